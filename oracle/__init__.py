@@ -1,0 +1,220 @@
+"""fp64 CPU oracle for the multi-tenant LoRA hot path (ctypes wrapper).
+
+TEST INFRASTRUCTURE. Only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import this package. The CUDA product
+path never imports it, and the two share no code.
+
+The arithmetic lives in ``oracle.c`` (plain C, fp64 accumulation); this module
+only builds it with gcc, loads it and marshals numpy arrays. Each function
+cites the passage of the pages it follows in ``oracle.c``:
+
+* LoRA algebra and the batched output ``Y = X.W + (x_i.A_i.B_i)``:
+  Punica README, section "How?".
+* Per-token adapter ids in one multi-tenant batch, -1 for none:
+  EpiLoRA abstract, sentence 1.
+* FP8 base GEMM whose epilogue adds each tenant's up-projection:
+  EpiLoRA abstract, sentences 2-4 (8-bit format read as E4M3 with per-row
+  scales; that reading is stated in ``oracle.c``).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile ``oracle.c`` into ``liboracle.so`` (gcc, OpenMP, no fast-math)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        cmd = ["gcc", "-O2", "-fopenmp", "-ffp-contract=off", "-fno-fast-math",
+               "-shared", "-fPIC", "-o", _LIB + ".tmp", _SRC, "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(_LIB + ".tmp", _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            build()
+            lib = ctypes.CDLL(_LIB)
+            P = ctypes.c_void_p
+            I = ctypes.c_int
+            lib.orc_bf16_decode.restype = ctypes.c_double
+            lib.orc_bf16_decode.argtypes = [ctypes.c_uint16]
+            lib.orc_e4m3_decode.restype = ctypes.c_double
+            lib.orc_e4m3_decode.argtypes = [ctypes.c_uint8]
+            lib.orc_e4m3_encode.restype = ctypes.c_uint8
+            lib.orc_e4m3_encode.argtypes = [ctypes.c_float]
+            lib.orc_build_segments.restype = None
+            lib.orc_build_segments.argtypes = [P, I, I, I, P, P, P, P, P, P]
+            lib.orc_lora_shrink.restype = None
+            lib.orc_lora_shrink.argtypes = [P, I, I, P, I, I, P, P, P]
+            lib.orc_lora_expand.restype = None
+            lib.orc_lora_expand.argtypes = [P, I, I, P, I, I, P, P, P, P, P]
+            lib.orc_lora_apply.restype = None
+            lib.orc_lora_apply.argtypes = [P, I, I, I, P, P, I, I, P, P, P, P, P]
+            lib.orc_linear_bf16_sampled.restype = None
+            lib.orc_linear_bf16_sampled.argtypes = [P, P, I, P, P, I, P]
+            lib.orc_quantize_rows.restype = None
+            lib.orc_quantize_rows.argtypes = [P, I, I, P, P]
+            lib.orc_fp8_gemm_lora_sampled.restype = None
+            lib.orc_fp8_gemm_lora_sampled.argtypes = [P, P, P, P, I, P, P, P, I, I, I,
+                                                      P, P, P, P, P, I, P]
+            lib.orc_num_threads.restype = I
+            lib.orc_set_num_threads.argtypes = [I]
+            _lib = lib
+    return _lib
+
+
+def _p(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _c(a, dtype):
+    return None if a is None else np.ascontiguousarray(a, dtype=dtype)
+
+
+def num_threads() -> int:
+    return _load().orc_num_threads()
+
+
+def set_num_threads(n: int) -> None:
+    _load().orc_set_num_threads(int(n))
+
+
+def bf16_decode(h: int) -> float:
+    return _load().orc_bf16_decode(int(h))
+
+
+def e4m3_decode(c: int) -> float:
+    return _load().orc_e4m3_decode(int(c))
+
+
+def e4m3_encode(f: float) -> int:
+    return int(_load().orc_e4m3_encode(float(f)))
+
+
+def bf16_to_f64(a: np.ndarray) -> np.ndarray:
+    """Decode an array of bf16 bit patterns (uint16) to fp64, element by element."""
+    lib = _load()
+    flat = np.asarray(a, dtype=np.uint16).ravel()
+    table = np.array([lib.orc_bf16_decode(i) for i in range(65536)], dtype=np.float64)
+    return table[flat].reshape(np.shape(a))
+
+
+def e4m3_to_f64(a: np.ndarray) -> np.ndarray:
+    lib = _load()
+    table = np.array([lib.orc_e4m3_decode(i) for i in range(256)], dtype=np.float64)
+    return table[np.asarray(a, dtype=np.uint8)]
+
+
+def build_segments(ids: np.ndarray, n_adapters: int, tile_t: int) -> dict:
+    lib = _load()
+    ids = _c(ids, np.int32)
+    T = ids.shape[0]
+    out = dict(
+        perm=np.zeros(T, np.int32),
+        indptr=np.zeros(n_adapters + 1, np.int32),
+        active=np.zeros(n_adapters, np.int32),
+        tile_ptr=np.zeros(n_adapters + 1, np.int32),
+        tok_adapter=np.zeros(T, np.int32),
+        counts=np.zeros(4, np.int32),
+    )
+    lib.orc_build_segments(_p(ids), T, n_adapters, tile_t, _p(out["perm"]), _p(out["indptr"]),
+                           _p(out["active"]), _p(out["tile_ptr"]), _p(out["tok_adapter"]),
+                           _p(out["counts"]))
+    return out
+
+
+def lora_shrink(x, A, ranks, ids) -> np.ndarray:
+    """x bf16 [T, h_in]; A bf16 [n_adapters, h_in, r_max]; returns v fp64 [T, r_max]."""
+    lib = _load()
+    x = _c(x, np.uint16); A = _c(A, np.uint16)
+    ranks = _c(ranks, np.int32); ids = _c(ids, np.int32)
+    T, h_in = x.shape
+    n_adapters, _, r_max = A.shape
+    v = np.zeros((T, r_max), np.float64)
+    lib.orc_lora_shrink(_p(x), T, h_in, _p(A), n_adapters, r_max, _p(ranks), _p(ids), _p(v))
+    return v
+
+
+def lora_expand(v, B, ranks, scales, ids, y_in) -> np.ndarray:
+    """v [T, r_max] (any float type, used exactly); B bf16 [n_adapters, r_max, h_out];
+    y_in bf16 [T, h_out]; returns y fp64 [T, h_out]."""
+    lib = _load()
+    v = _c(v, np.float64); B = _c(B, np.uint16)
+    ranks = _c(ranks, np.int32); scales = _c(scales, np.float32)
+    ids = _c(ids, np.int32); y_in = _c(y_in, np.uint16)
+    T, r_max = v.shape
+    n_adapters, _, h_out = B.shape
+    y = np.zeros((T, h_out), np.float64)
+    lib.orc_lora_expand(_p(v), T, r_max, _p(B), n_adapters, h_out, _p(ranks), _p(scales),
+                        _p(ids), _p(y_in), _p(y))
+    return y
+
+
+def lora_apply(x, A, B, ranks, scales, ids, y_in) -> np.ndarray:
+    lib = _load()
+    x = _c(x, np.uint16); A = _c(A, np.uint16); B = _c(B, np.uint16)
+    ranks = _c(ranks, np.int32); scales = _c(scales, np.float32)
+    ids = _c(ids, np.int32); y_in = _c(y_in, np.uint16)
+    T, h_in = x.shape
+    n_adapters, _, r_max = A.shape
+    h_out = B.shape[2]
+    y = np.zeros((T, h_out), np.float64)
+    lib.orc_lora_apply(_p(x), T, h_in, h_out, _p(A), _p(B), n_adapters, r_max, _p(ranks),
+                       _p(scales), _p(ids), _p(y_in), _p(y))
+    return y
+
+
+def linear_bf16_sampled(x, W, rows, cols) -> np.ndarray:
+    lib = _load()
+    x = _c(x, np.uint16); W = _c(W, np.uint16)
+    rows = _c(rows, np.int32); cols = _c(cols, np.int32)
+    out = np.zeros(rows.shape[0], np.float64)
+    lib.orc_linear_bf16_sampled(_p(x), _p(W), x.shape[1], _p(rows), _p(cols), rows.shape[0],
+                                _p(out))
+    return out
+
+
+def quantize_rows(x):
+    """x bf16 [M, K] -> (codes uint8 [M, K], scales fp32 [M])."""
+    lib = _load()
+    x = _c(x, np.uint16)
+    M, K = x.shape
+    xq = np.zeros((M, K), np.uint8)
+    sx = np.zeros(M, np.float32)
+    lib.orc_quantize_rows(_p(x), M, K, _p(xq), _p(sx))
+    return xq, sx
+
+
+def fp8_gemm_lora_sampled(xq, sx, Wq, sw, rows, cols, x=None, A=None, B=None, ranks=None,
+                          scales=None, ids=None) -> np.ndarray:
+    lib = _load()
+    xq = _c(xq, np.uint8); sx = _c(sx, np.float32)
+    Wq = _c(Wq, np.uint8); sw = _c(sw, np.float32)
+    rows = _c(rows, np.int32); cols = _c(cols, np.int32)
+    K = xq.shape[1]
+    N = Wq.shape[0]
+    if A is not None:
+        x = _c(x, np.uint16); A = _c(A, np.uint16); B = _c(B, np.uint16)
+        ranks = _c(ranks, np.int32); scales = _c(scales, np.float32); ids = _c(ids, np.int32)
+        n_adapters, _, r_max = A.shape
+    else:
+        n_adapters, r_max = 0, 0
+    out = np.zeros(rows.shape[0], np.float64)
+    lib.orc_fp8_gemm_lora_sampled(_p(xq), _p(sx), _p(Wq), _p(sw), K, _p(x), _p(A), _p(B),
+                                  n_adapters, r_max, N, _p(ranks), _p(scales), _p(ids),
+                                  _p(rows), _p(cols), rows.shape[0], _p(out))
+    return out

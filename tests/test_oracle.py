@@ -1,0 +1,451 @@
+"""Pins for the fp64 CPU oracle, independent of the oracle's own code.
+
+Each test checks the oracle against something the pages or mathematics fix:
+format definitions (OCP FP8 E4M3, bfloat16) re-checked against torch's own
+conversions, hand-worked examples (tests/golden/), brute force in exact
+rationals on tiny shapes, closed forms and invariants of the LoRA algebra
+(Punica README, "How?"), and a library sort for the segment order.
+"""
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from adapter_gemm_builder_b200 import workloads as wl
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+# ---------------------------------------------------------------- formats
+
+def test_bf16_decode_all_patterns_match_torch():
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    ours = oracle.bf16_to_f64(bits)
+    ref = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(torch.float64).numpy()
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(ours), nan)
+    assert np.array_equal(ours[~nan], ref[~nan])
+    assert np.array_equal(np.signbit(ours[~nan]), np.signbit(ref[~nan]))
+
+
+def test_e4m3_decode_all_codes_match_torch():
+    codes = np.arange(256, dtype=np.uint8)
+    ours = oracle.e4m3_to_f64(codes)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    nan = np.isnan(ref)
+    assert nan.sum() == 2 and nan[0x7F] and nan[0xFF]
+    assert np.array_equal(np.isnan(ours), nan)
+    assert np.array_equal(ours[~nan], ref[~nan])
+
+
+def _golden_e4m3():
+    rows = []
+    with open(os.path.join(GOLDEN, "e4m3_key_values.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            c, v = line.split()
+            rows.append((int(c, 16), float(v)))
+    return rows
+
+
+def test_e4m3_decode_golden_values():
+    for c, v in _golden_e4m3():
+        got = oracle.e4m3_decode(c)
+        if math.isnan(v):
+            assert math.isnan(got), hex(c)
+        else:
+            assert got == v and math.copysign(1, got) == math.copysign(1, v), hex(c)
+
+
+def test_e4m3_encode_roundtrip_every_finite_code():
+    for c in range(256):
+        v = oracle.e4m3_decode(c)
+        if math.isnan(v):
+            continue
+        assert oracle.e4m3_encode(v) == c, hex(c)
+
+
+def test_e4m3_encode_matches_torch_in_range():
+    rng = np.random.default_rng(123)
+    vals = np.concatenate([
+        rng.uniform(-448, 448, 4000),
+        rng.standard_normal(4000) * 3,
+        rng.standard_normal(2000) * 0.01,          # subnormal region
+        rng.uniform(-2 ** -9, 2 ** -9, 500),
+    ]).astype(np.float32)
+    ref = torch.from_numpy(vals).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    ours = np.array([oracle.e4m3_encode(float(v)) for v in vals], np.uint8)
+    assert np.array_equal(ours, ref)
+
+
+def test_e4m3_encode_ties_to_even_and_saturation():
+    # midpoint of 1.0 (0x38) and 1.125 (0x39): even code wins
+    assert oracle.e4m3_encode(1.0625) == 0x38
+    # midpoint of 1.125 (0x39) and 1.25 (0x3A)
+    assert oracle.e4m3_encode(1.1875) == 0x3A
+    # half the smallest subnormal ties between 0 and 2^-9: goes to 0
+    assert oracle.e4m3_encode(2.0 ** -10) == 0x00
+    assert oracle.e4m3_encode(1.5 * 2.0 ** -10) == 0x01
+    # every midpoint between consecutive positive codes goes to the even one
+    for c in range(0, 0x7E):
+        lo, hi = oracle.e4m3_decode(c), oracle.e4m3_decode(c + 1)
+        mid = (lo + hi) / 2
+        if float(np.float32(mid)) != mid:
+            continue
+        want = c if c % 2 == 0 else c + 1
+        assert oracle.e4m3_encode(mid) == want, hex(c)
+    # saturating conversion: beyond the largest finite value -> +-448
+    for v in (448.0, 449.0, 464.0, 480.0, 1e30, float("inf")):
+        assert oracle.e4m3_encode(v) == 0x7E
+        assert oracle.e4m3_encode(-v) == 0xFE
+    assert oracle.e4m3_encode(float("nan")) == 0x7F
+
+
+# ---------------------------------------------------------------- segments
+
+def _segments_by_sort(ids, n_adapters, tile_t):
+    T = len(ids)
+    key = [(ids[t] if 0 <= ids[t] < n_adapters else n_adapters, t) for t in range(T)]
+    order = sorted(range(T), key=lambda t: key[t])  # library sort, stable key
+    counts = [sum(1 for t in range(T) if key[t][0] == a) for a in range(n_adapters + 1)]
+    indptr = [sum(counts[:a]) for a in range(n_adapters + 1)]
+    active = [a for a in range(n_adapters) if counts[a] > 0]
+    tiles = [(counts[a] + tile_t - 1) // tile_t for a in active]
+    tile_ptr = [sum(tiles[:s]) for s in range(len(active) + 1)]
+    n_bad = sum(1 for i in ids if i != -1 and not (0 <= i < n_adapters))
+    return order, indptr, active, tile_ptr, n_bad
+
+
+SEG_KINDS = ["distinct", "identical", "uniform", "zipf", "sorted_zipf", "none", "bad", "single"]
+
+
+@pytest.mark.parametrize("kind", SEG_KINDS)
+def test_segments_match_sorted_order(kind):
+    rng = np.random.default_rng(SEG_KINDS.index(kind))
+    n_adapters, tile_t = 12, 4
+    if kind == "none":
+        ids = np.full(17, -1, np.int32)
+    elif kind == "bad":
+        ids = rng.integers(-3, n_adapters + 3, size=40).astype(np.int32)
+    elif kind == "single":
+        ids = np.array([5], np.int32)
+    elif kind == "distinct":
+        ids = wl.make_ids("distinct", rng, 12, n_adapters, none_frac=0.2)
+    else:
+        ids = wl.make_ids(kind, rng, 50, n_adapters, none_frac=0.1)
+    seg = oracle.build_segments(ids, n_adapters, tile_t)
+    order, indptr, active, tile_ptr, n_bad = _segments_by_sort(list(ids), n_adapters, tile_t)
+    assert seg["perm"].tolist() == order
+    assert seg["indptr"].tolist() == indptr
+    n_active = len(active)
+    assert seg["counts"].tolist() == [indptr[n_adapters], n_active, n_bad, tile_ptr[-1]]
+    assert seg["active"][:n_active].tolist() == active
+    assert seg["tile_ptr"][:n_active + 1].tolist() == tile_ptr
+    want_tok = [i if 0 <= i < n_adapters else -1 for i in ids]
+    assert seg["tok_adapter"].tolist() == want_tok
+
+
+def test_segments_empty_batch():
+    seg = oracle.build_segments(np.zeros(0, np.int32), 3, 64)
+    assert seg["counts"].tolist() == [0, 0, 0, 0]
+    assert seg["indptr"].tolist() == [0, 0, 0, 0]
+
+
+# ---------------------------------------------------------------- LoRA algebra
+
+def _read_worked_example():
+    d = {}
+    with open(os.path.join(GOLDEN, "lora_how_worked_example.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            k, *vals = line.split()
+            d.setdefault(k, []).append([float(v) for v in vals])
+    return d
+
+
+@pytest.mark.parametrize("s", [1.0, 2.0])
+def test_worked_example_of_how_section(s):
+    d = _read_worked_example()
+    W_h1h2 = np.array(d["W_row0"] + d["W_row1"])           # [H1=2, H2=3]
+    W = wl.to_bf16_bits(W_h1h2.T.copy())                    # stored [N=3][K=2]
+    A = np.stack([wl.to_bf16_bits(np.array(d["A0"][0]).reshape(2, 1)),
+                  wl.to_bf16_bits(np.array(d["A1"][0]).reshape(2, 1))])
+    B = np.stack([wl.to_bf16_bits(np.array(d["B0"][0]).reshape(1, 3)),
+                  wl.to_bf16_bits(np.array(d["B1"][0]).reshape(1, 3))])
+    toks = np.array(d["tok"])
+    ids = toks[:, 0].astype(np.int32)
+    x = wl.to_bf16_bits(toks[:, 1:])
+    rows = np.repeat(np.arange(3), 3).astype(np.int32)
+    cols = np.tile(np.arange(3), 3).astype(np.int32)
+    base = oracle.linear_bf16_sampled(x, W, rows, cols).reshape(3, 3)
+    assert np.array_equal(base, np.array(d["base"]))
+    y = oracle.lora_apply(x, A, B, np.array([1, 1], np.int32), np.array([s, s], np.float32),
+                          ids, wl.to_bf16_bits(base))
+    want = np.array(d["y_s1"] if s == 1.0 else d["y_s2"])
+    assert np.array_equal(y, want)
+
+
+def _frac_bf16(a):
+    return [[Fraction(float(v)) for v in row] for row in oracle.bf16_to_f64(a)]
+
+
+def _brute_force_apply(x, A, B, ranks, scales, ids, y_in):
+    """Exact rationals, straight from y = y_in + s * (x A) B per token."""
+    T = x.shape[0]
+    n_adapters, h_in, r_max = A.shape
+    h_out = B.shape[2]
+    X = _frac_bf16(x)
+    Y = _frac_bf16(y_in)
+    out = []
+    for t in range(T):
+        a = int(ids[t])
+        row = list(Y[t])
+        if 0 <= a < n_adapters:
+            r = int(ranks[a])
+            Aa = _frac_bf16(A[a][:, :r])
+            Ba = _frac_bf16(B[a][:r, :])
+            s = Fraction(float(scales[a]))
+            v = [sum(X[t][k] * Aa[k][j] for k in range(h_in)) for j in range(r)]
+            for n in range(h_out):
+                row[n] += s * sum(v[j] * Ba[j][n] for j in range(r))
+        out.append(row)
+    return out
+
+
+def _tiny_problem(seed, T=5, n_adapters=3, h_in=7, h_out=5, r_max=3, ints=False):
+    rng = np.random.default_rng(seed)
+    ids = rng.integers(-1, n_adapters, size=T).astype(np.int32)
+    ranks = rng.integers(1, r_max + 1, size=n_adapters).astype(np.int32)
+    scales = rng.choice(np.array([0.5, 1.0, 2.0, -1.5], np.float32), size=n_adapters)
+
+    def draw(shape, std):
+        if ints:
+            return wl.to_bf16_bits(rng.integers(-2, 3, size=shape).astype(np.float32))
+        return wl.normal_bf16(rng, shape, std)
+    x = draw((T, h_in), 1.0)
+    A = np.full((n_adapters, h_in, r_max), wl.BF16_NAN, np.uint16)
+    B = np.full((n_adapters, r_max, h_out), wl.BF16_NAN, np.uint16)
+    for a in range(n_adapters):
+        A[a, :, :ranks[a]] = draw((h_in, ranks[a]), 0.4)
+        B[a, :ranks[a], :] = draw((ranks[a], h_out), 0.6)
+    y_in = draw((T, h_out), 1.0)
+    return x, A, B, ranks, scales, ids, y_in
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_apply_exact_rationals_small_ints(seed):
+    args = _tiny_problem(seed, ints=True)
+    got = oracle.lora_apply(*args)
+    want = _brute_force_apply(*args)
+    assert [[Fraction(float(v)) for v in row] for row in got] == want
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_apply_rationals_random_bf16(seed):
+    args = _tiny_problem(100 + seed, T=6, n_adapters=2, h_in=8, h_out=4, r_max=3)
+    got = oracle.lora_apply(*args)
+    want = np.array([[float(v) for v in row] for row in _brute_force_apply(*args)])
+    assert np.allclose(got, want, rtol=1e-12, atol=1e-12)
+
+
+def test_shrink_then_expand_equals_apply():
+    x, A, B, ranks, scales, ids, y_in = _tiny_problem(7, T=9, n_adapters=4, h_in=16, h_out=12,
+                                                      r_max=4)
+    v = oracle.lora_shrink(x, A, ranks, ids)
+    y = oracle.lora_expand(v, B, ranks, scales, ids, y_in)
+    assert np.array_equal(y, oracle.lora_apply(x, A, B, ranks, scales, ids, y_in))
+    # padding beyond each adapter's rank is NaN in A and B and is never read
+    assert np.isfinite(v).all() and np.isfinite(y).all()
+
+
+def _random_problem(seed, T=24, n_adapters=5, h_in=64, h_out=40, r_max=8):
+    p = wl.make_lora_problem("t", seed, T=T, n_adapters=n_adapters, h_in=h_in, h_out=h_out,
+                             r_max=r_max, ids_kind="uniform", none_frac=0.2,
+                             rank_choices=(1, 3, 8), with_W=True)
+    return p
+
+
+def test_invariant_zero_B_gives_base_output():
+    p = _random_problem(1)
+    B0 = np.where(p.B[0] == wl.BF16_NAN, p.B[0], np.uint16(0))
+    y = oracle.lora_apply(p.x[0], p.A[0], B0, p.ranks, p.scales, p.ids, p.y_in[0])
+    assert np.array_equal(y, oracle.bf16_to_f64(p.y_in[0]))
+
+
+def test_invariant_no_adapter_rows_untouched():
+    p = _random_problem(2)
+    y = oracle.lora_apply(p.x[0], p.A[0], p.B[0], p.ranks, p.scales, p.ids, p.y_in[0])
+    none = p.ids == -1
+    assert none.any()
+    assert np.array_equal(y[none], oracle.bf16_to_f64(p.y_in[0][none]))
+    assert not np.array_equal(y[~none], oracle.bf16_to_f64(p.y_in[0][~none]))
+
+
+def test_invariant_permuting_tokens_permutes_outputs():
+    p = _random_problem(3)
+    y = oracle.lora_apply(p.x[0], p.A[0], p.B[0], p.ranks, p.scales, p.ids, p.y_in[0])
+    pi = np.random.default_rng(0).permutation(p.T)
+    y2 = oracle.lora_apply(p.x[0][pi], p.A[0], p.B[0], p.ranks, p.scales, p.ids[pi],
+                           p.y_in[0][pi])
+    assert np.array_equal(y2, y[pi])
+
+
+def test_invariant_merged_weight():
+    """x.W^T + s.(x.A).B == x.(W + s.(A.B)^T)^T, the README's identity, with the
+    merged product formed by numpy's matmul."""
+    p = _random_problem(4)
+    T, K, N = p.T, p.h_in, p.h_out
+    rows = np.repeat(np.arange(T), N).astype(np.int32)
+    cols = np.tile(np.arange(N), T).astype(np.int32)
+    base = oracle.linear_bf16_sampled(p.x[0], p.W[0], rows, cols).reshape(T, N)
+    # feed the exact fp64 base in through y_in = 0 and add it afterwards
+    zeros = np.zeros((T, N), np.uint16)
+    lora = oracle.lora_apply(p.x[0], p.A[0], p.B[0], p.ranks, p.scales, p.ids, zeros)
+    y = base + lora
+    X = oracle.bf16_to_f64(p.x[0])
+    W = oracle.bf16_to_f64(p.W[0])
+    for t in range(T):
+        a = p.ids[t]
+        if a < 0:
+            want = X[t] @ W.T
+        else:
+            r = p.ranks[a]
+            Aa = oracle.bf16_to_f64(p.A[0][a][:, :r])
+            Ba = oracle.bf16_to_f64(p.B[0][a][:r, :])
+            merged = W + float(p.scales[a]) * (Aa @ Ba).T
+            want = X[t] @ merged.T
+        assert np.allclose(y[t], want, rtol=1e-9, atol=1e-9)
+
+
+def test_rank1_closed_form():
+    """A = e_j (unit column), B = c * ones -> s * x[t, j] * c, exactly."""
+    T, h_in, h_out, j, c, s = 7, 32, 9, 5, 0.75, 2.0
+    rng = np.random.default_rng(9)
+    x = wl.normal_bf16(rng, (T, h_in))
+    A = np.zeros((1, h_in, 1), np.uint16)
+    A[0, j, 0] = wl.to_bf16_bits(np.array([1.0]))[0]
+    B = wl.to_bf16_bits(np.full((1, 1, h_out), c))
+    y = oracle.lora_apply(x, A, B, np.array([1], np.int32), np.array([s], np.float32),
+                          np.zeros(T, np.int32), np.zeros((T, h_out), np.uint16))
+    want = s * oracle.bf16_to_f64(x)[:, j:j + 1] * c * np.ones((1, h_out))
+    assert np.array_equal(y, want)
+
+
+def test_expand_uses_v_exactly():
+    rng = np.random.default_rng(5)
+    T, r, h_out = 4, 2, 3
+    v = rng.standard_normal((T, r)).astype(np.float32)
+    B = wl.to_bf16_bits(np.array([[[1.0, 2.0, 0.5], [-1.0, 0.25, 4.0]]]))
+    ids = np.array([0, -1, 0, 0], np.int32)
+    y = oracle.lora_expand(v, B, None, np.array([3.0], np.float32), ids,
+                           np.zeros((T, h_out), np.uint16))
+    Bf = np.array([[1.0, 2.0, 0.5], [-1.0, 0.25, 4.0]])
+    for t in range(T):
+        want = np.zeros(h_out) if ids[t] < 0 else 3.0 * (v[t].astype(np.float64) @ Bf)
+        assert np.allclose(y[t], want, rtol=1e-15, atol=0)
+
+
+# ---------------------------------------------------------------- FP8 path
+
+def test_quantize_rows_exact_row():
+    vals = np.array([[448, 224, 1, -2, 0.5, 0]], np.float32)
+    xq, sx = oracle.quantize_rows(wl.to_bf16_bits(vals))
+    assert sx[0] == 1.0
+    assert xq[0].tolist() == [0x7E, 0x76, 0x38, 0xC0, 0x30, 0x00]
+
+
+def test_quantize_rows_zero_row_scale_one():
+    xq, sx = oracle.quantize_rows(np.zeros((2, 16), np.uint16))
+    assert sx.tolist() == [1.0, 1.0] and not xq.any()
+
+
+def test_quantize_rows_scale_and_error_bound():
+    rng = np.random.default_rng(11)
+    x = wl.normal_bf16(rng, (8, 256), 3.0)
+    xq, sx = oracle.quantize_rows(x)
+    X = oracle.bf16_to_f64(x)
+    amax = np.abs(X).max(axis=1)
+    assert np.array_equal(sx, (amax.astype(np.float32) / np.float32(448.0)).astype(np.float32))
+    deq = oracle.e4m3_to_f64(xq) * sx[:, None].astype(np.float64)
+    # the largest element lands on the top code
+    for m in range(8):
+        k = int(np.argmax(np.abs(X[m])))
+        assert xq[m, k] & 0x7F == 0x7E
+    # relative error of a normal E4M3 value is at most 2^-4 (half of 2^-3)
+    big = np.abs(X) >= 2.0 ** -6 * sx[:, None]
+    rel = np.abs(deq - X)[big] / np.abs(X)[big]
+    assert rel.max() <= 2.0 ** -4 * (1 + 1e-6)
+    # agrees with a library E4M3 cast of the fp32 quotient
+    q = (X.astype(np.float32) / sx[:, None]).astype(np.float32)
+    ref = torch.from_numpy(q).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(xq, ref)
+
+
+def _brute_force_fp8(xq, sx, Wq, sw, x, A, B, ranks, scales, ids, m, n):
+    K = xq.shape[1]
+    acc = sum(Fraction(oracle.e4m3_decode(int(xq[m, k]))) *
+              Fraction(oracle.e4m3_decode(int(Wq[n, k]))) for k in range(K))
+    y = Fraction(float(sx[m])) * Fraction(float(sw[n])) * acc
+    a = int(ids[m])
+    if A is not None and 0 <= a < A.shape[0]:
+        r = int(ranks[a])
+        Xr = [Fraction(v) for v in oracle.bf16_to_f64(x[m])]
+        Aa = _frac_bf16(A[a][:, :r])
+        Ba = _frac_bf16(B[a][:r, :])
+        v = [sum(Xr[k] * Aa[k][j] for k in range(K)) for j in range(r)]
+        y += Fraction(float(scales[a])) * sum(v[j] * Ba[j][n] for j in range(r))
+    return y
+
+
+@pytest.mark.parametrize("with_lora", [False, True])
+def test_fp8_gemm_lora_bruteforce(with_lora):
+    rng = np.random.default_rng(21)
+    M, K, N = 4, 16, 6
+    p = wl.fp8_problem(M, K=K, N=N, n_adapters=3, r=2, seed=5, ids_kind="uniform",
+                       none_frac=0.3, W=wl.normal_bf16(rng, (N, K), 0.25))
+    xq, sx = oracle.quantize_rows(p.x)
+    Wq, sw = oracle.quantize_rows(p.W)
+    rows = np.repeat(np.arange(M), N).astype(np.int32)
+    cols = np.tile(np.arange(N), M).astype(np.int32)
+    kw = dict(x=p.x, A=p.A, B=p.B, ranks=p.ranks, scales=p.scales, ids=p.ids) if with_lora else {}
+    got = oracle.fp8_gemm_lora_sampled(xq, sx, Wq, sw, rows, cols, **kw)
+    for i in range(M * N):
+        want = _brute_force_fp8(xq, sx, Wq, sw, p.x, p.A if with_lora else None, p.B, p.ranks,
+                                p.scales, p.ids, rows[i], cols[i])
+        assert abs(got[i] - float(want)) <= 1e-12 * (1 + abs(float(want)))
+
+
+def test_fp8_gemm_small_int_exact():
+    """Small integers are exact in E4M3 with unit scales: the GEMM is exact."""
+    rng = np.random.default_rng(3)
+    M, K, N = 3, 32, 5
+    xi = rng.integers(-8, 9, size=(M, K)).astype(np.float32)
+    xi[:, 0] = 448.0  # pin amax so that sx == 1
+    wi = rng.integers(-8, 9, size=(N, K)).astype(np.float32)
+    wi[:, 0] = 448.0
+    xq, sx = oracle.quantize_rows(wl.to_bf16_bits(xi))
+    Wq, sw = oracle.quantize_rows(wl.to_bf16_bits(wi))
+    assert (sx == 1).all() and (sw == 1).all()
+    rows = np.repeat(np.arange(M), N).astype(np.int32)
+    cols = np.tile(np.arange(N), M).astype(np.int32)
+    got = oracle.fp8_gemm_lora_sampled(xq, sx, Wq, sw, rows, cols)
+    assert np.array_equal(got.reshape(M, N), xi.astype(np.float64) @ wi.T.astype(np.float64))
+
+
+def test_linear_bf16_matches_numpy():
+    rng = np.random.default_rng(8)
+    x = wl.normal_bf16(rng, (5, 33))
+    W = wl.normal_bf16(rng, (7, 33))
+    rows = np.repeat(np.arange(5), 7).astype(np.int32)
+    cols = np.tile(np.arange(7), 5).astype(np.int32)
+    got = oracle.linear_bf16_sampled(x, W, rows, cols).reshape(5, 7)
+    want = oracle.bf16_to_f64(x) @ oracle.bf16_to_f64(W).T
+    assert np.allclose(got, want, rtol=1e-13, atol=1e-13)
