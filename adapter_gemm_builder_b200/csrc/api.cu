@@ -1,0 +1,271 @@
+// api.cu -- the extern "C" entry points declared in include/lora.h.
+// Host-side argument checks, workspace carving and stream-ordered launches;
+// no allocation, no exceptions across the ABI.
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <string.h>
+
+#include "internal.h"
+#include "lora.h"
+
+using namespace lora;
+
+namespace {
+
+constexpr int kVersion = 1;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? LORA_OK : LORA_ERR_CUDA; }
+
+size_t align256(size_t x) { return (x + 255) / 256 * 256; }
+
+// Checks shared by every call that reads the pool.
+int check_pool(const lora_pool_t* pool)
+{
+    if (!pool || !pool->A || !pool->B) return LORA_ERR_INVALID_ARG;
+    if (pool->n_slices < 1 || pool->n_adapters < 1 || pool->h_in < 1 || pool->h_out < 1 ||
+        pool->r_max < 1)
+        return LORA_ERR_INVALID_ARG;
+    if (pool->n_slices > 65535 || pool->n_adapters > LORA_MAX_ADAPTERS) return LORA_ERR_UNSUPPORTED;
+    if (pool->r_max > LORA_MAX_RANK) return LORA_ERR_UNSUPPORTED;
+    if (pool->h_in % 8 || pool->h_out % 8 || pool->r_max % 8) return LORA_ERR_INVALID_ARG;
+    if (!aligned16(pool->A) || !aligned16(pool->B)) return LORA_ERR_INVALID_ARG;
+    if ((long long)pool->n_slices * pool->n_adapters * pool->h_in * pool->r_max > (1ll << 40))
+        return LORA_ERR_UNSUPPORTED;
+    return LORA_OK;
+}
+
+int check_segments(const lora_segments_t* seg, int n_adapters)
+{
+    if (!seg) return LORA_ERR_INVALID_ARG;
+    if (seg->T < 0 || seg->n_adapters != n_adapters) return LORA_ERR_INVALID_ARG;
+    if (!seg->indptr || !seg->active || !seg->tile_ptr || !seg->counts) return LORA_ERR_INVALID_ARG;
+    if (seg->T > 0 && (!seg->perm || !seg->tok_adapter)) return LORA_ERR_INVALID_ARG;
+    return LORA_OK;
+}
+
+size_t fp8_ws_layout(int M, int K, const lora_pool_t* pool, size_t* off_xq, size_t* off_sx,
+                     size_t* off_v)
+{
+    size_t off = 256;  // status word block
+    *off_xq = off;
+    off += align256((size_t)M * K);
+    *off_sx = off;
+    off += align256((size_t)M * 4);
+    *off_v = off;
+    if (pool) off += align256((size_t)M * pool->r_max * 4);
+    return off;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* lora_status_string(int s)
+{
+    switch (s) {
+    case LORA_OK: return "ok";
+    case LORA_ERR_INVALID_ARG: return "invalid argument";
+    case LORA_ERR_UNSUPPORTED: return "unsupported shape";
+    case LORA_ERR_BAD_ADAPTER_ID: return "adapter id outside [-1, n_adapters)";
+    case LORA_ERR_CUDA: return "CUDA error";
+    case LORA_ERR_WORKSPACE: return "workspace missing or too small";
+    case LORA_ERR_TIMEOUT: return "a bounded device wait timed out";
+    default: return "unknown status";
+    }
+}
+
+int lora_version(void) { return kVersion; }
+
+int lora_tile_tokens(void) { return LORA_TILE_TOKENS; }
+
+size_t lora_workspace_size(int op, int T, int K, const lora_pool_t* pool)
+{
+    if (T < 0) return (size_t)-1;
+    switch (op) {
+    case LORA_OP_SHRINK:
+    case LORA_OP_EXPAND:
+    case LORA_OP_APPLY: return 0;
+    case LORA_OP_FP8_GEMM: {
+        if (K <= 0) return (size_t)-1;
+        if (pool && check_pool(pool) != LORA_OK) return (size_t)-1;
+        size_t a, b, c;
+        return fp8_ws_layout(T, K, pool, &a, &b, &c);
+    }
+    default: return (size_t)-1;
+    }
+}
+
+int lora_workspace_init(void* ws, size_t ws_bytes, lora_stream_t stream)
+{
+    if (!ws || ws_bytes == 0) return LORA_ERR_INVALID_ARG;
+    return cuda_status(cudaMemsetAsync(ws, 0, ws_bytes, (cudaStream_t)stream));
+}
+
+int lora_workspace_status(void* ws, size_t ws_bytes, lora_stream_t stream, uint32_t* detail)
+{
+    if (!ws || ws_bytes < 256) return LORA_ERR_INVALID_ARG;
+    uint32_t word = 0;
+    cudaError_t e = cudaMemcpyAsync(&word, ws, sizeof(word), cudaMemcpyDeviceToHost,
+                                    (cudaStream_t)stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize((cudaStream_t)stream);
+    if (e != cudaSuccess) return LORA_ERR_CUDA;
+    if (detail) *detail = word;
+    if (word) {
+        e = cudaMemsetAsync(ws, 0, sizeof(uint32_t), (cudaStream_t)stream);
+        if (e == cudaSuccess) e = cudaStreamSynchronize((cudaStream_t)stream);
+        if (e != cudaSuccess) return LORA_ERR_CUDA;
+        return LORA_ERR_TIMEOUT;
+    }
+    return LORA_OK;
+}
+
+int lora_build_segments(const int32_t* ids, int T, int n_adapters, const lora_segments_t* seg,
+                        int sync_check, lora_stream_t stream)
+{
+    if (T < 0 || n_adapters < 1) return LORA_ERR_INVALID_ARG;
+    if (n_adapters > LORA_MAX_ADAPTERS || T >= (1 << 30)) return LORA_ERR_UNSUPPORTED;
+    if (T > 0 && !ids) return LORA_ERR_INVALID_ARG;
+    int st = check_segments(seg, n_adapters);
+    if (st != LORA_OK) return st;
+    if (seg->T != T) return LORA_ERR_INVALID_ARG;
+    cudaError_t e = launch_build_segments(ids, T, n_adapters, *seg, (cudaStream_t)stream);
+    if (e != cudaSuccess) return LORA_ERR_CUDA;
+    if (sync_check) {
+        int32_t counts[4];
+        e = cudaMemcpyAsync(counts, seg->counts, sizeof(counts), cudaMemcpyDeviceToHost,
+                            (cudaStream_t)stream);
+        if (e == cudaSuccess) e = cudaStreamSynchronize((cudaStream_t)stream);
+        if (e != cudaSuccess) return LORA_ERR_CUDA;
+        if (counts[2] != 0) return LORA_ERR_BAD_ADAPTER_ID;
+    }
+    return LORA_OK;
+}
+
+static int check_x(const void* x, int64_t x_slice_stride, const lora_pool_t* pool, int T)
+{
+    if (!x || !aligned16(x)) return LORA_ERR_INVALID_ARG;
+    if (x_slice_stride < 0 || x_slice_stride % 8) return LORA_ERR_INVALID_ARG;
+    if (x_slice_stride != 0 && x_slice_stride < (int64_t)T * pool->h_in) return LORA_ERR_INVALID_ARG;
+    return LORA_OK;
+}
+
+int lora_shrink(const void* x, int64_t x_slice_stride, const lora_pool_t* pool,
+                const lora_segments_t* seg, float* v, void* ws, size_t ws_bytes,
+                lora_stream_t stream)
+{
+    (void)ws;
+    (void)ws_bytes;
+    int st = check_pool(pool);
+    if (st != LORA_OK) return st;
+    if ((st = check_segments(seg, pool->n_adapters)) != LORA_OK) return st;
+    if (seg->T == 0) return LORA_OK;
+    if ((st = check_x(x, x_slice_stride, pool, seg->T)) != LORA_OK) return st;
+    if (!v || !aligned16(v)) return LORA_ERR_INVALID_ARG;
+    return cuda_status(launch_sgmv(SGMV_SHRINK, x, x_slice_stride, *pool, *seg, v, nullptr,
+                                   (cudaStream_t)stream, false));
+}
+
+int lora_expand(const float* v, const lora_pool_t* pool, const lora_segments_t* seg, void* y,
+                void* ws, size_t ws_bytes, lora_stream_t stream)
+{
+    (void)ws;
+    (void)ws_bytes;
+    int st = check_pool(pool);
+    if (st != LORA_OK) return st;
+    if ((st = check_segments(seg, pool->n_adapters)) != LORA_OK) return st;
+    if (seg->T == 0) return LORA_OK;
+    if (!v || !aligned16(v) || !y || !aligned16(y)) return LORA_ERR_INVALID_ARG;
+    return cuda_status(launch_sgmv(SGMV_EXPAND, nullptr, 0, *pool, *seg, const_cast<float*>(v), y,
+                                   (cudaStream_t)stream, false));
+}
+
+int lora_apply(const void* x, int64_t x_slice_stride, const lora_pool_t* pool,
+               const lora_segments_t* seg, void* y, void* ws, size_t ws_bytes,
+               lora_stream_t stream)
+{
+    (void)ws;
+    (void)ws_bytes;
+    int st = check_pool(pool);
+    if (st != LORA_OK) return st;
+    if ((st = check_segments(seg, pool->n_adapters)) != LORA_OK) return st;
+    if (seg->T == 0) return LORA_OK;
+    if ((st = check_x(x, x_slice_stride, pool, seg->T)) != LORA_OK) return st;
+    if (!y || !aligned16(y)) return LORA_ERR_INVALID_ARG;
+    return cuda_status(launch_sgmv(SGMV_APPLY, x, x_slice_stride, *pool, *seg, nullptr, y,
+                                   (cudaStream_t)stream, false));
+}
+
+int fp8_quantize_rows(const void* x, int M, int K, uint8_t* xq, float* sx, lora_stream_t stream)
+{
+    if (M < 0 || K <= 0 || K % 16) return LORA_ERR_INVALID_ARG;
+    if (M == 0) return LORA_OK;
+    if (!x || !xq || !sx || !aligned16(x) || !aligned16(xq)) return LORA_ERR_INVALID_ARG;
+    return cuda_status(launch_quantize_rows(x, nullptr, M, K, xq, sx, (cudaStream_t)stream));
+}
+
+int fp8_gemm_lora_epilogue(const void* x, int M, int K, int N, const uint8_t* Wq,
+                           const float* w_scale, const lora_pool_t* pool,
+                           const lora_segments_t* seg, void* y, void* ws, size_t ws_bytes,
+                           lora_stream_t stream)
+{
+    if (M < 1 || K < 16 || N < 8 || K % 16 || N % 8) return LORA_ERR_INVALID_ARG;
+    if (!x || !Wq || !w_scale || !y) return LORA_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(Wq) || !aligned16(y)) return LORA_ERR_INVALID_ARG;
+    if (M > (1 << 24)) return LORA_ERR_UNSUPPORTED;
+    if (pool) {
+        int st = check_pool(pool);
+        if (st != LORA_OK) return st;
+        if (pool->n_slices != 1 || pool->h_in != K || pool->h_out != N) return LORA_ERR_INVALID_ARG;
+        if ((st = check_segments(seg, pool->n_adapters)) != LORA_OK) return st;
+        if (seg->T != M) return LORA_ERR_INVALID_ARG;
+    }
+    size_t off_xq, off_sx, off_v;
+    const size_t need = fp8_ws_layout(M, K, pool, &off_xq, &off_sx, &off_v);
+    if (!ws || ws_bytes < need || !aligned16(ws)) return LORA_ERR_WORKSPACE;
+    uint8_t* w = static_cast<uint8_t*>(ws);
+    uint32_t* status = reinterpret_cast<uint32_t*>(w);
+    uint8_t* xq = w + off_xq;
+    float* sx = reinterpret_cast<float*>(w + off_sx);
+    float* v = pool ? reinterpret_cast<float*>(w + off_v) : nullptr;
+    cudaStream_t s = (cudaStream_t)stream;
+
+    // 1. activations -> E4M3, rows in segment order when adapters are present
+    cudaError_t e = launch_quantize_rows(x, pool ? seg->perm : nullptr, M, K, xq, sx, s);
+    if (e != cudaSuccess) return LORA_ERR_CUDA;
+    // 2. the down-projection, launched first
+    if (pool) {
+        e = launch_sgmv(SGMV_SHRINK, x, 0, *pool, *seg, v, nullptr, s, true);
+        if (e != cudaSuccess) return LORA_ERR_CUDA;
+    }
+    // 3. the GEMM, a programmatic dependent of the shrink when there is one
+    Fp8GemmArgs a = {};
+    a.M = M;
+    a.N = N;
+    a.K = K;
+    a.xq = xq;
+    a.sx = sx;
+    a.Wq = Wq;
+    a.sw = w_scale;
+    a.y = static_cast<uint16_t*>(y);
+    a.status = status;
+    a.lora = pool != nullptr;
+    if (pool) {
+        a.perm = seg->perm;
+        a.tok_adapter = seg->tok_adapter;
+        a.indptr = seg->indptr;
+        a.active = seg->active;
+        a.counts = seg->counts;
+        a.v = v;
+        a.B = static_cast<const uint16_t*>(pool->B);
+        a.ranks = pool->ranks;
+        a.scales = pool->scales;
+        a.n_adapters = pool->n_adapters;
+        a.r_max = pool->r_max;
+        a.pdl = true;
+    }
+    return cuda_status(launch_fp8_gemm(a, s));
+}
+
+}  // extern "C"

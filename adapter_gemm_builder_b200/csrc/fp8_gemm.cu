@@ -1,0 +1,610 @@
+// fp8_gemm.cu -- 8-bit (E4M3) base GEMM with the multi-tenant LoRA expand
+// fused into its epilogue, on the sm_100a tensor cores (tcgen05 + TMEM + TMA).
+//
+// The EpiLoRA abstract (sentences 3-4) observes that the GEMM needs the
+// adapter's down-projection only in its epilogue; so the down-projection runs
+// first, and the GEMM -- launched as a programmatic dependent kernel -- streams
+// its weights meanwhile and adds every tenant's up-projection before the store:
+//   y[m][n] = sx[m] * sw[n] * sum_k xq[m][k] Wq[n][k] + s_a * sum_j v[m][j] B[a][j][n].
+//
+// Design for decode-sized M (tokens) and large N x K weights:
+//  * swap-AB: the MMA's M dimension is 128 rows of W, its N dimension the
+//    tokens (16..256 per tile), so W -- the bytes that bound the kernel -- is
+//    read exactly once while all tokens ride along in one MMA.
+//  * persistent CTAs (one per SM), warp-specialised:
+//      warp 0  TMA producer: W and xq k-blocks into a ring of stages
+//              (128-byte or 64-byte swizzle, matching the MMA descriptors);
+//      warp 1  TMEM allocator and single-thread tcgen05.mma issuer
+//              (kind::f8f6f4, fp32 accumulators in TMEM, double-buffered so the
+//              epilogue of tile i overlaps the mainloop of tile i+1);
+//      warp 2  B stager: TMA-loads the [r x 128] slices of B_a for every
+//              adapter present in the tile's token block into shared memory,
+//              while the mainloop runs;
+//      warps 3..10 epilogue: tcgen05.ld of the accumulator, per-token and
+//              per-channel scales, the LoRA term on CUDA cores from shared
+//              memory, bf16 stores.
+//  * tokens are processed in segment order (rows of xq are permuted by the
+//    quantiser), so the adapter changes only at segment boundaries.
+//  * every mbarrier wait is bounded (2 s); on expiry the CTA records a status
+//    word in the workspace, drains what it issued and returns.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace lora {
+namespace {
+
+constexpr int kBlockM = 128;  // W rows per tile (MMA M)
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = (3 + kEpiWarps) * 32;
+constexpr int kMaxStages = 8;
+constexpr unsigned long long kTimeoutNs = 2000000000ull;
+
+struct GemmParams {
+    int M, N, K, BN, n_tb, n_nb, num_tiles, k_blocks, stages;
+    const float* sx;
+    const float* sw;
+    uint16_t* y;
+    uint32_t* status;
+    int lora;
+    const int32_t* perm;
+    const int32_t* tok_adapter;
+    const int32_t* indptr;
+    const int32_t* active;
+    const int32_t* counts;
+    const float* v;
+    const uint16_t* B;
+    const int32_t* ranks;
+    const float* scales;
+    int n_adapters, r_max, r8;
+    int n_slots;
+    uint32_t ring_off, slots_off, v_off, meta_off, bar_off;
+};
+
+__device__ __forceinline__ unsigned long long globaltimer()
+{
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Bounded wait on an mbarrier phase. Returns false if the CTA is aborting
+// (another role gave up) or if this wait itself timed out (then it raises the
+// abort flag and records `code` in the status word).
+__device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                             uint32_t* status, uint32_t code)
+{
+    if (ptx::mbar_try_wait(bar, parity)) return true;
+    const unsigned long long t0 = globaltimer();
+    while (true) {
+        if (ptx::mbar_try_wait(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if (globaltimer() - t0 > kTimeoutNs) {
+            *abort_flag = 1;
+            if (status) atomicOr(status, code);
+            return false;
+        }
+    }
+}
+// Bounded wait used while draining after an abort (no abort check).
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity)
+{
+    const unsigned long long t0 = globaltimer();
+    while (!ptx::mbar_try_wait(bar, parity))
+        if (globaltimer() - t0 > kTimeoutNs) return;
+}
+
+// UMMA shared-memory descriptor for a K-major operand tile whose rows are
+// SW bytes long (SW = 128 or 64), swizzled by TMA with the same width:
+// 8-row core groups SW*8 bytes apart (stride byte offset), version 1.
+template <int SW>
+__device__ __forceinline__ uint64_t make_desc(uint32_t saddr)
+{
+    constexpr uint64_t layout = (SW == 128) ? 2ull : 4ull;  // SWIZZLE_128B / SWIZZLE_64B
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) |
+           ((uint64_t)((SW * 8) >> 4) << 32) | ((uint64_t)1 << 46) | (layout << 61);
+}
+
+// Instruction descriptor: kind::f8f6f4, A = B = E4M3, both K-major, D fp32,
+// M = 128, N = n.
+__device__ __forceinline__ uint32_t make_idesc(int n)
+{
+    return (1u << 4) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(kBlockM >> 4) << 24);
+}
+
+
+template <int BK, int MAXR>
+__global__ void __launch_bounds__(kThreads, 1)
+fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
+                const __grid_constant__ CUtensorMap tmB, const GemmParams p)
+{
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    __shared__ uint32_t s_tmem;
+    __shared__ int s_abort;
+    __shared__ int s_nslots;
+    __shared__ int s_slot_adapter[256];
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // the swizzled TMA tiles need a 1024-byte aligned base
+    const uint32_t raw_u = ptx::smem_u32(smem_raw);
+    const uint32_t smem_u = (raw_u + 1023u) & ~1023u;
+    uint8_t* smem = smem_raw + (smem_u - raw_u);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + p.bar_off);
+    uint64_t* full = bars;                      // [stages]
+    uint64_t* empty = bars + kMaxStages;        // [stages]
+    uint64_t* tfull = bars + 2 * kMaxStages;    // [2]
+    uint64_t* tempty = tfull + 2;               // [2]
+    uint64_t* bfull = tempty + 2;               // [1]
+    uint64_t* bempty = bfull + 1;               // [1]
+    uint64_t* drain = bempty + 1;               // [1]
+    uint64_t* epibar = drain + 1;               // [1] epilogue-warps barrier
+    volatile int* abort_flag = &s_abort;
+
+    constexpr int kStageW = kBlockM * BK;
+    const int stage_bytes = kStageW + p.BN * BK;
+    const uint32_t ncols = (uint32_t)(2 * p.BN <= 32 ? 32 : (2 * p.BN <= 64 ? 64 : (2 * p.BN <= 128 ? 128 : (2 * p.BN <= 256 ? 256 : 512))));
+
+    if (threadIdx.x == 0) {
+        s_abort = 0;
+        s_nslots = 0;
+        for (int s = 0; s < p.stages; ++s) {
+            ptx::mbar_init(&full[s], 1);
+            ptx::mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            ptx::mbar_init(&tfull[b], 1);
+            ptx::mbar_init(&tempty[b], kEpiWarps);
+        }
+        ptx::mbar_init(bfull, 1);
+        ptx::mbar_init(bempty, kEpiWarps);
+        ptx::mbar_init(drain, 1);
+        ptx::mbar_init(epibar, kEpiWarps);
+        ptx::fence_mbar_init();
+    }
+    if (warp == 1) {
+        ptx::tmem_alloc(&s_tmem, ncols);
+        ptx::tmem_relinquish();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem_base = s_tmem;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            ptx::tma_prefetch_desc(&tmW);
+            ptx::tma_prefetch_desc(&tmX);
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t issued_phase[kMaxStages];
+            bool issued[kMaxStages];
+            for (int s = 0; s < kMaxStages; ++s) issued[s] = false;
+            bool ok = true;
+            for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
+                const int nb = t / p.n_tb, tb = t - nb * p.n_tb;
+                for (int kb = 0; kb < p.k_blocks; ++kb) {
+                    if (!wait_bounded(&empty[stage], phase ^ 1, abort_flag, p.status, 0x1u)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t sW = smem_u + p.ring_off + stage * stage_bytes;
+                    const uint32_t sX = sW + kStageW;
+                    ptx::mbar_arrive_expect_tx(&full[stage], (uint32_t)stage_bytes);
+                    ptx::tma_load_2d(sW, &tmW, &full[stage], kb * BK, nb * kBlockM);
+                    ptx::tma_load_2d(sX, &tmX, &full[stage], kb * BK, tb * p.BN);
+                    issued[stage] = true;
+                    issued_phase[stage] = phase;
+                    if (++stage == p.stages) {
+                        stage = 0;
+                        phase ^= 1;
+                    }
+                }
+            }
+            if (!ok)  // let every load this CTA issued land before it exits
+                for (int s = 0; s < p.stages; ++s)
+                    if (issued[s]) drain_wait(&full[s], issued_phase[s]);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            const uint32_t idesc = make_idesc(p.BN);
+            bool ok = true, any = false;
+            int i = 0;
+            for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x, ++i) {
+                const int buf = i & 1;
+                const uint32_t bphase = (uint32_t)((i >> 1) & 1);
+                if (!wait_bounded(&tempty[buf], bphase ^ 1, abort_flag, p.status, 0x2u)) {
+                    ok = false;
+                    break;
+                }
+                ptx::tc_fence_after();
+                const uint32_t d = tmem_base + (uint32_t)(buf * p.BN);
+                for (int kb = 0; kb < p.k_blocks; ++kb) {
+                    if (!wait_bounded(&full[stage], phase, abort_flag, p.status, 0x4u)) {
+                        ok = false;
+                        break;
+                    }
+                    ptx::tc_fence_after();
+                    const uint32_t sW = smem_u + p.ring_off + stage * stage_bytes;
+                    const uint32_t sX = sW + kStageW;
+#pragma unroll
+                    for (int kk = 0; kk < BK / 32; ++kk)
+                        ptx::tc_mma_f8(d, make_desc<BK>(sW + kk * 32), make_desc<BK>(sX + kk * 32),
+                                       idesc, (kb | kk) != 0 ? 1u : 0u);
+                    any = true;
+                    ptx::tc_commit(&empty[stage]);
+                    if (++stage == p.stages) {
+                        stage = 0;
+                        phase ^= 1;
+                    }
+                }
+                if (ok) ptx::tc_commit(&tfull[buf]);
+            }
+            if (!ok && any) {  // wait for the MMAs in flight before TMEM is freed
+                ptx::tc_commit(drain);
+                drain_wait(drain, 0);
+            }
+        }
+    } else if (warp == 2) {
+        // ------------------------------------------------------------ B stager
+        if (lane == 0 && p.lora) {
+            ptx::tma_prefetch_desc(&tmB);
+            const int n_valid = p.counts[0];
+            const int n_active = p.counts[1];
+            int i = 0;
+            bool pending = false;
+            uint32_t pending_phase = 0;
+            for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x, ++i) {
+                const int nb = t / p.n_tb, tb = t - nb * p.n_tb;
+                if (!wait_bounded(bempty, (uint32_t)((i & 1) ^ 1), abort_flag, p.status, 0x8u)) break;
+                const int p0 = tb * p.BN;
+                const int p1 = min(min(p.M, p0 + p.BN), n_valid);
+                // first active segment that ends after p0
+                int s = 0;
+                {
+                    int lo = 0, hi = n_active;  // first s with indptr[active[s]+1] > p0
+                    while (lo < hi) {
+                        const int mid = (lo + hi) >> 1;
+                        if (p.indptr[p.active[mid] + 1] > p0) hi = mid; else lo = mid + 1;
+                    }
+                    s = lo;
+                }
+                int nslots = 0;
+                uint32_t bytes = 0;
+                for (int s2 = s; s2 < n_active && nslots < p.n_slots; ++s2) {
+                    const int a = p.active[s2];
+                    if (p.indptr[a] >= p1) break;
+                    int r = p.ranks ? p.ranks[a] : p.r_max;
+                    r = max(1, min(r, p.r_max));
+                    bytes += (uint32_t)(((r + 7) >> 3) * 8 * 256);
+                    s_slot_adapter[nslots++] = a;
+                }
+                s_nslots = nslots;
+                if (bytes) ptx::mbar_arrive_expect_tx(bfull, bytes);
+                for (int q = 0; q < nslots; ++q) {
+                    const int a = s_slot_adapter[q];
+                    int r = p.ranks ? p.ranks[a] : p.r_max;
+                    r = max(1, min(r, p.r_max));
+                    const uint32_t dst = smem_u + p.slots_off + (uint32_t)(q * p.r8 * 256);
+                    for (int rb = 0; rb < ((r + 7) >> 3); ++rb)
+                        ptx::tma_load_2d(dst + rb * 2048, &tmB, bfull, nb * kBlockM,
+                                         a * p.r_max + rb * 8);
+                }
+                if (!bytes) ptx::mbar_arrive(bfull);
+                pending = true;
+                pending_phase = (uint32_t)(i & 1);
+            }
+            if (*abort_flag && pending) drain_wait(bfull, pending_phase);
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int ew = warp - 3;
+        const int quarter = warp & 3;         // TMEM lane quarter this warp may access
+        const int grp = ew >> 2;              // which half of the token chunks
+        const int etid = ew * 32 + lane;      // 0..255
+        const int n_local = quarter * 32 + lane;
+        int* s_m = reinterpret_cast<int*>(smem + p.meta_off);
+        int* s_a = s_m + p.BN;
+        float* s_sx = reinterpret_cast<float*>(s_a + p.BN);
+        float* s_v = reinterpret_cast<float*>(smem + p.v_off);
+        const uint16_t* slots = reinterpret_cast<const uint16_t*>(smem + p.slots_off);
+        if (p.lora) ptx::pdl_wait();  // v comes from the kernel this one depends on
+        // barrier among the epilogue warps, bounded like every other wait
+        uint32_t epi_phase = 0;
+        auto epi_sync = [&]() -> bool {
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(epibar);
+            const bool ok = wait_bounded(epibar, epi_phase, abort_flag, p.status, 0x40u);
+            epi_phase ^= 1;
+            return ok;
+        };
+
+        int i = 0;
+        for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x, ++i) {
+            const int nb = t / p.n_tb, tb = t - nb * p.n_tb;
+            const int buf = i & 1;
+            if (i == 0 || p.n_tb > 1) {
+                // stage this token block's metadata (and s_a * v) in shared memory
+                if (i > 0 && !epi_sync()) break;
+                for (int pl = etid; pl < p.BN; pl += kEpiWarps * 32) {
+                    const int pp = tb * p.BN + pl;
+                    int m = 0, a = -1;
+                    float sxp = 0.f;
+                    if (pp < p.M) {
+                        m = p.perm ? p.perm[pp] : pp;
+                        sxp = p.sx[pp];
+                        if (p.lora) a = p.tok_adapter[m];
+                    }
+                    s_m[pl] = m;
+                    s_a[pl] = a;
+                    s_sx[pl] = sxp;
+                    if (p.lora) {
+                        int r = 0;
+                        float sc = 0.f;
+                        if (a >= 0) {
+                            r = p.ranks ? p.ranks[a] : p.r_max;
+                            r = max(0, min(r, p.r_max));
+                            sc = p.scales ? p.scales[a] : 1.f;
+                        }
+                        for (int j = 0; j < p.r8; ++j)
+                            s_v[pl * p.r8 + j] = j < r ? sc * p.v[(size_t)m * p.r_max + j] : 0.f;
+                    }
+                }
+                if (!epi_sync()) break;
+            }
+            if (!wait_bounded(&tfull[buf], (uint32_t)((i >> 1) & 1), abort_flag, p.status, 0x10u))
+                break;
+            ptx::tc_fence_after();
+            if (p.lora && !wait_bounded(bfull, (uint32_t)(i & 1), abort_flag, p.status, 0x20u))
+                break;
+
+            const int n = nb * kBlockM + n_local;
+            const float swn = n < p.N ? p.sw[n] : 0.f;
+            const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * p.BN);
+            const int nslots = p.lora ? s_nslots : 0;
+            int slot = 0, cur_a = -2, cur_r = 0;
+            float breg[MAXR];
+#pragma unroll
+            for (int j = 0; j < MAXR; ++j) breg[j] = 0.f;
+
+            for (int c0 = grp * 16; c0 < p.BN; c0 += 32) {
+                if (tb * p.BN + c0 >= p.M) break;
+                float acc[16];
+                ptx::tmem_ld16(taddr + (uint32_t)c0, acc);
+#pragma unroll 1
+                for (int e = 0; e < 16; ++e) {
+                    const int pl = c0 + e;
+                    if (tb * p.BN + pl >= p.M) break;
+                    float out = acc[e] * s_sx[pl] * swn;
+                    if (p.lora) {
+                        const int a = s_a[pl];
+                        if (a >= 0) {
+                            if (a != cur_a) {
+                                cur_a = a;
+                                int r = p.ranks ? p.ranks[a] : p.r_max;
+                                cur_r = max(0, min(r, p.r_max));
+                                while (slot < nslots && s_slot_adapter[slot] != a) ++slot;
+                                if (slot < nslots) {
+                                    const uint16_t* sb = slots + (size_t)slot * p.r8 * 128 + n_local;
+#pragma unroll
+                                    for (int j = 0; j < MAXR; ++j)
+                                        breg[j] = j < cur_r ? __uint_as_float((uint32_t)sb[j * 128] << 16) : 0.f;
+                                } else {  // not staged: read B from global memory
+                                    const uint16_t* gb = p.B + ((size_t)a * p.r_max) * p.N + n;
+#pragma unroll
+                                    for (int j = 0; j < MAXR; ++j)
+                                        breg[j] = (j < cur_r && n < p.N)
+                                                      ? __uint_as_float((uint32_t)gb[(size_t)j * p.N] << 16)
+                                                      : 0.f;
+                                }
+                            }
+                            const float* vv = s_v + pl * p.r8;
+                            float l = 0.f;
+#pragma unroll
+                            for (int j = 0; j < MAXR; j += 4) {
+                                if (j < p.r8) {
+                                    const float4 v4 = *reinterpret_cast<const float4*>(vv + j);
+                                    l = fmaf(v4.x, breg[j], l);
+                                    l = fmaf(v4.y, breg[j + 1], l);
+                                    l = fmaf(v4.z, breg[j + 2], l);
+                                    l = fmaf(v4.w, breg[j + 3], l);
+                                }
+                            }
+                            out += l;
+                        }
+                    }
+                    if (n < p.N) {
+                        const __nv_bfloat16 o = __float2bfloat16_rn(out);
+                        p.y[(size_t)s_m[pl] * p.N + n] = *reinterpret_cast<const uint16_t*>(&o);
+                    }
+                }
+            }
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                ptx::mbar_arrive(&tempty[buf]);
+                if (p.lora) ptx::mbar_arrive(bempty);
+            }
+        }
+    }
+
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem_base, ncols);
+    }
+}
+
+// ---------------------------------------------------------------- host side
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000,
+                                             cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    }
+    return fn;
+}
+
+bool encode_2d(CUtensorMap* m, CUtensorMapDataType dt, int elem_bytes, const void* base,
+               uint64_t inner, uint64_t outer, uint32_t box_inner, uint32_t box_outer,
+               CUtensorMapSwizzle swz)
+{
+    EncodeTiledFn fn = get_encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {inner, outer};
+    const cuuint64_t strides[1] = {inner * (uint64_t)elem_bytes};
+    const cuuint32_t box[2] = {box_inner, box_outer};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int BK, int MAXR>
+cudaError_t launch_t(const GemmParams& p, const CUtensorMap& tmW, const CUtensorMap& tmX,
+                     const CUtensorMap& tmB, size_t smem, int grid, bool pdl, cudaStream_t stream)
+{
+    cudaError_t e = cudaFuncSetAttribute(fp8_gemm_kernel<BK, MAXR>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, fp8_gemm_kernel<BK, MAXR>, tmW, tmX, tmB, p);
+}
+
+size_t align_up(size_t a, size_t b) { return (a + b - 1) / b * b; }
+
+}  // namespace
+
+int device_sm_count()
+{
+    int dev = 0;
+    cudaGetDevice(&dev);
+    static int cached[64] = {0};
+    if (dev < 64 && cached[dev]) return cached[dev];
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (dev < 64) cached[dev] = n;
+    return n;
+}
+
+cudaError_t launch_fp8_gemm(const Fp8GemmArgs& a, cudaStream_t stream)
+{
+    GemmParams p = {};
+    p.M = a.M;
+    p.N = a.N;
+    p.K = a.K;
+    p.n_tb = (a.M + 255) / 256;
+    p.BN = (((a.M + p.n_tb - 1) / p.n_tb) + 15) / 16 * 16;
+    p.n_nb = (a.N + kBlockM - 1) / kBlockM;
+    p.num_tiles = p.n_nb * p.n_tb;
+    p.sx = a.sx;
+    p.sw = a.sw;
+    p.y = a.y;
+    p.status = a.status;
+    p.lora = a.lora ? 1 : 0;
+    p.perm = a.perm;
+    p.tok_adapter = a.tok_adapter;
+    p.indptr = a.indptr;
+    p.active = a.active;
+    p.counts = a.counts;
+    p.v = a.v;
+    p.B = a.B;
+    p.ranks = a.ranks;
+    p.scales = a.scales;
+    p.n_adapters = a.n_adapters;
+    p.r_max = a.lora ? a.r_max : 0;
+    p.r8 = a.lora ? (a.r_max + 7) / 8 * 8 : 0;
+
+    // shared-memory plan: ring | B slots | v | meta | barriers, within the
+    // opt-in per-block limit minus the kernel's static shared memory
+    int dev = 0, optin = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, fp8_gemm_kernel<128, 64>) != cudaSuccess) return cudaErrorInvalidValue;
+    const size_t kSmemMax = (size_t)(optin > 0 ? optin : 232448) - fa.sharedSizeBytes - 256;
+    const size_t meta = align_up((size_t)p.BN * 12, 128);
+    const size_t vbytes = align_up((size_t)p.BN * p.r8 * 4, 128);
+    const size_t bars = 8 * (2 * kMaxStages + 8);
+    const size_t slot_bytes = (size_t)p.r8 * 256;
+    int want_slots = a.lora ? (a.n_adapters < p.BN ? a.n_adapters : p.BN) : 0;
+    if (want_slots > 256) want_slots = 256;
+    auto fit = [&](int bk, int nslots) -> int {
+        const size_t stage_bytes = (size_t)kBlockM * bk + (size_t)p.BN * bk;
+        const size_t fixed = 1024 + meta + vbytes + bars + (size_t)nslots * slot_bytes;
+        if (fixed >= kSmemMax) return 0;
+        const size_t st = (kSmemMax - fixed) / stage_bytes;
+        return (int)(st > (size_t)kMaxStages ? kMaxStages : st);
+    };
+    // prefer 128-byte k-blocks, then 64-byte ones, with every adapter's B staged
+    // and >= 4 stages; then give up staging slots; then accept 2 stages
+    int BK = 128, slots = want_slots, stages = fit(128, want_slots);
+    if (stages < 4) { BK = 64; stages = fit(64, want_slots); }
+    while (stages < 4 && slots > 0) stages = fit(64, --slots);
+    if (stages < 4) stages = fit(64, 0);
+    if (stages < 2) return cudaErrorInvalidConfiguration;
+    p.stages = stages;
+    p.n_slots = slots;
+    p.k_blocks = (a.K + BK - 1) / BK;
+    const size_t stage_bytes = (size_t)kBlockM * BK + (size_t)p.BN * BK;
+    p.ring_off = 0;
+    p.slots_off = (uint32_t)align_up((size_t)stages * stage_bytes, 1024);
+    p.v_off = (uint32_t)align_up(p.slots_off + (size_t)slots * slot_bytes, 128);
+    p.meta_off = (uint32_t)(p.v_off + vbytes);
+    p.bar_off = (uint32_t)align_up(p.meta_off + meta, 8);
+    const size_t smem = align_up(p.bar_off + bars, 128) + 1024;  // + alignment slack
+
+    CUtensorMap tmW, tmX, tmB;
+    const CUtensorMapSwizzle swz = BK == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+    if (!encode_2d(&tmW, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.Wq, (uint64_t)a.K, (uint64_t)a.N, BK,
+                   kBlockM, swz) ||
+        !encode_2d(&tmX, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.xq, (uint64_t)a.K, (uint64_t)a.M, BK,
+                   (uint32_t)p.BN, swz))
+        return cudaErrorInvalidValue;
+    if (a.lora) {
+        if (!encode_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, a.B, (uint64_t)a.N,
+                       (uint64_t)a.n_adapters * a.r_max, 128, 8, CU_TENSOR_MAP_SWIZZLE_NONE))
+            return cudaErrorInvalidValue;
+    } else {
+        tmB = tmW;  // unused
+    }
+
+    int grid = device_sm_count();
+    if (grid <= 0) grid = 148;
+    if (grid > p.num_tiles) grid = p.num_tiles;
+    const bool small_r = p.r8 <= 16;
+    if (BK == 128)
+        return small_r ? launch_t<128, 16>(p, tmW, tmX, tmB, smem, grid, a.pdl, stream)
+                       : launch_t<128, 64>(p, tmW, tmX, tmB, smem, grid, a.pdl, stream);
+    return small_r ? launch_t<64, 16>(p, tmW, tmX, tmB, smem, grid, a.pdl, stream)
+                   : launch_t<64, 64>(p, tmW, tmX, tmB, smem, grid, a.pdl, stream);
+}
+
+}  // namespace lora

@@ -1,0 +1,54 @@
+// internal.h -- launchers shared between the C-ABI layer (api.cu) and the
+// kernel files. Every launcher enqueues on `stream` and returns the CUDA
+// error of the launch (cudaSuccess when nothing was launched).
+#pragma once
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "lora.h"
+
+namespace lora {
+
+// Kernel files expose these; arguments are validated by api.cu.
+cudaError_t launch_build_segments(const int32_t* ids, int T, int n_adapters,
+                                  const lora_segments_t& seg, cudaStream_t stream);
+
+enum SgmvMode { SGMV_SHRINK = 0, SGMV_EXPAND = 1, SGMV_APPLY = 2 };
+
+// x, v, y may be NULL where the mode does not use them.
+cudaError_t launch_sgmv(int mode, const void* x, int64_t x_slice_stride, const lora_pool_t& pool,
+                        const lora_segments_t& seg, float* v, void* y, cudaStream_t stream,
+                        bool pdl_trigger);
+
+// Per-row E4M3 quantisation; row p of the output is row perm[p] of x
+// (perm == NULL: identity).
+cudaError_t launch_quantize_rows(const void* x, const int32_t* perm, int M, int K, uint8_t* xq,
+                                 float* sx, cudaStream_t stream);
+
+struct Fp8GemmArgs {
+    int M, N, K;
+    const uint8_t* xq;   // e4m3 [M][K], rows in perm order
+    const float* sx;     // [M], perm order
+    const uint8_t* Wq;   // e4m3 [N][K]
+    const float* sw;     // [N]
+    uint16_t* y;         // bf16 [M][N]
+    uint32_t* status;    // device status word
+    // LoRA epilogue (lora == false: base only)
+    bool lora;
+    const int32_t* perm;        // [M]
+    const int32_t* tok_adapter; // [M]
+    const int32_t* indptr;      // [n_adapters+1]
+    const int32_t* active;      // [n_adapters]
+    const int32_t* counts;      // [4]
+    const float* v;             // fp32 [M][r_max], by token index
+    const uint16_t* B;          // bf16 [n_adapters][r_max][N]
+    const int32_t* ranks;
+    const float* scales;
+    int n_adapters, r_max;
+    bool pdl;                   // launch as a programmatic dependent of the previous kernel
+};
+cudaError_t launch_fp8_gemm(const Fp8GemmArgs& a, cudaStream_t stream);
+
+int device_sm_count();
+
+}  // namespace lora

@@ -1,0 +1,78 @@
+// quant.cu -- per-row FP8 (E4M3) quantisation for the 8-bit base GEMM.
+//
+// The pages make the base GEMM 8-bit (EpiLoRA abstract, sentence 2) without
+// fixing the scaling; rows are scaled by amax/448 so the largest magnitude of
+// each row lands on the largest finite E4M3 value, then rounded to nearest
+// even with saturation. One CTA per output row; both divisions are IEEE
+// binary32 divisions rounded to nearest (__fdiv_rn), so the result does not
+// depend on compiler flags.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace lora {
+namespace {
+
+constexpr int kThreads = 256;
+
+__global__ void __launch_bounds__(kThreads)
+quantize_rows_kernel(const uint16_t* __restrict__ x, const int32_t* __restrict__ perm, int K,
+                     uint8_t* __restrict__ xq, float* __restrict__ sx)
+{
+    __shared__ float s_red[kThreads / 32];
+    const int prow = blockIdx.x;
+    const int row = perm ? perm[prow] : prow;
+    const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)row * K);
+    const int n16 = K >> 3;  // 8 bf16 per 16-byte chunk
+
+    float amax = 0.f;
+    for (int i = threadIdx.x; i < n16; i += kThreads) {
+        const uint4 c = src[i];
+        const uint32_t w[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            amax = fmaxf(amax, fabsf(__uint_as_float(w[e] << 16)));
+            amax = fmaxf(amax, fabsf(__uint_as_float(w[e] & 0xffff0000u)));
+        }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+    if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = amax;
+    __syncthreads();
+    amax = s_red[0];
+#pragma unroll
+    for (int i = 1; i < kThreads / 32; ++i) amax = fmaxf(amax, s_red[i]);
+    const float s = (amax == 0.f) ? 1.f : __fdiv_rn(amax, 448.f);
+    if (threadIdx.x == 0) sx[prow] = s;
+
+    uint2* dst = reinterpret_cast<uint2*>(xq + (size_t)prow * K);
+    for (int i = threadIdx.x; i < n16; i += kThreads) {
+        const uint4 c = src[i];
+        const uint32_t w[4] = {c.x, c.y, c.z, c.w};
+        uint32_t out[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const float a0 = __fdiv_rn(__uint_as_float(w[2 * e] << 16), s);
+            const float a1 = __fdiv_rn(__uint_as_float(w[2 * e] & 0xffff0000u), s);
+            const float a2 = __fdiv_rn(__uint_as_float(w[2 * e + 1] << 16), s);
+            const float a3 = __fdiv_rn(__uint_as_float(w[2 * e + 1] & 0xffff0000u), s);
+            out[e] = (uint32_t)ptx::cvt_e4m3x2(a0, a1) | ((uint32_t)ptx::cvt_e4m3x2(a2, a3) << 16);
+        }
+        dst[i] = make_uint2(out[0], out[1]);
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_quantize_rows(const void* x, const int32_t* perm, int M, int K, uint8_t* xq,
+                                 float* sx, cudaStream_t stream)
+{
+    if (M == 0) return cudaSuccess;
+    quantize_rows_kernel<<<M, kThreads, 0, stream>>>(static_cast<const uint16_t*>(x), perm, K, xq,
+                                                      sx);
+    return cudaGetLastError();
+}
+
+}  // namespace lora

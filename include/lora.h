@@ -1,0 +1,237 @@
+/*
+ * lora.h -- C ABI of liblora, the multi-tenant LoRA hot path on B200 (sm_100a).
+ *
+ * The problem (Punica README, section "How?"): a base weight W and, for n
+ * adapters, LoRA matrices A_i [h_in, r_i] and B_i [r_i, h_out]. A batch X of
+ * tokens maps token by token to adapters, and the output is
+ *     Y = X.W + (x_1.A_1.B_1, ..., x_n.A_n.B_n),
+ * here with a per-adapter scale s_i on the added term. Every token carries an
+ * adapter id; -1 means "base model only" (EpiLoRA abstract, sentence 1: one
+ * base copy serves the requests of many tenants, each with its own adapter).
+ * The added term is computed as a shrink, v = x.A_i (rank r_i, fp32), and an
+ * expand, y += s_i.v.B_i: SGMV for runs of tokens that share an adapter, BGMV
+ * for one adapter per decode token (Punica README, "How?": Segmented Gather
+ * Matrix-Vector multiplication). fp8_gemm_lora_epilogue() fuses the expand
+ * into the epilogue of an 8-bit base GEMM whose down-projection is launched
+ * first while the GEMM streams its weights (EpiLoRA abstract, sentences 3-4).
+ *
+ * Conventions for every call:
+ *   - All array arguments are DEVICE pointers owned by the caller, unless a
+ *     comment says "host". The library never allocates device memory; calls
+ *     that need scratch space take a caller-owned workspace whose size comes
+ *     from lora_workspace_size() (the Punica README's file listing records the
+ *     same choice for SGMV: "use preallocated buffer").
+ *   - bf16 arrays hold IEEE bfloat16 bit patterns; "e4m3" arrays hold OCP FP8
+ *     E4M3 codes. Matrices are row-major with the last index contiguous.
+ *   - Calls are ordered on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and return once the work is enqueued. Errors that the host can
+ *     see (NULL pointers, bad sizes, misalignment, unsupported shapes, launch
+ *     failures) are returned before or instead of any launch; nothing is
+ *     thrown across the ABI.
+ *   - Pointers to bf16/e4m3/fp32 arrays must be 16-byte aligned, and every row
+ *     length in bytes a multiple of 16 (so h_in, h_out, r_max, K must be
+ *     multiples of 8 for bf16 rows, K a multiple of 16 for e4m3 rows).
+ *   - Adapter ids outside [-1, n_adapters) are counted as bad and served as
+ *     -1 (see lora_build_segments).
+ */
+#ifndef LORA_H_
+#define LORA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define LORA_API __attribute__((visibility("default")))
+#else
+#define LORA_API
+#endif
+
+struct CUstream_st;
+typedef struct CUstream_st* lora_stream_t; /* same object as cudaStream_t */
+
+typedef enum {
+    LORA_OK = 0,
+    LORA_ERR_INVALID_ARG = 1,    /* NULL pointer, size <= 0, misaligned pointer/stride */
+    LORA_ERR_UNSUPPORTED = 2,    /* shape outside the implemented limits below */
+    LORA_ERR_BAD_ADAPTER_ID = 3, /* sync_check found ids outside [-1, n_adapters) */
+    LORA_ERR_CUDA = 4,           /* a CUDA runtime call or launch failed */
+    LORA_ERR_WORKSPACE = 5,      /* workspace NULL or smaller than lora_workspace_size() */
+    LORA_ERR_TIMEOUT = 6         /* a bounded device-side wait gave up (see lora_workspace_status) */
+} lora_status_t;
+
+/* Implemented limits. */
+#define LORA_TILE_TOKENS 64    /* tokens per work tile of one adapter segment */
+#define LORA_MAX_RANK 64       /* largest r_max */
+#define LORA_MAX_ADAPTERS 16384
+
+/*
+ * Stacked adapter pool (the pages' per-adapter A_i, B_i, stacked; the
+ * `n_slices` dimension holds several projections that share the token ids,
+ * e.g. q/k/v/o of one layer, applied in one call).
+ *   A      bf16 [n_slices][n_adapters][h_in][r_max]
+ *   B      bf16 [n_slices][n_adapters][r_max][h_out]
+ *   ranks  int32 [n_adapters], each in 1..r_max; NULL = every adapter has rank r_max.
+ *          Entries of A with column >= r_i and of B with row >= r_i are never read.
+ *   scales fp32 [n_adapters] (s_i); NULL = 1.0.
+ */
+typedef struct {
+    const void* A;
+    const void* B;
+    const int32_t* ranks;
+    const float* scales;
+    int32_t n_slices;
+    int32_t n_adapters;
+    int32_t h_in;
+    int32_t h_out;
+    int32_t r_max;
+} lora_pool_t;
+
+/*
+ * Token grouping produced by lora_build_segments (device arrays, caller-owned,
+ * filled by the call). For a batch of T tokens:
+ *   perm        int32 [T]: token indices with a valid id, by ascending id and
+ *               ascending token index within an id; then the tokens without an
+ *               adapter, ascending.
+ *   indptr      int32 [n_adapters+1]: adapter a owns perm[indptr[a] .. indptr[a+1]);
+ *               indptr[n_adapters] = number of tokens with an adapter.
+ *   active      int32 [n_adapters]: ids with >= 1 token, ascending; -1 after n_active.
+ *   tile_ptr    int32 [n_adapters+1]: prefix sums over active segments of
+ *               ceil(count / LORA_TILE_TOKENS); entries past n_active hold the total.
+ *   tok_adapter int32 [T]: the id each token is served with (-1: none or bad id).
+ *   counts      int32 [4]: n_valid, n_active, n_bad_ids, n_tiles.
+ * T and n_adapters are host values describing the arrays.
+ */
+typedef struct {
+    int32_t* perm;
+    int32_t* indptr;
+    int32_t* active;
+    int32_t* tile_ptr;
+    int32_t* tok_adapter;
+    int32_t* counts;
+    int32_t T;
+    int32_t n_adapters;
+} lora_segments_t;
+
+/* Operation codes for lora_workspace_size. */
+#define LORA_OP_SHRINK 0
+#define LORA_OP_EXPAND 1
+#define LORA_OP_APPLY 2
+#define LORA_OP_FP8_GEMM 3
+
+/*
+ * Bytes of workspace an operation needs (0 if it needs none), or (size_t)-1
+ * for invalid arguments. For LORA_OP_FP8_GEMM, T is the
+ * token count M and `K` the GEMM's reduction size; `pool` may be NULL (no
+ * LoRA). The other operations ignore K.
+ * A workspace must be zeroed once after allocation (lora_workspace_init);
+ * afterwards the library keeps it in a reusable state.
+ */
+LORA_API size_t lora_workspace_size(int op, int T, int K, const lora_pool_t* pool);
+
+/* Zero a freshly allocated workspace (stream-ordered memset). */
+LORA_API int lora_workspace_init(void* ws, size_t ws_bytes, lora_stream_t stream);
+
+/*
+ * Read and clear the device status word of a workspace: synchronises
+ * `stream`, returns LORA_OK, or LORA_ERR_TIMEOUT if a kernel that used this
+ * workspace gave up on a bounded wait since the last query (its output is
+ * then undefined). *detail (host, may be NULL) receives the raw status word.
+ */
+LORA_API int lora_workspace_status(void* ws, size_t ws_bytes, lora_stream_t stream, uint32_t* detail);
+
+/*
+ * Group the tokens of one batch by adapter (the segments of SGMV; Punica
+ * README, "How?"). ids int32 [T] (device). Fills every array of *seg, whose
+ * T and n_adapters must equal the arguments. One single-CTA kernel: a stable
+ * counting sort, bit-exact and deterministic. Built once per batch and shared
+ * by every layer and projection of that batch.
+ * sync_check != 0: synchronise the stream and return LORA_ERR_BAD_ADAPTER_ID if
+ * any id was outside [-1, n_adapters). Without it, bad ids are only counted
+ * (counts[2]) and served as -1.
+ * T may be 0 (every output describes an empty batch). Limits: n_adapters <=
+ * LORA_MAX_ADAPTERS, T < 2^30.
+ */
+LORA_API int lora_build_segments(const int32_t* ids, int T, int n_adapters, const lora_segments_t* seg,
+                        int sync_check, lora_stream_t stream);
+
+/*
+ * Shrink (down-projection), for every slice s and token t with adapter a:
+ *   v[s][t][j] = sum_k x[s][t][k] * A[s][a][k][j]   for j < r_a  (fp32 accumulate)
+ *   v[s][t][j] = 0                                    for r_a <= j < r_max.
+ * Rows of tokens without an adapter are not written.
+ *   x  bf16 [n_slices][T][h_in], slice s at x + s * x_slice_stride elements
+ *      (x_slice_stride = 0 lets all slices share one x; otherwise >= T*h_in and
+ *      a multiple of 8).
+ *   v  fp32 [n_slices][T][r_max].
+ * Needs no workspace (ws may be NULL, ws_bytes 0). One kernel launch.
+ */
+LORA_API int lora_shrink(const void* x, int64_t x_slice_stride, const lora_pool_t* pool,
+                const lora_segments_t* seg, float* v, void* ws, size_t ws_bytes,
+                lora_stream_t stream);
+
+/*
+ * Expand (up-projection), in place on y, for every slice s and token t with adapter a:
+ *   y[s][t][n] = bf16( fp32(y[s][t][n]) + s_a * sum_{j < r_a} v[s][t][j] * B[s][a][j][n] )
+ * (one rounding, to nearest even); rows of tokens without an adapter are untouched.
+ *   v  fp32 [n_slices][T][r_max];  y bf16 [n_slices][T][h_out] (in/out).
+ * Needs no workspace. One kernel launch.
+ */
+LORA_API int lora_expand(const float* v, const lora_pool_t* pool, const lora_segments_t* seg, void* y,
+                void* ws, size_t ws_bytes, lora_stream_t stream);
+
+/*
+ * Shrink then expand (y += s_a * (x.A_a).B_a), with v kept on chip in fp32:
+ * one kernel launch, no workspace. Arguments as lora_shrink / lora_expand.
+ */
+LORA_API int lora_apply(const void* x, int64_t x_slice_stride, const lora_pool_t* pool,
+               const lora_segments_t* seg, void* y, void* ws, size_t ws_bytes,
+               lora_stream_t stream);
+
+/*
+ * Per-row FP8 quantisation (the activation step of the 8-bit GEMM; also used
+ * offline for weights with one scale per output channel):
+ *   sx[m] = fl32(amax_k |x[m][k]| / 448), or 1 if the row is all zero;
+ *   xq[m][k] = E4M3(fl32(x[m][k] / sx[m])), round to nearest even, saturating.
+ *   x bf16 [M][K]; xq e4m3 [M][K]; sx fp32 [M]. One kernel launch.
+ */
+LORA_API int fp8_quantize_rows(const void* x, int M, int K, uint8_t* xq, float* sx, lora_stream_t stream);
+
+/*
+ * 8-bit base GEMM with the LoRA expand fused into its epilogue (EpiLoRA
+ * abstract, sentences 3-4):
+ *   y[m][n] = bf16( sx[m] * w_scale[n] * sum_k xq[m][k] * Wq[n][k]
+ *                   + s_a * sum_{j < r_a} v[m][j] * B[0][a][j][n] ),
+ *   a = seg->tok_adapter[m]; the LoRA term is absent when a == -1 or pool == NULL;
+ *   xq, sx: x quantised per token as in fp8_quantize_rows;
+ *   v = x.A_a in fp32 from the unquantised bf16 x (as lora_shrink).
+ * Launch order: the activation quantiser, then the shrink (the
+ * down-projection, launched first as the page describes), then the GEMM as a
+ * programmatic dependent launch: its mainloop starts streaming Wq while the
+ * shrink runs and it waits for v only before its epilogue.
+ *   x bf16 [M][K]; Wq e4m3 [N][K]; w_scale fp32 [N]; y bf16 [M][N] (out).
+ *   pool: NULL for the base GEMM alone; else n_slices == 1, h_in == K, h_out == N.
+ *   seg: required when pool != NULL (built for these M tokens); may be NULL otherwise.
+ *   ws: lora_workspace_size(LORA_OP_FP8_GEMM, M, K, pool) bytes.
+ * Limits: K % 16 == 0, N % 8 == 0, M >= 1.
+ */
+LORA_API int fp8_gemm_lora_epilogue(const void* x, int M, int K, int N, const uint8_t* Wq,
+                           const float* w_scale, const lora_pool_t* pool,
+                           const lora_segments_t* seg, void* y, void* ws, size_t ws_bytes,
+                           lora_stream_t stream);
+
+/* Static string for a status code. */
+LORA_API const char* lora_status_string(int status);
+
+/* Library version, and the tile size kernels assume for lora_segments_t.tile_ptr. */
+LORA_API int lora_version(void);
+LORA_API int lora_tile_tokens(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LORA_H_ */

@@ -105,18 +105,24 @@ def e4m3_encode(f: float) -> int:
     return int(_load().orc_e4m3_encode(float(f)))
 
 
+_tables = {}
+
+
+def _table(name, n):
+    if name not in _tables:
+        f = getattr(_load(), name)
+        _tables[name] = np.array([f(i) for i in range(n)], dtype=np.float64)
+    return _tables[name]
+
+
 def bf16_to_f64(a: np.ndarray) -> np.ndarray:
-    """Decode an array of bf16 bit patterns (uint16) to fp64, element by element."""
-    lib = _load()
+    """Decode an array of bf16 bit patterns (uint16) to fp64 with orc_bf16_decode."""
     flat = np.asarray(a, dtype=np.uint16).ravel()
-    table = np.array([lib.orc_bf16_decode(i) for i in range(65536)], dtype=np.float64)
-    return table[flat].reshape(np.shape(a))
+    return _table("orc_bf16_decode", 65536)[flat].reshape(np.shape(a))
 
 
 def e4m3_to_f64(a: np.ndarray) -> np.ndarray:
-    lib = _load()
-    table = np.array([lib.orc_e4m3_decode(i) for i in range(256)], dtype=np.float64)
-    return table[np.asarray(a, dtype=np.uint8)]
+    return _table("orc_e4m3_decode", 256)[np.asarray(a, dtype=np.uint8)]
 
 
 def build_segments(ids: np.ndarray, n_adapters: int, tile_t: int) -> dict:

@@ -1,0 +1,244 @@
+"""GPU parity of the segment builder and the SGMV shrink / expand / apply kernels
+against the fp64 oracle, through the C ABI, on seeded inputs (workloads.py).
+
+Tolerance (the stated bar for bf16 inputs with fp32 accumulation):
+max |gpu - oracle| <= 2e-2 * (1 + |oracle|) elementwise. Integer work (the
+segments) is bit-exact; small-integer inputs make the float results exact, so
+there the GPU must equal the oracle rounded once to bf16."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from adapter_gemm_builder_b200 import lora as L
+from adapter_gemm_builder_b200 import workloads as wl
+from gpu_util import (TOL_BF16, DeviceProblem, assert_close, dev, dev_bf16, f64, host_bf16_bits,
+                      oracle_apply, rne_bf16_bits)
+
+pytestmark = pytest.mark.gpu
+TT = 64
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a GPU")
+    L.load()
+
+
+# ------------------------------------------------------------------ segments
+
+def _check_segments(ids, n_adapters):
+    T = len(ids)
+    seg = L.Segments(T, n_adapters)
+    L.lora_build_segments(dev(ids) if T else torch.empty(0, dtype=torch.int32, device="cuda"),
+                          n_adapters, seg)
+    torch.cuda.synchronize()
+    want = oracle.build_segments(ids, n_adapters, TT)
+    counts = seg.counts.cpu().numpy()
+    assert counts.tolist() == want["counts"].tolist()
+    assert seg.indptr.cpu().numpy().tolist() == want["indptr"].tolist()
+    assert seg.active.cpu().numpy().tolist() == want["active"].tolist()
+    assert seg.tile_ptr.cpu().numpy().tolist() == want["tile_ptr"].tolist()
+    if T:
+        assert seg.perm.cpu().numpy()[:T].tolist() == want["perm"].tolist()
+        assert seg.tok_adapter.cpu().numpy()[:T].tolist() == want["tok_adapter"].tolist()
+
+
+@pytest.mark.parametrize("kind,T,n", [
+    ("distinct", 36, 32), ("identical", 36, 32), ("uniform", 1000, 7), ("zipf", 512, 256),
+    ("sorted_zipf", 2300, 8), ("uniform", 5000, 3000), ("zipf", 4097, 1), ("uniform", 1, 5),
+    ("zipf", 70000, 16384),
+])
+def test_segments_bitexact(kind, T, n):
+    rng = np.random.default_rng(T + n)
+    ids = wl.make_ids(kind if kind != "distinct" else "distinct", rng, T, n,
+                      none_frac=0.05 if kind != "identical" else 0.0)
+    _check_segments(ids, n)
+
+
+def test_segments_edge_cases():
+    _check_segments(np.zeros(0, np.int32), 4)               # empty batch
+    _check_segments(np.full(300, -1, np.int32), 9)          # nobody has an adapter
+    rng = np.random.default_rng(3)
+    bad = rng.integers(-5, 15, size=777).astype(np.int32)    # out-of-range ids
+    _check_segments(bad, 10)
+
+
+def test_segments_sync_check_reports_bad_ids():
+    ids = np.array([0, 1, 7, -1, 2], np.int32)
+    seg = L.Segments(5, 3)
+    with pytest.raises(L.LoraError) as e:
+        L.lora_build_segments(dev(ids), 3, seg, sync_check=True)
+    assert e.value.status == L.LORA_ERR_BAD_ADAPTER_ID
+    L.lora_build_segments(dev(np.array([0, -1, 2], np.int32)), 3, L.Segments(3, 3),
+                          sync_check=True)
+
+
+# ------------------------------------------------------------------ problems
+
+def _small(seed, T=150, n_adapters=6, h_in=520, h_out=392, r_max=24, kind="zipf", n_slices=1,
+           rank_choices=(1, 5, 8, 13, 24), none_frac=0.1):
+    return wl.make_lora_problem("t", seed, T=T, n_adapters=n_adapters, h_in=h_in, h_out=h_out,
+                                r_max=r_max, ids_kind=kind, none_frac=none_frac,
+                                rank_choices=rank_choices, n_slices=n_slices)
+
+
+SMALL_CASES = {
+    "ragged_mixed_ranks": dict(seed=11),
+    "multi_tile_segment": dict(seed=12, T=300, n_adapters=3, kind="sorted_zipf"),
+    "decode_distinct": dict(seed=13, T=40, n_adapters=48, kind="distinct", h_in=2048,
+                            h_out=1024, r_max=16, rank_choices=(16,)),
+    "rank64_slices": dict(seed=14, T=90, n_adapters=9, r_max=64, rank_choices=(8, 16, 32, 64),
+                          n_slices=3, h_in=640, h_out=512),
+    "tiny_dims": dict(seed=15, T=7, n_adapters=2, h_in=8, h_out=8, r_max=8, rank_choices=(3, 8)),
+    "single_token": dict(seed=16, T=1, n_adapters=1, none_frac=0.0),
+}
+
+
+@pytest.mark.parametrize("case", list(SMALL_CASES))
+def test_apply_parity_small(case):
+    p = _small(**SMALL_CASES[case])
+    d = DeviceProblem(p)
+    y = d.y_in()
+    L.lora_apply(d.x, d.pool, d.seg, y)
+    torch.cuda.synchronize()
+    got = f64(host_bf16_bits(y))
+    want = oracle_apply(p)
+    assert_close(got, want, TOL_BF16, case)
+    none = p.ids == -1
+    assert np.array_equal(host_bf16_bits(y)[:, none], p.y_in[:, none])  # untouched, bit-exact
+
+
+@pytest.mark.parametrize("case", list(SMALL_CASES))
+def test_shrink_parity_small(case):
+    p = _small(**SMALL_CASES[case])
+    d = DeviceProblem(p)
+    v = torch.full((p.n_slices, p.T, p.r_max), float("nan"), device="cuda")
+    L.lora_shrink(d.x, d.pool, d.seg, v)
+    torch.cuda.synchronize()
+    got = v.cpu().numpy().astype(np.float64)
+    for s in range(p.n_slices):
+        want = oracle.lora_shrink(p.x[s], p.A[s], p.ranks, p.ids)
+        has = p.ids >= 0
+        assert_close(got[s][has], want[has], TOL_BF16, f"{case} slice {s}")
+        assert np.isnan(got[s][~has]).all()  # rows without an adapter are not written
+
+
+@pytest.mark.parametrize("case", list(SMALL_CASES))
+def test_expand_parity_small(case):
+    p = _small(**SMALL_CASES[case])
+    d = DeviceProblem(p)
+    rng = np.random.default_rng(99)
+    v = rng.standard_normal((p.n_slices, p.T, p.r_max)).astype(np.float32)
+    y = d.y_in()
+    L.lora_expand(dev(v), d.pool, d.seg, y)
+    torch.cuda.synchronize()
+    got = f64(host_bf16_bits(y))
+    for s in range(p.n_slices):
+        want = oracle.lora_expand(v[s], p.B[s], p.ranks, p.scales, p.ids, p.y_in[s])
+        assert_close(got[s], want, TOL_BF16, f"{case} slice {s}")
+
+
+def test_apply_exact_small_integers():
+    """Small-integer inputs: every product and sum is exact in fp32, so the GPU
+    result must equal the exact value rounded once to bf16."""
+    rng = np.random.default_rng(5)
+    T, n_adapters, h_in, h_out, r_max = 130, 5, 1024, 264, 32
+    p = _small(21, T=T, n_adapters=n_adapters, h_in=h_in, h_out=h_out, r_max=r_max,
+               rank_choices=(3, 16, 32))
+    p.x[:] = wl.to_bf16_bits(rng.integers(-2, 3, size=p.x.shape).astype(np.float32))
+    for a in range(n_adapters):
+        r = p.ranks[a]
+        p.A[:, a, :, :r] = wl.to_bf16_bits(rng.integers(-2, 3, size=(1, h_in, r)).astype(np.float32))
+        p.B[:, a, :r, :] = wl.to_bf16_bits(rng.integers(-2, 3, size=(1, r, h_out)).astype(np.float32))
+    p.y_in[:] = wl.to_bf16_bits(rng.integers(-8, 9, size=p.y_in.shape).astype(np.float32))
+    p.scales[:] = 2.0
+    d = DeviceProblem(p)
+    y = d.y_in()
+    L.lora_apply(d.x, d.pool, d.seg, y)
+    v = torch.zeros((1, T, r_max), device="cuda")
+    L.lora_shrink(d.x, d.pool, d.seg, v)
+    torch.cuda.synchronize()
+    want = oracle_apply(p)
+    assert np.array_equal(host_bf16_bits(y), rne_bf16_bits(want))
+    v_want = oracle.lora_shrink(p.x[0], p.A[0], p.ranks, p.ids)
+    has = p.ids >= 0
+    assert np.array_equal(v.cpu().numpy()[0][has].astype(np.float64), v_want[has])
+
+
+def test_apply_invariants_on_gpu():
+    p = _small(31, T=200, n_adapters=8, h_in=512, h_out=256, r_max=16, rank_choices=(16,))
+    d = DeviceProblem(p)
+    # B = 0 leaves y unchanged, bit for bit
+    zB = L.Pool(d.A, torch.zeros_like(d.B), d.ranks, d.scales)
+    y = d.y_in()
+    L.lora_apply(d.x, zB, d.seg, y)
+    torch.cuda.synchronize()
+    assert np.array_equal(host_bf16_bits(y), p.y_in)
+    # permuting tokens permutes outputs
+    y1 = d.y_in()
+    L.lora_apply(d.x, d.pool, d.seg, y1)
+    pi = np.random.default_rng(1).permutation(p.T)
+    p2 = wl.LoraProblem("perm", p.x[:, pi], p.A, p.B, p.ids[pi], p.ranks, p.scales, p.y_in[:, pi])
+    d2 = DeviceProblem(p2)
+    y2 = d2.y_in()
+    L.lora_apply(d2.x, d2.pool, d2.seg, y2)
+    torch.cuda.synchronize()
+    assert_close(f64(host_bf16_bits(y2)), f64(host_bf16_bits(y1))[:, pi], TOL_BF16, "permutation")
+
+
+def test_shared_x_across_slices():
+    p = _small(41, T=64, n_slices=3, h_in=256, h_out=128, r_max=16, rank_choices=(16,))
+    p.x[1] = p.x[0]
+    p.x[2] = p.x[0]
+    d = DeviceProblem(p)
+    y = d.y_in()
+    L.lora_apply(d.x[0], d.pool, d.seg, y, x_slice_stride=0)
+    torch.cuda.synchronize()
+    assert_close(f64(host_bf16_bits(y)), oracle_apply(p), TOL_BF16, "shared x")
+
+
+# ------------------------------------------------------------------ the named workloads, full size
+
+def test_sgmv_tiny_full():
+    p = wl.sgmv_tiny()
+    d = DeviceProblem(p)
+    y = d.y_in()
+    L.lora_apply(d.x, d.pool, d.seg, y)
+    torch.cuda.synchronize()
+    assert_close(f64(host_bf16_bits(y)), oracle_apply(p), TOL_BF16, "sgmv_tiny")
+
+
+@pytest.mark.parametrize("kind", ["distinct", "identical"])
+def test_bgmv_decode_full(kind):
+    p = wl.bgmv_decode(ids_kind=kind)
+    d = DeviceProblem(p)
+    y = d.y_in()
+    L.lora_apply(d.x, d.pool, d.seg, y)
+    torch.cuda.synchronize()
+    assert_close(f64(host_bf16_bits(y)), oracle_apply(p), TOL_BF16, f"bgmv_decode {kind}")
+
+
+def test_sgmv_prefill_full_sampled_tokens():
+    p = wl.sgmv_prefill()
+    d = DeviceProblem(p)
+    y = d.y_in()
+    L.lora_apply(d.x, d.pool, d.seg, y)
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(0)
+    rows = np.sort(rng.choice(p.T, size=192, replace=False))
+    # include the first and last token of every segment (tile boundaries)
+    starts = np.concatenate([[0], np.cumsum(np.bincount(p.ids))])
+    rows = np.unique(np.concatenate([rows, starts[:-1], starts[1:] - 1]))
+    got = f64(host_bf16_bits(y))[:, rows]
+    assert_close(got, oracle_apply(p, rows=rows), TOL_BF16, "sgmv_prefill")
+
+
+def test_many_tenants_full():
+    p = wl.many_tenants()
+    d = DeviceProblem(p)
+    y = d.y_in()
+    L.lora_apply(d.x, d.pool, d.seg, y)
+    torch.cuda.synchronize()
+    assert_close(f64(host_bf16_bits(y)), oracle_apply(p), TOL_BF16, "many_tenants")

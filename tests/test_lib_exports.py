@@ -1,0 +1,154 @@
+"""The C-ABI library builds for sm_100a, loads, and exports every symbol that
+include/lora.h declares; host-side argument checks answer before any launch.
+No compute call is made here (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from adapter_gemm_builder_b200 import build as lbuild
+from adapter_gemm_builder_b200 import lora as L
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    lbuild.build()
+    return L.load()
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "lora.h")).read()
+    return re.findall(r"LORA_API\s+[\w\s\*]+?\b(\w+)\s*\(", src)
+
+
+def test_header_declares_the_boundary():
+    names = set(_declared())
+    for n in ["lora_build_segments", "lora_shrink", "lora_expand", "lora_apply",
+              "fp8_gemm_lora_epilogue"]:
+        assert n in names
+    assert names == set(L.EXPORTED)
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in _declared():
+        assert hasattr(lib, name), name
+        assert ctypes.cast(getattr(lib, name), ctypes.c_void_p).value
+
+
+def test_library_is_sm100a_only():
+    # every object is compiled with -gencode arch=compute_100a,code=sm_100a
+    assert lbuild.ARCH == ["-gencode", "arch=compute_100a,code=sm_100a"]
+
+
+def test_version_and_constants(lib):
+    assert lib.lora_version() >= 1
+    assert lib.lora_tile_tokens() == 64
+    assert lib.lora_status_string(L.LORA_ERR_TIMEOUT).decode()
+
+
+def _pool(**kw):
+    d = dict(A=16, B=32, ranks=None, scales=None, n_slices=1, n_adapters=4, h_in=64, h_out=64,
+             r_max=16)
+    d.update(kw)
+    return L.lora_pool_t(d["A"], d["B"], d["ranks"], d["scales"], d["n_slices"], d["n_adapters"],
+                         d["h_in"], d["h_out"], d["r_max"])
+
+
+def test_workspace_sizes(lib):
+    assert lib.lora_workspace_size(L.LORA_OP_APPLY, 10, 0, None) == 0
+    assert lib.lora_workspace_size(L.LORA_OP_SHRINK, 10, 0, None) == 0
+    p = _pool(h_in=8192, h_out=28672)
+    n = lib.lora_workspace_size(L.LORA_OP_FP8_GEMM, 256, 8192, ctypes.byref(p))
+    assert n >= 256 + 256 * 8192 + 256 * 4 + 256 * 16 * 4
+    n0 = lib.lora_workspace_size(L.LORA_OP_FP8_GEMM, 256, 8192, None)
+    assert n0 < n
+    assert lib.lora_workspace_size(99, 1, 1, None) == ctypes.c_size_t(-1).value
+    assert lib.lora_workspace_size(L.LORA_OP_FP8_GEMM, 4, 0, None) == ctypes.c_size_t(-1).value
+
+
+def _seg(T=8, n=4):
+    return L.lora_segments_t(16, 32, 48, 64, 80, 96, T, n)
+
+
+@pytest.mark.parametrize("bad,code", [
+    (dict(r_max=72), L.LORA_ERR_UNSUPPORTED),
+    (dict(r_max=12), L.LORA_ERR_INVALID_ARG),
+    (dict(h_in=100), L.LORA_ERR_INVALID_ARG),
+    (dict(A=None), L.LORA_ERR_INVALID_ARG),
+    (dict(A=24), L.LORA_ERR_INVALID_ARG),            # misaligned
+    (dict(n_adapters=0), L.LORA_ERR_INVALID_ARG),
+    (dict(n_adapters=20000), L.LORA_ERR_UNSUPPORTED),
+])
+def test_pool_checks_before_launch(lib, bad, code):
+    p = _pool(**bad)
+    s = _seg(n=p.n_adapters)
+    st = lib.lora_apply(ctypes.c_void_p(1024), 0, ctypes.byref(p), ctypes.byref(s),
+                        ctypes.c_void_p(2048), None, 0, None)
+    assert st == code
+
+
+def test_segment_and_pointer_checks(lib):
+    p = _pool()
+    s = _seg(n=5)  # n_adapters mismatch
+    assert lib.lora_shrink(ctypes.c_void_p(1024), 0, ctypes.byref(p), ctypes.byref(s),
+                           ctypes.c_void_p(2048), None, 0, None) == L.LORA_ERR_INVALID_ARG
+    s = _seg()
+    assert lib.lora_shrink(None, 0, ctypes.byref(p), ctypes.byref(s), ctypes.c_void_p(2048), None,
+                           0, None) == L.LORA_ERR_INVALID_ARG
+    assert lib.lora_shrink(ctypes.c_void_p(1024), 12, ctypes.byref(p), ctypes.byref(s),
+                           ctypes.c_void_p(2048), None, 0, None) == L.LORA_ERR_INVALID_ARG
+    assert lib.lora_expand(ctypes.c_void_p(1028), ctypes.byref(p), ctypes.byref(s),
+                           ctypes.c_void_p(2048), None, 0, None) == L.LORA_ERR_INVALID_ARG
+    # empty batch: nothing to do, no launch
+    s0 = _seg(T=0)
+    assert lib.lora_apply(ctypes.c_void_p(1024), 0, ctypes.byref(p), ctypes.byref(s0),
+                          ctypes.c_void_p(2048), None, 0, None) == L.LORA_OK
+
+
+def test_fp8_checks_before_launch(lib):
+    x, w, sw, y = (ctypes.c_void_p(v) for v in (1024, 2048, 4096, 8192))
+    ws = ctypes.c_void_p(16384)
+    # K not a multiple of 16
+    assert lib.fp8_gemm_lora_epilogue(x, 4, 24, 64, w, sw, None, None, y, ws, 1 << 20,
+                                      None) == L.LORA_ERR_INVALID_ARG
+    # workspace too small
+    assert lib.fp8_gemm_lora_epilogue(x, 4, 64, 64, w, sw, None, None, y, ws, 16,
+                                      None) == L.LORA_ERR_WORKSPACE
+    # LoRA pool that does not match the GEMM
+    p = _pool(h_in=64, h_out=128)
+    s = _seg(T=4)
+    assert lib.fp8_gemm_lora_epilogue(x, 4, 64, 64, w, sw, ctypes.byref(p), ctypes.byref(s), y, ws,
+                                      1 << 20, None) == L.LORA_ERR_INVALID_ARG
+    # segments for a different token count
+    p = _pool(h_in=64, h_out=64)
+    s = _seg(T=5)
+    assert lib.fp8_gemm_lora_epilogue(x, 4, 64, 64, w, sw, ctypes.byref(p), ctypes.byref(s), y, ws,
+                                      1 << 20, None) == L.LORA_ERR_INVALID_ARG
+    assert lib.fp8_quantize_rows(x, 4, 8, w, sw, None) == L.LORA_ERR_INVALID_ARG
+    assert lib.fp8_quantize_rows(x, 0, 16, w, sw, None) == L.LORA_OK
+
+
+def test_build_segments_checks(lib):
+    s = _seg(T=8, n=4)
+    assert lib.lora_build_segments(None, 8, 4, ctypes.byref(s), 0, None) == L.LORA_ERR_INVALID_ARG
+    assert lib.lora_build_segments(ctypes.c_void_p(64), 9, 4, ctypes.byref(s), 0,
+                                   None) == L.LORA_ERR_INVALID_ARG
+    assert lib.lora_build_segments(ctypes.c_void_p(64), 8, 0, ctypes.byref(s), 0,
+                                   None) == L.LORA_ERR_INVALID_ARG
+    big = _seg(T=8, n=20000)
+    assert lib.lora_build_segments(ctypes.c_void_p(64), 8, 20000, ctypes.byref(big), 0,
+                                   None) == L.LORA_ERR_UNSUPPORTED
+
+
+def test_binding_fails_loudly_without_library(tmp_path):
+    missing = str(tmp_path / "liblora.so")
+    saved = L._lib
+    L._lib = None
+    try:
+        with pytest.raises(L.LoraLibraryMissing):
+            L.load(missing)
+    finally:
+        L._lib = saved
