@@ -30,8 +30,10 @@ int check_pool(const lora_pool_t* pool)
     if (pool->n_slices > 65535 || pool->n_adapters > LORA_MAX_ADAPTERS) return LORA_ERR_UNSUPPORTED;
     if (pool->r_max > LORA_MAX_RANK) return LORA_ERR_UNSUPPORTED;
     if (pool->h_in % 8 || pool->h_out % 8 || pool->r_max % 8) return LORA_ERR_INVALID_ARG;
+    if (pool->r_max & (pool->r_max - 1)) return LORA_ERR_UNSUPPORTED;  // 8, 16, 32 or 64
     if (!aligned16(pool->A) || !aligned16(pool->B)) return LORA_ERR_INVALID_ARG;
-    if ((long long)pool->n_slices * pool->n_adapters * pool->h_in * pool->r_max > (1ll << 40))
+    if ((long long)pool->n_slices * pool->n_adapters * pool->h_in >= (1ll << 31) ||
+        (long long)pool->n_slices * pool->n_adapters * pool->r_max >= (1ll << 31))
         return LORA_ERR_UNSUPPORTED;
     return LORA_OK;
 }
@@ -40,7 +42,8 @@ int check_segments(const lora_segments_t* seg, int n_adapters)
 {
     if (!seg) return LORA_ERR_INVALID_ARG;
     if (seg->T < 0 || seg->n_adapters != n_adapters) return LORA_ERR_INVALID_ARG;
-    if (!seg->indptr || !seg->active || !seg->tile_ptr || !seg->counts) return LORA_ERR_INVALID_ARG;
+    if (!seg->indptr || !seg->active || !seg->tiles || !seg->counts) return LORA_ERR_INVALID_ARG;
+    if (!aligned16(seg->tiles)) return LORA_ERR_INVALID_ARG;
     if (seg->T > 0 && (!seg->perm || !seg->tok_adapter)) return LORA_ERR_INVALID_ARG;
     return LORA_OK;
 }
@@ -79,6 +82,30 @@ const char* lora_status_string(int s)
 int lora_version(void) { return kVersion; }
 
 int lora_tile_tokens(void) { return LORA_TILE_TOKENS; }
+
+int lora_max_tiles(int T, int n_adapters)
+{
+    if (T < 0 || n_adapters < 1) return -1;
+    return max_tiles_for(T, n_adapters);
+}
+
+int lora_segments_status(const lora_segments_t* seg, lora_stream_t stream, uint32_t* detail)
+{
+    if (!seg || !seg->counts) return LORA_ERR_INVALID_ARG;
+    int32_t word = 0;
+    int32_t* dev = seg->counts + kSegStatusSlot;
+    cudaError_t e = cudaMemcpyAsync(&word, dev, sizeof(word), cudaMemcpyDeviceToHost,
+                                    (cudaStream_t)stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize((cudaStream_t)stream);
+    if (e != cudaSuccess) return LORA_ERR_CUDA;
+    if (detail) *detail = (uint32_t)word;
+    if (word) {
+        e = cudaMemsetAsync(dev, 0, sizeof(int32_t), (cudaStream_t)stream);
+        if (e == cudaSuccess) e = cudaStreamSynchronize((cudaStream_t)stream);
+        return e == cudaSuccess ? LORA_ERR_TIMEOUT : LORA_ERR_CUDA;
+    }
+    return LORA_OK;
+}
 
 size_t lora_workspace_size(int op, int T, int K, const lora_pool_t* pool)
 {

@@ -2,6 +2,7 @@
 // kernel files. Every launcher enqueues on `stream` and returns the CUDA
 // error of the launch (cudaSuccess when nothing was launched).
 #pragma once
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -50,5 +51,16 @@ struct Fp8GemmArgs {
 cudaError_t launch_fp8_gemm(const Fp8GemmArgs& a, cudaStream_t stream);
 
 int device_sm_count();
+
+// Rows of lora_segments_t.tiles for T tokens over n_adapters.
+int max_tiles_for(int T, int n_adapters);
+
+// 2-D tiled tensor map (inner dimension contiguous); false on failure.
+bool encode_tmap_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner,
+                    uint64_t outer, uint64_t row_stride_bytes, uint32_t box_inner,
+                    uint32_t box_outer, CUtensorMapSwizzle swz);
+
+// Slot of the device status word in lora_segments_t.counts.
+constexpr int kSegStatusSlot = 4;
 
 }  // namespace lora

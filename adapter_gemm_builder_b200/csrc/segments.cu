@@ -1,29 +1,37 @@
 // segments.cu -- group the tokens of a batch by adapter id.
 //
 // The SGMV of the Punica README ("How?") works on segments: runs of tokens
-// that map to the same adapter. One CTA of 1024 threads builds them with a
-// stable counting sort: a shared-memory histogram, block-wide prefix sums
-// for the segment starts, the list of active adapters and their tile counts,
-// then a scatter that keeps token order inside every segment (tokens are
-// taken 1024 at a time, warp by warp, and within a warp the lanes that share
-// an id rank themselves with __match_any_sync). The result is unique, so it
-// is bit-exact and independent of thread timing.
+// that map to the same adapter. One CTA builds them with a stable counting
+// sort and cuts every segment into work tiles of at most LORA_TILE_TOKENS
+// tokens. The order is unique (ascending id, ascending token index inside an
+// id, the tokens without an adapter last), so the result is bit-exact and
+// independent of thread timing.
+//
+// Two paths:
+//  * small batches (T <= 1024 and a per-warp count table that fits shared
+//    memory): one thread per token. Each warp ranks its lanes that share an
+//    id with __match_any_sync and records per-id counts in its own row of a
+//    [warps][bins] table; a column-wise exclusive scan of that table gives
+//    every warp its offset inside each segment and the histogram itself.
+//  * large batches: a histogram, then 1024 tokens per round scattered warp by
+//    warp (the same per-warp ranking) to keep token order.
 #include <cuda_runtime.h>
 
 #include "internal.h"
+#include "ptx.cuh"
 
 namespace lora {
 namespace {
 
-constexpr int kThreads = 1024;
-constexpr int kWarps = kThreads / 32;
+constexpr int kMaxThreads = 1024;
+constexpr int kTile = LORA_TILE_TOKENS;
 
-// Exclusive block-wide scan of one 64-bit value per thread; returns the
-// thread's exclusive prefix and writes the block total to *total.
+// Exclusive block-wide scan of one 64-bit value per thread (any blockDim that
+// is a multiple of 32); *total receives the sum. Ends with __syncthreads.
 __device__ long long block_exclusive_scan(long long val, long long* total)
 {
-    __shared__ long long warp_sums[kWarps];
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    __shared__ long long warp_sums[32];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
     long long incl = val;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
@@ -33,111 +41,172 @@ __device__ long long block_exclusive_scan(long long val, long long* total)
     if (lane == 31) warp_sums[warp] = incl;
     __syncthreads();
     if (warp == 0) {
-        long long w = warp_sums[lane];
+        long long w = lane < nw ? warp_sums[lane] : 0;
         long long wi = w;
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
             long long n = __shfl_up_sync(0xffffffffu, wi, off);
             if (lane >= off) wi += n;
         }
-        warp_sums[lane] = wi - w;  // exclusive prefix of warp totals
+        if (lane < nw) warp_sums[lane] = wi - w;
         if (lane == 31) *total = wi;
     }
     __syncthreads();
-    long long excl = incl - val + warp_sums[warp];
+    const long long excl = incl - val + warp_sums[warp];
     __syncthreads();
     return excl;
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
-build_segments_kernel(const int32_t* __restrict__ ids, int T, int n_adapters,
-                      int32_t* __restrict__ perm, int32_t* __restrict__ indptr,
-                      int32_t* __restrict__ active, int32_t* __restrict__ tile_ptr,
-                      int32_t* __restrict__ tok_adapter, int32_t* __restrict__ counts)
+struct SegOut {
+    int32_t* perm;
+    int32_t* indptr;
+    int32_t* active;
+    int32_t* tiles;
+    int32_t* tok_adapter;
+    int32_t* counts;
+};
+
+// Given per-bin counts hist[0..nb) in shared memory (nb = n_adapters + 1),
+// write starts[] (shared) and indptr, then the active list, the tile table
+// and the counts. Every thread of the block must call it.
+__device__ void finish_tables(const int32_t* hist, int32_t* starts, int n_adapters, int max_tiles,
+                              int n_bad, const SegOut& o)
 {
-    extern __shared__ int32_t smem[];
-    const int nb = n_adapters + 1;  // bins: adapters, then "no adapter"
-    int32_t* hist = smem;           // [nb]
-    int32_t* cursor = smem + nb;    // [nb]
     __shared__ long long s_total;
-    __shared__ int s_bad;
-
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    for (int i = tid; i < nb; i += kThreads) hist[i] = 0;
-    if (tid == 0) s_bad = 0;
-    __syncthreads();
-
-    // 1. histogram + per-token served id
-    int bad = 0;
-    for (int t = tid; t < T; t += kThreads) {
-        const int id = ids[t];
-        const bool ok = id >= 0 && id < n_adapters;
-        if (!ok && id != -1) ++bad;
-        tok_adapter[t] = ok ? id : -1;
-        atomicAdd(&hist[ok ? id : n_adapters], 1);
-    }
-    if (bad) atomicAdd(&s_bad, bad);
-    __syncthreads();
-
-    // 2. segment starts: exclusive scan of hist over contiguous chunks
-    const int chunk = (nb + kThreads - 1) / kThreads;
+    const int nb = n_adapters + 1;
+    const int tid = threadIdx.x, nthr = blockDim.x;
+    const int chunk = (nb + nthr - 1) / nthr;
     const int c0 = min(nb, tid * chunk), c1 = min(nb, c0 + chunk);
     long long local = 0;
     for (int i = c0; i < c1; ++i) local += hist[i];
     long long base = block_exclusive_scan(local, &s_total);
     for (int i = c0; i < c1; ++i) {
-        cursor[i] = (int32_t)base;
-        indptr[i] = (int32_t)base;
+        starts[i] = (int32_t)base;
+        o.indptr[i] = (int32_t)base;
         base += hist[i];
     }
-
-    // 3. active adapters (count > 0) and their tiles: one packed scan of
-    //    (#active << 32 | #tiles) over the adapter bins
-    const int ca0 = min(n_adapters, tid * chunk), ca1 = min(n_adapters, ca0 + chunk);
+    // active adapters and their tiles: one packed scan of (#active << 32 | #tiles)
+    const int ca0 = min(n_adapters, c0), ca1 = min(n_adapters, c1);
     long long pk = 0;
     for (int a = ca0; a < ca1; ++a)
-        if (hist[a] > 0)
-            pk += (1ll << 32) + (hist[a] + LORA_TILE_TOKENS - 1) / LORA_TILE_TOKENS;
-    __syncthreads();
-    long long pbase = block_exclusive_scan(pk, &s_total);
-    {
-        int pos = (int)(pbase >> 32);
-        int tiles = (int)(pbase & 0xffffffffll);
-        for (int a = ca0; a < ca1; ++a) {
-            if (hist[a] > 0) {
-                active[pos] = a;
-                tile_ptr[pos] = tiles;
-                ++pos;
-                tiles += (hist[a] + LORA_TILE_TOKENS - 1) / LORA_TILE_TOKENS;
-            }
+        if (hist[a] > 0) pk += (1ll << 32) + (hist[a] + kTile - 1) / kTile;
+    const long long pbase = block_exclusive_scan(pk, &s_total);
+    int pos = (int)(pbase >> 32);
+    int tile = (int)(pbase & 0xffffffffll);
+    for (int a = ca0; a < ca1; ++a) {
+        const int c = hist[a];
+        if (c > 0) {
+            o.active[pos] = a;
+            for (int off = 0; off < c; off += kTile, ++tile)
+                reinterpret_cast<int4*>(o.tiles)[tile] =
+                    make_int4(a, starts[a] + off, min(kTile, c - off), pos);
+            ++pos;
         }
     }
-    __syncthreads();
     const int n_active = (int)(s_total >> 32);
     const int n_tiles = (int)(s_total & 0xffffffffll);
-    for (int s = n_active + tid; s < n_adapters; s += kThreads) active[s] = -1;
-    for (int s = n_active + tid; s <= n_adapters; s += kThreads) tile_ptr[s] = n_tiles;
+    for (int s = n_active + tid; s < n_adapters; s += nthr) o.active[s] = -1;
+    for (int g = n_tiles + tid; g < max_tiles; g += nthr)
+        reinterpret_cast<int4*>(o.tiles)[g] = make_int4(-1, 0, 0, -1);
     if (tid == 0) {
-        counts[0] = cursor[n_adapters];  // start of the no-adapter tail = #valid
-        counts[1] = n_active;
-        counts[2] = s_bad;
-        counts[3] = n_tiles;
+        o.counts[0] = starts[n_adapters];
+        o.counts[1] = n_active;
+        o.counts[2] = n_bad;
+        o.counts[3] = n_tiles;
+        o.counts[4] = 0;  // device status word
+        o.counts[5] = o.counts[6] = o.counts[7] = 0;
     }
     __syncthreads();
+}
 
-    // 4. stable scatter, 1024 tokens per round, one warp at a time
-    for (int t0 = 0; t0 < T; t0 += kThreads) {
+__device__ __forceinline__ int bin_of(int id, int n_adapters)
+{
+    return (id >= 0 && id < n_adapters) ? id : n_adapters;
+}
+
+// Small batches: blockDim >= T, shared memory = (warps + 2) * nb ints.
+__global__ void __launch_bounds__(kMaxThreads, 1)
+segments_small_kernel(const int32_t* __restrict__ ids, int T, int n_adapters, int max_tiles, SegOut o)
+{
+    extern __shared__ int32_t smem[];
+    __shared__ int s_bad;
+    // PDL: whatever ran before may still be writing our outputs; wait, then
+    // let the consumer of the segments launch early.
+    ptx::pdl_wait();
+    ptx::pdl_launch_dependents();
+    const int nb = n_adapters + 1;
+    const int nw = blockDim.x >> 5;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    int32_t* cnt = smem;             // [nw][nb] per-warp counts, then offsets
+    int32_t* hist = smem + nw * nb;  // [nb]
+    int32_t* starts = hist + nb;     // [nb]
+    for (int i = tid; i < nw * nb; i += blockDim.x) cnt[i] = 0;
+    if (tid == 0) s_bad = 0;
+    __syncthreads();
+
+    const bool in = tid < T;
+    int id = -1, bin = -2 - lane;
+    if (in) {
+        id = ids[tid];
+        bin = bin_of(id, n_adapters);
+        o.tok_adapter[tid] = bin < n_adapters ? id : -1;
+    }
+    const unsigned bad = __ballot_sync(0xffffffffu, in && bin == n_adapters && id != -1);
+    if (lane == 0 && bad) atomicAdd(&s_bad, __popc(bad));
+    const unsigned peers = __match_any_sync(0xffffffffu, bin);
+    const int rank = __popc(peers & ((1u << lane) - 1u));
+    if (in && lane == __ffs(peers) - 1) cnt[warp * nb + bin] = __popc(peers);
+    __syncthreads();
+    // column scan: offset of each warp inside every bin, and the histogram
+    for (int b = tid; b < nb; b += blockDim.x) {
+        int run = 0;
+        for (int w = 0; w < nw; ++w) {
+            const int c = cnt[w * nb + b];
+            cnt[w * nb + b] = run;
+            run += c;
+        }
+        hist[b] = run;
+    }
+    __syncthreads();
+    finish_tables(hist, starts, n_adapters, max_tiles, s_bad, o);
+    if (in) o.perm[starts[bin] + cnt[warp * nb + bin] + rank] = tid;
+}
+
+// Large batches: 1024 threads, shared memory = 2 * nb ints.
+__global__ void __launch_bounds__(kMaxThreads, 1)
+segments_large_kernel(const int32_t* __restrict__ ids, int T, int n_adapters, int max_tiles, SegOut o)
+{
+    extern __shared__ int32_t smem[];
+    __shared__ int s_bad;
+    ptx::pdl_wait();
+    ptx::pdl_launch_dependents();
+    const int nb = n_adapters + 1;
+    int32_t* hist = smem;         // [nb]
+    int32_t* cursor = smem + nb;  // [nb] starts, then running cursors
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
+    for (int i = tid; i < nb; i += blockDim.x) hist[i] = 0;
+    if (tid == 0) s_bad = 0;
+    __syncthreads();
+    int bad = 0;
+    for (int t = tid; t < T; t += blockDim.x) {
+        const int id = ids[t];
+        const int bin = bin_of(id, n_adapters);
+        if (bin == n_adapters && id != -1) ++bad;
+        o.tok_adapter[t] = bin < n_adapters ? id : -1;
+        atomicAdd(&hist[bin], 1);
+    }
+    if (bad) atomicAdd(&s_bad, bad);
+    __syncthreads();
+    finish_tables(hist, cursor, n_adapters, max_tiles, s_bad, o);
+
+    for (int t0 = 0; t0 < T; t0 += blockDim.x) {
         const int t = t0 + tid;
         const bool in = t < T;
-        int bin = -2 - lane;  // unique per lane when out of range
-        if (in) {
-            const int id = ids[t];
-            bin = (id >= 0 && id < n_adapters) ? id : n_adapters;
-        }
+        const int bin = in ? bin_of(ids[t], n_adapters) : -2 - lane;
         const unsigned peers = __match_any_sync(0xffffffffu, bin);
         const int leader = __ffs(peers) - 1;
         const int rank = __popc(peers & ((1u << lane) - 1u));
-        for (int w = 0; w < kWarps; ++w) {
+        for (int w = 0; w < nw; ++w) {
             if (warp == w) {
                 int p = 0;
                 if (in && lane == leader) {
@@ -145,7 +214,7 @@ build_segments_kernel(const int32_t* __restrict__ ids, int T, int n_adapters,
                     cursor[bin] = p + __popc(peers);
                 }
                 p = __shfl_sync(0xffffffffu, p, leader);
-                if (in) perm[p + rank] = t;
+                if (in) o.perm[p + rank] = t;
             }
             __syncthreads();
         }
@@ -154,20 +223,44 @@ build_segments_kernel(const int32_t* __restrict__ ids, int T, int n_adapters,
 
 }  // namespace
 
+int max_tiles_for(int T, int n_adapters)
+{
+    return (n_adapters < T ? n_adapters : T) + (T + kTile - 1) / kTile;
+}
+
 cudaError_t launch_build_segments(const int32_t* ids, int T, int n_adapters,
                                   const lora_segments_t& seg, cudaStream_t stream)
 {
-    const size_t smem = sizeof(int32_t) * 2 * (size_t)(n_adapters + 1);
-    if (smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(build_segments_kernel,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             2 * (LORA_MAX_ADAPTERS + 1) * (int)sizeof(int32_t));
+    SegOut o{seg.perm, seg.indptr, seg.active, seg.tiles, seg.tok_adapter, seg.counts};
+    const int nb = n_adapters + 1;
+    const int mt = max_tiles_for(T, n_adapters);
+    const int threads_small = T <= 64 ? 64 : (T + 31) / 32 * 32;
+    const size_t smem_small = sizeof(int32_t) * (size_t)(threads_small / 32 + 2) * nb;
+    const bool small = T <= kMaxThreads && smem_small <= 96 * 1024;
+
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cfg.stream = stream;
+    cfg.gridDim = dim3(1, 1, 1);
+    cudaError_t e;
+    if (small) {
+        cfg.blockDim = dim3(threads_small, 1, 1);
+        cfg.dynamicSmemBytes = smem_small;
+        e = cudaFuncSetAttribute(segments_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 96 * 1024);
         if (e != cudaSuccess) return e;
+        return cudaLaunchKernelEx(&cfg, segments_small_kernel, ids, T, n_adapters, mt, o);
     }
-    build_segments_kernel<<<1, kThreads, smem, stream>>>(ids, T, n_adapters, seg.perm, seg.indptr,
-                                                         seg.active, seg.tile_ptr, seg.tok_adapter,
-                                                         seg.counts);
-    return cudaGetLastError();
+    cfg.blockDim = dim3(kMaxThreads, 1, 1);
+    cfg.dynamicSmemBytes = sizeof(int32_t) * 2 * (size_t)nb;
+    e = cudaFuncSetAttribute(segments_large_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             2 * (LORA_MAX_ADAPTERS + 1) * (int)sizeof(int32_t));
+    if (e != cudaSuccess) return e;
+    return cudaLaunchKernelEx(&cfg, segments_large_kernel, ids, T, n_adapters, mt, o);
 }
 
 }  // namespace lora

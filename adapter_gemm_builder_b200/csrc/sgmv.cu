@@ -1,35 +1,43 @@
 // sgmv.cu -- Segmented Gather Matrix-Vector multiplication for multi-tenant
 // LoRA (Punica README, "How?": the added term (x_i.A_i.B_i) for a batch whose
-// tokens map to different adapters, computed for all adapters in one kernel).
+// tokens map to different adapters, for all adapters in one kernel).
 //
 // One kernel, three modes:
 //   SHRINK  v = x.A_a            (fp32, written to global)
 //   EXPAND  y += s_a * v.B_a     (v read from global, y bf16 read-modify-write)
 //   APPLY   y += s_a * (x.A_a).B_a, with v kept on chip
 //
-// Work decomposition. The segment builder cuts every adapter's run of tokens
-// into tiles of up to LORA_TILE_TOKENS tokens. A tile is handled by a
-// thread-block cluster of C CTAs (C <= 8): in the shrink, CTA c owns the
-// c-th slice of h_in (split-K) and produces a partial v for the tile's tokens;
-// the partials are reduced through distributed shared memory (reduce-scatter
-// then all-gather), so no global workspace and no second pass is needed; in
-// the expand, CTA c owns the c-th slice of h_out. gridDim.y is the slice
-// (projection) index, so q/k/v/o of one layer run in one launch.
+// Work. The segment builder cuts every adapter's run of tokens into tiles of
+// at most LORA_TILE_TOKENS tokens (one row of lora_segments_t.tiles each). A
+// tile is handled by a thread-block cluster of C CTAs: in the shrink CTA c
+// owns the c-th slice of h_in (split-K) and computes a partial v for the
+// tile's tokens; in the expand it owns the c-th slice of h_out. gridDim.y is
+// the slice (projection) index, so q/k/v/o run in one launch.
 //
-// Memory path. Every operand streams global -> shared with 16-byte cp.async
-// (zero-filling the bytes past an adapter's rank or past the end of a row,
-// so the padding of the pool is never read) through a 4-stage ring of 16 KB
-// stages. The stage shape adapts to the tile: a k-block holds BK rows of A_a
-// (r8 columns) plus BK columns of the tile's x rows, with BK chosen so the
-// stage is full whatever the rank and token count; decode tiles with one
-// token therefore stream ~15 KB of A per stage. Shared layouts are chosen
-// for conflict-free ldmatrix: A and B in 8-column blocks (each 8x8 matrix is
-// 128 contiguous bytes), x and y rows with a 16-byte-chunk XOR swizzle.
+// Memory path (the kernel is bound by HBM bytes and by latency). A producer
+// warp fills a ring of 3 stages with 16-byte cp.async from all 32 lanes,
+// completing on the stage's mbarrier: the k rows of A_a (only its r8 columns;
+// bytes past the rank are zero-filled, so the pool's padding is never read),
+// the gathered x rows of the tile's tokens, then the r rows of B_a and the
+// gathered y rows. Row pitches are padded by 16 bytes so that the ldmatrix
+// reads of the tensor-core path are free of bank conflicts. A decode tile
+// (one token, rank 16) moves its whole A and B slices in one stage each.
 //
-// Math. bf16 tensor-core MMA (m16n8k16, fp32 accumulate) for both products.
-// The expand's left operand v is fp32; it is split as v = hi + lo with hi, lo
-// in bf16 and both halves are multiplied, which keeps ~16 mantissa bits of v
-// (bf16 x bf16 products are exact in fp32).
+// Math. Tiles of at most 4 tokens (decode) use CUDA-core FMAs: the products
+// are few and a 16-row MMA would be mostly padding. Larger tiles use bf16
+// tensor-core MMA (m16n8k16, fp32 accumulate) with all tile-invariant
+// addressing hoisted out of the k loop; their expand operand v (fp32) is
+// split as v = hi + lo in bf16 and both halves are multiplied (~16 bits of v).
+//
+// Reduction of v. Partials travel by distributed shared memory with st.async:
+// each store lands in a peer's shared memory and counts as transaction bytes
+// on that peer's mbarrier, which expects exactly the bytes it must receive.
+// With few rows all CTAs receive all partials (one exchange); with many rows
+// a reduce-scatter by row is followed by an all-gather. Every wait is
+// bounded (2 s); on expiry the kernel records a status word in
+// lora_segments_t.counts and stops computing, but still takes part in every
+// barrier.
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -39,12 +47,15 @@
 namespace lora {
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kWarps = kThreads / 32;
-constexpr int kStages = 4;
-constexpr int kStageBytes = 16384;
-constexpr int kTT = LORA_TILE_TOKENS;  // 64
+constexpr int kComputeWarps = 8;
+constexpr int kCompute = kComputeWarps * 32;
+constexpr int kThreads = kCompute + 32;  // + one producer warp
+constexpr int kStages = 3;
+constexpr int kTT = LORA_TILE_TOKENS;    // 64
 constexpr int kMaxCluster = 8;
+constexpr int kOnePhaseBytes = 8192;     // all-to-all exchange of v up to this size per CTA
+constexpr int kSmallTile = 4;            // tiles of <= 4 tokens use CUDA-core FMAs
+constexpr unsigned long long kTimeoutNs = 2000000000ull;
 
 struct SgmvParams {
     const uint16_t* x;
@@ -54,27 +65,19 @@ struct SgmvParams {
     const int32_t* ranks;
     const float* scales;
     const int32_t* perm;
-    const int32_t* indptr;
-    const int32_t* active;
-    const int32_t* tile_ptr;
-    const int32_t* counts;
+    const int4* tiles;
+    int32_t* counts;
     float* v;
     uint16_t* y;
     int T, n_adapters, h_in, h_out, r_max;
-    int csize;     // CTAs per tile
-    int kc, nc;    // h_in / h_out slice per CTA (multiples of 8)
-    int rp;        // row pitch (floats) of the partial / reduced v buffers = round_up(r_max, 16)
-    int vpitch;    // row pitch (bf16) of the hi/lo v operand = rp + 8
+    int csize;       // CTAs per tile
+    int kc, nc;      // h_in / h_out slice per CTA (multiples of 64 except at the end)
+    int rp;          // round_up(r_max, 16): row pitch (floats) of the v buffers
+    int stage_bytes; // one ring stage
+    uint32_t off_rb, off_vf, off_bar;
 };
 
 __device__ __forceinline__ int round_up(int a, int b) { return (a + b - 1) / b * b; }
-
-// XOR-swizzled byte offset of 16-byte chunk `ch` of row `row` in a row-major
-// tile of `row_bytes` per row (row_bytes a multiple of 128).
-__device__ __forceinline__ uint32_t swz(int row, int ch, int row_bytes)
-{
-    return (uint32_t)(row * row_bytes + ((ch ^ (row & 7)) << 4));
-}
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
 {
@@ -82,314 +85,572 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
     return *reinterpret_cast<uint32_t*>(&h);
 }
 
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// Bounded wait by ONE thread; on expiry raises the CTA abort flag and the
+// status word. The clock and the abort flag are read every 256 probes only.
+template <bool kClusterScope>
+__device__ bool wait_one(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int32_t* status,
+                         int code)
+{
+    auto probe = [&]() {
+        return kClusterScope ? ptx::mbar_try_wait_cluster(bar, parity) : ptx::mbar_try_wait(bar, parity);
+    };
+    if (probe()) return true;
+    const unsigned long long t0 = ptx::globaltimer();
+    for (unsigned n = 1;; ++n) {
+        if (probe()) return true;
+        if ((n & 255) == 0) {
+            if (*abort_flag) return false;
+            if (ptx::globaltimer() - t0 > kTimeoutNs) {
+                *abort_flag = 1;
+                atomicOr(status, code);
+                return false;
+            }
+        }
+    }
+}
+
+// Bounded wait by a WHOLE warp (all 32 lanes must call it): lane 0 polls,
+// the others then observe the completed phase themselves (acquire).
+template <bool kClusterScope>
+__device__ bool wait_all(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int32_t* status,
+                         int code)
+{
+    bool ok = true;
+    if ((threadIdx.x & 31) == 0) ok = wait_one<kClusterScope>(bar, parity, abort_flag, status, code);
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    if (ok && (threadIdx.x & 31) != 0)
+        kClusterScope ? ptx::mbar_try_wait_cluster(bar, parity) : ptx::mbar_try_wait(bar, parity);
+    return ok;
+}
+
 template <int MODE>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 2)
 sgmv_kernel(const SgmvParams p)
 {
-    extern __shared__ __align__(128) uint8_t smem[];
+    extern __shared__ __align__(128) uint8_t smem_raw[];
     __shared__ int s_tok[kTT];
-    __shared__ __align__(16) uint32_t s_zero[4];
+    __shared__ int s_abort;
 
-    // Let a programmatic dependent (the FP8 GEMM) launch as early as possible.
-    ptx::pdl_launch_dependents();
-
+    constexpr bool kClustered = MODE != SGMV_EXPAND;
+    const uint32_t raw_u = ptx::smem_u32(smem_raw);
+    const uint32_t base_u = (raw_u + 127u) & ~127u;
+    uint8_t* smem = smem_raw + (base_u - raw_u);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int C = p.csize;
-    const int rank = (MODE == SGMV_EXPAND) ? (int)(blockIdx.x % C) : (int)ptx::cluster_ctarank();
-    const int g = blockIdx.x / C;  // tile index
+    const int rank = kClustered ? (int)ptx::cluster_ctarank() : (int)(blockIdx.x % C);
+    const int g = blockIdx.x / C;
     const int slice = blockIdx.y;
+    const int SB = p.stage_bytes;
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + p.off_bar);
+    uint64_t* empty = full + kStages;
+    uint64_t* red1 = empty + kStages;
+    uint64_t* red2 = red1 + 1;
+    volatile int* abort_flag = &s_abort;
+    int32_t* status = p.counts + kSegStatusSlot;
 
-    const int n_tiles = p.counts[3];
-    if (g >= n_tiles) return;  // the whole cluster leaves together (same g)
-    const int n_active = p.counts[1];
-
-    // tile -> active segment (largest s with tile_ptr[s] <= g)
-    int lo = 0, hi = n_active - 1;
-    while (lo < hi) {
-        int mid = (lo + hi + 1) >> 1;
-        if (p.tile_ptr[mid] <= g) lo = mid; else hi = mid - 1;
+    if (tid == 0) {
+        s_abort = 0;
+        for (int s = 0; s < kStages; ++s) {
+            ptx::mbar_init(&full[s], 32);  // the 32 producer lanes' cp.async groups
+            ptx::mbar_init(&empty[s], 1);
+        }
+        ptx::mbar_init(red1, 1);
+        ptx::mbar_init(red2, 1);
+        ptx::fence_mbar_init();
     }
-    const int seg = lo;
-    const int a = p.active[seg];
-    const int seg_begin = p.indptr[a], seg_len = p.indptr[a + 1] - seg_begin;
-    const int tok0 = seg_begin + (g - p.tile_ptr[seg]) * kTT;
-    const int nt = min(kTT, seg_begin + seg_len - tok0);  // tokens in this tile, 1..64
+    // the previous kernel in the stream (e.g. the segment builder) may still run
+    ptx::pdl_wait();
+    ptx::pdl_launch_dependents();
+
+    const int4 tl = p.tiles[g];
+    const int nt = tl.z;
+    if (nt <= 0) return;  // unused tile row: the whole cluster leaves together
+    const int a = tl.x, tok0 = tl.y;
     int r = p.ranks ? p.ranks[a] : p.r_max;
-    r = max(0, min(r, p.r_max));
+    r = max(1, min(r, p.r_max));
     const float scale = p.scales ? p.scales[a] : 1.0f;
-    const int r8 = round_up(max(r, 1), 8), r16 = round_up(max(r, 1), 16);
+    const int r8 = round_up(r, 8), r16 = round_up(r, 16);
+    const bool small = nt <= kSmallTile;
     const int Mt = (nt + 15) >> 4;
+    const int Mtr = small ? nt : Mt * 16;  // x / y rows held per stage (tail rows zero)
+    if (tid < nt) s_tok[tid] = p.perm[tok0 + tid];
 
-    if (tid < kTT) s_tok[tid] = tid < nt ? p.perm[tok0 + tid] : 0;
-    if (tid < 4) s_zero[tid] = 0u;
-
-    uint8_t* ring = smem;
-    // [sP partial v | hi/lo operand (aliases sP)] then [sR reduced v]
-    float* sP = reinterpret_cast<float*>(smem + kStages * kStageBytes);  // [kTT][rp]
-    uint16_t* sVh = reinterpret_cast<uint16_t*>(sP);                     // [kTT][vpitch]
-    uint16_t* sVl = sVh + kTT * p.vpitch;                                // [kTT][vpitch]
-    const int region0 = max(kTT * p.rp * 4, 2 * kTT * p.vpitch * 2);
-    float* sR = reinterpret_cast<float*>(smem + kStages * kStageBytes + region0);  // [kTT][rp]
-    const uint32_t ring_u = ptx::smem_u32(ring);
-    const uint32_t zero_u = ptx::smem_u32(s_zero);
-
-    // ---- shrink geometry: this CTA's slice of h_in
+    // ---- geometry (identical in every role)
+    // bytes per A row in shared memory: small tiles take the contiguous rows of the pool
+    // with one bulk copy (r_max columns); large tiles take r8 columns with a padded pitch
+    const int apitch = small ? p.r_max * 2 : r8 * 2 + 16;
     const int k_begin = min(p.h_in, rank * p.kc);
-    const int k_end = min(p.h_in, k_begin + p.kc);
-    const int BK = ((kStageBytes / (2 * (r8 + nt))) / 64) * 64;  // >= 64
-    const int nK = (MODE == SGMV_EXPAND) ? 0 : (k_end - k_begin + BK - 1) / BK;
-    // ---- expand geometry: this CTA's slice of h_out
+    const int k_len = min(p.h_in, k_begin + p.kc) - k_begin;
+    int BK = ((SB - 16 * Mtr) / (apitch + 2 * Mtr)) / 64 * 64;
+    BK = min(BK, round_up(max(k_len, 1), 64));
+    const int nK = (MODE == SGMV_EXPAND) ? 0 : (k_len + BK - 1) / BK;
+    const int xp = BK * 2 + 16;  // x row pitch (bytes)
     const int n_begin = min(p.h_out, rank * p.nc);
-    const int n_end = min(p.h_out, n_begin + p.nc);
-    const int BN = ((kStageBytes / (2 * (r16 + nt))) / 64) * 64;  // >= 64
-    const int nN = (MODE == SGMV_SHRINK) ? 0 : (n_end - n_begin + BN - 1) / BN;
+    const int n_len = min(p.h_out, n_begin + p.nc) - n_begin;
+    int BN = ((SB / (r16 + Mtr) - 16) / 2) / 64 * 64;
+    BN = min(BN, round_up(max(n_len, 1), 64));
+    const int nN = (MODE == SGMV_SHRINK) ? 0 : (n_len + BN - 1) / BN;
+    const int bp = BN * 2 + 16;  // B and y row pitch (bytes)
     const int nItems = nK + nN;
-
     const size_t sa = (size_t)slice * p.n_adapters + a;
     const uint16_t* Ag = p.A + sa * (size_t)p.h_in * p.r_max;
     const uint16_t* Bg = p.B + sa * (size_t)p.r_max * p.h_out;
     const uint16_t* xg = p.x ? p.x + (size_t)slice * p.x_slice_stride : nullptr;
     uint16_t* yg = p.y ? p.y + (size_t)slice * p.T * p.h_out : nullptr;
+
+    // bytes this CTA receives in the v exchange
+    const bool one_phase = C * nt * r8 * 4 <= kOnePhaseBytes;
+    const int rows_per = (nt + C - 1) / C;
+    const int mine = nt > rank ? (nt - rank + C - 1) / C : 0;
+    if (kClustered && tid == 0) {
+        ptx::mbar_arrive_expect_tx(red1, (uint32_t)((one_phase ? C * nt : C * mine) * r8 * 4));
+        ptx::mbar_arrive_expect_tx(red2, one_phase ? 0u : (uint32_t)(nt * r8 * 4));
+    }
     __syncthreads();
+    if (kClustered) ptx::cluster_arrive();  // barriers initialised; matched before any remote access
 
-    // Issue the loads of work item `it` into ring stage `st`.
-    auto load_item = [&](int it, int st) {
-        const uint32_t base = ring_u + st * kStageBytes;
-        if (it < nK) {
-            const int k0 = k_begin + it * BK;
-            const int kb = min(BK, k_end - k0);
-            const int ncb = r8 >> 3;
-            // A rows k0..k0+BK, column blocks of 8: smem [cb][BK][8]
-            for (int i = tid; i < BK * ncb; i += kThreads) {
-                const int kk = i / ncb, cb = i - kk * ncb;
-                const int valid = (kk < kb) ? max(0, min(8, r - cb * 8)) : 0;
-                const uint16_t* src = valid ? Ag + (size_t)(k0 + kk) * p.r_max + cb * 8 : Ag;
-                ptx::cp_async16(base + (uint32_t)((cb * BK + kk) << 4), src, valid * 2);
-            }
-            // x rows of the tile: smem [nt][BK], swizzled
-            const uint32_t xb = base + (uint32_t)(r8 * BK * 2);
-            const int nch = BK >> 3;
-            for (int i = tid; i < nt * nch; i += kThreads) {
-                const int row = i / nch, ch = i - row * nch;
-                const bool ok = ch * 8 < kb;
-                const uint16_t* src =
-                    ok ? xg + (size_t)s_tok[row] * p.h_in + k0 + ch * 8 : xg;
-                ptx::cp_async16(xb + swz(row, ch, BK * 2), src, ok ? 16 : 0);
-            }
-        } else {
-            const int n0 = n_begin + (it - nK) * BN;
-            const int nb = min(BN, n_end - n0);
-            const int ncb = BN >> 3;
-            // B rows 0..r16, column blocks of 8: smem [cb][r16][8]
-            for (int i = tid; i < r16 * ncb; i += kThreads) {
-                const int j = i / ncb, cb = i - j * ncb;
-                const bool ok = j < r && cb * 8 < nb;
-                const uint16_t* src = ok ? Bg + (size_t)j * p.h_out + n0 + cb * 8 : Bg;
-                ptx::cp_async16(base + (uint32_t)((cb * r16 + j) << 4), src, ok ? 16 : 0);
-            }
-            // y rows of the tile: smem [nt][BN], swizzled
-            const uint32_t yb = base + (uint32_t)(r16 * BN * 2);
-            for (int i = tid; i < nt * ncb; i += kThreads) {
-                const int row = i / ncb, ch = i - row * ncb;
-                const bool ok = ch * 8 < nb;
-                const uint16_t* src =
-                    ok ? yg + (size_t)s_tok[row] * p.h_out + n0 + ch * 8 : yg;
-                ptx::cp_async16(yb + swz(row, ch, BN * 2), src, ok ? 16 : 0);
-            }
-        }
-    };
-
-    // Shrink accumulators: warp w owns output tiles [w*tpw, (w+1)*tpw) of the
-    // (Mt x r8/8) grid of 16x8 tiles, row-major.
-    const int nNT = r8 >> 3;
-    const int tiles_s = Mt * nNT;
-    const int tpw_s = (tiles_s + kWarps - 1) / kWarps;  // <= 4
-    float acc[4][4];
-#pragma unroll
-    for (int q = 0; q < 4; ++q)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) acc[q][e] = 0.f;
-
-
-    // Partial v of this CTA -> sP, then the cluster-wide reduction of v
-    // (reduce-scatter by rows, then, for APPLY, all-gather as the bf16 hi/lo
-    // operand of the expand). Called once by every CTA of a shrinking mode.
-    auto finish_shrink = [&]() {
-        {
-            const int gq = lane >> 2, tq = lane & 3;
-            const int q0 = warp * tpw_s;
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const int t = q0 + q;
-                if (q < tpw_s && t < tiles_s) {
-                    const int mt = t / nNT, ntl = t - mt * nNT;
-                    const int row = mt * 16 + gq, col = ntl * 8 + tq * 2;
-                    if (row < nt)
-                        *reinterpret_cast<float2*>(&sP[row * p.rp + col]) =
-                            make_float2(acc[q][0], acc[q][1]);
-                    if (row + 8 < nt)
-                        *reinterpret_cast<float2*>(&sP[(row + 8) * p.rp + col]) =
-                            make_float2(acc[q][2], acc[q][3]);
+    if (warp == kComputeWarps) {
+        // ================================================================ producer warp
+        for (int it = 0; it < nItems; ++it) {
+            const int st = it % kStages;
+            const uint32_t ph = (uint32_t)((it / kStages) & 1);
+            if (!wait_all<false>(&empty[st], ph ^ 1, abort_flag, status, 0x100)) break;
+            const uint32_t base = base_u + st * SB;
+            if (small) {
+                // decode-sized tile: a handful of 1-D bulk copies, all issued by lane 0
+                if (lane == 0) {
+                    if (it < nK) {
+                        const int k0 = k_begin + it * BK;
+                        const int kb = min(BK, k_begin + k_len - k0);
+                        const uint32_t xb = base + (uint32_t)(BK * apitch);
+                        ptx::mbar_arrive_expect_tx(&full[st], (uint32_t)((p.r_max + nt) * kb * 2));
+                        ptx::bulk_g2s(base, Ag + (size_t)k0 * p.r_max, (uint32_t)(kb * p.r_max * 2), &full[st]);
+                        for (int row = 0; row < nt; ++row)
+                            ptx::bulk_g2s(xb + row * xp, xg + (size_t)s_tok[row] * p.h_in + k0, (uint32_t)(kb * 2),
+                                          &full[st]);
+                    } else {
+                        const int n0 = n_begin + (it - nK) * BN;
+                        const int nb = min(BN, n_begin + n_len - n0);
+                        const uint32_t yb = base + (uint32_t)(r16 * bp);
+                        ptx::mbar_arrive_expect_tx(&full[st], (uint32_t)((r + nt) * nb * 2));
+                        for (int j = 0; j < r; ++j)
+                            ptx::bulk_g2s(base + j * bp, Bg + (size_t)j * p.h_out + n0, (uint32_t)(nb * 2), &full[st]);
+                        for (int row = 0; row < nt; ++row)
+                            ptx::bulk_g2s(yb + row * bp, yg + (size_t)s_tok[row] * p.h_out + n0, (uint32_t)(nb * 2),
+                                          &full[st]);
+                    }
+                } else {
+                    ptx::mbar_arrive(&full[st]);
                 }
+                continue;
             }
-        }
-        ptx::cluster_sync();  // every CTA's partial is in its sP
-        const uint32_t sP_u = ptx::smem_u32(sP);
-        const uint32_t sR_u = ptx::smem_u32(sR);
-        const int rows_mine = (nt > rank) ? (nt - rank + C - 1) / C : 0;
-        const int cols = (MODE == SGMV_SHRINK) ? p.r_max : r8;
-        for (int i = tid; i < rows_mine * cols; i += kThreads) {
-            const int row = rank + (i / cols) * C, j = i % cols;
-            float sum = 0.f;
-            if (j < r8) {
-                for (int c = 0; c < C; ++c)
-                    sum += ptx::ld_dsmem_f32(ptx::mapa(sP_u + (uint32_t)((row * p.rp + j) * 4), c));
-            }
-            if (MODE == SGMV_SHRINK)
-                p.v[((size_t)slice * p.T + s_tok[row]) * p.r_max + j] = (j < r) ? sum : 0.f;
-            else
-                sR[row * p.rp + j] = sum;
-        }
-        ptx::cluster_sync();  // reductions done; nobody reads sP any more
-        if (MODE == SGMV_APPLY) {
-            for (int i = tid; i < nt * r16; i += kThreads) {
-                const int row = i / r16, j = i - row * r16;
-                const float val =
-                    j < r ? ptx::ld_dsmem_f32(
-                                ptx::mapa(sR_u + (uint32_t)((row * p.rp + j) * 4), row % C))
-                          : 0.f;
-                const __nv_bfloat16 h = __float2bfloat16_rn(val);
-                const __nv_bfloat16 l = __float2bfloat16_rn(val - __bfloat162float(h));
-                sVh[row * p.vpitch + j] = *reinterpret_cast<const uint16_t*>(&h);
-                sVl[row * p.vpitch + j] = *reinterpret_cast<const uint16_t*>(&l);
-            }
-            ptx::cluster_arrive();  // matched by the wait before exit
-        }
-    };
-
-    // ---- prologue
-#pragma unroll
-    for (int i = 0; i < kStages - 1; ++i) {
-        if (i < nItems) load_item(i, i);
-        ptx::cp_async_commit();
-    }
-
-    if (MODE == SGMV_EXPAND) {
-        // v (fp32, global) -> hi/lo bf16 operand
-        for (int i = tid; i < nt * r16; i += kThreads) {
-            const int row = i / r16, j = i - row * r16;
-            const float val =
-                j < r ? p.v[((size_t)slice * p.T + s_tok[row]) * p.r_max + j] : 0.f;
-            const __nv_bfloat16 h = __float2bfloat16_rn(val);
-            const __nv_bfloat16 l = __float2bfloat16_rn(val - __bfloat162float(h));
-            sVh[row * p.vpitch + j] = *reinterpret_cast<const uint16_t*>(&h);
-            sVl[row * p.vpitch + j] = *reinterpret_cast<const uint16_t*>(&l);
-        }
-    }
-
-    if (MODE != SGMV_EXPAND && nK == 0) finish_shrink();
-
-    for (int it = 0; it < nItems; ++it) {
-        ptx::cp_async_wait<kStages - 2>();
-        __syncthreads();
-        {
-            const int nx = it + kStages - 1;
-            if (nx < nItems) load_item(nx, nx % kStages);
-            ptx::cp_async_commit();
-        }
-        const int st = it % kStages;
-        const uint32_t base = ring_u + st * kStageBytes;
-
-        if (it < nK) {
-            // ------------------------------------------------ shrink k-block
-            const int k0 = k_begin + it * BK;
-            const int kb = min(BK, k_end - k0);
-            const uint32_t xb = base + (uint32_t)(r8 * BK * 2);
-            const int ksteps = (kb + 15) >> 4;
-            const int q0 = warp * tpw_s;
-            for (int ks = 0; ks < ksteps; ++ks) {
-                uint32_t af[4];
-                int cur_mt = -1;
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const int t = q0 + q;
-                    if (q < tpw_s && t < tiles_s) {
-                        const int mt = t / nNT, ntl = t - mt * nNT;
-                        if (mt != cur_mt) {
-                            const int row = mt * 16 + (lane & 15);
-                            const int ch = ks * 2 + (lane >> 4);
-                            const uint32_t addr = row < nt ? xb + swz(row, ch, BK * 2) : zero_u;
-                            ptx::ldsm_x4(addr, af[0], af[1], af[2], af[3]);
-                            cur_mt = mt;
-                        }
-                        uint32_t b0, b1;
-                        ptx::ldsm_x2_t(base + (uint32_t)((ntl * BK + ks * 16 + (lane & 15)) << 4),
-                                       b0, b1);
-                        ptx::mma_bf16_16816(acc[q], af, b0, b1);
+            if (it < nK) {
+                const int k0 = k_begin + it * BK;
+                const int kb = min(BK, k_begin + k_len - k0);
+                // A rows k0 .. k0+BK (rows >= kb and bytes past the rank zero-filled);
+                // (row, 16-byte chunk) pairs spread over the lanes, chunks padded to a power of 2
+                const int ncb = r8 >> 3;
+                const int lgc = ncb <= 1 ? 0 : (ncb <= 2 ? 1 : (ncb <= 4 ? 2 : 3));
+                for (int i = lane; i < (BK << lgc); i += 32) {
+                    const int kk = i >> lgc, c = i & ((1 << lgc) - 1);
+                    if (c < ncb) {
+                        const int valid = kk < kb ? min(8, r - c * 8) : 0;
+                        ptx::cp_async16(base + kk * apitch + c * 16,
+                                        valid > 0 ? Ag + (size_t)(k0 + kk) * p.r_max + c * 8 : Ag,
+                                        valid > 0 ? valid * 2 : 0);
+                    }
+                }
+                // x rows of the tile's tokens (rows >= nt and columns >= kb zero-filled)
+                const uint32_t xb = base + (uint32_t)(BK * apitch);
+                for (int row = 0; row < Mtr; ++row) {
+                    const uint16_t* src = xg + (size_t)s_tok[row < nt ? row : 0] * p.h_in + k0;
+                    for (int ch = lane; ch < (BK >> 3); ch += 32) {
+                        const bool ok = row < nt && ch * 8 < kb;
+                        ptx::cp_async16(xb + row * xp + ch * 16, ok ? src + ch * 8 : xg, ok ? 16 : 0);
+                    }
+                }
+            } else {
+                const int n0 = n_begin + (it - nK) * BN;
+                const int nb = min(BN, n_begin + n_len - n0);
+                // B rows 0 .. r16 (rows >= r zero-filled), columns n0 .. n0+BN
+                for (int j = 0; j < r16; ++j)
+                    for (int ch = lane; ch < (BN >> 3); ch += 32) {
+                        const bool ok = j < r && ch * 8 < nb;
+                        ptx::cp_async16(base + j * bp + ch * 16, ok ? Bg + (size_t)j * p.h_out + n0 + ch * 8 : Bg,
+                                        ok ? 16 : 0);
+                    }
+                const uint32_t yb = base + (uint32_t)(r16 * bp);
+                for (int row = 0; row < Mtr; ++row) {
+                    const uint16_t* src = yg + (size_t)s_tok[row < nt ? row : 0] * p.h_out + n0;
+                    for (int ch = lane; ch < (BN >> 3); ch += 32) {
+                        const bool ok = row < nt && ch * 8 < nb;
+                        ptx::cp_async16(yb + row * bp + ch * 16, ok ? src + ch * 8 : yg, ok ? 16 : 0);
                     }
                 }
             }
-        } else {
-            // ------------------------------------------------ expand n-block
-            const int n0 = n_begin + (it - nK) * BN;
-            const int nb = min(BN, n_end - n0);
-            const uint32_t yb = base + (uint32_t)(r16 * BN * 2);
-            const int nNTe = BN >> 3;
-            const int tiles_e = Mt * nNTe;
-            const int tpw_e = (tiles_e + kWarps - 1) / kWarps;
-            const int ksteps = r16 >> 4;
-            const int gq = lane >> 2, tq = lane & 3;
-            const uint32_t vh_u = ptx::smem_u32(sVh), vl_u = ptx::smem_u32(sVl);
-            for (int q = 0; q < tpw_e; ++q) {
-                const int t = warp * tpw_e + q;
-                if (t >= tiles_e) break;
-                const int mt = t / nNTe, ntl = t - mt * nNTe;
-                if (ntl * 8 >= nb) continue;
-                float c[4] = {0.f, 0.f, 0.f, 0.f};
-                for (int ks = 0; ks < ksteps; ++ks) {
-                    const int row = mt * 16 + (lane & 15);
-                    const uint32_t off = (uint32_t)((row * p.vpitch + ks * 16 + (lane >> 4) * 8) * 2);
-                    uint32_t ah[4], al[4];
-                    ptx::ldsm_x4(row < nt ? vh_u + off : zero_u, ah[0], ah[1], ah[2], ah[3]);
-                    ptx::ldsm_x4(row < nt ? vl_u + off : zero_u, al[0], al[1], al[2], al[3]);
-                    uint32_t b0, b1;
-                    ptx::ldsm_x2_t(base + (uint32_t)((ntl * r16 + ks * 16 + (lane & 15)) << 4), b0,
-                                   b1);
-                    ptx::mma_bf16_16816(c, ah, b0, b1);
-                    ptx::mma_bf16_16816(c, al, b0, b1);
+            ptx::cp_async_arrive_noinc(&full[st]);
+        }
+        ptx::cp_async_wait<0>();
+        if (small && lane == 0 && *abort_flag) {  // let the bulk copies that were issued land
+            const unsigned long long t0 = ptx::globaltimer();
+            for (int it = (nItems > kStages ? nItems - kStages : 0); it < nItems; ++it)
+                while (!ptx::mbar_try_wait(&full[it % kStages], (uint32_t)((it / kStages) & 1)) &&
+                       ptx::globaltimer() - t0 < kTimeoutNs) {
                 }
-                // y(smem) = bf16(fp32(y) + s * c)
-                const int col = ntl * 8 + tq * 2;
+        }
+        __syncwarp();
+        if (kClustered) ptx::cluster_wait();
+    } else {
+        // ================================================================ compute warps
+        float* VF = reinterpret_cast<float*>(smem + p.off_vf);       // [kTT][rp]: partial, then v
+        float* RB = reinterpret_cast<float*>(smem + p.off_rb);       // exchange receive buffer
+        uint16_t* Vh = reinterpret_cast<uint16_t*>(smem + p.off_rb); // [kTT][rp+8] (aliases RB)
+        uint16_t* Vl = Vh + kTT * (p.rp + 8);
+        const int vpitch = p.rp + 8;
+        const uint32_t vf_u = base_u + p.off_vf, rb_u = base_u + p.off_rb;
+        const uint32_t red1_u = ptx::smem_u32(red1), red2_u = ptx::smem_u32(red2);
+
+        // small tiles: thread owns 8 columns (chunk c) of A over rows k = rg, rg + rstride, ...;
+        // chunks per row are padded to a power of two (ncbp) so a warp reduces by shuffles
+        const int ncb = r8 >> 3;
+        const int lg = ncb <= 1 ? 0 : (ncb <= 2 ? 1 : (ncb <= 4 ? 2 : 3));
+        const int ncbp = 1 << lg;
+        const int c_own = tid & (ncbp - 1), rg = tid >> lg, rstride = kCompute >> lg;
+        // large tiles: warp w owns 16x8 output tiles [w*tpw, (w+1)*tpw) of the (Mt x r8/8) grid
+        const int nNT = r8 >> 3;
+        const int tiles_s = Mt * nNT;
+        const int tpw_s = (tiles_s + kComputeWarps - 1) / kComputeWarps;  // <= 4
+        // one register file for both paths (a tile takes exactly one of them):
+        // small: R[t*8+e] = token t, column c_own*8+e; large: R[q*4+e] = MMA tile q
+        float R[kSmallTile * 8];
+#pragma unroll
+        for (int i = 0; i < kSmallTile * 8; ++i) R[i] = 0.f;
+#define SACC(t, e) R[(t) * 8 + (e)]
+#define ACC(q) (&R[(q) * 4])
+
+        // ---- v for the expand: hi/lo operand (large tiles) or VF as is (small tiles)
+        auto stage_v = [&](auto get) {
+            if (small) {
+                for (int i = tid; i < nt * r16; i += kCompute) {
+                    const int row = i / r16, j = i - row * r16;
+                    VF[row * p.rp + j] = j < r ? get(row, j) : 0.f;
+                }
+            } else {
+                for (int i = tid; i < Mtr * r16; i += kCompute) {
+                    const int row = i / r16, j = i - row * r16;
+                    const float val = (j < r && row < nt) ? get(row, j) : 0.f;
+                    const __nv_bfloat16 h = __float2bfloat16_rn(val);
+                    const __nv_bfloat16 l = __float2bfloat16_rn(val - __bfloat162float(h));
+                    Vh[row * vpitch + j] = *reinterpret_cast<const uint16_t*>(&h);
+                    Vl[row * vpitch + j] = *reinterpret_cast<const uint16_t*>(&l);
+                }
+            }
+            ptx::named_sync(1, kCompute);
+        };
+
+        // ---- partial v of this CTA -> VF, cluster exchange, v in VF (all rows)
+        auto reduce_v = [&]() {
+            if (small) {
+                // lanes sharing a chunk (lane % ncbp) reduce by shuffles, then warps through VF
+                for (int off = 16; off >= ncbp; off >>= 1)
+#pragma unroll
+                    for (int t = 0; t < kSmallTile; ++t)
+                        if (t < nt)  // uniform
+#pragma unroll
+                            for (int e = 0; e < 8; ++e)
+                                SACC(t, e) += __shfl_xor_sync(0xffffffffu, SACC(t, e), off);
+                if (lane < ncbp) {
+#pragma unroll
+                    for (int t = 0; t < kSmallTile; ++t)
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) VF[((warp * ncbp + lane) * kSmallTile + t) * 8 + e] = SACC(t, e);
+                }
+                ptx::named_sync(1, kCompute);
+                // column j = c*8+e of token t: sum the slots of the threads that own chunk c
+                float part[2] = {0.f, 0.f};
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
-                    const int row = mt * 16 + gq + h * 8;
-                    if (row < nt) {
-                        uint32_t* py = reinterpret_cast<uint32_t*>(
-                            smem + (yb - ring_u) + swz(row, col >> 3, BN * 2) + (col & 7) * 2);
-                        __nv_bfloat162 yv = *reinterpret_cast<__nv_bfloat162*>(py);
-                        const float y0 = __bfloat162float(yv.x) + scale * c[h * 2 + 0];
-                        const float y1 = __bfloat162float(yv.y) + scale * c[h * 2 + 1];
-                        *py = pack_bf16x2(y0, y1);
+                    const int idx = tid + h * kCompute;
+                    if (idx < nt * r8) {
+                        const int t = idx / r8, j = idx - t * r8, c = j >> 3, e = j & 7;
+                        for (int w = 0; w < kComputeWarps; ++w)
+                            part[h] += VF[((w * ncbp + c) * kSmallTile + t) * 8 + e];
+                    }
+                }
+                ptx::named_sync(1, kCompute);
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int idx = tid + h * kCompute;
+                    if (idx < nt * r8) VF[(idx / r8) * p.rp + idx % r8] = part[h];
+                }
+            } else {
+                const int gq = lane >> 2, tq = lane & 3;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int t = warp * tpw_s + q;
+                    if (q < tpw_s && t < tiles_s) {
+                        const int mt = t / nNT, ntl = t - mt * nNT;
+                        const int row = mt * 16 + gq, col = ntl * 8 + tq * 2;
+                        if (row < nt)
+                            *reinterpret_cast<float2*>(&VF[row * p.rp + col]) = make_float2(ACC(q)[0], ACC(q)[1]);
+                        if (row + 8 < nt)
+                            *reinterpret_cast<float2*>(&VF[(row + 8) * p.rp + col]) =
+                                make_float2(ACC(q)[2], ACC(q)[3]);
                     }
                 }
             }
-            __syncthreads();
-            // store the updated y rows (16 B per thread, coalesced per row)
-            const int ncb = BN >> 3;
-            for (int i = tid; i < nt * ncb; i += kThreads) {
-                const int row = i / ncb, ch = i - row * ncb;
-                if (ch * 8 < nb) {
-                    const uint4 val =
-                        *reinterpret_cast<const uint4*>(smem + (yb - ring_u) + swz(row, ch, BN * 2));
-                    *reinterpret_cast<uint4*>(yg + (size_t)s_tok[row] * p.h_out + n0 + ch * 8) = val;
+            ptx::named_sync(1, kCompute);
+            ptx::cluster_wait();  // every CTA of the cluster has initialised its barriers
+            if (one_phase) {
+                for (int i = tid; i < nt * r8; i += kCompute) {
+                    const int row = i / r8, j = i - row * r8;
+                    const float val = VF[row * p.rp + j];
+                    const uint32_t off = (uint32_t)(((rank * nt + row) * r8 + j) * 4);
+                    for (int d = 0; d < C; ++d)
+                        ptx::st_async_f32(ptx::mapa(rb_u + off, d), val, ptx::mapa(red1_u, d));
+                }
+            } else {
+                for (int i = tid; i < nt * r8; i += kCompute) {
+                    const int row = i / r8, j = i - row * r8;
+                    const uint32_t off = (uint32_t)(((rank * rows_per + row / C) * r8 + j) * 4);
+                    ptx::st_async_f32(ptx::mapa(rb_u + off, row % C), VF[row * p.rp + j],
+                                      ptx::mapa(red1_u, row % C));
                 }
             }
+            wait_all<true>(red1, 0, abort_flag, status, 0x200);
+            ptx::named_sync(1, kCompute);  // every thread of this CTA has sent its share
+            if (one_phase) {
+                for (int i = tid; i < nt * r8; i += kCompute) {
+                    const int row = i / r8, j = i - row * r8;
+                    float s = 0.f;
+                    for (int c = 0; c < C; ++c) s += RB[(c * nt + row) * r8 + j];
+                    VF[row * p.rp + j] = s;
+                }
+            } else {
+                // VF is written by the peers from here on; this CTA's partial was sent already
+                for (int i = tid; i < mine * r8; i += kCompute) {
+                    const int li = i / r8, j = i - li * r8;
+                    const int row = rank + li * C;
+                    float s = 0.f;
+                    for (int c = 0; c < C; ++c) s += RB[(c * rows_per + li) * r8 + j];
+                    const uint32_t off = (uint32_t)((row * p.rp + j) * 4);
+                    for (int d = 0; d < C; ++d)
+                        ptx::st_async_f32(ptx::mapa(vf_u + off, d), s, ptx::mapa(red2_u, d));
+                }
+                wait_all<true>(red2, 0, abort_flag, status, 0x400);
+            }
+            ptx::named_sync(1, kCompute);
+            if (MODE == SGMV_SHRINK) {
+                for (int i = tid; i < nt * p.r_max; i += kCompute) {
+                    const int row = i / p.r_max, j = i - row * p.r_max;
+                    if (row % C == rank)
+                        p.v[((size_t)slice * p.T + s_tok[row]) * p.r_max + j] = j < r ? VF[row * p.rp + j] : 0.f;
+                }
+            } else if (!small) {
+                stage_v([&](int row, int j) { return VF[row * p.rp + j]; });
+            }
+        };
+
+        if (MODE == SGMV_EXPAND)
+            stage_v([&](int row, int j) { return p.v[((size_t)slice * p.T + s_tok[row]) * p.r_max + j]; });
+
+        // hoisted large-tile shrink addressing: warp tiles (mt, ntl)
+        int l_mt[4], l_ntl[4];
+        bool l_ok[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int t = warp * tpw_s + q;
+            l_ok[q] = q < tpw_s && t < tiles_s;
+            l_mt[q] = l_ok[q] ? t / nNT : 0;
+            l_ntl[q] = l_ok[q] ? t - l_mt[q] * nNT : 0;
         }
 
-        if (it == nK - 1 && MODE != SGMV_EXPAND) finish_shrink();
+        for (int it = 0; it < nK; ++it) {
+            // -------------------------------------------------------- shrink k-block
+            const int st = it % kStages;
+            const uint32_t ph = (uint32_t)((it / kStages) & 1);
+            const uint32_t base = base_u + st * SB;
+            const bool ok = wait_all<false>(&full[st], ph, abort_flag, status, 0x800) && !*abort_flag;
+            const int k0 = k_begin + it * BK;
+            const int kb = min(BK, k_begin + k_len - k0);
+            const uint32_t xb = base + (uint32_t)(BK * apitch);
+            if (ok && small) {
+                if (c_own < ncb) {
+                    for (int k = rg; k < kb; k += rstride) {
+                        const uint4 av = *reinterpret_cast<const uint4*>(smem + (base - base_u) + k * apitch + c_own * 16);
+                        const float af[8] = {bf16_lo(av.x), bf16_hi(av.x), bf16_lo(av.y), bf16_hi(av.y),
+                                             bf16_lo(av.z), bf16_hi(av.z), bf16_lo(av.w), bf16_hi(av.w)};
+#pragma unroll
+                        for (int t = 0; t < kSmallTile; ++t) {
+                            if (t < nt) {
+                                const float xv = __uint_as_float(
+                                    (uint32_t)(*reinterpret_cast<const uint16_t*>(smem + (xb - base_u) + t * xp + k * 2))
+                                    << 16);
+#pragma unroll
+                                for (int e = 0; e < 8; ++e) SACC(t, e) = fmaf(xv, af[e], SACC(t, e));
+                            }
+                        }
+                    }
+                }
+            } else if (ok) {
+                const int ksteps = (kb + 15) >> 4;
+                uint32_t xaddr[4], aaddr[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    xaddr[q] = xb + (uint32_t)((l_mt[q] * 16 + (lane & 15)) * xp + (lane >> 4) * 16);
+                    aaddr[q] = base + (uint32_t)((lane & 15) * apitch + l_ntl[q] * 16);
+                }
+                for (int ks = 0; ks < ksteps; ++ks) {
+                    uint32_t af[4][4], bf[4][2];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        if (l_ok[q]) {
+                            if (q == 0 || l_mt[q] != l_mt[q - 1])
+                                ptx::ldsm_x4(xaddr[q] + ks * 32, af[q][0], af[q][1], af[q][2], af[q][3]);
+                            else
+#pragma unroll
+                                for (int e = 0; e < 4; ++e) af[q][e] = af[q - 1][e];
+                            ptx::ldsm_x2_t(aaddr[q] + (uint32_t)(ks * 16 * apitch), bf[q][0], bf[q][1]);
+                        }
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        if (l_ok[q]) ptx::mma_bf16_16816(ACC(q), af[q], bf[q][0], bf[q][1]);
+                }
+            }
+            ptx::named_sync(1, kCompute);
+            if (tid == 0) ptx::mbar_arrive(&empty[st]);
+        }
+        if (MODE != SGMV_EXPAND) reduce_v();
+
+        for (int it = nK; it < nItems; ++it) {
+            // -------------------------------------------------------- expand n-block
+            const int st = it % kStages;
+            const uint32_t ph = (uint32_t)((it / kStages) & 1);
+            const uint32_t base = base_u + st * SB;
+            const bool ok = wait_all<false>(&full[st], ph, abort_flag, status, 0x800) && !*abort_flag;
+            const int n0 = n_begin + (it - nK) * BN;
+            const int nb = min(BN, n_begin + n_len - n0);
+            const uint32_t yb = base + (uint32_t)(r16 * bp);
+            if (ok && small) {
+                // one column pair per thread: y[t][n..n+1] += s * sum_j v[t][j] * B[j][n..n+1]
+                for (int pp = tid; pp < (nb >> 1); pp += kCompute) {
+                    const int n = pp * 2;
+                    float s0[kSmallTile], s1[kSmallTile];
+#pragma unroll
+                    for (int t = 0; t < kSmallTile; ++t) s0[t] = s1[t] = 0.f;
+                    const uint8_t* bcol = smem + (base - base_u) + n * 2;
+                    for (int j = 0; j < r; ++j) {
+                        const uint32_t bw = *reinterpret_cast<const uint32_t*>(bcol + j * bp);
+                        const float b0 = bf16_lo(bw), b1 = bf16_hi(bw);
+#pragma unroll
+                        for (int t = 0; t < kSmallTile; ++t)
+                            if (t < nt) {
+                                const float vv = VF[t * p.rp + j];
+                                s0[t] = fmaf(vv, b0, s0[t]);
+                                s1[t] = fmaf(vv, b1, s1[t]);
+                            }
+                    }
+#pragma unroll
+                    for (int t = 0; t < kSmallTile; ++t)
+                        if (t < nt) {
+                            const uint32_t yw = *reinterpret_cast<const uint32_t*>(smem + (yb - base_u) + t * bp + n * 2);
+                            *reinterpret_cast<uint32_t*>(yg + (size_t)s_tok[t] * p.h_out + n0 + n) =
+                                pack_bf16x2(bf16_lo(yw) + scale * s0[t], bf16_hi(yw) + scale * s1[t]);
+                        }
+                }
+            } else if (ok) {
+                const int nNTe = (nb + 7) >> 3;
+                const int tiles_e = Mt * nNTe;
+                const int tpw_e = (tiles_e + kComputeWarps - 1) / kComputeWarps;
+                const int ksteps = r16 >> 4;
+                const int gq = lane >> 2, tq = lane & 3;
+                const uint32_t vh_u = ptx::smem_u32(Vh), vl_u = ptx::smem_u32(Vl);
+                for (int q = 0; q < tpw_e; ++q) {
+                    const int t = warp * tpw_e + q;
+                    if (t >= tiles_e) break;
+                    const int mt = t / nNTe, ntl = t - mt * nNTe;
+                    const int row = mt * 16 + (lane & 15);
+                    const uint32_t voff = (uint32_t)((row * vpitch + (lane >> 4) * 8) * 2);
+                    const uint32_t bbase = base + (uint32_t)((lane & 15) * bp + ntl * 16);
+                    uint32_t ah[4][4], al[4][4], b[4][2];
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)
+                        if (ks < ksteps) {
+                            ptx::ldsm_x4(vh_u + voff + ks * 32, ah[ks][0], ah[ks][1], ah[ks][2], ah[ks][3]);
+                            ptx::ldsm_x4(vl_u + voff + ks * 32, al[ks][0], al[ks][1], al[ks][2], al[ks][3]);
+                            ptx::ldsm_x2_t(bbase + ks * 16 * bp, b[ks][0], b[ks][1]);
+                        }
+                    float c[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)
+                        if (ks < ksteps) {
+                            ptx::mma_bf16_16816(c[0], ah[ks], b[ks][0], b[ks][1]);
+                            ptx::mma_bf16_16816(c[1], al[ks], b[ks][0], b[ks][1]);
+                        }
+                    const int col = ntl * 8 + tq * 2;
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const int rr = mt * 16 + gq + h * 8;
+                        if (rr < nt) {
+                            uint32_t* py = reinterpret_cast<uint32_t*>(smem + (yb - base_u) + rr * bp + col * 2);
+                            const uint32_t yw = *py;
+                            *py = pack_bf16x2(bf16_lo(yw) + scale * (c[0][h * 2] + c[1][h * 2]),
+                                              bf16_hi(yw) + scale * (c[0][h * 2 + 1] + c[1][h * 2 + 1]));
+                        }
+                    }
+                }
+            }
+            // large tiles: updated y rows -> global, 16 bytes per thread, coalesced (uniform branch)
+            if (!small) {
+                ptx::named_sync(1, kCompute);
+                if (ok) {
+                    const int nch = nb >> 3;
+                    for (int i = tid; i < nt * nch; i += kCompute) {
+                        const int rr = i / nch, ch = i - rr * nch;
+                        *reinterpret_cast<uint4*>(yg + (size_t)s_tok[rr] * p.h_out + n0 + ch * 8) =
+                            *reinterpret_cast<const uint4*>(smem + (yb - base_u) + rr * bp + ch * 16);
+                    }
+                }
+            }
+            ptx::named_sync(1, kCompute);
+            if (tid == 0) ptx::mbar_arrive(&empty[st]);
+        }
     }
-    ptx::cp_async_wait<0>();
-    if (MODE == SGMV_APPLY) ptx::cluster_wait();  // peers may read this CTA's sR until here
+    // no CTA leaves while a peer may still address its shared memory
+    if (kClustered) ptx::cluster_sync();
+}
+#undef SACC
+#undef ACC
+
+template <int MODE>
+cudaError_t launch_mode(const SgmvParams& p, dim3 grid, int C, size_t smem, cudaStream_t stream)
+{
+    auto kern = sgmv_kernel<MODE>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    int n = 0;
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+    if (MODE != SGMV_EXPAND) {
+        attr[n].id = cudaLaunchAttributeClusterDimension;
+        attr[n].val.clusterDim.x = (unsigned)C;
+        attr[n].val.clusterDim.y = 1;
+        attr[n].val.clusterDim.z = 1;
+        ++n;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = n;
+    return cudaLaunchKernelEx(&cfg, kern, p);
 }
 
 }  // namespace
@@ -399,7 +660,8 @@ cudaError_t launch_sgmv(int mode, const void* x, int64_t x_slice_stride, const l
                         bool pdl_trigger)
 {
     (void)pdl_trigger;
-    SgmvParams p;
+    if (seg.T == 0) return cudaSuccess;
+    SgmvParams p = {};
     p.x = static_cast<const uint16_t*>(x);
     p.x_slice_stride = x_slice_stride;
     p.A = static_cast<const uint16_t*>(pool.A);
@@ -407,9 +669,7 @@ cudaError_t launch_sgmv(int mode, const void* x, int64_t x_slice_stride, const l
     p.ranks = pool.ranks;
     p.scales = pool.scales;
     p.perm = seg.perm;
-    p.indptr = seg.indptr;
-    p.active = seg.active;
-    p.tile_ptr = seg.tile_ptr;
+    p.tiles = reinterpret_cast<const int4*>(seg.tiles);
     p.counts = seg.counts;
     p.v = v;
     p.y = static_cast<uint16_t*>(y);
@@ -418,55 +678,36 @@ cudaError_t launch_sgmv(int mode, const void* x, int64_t x_slice_stride, const l
     p.h_in = pool.h_in;
     p.h_out = pool.h_out;
     p.r_max = pool.r_max;
-    if (seg.T == 0) return cudaSuccess;
-
-    // CTAs per tile: enough h_in per CTA to amortise the tile set-up
-    int C = (pool.h_in + 255) / 256;
+    int C = (pool.h_in + 511) / 512;
     C = C < 1 ? 1 : (C > kMaxCluster ? kMaxCluster : C);
     p.csize = C;
-    p.kc = ((pool.h_in + C - 1) / C + 7) / 8 * 8;
-    p.nc = ((pool.h_out + C - 1) / C + 7) / 8 * 8;
+    p.kc = ((pool.h_in + C - 1) / C + 63) / 64 * 64;
+    p.nc = ((pool.h_out + C - 1) / C + 63) / 64 * 64;
     p.rp = (pool.r_max + 15) / 16 * 16;
-    p.vpitch = p.rp + 8;
+    // stages: 32 KB while the v buffers stay small, 24 KB otherwise (2 CTAs per SM)
+    p.stage_bytes = p.rp <= 16 ? 32768 : 24576;
 
-    const int max_tiles = (pool.n_adapters < seg.T ? pool.n_adapters : seg.T) +
-                          (seg.T + LORA_TILE_TOKENS - 1) / LORA_TILE_TOKENS;
-    const size_t v_bytes = (size_t)kTT * p.rp * 4;                 // sP / sR
-    const size_t vhl_bytes = (size_t)2 * kTT * p.vpitch * 2;       // hi + lo
-    const size_t smem = kStages * kStageBytes + (v_bytes > vhl_bytes ? v_bytes : vhl_bytes) + v_bytes;
-    // (layout: ring | sP or hi/lo v | sR; must match the kernel)
+    // shared memory: ring | exchange buffer (aliased by the hi/lo operand) | v | barriers
+    const size_t ring = (size_t)kStages * p.stage_bytes;
+    const size_t rows_per = (kTT + C - 1) / C;
+    size_t rb = (size_t)C * rows_per * p.rp * 4;
+    if (rb < (size_t)kOnePhaseBytes) rb = kOnePhaseBytes;
+    const size_t hilo = (size_t)2 * kTT * (p.rp + 8) * 2;
+    if (rb < hilo) rb = hilo;
+    rb = (rb + 127) / 128 * 128;
+    size_t vf = (size_t)kTT * p.rp * 4;
+    const size_t partials = (size_t)kComputeWarps * 8 * kSmallTile * 8 * 4;  // small-tile warp partials
+    if (vf < partials) vf = partials;
+    p.off_rb = (uint32_t)ring;
+    p.off_vf = (uint32_t)(ring + rb);
+    p.off_bar = (uint32_t)(ring + rb + vf);
+    const size_t smem = p.off_bar + 8 * (2 * kStages + 2) + 128;  // + base alignment slack
 
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(max_tiles * C), (unsigned)pool.n_slices, 1);
-    cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    int nattr = 0;
-    if (mode != SGMV_EXPAND) {
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = (unsigned)C;
-        attr[0].val.clusterDim.y = 1;
-        attr[0].val.clusterDim.z = 1;
-        nattr = 1;
-    }
-    cfg.attrs = attr;
-    cfg.numAttrs = nattr;
-
-    cudaError_t e;
+    const dim3 grid((unsigned)(max_tiles_for(seg.T, pool.n_adapters) * C), (unsigned)pool.n_slices, 1);
     switch (mode) {
-    case SGMV_SHRINK:
-        e = cudaFuncSetAttribute(sgmv_kernel<SGMV_SHRINK>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        return cudaLaunchKernelEx(&cfg, sgmv_kernel<SGMV_SHRINK>, p);
-    case SGMV_EXPAND:
-        e = cudaFuncSetAttribute(sgmv_kernel<SGMV_EXPAND>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        return cudaLaunchKernelEx(&cfg, sgmv_kernel<SGMV_EXPAND>, p);
-    default:
-        e = cudaFuncSetAttribute(sgmv_kernel<SGMV_APPLY>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        return cudaLaunchKernelEx(&cfg, sgmv_kernel<SGMV_APPLY>, p);
+    case SGMV_SHRINK: return launch_mode<SGMV_SHRINK>(p, grid, C, smem, stream);
+    case SGMV_EXPAND: return launch_mode<SGMV_EXPAND>(p, grid, C, smem, stream);
+    default: return launch_mode<SGMV_APPLY>(p, grid, C, smem, stream);
     }
 }
 

@@ -32,7 +32,8 @@ LORA_OP_FP8_GEMM = 3
 EXPORTED = [
     "lora_workspace_size", "lora_workspace_init", "lora_workspace_status", "lora_build_segments",
     "lora_shrink", "lora_expand", "lora_apply", "fp8_quantize_rows", "fp8_gemm_lora_epilogue",
-    "lora_status_string", "lora_version", "lora_tile_tokens",
+    "lora_status_string", "lora_version", "lora_tile_tokens", "lora_max_tiles",
+    "lora_segments_status",
 ]
 
 
@@ -55,7 +56,7 @@ class lora_pool_t(ctypes.Structure):
 
 class lora_segments_t(ctypes.Structure):
     _fields_ = [("perm", ctypes.c_void_p), ("indptr", ctypes.c_void_p),
-                ("active", ctypes.c_void_p), ("tile_ptr", ctypes.c_void_p),
+                ("active", ctypes.c_void_p), ("tiles", ctypes.c_void_p),
                 ("tok_adapter", ctypes.c_void_p), ("counts", ctypes.c_void_p),
                 ("T", ctypes.c_int32), ("n_adapters", ctypes.c_int32)]
 
@@ -89,6 +90,8 @@ def load(path: str = LIB_PATH):
             "lora_status_string": (ctypes.c_char_p, [I]),
             "lora_version": (I, []),
             "lora_tile_tokens": (I, []),
+            "lora_max_tiles": (I, [I, I]),
+            "lora_segments_status": (I, [P, P, P]),
         }
         for name, (res, args) in sig.items():
             f = getattr(lib, name)
@@ -116,6 +119,11 @@ def _stream(stream):
 
 def tile_tokens() -> int:
     return load().lora_tile_tokens()
+
+
+def max_tiles(T: int, n_adapters: int) -> int:
+    """Rows of Segments.tiles (same formula as lora_max_tiles)."""
+    return min(n_adapters, T) + (T + 63) // 64
 
 
 class Pool:
@@ -148,11 +156,11 @@ class Segments:
         self.perm = torch.empty(max(T, 1), **i32)
         self.indptr = torch.empty(n_adapters + 1, **i32)
         self.active = torch.empty(n_adapters, **i32)
-        self.tile_ptr = torch.empty(n_adapters + 1, **i32)
+        self.tiles = torch.empty((max(max_tiles(T, n_adapters), 1), 4), **i32)
         self.tok_adapter = torch.empty(max(T, 1), **i32)
-        self.counts = torch.empty(4, **i32)
+        self.counts = torch.zeros(8, **i32)
         self.c = lora_segments_t(self.perm.data_ptr(), self.indptr.data_ptr(),
-                                 self.active.data_ptr(), self.tile_ptr.data_ptr(),
+                                 self.active.data_ptr(), self.tiles.data_ptr(),
                                  self.tok_adapter.data_ptr(), self.counts.data_ptr(), T,
                                  n_adapters)
 
@@ -179,6 +187,12 @@ def workspace(op: int, T: int, K: int = 0, pool: Pool | None = None, device="cud
 def lora_workspace_status(ws: torch.Tensor, stream=None) -> tuple[int, int]:
     detail = ctypes.c_uint32(0)
     st = load().lora_workspace_status(_ptr(ws), ws.numel(), _stream(stream), ctypes.byref(detail))
+    return st, detail.value
+
+
+def lora_segments_status(seg: "Segments", stream=None) -> tuple[int, int]:
+    detail = ctypes.c_uint32(0)
+    st = load().lora_segments_status(ctypes.byref(seg.c), _stream(stream), ctypes.byref(detail))
     return st, detail.value
 
 

@@ -74,6 +74,7 @@ typedef enum {
  * e.g. q/k/v/o of one layer, applied in one call).
  *   A      bf16 [n_slices][n_adapters][h_in][r_max]
  *   B      bf16 [n_slices][n_adapters][r_max][h_out]
+ *   r_max  the padded rank of the pool: 8, 16, 32 or 64.
  *   ranks  int32 [n_adapters], each in 1..r_max; NULL = every adapter has rank r_max.
  *          Entries of A with column >= r_i and of B with row >= r_i are never read.
  *   scales fp32 [n_adapters] (s_i); NULL = 1.0.
@@ -99,22 +100,36 @@ typedef struct {
  *   indptr      int32 [n_adapters+1]: adapter a owns perm[indptr[a] .. indptr[a+1]);
  *               indptr[n_adapters] = number of tokens with an adapter.
  *   active      int32 [n_adapters]: ids with >= 1 token, ascending; -1 after n_active.
- *   tile_ptr    int32 [n_adapters+1]: prefix sums over active segments of
- *               ceil(count / LORA_TILE_TOKENS); entries past n_active hold the total.
+ *   tiles       int32 [lora_max_tiles(T, n_adapters)][4]: every active segment
+ *               cut, in order, into runs of at most LORA_TILE_TOKENS tokens:
+ *               {adapter, first position in perm, token count, segment index};
+ *               the rows after the last run are {-1, 0, 0, -1}. One row is one
+ *               unit of work of the SGMV kernels.
  *   tok_adapter int32 [T]: the id each token is served with (-1: none or bad id).
- *   counts      int32 [4]: n_valid, n_active, n_bad_ids, n_tiles.
+ *   counts      int32 [8]: n_valid, n_active, n_bad_ids, n_tiles, then a device
+ *               status word (0 = ok; set by a kernel using these segments whose
+ *               bounded wait gave up, see lora_segments_status) and 3 reserved.
  * T and n_adapters are host values describing the arrays.
  */
 typedef struct {
     int32_t* perm;
     int32_t* indptr;
     int32_t* active;
-    int32_t* tile_ptr;
+    int32_t* tiles;
     int32_t* tok_adapter;
     int32_t* counts;
     int32_t T;
     int32_t n_adapters;
 } lora_segments_t;
+
+/*
+ * Read and clear the status word of a segments object (counts[4]):
+ * synchronises `stream`; LORA_OK, or LORA_ERR_TIMEOUT if an SGMV kernel that
+ * used these segments gave up on a bounded wait (its output is then
+ * undefined). *detail (host, may be NULL) receives the raw word. The word is
+ * also cleared by every lora_build_segments on the same object.
+ */
+LORA_API int lora_segments_status(const lora_segments_t* seg, lora_stream_t stream, uint32_t* detail);
 
 /* Operation codes for lora_workspace_size. */
 #define LORA_OP_SHRINK 0
@@ -226,9 +241,13 @@ LORA_API int fp8_gemm_lora_epilogue(const void* x, int M, int K, int N, const ui
 /* Static string for a status code. */
 LORA_API const char* lora_status_string(int status);
 
-/* Library version, and the tile size kernels assume for lora_segments_t.tile_ptr. */
+/* Library version, and the tile size kernels assume for lora_segments_t.tiles. */
 LORA_API int lora_version(void);
 LORA_API int lora_tile_tokens(void);
+
+/* Rows of lora_segments_t.tiles for a batch of T tokens over n_adapters:
+ * min(n_adapters, T) + ceil(T / LORA_TILE_TOKENS); -1 for invalid arguments. */
+LORA_API int lora_max_tiles(int T, int n_adapters);
 
 #ifdef __cplusplus
 }

@@ -36,10 +36,11 @@ def _check_segments(ids, n_adapters):
     torch.cuda.synchronize()
     want = oracle.build_segments(ids, n_adapters, TT)
     counts = seg.counts.cpu().numpy()
-    assert counts.tolist() == want["counts"].tolist()
+    assert counts[:4].tolist() == want["counts"].tolist()
+    assert counts[4:].tolist() == [0, 0, 0, 0]
     assert seg.indptr.cpu().numpy().tolist() == want["indptr"].tolist()
     assert seg.active.cpu().numpy().tolist() == want["active"].tolist()
-    assert seg.tile_ptr.cpu().numpy().tolist() == want["tile_ptr"].tolist()
+    assert seg.tiles.cpu().numpy()[:len(want["tiles"])].tolist() == want["tiles"].tolist()
     if T:
         assert seg.perm.cpu().numpy()[:T].tolist() == want["perm"].tolist()
         assert seg.tok_adapter.cpu().numpy()[:T].tolist() == want["tok_adapter"].tolist()
@@ -77,8 +78,8 @@ def test_segments_sync_check_reports_bad_ids():
 
 # ------------------------------------------------------------------ problems
 
-def _small(seed, T=150, n_adapters=6, h_in=520, h_out=392, r_max=24, kind="zipf", n_slices=1,
-           rank_choices=(1, 5, 8, 13, 24), none_frac=0.1):
+def _small(seed, T=150, n_adapters=6, h_in=520, h_out=392, r_max=32, kind="zipf", n_slices=1,
+           rank_choices=(1, 5, 8, 13, 24, 32), none_frac=0.1):
     return wl.make_lora_problem("t", seed, T=T, n_adapters=n_adapters, h_in=h_in, h_out=h_out,
                                 r_max=r_max, ids_kind=kind, none_frac=none_frac,
                                 rank_choices=rank_choices, n_slices=n_slices)
@@ -93,6 +94,10 @@ SMALL_CASES = {
                           n_slices=3, h_in=640, h_out=512),
     "tiny_dims": dict(seed=15, T=7, n_adapters=2, h_in=8, h_out=8, r_max=8, rank_choices=(3, 8)),
     "single_token": dict(seed=16, T=1, n_adapters=1, none_frac=0.0),
+    "medium_tiles": dict(seed=17, T=120, n_adapters=10, h_in=1024, h_out=768, r_max=16,
+                         rank_choices=(16,), kind="uniform"),
+    "rank8_pool": dict(seed=18, T=33, n_adapters=4, h_in=256, h_out=136, r_max=8,
+                       rank_choices=(3, 8)),
 }
 
 

@@ -46,6 +46,9 @@ def test_library_is_sm100a_only():
 def test_version_and_constants(lib):
     assert lib.lora_version() >= 1
     assert lib.lora_tile_tokens() == 64
+    assert lib.lora_max_tiles(36, 32) == 32 + 1
+    assert lib.lora_max_tiles(512, 256) == 256 + 8
+    assert lib.lora_max_tiles(-1, 4) == -1
     assert lib.lora_status_string(L.LORA_ERR_TIMEOUT).decode()
 
 
@@ -76,6 +79,7 @@ def _seg(T=8, n=4):
 @pytest.mark.parametrize("bad,code", [
     (dict(r_max=72), L.LORA_ERR_UNSUPPORTED),
     (dict(r_max=12), L.LORA_ERR_INVALID_ARG),
+    (dict(r_max=24), L.LORA_ERR_UNSUPPORTED),
     (dict(h_in=100), L.LORA_ERR_INVALID_ARG),
     (dict(A=None), L.LORA_ERR_INVALID_ARG),
     (dict(A=24), L.LORA_ERR_INVALID_ARG),            # misaligned

@@ -116,10 +116,12 @@ def _segments_by_sort(ids, n_adapters, tile_t):
     counts = [sum(1 for t in range(T) if key[t][0] == a) for a in range(n_adapters + 1)]
     indptr = [sum(counts[:a]) for a in range(n_adapters + 1)]
     active = [a for a in range(n_adapters) if counts[a] > 0]
-    tiles = [(counts[a] + tile_t - 1) // tile_t for a in active]
-    tile_ptr = [sum(tiles[:s]) for s in range(len(active) + 1)]
+    tiles = []
+    for s, a in enumerate(active):
+        for off in range(0, counts[a], tile_t):
+            tiles.append([a, indptr[a] + off, min(tile_t, counts[a] - off), s])
     n_bad = sum(1 for i in ids if i != -1 and not (0 <= i < n_adapters))
-    return order, indptr, active, tile_ptr, n_bad
+    return order, indptr, active, tiles, n_bad
 
 
 SEG_KINDS = ["distinct", "identical", "uniform", "zipf", "sorted_zipf", "none", "bad", "single"]
@@ -140,13 +142,15 @@ def test_segments_match_sorted_order(kind):
     else:
         ids = wl.make_ids(kind, rng, 50, n_adapters, none_frac=0.1)
     seg = oracle.build_segments(ids, n_adapters, tile_t)
-    order, indptr, active, tile_ptr, n_bad = _segments_by_sort(list(ids), n_adapters, tile_t)
+    order, indptr, active, tiles, n_bad = _segments_by_sort(list(ids), n_adapters, tile_t)
     assert seg["perm"].tolist() == order
     assert seg["indptr"].tolist() == indptr
     n_active = len(active)
-    assert seg["counts"].tolist() == [indptr[n_adapters], n_active, n_bad, tile_ptr[-1]]
+    assert seg["counts"].tolist() == [indptr[n_adapters], n_active, n_bad, len(tiles)]
     assert seg["active"][:n_active].tolist() == active
-    assert seg["tile_ptr"][:n_active + 1].tolist() == tile_ptr
+    assert seg["tiles"][:len(tiles)].tolist() == tiles
+    assert (seg["tiles"][len(tiles):] == [-1, 0, 0, -1]).all()
+    assert len(tiles) <= oracle.max_tiles(len(ids), n_adapters, tile_t)
     want_tok = [i if 0 <= i < n_adapters else -1 for i in ids]
     assert seg["tok_adapter"].tolist() == want_tok
 
