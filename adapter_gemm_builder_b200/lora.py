@@ -33,7 +33,7 @@ EXPORTED = [
     "lora_workspace_size", "lora_workspace_init", "lora_workspace_status", "lora_build_segments",
     "lora_shrink", "lora_expand", "lora_apply", "fp8_quantize_rows", "fp8_gemm_lora_epilogue",
     "lora_status_string", "lora_version", "lora_tile_tokens", "lora_max_tiles",
-    "lora_segments_status",
+    "lora_segments_status", "fp8_gemm_lora_epilogue_noalloc", "lora_noalloc_scratch_bytes",
 ]
 
 
@@ -92,6 +92,8 @@ def load(path: str = LIB_PATH):
             "lora_tile_tokens": (I, []),
             "lora_max_tiles": (I, [I, I]),
             "lora_segments_status": (I, [P, P, P]),
+            "fp8_gemm_lora_epilogue_noalloc": (I, [P, I, I, I, P, P, P, P, P, P]),
+            "lora_noalloc_scratch_bytes": (Z, []),
         }
         for name, (res, args) in sig.items():
             f = getattr(lib, name)
@@ -242,3 +244,14 @@ def fp8_gemm_lora_epilogue(x: torch.Tensor, Wq: torch.Tensor, w_scale: torch.Ten
     _check(load().fp8_gemm_lora_epilogue(
         _ptr(x), M, K, N, _ptr(Wq), _ptr(w_scale), ctypes.byref(pool.c) if pool else None,
         ctypes.byref(seg.c) if seg else None, _ptr(y), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def fp8_gemm_lora_epilogue_noalloc(x: torch.Tensor, Wq: torch.Tensor, w_scale: torch.Tensor,
+                                   pool: Pool | None, seg: Segments | None, y: torch.Tensor,
+                                   stream=None) -> None:
+    """fp8_gemm_lora_epilogue without a caller workspace (scratch inside the library)."""
+    M, K = x.shape
+    N = Wq.shape[0]
+    _check(load().fp8_gemm_lora_epilogue_noalloc(
+        _ptr(x), M, K, N, _ptr(Wq), _ptr(w_scale), ctypes.byref(pool.c) if pool else None,
+        ctypes.byref(seg.c) if seg else None, _ptr(y), _stream(stream)))

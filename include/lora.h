@@ -238,6 +238,32 @@ LORA_API int fp8_gemm_lora_epilogue(const void* x, int M, int K, int N, const ui
                            const lora_segments_t* seg, void* y, void* ws, size_t ws_bytes,
                            lora_stream_t stream);
 
+/*
+ * fp8_gemm_lora_epilogue for callers that cannot allocate device memory
+ * (the pages have no counterpart of this call): for example a plugin inside
+ * a serving engine that plans all device memory itself and only hands over
+ * inputs and outputs, or a hot path that must not call cudaMalloc, which can
+ * synchronise the device. Same arguments and results as
+ * fp8_gemm_lora_epilogue, minus the workspace: the scratch space lives in a
+ * fixed array of lora_noalloc_scratch_bytes() (8 MiB) inside the library's
+ * own device memory, held by every GPU that loads the library until the
+ * process exits. Calls whose workspace would exceed it return
+ * LORA_ERR_WORKSPACE. The call allocates nothing (no cudaMalloc or
+ * cudaFree); it clears the array's status word with a stream-ordered memset.
+ * The first call on each device looks up the array's device address (with
+ * that device current); make that first call before any stream capture.
+ * Every call shares the one array: calls that may overlap on the GPU (other
+ * streams, other threads) race on it and must be ordered by the caller.
+ * lora_workspace_status() does not apply; a bounded-wait timeout is not
+ * reported by this entry point.
+ */
+LORA_API int fp8_gemm_lora_epilogue_noalloc(const void* x, int M, int K, int N, const uint8_t* Wq,
+                                            const float* w_scale, const lora_pool_t* pool,
+                                            const lora_segments_t* seg, void* y, lora_stream_t stream);
+
+/* Bytes of the built-in scratch array used by fp8_gemm_lora_epilogue_noalloc. */
+LORA_API size_t lora_noalloc_scratch_bytes(void);
+
 /* Static string for a status code. */
 LORA_API const char* lora_status_string(int status);
 
