@@ -60,6 +60,11 @@ bool encode_tmap_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, ui
                     uint64_t outer, uint64_t row_stride_bytes, uint32_t box_inner,
                     uint32_t box_outer, CUtensorMapSwizzle swz);
 
+// 3-D tiled tensor map: dims innermost first, strides (bytes) of dims 1 and 2;
+// out-of-range box elements are filled with zeros. false on failure.
+bool encode_tmap_3d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, const uint64_t dims[3],
+                    const uint64_t strides_bytes[2], const uint32_t box[3], CUtensorMapSwizzle swz);
+
 // Slot of the device status word in lora_segments_t.counts.
 constexpr int kSegStatusSlot = 4;
 

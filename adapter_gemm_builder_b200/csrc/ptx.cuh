@@ -172,6 +172,16 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, uint
         "l"(reinterpret_cast<uint64_t>(tmap)), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
         : "memory");
 }
+// 3-D tiled tensor load (no multicast), completion as transaction bytes on `bar`.
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const void* tmap, uint64_t* bar, int32_t c0,
+                                            int32_t c1, int32_t c2)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5}], [%2];\n" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
+        : "memory");
+}
 
 // 1-D bulk copy global -> this CTA's shared memory (16-byte aligned
 // addresses, size a multiple of 16); completion as transaction bytes on `bar`.
@@ -214,6 +224,16 @@ __device__ __forceinline__ void st_async_f32(uint32_t addr, float v, uint32_t re
 {
     asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];\n" ::"r"(addr),
                  "r"(__float_as_uint(v)), "r"(remote_bar)
+                 : "memory");
+}
+// Four floats (16-byte aligned) to a peer's shared memory, counted as 16
+// transaction bytes on its mbarrier.
+__device__ __forceinline__ void st_async_f32x4(uint32_t addr, float4 v, uint32_t remote_bar)
+{
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];\n" ::"r"(
+                     addr),
+                 "r"(__float_as_uint(v.x)), "r"(__float_as_uint(v.y)), "r"(__float_as_uint(v.z)),
+                 "r"(__float_as_uint(v.w)), "r"(remote_bar)
                  : "memory");
 }
 __device__ __forceinline__ void st_cluster_f32(uint32_t addr, float v)

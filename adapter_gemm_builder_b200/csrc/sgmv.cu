@@ -15,13 +15,19 @@
 // the slice (projection) index, so q/k/v/o run in one launch.
 //
 // Memory path (the kernel is bound by HBM bytes and by latency). A producer
-// warp fills a ring of 3 stages with 16-byte cp.async from all 32 lanes,
-// completing on the stage's mbarrier: the k rows of A_a (only its r8 columns;
-// bytes past the rank are zero-filled, so the pool's padding is never read),
-// the gathered x rows of the tile's tokens, then the r rows of B_a and the
-// gathered y rows. Row pitches are padded by 16 bytes so that the ldmatrix
-// reads of the tensor-core path are free of bank conflicts. A decode tile
-// (one token, rank 16) moves its whole A and B slices in one stage each.
+// warp fills a ring of 3 stages whose copies all complete on the stage's
+// mbarrier. The k rows of A_a come as tensor-map boxes of only the adapter's
+// live columns (128-, 64- or 32-byte swizzled rows: the pool's padding past
+// the rank is never read and the tensor-core reads are free of bank
+// conflicts) or, for a decode tile whose rank rounds to r_max, as one
+// contiguous 1-D bulk copy. Decode tiles take their few x, B and y rows as
+// 1-D bulk copies, issued from all lanes in parallel (a copy instruction
+// costs ~35 ns of issue, so one lane issuing many small copies would
+// serialise). Tensor-core tiles keep x, B_a and y in blocks of 64 columns
+// whose 128-byte rows are swizzled (bank-conflict free for ldmatrix): B_a
+// comes as tensor-map boxes, and so do x and y when the tile's tokens are
+// consecutive rows (pre-sorted batches); otherwise the rows are gathered with
+// 16-byte cp.async spread over all 32 lanes, written in the same layout.
 //
 // Math. Tiles of at most 4 tokens (decode) use CUDA-core FMAs: the products
 // are few and a 16-row MMA would be mostly padding. Larger tiles use bf16
@@ -40,6 +46,7 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
+#include <string.h>
 
 #include "internal.h"
 #include "ptx.cuh"
@@ -57,6 +64,17 @@ constexpr int kOnePhaseBytes = 8192;     // all-to-all exchange of v up to this 
 constexpr int kSmallTile = 4;            // tiles of <= 4 tokens use CUDA-core FMAs
 constexpr unsigned long long kTimeoutNs = 2000000000ull;
 
+// Tensor maps of the pools. a[i]: A viewed as {r_max, h_in, n_slices *
+// n_adapters}, box {8 << i, 64, 1} (swizzle = the box row width);
+// b[i]: B viewed as {h_out, r_max, n_slices * n_adapters}, box
+// {64, min(16 (i + 1), r_max), 1}, 128-byte swizzle.
+// x: {h_in, T, slices of x}, y: {h_out, T, n_slices}, box {64, 16, 1}, 128-byte swizzle.
+struct AMaps {
+    CUtensorMap m[4];
+    CUtensorMap b[4];
+    CUtensorMap x, y;
+};
+
 struct SgmvParams {
     const uint16_t* x;
     long long x_slice_stride;
@@ -71,9 +89,10 @@ struct SgmvParams {
     uint16_t* y;
     int T, n_adapters, h_in, h_out, r_max;
     int csize;       // CTAs per tile
-    int kc, nc;      // h_in / h_out slice per CTA (multiples of 64 except at the end)
+    int kc, nc;      // h_in / h_out slice per CTA (kc a multiple of 128, nc of 64)
     int rp;          // round_up(r_max, 16): row pitch (floats) of the v buffers
     int stage_bytes; // one ring stage
+    int xy_maps;     // tensor maps of x and y are valid (consecutive-row tiles use them)
     uint32_t off_rb, off_vf, off_bar;
 };
 
@@ -87,6 +106,40 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// Byte offset of 16-byte chunk c of A row k in a stage: rows are `pitch` bytes;
+// a swizzled tensor-map box XORs the chunk index with bits 7.. of the row's
+// offset (mask `swz`: 7, 3, 1 for 128-, 64-, 32-byte rows; 0 unswizzled).
+__device__ __forceinline__ uint32_t a_chunk(int k, int c, int pitch, int swz)
+{
+    const uint32_t off = (uint32_t)(k * pitch);
+    return off + (uint32_t)((c ^ (int)((off >> 7) & (uint32_t)swz)) << 4);
+}
+
+// Byte offset of 16-byte chunk c (8 columns) of row `row` in a block-swizzled
+// tile: blocks of 64 columns, each `rows` rows of 128 bytes, 128-byte swizzle.
+__device__ __forceinline__ uint32_t blk_chunk(int row, int c, int rows)
+{
+    return (uint32_t)((c >> 3) * rows * 128 + row * 128 + (((c & 7) ^ (row & 7)) << 4));
+}
+
+// Gather `nt` rows of `cpr` 16-byte chunks with cp.async from all 32 lanes:
+// row i of the tile is global row tok[i] (src + tok[i] * row_elems), written
+// block-swizzled at dst.
+__device__ __forceinline__ void gather_rows(uint32_t dst, const uint16_t* src, size_t row_elems,
+                                            const int* tok, int nt, int cpr, int rows, int lane)
+{
+    if (cpr <= 32 && (cpr & (cpr - 1)) == 0) {  // whole blocks: no division
+        const int lg = __ffs(cpr) - 1, c = lane & (cpr - 1);
+        for (int row = lane >> lg; row < nt; row += 32 >> lg)
+            ptx::cp_async16(dst + blk_chunk(row, c, rows), src + (size_t)tok[row] * row_elems + c * 8, 16);
+    } else {
+        for (int i = lane; i < nt * cpr; i += 32) {
+            const int row = i / cpr, c = i - row * cpr;
+            ptx::cp_async16(dst + blk_chunk(row, c, rows), src + (size_t)tok[row] * row_elems + c * 8, 16);
+        }
+    }
+}
 
 // Bounded wait by ONE thread; on expiry raises the CTA abort flag and the
 // status word. The clock and the abort flag are read every 256 probes only.
@@ -128,15 +181,15 @@ __device__ bool wait_all(uint64_t* bar, uint32_t parity, volatile int* abort_fla
 
 template <int MODE>
 __global__ void __launch_bounds__(kThreads, 2)
-sgmv_kernel(const SgmvParams p)
+sgmv_kernel(const __grid_constant__ AMaps am, const SgmvParams p)
 {
-    extern __shared__ __align__(128) uint8_t smem_raw[];
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
     __shared__ int s_tok[kTT];
     __shared__ int s_abort;
 
     constexpr bool kClustered = MODE != SGMV_EXPAND;
     const uint32_t raw_u = ptx::smem_u32(smem_raw);
-    const uint32_t base_u = (raw_u + 127u) & ~127u;
+    const uint32_t base_u = (raw_u + 1023u) & ~1023u;  // swizzled boxes need 1024-byte alignment
     uint8_t* smem = smem_raw + (base_u - raw_u);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int C = p.csize;
@@ -154,7 +207,7 @@ sgmv_kernel(const SgmvParams p)
     if (tid == 0) {
         s_abort = 0;
         for (int s = 0; s < kStages; ++s) {
-            ptx::mbar_init(&full[s], 32);  // the 32 producer lanes' cp.async groups
+            ptx::mbar_init(&full[s], 33);  // lane 0's expect_tx + one arrival per producer lane
             ptx::mbar_init(&empty[s], 1);
         }
         ptx::mbar_init(red1, 1);
@@ -179,21 +232,48 @@ sgmv_kernel(const SgmvParams p)
     if (tid < nt) s_tok[tid] = p.perm[tok0 + tid];
 
     // ---- geometry (identical in every role)
-    // bytes per A row in shared memory: small tiles take the contiguous rows of the pool
-    // with one bulk copy (r_max columns); large tiles take r8 columns with a padded pitch
-    const int apitch = small ? p.r_max * 2 : r8 * 2 + 16;
+    // A rows in shared memory: tensor-map boxes of rA >= r live columns (rA the power of
+    // two >= r8; dense, swizzled when rA >= 16), or for decode tiles whose rank rounds to
+    // r_max the pool's contiguous rows
+    const int a_map = r8 <= 8 ? 0 : 32 - __clz((r8 >> 3) - 1);  // log2(rA / 8)
+    const int rA = 8 << a_map;
+    const bool a_tma = !small || rA < p.r_max;
+    const int apitch = a_tma ? rA * 2 : p.r_max * 2;
+    const int a_swz = (a_tma && rA >= 16) ? (rA >> 3) - 1 : 0;
     const int k_begin = min(p.h_in, rank * p.kc);
     const int k_len = min(p.h_in, k_begin + p.kc) - k_begin;
-    int BK = ((SB - 16 * Mtr) / (apitch + 2 * Mtr)) / 64 * 64;
-    BK = min(BK, round_up(max(k_len, 1), 64));
+    int BK;
+    if (small) {
+        BK = ((SB - 16 * Mtr) / (apitch + 2 * Mtr)) / 64 * 64;
+        BK = min(BK, round_up(max(k_len, 1), 64));
+    } else {
+        // a divisor of kc (a multiple of 128), so only the last block of h_in is partial
+        BK = 64;
+        for (int b = 256; b > 64; b >>= 1)
+            if (p.kc % b == 0 && b * (apitch + 2 * Mtr) <= SB) {
+                BK = b;
+                break;
+            }
+    }
     const int nK = (MODE == SGMV_EXPAND) ? 0 : (k_len + BK - 1) / BK;
-    const int xp = BK * 2 + 16;  // x row pitch (bytes)
+    const int xp = BK * 2 + 16;  // x row pitch of decode tiles (bytes)
     const int n_begin = min(p.h_out, rank * p.nc);
     const int n_len = min(p.h_out, n_begin + p.nc) - n_begin;
-    int BN = ((SB / (r16 + Mtr) - 16) / 2) / 64 * 64;
+    // expand blocks: decode tiles keep B rows j < r and y rows at the padded pitch bp;
+    // tensor-core tiles keep B (r16 rows) and y (Mtr rows) in swizzled 64-column blocks
+    int BN;
+    if (small) {
+        BN = ((SB / (r16 + Mtr) - 16) / 2) / 64 * 64;
+    } else {
+        BN = 64;  // a power of two, so the gathers need no division
+        while (BN < 256 && 2 * BN * (2 * r16 + 2 * Mtr) <= SB) BN *= 2;
+    }
     BN = min(BN, round_up(max(n_len, 1), 64));
     const int nN = (MODE == SGMV_SHRINK) ? 0 : (n_len + BN - 1) / BN;
-    const int bp = BN * 2 + 16;  // B and y row pitch (bytes)
+    const int bp = BN * 2 + 16;  // y row pitch (and B row pitch of decode tiles), bytes
+    const int b_map = (r16 >> 4) - 1;
+    const int rB = min(r16, p.r_max);                               // rows per B box
+    const uint32_t y_off = small ? (uint32_t)(r16 * bp) : (uint32_t)((BN >> 6) * r16 * 128);
     const int nItems = nK + nN;
     const size_t sa = (size_t)slice * p.n_adapters + a;
     const uint16_t* Ag = p.A + sa * (size_t)p.h_in * p.r_max;
@@ -214,89 +294,101 @@ sgmv_kernel(const SgmvParams p)
 
     if (warp == kComputeWarps) {
         // ================================================================ producer warp
+        if (lane == 0 && a_tma && nK > 0) ptx::tma_prefetch_desc(&am.m[a_map]);
+        if (lane == 0 && !small && nN > 0) ptx::tma_prefetch_desc(&am.b[b_map]);
+        // consecutive token rows (a pre-sorted batch): x and y rows come as tensor-map boxes
+        bool contig = false;
+        if (!small && p.xy_maps) {
+            const int t0 = s_tok[0];
+            contig = __all_sync(0xffffffffu, (lane >= nt || s_tok[lane] == t0 + lane) &&
+                                                 (lane + 32 >= nt || s_tok[lane + 32] == t0 + lane + 32));
+        }
+        const int xs = p.x_slice_stride ? slice : 0;
+        int issued = 0;
         for (int it = 0; it < nItems; ++it) {
             const int st = it % kStages;
             const uint32_t ph = (uint32_t)((it / kStages) & 1);
             if (!wait_all<false>(&empty[st], ph ^ 1, abort_flag, status, 0x100)) break;
             const uint32_t base = base_u + st * SB;
-            if (small) {
-                // decode-sized tile: a handful of 1-D bulk copies, all issued by lane 0
-                if (lane == 0) {
-                    if (it < nK) {
-                        const int k0 = k_begin + it * BK;
-                        const int kb = min(BK, k_begin + k_len - k0);
-                        const uint32_t xb = base + (uint32_t)(BK * apitch);
-                        ptx::mbar_arrive_expect_tx(&full[st], (uint32_t)((p.r_max + nt) * kb * 2));
-                        ptx::bulk_g2s(base, Ag + (size_t)k0 * p.r_max, (uint32_t)(kb * p.r_max * 2), &full[st]);
-                        for (int row = 0; row < nt; ++row)
-                            ptx::bulk_g2s(xb + row * xp, xg + (size_t)s_tok[row] * p.h_in + k0, (uint32_t)(kb * 2),
-                                          &full[st]);
-                    } else {
-                        const int n0 = n_begin + (it - nK) * BN;
-                        const int nb = min(BN, n_begin + n_len - n0);
-                        const uint32_t yb = base + (uint32_t)(r16 * bp);
-                        ptx::mbar_arrive_expect_tx(&full[st], (uint32_t)((r + nt) * nb * 2));
-                        for (int j = 0; j < r; ++j)
-                            ptx::bulk_g2s(base + j * bp, Bg + (size_t)j * p.h_out + n0, (uint32_t)(nb * 2), &full[st]);
-                        for (int row = 0; row < nt; ++row)
-                            ptx::bulk_g2s(yb + row * bp, yg + (size_t)s_tok[row] * p.h_out + n0, (uint32_t)(nb * 2),
-                                          &full[st]);
-                    }
-                } else {
-                    ptx::mbar_arrive(&full[st]);
-                }
-                continue;
-            }
+            // lane 0 announces the stage's tensor-map / bulk bytes before any lane issues a
+            // copy; then every lane arrives once its own copies have landed (33 arrivals)
             if (it < nK) {
                 const int k0 = k_begin + it * BK;
                 const int kb = min(BK, k_begin + k_len - k0);
-                // A rows k0 .. k0+BK (rows >= kb and bytes past the rank zero-filled);
-                // (row, 16-byte chunk) pairs spread over the lanes, chunks padded to a power of 2
-                const int ncb = r8 >> 3;
-                const int lgc = ncb <= 1 ? 0 : (ncb <= 2 ? 1 : (ncb <= 4 ? 2 : 3));
-                for (int i = lane; i < (BK << lgc); i += 32) {
-                    const int kk = i >> lgc, c = i & ((1 << lgc) - 1);
-                    if (c < ncb) {
-                        const int valid = kk < kb ? min(8, r - c * 8) : 0;
-                        ptx::cp_async16(base + kk * apitch + c * 16,
-                                        valid > 0 ? Ag + (size_t)(k0 + kk) * p.r_max + c * 8 : Ag,
-                                        valid > 0 ? valid * 2 : 0);
-                    }
-                }
-                // x rows of the tile's tokens (rows >= nt and columns >= kb zero-filled)
+                const int nbox = (kb + 63) >> 6;  // 64-row boxes; rows past h_in read as zero
                 const uint32_t xb = base + (uint32_t)(BK * apitch);
-                for (int row = 0; row < Mtr; ++row) {
-                    const uint16_t* src = xg + (size_t)s_tok[row < nt ? row : 0] * p.h_in + k0;
-                    for (int ch = lane; ch < (BK >> 3); ch += 32) {
-                        const bool ok = row < nt && ch * 8 < kb;
-                        ptx::cp_async16(xb + row * xp + ch * 16, ok ? src + ch * 8 : xg, ok ? 16 : 0);
-                    }
+                if (lane == 0) {
+                    uint32_t bytes = a_tma ? (uint32_t)(nbox * 64 * apitch) : (uint32_t)(kb * apitch);
+                    if (small) bytes += (uint32_t)(nt * kb * 2);
+                    else if (contig) bytes += (uint32_t)(nbox * Mt * 16 * 128);
+                    ptx::mbar_arrive_expect_tx(&full[st], bytes);
+                }
+                __syncwarp();
+                // one copy instruction per lane (a copy costs ~150 ns of issue to its thread):
+                // lanes 0..nA-1 the A boxes (or the one A bulk copy), then the x boxes or rows
+                const int nA = a_tma ? nbox : 1;
+                if (lane < nA) {
+                    if (a_tma)
+                        ptx::tma_load_3d(base + (uint32_t)(lane * 64 * apitch), &am.m[a_map], &full[st], 0,
+                                         k0 + lane * 64, (int)sa);
+                    else
+                        ptx::bulk_g2s(base, Ag + (size_t)k0 * p.r_max, (uint32_t)(kb * apitch), &full[st]);
+                }
+                if (small) {
+                    for (int row = lane - nA; row < nt; row += 32)
+                        if (row >= 0)
+                            ptx::bulk_g2s(xb + row * xp, xg + (size_t)s_tok[row] * p.h_in + k0, (uint32_t)(kb * 2),
+                                          &full[st]);
+                    ptx::mbar_arrive(&full[st]);
+                } else {
+                    if (contig)  // columns past h_in read as zero
+                        for (int i = lane - nA; i < nbox * Mt; i += 32)
+                            if (i >= 0)
+                                ptx::tma_load_3d(xb + (uint32_t)(((i / Mt) * Mtr + (i % Mt) * 16) * 128), &am.x, &full[st],
+                                                 k0 + (i / Mt) * 64, s_tok[0] + (i % Mt) * 16, xs);
+                    if (!contig) gather_rows(xb, xg + k0, (size_t)p.h_in, s_tok, nt, kb >> 3, Mtr, lane);
+                    ptx::cp_async_arrive_noinc(&full[st]);
                 }
             } else {
                 const int n0 = n_begin + (it - nK) * BN;
                 const int nb = min(BN, n_begin + n_len - n0);
-                // B rows 0 .. r16 (rows >= r zero-filled), columns n0 .. n0+BN
-                for (int j = 0; j < r16; ++j)
-                    for (int ch = lane; ch < (BN >> 3); ch += 32) {
-                        const bool ok = j < r && ch * 8 < nb;
-                        ptx::cp_async16(base + j * bp + ch * 16, ok ? Bg + (size_t)j * p.h_out + n0 + ch * 8 : Bg,
-                                        ok ? 16 : 0);
+                const uint32_t yb = base + y_off;
+                if (small) {
+                    if (lane == 0) ptx::mbar_arrive_expect_tx(&full[st], (uint32_t)((r + nt) * nb * 2));
+                    __syncwarp();
+                    for (int i = lane; i < r + nt; i += 32) {
+                        if (i < r)
+                            ptx::bulk_g2s(base + i * bp, Bg + (size_t)i * p.h_out + n0, (uint32_t)(nb * 2), &full[st]);
+                        else
+                            ptx::bulk_g2s(yb + (i - r) * bp, yg + (size_t)s_tok[i - r] * p.h_out + n0,
+                                          (uint32_t)(nb * 2), &full[st]);
                     }
-                const uint32_t yb = base + (uint32_t)(r16 * bp);
-                for (int row = 0; row < Mtr; ++row) {
-                    const uint16_t* src = yg + (size_t)s_tok[row < nt ? row : 0] * p.h_out + n0;
-                    for (int ch = lane; ch < (BN >> 3); ch += 32) {
-                        const bool ok = row < nt && ch * 8 < nb;
-                        ptx::cp_async16(yb + row * bp + ch * 16, ok ? src + ch * 8 : yg, ok ? 16 : 0);
-                    }
+                    ptx::mbar_arrive(&full[st]);
+                } else {
+                    const int nbox = (nb + 63) >> 6;
+                    if (lane == 0)
+                        ptx::mbar_arrive_expect_tx(&full[st], (uint32_t)(nbox * 64 * rB * 2) +
+                                                                  (contig ? (uint32_t)(nbox * Mt * 16 * 128) : 0u));
+                    __syncwarp();
+                    if (lane < nbox)
+                        ptx::tma_load_3d(base + (uint32_t)(lane * r16 * 128), &am.b[b_map], &full[st], n0 + lane * 64,
+                                         0, (int)sa);
+                    if (contig)
+                        for (int i = lane - nbox; i < nbox * Mt; i += 32)
+                            if (i >= 0)
+                                ptx::tma_load_3d(yb + (uint32_t)(((i / Mt) * Mtr + (i % Mt) * 16) * 128), &am.y,
+                                                 &full[st], n0 + (i / Mt) * 64, s_tok[0] + (i % Mt) * 16, slice);
+                    if (!contig) gather_rows(yb, yg + n0, (size_t)p.h_out, s_tok, nt, nb >> 3, Mtr, lane);
+                    ptx::cp_async_arrive_noinc(&full[st]);
                 }
             }
-            ptx::cp_async_arrive_noinc(&full[st]);
+            ++issued;
         }
+        ptx::cp_async_commit();
         ptx::cp_async_wait<0>();
-        if (small && lane == 0 && *abort_flag) {  // let the bulk copies that were issued land
+        if (lane == 0 && *abort_flag) {  // let the copies that were issued land before leaving
             const unsigned long long t0 = ptx::globaltimer();
-            for (int it = (nItems > kStages ? nItems - kStages : 0); it < nItems; ++it)
+            for (int it = (issued > kStages ? issued - kStages : 0); it < issued; ++it)
                 while (!ptx::mbar_try_wait(&full[it % kStages], (uint32_t)((it / kStages) & 1)) &&
                        ptx::globaltimer() - t0 < kTimeoutNs) {
                 }
@@ -404,41 +496,48 @@ sgmv_kernel(const SgmvParams p)
             }
             ptx::named_sync(1, kCompute);
             ptx::cluster_wait();  // every CTA of the cluster has initialised its barriers
+            // 16-byte pieces: 4 consecutive columns j of one row
+            const int q8 = r8 >> 2;
+            auto add4 = [](float4 a4, float4 b4) {
+                return make_float4(a4.x + b4.x, a4.y + b4.y, a4.z + b4.z, a4.w + b4.w);
+            };
             if (one_phase) {
-                for (int i = tid; i < nt * r8; i += kCompute) {
-                    const int row = i / r8, j = i - row * r8;
-                    const float val = VF[row * p.rp + j];
+                for (int i = tid; i < nt * q8; i += kCompute) {
+                    const int row = i / q8, j = (i - row * q8) * 4;
+                    const float4 val = *reinterpret_cast<const float4*>(&VF[row * p.rp + j]);
                     const uint32_t off = (uint32_t)(((rank * nt + row) * r8 + j) * 4);
                     for (int d = 0; d < C; ++d)
-                        ptx::st_async_f32(ptx::mapa(rb_u + off, d), val, ptx::mapa(red1_u, d));
+                        ptx::st_async_f32x4(ptx::mapa(rb_u + off, d), val, ptx::mapa(red1_u, d));
                 }
             } else {
-                for (int i = tid; i < nt * r8; i += kCompute) {
-                    const int row = i / r8, j = i - row * r8;
+                for (int i = tid; i < nt * q8; i += kCompute) {
+                    const int row = i / q8, j = (i - row * q8) * 4;
                     const uint32_t off = (uint32_t)(((rank * rows_per + row / C) * r8 + j) * 4);
-                    ptx::st_async_f32(ptx::mapa(rb_u + off, row % C), VF[row * p.rp + j],
-                                      ptx::mapa(red1_u, row % C));
+                    ptx::st_async_f32x4(ptx::mapa(rb_u + off, row % C),
+                                        *reinterpret_cast<const float4*>(&VF[row * p.rp + j]), ptx::mapa(red1_u, row % C));
                 }
             }
             wait_all<true>(red1, 0, abort_flag, status, 0x200);
             ptx::named_sync(1, kCompute);  // every thread of this CTA has sent its share
             if (one_phase) {
-                for (int i = tid; i < nt * r8; i += kCompute) {
-                    const int row = i / r8, j = i - row * r8;
-                    float s = 0.f;
-                    for (int c = 0; c < C; ++c) s += RB[(c * nt + row) * r8 + j];
-                    VF[row * p.rp + j] = s;
+                for (int i = tid; i < nt * q8; i += kCompute) {
+                    const int row = i / q8, j = (i - row * q8) * 4;
+                    float4 s4 = make_float4(0.f, 0.f, 0.f, 0.f);
+                    for (int c = 0; c < C; ++c)
+                        s4 = add4(s4, *reinterpret_cast<const float4*>(&RB[(c * nt + row) * r8 + j]));
+                    *reinterpret_cast<float4*>(&VF[row * p.rp + j]) = s4;
                 }
             } else {
                 // VF is written by the peers from here on; this CTA's partial was sent already
-                for (int i = tid; i < mine * r8; i += kCompute) {
-                    const int li = i / r8, j = i - li * r8;
+                for (int i = tid; i < mine * q8; i += kCompute) {
+                    const int li = i / q8, j = (i - li * q8) * 4;
                     const int row = rank + li * C;
-                    float s = 0.f;
-                    for (int c = 0; c < C; ++c) s += RB[(c * rows_per + li) * r8 + j];
+                    float4 s4 = make_float4(0.f, 0.f, 0.f, 0.f);
+                    for (int c = 0; c < C; ++c)
+                        s4 = add4(s4, *reinterpret_cast<const float4*>(&RB[(c * rows_per + li) * r8 + j]));
                     const uint32_t off = (uint32_t)((row * p.rp + j) * 4);
                     for (int d = 0; d < C; ++d)
-                        ptx::st_async_f32(ptx::mapa(vf_u + off, d), s, ptx::mapa(red2_u, d));
+                        ptx::st_async_f32x4(ptx::mapa(vf_u + off, d), s4, ptx::mapa(red2_u, d));
                 }
                 wait_all<true>(red2, 0, abort_flag, status, 0x400);
             }
@@ -480,7 +579,8 @@ sgmv_kernel(const SgmvParams p)
             if (ok && small) {
                 if (c_own < ncb) {
                     for (int k = rg; k < kb; k += rstride) {
-                        const uint4 av = *reinterpret_cast<const uint4*>(smem + (base - base_u) + k * apitch + c_own * 16);
+                        const uint4 av =
+                            *reinterpret_cast<const uint4*>(smem + (base - base_u) + a_chunk(k, c_own, apitch, a_swz));
                         const float af[8] = {bf16_lo(av.x), bf16_hi(av.x), bf16_lo(av.y), bf16_hi(av.y),
                                              bf16_lo(av.z), bf16_hi(av.z), bf16_lo(av.w), bf16_hi(av.w)};
 #pragma unroll
@@ -497,19 +597,30 @@ sgmv_kernel(const SgmvParams p)
                 }
             } else if (ok) {
                 const int ksteps = (kb + 15) >> 4;
-                uint32_t xaddr[4], aaddr[4];
+                if (kb & 15) {  // last block of h_in: x columns kb..kb+8 may hold stale bytes; zero them
+                    if (tid < nt)
+                        *reinterpret_cast<uint4*>(smem + (xb - base_u) + blk_chunk(tid, kb >> 3, Mtr)) =
+                            make_uint4(0, 0, 0, 0);
+                    ptx::fence_proxy_async_smem();  // generic writes to a stage that bulk copies refill
+                    ptx::named_sync(1, kCompute);
+                }
+                // x rows in swizzled 64-column blocks: row (l_mt*16 + lane%16), k chunk 2*ks + lane/16
+                uint32_t xrow[4], aaddr[4];
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
-                    xaddr[q] = xb + (uint32_t)((l_mt[q] * 16 + (lane & 15)) * xp + (lane >> 4) * 16);
-                    aaddr[q] = base + (uint32_t)((lane & 15) * apitch + l_ntl[q] * 16);
+                    xrow[q] = xb + (uint32_t)((l_mt[q] * 16 + (lane & 15)) * 128);
+                    aaddr[q] = base + a_chunk(lane & 15, l_ntl[q], apitch, a_swz);
                 }
+                const int xr7 = lane & 7, xhi = lane >> 4;
                 for (int ks = 0; ks < ksteps; ++ks) {
+                    const uint32_t xoff =
+                        (uint32_t)((ks >> 2) * Mtr * 128 + (((((ks & 3) << 1) | xhi) ^ xr7) << 4));
                     uint32_t af[4][4], bf[4][2];
 #pragma unroll
                     for (int q = 0; q < 4; ++q)
                         if (l_ok[q]) {
                             if (q == 0 || l_mt[q] != l_mt[q - 1])
-                                ptx::ldsm_x4(xaddr[q] + ks * 32, af[q][0], af[q][1], af[q][2], af[q][3]);
+                                ptx::ldsm_x4(xrow[q] + xoff, af[q][0], af[q][1], af[q][2], af[q][3]);
                             else
 #pragma unroll
                                 for (int e = 0; e < 4; ++e) af[q][e] = af[q - 1][e];
@@ -533,7 +644,7 @@ sgmv_kernel(const SgmvParams p)
             const bool ok = wait_all<false>(&full[st], ph, abort_flag, status, 0x800) && !*abort_flag;
             const int n0 = n_begin + (it - nK) * BN;
             const int nb = min(BN, n_begin + n_len - n0);
-            const uint32_t yb = base + (uint32_t)(r16 * bp);
+            const uint32_t yb = base + y_off;
             if (ok && small) {
                 // one column pair per thread: y[t][n..n+1] += s * sum_j v[t][j] * B[j][n..n+1]
                 for (int pp = tid; pp < (nb >> 1); pp += kCompute) {
@@ -562,26 +673,40 @@ sgmv_kernel(const SgmvParams p)
                         }
                 }
             } else if (ok) {
+                if (r != r16) {  // B rows r..r16 of every box hold padding or nothing: zero them
+                    const int zr = r16 - r, nbx = (nb + 63) >> 6;
+                    for (int i = tid; i < nbx * zr * 8; i += kCompute) {
+                        const int bx = i / (zr * 8), rem = i - bx * zr * 8;
+                        *reinterpret_cast<uint4*>(smem + (base - base_u) + bx * r16 * 128 + (r + (rem >> 3)) * 128 +
+                                                  (rem & 7) * 16) = make_uint4(0, 0, 0, 0);
+                    }
+                    ptx::fence_proxy_async_smem();  // generic writes to a stage that bulk copies refill
+                    ptx::named_sync(1, kCompute);
+                }
                 const int nNTe = (nb + 7) >> 3;
                 const int tiles_e = Mt * nNTe;
                 const int tpw_e = (tiles_e + kComputeWarps - 1) / kComputeWarps;
                 const int ksteps = r16 >> 4;
                 const int gq = lane >> 2, tq = lane & 3;
                 const uint32_t vh_u = ptx::smem_u32(Vh), vl_u = ptx::smem_u32(Vl);
-                for (int q = 0; q < tpw_e; ++q) {
+                for (int q0 = 0; q0 < tpw_e; q0 += 4)
+#pragma unroll
+                for (int q = q0; q < q0 + 4; ++q) {  // 4 tiles unrolled so their MMA chains overlap
                     const int t = warp * tpw_e + q;
-                    if (t >= tiles_e) break;
+                    if (q >= tpw_e || t >= tiles_e) continue;
                     const int mt = t / nNTe, ntl = t - mt * nNTe;
                     const int row = mt * 16 + (lane & 15);
                     const uint32_t voff = (uint32_t)((row * vpitch + (lane >> 4) * 8) * 2);
-                    const uint32_t bbase = base + (uint32_t)((lane & 15) * bp + ntl * 16);
+                    // row j = ks*16 + (lane & 15) of box ntl/8, 16-byte chunk ntl%8 XOR (j & 7)
+                    const uint32_t bbase = base + (uint32_t)((ntl >> 3) * r16 * 128 + (lane & 15) * 128 +
+                                                             ((((ntl & 7) ^ (lane & 7))) << 4));
                     uint32_t ah[4][4], al[4][4], b[4][2];
 #pragma unroll
                     for (int ks = 0; ks < 4; ++ks)
                         if (ks < ksteps) {
                             ptx::ldsm_x4(vh_u + voff + ks * 32, ah[ks][0], ah[ks][1], ah[ks][2], ah[ks][3]);
                             ptx::ldsm_x4(vl_u + voff + ks * 32, al[ks][0], al[ks][1], al[ks][2], al[ks][3]);
-                            ptx::ldsm_x2_t(bbase + ks * 16 * bp, b[ks][0], b[ks][1]);
+                            ptx::ldsm_x2_t(bbase + ks * 16 * 128, b[ks][0], b[ks][1]);
                         }
                     float c[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
@@ -595,7 +720,8 @@ sgmv_kernel(const SgmvParams p)
                     for (int h = 0; h < 2; ++h) {
                         const int rr = mt * 16 + gq + h * 8;
                         if (rr < nt) {
-                            uint32_t* py = reinterpret_cast<uint32_t*>(smem + (yb - base_u) + rr * bp + col * 2);
+                            uint32_t* py =
+                                reinterpret_cast<uint32_t*>(smem + (yb - base_u) + blk_chunk(rr, ntl, Mtr) + tq * 4);
                             const uint32_t yw = *py;
                             *py = pack_bf16x2(bf16_lo(yw) + scale * (c[0][h * 2] + c[1][h * 2]),
                                               bf16_hi(yw) + scale * (c[0][h * 2 + 1] + c[1][h * 2 + 1]));
@@ -605,13 +731,19 @@ sgmv_kernel(const SgmvParams p)
             }
             // large tiles: updated y rows -> global, 16 bytes per thread, coalesced (uniform branch)
             if (!small) {
+                ptx::fence_proxy_async_smem();  // the RMW wrote a stage that bulk copies refill
                 ptx::named_sync(1, kCompute);
                 if (ok) {
                     const int nch = nb >> 3;
-                    for (int i = tid; i < nt * nch; i += kCompute) {
-                        const int rr = i / nch, ch = i - rr * nch;
+                    auto put = [&](int rr, int ch) {
                         *reinterpret_cast<uint4*>(yg + (size_t)s_tok[rr] * p.h_out + n0 + ch * 8) =
-                            *reinterpret_cast<const uint4*>(smem + (yb - base_u) + rr * bp + ch * 16);
+                            *reinterpret_cast<const uint4*>(smem + (yb - base_u) + blk_chunk(rr, ch, Mtr));
+                    };
+                    if ((nch & (nch - 1)) == 0 && nch <= 32) {
+                        const int lg = __ffs(nch) - 1;
+                        for (int rr = tid >> lg; rr < nt; rr += kCompute >> lg) put(rr, tid & (nch - 1));
+                    } else {
+                        for (int i = tid; i < nt * nch; i += kCompute) put(i / nch, i % nch);
                     }
                 }
             }
@@ -626,7 +758,7 @@ sgmv_kernel(const SgmvParams p)
 #undef ACC
 
 template <int MODE>
-cudaError_t launch_mode(const SgmvParams& p, dim3 grid, int C, size_t smem, cudaStream_t stream)
+cudaError_t launch_mode(const AMaps& am, const SgmvParams& p, dim3 grid, int C, size_t smem, cudaStream_t stream)
 {
     auto kern = sgmv_kernel<MODE>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -650,7 +782,26 @@ cudaError_t launch_mode(const SgmvParams& p, dim3 grid, int C, size_t smem, cuda
     }
     cfg.attrs = attr;
     cfg.numAttrs = n;
-    return cudaLaunchKernelEx(&cfg, kern, p);
+    return cudaLaunchKernelEx(&cfg, kern, am, p);
+}
+
+// Dynamic shared memory one CTA may take so that two fit on an SM (per device).
+size_t sgmv_smem_per_cta()
+{
+    int dev = 0;
+    cudaGetDevice(&dev);
+    static size_t cached[64] = {0};
+    if (dev >= 0 && dev < 64 && cached[dev]) return cached[dev];
+    int per_sm = 0, reserved = 0;
+    cudaDeviceGetAttribute(&per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
+    cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev);
+    cudaFuncAttributes fa;
+    size_t stat = 1024;
+    if (cudaFuncGetAttributes(&fa, sgmv_kernel<SGMV_APPLY>) == cudaSuccess) stat = fa.sharedSizeBytes;
+    if (per_sm <= 0) per_sm = 233472;
+    const size_t b = (size_t)per_sm / 2 - (size_t)reserved - stat;
+    if (dev >= 0 && dev < 64) cached[dev] = b;
+    return b;
 }
 
 }  // namespace
@@ -681,14 +832,11 @@ cudaError_t launch_sgmv(int mode, const void* x, int64_t x_slice_stride, const l
     int C = (pool.h_in + 511) / 512;
     C = C < 1 ? 1 : (C > kMaxCluster ? kMaxCluster : C);
     p.csize = C;
-    p.kc = ((pool.h_in + C - 1) / C + 63) / 64 * 64;
+    p.kc = ((pool.h_in + C - 1) / C + 127) / 128 * 128;
     p.nc = ((pool.h_out + C - 1) / C + 63) / 64 * 64;
     p.rp = (pool.r_max + 15) / 16 * 16;
-    // stages: 32 KB while the v buffers stay small, 24 KB otherwise (2 CTAs per SM)
-    p.stage_bytes = p.rp <= 16 ? 32768 : 24576;
 
     // shared memory: ring | exchange buffer (aliased by the hi/lo operand) | v | barriers
-    const size_t ring = (size_t)kStages * p.stage_bytes;
     const size_t rows_per = (kTT + C - 1) / C;
     size_t rb = (size_t)C * rows_per * p.rp * 4;
     if (rb < (size_t)kOnePhaseBytes) rb = kOnePhaseBytes;
@@ -698,16 +846,79 @@ cudaError_t launch_sgmv(int mode, const void* x, int64_t x_slice_stride, const l
     size_t vf = (size_t)kTT * p.rp * 4;
     const size_t partials = (size_t)kComputeWarps * 8 * kSmallTile * 8 * 4;  // small-tile warp partials
     if (vf < partials) vf = partials;
+    // stages (multiples of 1024 bytes, at most 32 KB) sized so that two CTAs fit on an SM
+    const size_t bars = 8 * (2 * kStages + 2);
+    const size_t fixed = rb + vf + bars + 1024;  // + base alignment slack
+    const size_t budget = sgmv_smem_per_cta();
+    if (budget <= fixed + (size_t)kStages * 8192) return cudaErrorInvalidConfiguration;
+    size_t sb = (budget - fixed) / kStages / 1024 * 1024;
+    p.stage_bytes = (int)(sb > 32768 ? 32768 : sb);
+    // a tensor-core tile (64 tokens, rank 64) needs 64-column blocks and 64-row k-blocks
+    if (p.stage_bytes < 20480) return cudaErrorInvalidConfiguration;
+    const size_t ring = (size_t)kStages * p.stage_bytes;
     p.off_rb = (uint32_t)ring;
     p.off_vf = (uint32_t)(ring + rb);
     p.off_bar = (uint32_t)(ring + rb + vf);
-    const size_t smem = p.off_bar + 8 * (2 * kStages + 2) + 128;  // + base alignment slack
+    const size_t smem = p.off_bar + bars + 1024;  // + base alignment slack
+
+    AMaps am;
+    memset(&am, 0, sizeof(am));
+    if (mode != SGMV_EXPAND) {
+        const uint64_t dims[3] = {(uint64_t)pool.r_max, (uint64_t)pool.h_in,
+                                  (uint64_t)pool.n_slices * (uint64_t)pool.n_adapters};
+        const uint64_t strides[2] = {(uint64_t)pool.r_max * 2, (uint64_t)pool.h_in * pool.r_max * 2};
+        for (int i = 0; i < 4; ++i) {
+            const int r8 = 8 << i;
+            if (r8 > pool.r_max) break;
+            const uint32_t box[3] = {(uint32_t)r8, 64, 1};
+            const CUtensorMapSwizzle swz = r8 == 8 ? CU_TENSOR_MAP_SWIZZLE_NONE
+                                         : r8 == 16 ? CU_TENSOR_MAP_SWIZZLE_32B
+                                         : r8 == 32 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                    : CU_TENSOR_MAP_SWIZZLE_128B;
+            if (!encode_tmap_3d(&am.m[i], CU_TENSOR_MAP_DATA_TYPE_UINT16, pool.A, dims, strides, box, swz))
+                return cudaErrorInvalidValue;
+        }
+    }
+    if (mode != SGMV_SHRINK) {
+        const uint64_t dims[3] = {(uint64_t)pool.h_out, (uint64_t)pool.r_max,
+                                  (uint64_t)pool.n_slices * (uint64_t)pool.n_adapters};
+        const uint64_t strides[2] = {(uint64_t)pool.h_out * 2, (uint64_t)pool.r_max * pool.h_out * 2};
+        for (int i = 0; i < 4; ++i) {
+            if (16 * i >= pool.r_max) break;
+            const int rows = 16 * (i + 1) < pool.r_max ? 16 * (i + 1) : pool.r_max;
+            const uint32_t box[3] = {64, (uint32_t)rows, 1};
+            if (!encode_tmap_3d(&am.b[i], CU_TENSOR_MAP_DATA_TYPE_UINT16, pool.B, dims, strides, box,
+                                CU_TENSOR_MAP_SWIZZLE_128B))
+                return cudaErrorInvalidValue;
+        }
+    }
+
+    // x and y as {columns, T, slices}, box {64, 16, 1}: for tiles of consecutive tokens
+    p.xy_maps = 0;
+    if (pool.h_in >= 64 && pool.h_out >= 64 && seg.T >= 16) {
+        bool ok = true;
+        const uint32_t box[3] = {64, 16, 1};
+        if (mode != SGMV_EXPAND) {
+            const uint64_t xs = x_slice_stride ? (uint64_t)x_slice_stride * 2 : (uint64_t)seg.T * pool.h_in * 2;
+            const uint64_t dims[3] = {(uint64_t)pool.h_in, (uint64_t)seg.T, x_slice_stride ? (uint64_t)pool.n_slices : 1u};
+            const uint64_t strides[2] = {(uint64_t)pool.h_in * 2, xs};
+            ok = ok && encode_tmap_3d(&am.x, CU_TENSOR_MAP_DATA_TYPE_UINT16, x, dims, strides, box,
+                                      CU_TENSOR_MAP_SWIZZLE_128B);
+        }
+        if (mode != SGMV_SHRINK) {
+            const uint64_t dims[3] = {(uint64_t)pool.h_out, (uint64_t)seg.T, (uint64_t)pool.n_slices};
+            const uint64_t strides[2] = {(uint64_t)pool.h_out * 2, (uint64_t)seg.T * pool.h_out * 2};
+            ok = ok && encode_tmap_3d(&am.y, CU_TENSOR_MAP_DATA_TYPE_UINT16, y, dims, strides, box,
+                                      CU_TENSOR_MAP_SWIZZLE_128B);
+        }
+        p.xy_maps = ok ? 1 : 0;
+    }
 
     const dim3 grid((unsigned)(max_tiles_for(seg.T, pool.n_adapters) * C), (unsigned)pool.n_slices, 1);
     switch (mode) {
-    case SGMV_SHRINK: return launch_mode<SGMV_SHRINK>(p, grid, C, smem, stream);
-    case SGMV_EXPAND: return launch_mode<SGMV_EXPAND>(p, grid, C, smem, stream);
-    default: return launch_mode<SGMV_APPLY>(p, grid, C, smem, stream);
+    case SGMV_SHRINK: return launch_mode<SGMV_SHRINK>(am, p, grid, C, smem, stream);
+    case SGMV_EXPAND: return launch_mode<SGMV_EXPAND>(am, p, grid, C, smem, stream);
+    default: return launch_mode<SGMV_APPLY>(am, p, grid, C, smem, stream);
     }
 }
 
