@@ -48,8 +48,10 @@ int check_segments(const lora_segments_t* seg, int n_adapters)
     return LORA_OK;
 }
 
+// FP8 workspace: status | xq | sx | v (with a pool) | sync words | partials.
+// [off_v, off_part) is zeroed by the quantiser on every call.
 size_t fp8_ws_layout(int M, int K, const lora_pool_t* pool, size_t* off_xq, size_t* off_sx,
-                     size_t* off_v)
+                     size_t* off_v, size_t* off_sync, size_t* off_part)
 {
     size_t off = 256;  // status word block
     *off_xq = off;
@@ -58,6 +60,10 @@ size_t fp8_ws_layout(int M, int K, const lora_pool_t* pool, size_t* off_xq, size
     off += align256((size_t)M * 4);
     *off_v = off;
     if (pool) off += align256((size_t)M * pool->r_max * 4);
+    *off_sync = off;  // [0]: down-projection count, [16 ..]: one flag per SM
+    off += align256((size_t)(16 + device_sm_count()) * 4);
+    *off_part = off;
+    off += align256(fp8_gemm_partial_bytes(M));
     return off;
 }
 
@@ -117,8 +123,9 @@ size_t lora_workspace_size(int op, int T, int K, const lora_pool_t* pool)
     case LORA_OP_FP8_GEMM: {
         if (K <= 0) return (size_t)-1;
         if (pool && check_pool(pool) != LORA_OK) return (size_t)-1;
-        size_t a, b, c;
-        return fp8_ws_layout(T, K, pool, &a, &b, &c);
+        if (T < 1) return (size_t)-1;
+        size_t a, b, c, d, e;
+        return fp8_ws_layout(T, K, pool, &a, &b, &c, &d, &e);
     }
     default: return (size_t)-1;
     }
@@ -229,7 +236,7 @@ int fp8_quantize_rows(const void* x, int M, int K, uint8_t* xq, float* sx, lora_
     if (M < 0 || K <= 0 || K % 16) return LORA_ERR_INVALID_ARG;
     if (M == 0) return LORA_OK;
     if (!x || !xq || !sx || !aligned16(x) || !aligned16(xq)) return LORA_ERR_INVALID_ARG;
-    return cuda_status(launch_quantize_rows(x, nullptr, M, K, xq, sx, (cudaStream_t)stream));
+    return cuda_status(launch_quantize_rows(x, nullptr, M, K, xq, sx, nullptr, 0, (cudaStream_t)stream));
 }
 
 int fp8_gemm_lora_epilogue(const void* x, int M, int K, int N, const uint8_t* Wq,
@@ -248,25 +255,25 @@ int fp8_gemm_lora_epilogue(const void* x, int M, int K, int N, const uint8_t* Wq
         if ((st = check_segments(seg, pool->n_adapters)) != LORA_OK) return st;
         if (seg->T != M) return LORA_ERR_INVALID_ARG;
     }
-    size_t off_xq, off_sx, off_v;
-    const size_t need = fp8_ws_layout(M, K, pool, &off_xq, &off_sx, &off_v);
+    size_t off_xq, off_sx, off_v, off_sync, off_part;
+    const size_t need = fp8_ws_layout(M, K, pool, &off_xq, &off_sx, &off_v, &off_sync, &off_part);
     if (!ws || ws_bytes < need || !aligned16(ws)) return LORA_ERR_WORKSPACE;
     uint8_t* w = static_cast<uint8_t*>(ws);
     uint32_t* status = reinterpret_cast<uint32_t*>(w);
     uint8_t* xq = w + off_xq;
     float* sx = reinterpret_cast<float*>(w + off_sx);
     float* v = pool ? reinterpret_cast<float*>(w + off_v) : nullptr;
+    int* sync = reinterpret_cast<int*>(w + off_sync);
     cudaStream_t s = (cudaStream_t)stream;
 
-    // 1. activations -> E4M3, rows in segment order when adapters are present
-    cudaError_t e = launch_quantize_rows(x, pool ? seg->perm : nullptr, M, K, xq, sx, s);
+    // 1. activations -> E4M3, rows in segment order when adapters are present; the
+    //    same kernel zeroes v and the GEMM's synchronisation words
+    cudaError_t e = launch_quantize_rows(x, pool ? seg->perm : nullptr, M, K, xq, sx, w + off_v,
+                                         (off_part - off_v) / 4, s);
     if (e != cudaSuccess) return LORA_ERR_CUDA;
-    // 2. the down-projection, launched first
-    if (pool) {
-        e = launch_sgmv(SGMV_SHRINK, x, 0, *pool, *seg, v, nullptr, s, true);
-        if (e != cudaSuccess) return LORA_ERR_CUDA;
-    }
-    // 3. the GEMM, a programmatic dependent of the shrink when there is one
+    // 2. the GEMM, a programmatic dependent of the quantiser: its weights start
+    //    streaming at once, the down-projection runs in its epilogue warps meanwhile
+    //    and the up-projection in its epilogue
     Fp8GemmArgs a = {};
     a.M = M;
     a.N = N;
@@ -277,6 +284,9 @@ int fp8_gemm_lora_epilogue(const void* x, int M, int K, int N, const uint8_t* Wq
     a.sw = w_scale;
     a.y = static_cast<uint16_t*>(y);
     a.status = status;
+    a.partials = reinterpret_cast<float*>(w + off_part);
+    a.v_done = sync;
+    a.flags = sync + 16;
     a.lora = pool != nullptr;
     if (pool) {
         a.perm = seg->perm;
@@ -285,12 +295,13 @@ int fp8_gemm_lora_epilogue(const void* x, int M, int K, int N, const uint8_t* Wq
         a.active = seg->active;
         a.counts = seg->counts;
         a.v = v;
+        a.x = static_cast<const uint16_t*>(x);
+        a.A = static_cast<const uint16_t*>(pool->A);
         a.B = static_cast<const uint16_t*>(pool->B);
         a.ranks = pool->ranks;
         a.scales = pool->scales;
         a.n_adapters = pool->n_adapters;
         a.r_max = pool->r_max;
-        a.pdl = true;
     }
     return cuda_status(launch_fp8_gemm(a, s));
 }

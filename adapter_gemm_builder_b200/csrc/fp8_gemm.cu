@@ -1,32 +1,41 @@
-// fp8_gemm.cu -- 8-bit (E4M3) base GEMM with the multi-tenant LoRA expand
-// fused into its epilogue, on the sm_100a tensor cores (tcgen05 + TMEM + TMA).
+// fp8_gemm.cu -- 8-bit (E4M3) base GEMM with the multi-tenant LoRA term fused
+// into it, on the sm_100a tensor cores (tcgen05 + TMEM + TMA).
 //
 // The EpiLoRA abstract (sentences 3-4) observes that the GEMM needs the
-// adapter's down-projection only in its epilogue; so the down-projection runs
-// first, and the GEMM -- launched as a programmatic dependent kernel -- streams
-// its weights meanwhile and adds every tenant's up-projection before the store:
-//   y[m][n] = sx[m] * sw[n] * sum_k xq[m][k] Wq[n][k] + s_a * sum_j v[m][j] B[a][j][n].
+// adapter's down-projection only in its epilogue, so the down-projection can
+// run while the weights stream:
+//   y[m][n] = sx[m] * sw[n] * sum_k xq[m][k] Wq[n][k] + s_a * sum_j v[m][j] B[a][j][n],
+//   v[m][j] = sum_k x[m][k] A[a][k][j]       (a = adapter of token m, bf16 x).
 //
 // Design for decode-sized M (tokens) and large N x K weights:
 //  * swap-AB: the MMA's M dimension is 128 rows of W, its N dimension the
 //    tokens (16..256 per tile), so W -- the bytes that bound the kernel -- is
 //    read exactly once while all tokens ride along in one MMA.
-//  * persistent CTAs (one per SM), warp-specialised:
+//  * stream-K: the (tile, k-block) units are split evenly over one persistent
+//    CTA per SM, so no SM idles in a last partial wave. A tile cut between two
+//    CTAs is finished by the CTA holding its first k-blocks (the last work of
+//    that CTA): the others store fp32 partial accumulators to the workspace
+//    first thing and raise a flag; the finisher adds them before its epilogue.
+//  * warp roles in each CTA:
 //      warp 0  TMA producer: W and xq k-blocks into a ring of stages
-//              (128-byte or 64-byte swizzle, matching the MMA descriptors);
+//              (128- or 64-byte swizzle, matching the MMA descriptors); its
+//              first W loads are issued before the wait on the quantiser;
 //      warp 1  TMEM allocator and single-thread tcgen05.mma issuer
 //              (kind::f8f6f4, fp32 accumulators in TMEM, double-buffered so the
-//              epilogue of tile i overlaps the mainloop of tile i+1);
-//      warp 2  B stager: TMA-loads the [r x 128] slices of B_a for every
-//              adapter present in the tile's token block into shared memory,
-//              while the mainloop runs;
-//      warps 3..10 epilogue: tcgen05.ld of the accumulator, per-token and
-//              per-channel scales, the LoRA term on CUDA cores from shared
-//              memory, bf16 stores.
+//              epilogue of one segment overlaps the mainloop of the next);
+//      warp 2  B stager: TMA-loads the [r x 128] slices of B_a of every
+//              adapter of the tile's token block into shared memory;
+//      warps 3..10 the down-projection first -- while the first weights
+//              stream, each CTA computes v over its own 64-column slice of K
+//              for every token (bf16 x, fp32 sums, vector atomics into v,
+//              then a completion count) -- and then the epilogue: tcgen05.ld
+//              of the accumulator, per-token and per-channel scales, the LoRA
+//              term on CUDA cores from shared memory, bf16 stores.
 //  * tokens are processed in segment order (rows of xq are permuted by the
-//    quantiser), so the adapter changes only at segment boundaries.
-//  * every mbarrier wait is bounded (2 s); on expiry the CTA records a status
-//    word in the workspace, drains what it issued and returns.
+//    quantiser, v is kept in that order), so the adapter changes only at
+//    segment boundaries.
+//  * every wait (mbarrier, flag, count) is bounded (2 s); on expiry the CTA
+//    records a status word in the workspace, drains what it issued and returns.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -39,23 +48,31 @@ namespace {
 
 constexpr int kBlockM = 128;  // W rows per tile (MMA M)
 constexpr int kEpiWarps = 8;
+constexpr int kEpiThreads = kEpiWarps * 32;
 constexpr int kThreads = (3 + kEpiWarps) * 32;
 constexpr int kMaxStages = 8;
+constexpr int kShrinkCols = 64;  // K columns of the down-projection per work item
 constexpr unsigned long long kTimeoutNs = 2000000000ull;
 
 struct GemmParams {
     int M, N, K, BN, n_tb, n_nb, num_tiles, k_blocks, stages;
+    long long units;  // num_tiles * k_blocks, split evenly over the grid
     const float* sx;
     const float* sw;
     uint16_t* y;
     uint32_t* status;
+    float* partials;  // [gridDim.x][128][BN] fp32 stream-K partial accumulators
+    int* flags;       // [gridDim.x] partial of CTA c stored
+    int* v_done;      // down-projection items finished
     int lora;
+    const uint16_t* x;  // bf16 [M][K] (unquantised, by token index)
+    const uint16_t* A;  // bf16 [n_adapters][K][r_max]
     const int32_t* perm;
     const int32_t* tok_adapter;
     const int32_t* indptr;
     const int32_t* active;
     const int32_t* counts;
-    const float* v;
+    float* v;  // fp32 [M][r_max], segment (perm) order, zeroed by the quantiser
     const uint16_t* B;
     const int32_t* ranks;
     const float* scales;
@@ -92,6 +109,25 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity)
         if (globaltimer() - t0 > kTimeoutNs) return;
 }
 
+// Bounded wait until the global counter reaches `target` (acquire, GPU scope).
+__device__ __forceinline__ bool wait_count(const int* ctr, int target, volatile int* abort_flag,
+                                           uint32_t* status, uint32_t code)
+{
+    const unsigned long long t0 = globaltimer();
+    while (true) {
+        int v;
+        asm volatile("ld.acquire.gpu.global.b32 %0, [%1];\n" : "=r"(v) : "l"(ctr) : "memory");
+        if (v >= target) return true;
+        if (*abort_flag) return false;
+        if (globaltimer() - t0 > kTimeoutNs) {
+            *abort_flag = 1;
+            if (status) atomicOr(status, code);
+            return false;
+        }
+        __nanosleep(64);
+    }
+}
+
 // UMMA shared-memory descriptor for a K-major operand tile whose rows are
 // SW bytes long (SW = 128 or 64), swizzled by TMA with the same width:
 // 8-row core groups SW*8 bytes apart (stride byte offset), version 1.
@@ -110,6 +146,23 @@ __device__ __forceinline__ uint32_t make_idesc(int n)
     return (1u << 4) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(kBlockM >> 4) << 24);
 }
 
+// Stream-K schedule: CTA c owns units [c*U/G, (c+1)*U/G) of the (tile,
+// k-block) sequence; a segment is the part of one tile inside that range.
+struct Seg {
+    int tile, kb0, kb1;
+};
+__device__ __forceinline__ long long unit_begin(long long U, int c, int G) { return U * c / G; }
+
+// Next segment starting at unit u (< u_end).
+__device__ __forceinline__ Seg seg_at(long long u, long long u_end, int KB)
+{
+    Seg s;
+    s.tile = (int)(u / KB);
+    s.kb0 = (int)(u - (long long)s.tile * KB);
+    const long long left = u_end - u;
+    s.kb1 = (left < (long long)(KB - s.kb0)) ? s.kb0 + (int)left : KB;
+    return s;
+}
 
 template <int BK, int MAXR>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -121,6 +174,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
     __shared__ int s_abort;
     __shared__ int s_nslots;
     __shared__ int s_slot_adapter[256];
+    __shared__ int s_slot_rank[256];
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     // the swizzled TMA tiles need a 1024-byte aligned base
@@ -141,6 +195,8 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
     constexpr int kStageW = kBlockM * BK;
     const int stage_bytes = kStageW + p.BN * BK;
     const uint32_t ncols = (uint32_t)(2 * p.BN <= 32 ? 32 : (2 * p.BN <= 64 ? 64 : (2 * p.BN <= 128 ? 128 : (2 * p.BN <= 256 ? 256 : 512))));
+    const int G = gridDim.x, cta = blockIdx.x, KB = p.k_blocks;
+    const long long u_begin = unit_begin(p.units, cta, G), u_end = unit_begin(p.units, cta + 1, G);
 
     if (threadIdx.x == 0) {
         s_abort = 0;
@@ -178,10 +234,25 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
             uint32_t issued_phase[kMaxStages];
             bool issued[kMaxStages];
             for (int s = 0; s < kMaxStages; ++s) issued[s] = false;
+            // the first ring of W loads goes out before the wait on the quantiser
+            // (xq is its output, W is not); their xq loads follow the wait
+            bool waited = false;
+            int n_def = 0, def_kb[kMaxStages], def_tb[kMaxStages];
+            auto flush_deferred = [&]() {
+                ptx::pdl_wait();
+                waited = true;
+                for (int d = 0; d < n_def; ++d) {
+                    const uint32_t sX = smem_u + p.ring_off + d * stage_bytes + kStageW;
+                    ptx::tma_load_2d(sX, &tmX, &full[d], def_kb[d] * BK, def_tb[d] * p.BN);
+                }
+            };
             bool ok = true;
-            for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
-                const int nb = t / p.n_tb, tb = t - nb * p.n_tb;
-                for (int kb = 0; kb < p.k_blocks; ++kb) {
+            for (long long u = u_begin; u < u_end && ok;) {
+                const Seg sg = seg_at(u, u_end, KB);
+                u += sg.kb1 - sg.kb0;
+                const int nb = sg.tile / p.n_tb, tb = sg.tile - nb * p.n_tb;
+                for (int kb = sg.kb0; kb < sg.kb1; ++kb) {
+                    if (!waited && n_def == p.stages) flush_deferred();
                     if (!wait_bounded(&empty[stage], phase ^ 1, abort_flag, p.status, 0x1u)) {
                         ok = false;
                         break;
@@ -190,7 +261,13 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
                     const uint32_t sX = sW + kStageW;
                     ptx::mbar_arrive_expect_tx(&full[stage], (uint32_t)stage_bytes);
                     ptx::tma_load_2d(sW, &tmW, &full[stage], kb * BK, nb * kBlockM);
-                    ptx::tma_load_2d(sX, &tmX, &full[stage], kb * BK, tb * p.BN);
+                    if (waited) {
+                        ptx::tma_load_2d(sX, &tmX, &full[stage], kb * BK, tb * p.BN);
+                    } else {  // first ring pass: stage == n_def
+                        def_kb[n_def] = kb;
+                        def_tb[n_def] = tb;
+                        ++n_def;
+                    }
                     issued[stage] = true;
                     issued_phase[stage] = phase;
                     if (++stage == p.stages) {
@@ -199,6 +276,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
                     }
                 }
             }
+            if (!waited) flush_deferred();
             if (!ok)  // let every load this CTA issued land before it exits
                 for (int s = 0; s < p.stages; ++s)
                     if (issued[s]) drain_wait(&full[s], issued_phase[s]);
@@ -211,7 +289,9 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
             const uint32_t idesc = make_idesc(p.BN);
             bool ok = true, any = false;
             int i = 0;
-            for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x, ++i) {
+            for (long long u = u_begin; u < u_end && ok; ++i) {
+                const Seg sg = seg_at(u, u_end, KB);
+                u += sg.kb1 - sg.kb0;
                 const int buf = i & 1;
                 const uint32_t bphase = (uint32_t)((i >> 1) & 1);
                 if (!wait_bounded(&tempty[buf], bphase ^ 1, abort_flag, p.status, 0x2u)) {
@@ -220,7 +300,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
                 }
                 ptx::tc_fence_after();
                 const uint32_t d = tmem_base + (uint32_t)(buf * p.BN);
-                for (int kb = 0; kb < p.k_blocks; ++kb) {
+                for (int kb = sg.kb0; kb < sg.kb1; ++kb) {
                     if (!wait_bounded(&full[stage], phase, abort_flag, p.status, 0x4u)) {
                         ok = false;
                         break;
@@ -230,8 +310,8 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
                     const uint32_t sX = sW + kStageW;
 #pragma unroll
                     for (int kk = 0; kk < BK / 32; ++kk)
-                        ptx::tc_mma_f8(d, make_desc<BK>(sW + kk * 32), make_desc<BK>(sX + kk * 32),
-                                       idesc, (kb | kk) != 0 ? 1u : 0u);
+                        ptx::tc_mma_f8(d, make_desc<BK>(sW + kk * 32), make_desc<BK>(sX + kk * 32), idesc,
+                                       (kb > sg.kb0 || kk != 0) ? 1u : 0u);
                     any = true;
                     ptx::tc_commit(&empty[stage]);
                     if (++stage == p.stages) {
@@ -248,57 +328,65 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
         }
     } else if (warp == 2) {
         // ------------------------------------------------------------ B stager
+        // stages B for every segment that ends in an epilogue (kb0 == 0)
         if (lane == 0 && p.lora) {
             ptx::tma_prefetch_desc(&tmB);
             const int n_valid = p.counts[0];
             const int n_active = p.counts[1];
-            int i = 0;
+            int j = 0, slots_tb = -1, nslots = 0;
+            uint32_t bytes = 0;
             bool pending = false;
             uint32_t pending_phase = 0;
-            for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x, ++i) {
-                const int nb = t / p.n_tb, tb = t - nb * p.n_tb;
-                if (!wait_bounded(bempty, (uint32_t)((i & 1) ^ 1), abort_flag, p.status, 0x8u)) break;
-                const int p0 = tb * p.BN;
-                const int p1 = min(min(p.M, p0 + p.BN), n_valid);
-                // first active segment that ends after p0
-                int s = 0;
-                {
-                    int lo = 0, hi = n_active;  // first s with indptr[active[s]+1] > p0
-                    while (lo < hi) {
-                        const int mid = (lo + hi) >> 1;
-                        if (p.indptr[p.active[mid] + 1] > p0) hi = mid; else lo = mid + 1;
+            for (long long u = u_begin; u < u_end;) {
+                const Seg sg = seg_at(u, u_end, KB);
+                u += sg.kb1 - sg.kb0;
+                if (sg.kb0 != 0) continue;  // partial accumulators only: no epilogue here
+                const int nb = sg.tile / p.n_tb, tb = sg.tile - nb * p.n_tb;
+                if (!wait_bounded(bempty, (uint32_t)((j & 1) ^ 1), abort_flag, p.status, 0x8u)) break;
+                if (tb != slots_tb) {
+                    // the adapters of this token block (kept while the block does not change)
+                    slots_tb = tb;
+                    const int p0 = tb * p.BN;
+                    const int p1 = min(min(p.M, p0 + p.BN), n_valid);
+                    int s = 0;  // first active segment that ends after p0
+                    {
+                        int lo = 0, hi = n_active;
+                        while (lo < hi) {
+                            const int mid = (lo + hi) >> 1;
+                            if (p.indptr[p.active[mid] + 1] > p0) hi = mid; else lo = mid + 1;
+                        }
+                        s = lo;
                     }
-                    s = lo;
+                    nslots = 0;
+                    bytes = 0;
+                    for (int s2 = s; s2 < n_active && nslots < p.n_slots; ++s2) {
+                        const int a = p.active[s2];
+                        if (p.indptr[a] >= p1) break;
+                        int r = p.ranks ? p.ranks[a] : p.r_max;
+                        r = max(1, min(r, p.r_max));
+                        bytes += (uint32_t)(((r + 7) >> 3) * 8 * 256);
+                        s_slot_rank[nslots] = r;
+                        s_slot_adapter[nslots++] = a;
+                    }
+                    s_nslots = nslots;
                 }
-                int nslots = 0;
-                uint32_t bytes = 0;
-                for (int s2 = s; s2 < n_active && nslots < p.n_slots; ++s2) {
-                    const int a = p.active[s2];
-                    if (p.indptr[a] >= p1) break;
-                    int r = p.ranks ? p.ranks[a] : p.r_max;
-                    r = max(1, min(r, p.r_max));
-                    bytes += (uint32_t)(((r + 7) >> 3) * 8 * 256);
-                    s_slot_adapter[nslots++] = a;
-                }
-                s_nslots = nslots;
                 if (bytes) ptx::mbar_arrive_expect_tx(bfull, bytes);
                 for (int q = 0; q < nslots; ++q) {
                     const int a = s_slot_adapter[q];
-                    int r = p.ranks ? p.ranks[a] : p.r_max;
-                    r = max(1, min(r, p.r_max));
+                    const int r = s_slot_rank[q];
                     const uint32_t dst = smem_u + p.slots_off + (uint32_t)(q * p.r8 * 256);
                     for (int rb = 0; rb < ((r + 7) >> 3); ++rb)
-                        ptx::tma_load_2d(dst + rb * 2048, &tmB, bfull, nb * kBlockM,
-                                         a * p.r_max + rb * 8);
+                        ptx::tma_load_2d(dst + rb * 2048, &tmB, bfull, nb * kBlockM, a * p.r_max + rb * 8);
                 }
                 if (!bytes) ptx::mbar_arrive(bfull);
                 pending = true;
-                pending_phase = (uint32_t)(i & 1);
+                pending_phase = (uint32_t)(j & 1);
+                ++j;
             }
             if (*abort_flag && pending) drain_wait(bfull, pending_phase);
         }
     } else {
-        // ------------------------------------------------------------ epilogue
+        // ------------------------------------------------------------ epilogue warps
         const int ew = warp - 3;
         const int quarter = warp & 3;         // TMEM lane quarter this warp may access
         const int grp = ew >> 2;              // which half of the token chunks
@@ -306,10 +394,11 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
         const int n_local = quarter * 32 + lane;
         int* s_m = reinterpret_cast<int*>(smem + p.meta_off);
         int* s_a = s_m + p.BN;
-        float* s_sx = reinterpret_cast<float*>(s_a + p.BN);
+        int* s_r = s_a + p.BN;  // rank of the token's adapter
+        int* s_q = s_r + p.BN;  // B slot of the token's adapter (-1: none, -2: not staged)
+        float* s_sx = reinterpret_cast<float*>(s_q + p.BN);
         float* s_v = reinterpret_cast<float*>(smem + p.v_off);
         const uint16_t* slots = reinterpret_cast<const uint16_t*>(smem + p.slots_off);
-        if (p.lora) ptx::pdl_wait();  // v comes from the kernel this one depends on
         // barrier among the epilogue warps, bounded like every other wait
         uint32_t epi_phase = 0;
         auto epi_sync = [&]() -> bool {
@@ -319,15 +408,107 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
             epi_phase ^= 1;
             return ok;
         };
+        ptx::pdl_wait();  // xq, sx and the zeroed v / flags / count come from the quantiser
+        bool ok = true;
 
-        int i = 0;
-        for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x, ++i) {
-            const int nb = t / p.n_tb, tb = t - nb * p.n_tb;
+        // ---- down-projection: work item q = 64 columns of K for every token
+        const int n_chunks = (p.K + kShrinkCols - 1) / kShrinkCols;
+        if (p.lora) {
+            const int ng = p.r_max >> 3;  // groups of 8 rank columns (a power of two)
+            const int lg = __ffs(ng) - 1;
+            // with few (token, group) pairs, split the 64 columns over up to 4 threads
+            int ls = 0;
+            while (ls < 2 && (p.M << (lg + ls + 1)) <= kEpiThreads) ++ls;
+            const int kspan = kShrinkCols >> ls;  // 64, 32 or 16 columns per thread
+            for (int q = cta; q < n_chunks && ok; q += G) {
+                for (int w = etid; w < (p.M << (lg + ls)); w += kEpiThreads) {
+                    const int pg = w >> ls, sub = w & ((1 << ls) - 1);
+                    const int pp = pg >> lg, g = pg & (ng - 1);
+                    const int k0 = q * kShrinkCols + sub * kspan;
+                    const int kw = min(kspan, p.K - k0);  // a multiple of 16 (or <= 0)
+                    if (kw <= 0) continue;
+                    const int m = p.perm[pp];
+                    const int a = p.tok_adapter[m];
+                    if (a < 0) continue;
+                    int r = p.ranks ? p.ranks[a] : p.r_max;
+                    r = max(1, min(r, p.r_max));
+                    if (8 * g >= r) continue;
+                    const uint4* xr = reinterpret_cast<const uint4*>(p.x + (size_t)m * p.K + k0);
+                    const uint16_t* ar = p.A + ((size_t)a * p.K + k0) * p.r_max + 8 * g;
+                    float acc[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+                    for (int kk = 0; kk < kw; kk += 16) {
+                        // 16 columns: all 18 loads in flight before the first FMA
+                        const uint4 xv0 = __ldg(xr + (kk >> 3)), xv1 = __ldg(xr + (kk >> 3) + 1);
+                        uint4 av[16];
+#pragma unroll
+                        for (int h = 0; h < 16; ++h)
+                            av[h] = __ldg(reinterpret_cast<const uint4*>(ar + (size_t)(kk + h) * p.r_max));
+                        const uint32_t xw[8] = {xv0.x, xv0.y, xv0.z, xv0.w, xv1.x, xv1.y, xv1.z, xv1.w};
+#pragma unroll
+                        for (int h = 0; h < 16; ++h) {
+                            const float xf = __uint_as_float((h & 1) ? (xw[h >> 1] & 0xffff0000u) : (xw[h >> 1] << 16));
+                            const uint32_t aw[4] = {av[h].x, av[h].y, av[h].z, av[h].w};
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                acc[2 * e] = fmaf(xf, __uint_as_float(aw[e] << 16), acc[2 * e]);
+                                acc[2 * e + 1] = fmaf(xf, __uint_as_float(aw[e] & 0xffff0000u), acc[2 * e + 1]);
+                            }
+                        }
+                    }
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        if (8 * g + e >= r) acc[e] = 0.f;  // the pool's padding past the rank
+                    float* vd = p.v + (size_t)pp * p.r_max + 8 * g;
+                    atomicAdd(reinterpret_cast<float4*>(vd), make_float4(acc[0], acc[1], acc[2], acc[3]));
+                    atomicAdd(reinterpret_cast<float4*>(vd + 4), make_float4(acc[4], acc[5], acc[6], acc[7]));
+                }
+                __threadfence();
+                ok = epi_sync();
+                if (ok && etid == 0) atomicAdd(p.v_done, 1);
+            }
+        }
+
+        // ---- epilogues of this CTA's segments
+        int i = 0, jb = 0, staged_tb = -1, slotted_tb = -1;
+        bool v_ready = !p.lora;
+        for (long long u = u_begin; u < u_end && ok; ++i) {
+            const Seg sg = seg_at(u, u_end, KB);
+            u += sg.kb1 - sg.kb0;
+            const int nb = sg.tile / p.n_tb, tb = sg.tile - nb * p.n_tb;
             const int buf = i & 1;
-            if (i == 0 || p.n_tb > 1) {
-                // stage this token block's metadata (and s_a * v) in shared memory
-                if (i > 0 && !epi_sync()) break;
-                for (int pl = etid; pl < p.BN; pl += kEpiWarps * 32) {
+            const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * p.BN);
+            if (sg.kb0 > 0) {
+                // later k-blocks of a tile another CTA finishes: fp32 partials to the workspace
+                if (!wait_bounded(&tfull[buf], (uint32_t)((i >> 1) & 1), abort_flag, p.status, 0x10u)) break;
+                ptx::tc_fence_after();
+                // layout [cta][16-column chunk][column][128 rows]: each store of a warp
+                // covers 128 contiguous bytes
+                for (int c0 = grp * 16; c0 < p.BN; c0 += 32) {
+                    float acc[16];
+                    ptx::tmem_ld16(taddr + (uint32_t)c0, acc);
+                    float* dst = p.partials + (((size_t)cta * (p.BN >> 4) + (c0 >> 4)) * 16) * kBlockM + n_local;
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) __stcg(dst + e * kBlockM, acc[e]);
+                }
+                ptx::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(&tempty[buf]);
+                __threadfence();
+                if (!(ok = epi_sync())) break;
+                if (etid == 0) atomicExch(p.flags + cta, 1);
+                continue;
+            }
+            if (staged_tb != tb) {
+                if (!v_ready) {  // every CTA's share of the down-projection is in v
+                    if (etid == 0) ok = wait_count(p.v_done, n_chunks, abort_flag, p.status, 0x80u);
+                    if (!(ok = epi_sync() && ok)) break;
+                    v_ready = true;
+                }
+                // this token block's metadata and s_a * v in shared memory
+                if (staged_tb >= 0 && !(ok = epi_sync())) break;
+                for (int pl = etid; pl < p.BN; pl += kEpiThreads) {
                     const int pp = tb * p.BN + pl;
                     int m = 0, a = -1;
                     float sxp = 0.f;
@@ -339,6 +520,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
                     s_m[pl] = m;
                     s_a[pl] = a;
                     s_sx[pl] = sxp;
+                    s_r[pl] = 0;
                     if (p.lora) {
                         int r = 0;
                         float sc = 0.f;
@@ -347,59 +529,89 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
                             r = max(0, min(r, p.r_max));
                             sc = p.scales ? p.scales[a] : 1.f;
                         }
+                        s_r[pl] = r;
                         for (int j = 0; j < p.r8; ++j)
-                            s_v[pl * p.r8 + j] = j < r ? sc * p.v[(size_t)m * p.r_max + j] : 0.f;
+                            s_v[pl * p.r8 + j] = j < r ? sc * __ldcg(p.v + (size_t)pp * p.r_max + j) : 0.f;
                     }
                 }
-                if (!epi_sync()) break;
+                if (!(ok = epi_sync())) break;
+                staged_tb = tb;
             }
-            if (!wait_bounded(&tfull[buf], (uint32_t)((i >> 1) & 1), abort_flag, p.status, 0x10u))
-                break;
+            if (!(ok = wait_bounded(&tfull[buf], (uint32_t)((i >> 1) & 1), abort_flag, p.status, 0x10u))) break;
             ptx::tc_fence_after();
-            if (p.lora && !wait_bounded(bfull, (uint32_t)(i & 1), abort_flag, p.status, 0x20u))
-                break;
+            if (p.lora && !(ok = wait_bounded(bfull, (uint32_t)(jb & 1), abort_flag, p.status, 0x20u))) break;
+            if (p.lora && slotted_tb != tb) {  // each token's B slot (the stager's list is fixed per block)
+                const int nsl = s_nslots;
+                for (int pl = etid; pl < p.BN; pl += kEpiThreads) {
+                    const int a = s_a[pl];
+                    int q = -1;
+                    if (a >= 0) {
+                        q = -2;
+                        for (int t = 0; t < nsl; ++t)
+                            if (s_slot_adapter[t] == a) { q = t; break; }
+                    }
+                    s_q[pl] = q;
+                }
+                if (!(ok = epi_sync())) break;
+                slotted_tb = tb;
+            }
+            // the CTAs after this one that hold later k-blocks of this tile
+            int c_hi = cta + 1;
+            if (sg.kb1 < KB) {
+                const long long tile_end = (long long)(sg.tile + 1) * KB;
+                while (c_hi < G && unit_begin(p.units, c_hi, G) < tile_end) ++c_hi;
+                if (etid == 0)
+                    for (int cc = cta + 1; cc < c_hi && ok; ++cc)
+                        ok = wait_count(p.flags + cc, 1, abort_flag, p.status, 0x100u);
+                if (!(ok = epi_sync() && ok)) break;
+            }
 
             const int n = nb * kBlockM + n_local;
             const float swn = n < p.N ? p.sw[n] : 0.f;
-            const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * p.BN);
-            const int nslots = p.lora ? s_nslots : 0;
-            int slot = 0, cur_a = -2, cur_r = 0;
+            int cur_a = -2;
             float breg[MAXR];
 #pragma unroll
             for (int j = 0; j < MAXR; ++j) breg[j] = 0.f;
 
+            // 16 tokens per chunk, fully unrolled so the accumulator stays in registers
             for (int c0 = grp * 16; c0 < p.BN; c0 += 32) {
-                if (tb * p.BN + c0 >= p.M) break;
+                const int valid_n = min(16, p.M - (tb * p.BN + c0));  // tokens of this chunk
+                if (valid_n <= 0) break;
                 float acc[16];
                 ptx::tmem_ld16(taddr + (uint32_t)c0, acc);
-#pragma unroll 1
-                for (int e = 0; e < 16; ++e) {
-                    const int pl = c0 + e;
-                    if (tb * p.BN + pl >= p.M) break;
-                    float out = acc[e] * s_sx[pl] * swn;
-                    if (p.lora) {
-                        const int a = s_a[pl];
-                        if (a >= 0) {
-                            if (a != cur_a) {
-                                cur_a = a;
-                                int r = p.ranks ? p.ranks[a] : p.r_max;
-                                cur_r = max(0, min(r, p.r_max));
-                                while (slot < nslots && s_slot_adapter[slot] != a) ++slot;
-                                if (slot < nslots) {
-                                    const uint16_t* sb = slots + (size_t)slot * p.r8 * 128 + n_local;
+                for (int cc = cta + 1; cc < c_hi; ++cc) {  // partial sums of the later k-blocks
+                    const float* src = p.partials + (((size_t)cc * (p.BN >> 4) + (c0 >> 4)) * 16) * kBlockM + n_local;
 #pragma unroll
-                                    for (int j = 0; j < MAXR; ++j)
-                                        breg[j] = j < cur_r ? __uint_as_float((uint32_t)sb[j * 128] << 16) : 0.f;
-                                } else {  // not staged: read B from global memory
-                                    const uint16_t* gb = p.B + ((size_t)a * p.r_max) * p.N + n;
+                    for (int e = 0; e < 16; ++e) acc[e] += __ldcg(src + e * kBlockM);
+                }
+                float lo[16];
 #pragma unroll
-                                    for (int j = 0; j < MAXR; ++j)
-                                        breg[j] = (j < cur_r && n < p.N)
-                                                      ? __uint_as_float((uint32_t)gb[(size_t)j * p.N] << 16)
-                                                      : 0.f;
-                                }
-                            }
-                            const float* vv = s_v + pl * p.r8;
+                for (int e = 0; e < 16; ++e) lo[e] = 0.f;
+                if (p.lora) {
+                    // LoRA term l[e] = sum_j s_a v[e][j] B[a_e][j][n]; branch-free over the 16
+                    // tokens so their FMA chains overlap (the chunk's tests are warp-uniform)
+                    const int a0 = s_a[c0];
+                    bool uni = true;
+#pragma unroll
+                    for (int e = 1; e < 16; ++e) {
+                        const int ae = s_a[c0 + e];
+                        uni = uni && (e >= valid_n || ae == a0 || ae < 0);
+                    }
+                    bool far = false;  // some token's B is not staged in shared memory
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) far = far || (e < valid_n && s_q[c0 + e] == -2);
+                    if (uni && a0 >= 0 && !far) {
+                        if (a0 != cur_a) {  // one adapter: its B column in registers
+                            cur_a = a0;
+                            const int r = s_r[c0];
+                            const uint16_t* sb = slots + (size_t)s_q[c0] * p.r8 * 128 + n_local;
+#pragma unroll
+                            for (int j = 0; j < MAXR; ++j)
+                                breg[j] = j < r ? __uint_as_float((uint32_t)sb[j * 128] << 16) : 0.f;
+                        }
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) {
+                            const float* vv = s_v + (c0 + e) * p.r8;
                             float l = 0.f;
 #pragma unroll
                             for (int j = 0; j < MAXR; j += 4) {
@@ -411,12 +623,57 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
                                     l = fmaf(v4.w, breg[j + 3], l);
                                 }
                             }
-                            out += l;
+                            lo[e] = l;  // s_v is zero for tokens without an adapter
                         }
+                    } else if (!far) {
+                        // several adapters: each token reads its own B column from its slot
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) {
+                            const int q = max(s_q[c0 + e], 0);
+                            const int re = s_r[c0 + e];  // 0 for tokens without an adapter
+                            const uint16_t* sb = slots + (size_t)q * p.r8 * 128 + n_local;
+                            const float* vv = s_v + (c0 + e) * p.r8;
+                            // slot rows past the rank hold the pool's padding: masked, not multiplied
+                            auto bv = [&](int j) {
+                                return j < re ? __uint_as_float((uint32_t)sb[j * 128] << 16) : 0.f;
+                            };
+                            float l = 0.f;
+#pragma unroll
+                            for (int j = 0; j < MAXR; j += 4) {
+                                if (j < p.r8) {
+                                    const float4 v4 = *reinterpret_cast<const float4*>(vv + j);
+                                    l = fmaf(v4.x, bv(j), l);
+                                    l = fmaf(v4.y, bv(j + 1), l);
+                                    l = fmaf(v4.z, bv(j + 2), l);
+                                    l = fmaf(v4.w, bv(j + 3), l);
+                                }
+                            }
+                            lo[e] = l;
+                        }
+                        cur_a = -2;
+                    } else {
+                        // some adapter's B was not staged: read B columns from global memory
+                        for (int e = 0; e < valid_n; ++e) {
+                            const int a = s_a[c0 + e];
+                            if (a < 0) continue;
+                            const int r = s_r[c0 + e];
+                            const uint16_t* gb = p.B + ((size_t)a * p.r_max) * p.N + n;
+                            const float* vv = s_v + (c0 + e) * p.r8;
+                            float l = 0.f;
+                            for (int j = 0; j < r; ++j)
+                                l = fmaf(vv[j], n < p.N ? __uint_as_float((uint32_t)gb[(size_t)j * p.N] << 16) : 0.f, l);
+                            lo[e] = l;
+                        }
+                        cur_a = -2;
                     }
-                    if (n < p.N) {
+                }
+                if (n < p.N) {
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        if (e >= valid_n) break;
+                        const float out = acc[e] * s_sx[c0 + e] * swn + lo[e];
                         const __nv_bfloat16 o = __float2bfloat16_rn(out);
-                        p.y[(size_t)s_m[pl] * p.N + n] = *reinterpret_cast<const uint16_t*>(&o);
+                        p.y[(size_t)s_m[c0 + e] * p.N + n] = *reinterpret_cast<const uint16_t*>(&o);
                     }
                 }
             }
@@ -426,6 +683,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
                 ptx::mbar_arrive(&tempty[buf]);
                 if (p.lora) ptx::mbar_arrive(bempty);
             }
+            ++jb;
         }
     }
 
@@ -449,7 +707,7 @@ bool encode_2d(CUtensorMap* m, CUtensorMapDataType dt, int elem_bytes, const voi
 
 template <int BK, int MAXR>
 cudaError_t launch_t(const GemmParams& p, const CUtensorMap& tmW, const CUtensorMap& tmX,
-                     const CUtensorMap& tmB, size_t smem, int grid, bool pdl, cudaStream_t stream)
+                     const CUtensorMap& tmB, size_t smem, int grid, cudaStream_t stream)
 {
     cudaError_t e = cudaFuncSetAttribute(fp8_gemm_kernel<BK, MAXR>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -459,11 +717,12 @@ cudaError_t launch_t(const GemmParams& p, const CUtensorMap& tmW, const CUtensor
     cfg.blockDim = dim3(kThreads, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
+    // a programmatic dependent of the quantiser: the first W loads overlap it
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = pdl ? 1 : 0;
+    cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, fp8_gemm_kernel<BK, MAXR>, tmW, tmX, tmB, p);
 }
 
@@ -476,11 +735,23 @@ int device_sm_count()
     int dev = 0;
     cudaGetDevice(&dev);
     static int cached[64] = {0};
-    if (dev < 64 && cached[dev]) return cached[dev];
+    if (dev >= 0 && dev < 64 && cached[dev]) return cached[dev];
     int n = 0;
     cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (dev < 64) cached[dev] = n;
+    if (n <= 0) n = 148;
+    if (dev >= 0 && dev < 64) cached[dev] = n;
     return n;
+}
+
+int fp8_gemm_tile_n(int M)
+{
+    const int n_tb = (M + 255) / 256;
+    return (((M + n_tb - 1) / n_tb) + 15) / 16 * 16;
+}
+
+size_t fp8_gemm_partial_bytes(int M)
+{
+    return (size_t)device_sm_count() * kBlockM * (size_t)fp8_gemm_tile_n(M) * 4;
 }
 
 cudaError_t launch_fp8_gemm(const Fp8GemmArgs& a, cudaStream_t stream)
@@ -490,14 +761,19 @@ cudaError_t launch_fp8_gemm(const Fp8GemmArgs& a, cudaStream_t stream)
     p.N = a.N;
     p.K = a.K;
     p.n_tb = (a.M + 255) / 256;
-    p.BN = (((a.M + p.n_tb - 1) / p.n_tb) + 15) / 16 * 16;
+    p.BN = fp8_gemm_tile_n(a.M);
     p.n_nb = (a.N + kBlockM - 1) / kBlockM;
     p.num_tiles = p.n_nb * p.n_tb;
     p.sx = a.sx;
     p.sw = a.sw;
     p.y = a.y;
     p.status = a.status;
+    p.partials = a.partials;
+    p.flags = a.flags;
+    p.v_done = a.v_done;
     p.lora = a.lora ? 1 : 0;
+    p.x = a.x;
+    p.A = a.A;
     p.perm = a.perm;
     p.tok_adapter = a.tok_adapter;
     p.indptr = a.indptr;
@@ -519,7 +795,7 @@ cudaError_t launch_fp8_gemm(const Fp8GemmArgs& a, cudaStream_t stream)
     cudaFuncAttributes fa;
     if (cudaFuncGetAttributes(&fa, fp8_gemm_kernel<128, 64>) != cudaSuccess) return cudaErrorInvalidValue;
     const size_t kSmemMax = (size_t)(optin > 0 ? optin : 232448) - fa.sharedSizeBytes - 256;
-    const size_t meta = align_up((size_t)p.BN * 12, 128);
+    const size_t meta = align_up((size_t)p.BN * 20, 128);  // token, adapter, rank, slot, sx
     const size_t vbytes = align_up((size_t)p.BN * p.r8 * 4, 128);
     const size_t bars = 8 * (2 * kMaxStages + 8);
     const size_t slot_bytes = (size_t)p.r8 * 256;
@@ -542,6 +818,7 @@ cudaError_t launch_fp8_gemm(const Fp8GemmArgs& a, cudaStream_t stream)
     p.stages = stages;
     p.n_slots = slots;
     p.k_blocks = (a.K + BK - 1) / BK;
+    p.units = (long long)p.num_tiles * p.k_blocks;
     const size_t stage_bytes = (size_t)kBlockM * BK + (size_t)p.BN * BK;
     p.ring_off = 0;
     p.slots_off = (uint32_t)align_up((size_t)stages * stage_bytes, 1024);
@@ -565,15 +842,15 @@ cudaError_t launch_fp8_gemm(const Fp8GemmArgs& a, cudaStream_t stream)
         tmB = tmW;  // unused
     }
 
-    int grid = device_sm_count();
-    if (grid <= 0) grid = 148;
-    if (grid > p.num_tiles) grid = p.num_tiles;
+    // one persistent CTA per SM (the partial buffers and flags are sized for that)
+    long long grid = device_sm_count();
+    if (grid > p.units) grid = p.units;
     const bool small_r = p.r8 <= 16;
     if (BK == 128)
-        return small_r ? launch_t<128, 16>(p, tmW, tmX, tmB, smem, grid, a.pdl, stream)
-                       : launch_t<128, 64>(p, tmW, tmX, tmB, smem, grid, a.pdl, stream);
-    return small_r ? launch_t<64, 16>(p, tmW, tmX, tmB, smem, grid, a.pdl, stream)
-                   : launch_t<64, 64>(p, tmW, tmX, tmB, smem, grid, a.pdl, stream);
+        return small_r ? launch_t<128, 16>(p, tmW, tmX, tmB, smem, (int)grid, stream)
+                       : launch_t<128, 64>(p, tmW, tmX, tmB, smem, (int)grid, stream);
+    return small_r ? launch_t<64, 16>(p, tmW, tmX, tmB, smem, (int)grid, stream)
+                   : launch_t<64, 64>(p, tmW, tmX, tmB, smem, (int)grid, stream);
 }
 
 }  // namespace lora

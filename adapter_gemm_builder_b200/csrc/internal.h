@@ -22,9 +22,10 @@ cudaError_t launch_sgmv(int mode, const void* x, int64_t x_slice_stride, const l
                         bool pdl_trigger);
 
 // Per-row E4M3 quantisation; row p of the output is row perm[p] of x
-// (perm == NULL: identity).
+// (perm == NULL: identity). The kernel also zeroes zero_words 32-bit words at
+// `zero` (may be NULL) and lets a programmatic dependent launch start early.
 cudaError_t launch_quantize_rows(const void* x, const int32_t* perm, int M, int K, uint8_t* xq,
-                                 float* sx, cudaStream_t stream);
+                                 float* sx, void* zero, size_t zero_words, cudaStream_t stream);
 
 struct Fp8GemmArgs {
     int M, N, K;
@@ -34,21 +35,29 @@ struct Fp8GemmArgs {
     const float* sw;     // [N]
     uint16_t* y;         // bf16 [M][N]
     uint32_t* status;    // device status word
+    float* partials;     // fp32 [SMs][128][fp8_gemm_tile_n(M)] stream-K partials
+    int* flags;          // [SMs], zero on entry
+    int* v_done;         // zero on entry
     // LoRA epilogue (lora == false: base only)
     bool lora;
+    const uint16_t* x;          // bf16 [M][K], by token index (the down-projection's input)
+    const uint16_t* A;          // bf16 [n_adapters][K][r_max]
     const int32_t* perm;        // [M]
     const int32_t* tok_adapter; // [M]
     const int32_t* indptr;      // [n_adapters+1]
     const int32_t* active;      // [n_adapters]
     const int32_t* counts;      // [4]
-    const float* v;             // fp32 [M][r_max], by token index
+    float* v;                   // fp32 [M][r_max], segment order, zero on entry
     const uint16_t* B;          // bf16 [n_adapters][r_max][N]
     const int32_t* ranks;
     const float* scales;
     int n_adapters, r_max;
-    bool pdl;                   // launch as a programmatic dependent of the previous kernel
 };
+// Launched as a programmatic dependent of the previous kernel (the quantiser).
 cudaError_t launch_fp8_gemm(const Fp8GemmArgs& a, cudaStream_t stream);
+// Token columns of a GEMM tile for M tokens, and the bytes of partial sums.
+int fp8_gemm_tile_n(int M);
+size_t fp8_gemm_partial_bytes(int M);
 
 int device_sm_count();
 

@@ -19,9 +19,16 @@ constexpr int kThreads = 256;
 
 __global__ void __launch_bounds__(kThreads)
 quantize_rows_kernel(const uint16_t* __restrict__ x, const int32_t* __restrict__ perm, int K,
-                     uint8_t* __restrict__ xq, float* __restrict__ sx)
+                     uint8_t* __restrict__ xq, float* __restrict__ sx, uint32_t* __restrict__ zero,
+                     size_t zero_words)
 {
     __shared__ float s_red[kThreads / 32];
+    ptx::pdl_launch_dependents();  // the GEMM may start streaming its weights now
+    if (zero) {  // scratch the dependent GEMM accumulates into (block b: its slice)
+        const size_t per = (zero_words + gridDim.x - 1) / gridDim.x;
+        const size_t z0 = per * blockIdx.x, z1 = min(zero_words, z0 + per);
+        for (size_t i = z0 + threadIdx.x; i < z1; i += kThreads) zero[i] = 0u;
+    }
     const int prow = blockIdx.x;
     const int row = perm ? perm[prow] : prow;
     const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)row * K);
@@ -67,11 +74,11 @@ quantize_rows_kernel(const uint16_t* __restrict__ x, const int32_t* __restrict__
 }  // namespace
 
 cudaError_t launch_quantize_rows(const void* x, const int32_t* perm, int M, int K, uint8_t* xq,
-                                 float* sx, cudaStream_t stream)
+                                 float* sx, void* zero, size_t zero_words, cudaStream_t stream)
 {
     if (M == 0) return cudaSuccess;
     quantize_rows_kernel<<<M, kThreads, 0, stream>>>(static_cast<const uint16_t*>(x), perm, K, xq,
-                                                      sx);
+                                                      sx, static_cast<uint32_t*>(zero), zero_words);
     return cudaGetLastError();
 }
 

@@ -715,7 +715,6 @@ sgmv_kernel(const __grid_constant__ AMaps am, const SgmvParams p)
                             ptx::mma_bf16_16816(c[0], ah[ks], b[ks][0], b[ks][1]);
                             ptx::mma_bf16_16816(c[1], al[ks], b[ks][0], b[ks][1]);
                         }
-                    const int col = ntl * 8 + tq * 2;
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
                         const int rr = mt * 16 + gq + h * 8;
