@@ -76,7 +76,7 @@ struct GemmParams {
     const uint16_t* B;
     const int32_t* ranks;
     const float* scales;
-    int n_adapters, r_max, r8;
+    int n_adapters, r_max, r8, r16;
     int n_slots;
     uint32_t ring_off, slots_off, v_off, meta_off, bar_off;
 };
@@ -146,6 +146,28 @@ __device__ __forceinline__ uint32_t make_idesc(int n)
     return (1u << 4) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(kBlockM >> 4) << 24);
 }
 
+// Instruction descriptor: kind::f16 with A = B = bf16, both K-major, D fp32,
+// M = 128, N = n.
+__device__ __forceinline__ uint32_t make_idesc_bf16(int n)
+{
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(kBlockM >> 4) << 24);
+}
+
+// UMMA descriptor for a K-major bf16 tile without swizzle: 8-row x 16-byte
+// core matrices of 128 contiguous bytes, 128 bytes apart along K (leading
+// byte offset) and kg * 128 bytes apart along M / N (stride byte offset).
+__device__ __forceinline__ uint64_t make_desc_kmajor(uint32_t saddr, int kg)
+{
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)(128 >> 4) << 16) |
+           ((uint64_t)((kg * 128) >> 4) << 32) | ((uint64_t)1 << 46);
+}
+
+// Byte offset of (row, 8-column group kg) in such a tile with kg_n groups per row.
+__device__ __forceinline__ uint32_t kmajor_off(int row, int kg, int kg_n)
+{
+    return (uint32_t)((((row >> 3) * kg_n + kg) << 7) + ((row & 7) << 4));
+}
+
 // Stream-K schedule: CTA c owns units [c*U/G, (c+1)*U/G) of the (tile,
 // k-block) sequence; a segment is the part of one tile inside that range.
 struct Seg {
@@ -175,6 +197,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
     __shared__ int s_nslots;
     __shared__ int s_slot_adapter[256];
     __shared__ int s_slot_rank[256];
+    __shared__ int4 s_lq[256];  // per slot: first / end token (block-relative), V' byte offset
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     // the swizzled TMA tiles need a 1024-byte aligned base
@@ -190,6 +213,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
     uint64_t* bempty = bfull + 1;               // [1]
     uint64_t* drain = bempty + 1;               // [1]
     uint64_t* epibar = drain + 1;               // [1] epilogue-warps barrier
+    uint64_t* lready = epibar + 1;              // [1] LoRA operands of the segment built
     volatile int* abort_flag = &s_abort;
 
     constexpr int kStageW = kBlockM * BK;
@@ -213,6 +237,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
         ptx::mbar_init(bempty, kEpiWarps);
         ptx::mbar_init(drain, 1);
         ptx::mbar_init(epibar, kEpiWarps);
+        ptx::mbar_init(lready, 1);
         ptx::fence_mbar_init();
     }
     if (warp == 1) {
@@ -288,7 +313,9 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
             uint32_t phase = 0;
             const uint32_t idesc = make_idesc(p.BN);
             bool ok = true, any = false;
-            int i = 0;
+            int i = 0, lj = 0;
+            const uint32_t slots_u = smem_u + p.slots_off, vq_u = smem_u + p.v_off;
+            const int kgq = p.r16 >> 3;
             for (long long u = u_begin; u < u_end && ok; ++i) {
                 const Seg sg = seg_at(u, u_end, KB);
                 u += sg.kb1 - sg.kb0;
@@ -317,6 +344,26 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
                     if (++stage == p.stages) {
                         stage = 0;
                         phase ^= 1;
+                    }
+                }
+                if (ok && p.lora && sg.kb0 == 0) {
+                    // the up-projection into the same accumulator: per staged adapter q,
+                    // D[n][t] += (B_q[j][n] / sw[n]) * (s_q v[t][j] / sx[t]) over its tokens
+                    if (!wait_bounded(lready, (uint32_t)(lj & 1), abort_flag, p.status, 0x200u)) {
+                        ok = false;
+                        break;
+                    }
+                    ++lj;
+                    ptx::tc_fence_after();
+                    const int nsl = s_nslots;
+                    for (int q = 0; q < nsl; ++q) {
+                        const int4 lq = s_lq[q];
+                        const int c0 = lq.x & ~15, w = ((lq.y + 15) & ~15) - c0;
+                        const uint32_t idl = make_idesc_bf16(w);
+                        for (int ks = 0; ks < (p.r16 >> 4); ++ks)
+                            ptx::tc_mma_f16(d + (uint32_t)c0,
+                                            make_desc_kmajor(slots_u + (uint32_t)(q * p.r16 * 256 + ks * 256), kgq),
+                                            make_desc_kmajor(vq_u + (uint32_t)(lq.z + ks * 256), kgq), idl, 1u);
                     }
                 }
                 if (ok) ptx::tc_commit(&tfull[buf]);
@@ -366,6 +413,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
                         r = max(1, min(r, p.r_max));
                         bytes += (uint32_t)(((r + 7) >> 3) * 8 * 256);
                         s_slot_rank[nslots] = r;
+                        s_lq[nslots] = make_int4(max(p.indptr[a], p0) - p0, min(p.indptr[a + 1], p1) - p0, 0, 0);
                         s_slot_adapter[nslots++] = a;
                     }
                     s_nslots = nslots;
@@ -374,7 +422,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
                 for (int q = 0; q < nslots; ++q) {
                     const int a = s_slot_adapter[q];
                     const int r = s_slot_rank[q];
-                    const uint32_t dst = smem_u + p.slots_off + (uint32_t)(q * p.r8 * 256);
+                    const uint32_t dst = smem_u + p.slots_off + (uint32_t)(q * p.r16 * 256);
                     for (int rb = 0; rb < ((r + 7) >> 3); ++rb)
                         ptx::tma_load_2d(dst + rb * 2048, &tmB, bfull, nb * kBlockM, a * p.r_max + rb * 8);
                 }
@@ -397,8 +445,9 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
         int* s_r = s_a + p.BN;  // rank of the token's adapter
         int* s_q = s_r + p.BN;  // B slot of the token's adapter (-1: none, -2: not staged)
         float* s_sx = reinterpret_cast<float*>(s_q + p.BN);
-        float* s_v = reinterpret_cast<float*>(smem + p.v_off);
-        const uint16_t* slots = reinterpret_cast<const uint16_t*>(smem + p.slots_off);
+        uint8_t* vq = smem + p.v_off;     // V' tiles of the staged adapters (K-major bf16)
+        uint8_t* slots = smem + p.slots_off;  // B of the staged adapters, then B' in place
+        const int kgq = p.r16 >> 3;
         // barrier among the epilogue warps, bounded like every other wait
         uint32_t epi_phase = 0;
         auto epi_sync = [&]() -> bool {
@@ -530,31 +579,94 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
                             sc = p.scales ? p.scales[a] : 1.f;
                         }
                         s_r[pl] = r;
-                        for (int j = 0; j < p.r8; ++j)
-                            s_v[pl * p.r8 + j] = j < r ? sc * __ldcg(p.v + (size_t)pp * p.r_max + j) : 0.f;
+                        (void)sc;
                     }
                 }
                 if (!(ok = epi_sync())) break;
                 staged_tb = tb;
             }
+            // the LoRA operands of this segment first: the MMA warp adds them to the
+            // accumulator before it signals tfull
+            if (p.lora && !(ok = wait_bounded(bfull, (uint32_t)(jb & 1), abort_flag, p.status, 0x20u))) break;
+            if (p.lora) {
+                const int nsl = s_nslots;
+                if (slotted_tb != tb) {
+                    // per token: its slot (-2: adapter not staged, done on CUDA cores below);
+                    // per slot q: V'_q[t][j] = s_q v[t][j] / sx[t] for its tokens t (zero for the
+                    // other tokens of its 16-aligned column range), K-major bf16
+                    for (int pl = etid; pl < p.BN; pl += kEpiThreads) {
+                        const int a = s_a[pl];
+                        int q = -1;
+                        if (a >= 0) {
+                            q = -2;
+                            for (int t = 0; t < nsl; ++t)
+                                if (s_slot_adapter[t] == a) { q = t; break; }
+                        }
+                        s_q[pl] = q;
+                    }
+                    int off = 0;
+                    for (int q = 0; q < nsl; ++q) {
+                        const int4 lq = s_lq[q];
+                        const int c0 = lq.x & ~15, w = ((lq.y + 15) & ~15) - c0;
+                        const int a = s_slot_adapter[q], r = s_slot_rank[q];
+                        const float sc = p.scales ? p.scales[a] : 1.f;
+                        if (etid == 0) s_lq[q].z = off;
+                        for (int idx = etid; idx < w * kgq; idx += kEpiThreads) {
+                            const int rr = idx / kgq, kg = idx - rr * kgq;
+                            const int t = c0 + rr, pp = tb * p.BN + t;
+                            const bool mine = t >= lq.x && t < lq.y;
+                            const float f = mine ? sc / s_sx[t] : 0.f;
+                            uint32_t wv[4];
+#pragma unroll
+                            for (int h = 0; h < 4; ++h) {
+                                const int j = kg * 8 + 2 * h;
+                                const float v0 = (mine && j < r) ? f * __ldcg(p.v + (size_t)pp * p.r_max + j) : 0.f;
+                                const float v1 = (mine && j + 1 < r) ? f * __ldcg(p.v + (size_t)pp * p.r_max + j + 1) : 0.f;
+                                __nv_bfloat162 hv = __floats2bfloat162_rn(v0, v1);
+                                wv[h] = *reinterpret_cast<uint32_t*>(&hv);
+                            }
+                            *reinterpret_cast<uint4*>(vq + off + kmajor_off(rr, kg, kgq)) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+                        }
+                        off += w * kgq * 16;
+                    }
+                    slotted_tb = tb;
+                }
+                // B'_q[n][j] = B_q[j][n] / sw[n] in place, K-major: every thread first reads
+                // its (n, slot) columns, then (after a barrier) writes them transposed
+                const float inv_sw2 = (nb * kBlockM + (etid & 127) < p.N) ? 1.f / p.sw[nb * kBlockM + (etid & 127)] : 0.f;
+                for (int q0 = 0; q0 < nsl && ok; q0 += 2) {
+                    const int q = q0 + (etid >> 7), nn = etid & 127;
+                    float col[MAXR];
+                    const bool act = q < nsl;
+                    const int r = act ? s_slot_rank[q] : 0;
+                    const uint16_t* raw = reinterpret_cast<const uint16_t*>(slots + (size_t)(act ? q : 0) * p.r16 * 256) + nn;
+#pragma unroll
+                    for (int j = 0; j < MAXR; ++j)
+                        col[j] = (j < r) ? __uint_as_float((uint32_t)raw[j * 128] << 16) * inv_sw2 : 0.f;
+                    if (!(ok = epi_sync())) break;
+                    if (act) {
+                        uint8_t* dst = slots + (size_t)q * p.r16 * 256;
+#pragma unroll
+                        for (int kg = 0; kg < MAXR / 8; ++kg) {
+                            if (kg >= kgq) break;
+                            uint32_t wv[4];
+#pragma unroll
+                            for (int h = 0; h < 4; ++h) {
+                                __nv_bfloat162 hv = __floats2bfloat162_rn(col[kg * 8 + 2 * h], col[kg * 8 + 2 * h + 1]);
+                                wv[h] = *reinterpret_cast<uint32_t*>(&hv);
+                            }
+                            *reinterpret_cast<uint4*>(dst + kmajor_off(nn, kg, kgq)) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+                        }
+                    }
+                    // the next pair reads other slots: no barrier before it
+                }
+                if (!ok) break;
+                ptx::fence_proxy_async_smem();  // generic writes, read by the tensor core (async proxy)
+                if (!(ok = epi_sync())) break;
+                if (etid == 0) ptx::mbar_arrive(lready);
+            }
             if (!(ok = wait_bounded(&tfull[buf], (uint32_t)((i >> 1) & 1), abort_flag, p.status, 0x10u))) break;
             ptx::tc_fence_after();
-            if (p.lora && !(ok = wait_bounded(bfull, (uint32_t)(jb & 1), abort_flag, p.status, 0x20u))) break;
-            if (p.lora && slotted_tb != tb) {  // each token's B slot (the stager's list is fixed per block)
-                const int nsl = s_nslots;
-                for (int pl = etid; pl < p.BN; pl += kEpiThreads) {
-                    const int a = s_a[pl];
-                    int q = -1;
-                    if (a >= 0) {
-                        q = -2;
-                        for (int t = 0; t < nsl; ++t)
-                            if (s_slot_adapter[t] == a) { q = t; break; }
-                    }
-                    s_q[pl] = q;
-                }
-                if (!(ok = epi_sync())) break;
-                slotted_tb = tb;
-            }
             // the CTAs after this one that hold later k-blocks of this tile
             int c_hi = cta + 1;
             if (sg.kb1 < KB) {
@@ -568,10 +680,6 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
 
             const int n = nb * kBlockM + n_local;
             const float swn = n < p.N ? p.sw[n] : 0.f;
-            int cur_a = -2;
-            float breg[MAXR];
-#pragma unroll
-            for (int j = 0; j < MAXR; ++j) breg[j] = 0.f;
 
             // 16 tokens per chunk, fully unrolled so the accumulator stays in registers
             for (int c0 = grp * 16; c0 < p.BN; c0 += 32) {
@@ -588,83 +696,25 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
 #pragma unroll
                 for (int e = 0; e < 16; ++e) lo[e] = 0.f;
                 if (p.lora) {
-                    // LoRA term l[e] = sum_j s_a v[e][j] B[a_e][j][n]; branch-free over the 16
-                    // tokens so their FMA chains overlap (the chunk's tests are warp-uniform)
-                    const int a0 = s_a[c0];
-                    bool uni = true;
-#pragma unroll
-                    for (int e = 1; e < 16; ++e) {
-                        const int ae = s_a[c0 + e];
-                        uni = uni && (e >= valid_n || ae == a0 || ae < 0);
-                    }
-                    bool far = false;  // some token's B is not staged in shared memory
+                    // adapters that found no shared-memory slot: their term on CUDA cores, B
+                    // and v from global memory (the staged ones are in the accumulator)
+                    bool far = false;
 #pragma unroll
                     for (int e = 0; e < 16; ++e) far = far || (e < valid_n && s_q[c0 + e] == -2);
-                    if (uni && a0 >= 0 && !far) {
-                        if (a0 != cur_a) {  // one adapter: its B column in registers
-                            cur_a = a0;
-                            const int r = s_r[c0];
-                            const uint16_t* sb = slots + (size_t)s_q[c0] * p.r8 * 128 + n_local;
-#pragma unroll
-                            for (int j = 0; j < MAXR; ++j)
-                                breg[j] = j < r ? __uint_as_float((uint32_t)sb[j * 128] << 16) : 0.f;
-                        }
-#pragma unroll
-                        for (int e = 0; e < 16; ++e) {
-                            const float* vv = s_v + (c0 + e) * p.r8;
-                            float l = 0.f;
-#pragma unroll
-                            for (int j = 0; j < MAXR; j += 4) {
-                                if (j < p.r8) {
-                                    const float4 v4 = *reinterpret_cast<const float4*>(vv + j);
-                                    l = fmaf(v4.x, breg[j], l);
-                                    l = fmaf(v4.y, breg[j + 1], l);
-                                    l = fmaf(v4.z, breg[j + 2], l);
-                                    l = fmaf(v4.w, breg[j + 3], l);
-                                }
-                            }
-                            lo[e] = l;  // s_v is zero for tokens without an adapter
-                        }
-                    } else if (!far) {
-                        // several adapters: each token reads its own B column from its slot
-#pragma unroll
-                        for (int e = 0; e < 16; ++e) {
-                            const int q = max(s_q[c0 + e], 0);
-                            const int re = s_r[c0 + e];  // 0 for tokens without an adapter
-                            const uint16_t* sb = slots + (size_t)q * p.r8 * 128 + n_local;
-                            const float* vv = s_v + (c0 + e) * p.r8;
-                            // slot rows past the rank hold the pool's padding: masked, not multiplied
-                            auto bv = [&](int j) {
-                                return j < re ? __uint_as_float((uint32_t)sb[j * 128] << 16) : 0.f;
-                            };
-                            float l = 0.f;
-#pragma unroll
-                            for (int j = 0; j < MAXR; j += 4) {
-                                if (j < p.r8) {
-                                    const float4 v4 = *reinterpret_cast<const float4*>(vv + j);
-                                    l = fmaf(v4.x, bv(j), l);
-                                    l = fmaf(v4.y, bv(j + 1), l);
-                                    l = fmaf(v4.z, bv(j + 2), l);
-                                    l = fmaf(v4.w, bv(j + 3), l);
-                                }
-                            }
-                            lo[e] = l;
-                        }
-                        cur_a = -2;
-                    } else {
-                        // some adapter's B was not staged: read B columns from global memory
+                    if (far) {
                         for (int e = 0; e < valid_n; ++e) {
-                            const int a = s_a[c0 + e];
-                            if (a < 0) continue;
-                            const int r = s_r[c0 + e];
+                            if (s_q[c0 + e] != -2) continue;
+                            const int a = s_a[c0 + e], r = s_r[c0 + e];
+                            const float sc = p.scales ? p.scales[a] : 1.f;
                             const uint16_t* gb = p.B + ((size_t)a * p.r_max) * p.N + n;
-                            const float* vv = s_v + (c0 + e) * p.r8;
+                            const float* vg = p.v + (size_t)(tb * p.BN + c0 + e) * p.r_max;
                             float l = 0.f;
                             for (int j = 0; j < r; ++j)
-                                l = fmaf(vv[j], n < p.N ? __uint_as_float((uint32_t)gb[(size_t)j * p.N] << 16) : 0.f, l);
-                            lo[e] = l;
+                                l = fmaf(__ldcg(vg + j), n < p.N ? __uint_as_float((uint32_t)gb[(size_t)j * p.N] << 16) : 0.f, l);
+#pragma unroll
+                            for (int e2 = 0; e2 < 16; ++e2)
+                                if (e2 == e) lo[e2] = sc * l;
                         }
-                        cur_a = -2;
                     }
                 }
                 if (n < p.N) {
@@ -786,6 +836,7 @@ cudaError_t launch_fp8_gemm(const Fp8GemmArgs& a, cudaStream_t stream)
     p.n_adapters = a.n_adapters;
     p.r_max = a.lora ? a.r_max : 0;
     p.r8 = a.lora ? (a.r_max + 7) / 8 * 8 : 0;
+    p.r16 = a.lora ? (a.r_max + 15) / 16 * 16 : 0;
 
     // shared-memory plan: ring | B slots | v | meta | barriers, within the
     // opt-in per-block limit minus the kernel's static shared memory
@@ -796,14 +847,18 @@ cudaError_t launch_fp8_gemm(const Fp8GemmArgs& a, cudaStream_t stream)
     if (cudaFuncGetAttributes(&fa, fp8_gemm_kernel<128, 64>) != cudaSuccess) return cudaErrorInvalidValue;
     const size_t kSmemMax = (size_t)(optin > 0 ? optin : 232448) - fa.sharedSizeBytes - 256;
     const size_t meta = align_up((size_t)p.BN * 20, 128);  // token, adapter, rank, slot, sx
-    const size_t vbytes = align_up((size_t)p.BN * p.r8 * 4, 128);
-    const size_t bars = 8 * (2 * kMaxStages + 8);
-    const size_t slot_bytes = (size_t)p.r8 * 256;
+    const size_t bars = 8 * (2 * kMaxStages + 9);
+    // a slot holds one adapter's B[j][128 n] as loaded, then B'[128 n][r16] in place
+    const size_t slot_bytes = (size_t)p.r16 * 256;
+    // V' tiles: each staged adapter's 16-aligned token range, r16 bf16 per token
+    auto vq_bytes = [&](int nslots) -> size_t {
+        return a.lora ? align_up(((size_t)p.BN + 32 * (size_t)nslots) * p.r16 * 2, 128) : 0;
+    };
     int want_slots = a.lora ? (a.n_adapters < p.BN ? a.n_adapters : p.BN) : 0;
     if (want_slots > 256) want_slots = 256;
     auto fit = [&](int bk, int nslots) -> int {
         const size_t stage_bytes = (size_t)kBlockM * bk + (size_t)p.BN * bk;
-        const size_t fixed = 1024 + meta + vbytes + bars + (size_t)nslots * slot_bytes;
+        const size_t fixed = 1024 + meta + vq_bytes(nslots) + bars + (size_t)nslots * slot_bytes;
         if (fixed >= kSmemMax) return 0;
         const size_t st = (kSmemMax - fixed) / stage_bytes;
         return (int)(st > (size_t)kMaxStages ? kMaxStages : st);
@@ -823,7 +878,7 @@ cudaError_t launch_fp8_gemm(const Fp8GemmArgs& a, cudaStream_t stream)
     p.ring_off = 0;
     p.slots_off = (uint32_t)align_up((size_t)stages * stage_bytes, 1024);
     p.v_off = (uint32_t)align_up(p.slots_off + (size_t)slots * slot_bytes, 128);
-    p.meta_off = (uint32_t)(p.v_off + vbytes);
+    p.meta_off = (uint32_t)(p.v_off + vq_bytes(slots));
     p.bar_off = (uint32_t)align_up(p.meta_off + meta, 8);
     const size_t smem = align_up(p.bar_off + bars, 128) + 1024;  // + alignment slack
 

@@ -312,6 +312,18 @@ __device__ __forceinline__ void tc_mma_f8(uint32_t d_tmem, uint64_t a_desc, uint
         : "memory");
 }
 // Arrive on `bar` once all previously issued tcgen05.mma of this thread complete.
+// D (TMEM, fp32) (+)= A * B for 16-bit operands (kind::f16; bf16 per the
+// instruction descriptor), K = 16 per instruction.
+__device__ __forceinline__ void tc_mma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                           uint32_t idesc, uint32_t accumulate)
+{
+    asm volatile(
+        "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\n"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n}\n" ::"r"(
+            d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(0u), "r"(0u), "r"(0u), "r"(0u)
+        : "memory");
+}
 __device__ __forceinline__ void tc_commit(uint64_t* bar)
 {
     asm volatile(
