@@ -214,6 +214,12 @@ sgmv_kernel(const __grid_constant__ AMaps am, const SgmvParams p)
         ptx::mbar_init(red2, 1);
         ptx::fence_mbar_init();
     }
+    // Cluster barrier, phase 0: this CTA's mbarriers exist (peers wait for it before
+    // their first remote store); phase 1: this CTA makes no more remote accesses (every
+    // CTA waits for it before leaving). Phase 0 is announced before the wait on the
+    // previous kernel, so it overlaps that kernel's tail.
+    __syncthreads();
+    if (kClustered) ptx::cluster_arrive();
     // the previous kernel in the stream (e.g. the segment builder) may still run
     ptx::pdl_wait();
     ptx::pdl_launch_dependents();
@@ -290,7 +296,6 @@ sgmv_kernel(const __grid_constant__ AMaps am, const SgmvParams p)
         ptx::mbar_arrive_expect_tx(red2, one_phase ? 0u : (uint32_t)(nt * r8 * 4));
     }
     __syncthreads();
-    if (kClustered) ptx::cluster_arrive();  // barriers initialised; matched before any remote access
 
     if (warp == kComputeWarps) {
         // ================================================================ producer warp
@@ -394,7 +399,10 @@ sgmv_kernel(const __grid_constant__ AMaps am, const SgmvParams p)
                 }
         }
         __syncwarp();
-        if (kClustered) ptx::cluster_wait();
+        if (kClustered) {  // no remote accesses from this warp
+            ptx::cluster_wait();
+            ptx::cluster_arrive();
+        }
     } else {
         // ================================================================ compute warps
         float* VF = reinterpret_cast<float*>(smem + p.off_vf);       // [kTT][rp]: partial, then v
@@ -517,6 +525,7 @@ sgmv_kernel(const __grid_constant__ AMaps am, const SgmvParams p)
                                         *reinterpret_cast<const float4*>(&VF[row * p.rp + j]), ptx::mapa(red1_u, row % C));
                 }
             }
+            if (one_phase) ptx::cluster_arrive();  // phase 1: this thread's remote stores are issued
             wait_all<true>(red1, 0, abort_flag, status, 0x200);
             ptx::named_sync(1, kCompute);  // every thread of this CTA has sent its share
             if (one_phase) {
@@ -539,6 +548,7 @@ sgmv_kernel(const __grid_constant__ AMaps am, const SgmvParams p)
                     for (int d = 0; d < C; ++d)
                         ptx::st_async_f32x4(ptx::mapa(vf_u + off, d), s4, ptx::mapa(red2_u, d));
                 }
+                ptx::cluster_arrive();  // phase 1: this thread's remote stores are issued
                 wait_all<true>(red2, 0, abort_flag, status, 0x400);
             }
             ptx::named_sync(1, kCompute);
@@ -751,7 +761,7 @@ sgmv_kernel(const __grid_constant__ AMaps am, const SgmvParams p)
         }
     }
     // no CTA leaves while a peer may still address its shared memory
-    if (kClustered) ptx::cluster_sync();
+    if (kClustered) ptx::cluster_wait();
 }
 #undef SACC
 #undef ACC
