@@ -316,11 +316,46 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
             int i = 0, lj = 0;
             const uint32_t slots_u = smem_u + p.slots_off, vq_u = smem_u + p.v_off;
             const int kgq = p.r16 >> 3;
+            // the up-projection of a finished segment waits for its operands (lready) without
+            // holding up the next segment's k-blocks: it is issued as soon as they are built
+            int pend_buf = -1;
+            auto issue_lora = [&](int pbuf) {
+                ++lj;
+                ptx::tc_fence_after();
+                const uint32_t dp = tmem_base + (uint32_t)(pbuf * p.BN);
+                const int nsl = s_nslots;
+                for (int q = 0; q < nsl; ++q) {
+                    // D[n][t] += (B_q[j][n] / sw[n]) * (s_q v[t][j] / sx[t]) over adapter q's tokens
+                    const int4 lq = s_lq[q];
+                    const int c0 = lq.x & ~15, w = ((lq.y + 15) & ~15) - c0;
+                    const uint32_t idl = make_idesc_bf16(w);
+                    for (int ks = 0; ks < (p.r16 >> 4); ++ks)
+                        ptx::tc_mma_f16(dp + (uint32_t)c0,
+                                        make_desc_kmajor(slots_u + (uint32_t)(q * p.r16 * 256 + ks * 256), kgq),
+                                        make_desc_kmajor(vq_u + (uint32_t)(lq.z + ks * 256), kgq), idl, 1u);
+                }
+                ptx::tc_commit(&tfull[pbuf]);
+            };
+            auto resolve_pending = [&](bool block) -> bool {
+                if (pend_buf < 0) return true;
+                if (block) {
+                    if (!wait_bounded(lready, (uint32_t)(lj & 1), abort_flag, p.status, 0x200u)) return false;
+                } else if (!ptx::mbar_try_wait(lready, (uint32_t)(lj & 1))) {
+                    return true;
+                }
+                issue_lora(pend_buf);
+                pend_buf = -1;
+                return true;
+            };
             for (long long u = u_begin; u < u_end && ok; ++i) {
                 const Seg sg = seg_at(u, u_end, KB);
                 u += sg.kb1 - sg.kb0;
                 const int buf = i & 1;
                 const uint32_t bphase = (uint32_t)((i >> 1) & 1);
+                if (pend_buf == buf && !resolve_pending(true)) {  // that buffer's epilogue comes first
+                    ok = false;
+                    break;
+                }
                 if (!wait_bounded(&tempty[buf], bphase ^ 1, abort_flag, p.status, 0x2u)) {
                     ok = false;
                     break;
@@ -328,7 +363,8 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
                 ptx::tc_fence_after();
                 const uint32_t d = tmem_base + (uint32_t)(buf * p.BN);
                 for (int kb = sg.kb0; kb < sg.kb1; ++kb) {
-                    if (!wait_bounded(&full[stage], phase, abort_flag, p.status, 0x4u)) {
+                    if (!resolve_pending(false) ||
+                        !wait_bounded(&full[stage], phase, abort_flag, p.status, 0x4u)) {
                         ok = false;
                         break;
                     }
@@ -346,28 +382,23 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
                         phase ^= 1;
                     }
                 }
-                if (ok && p.lora && sg.kb0 == 0) {
-                    // the up-projection into the same accumulator: per staged adapter q,
-                    // D[n][t] += (B_q[j][n] / sw[n]) * (s_q v[t][j] / sx[t]) over its tokens
-                    if (!wait_bounded(lready, (uint32_t)(lj & 1), abort_flag, p.status, 0x200u)) {
+                if (!ok) break;
+                if (p.lora && sg.kb0 == 0) {
+                    // an earlier segment's up-projection goes first (lready phases are in order)
+                    if (!resolve_pending(true)) {
                         ok = false;
                         break;
                     }
-                    ++lj;
-                    ptx::tc_fence_after();
-                    const int nsl = s_nslots;
-                    for (int q = 0; q < nsl; ++q) {
-                        const int4 lq = s_lq[q];
-                        const int c0 = lq.x & ~15, w = ((lq.y + 15) & ~15) - c0;
-                        const uint32_t idl = make_idesc_bf16(w);
-                        for (int ks = 0; ks < (p.r16 >> 4); ++ks)
-                            ptx::tc_mma_f16(d + (uint32_t)c0,
-                                            make_desc_kmajor(slots_u + (uint32_t)(q * p.r16 * 256 + ks * 256), kgq),
-                                            make_desc_kmajor(vq_u + (uint32_t)(lq.z + ks * 256), kgq), idl, 1u);
+                    pend_buf = buf;
+                    if (!resolve_pending(false)) {
+                        ok = false;
+                        break;
                     }
+                } else {
+                    ptx::tc_commit(&tfull[buf]);
                 }
-                if (ok) ptx::tc_commit(&tfull[buf]);
             }
+            if (ok && !resolve_pending(true)) ok = false;
             if (!ok && any) {  // wait for the MMAs in flight before TMEM is freed
                 ptx::tc_commit(drain);
                 drain_wait(drain, 0);

@@ -646,6 +646,25 @@ sgmv_kernel(const __grid_constant__ AMaps am, const SgmvParams p)
         }
         if (MODE != SGMV_EXPAND) reduce_v();
 
+        // tensor-core expand: warp w owns m-tile mt_w = w % Mt (rows mt_w*16 ..) and the
+        // n-tiles ntl = w / Mt + k * nw_mt of every n-block; its V fragments (hi and lo,
+        // all rank steps) are loaded once here and stay in registers for every n-block
+        const int mt_w = warp % Mt;
+        const int nw_mt = (kComputeWarps - mt_w + Mt - 1) / Mt;
+        const int ntl0 = warp / Mt;
+        const int ksteps_e = r16 >> 4;
+        uint32_t vah[4][4], val[4][4];
+        if (!small && nN > 0) {
+            const uint32_t voff = (uint32_t)(((mt_w * 16 + (lane & 15)) * vpitch + (lane >> 4) * 8) * 2);
+            const uint32_t vh_u = ptx::smem_u32(Vh), vl_u = ptx::smem_u32(Vl);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                if (ks < ksteps_e) {
+                    ptx::ldsm_x4(vh_u + voff + ks * 32, vah[ks][0], vah[ks][1], vah[ks][2], vah[ks][3]);
+                    ptx::ldsm_x4(vl_u + voff + ks * 32, val[ks][0], val[ks][1], val[ks][2], val[ks][3]);
+                }
+        }
+
         for (int it = nK; it < nItems; ++it) {
             // -------------------------------------------------------- expand n-block
             const int st = it % kStages;
@@ -694,40 +713,25 @@ sgmv_kernel(const __grid_constant__ AMaps am, const SgmvParams p)
                     ptx::named_sync(1, kCompute);
                 }
                 const int nNTe = (nb + 7) >> 3;
-                const int tiles_e = Mt * nNTe;
-                const int tpw_e = (tiles_e + kComputeWarps - 1) / kComputeWarps;
-                const int ksteps = r16 >> 4;
                 const int gq = lane >> 2, tq = lane & 3;
-                const uint32_t vh_u = ptx::smem_u32(Vh), vl_u = ptx::smem_u32(Vl);
-                for (int q0 = 0; q0 < tpw_e; q0 += 4)
-#pragma unroll
-                for (int q = q0; q < q0 + 4; ++q) {  // 4 tiles unrolled so their MMA chains overlap
-                    const int t = warp * tpw_e + q;
-                    if (q >= tpw_e || t >= tiles_e) continue;
-                    const int mt = t / nNTe, ntl = t - mt * nNTe;
-                    const int row = mt * 16 + (lane & 15);
-                    const uint32_t voff = (uint32_t)((row * vpitch + (lane >> 4) * 8) * 2);
+                for (int ntl = ntl0; ntl < nNTe; ntl += nw_mt) {
                     // row j = ks*16 + (lane & 15) of box ntl/8, 16-byte chunk ntl%8 XOR (j & 7)
                     const uint32_t bbase = base + (uint32_t)((ntl >> 3) * r16 * 128 + (lane & 15) * 128 +
                                                              ((((ntl & 7) ^ (lane & 7))) << 4));
-                    uint32_t ah[4][4], al[4][4], b[4][2];
+                    uint32_t b[4][2];
 #pragma unroll
                     for (int ks = 0; ks < 4; ++ks)
-                        if (ks < ksteps) {
-                            ptx::ldsm_x4(vh_u + voff + ks * 32, ah[ks][0], ah[ks][1], ah[ks][2], ah[ks][3]);
-                            ptx::ldsm_x4(vl_u + voff + ks * 32, al[ks][0], al[ks][1], al[ks][2], al[ks][3]);
-                            ptx::ldsm_x2_t(bbase + ks * 16 * 128, b[ks][0], b[ks][1]);
-                        }
+                        if (ks < ksteps_e) ptx::ldsm_x2_t(bbase + ks * 16 * 128, b[ks][0], b[ks][1]);
                     float c[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
                     for (int ks = 0; ks < 4; ++ks)
-                        if (ks < ksteps) {
-                            ptx::mma_bf16_16816(c[0], ah[ks], b[ks][0], b[ks][1]);
-                            ptx::mma_bf16_16816(c[1], al[ks], b[ks][0], b[ks][1]);
+                        if (ks < ksteps_e) {
+                            ptx::mma_bf16_16816(c[0], vah[ks], b[ks][0], b[ks][1]);
+                            ptx::mma_bf16_16816(c[1], val[ks], b[ks][0], b[ks][1]);
                         }
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
-                        const int rr = mt * 16 + gq + h * 8;
+                        const int rr = mt_w * 16 + gq + h * 8;
                         if (rr < nt) {
                             uint32_t* py =
                                 reinterpret_cast<uint32_t*>(smem + (yb - base_u) + blk_chunk(rr, ntl, Mtr) + tq * 4);
