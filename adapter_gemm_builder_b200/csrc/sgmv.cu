@@ -842,15 +842,23 @@ cudaError_t launch_sgmv(int mode, const void* x, int64_t x_slice_stride, const l
     p.h_in = pool.h_in;
     p.h_out = pool.h_out;
     p.r_max = pool.r_max;
-    // CTAs per tile: up to one per 512 columns of h_in (at most 8), but no more than
-    // fill about eight waves of two CTAs per SM over the tile rows of all slices, so many
-    // small tiles (many tenants) take fewer CTAs each (2 at 4 x 264 tile rows)
+    // CTAs per tile: up to one per 512 columns of h_in (at most 8). When that would
+    // need more than one wave of two CTAs per SM but the tile rows alone fit in one,
+    // take as many per tile as keep one wave (no near-empty last wave: prefill gets 5);
+    // with more tile rows than that (many tenants), 2 per tile, then 1
     int C = (pool.h_in + 511) / 512;
     C = C < 1 ? 1 : (C > kMaxCluster ? kMaxCluster : C);
     {
         const long long rows = (long long)max_tiles_for(seg.T, pool.n_adapters) * pool.n_slices;
-        const long long cap = 16LL * device_sm_count();
-        while (C > 1 && rows * C > cap) C >>= 1;
+        const long long slots = 2LL * device_sm_count();
+        if (rows * C > slots) {
+            if (rows <= slots) {
+                C = (int)(slots / rows);
+            } else {
+                C = C < 2 ? C : 2;
+                if (rows * C > 8 * slots) C = 1;
+            }
+        }
     }
     p.csize = C;
     p.kc = ((pool.h_in + C - 1) / C + 127) / 128 * 128;
