@@ -115,3 +115,18 @@ def test_fp8_gemm_lora_full_size_sampled(M):
     assert np.array_equal(Wq[need], Wq_o) and np.array_equal(sw[need], sw_o)
     want = _oracle_fp8(p, Wq, sw, rows, cols, True)
     assert_close(f64(y[rows, cols]), want, TOL_FP8, f"fp8 full M{M}")
+
+
+@pytest.mark.parametrize("M,K,N,n_adapters,r,kind", [
+    (48, 512, 256, 6, 8, "zipf"),         # r_max 8: B staged as 8-row boxes, rank steps of 16
+    (48, 512, 256, 6, 32, "zipf"),        # r_max 32: two rank steps per adapter
+    (64, 256, 256, 64, 16, "distinct"),   # one adapter per token: more adapters than slots
+    (40, 256, 384, 3, 16, "identical"),   # a single adapter over the whole token block
+])
+def test_fp8_gemm_lora_rank_and_id_mixes(M, K, N, n_adapters, r, kind):
+    p, Wq, sw, y = _fp8_case(M, K, N, n_adapters=n_adapters, r=r, seed=M + r, kind=kind,
+                             none_frac=0.0 if kind != "zipf" else 0.1)
+    rows = np.repeat(np.arange(M), N).astype(np.int32)
+    cols = np.tile(np.arange(N), M).astype(np.int32)
+    want = _oracle_fp8(p, Wq, sw, rows, cols, True).reshape(M, N)
+    assert_close(f64(y), want, TOL_FP8, f"fp8 r{r} {kind}")
