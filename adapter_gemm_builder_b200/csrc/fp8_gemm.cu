@@ -712,16 +712,33 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
             const int n = nb * kBlockM + n_local;
             const float swn = n < p.N ? p.sw[n] : 0.f;
 
+            // partial sums of the later k-blocks for 16 columns (zero when nobody else has any);
+            // the next chunk's are loaded while this one is processed
+            const bool fixup = c_hi > cta + 1;
+            auto load_part = [&](int c, float* out) {
+#pragma unroll
+                for (int e = 0; e < 16; ++e) out[e] = 0.f;
+                for (int cc = cta + 1; cc < c_hi; ++cc) {
+                    const float* src = p.partials + (((size_t)cc * (p.BN >> 4) + (c >> 4)) * 16) * kBlockM + n_local;
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) out[e] += __ldcg(src + e * kBlockM);
+                }
+            };
+            float pf[16];
+            if (fixup && tb * p.BN + grp * 16 < p.M) load_part(grp * 16, pf);
             // 16 tokens per chunk, fully unrolled so the accumulator stays in registers
             for (int c0 = grp * 16; c0 < p.BN; c0 += 32) {
                 const int valid_n = min(16, p.M - (tb * p.BN + c0));  // tokens of this chunk
                 if (valid_n <= 0) break;
                 float acc[16];
                 ptx::tmem_ld16(taddr + (uint32_t)c0, acc);
-                for (int cc = cta + 1; cc < c_hi; ++cc) {  // partial sums of the later k-blocks
-                    const float* src = p.partials + (((size_t)cc * (p.BN >> 4) + (c0 >> 4)) * 16) * kBlockM + n_local;
+                const int c1 = c0 + 32;
+                const bool more = fixup && c1 < p.BN && tb * p.BN + c1 < p.M;
+                float pn[16];
+                if (more) load_part(c1, pn);
+                if (fixup) {
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) acc[e] += __ldcg(src + e * kBlockM);
+                    for (int e = 0; e < 16; ++e) acc[e] += pf[e];
                 }
                 float lo[16];
 #pragma unroll
@@ -756,6 +773,10 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
                         const __nv_bfloat16 o = __float2bfloat16_rn(out);
                         p.y[(size_t)s_m[c0 + e] * p.N + n] = *reinterpret_cast<const uint16_t*>(&o);
                     }
+                }
+                if (more) {
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) pf[e] = pn[e];
                 }
             }
             ptx::tc_fence_before();
