@@ -201,11 +201,13 @@ def dist_setup(args):
 
 
 def dist_max(val, world):
+    """Max of a per-rank value over all ranks (NCCL on the GPU, gloo on the host)."""
     if world == 1:
         return val
     import torch
     import torch.distributed as dist
-    t = torch.tensor([val], dtype=torch.float64, device="cuda")
+    device = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([val], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
