@@ -23,7 +23,11 @@ quantize_rows_kernel(const uint16_t* __restrict__ x, const int32_t* __restrict__
                      size_t zero_words)
 {
     __shared__ float s_red[kThreads / 32];
-    ptx::pdl_launch_dependents();  // the GEMM may start streaming its weights now
+    // launched as a programmatic dependent of the previous kernel (which may produce x
+    // or still read this call's scratch): wait for it, then let the GEMM start streaming
+    // its weights
+    ptx::pdl_wait();
+    ptx::pdl_launch_dependents();
     if (zero) {  // scratch the dependent GEMM accumulates into (block b: its slice)
         const size_t per = (zero_words + gridDim.x - 1) / gridDim.x;
         const size_t z0 = per * blockIdx.x, z1 = min(zero_words, z0 + per);
@@ -77,9 +81,17 @@ cudaError_t launch_quantize_rows(const void* x, const int32_t* perm, int M, int 
                                  float* sx, void* zero, size_t zero_words, cudaStream_t stream)
 {
     if (M == 0) return cudaSuccess;
-    quantize_rows_kernel<<<M, kThreads, 0, stream>>>(static_cast<const uint16_t*>(x), perm, K, xq,
-                                                      sx, static_cast<uint32_t*>(zero), zero_words);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)M, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, quantize_rows_kernel, static_cast<const uint16_t*>(x), perm, K, xq, sx,
+                              static_cast<uint32_t*>(zero), zero_words);
 }
 
 }  // namespace lora
