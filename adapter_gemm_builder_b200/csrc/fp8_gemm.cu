@@ -61,7 +61,8 @@ struct GemmParams {
     const float* sw;
     uint16_t* y;
     uint32_t* status;
-    float* partials;  // [gridDim.x][128][BN] fp32 stream-K partial accumulators
+    float* partials;  // fp32 stream-K partial accumulators, [gridDim.x][BN/16][4][128][4]
+                      // (per 16-token chunk: four float4 planes over the 128 rows)
     int* flags;       // [gridDim.x] partial of CTA c stored
     int* v_done;      // down-projection items finished
     int lora;
@@ -82,6 +83,24 @@ struct GemmParams {
 };
 
 using ptx::globaltimer;
+
+// Transpose an 8x8 matrix of 32-bit words held by 8 consecutive lanes (lane j of
+// the group holds row j in w[0..7]); afterwards lane j holds column j. Three
+// butterfly stages swap the off-diagonal blocks of 4x4, 2x2 and 1x1 words.
+__device__ __forceinline__ void transpose8x8(uint32_t (&w)[8], int lane)
+{
+#pragma unroll
+    for (int s = 4; s >= 1; s >>= 1) {
+        const bool upper = (lane & s) != 0;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            if (k & s) continue;
+            const uint32_t send = upper ? w[k] : w[k | s];
+            const uint32_t recv = __shfl_xor_sync(0xffffffffu, send, s);
+            if (upper) w[k] = recv; else w[k | s] = recv;
+        }
+    }
+}
 
 // Bounded wait on an mbarrier phase. Returns false if the CTA is aborting
 // (another role gave up) or if this wait itself timed out (then it raises the
@@ -244,6 +263,8 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
         ptx::tmem_alloc(&s_tmem, ncols);
         ptx::tmem_relinquish();
     }
+    // __syncthreads is an aligned barrier: every warp reaches it converged
+    __syncwarp();
     ptx::tc_fence_before();
     __syncthreads();
     ptx::tc_fence_after();
@@ -563,14 +584,15 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
                 // later k-blocks of a tile another CTA finishes: fp32 partials to the workspace
                 if (!wait_bounded(&tfull[buf], (uint32_t)((i >> 1) & 1), abort_flag, p.status, 0x10u)) break;
                 ptx::tc_fence_after();
-                // layout [cta][16-column chunk][column][128 rows]: each store of a warp
-                // covers 128 contiguous bytes
+                // per 16-column chunk four planes [128 rows][4 columns]: each store of a
+                // warp covers 512 contiguous bytes
                 for (int c0 = grp * 16; c0 < p.BN; c0 += 32) {
                     float acc[16];
                     ptx::tmem_ld16(taddr + (uint32_t)c0, acc);
-                    float* dst = p.partials + (((size_t)cta * (p.BN >> 4) + (c0 >> 4)) * 16) * kBlockM + n_local;
+                    float4* dst = reinterpret_cast<float4*>(p.partials + ((size_t)cta * (p.BN >> 4) + (c0 >> 4)) * 2048) + n_local;
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) __stcg(dst + e * kBlockM, acc[e]);
+                    for (int q = 0; q < 4; ++q)
+                        __stcg(dst + q * kBlockM, make_float4(acc[4 * q], acc[4 * q + 1], acc[4 * q + 2], acc[4 * q + 3]));
                 }
                 ptx::tc_fence_before();
                 __syncwarp();
@@ -715,30 +737,49 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
             // partial sums of the later k-blocks for 16 columns (zero when nobody else has any);
             // the next chunk's are loaded while this one is processed
             const bool fixup = c_hi > cta + 1;
-            auto load_part = [&](int c, float* out) {
+            // the partial sums of the next CTA (the usual single contributor) are loaded two
+            // chunks ahead of their use, as raw registers; those of any further CTA are added
+            // when their chunk is processed
+            auto part_src = [&](int cc, int c) {
+                return reinterpret_cast<const float4*>(p.partials + ((size_t)cc * (p.BN >> 4) + (c >> 4)) * 2048) + n_local;
+            };
+            auto part_issue = [&](int c, float4 (&dst)[4]) {
+                if (fixup && c < p.BN && tb * p.BN + c < p.M) {
+                    const float4* src = part_src(cta + 1, c);
 #pragma unroll
-                for (int e = 0; e < 16; ++e) out[e] = 0.f;
-                for (int cc = cta + 1; cc < c_hi; ++cc) {
-                    const float* src = p.partials + (((size_t)cc * (p.BN >> 4) + (c >> 4)) * 16) * kBlockM + n_local;
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) out[e] += __ldcg(src + e * kBlockM);
+                    for (int q = 0; q < 4; ++q) dst[q] = __ldcg(src + q * kBlockM);
                 }
             };
-            float pf[16];
-            if (fixup && tb * p.BN + grp * 16 < p.M) load_part(grp * 16, pf);
+            float4 pa[4], pb[4];  // chunk c0 and chunk c0 + 32 of this warp
+            part_issue(grp * 16, pa);
+            part_issue(grp * 16 + 32, pb);
             // 16 tokens per chunk, fully unrolled so the accumulator stays in registers
             for (int c0 = grp * 16; c0 < p.BN; c0 += 32) {
                 const int valid_n = min(16, p.M - (tb * p.BN + c0));  // tokens of this chunk
                 if (valid_n <= 0) break;
                 float acc[16];
                 ptx::tmem_ld16(taddr + (uint32_t)c0, acc);
-                const int c1 = c0 + 32;
-                const bool more = fixup && c1 < p.BN && tb * p.BN + c1 < p.M;
-                float pn[16];
-                if (more) load_part(c1, pn);
                 if (fixup) {
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) acc[e] += pf[e];
+                    for (int q = 0; q < 4; ++q) {
+                        acc[4 * q] += pa[q].x;
+                        acc[4 * q + 1] += pa[q].y;
+                        acc[4 * q + 2] += pa[q].z;
+                        acc[4 * q + 3] += pa[q].w;
+                        pa[q] = pb[q];
+                    }
+                    part_issue(c0 + 64, pb);
+                    for (int cc = cta + 2; cc < c_hi; ++cc) {
+                        const float4* src = part_src(cc, c0);
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            const float4 f = __ldcg(src + q * kBlockM);
+                            acc[4 * q] += f.x;
+                            acc[4 * q + 1] += f.y;
+                            acc[4 * q + 2] += f.z;
+                            acc[4 * q + 3] += f.w;
+                        }
+                    }
                 }
                 float lo[16];
 #pragma unroll
@@ -765,18 +806,43 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
                         }
                     }
                 }
-                if (n < p.N) {
+                {
+                    // y is 16-byte aligned and N % 8 == 0 (checked by the caller): after an 8x8
+                    // transpose inside each group of 8 lanes, a lane holds two token rows of 8
+                    // consecutive columns, so a chunk takes two 16-byte stores instead of 16
+                    float sxv[16];
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        if (e >= valid_n) break;
-                        const float out = acc[e] * s_sx[c0 + e] * swn + lo[e];
-                        const __nv_bfloat16 o = __float2bfloat16_rn(out);
-                        p.y[(size_t)s_m[c0 + e] * p.N + n] = *reinterpret_cast<const uint16_t*>(&o);
+                    for (int q = 0; q < 4; ++q) {
+                        const float4 f = reinterpret_cast<const float4*>(s_sx + c0)[q];
+                        sxv[4 * q] = f.x;
+                        sxv[4 * q + 1] = f.y;
+                        sxv[4 * q + 2] = f.z;
+                        sxv[4 * q + 3] = f.w;
                     }
-                }
-                if (more) {
+                    uint32_t w[8];
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) pf[e] = pn[e];
+                    for (int k = 0; k < 8; ++k) {
+                        const float o0 = acc[2 * k] * sxv[2 * k] * swn + lo[2 * k];
+                        const float o1 = acc[2 * k + 1] * sxv[2 * k + 1] * swn + lo[2 * k + 1];
+                        __nv_bfloat162 h = __floats2bfloat162_rn(o0, o1);
+                        w[k] = *reinterpret_cast<uint32_t*>(&h);
+                    }
+                    transpose8x8(w, lane);
+                    const int j = lane & 7;                                 // token pair of this lane
+                    const int ng = nb * kBlockM + quarter * 32 + (lane & ~7);  // its 8 columns
+                    const int2 rows = reinterpret_cast<const int2*>(s_m + c0)[j];
+                    if (ng < p.N) {                                         // N % 8 == 0: all 8 or none
+                        if (2 * j < valid_n) {
+                            const uint4 r0 = make_uint4(__byte_perm(w[0], w[1], 0x5410), __byte_perm(w[2], w[3], 0x5410),
+                                                        __byte_perm(w[4], w[5], 0x5410), __byte_perm(w[6], w[7], 0x5410));
+                            *reinterpret_cast<uint4*>(p.y + (size_t)rows.x * p.N + ng) = r0;
+                        }
+                        if (2 * j + 1 < valid_n) {
+                            const uint4 r1 = make_uint4(__byte_perm(w[0], w[1], 0x7632), __byte_perm(w[2], w[3], 0x7632),
+                                                        __byte_perm(w[4], w[5], 0x7632), __byte_perm(w[6], w[7], 0x7632));
+                            *reinterpret_cast<uint4*>(p.y + (size_t)rows.y * p.N + ng) = r1;
+                        }
+                    }
                 }
             }
             ptx::tc_fence_before();
@@ -789,6 +855,9 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
         }
     }
 
+    // the single-lane roles of warps 0-2 rejoin their warps before the aligned barrier
+    // (otherwise a lane arriving late is not held by it)
+    __syncwarp();
     ptx::tc_fence_before();
     __syncthreads();
     if (warp == 1) {

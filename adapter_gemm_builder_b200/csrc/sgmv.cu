@@ -214,6 +214,7 @@ sgmv_kernel(const __grid_constant__ AMaps am, const SgmvParams p)
         ptx::mbar_init(red2, 1);
         ptx::fence_mbar_init();
     }
+    __syncwarp();  // __syncthreads is an aligned barrier: warps reach it converged
     // Cluster barrier, phase 0: this CTA's mbarriers exist (peers wait for it before
     // their first remote store); phase 1: this CTA makes no more remote accesses (every
     // CTA waits for it before leaving). Phase 0 is announced before the wait on the
@@ -295,6 +296,7 @@ sgmv_kernel(const __grid_constant__ AMaps am, const SgmvParams p)
         ptx::mbar_arrive_expect_tx(red1, (uint32_t)((one_phase ? C * nt : C * mine) * r8 * 4));
         ptx::mbar_arrive_expect_tx(red2, one_phase ? 0u : (uint32_t)(nt * r8 * 4));
     }
+    __syncwarp();
     __syncthreads();
 
     if (warp == kComputeWarps) {

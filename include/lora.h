@@ -223,10 +223,11 @@ LORA_API int fp8_quantize_rows(const void* x, int M, int K, uint8_t* xq, float* 
  *   a = seg->tok_adapter[m]; the LoRA term is absent when a == -1 or pool == NULL;
  *   xq, sx: x quantised per token as in fp8_quantize_rows;
  *   v = x.A_a in fp32 from the unquantised bf16 x (as lora_shrink).
- * Launch order: the activation quantiser, then the shrink (the
- * down-projection, launched first as the page describes), then the GEMM as a
- * programmatic dependent launch: its mainloop starts streaming Wq while the
- * shrink runs and it waits for v only before its epilogue.
+ * Two launches: the activation quantiser, then the GEMM as its programmatic
+ * dependent. The GEMM's mainloop starts streaming Wq at once. Its epilogue
+ * warps compute the down-projection v meanwhile; the page runs it first as a
+ * separate shrink. Each CTA waits for the whole v only before its first
+ * epilogue.
  *   x bf16 [M][K]; Wq e4m3 [N][K]; w_scale fp32 [N]; y bf16 [M][N] (out).
  *   pool: NULL for the base GEMM alone; else n_slices == 1, h_in == K, h_out == N.
  *   seg: required when pool != NULL (built for these M tokens); may be NULL otherwise.

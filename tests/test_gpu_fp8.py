@@ -130,3 +130,21 @@ def test_fp8_gemm_lora_rank_and_id_mixes(M, K, N, n_adapters, r, kind):
     cols = np.tile(np.arange(N), M).astype(np.int32)
     want = _oracle_fp8(p, Wq, sw, rows, cols, True).reshape(M, N)
     assert_close(f64(y), want, TOL_FP8, f"fp8 r{r} {kind}")
+
+
+
+def test_fp8_gemm_rejects_unaligned_y():
+    """y must start on a 16-byte boundary (the epilogue writes 16-byte row pieces):
+    a y two bytes past one is refused before anything is launched."""
+    M, K, N = 16, 256, 256
+    x = torch.zeros((M, K), dtype=torch.bfloat16, device="cuda")
+    Wq = torch.zeros((N, K), dtype=torch.uint8, device="cuda")
+    sw = torch.ones(N, dtype=torch.float32, device="cuda")
+    y_buf = torch.full((M * N + 1,), float("nan"), dtype=torch.bfloat16, device="cuda")
+    ws = L.workspace(L.LORA_OP_FP8_GEMM, M, K, None)
+    with pytest.raises(L.LoraError) as err:
+        L.fp8_gemm_lora_epilogue(x, Wq, sw, None, None, y_buf[1:].view(M, N), ws)
+    assert err.value.status == L.LORA_ERR_INVALID_ARG
+    L.fp8_gemm_lora_epilogue(x, Wq, sw, None, None, y_buf[:-1].view(M, N), ws)
+    torch.cuda.synchronize()
+    assert torch.count_nonzero(y_buf[:-1]).item() == 0  # all-zero x: y = 0
