@@ -59,7 +59,7 @@ size_t fp8_ws_layout(int M, int K, const lora_pool_t* pool, size_t* off_xq, size
     *off_sx = off;
     off += align256((size_t)M * 4);
     *off_v = off;
-    if (pool) off += align256((size_t)M * pool->r_max * 4);
+    if (pool) off += align256((size_t)fp8_gemm_v_copies(M) * M * pool->r_max * 4);
     *off_sync = off;  // [0]: down-projection count, [16 ..]: one flag per SM
     off += align256((size_t)(16 + device_sm_count()) * 4);
     *off_part = off;

@@ -73,7 +73,9 @@ struct GemmParams {
     const int32_t* indptr;
     const int32_t* active;
     const int32_t* counts;
-    float* v;  // fp32 [M][r_max], segment (perm) order, zeroed by the quantiser
+    float* v;  // fp32 [v_rep][M][r_max], segment (perm) order, zeroed by the quantiser: the
+               // down-projection of K chunk q adds into copy q % v_rep (fewer atomics per address)
+    int v_rep, lg_rep;  // copies of v (a power of two), log2
     const uint16_t* B;
     const int32_t* ranks;
     const float* scales;
@@ -521,21 +523,30 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
             int ls = 0;
             while (ls < 2 && (p.M << (lg + ls + 1)) <= kEpiThreads) ++ls;
             const int kspan = kShrinkCols >> ls;  // 64, 32 or 16 columns per thread
+            const int total = p.M << (lg + ls);
             for (int q = cta; q < n_chunks && ok; q += G) {
-                for (int w = etid; w < (p.M << (lg + ls)); w += kEpiThreads) {
+                float* vcopy = p.v + (size_t)(q & (p.v_rep - 1)) * p.M * p.r_max;
+                // work items w: (token, group of 8 ranks, K sub-range); the 2^ls sub-ranges of
+                // one (token, group) sit in consecutive lanes, the loop is uniform per warp
+                for (int wb = ew * 32; wb < total; wb += kEpiThreads) {
+                    const int w = wb + lane;
                     const int pg = w >> ls, sub = w & ((1 << ls) - 1);
                     const int pp = pg >> lg, g = pg & (ng - 1);
                     const int k0 = q * kShrinkCols + sub * kspan;
-                    const int kw = min(kspan, p.K - k0);  // a multiple of 16 (or <= 0)
-                    if (kw <= 0) continue;
-                    const int m = p.perm[pp];
-                    const int a = p.tok_adapter[m];
-                    if (a < 0) continue;
-                    int r = p.ranks ? p.ranks[a] : p.r_max;
-                    r = max(1, min(r, p.r_max));
-                    if (8 * g >= r) continue;
+                    int kw = min(kspan, p.K - k0);  // a multiple of 16 (or <= 0)
+                    int r = 0, m = 0, a = -1;
+                    if (w < total && kw > 0) {
+                        m = p.perm[pp];
+                        a = p.tok_adapter[m];
+                        if (a >= 0) {
+                            r = p.ranks ? p.ranks[a] : p.r_max;
+                            r = max(1, min(r, p.r_max));
+                        }
+                    }
+                    const bool live = a >= 0 && 8 * g < r;
+                    if (!live) kw = 0;
                     const uint4* xr = reinterpret_cast<const uint4*>(p.x + (size_t)m * p.K + k0);
-                    const uint16_t* ar = p.A + ((size_t)a * p.K + k0) * p.r_max + 8 * g;
+                    const uint16_t* ar = p.A + ((size_t)max(a, 0) * p.K + k0) * p.r_max + 8 * g;
                     float acc[8];
 #pragma unroll
                     for (int e = 0; e < 8; ++e) acc[e] = 0.f;
@@ -561,9 +572,16 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
 #pragma unroll
                     for (int e = 0; e < 8; ++e)
                         if (8 * g + e >= r) acc[e] = 0.f;  // the pool's padding past the rank
-                    float* vd = p.v + (size_t)pp * p.r_max + 8 * g;
-                    atomicAdd(reinterpret_cast<float4*>(vd), make_float4(acc[0], acc[1], acc[2], acc[3]));
-                    atomicAdd(reinterpret_cast<float4*>(vd + 4), make_float4(acc[4], acc[5], acc[6], acc[7]));
+                    // the sub-ranges' sums meet in their first lane: one pair of atomics per item
+                    for (int o = 1; o < (1 << ls); o <<= 1) {
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], o);
+                    }
+                    if (live && sub == 0 && w < total) {
+                        float* vd = vcopy + (size_t)pp * p.r_max + 8 * g;
+                        atomicAdd(reinterpret_cast<float4*>(vd), make_float4(acc[0], acc[1], acc[2], acc[3]));
+                        atomicAdd(reinterpret_cast<float4*>(vd + 4), make_float4(acc[4], acc[5], acc[6], acc[7]));
+                    }
                 }
                 __threadfence();
                 ok = epi_sync();
@@ -646,41 +664,89 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
                 if (slotted_tb != tb) {
                     // per token: its slot (-2: adapter not staged, done on CUDA cores below);
                     // per slot q: V'_q[t][j] = s_q v[t][j] / sx[t] for its tokens t (zero for the
-                    // other tokens of its 16-aligned column range), K-major bf16
-                    for (int pl = etid; pl < p.BN; pl += kEpiThreads) {
+                    // other tokens of its 16-aligned column range), K-major bf16. Each thread owns
+                    // at most one token (BN <= 256): it loads that token's v row first, so the
+                    // whole build waits for one round trip to memory, not one per slot
+                    // lane (token pl, copy cp): v_rep consecutive lanes load the copies of one
+                    // token's v row and sum them with shuffles (BN * v_rep <= 256)
+                    const int pl = etid >> p.lg_rep, cp = etid & (p.v_rep - 1);
+                    int q_own = -1;
+                    float4 vr[4];  // v[token][0..16) (a larger rank loads the rest later)
+#pragma unroll
+                    for (int h = 0; h < 4; ++h) vr[h] = make_float4(0.f, 0.f, 0.f, 0.f);
+                    const float4* vg = reinterpret_cast<const float4*>(
+                        p.v + ((size_t)cp * p.M + tb * p.BN + min(pl, p.BN - 1)) * p.r_max);
+                    if (pl < p.BN) {
                         const int a = s_a[pl];
-                        int q = -1;
                         if (a >= 0) {
-                            q = -2;
+                            q_own = -2;
                             for (int t = 0; t < nsl; ++t)
-                                if (s_slot_adapter[t] == a) { q = t; break; }
+                                if (s_slot_adapter[t] == a) { q_own = t; break; }
                         }
-                        s_q[pl] = q;
+                        if (cp == 0) s_q[pl] = q_own;
+                        if (q_own >= 0) {
+#pragma unroll
+                            for (int h = 0; h < 4; ++h)
+                                if (4 * h < p.r_max) vr[h] = __ldcg(vg + h);
+                        }
                     }
+                    // zero every slot's tile and publish its byte offset
                     int off = 0;
                     for (int q = 0; q < nsl; ++q) {
                         const int4 lq = s_lq[q];
-                        const int c0 = lq.x & ~15, w = ((lq.y + 15) & ~15) - c0;
-                        const int a = s_slot_adapter[q], r = s_slot_rank[q];
-                        const float sc = p.scales ? p.scales[a] : 1.f;
+                        const int w = ((lq.y + 15) & ~15) - (lq.x & ~15);
                         if (etid == 0) s_lq[q].z = off;
-                        for (int idx = etid; idx < w * kgq; idx += kEpiThreads) {
-                            const int rr = idx / kgq, kg = idx - rr * kgq;
-                            const int t = c0 + rr, pp = tb * p.BN + t;
-                            const bool mine = t >= lq.x && t < lq.y;
-                            const float f = mine ? sc / s_sx[t] : 0.f;
+                        for (int i = etid; i < w * kgq; i += kEpiThreads)
+                            *reinterpret_cast<uint4*>(vq + off + i * 16) = make_uint4(0u, 0u, 0u, 0u);
+                        off += w * kgq * 16;
+                    }
+                    if (!(ok = epi_sync())) break;
+                    auto sum_copies = [&](float4& f) {
+                        for (int o = 1; o < p.v_rep; o <<= 1) {
+                            f.x += __shfl_xor_sync(0xffffffffu, f.x, o);
+                            f.y += __shfl_xor_sync(0xffffffffu, f.y, o);
+                            f.z += __shfl_xor_sync(0xffffffffu, f.z, o);
+                            f.w += __shfl_xor_sync(0xffffffffu, f.w, o);
+                        }
+                    };
+#pragma unroll
+                    for (int h = 0; h < 4; ++h) sum_copies(vr[h]);
+                    {  // this token's row of its slot's tile (lane cp == 0 writes it)
+                        const int4 lq = s_lq[max(q_own, 0)];
+                        const int rr = pl - (lq.x & ~15);
+                        const int r = q_own >= 0 ? s_slot_rank[q_own] : 0;
+                        const float f = q_own >= 0 ? (p.scales ? p.scales[s_slot_adapter[q_own]] : 1.f) / s_sx[pl] : 0.f;
+#pragma unroll
+                        for (int kg = 0; kg < MAXR / 8; ++kg) {
+                            if (kg >= kgq) break;
+                            float vv[8];
+                            const bool in_row = q_own >= 0 && 8 * kg < p.r_max;  // r_max: a multiple of 8
+                            float4 f0 = make_float4(0.f, 0.f, 0.f, 0.f), f1 = f0;
+                            if (kg < 2) {
+                                f0 = vr[2 * kg];
+                                f1 = vr[2 * kg + 1];
+                            } else {
+                                if (in_row) {
+                                    f0 = __ldcg(vg + 2 * kg);
+                                    f1 = __ldcg(vg + 2 * kg + 1);
+                                }
+                                sum_copies(f0);
+                                sum_copies(f1);
+                            }
+                            if (q_own < 0 || cp != 0) continue;
+                            vv[0] = f0.x; vv[1] = f0.y; vv[2] = f0.z; vv[3] = f0.w;
+                            vv[4] = f1.x; vv[5] = f1.y; vv[6] = f1.z; vv[7] = f1.w;
                             uint32_t wv[4];
 #pragma unroll
                             for (int h = 0; h < 4; ++h) {
                                 const int j = kg * 8 + 2 * h;
-                                const float v0 = (mine && j < r) ? f * __ldcg(p.v + (size_t)pp * p.r_max + j) : 0.f;
-                                const float v1 = (mine && j + 1 < r) ? f * __ldcg(p.v + (size_t)pp * p.r_max + j + 1) : 0.f;
+                                const float v0 = j < r ? f * vv[2 * h] : 0.f;
+                                const float v1 = j + 1 < r ? f * vv[2 * h + 1] : 0.f;
                                 __nv_bfloat162 hv = __floats2bfloat162_rn(v0, v1);
                                 wv[h] = *reinterpret_cast<uint32_t*>(&hv);
                             }
-                            *reinterpret_cast<uint4*>(vq + off + kmajor_off(rr, kg, kgq)) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+                            *reinterpret_cast<uint4*>(vq + lq.z + kmajor_off(rr, kg, kgq)) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
                         }
-                        off += w * kgq * 16;
                     }
                     slotted_tb = tb;
                 }
@@ -798,8 +864,11 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
                             const uint16_t* gb = p.B + ((size_t)a * p.r_max) * p.N + n;
                             const float* vg = p.v + (size_t)(tb * p.BN + c0 + e) * p.r_max;
                             float l = 0.f;
-                            for (int j = 0; j < r; ++j)
-                                l = fmaf(__ldcg(vg + j), n < p.N ? __uint_as_float((uint32_t)gb[(size_t)j * p.N] << 16) : 0.f, l);
+                            for (int j = 0; j < r; ++j) {
+                                float vj = 0.f;
+                                for (int c = 0; c < p.v_rep; ++c) vj += __ldcg(vg + (size_t)c * p.M * p.r_max + j);
+                                l = fmaf(vj, n < p.N ? __uint_as_float((uint32_t)gb[(size_t)j * p.N] << 16) : 0.f, l);
+                            }
 #pragma unroll
                             for (int e2 = 0; e2 < 16; ++e2)
                                 if (e2 == e) lo[e2] = sc * l;
@@ -920,6 +989,15 @@ int fp8_gemm_tile_n(int M)
     return (((M + n_tb - 1) / n_tb) + 15) / 16 * 16;
 }
 
+int fp8_gemm_v_copies(int M)
+{
+    // as many copies as the V' build has lanes to spare per token (at most 8)
+    const int bn = fp8_gemm_tile_n(M);
+    int c = 1;
+    while (c < 8 && bn * c * 2 <= kEpiThreads) c *= 2;
+    return c;
+}
+
 size_t fp8_gemm_partial_bytes(int M)
 {
     return (size_t)device_sm_count() * kBlockM * (size_t)fp8_gemm_tile_n(M) * 4;
@@ -951,6 +1029,8 @@ cudaError_t launch_fp8_gemm(const Fp8GemmArgs& a, cudaStream_t stream)
     p.active = a.active;
     p.counts = a.counts;
     p.v = a.v;
+    p.v_rep = fp8_gemm_v_copies(a.M);
+    p.lg_rep = __builtin_ctz((unsigned)p.v_rep);
     p.B = a.B;
     p.ranks = a.ranks;
     p.scales = a.scales;

@@ -58,6 +58,8 @@ cudaError_t launch_fp8_gemm(const Fp8GemmArgs& a, cudaStream_t stream);
 // Token columns of a GEMM tile for M tokens, and the bytes of partial sums.
 int fp8_gemm_tile_n(int M);
 size_t fp8_gemm_partial_bytes(int M);
+// copies of the down-projection v the fused GEMM spreads its atomics over (a power of two)
+int fp8_gemm_v_copies(int M);
 
 int device_sm_count();
 
