@@ -73,6 +73,7 @@ struct GemmParams {
     const int32_t* indptr;
     const int32_t* active;
     const int32_t* counts;
+    int v_adapters;  // adapters of a token block whose V' tiles fit (the rest: CUDA cores)
     float* v;  // fp32 [v_rep][M][r_max], segment (perm) order, zeroed by the quantiser: the
                // down-projection of K chunk q adds into copy q % v_rep (fewer atomics per address)
     int v_rep, lg_rep;  // copies of v (a power of two), log2
@@ -215,7 +216,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     __shared__ uint32_t s_tmem;
     __shared__ int s_abort;
-    __shared__ int s_nslots;
+    __shared__ int s_nact;  // adapters of the current token block on the tensor cores
     __shared__ int s_slot_adapter[256];
     __shared__ int s_slot_rank[256];
     __shared__ int4 s_lq[256];  // per slot: first / end token (block-relative), V' byte offset
@@ -245,7 +246,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
 
     if (threadIdx.x == 0) {
         s_abort = 0;
-        s_nslots = 0;
+        s_nact = 0;
         for (int s = 0; s < p.stages; ++s) {
             ptx::mbar_init(&full[s], 1);
             ptx::mbar_init(&empty[s], 1);
@@ -255,7 +256,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
             ptx::mbar_init(&tempty[b], kEpiWarps);
         }
         ptx::mbar_init(bfull, 1);
-        ptx::mbar_init(bempty, kEpiWarps);
+        ptx::mbar_init(bempty, 1);  // tcgen05.commit of a LoRA phase
         ptx::mbar_init(drain, 1);
         ptx::mbar_init(epibar, kEpiWarps);
         ptx::mbar_init(lready, 1);
@@ -339,35 +340,64 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
             int i = 0, lj = 0;
             const uint32_t slots_u = smem_u + p.slots_off, vq_u = smem_u + p.v_off;
             const int kgq = p.r16 >> 3;
-            // the up-projection of a finished segment waits for its operands (lready) without
-            // holding up the next segment's k-blocks: it is issued as soon as they are built
-            int pend_buf = -1;
-            auto issue_lora = [&](int pbuf) {
+            // The up-projection of a y-segment (one that ends in an epilogue) comes in
+            // phases of at most n_slots adapters: the epilogue warps build a phase's
+            // operands and signal lready, this thread adds them to the segment's
+            // accumulator between its own k-blocks (after the segment's first k-block,
+            // which starts the accumulator) and commits bempty, which frees the slots
+            // for the next phase. tfull follows the last k-block and the last phase.
+            // At most two y-segments wait for phases (the two TMEM buffers), in order.
+            int fq_buf[2] = {0, 0}, fq_ph[2] = {0, 0};
+            bool fq_base_done[2] = {false, false};
+            int fq_n = 0;
+            auto issue_phase = [&]() {
                 ++lj;
                 ptx::tc_fence_after();
+                const int pbuf = fq_buf[0];
                 const uint32_t dp = tmem_base + (uint32_t)(pbuf * p.BN);
-                const int nsl = s_nslots;
-                for (int q = 0; q < nsl; ++q) {
-                    // D[n][t] += (B_q[j][n] / sw[n]) * (s_q v[t][j] / sx[t]) over adapter q's tokens
-                    const int4 lq = s_lq[q];
+                const int nact = s_nact;
+                const int e0 = fq_ph[0] * p.n_slots, e1 = min(nact, e0 + p.n_slots);
+                for (int e = e0; e < e1; ++e) {
+                    // D[n][t] += (B_a[j][n] / sw[n]) * (s_a v[t][j] / sx[t]) over adapter a's tokens
+                    const int4 lq = s_lq[e];
                     const int c0 = lq.x & ~15, w = ((lq.y + 15) & ~15) - c0;
                     const uint32_t idl = make_idesc_bf16(w);
+                    const uint32_t sb = slots_u + (uint32_t)((e - e0) * p.r16 * 256);
                     for (int ks = 0; ks < (p.r16 >> 4); ++ks)
-                        ptx::tc_mma_f16(dp + (uint32_t)c0,
-                                        make_desc_kmajor(slots_u + (uint32_t)(q * p.r16 * 256 + ks * 256), kgq),
+                        ptx::tc_mma_f16(dp + (uint32_t)c0, make_desc_kmajor(sb + (uint32_t)(ks * 256), kgq),
                                         make_desc_kmajor(vq_u + (uint32_t)(lq.z + ks * 256), kgq), idl, 1u);
                 }
-                ptx::tc_commit(&tfull[pbuf]);
+                ptx::tc_commit(bempty);  // the slots may be refilled once these MMAs are done
+                ++fq_ph[0];
+                if (e1 >= nact) {  // that was the segment's last phase
+                    if (fq_base_done[0]) ptx::tc_commit(&tfull[pbuf]);
+                    else fq_ph[0] = -1;  // tfull goes with the segment's last k-block
+                    if (fq_base_done[0]) {
+                        fq_buf[0] = fq_buf[1];
+                        fq_ph[0] = fq_ph[1];
+                        fq_base_done[0] = fq_base_done[1];
+                        --fq_n;
+                    }
+                }
             };
-            auto resolve_pending = [&](bool block) -> bool {
-                if (pend_buf < 0) return true;
+            // issue the next phase of the oldest waiting segment if its operands are ready
+            // (block: wait for them, bounded)
+            auto lora_step = [&](bool block) -> bool {
+                if (fq_n == 0 || fq_ph[0] < 0) return true;
                 if (block) {
                     if (!wait_bounded(lready, (uint32_t)(lj & 1), abort_flag, p.status, 0x200u)) return false;
-                } else if (!ptx::mbar_try_wait(lready, (uint32_t)(lj & 1))) {
+                } else if (!ptx::mbar_test_wait(lready, (uint32_t)(lj & 1))) {  // no suspend
                     return true;
                 }
-                issue_lora(pend_buf);
-                pend_buf = -1;
+                issue_phase();
+                return true;
+            };
+            // every phase of the waiting segment that uses TMEM buffer b
+            auto lora_flush = [&](int b) -> bool {
+                while (fq_n > 0 && (b < 0 || fq_buf[0] == b || (fq_n > 1 && fq_buf[1] == b))) {
+                    if (fq_ph[0] < 0) return true;  // its k-blocks are not all issued yet
+                    if (!lora_step(true)) return false;
+                }
                 return true;
             };
             for (long long u = u_begin; u < u_end && ok; ++i) {
@@ -375,7 +405,8 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
                 u += sg.kb1 - sg.kb0;
                 const int buf = i & 1;
                 const uint32_t bphase = (uint32_t)((i >> 1) & 1);
-                if (pend_buf == buf && !resolve_pending(true)) {  // that buffer's epilogue comes first
+                const bool yseg = p.lora && sg.kb0 == 0;
+                if (!lora_flush(buf)) {  // that buffer's epilogue comes first
                     ok = false;
                     break;
                 }
@@ -386,7 +417,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
                 ptx::tc_fence_after();
                 const uint32_t d = tmem_base + (uint32_t)(buf * p.BN);
                 for (int kb = sg.kb0; kb < sg.kb1; ++kb) {
-                    if (!resolve_pending(false) ||
+                    if (!lora_step(false) ||
                         !wait_bounded(&full[stage], phase, abort_flag, p.status, 0x4u)) {
                         ok = false;
                         break;
@@ -404,24 +435,26 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
                         stage = 0;
                         phase ^= 1;
                     }
+                    if (yseg && kb == sg.kb0) {  // the accumulator is started: phases may follow
+                        fq_buf[fq_n] = buf;
+                        fq_ph[fq_n] = 0;
+                        fq_base_done[fq_n] = false;
+                        ++fq_n;
+                    }
                 }
                 if (!ok) break;
-                if (p.lora && sg.kb0 == 0) {
-                    // an earlier segment's up-projection goes first (lready phases are in order)
-                    if (!resolve_pending(true)) {
-                        ok = false;
-                        break;
-                    }
-                    pend_buf = buf;
-                    if (!resolve_pending(false)) {
-                        ok = false;
-                        break;
+                if (yseg) {
+                    const int q = fq_n - 1;  // this segment's entry (the newest)
+                    fq_base_done[q] = true;
+                    if (fq_ph[q] < 0) {  // its phases were all issued already
+                        ptx::tc_commit(&tfull[buf]);
+                        --fq_n;  // it is the only entry: an older one would be ahead of it
                     }
                 } else {
                     ptx::tc_commit(&tfull[buf]);
                 }
             }
-            if (ok && !resolve_pending(true)) ok = false;
+            if (ok && !lora_flush(-1)) ok = false;
             if (!ok && any) {  // wait for the MMAs in flight before TMEM is freed
                 ptx::tc_commit(drain);
                 drain_wait(drain, 0);
@@ -429,61 +462,62 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
         }
     } else if (warp == 2) {
         // ------------------------------------------------------------ B stager
-        // stages B for every segment that ends in an epilogue (kb0 == 0)
+        // for every segment that ends in an epilogue (kb0 == 0): the B slices of the
+        // adapters of its token block, in phases of at most n_slots adapters; a phase
+        // waits for bempty (the MMAs of the previous phase are done)
         if (lane == 0 && p.lora) {
             ptx::tma_prefetch_desc(&tmB);
             const int n_valid = p.counts[0];
             const int n_active = p.counts[1];
-            int j = 0, slots_tb = -1, nslots = 0;
-            uint32_t bytes = 0;
+            int j = 0, slots_tb = -1, nact = 0;
             bool pending = false;
             uint32_t pending_phase = 0;
-            for (long long u = u_begin; u < u_end;) {
+            bool ok = true;
+            for (long long u = u_begin; u < u_end && ok;) {
                 const Seg sg = seg_at(u, u_end, KB);
                 u += sg.kb1 - sg.kb0;
                 if (sg.kb0 != 0) continue;  // partial accumulators only: no epilogue here
                 const int nb = sg.tile / p.n_tb, tb = sg.tile - nb * p.n_tb;
-                if (!wait_bounded(bempty, (uint32_t)((j & 1) ^ 1), abort_flag, p.status, 0x8u)) break;
-                if (tb != slots_tb) {
-                    // the adapters of this token block (kept while the block does not change)
-                    slots_tb = tb;
-                    const int p0 = tb * p.BN;
-                    const int p1 = min(min(p.M, p0 + p.BN), n_valid);
-                    int s = 0;  // first active segment that ends after p0
-                    {
-                        int lo = 0, hi = n_active;
+                for (int ph = 0;; ++ph) {
+                    if (!(ok = wait_bounded(bempty, (uint32_t)((j & 1) ^ 1), abort_flag, p.status, 0x8u))) break;
+                    if (ph == 0 && tb != slots_tb) {
+                        // the adapters of this token block (kept while the block does not change)
+                        slots_tb = tb;
+                        const int p0 = tb * p.BN;
+                        const int p1 = min(min(p.M, p0 + p.BN), n_valid);
+                        int lo = 0, hi = n_active;  // first active segment that ends after p0
                         while (lo < hi) {
                             const int mid = (lo + hi) >> 1;
                             if (p.indptr[p.active[mid] + 1] > p0) hi = mid; else lo = mid + 1;
                         }
-                        s = lo;
+                        nact = 0;
+                        for (int s2 = lo; s2 < n_active && nact < p.v_adapters; ++s2) {
+                            const int a = p.active[s2];
+                            if (p.indptr[a] >= p1) break;
+                            int r = p.ranks ? p.ranks[a] : p.r_max;
+                            r = max(1, min(r, p.r_max));
+                            s_slot_rank[nact] = r;
+                            s_lq[nact] = make_int4(max(p.indptr[a], p0) - p0, min(p.indptr[a + 1], p1) - p0, 0, 0);
+                            s_slot_adapter[nact++] = a;
+                        }
+                        s_nact = nact;
                     }
-                    nslots = 0;
-                    bytes = 0;
-                    for (int s2 = s; s2 < n_active && nslots < p.n_slots; ++s2) {
-                        const int a = p.active[s2];
-                        if (p.indptr[a] >= p1) break;
-                        int r = p.ranks ? p.ranks[a] : p.r_max;
-                        r = max(1, min(r, p.r_max));
-                        bytes += (uint32_t)(((r + 7) >> 3) * 8 * 256);
-                        s_slot_rank[nslots] = r;
-                        s_lq[nslots] = make_int4(max(p.indptr[a], p0) - p0, min(p.indptr[a + 1], p1) - p0, 0, 0);
-                        s_slot_adapter[nslots++] = a;
+                    const int e0 = ph * p.n_slots, e1 = min(nact, e0 + p.n_slots);
+                    uint32_t bytes = 0;
+                    for (int e = e0; e < e1; ++e) bytes += (uint32_t)(((s_slot_rank[e] + 7) >> 3) * 2048);
+                    if (bytes) ptx::mbar_arrive_expect_tx(bfull, bytes);
+                    for (int e = e0; e < e1; ++e) {
+                        const int a = s_slot_adapter[e];
+                        const uint32_t dst = smem_u + p.slots_off + (uint32_t)((e - e0) * p.r16 * 256);
+                        for (int rb = 0; rb < ((s_slot_rank[e] + 7) >> 3); ++rb)
+                            ptx::tma_load_2d(dst + rb * 2048, &tmB, bfull, nb * kBlockM, a * p.r_max + rb * 8);
                     }
-                    s_nslots = nslots;
+                    if (!bytes) ptx::mbar_arrive(bfull);
+                    pending = true;
+                    pending_phase = (uint32_t)(j & 1);
+                    ++j;
+                    if (e1 >= nact) break;  // the segment's last phase
                 }
-                if (bytes) ptx::mbar_arrive_expect_tx(bfull, bytes);
-                for (int q = 0; q < nslots; ++q) {
-                    const int a = s_slot_adapter[q];
-                    const int r = s_slot_rank[q];
-                    const uint32_t dst = smem_u + p.slots_off + (uint32_t)(q * p.r16 * 256);
-                    for (int rb = 0; rb < ((r + 7) >> 3); ++rb)
-                        ptx::tma_load_2d(dst + rb * 2048, &tmB, bfull, nb * kBlockM, a * p.r_max + rb * 8);
-                }
-                if (!bytes) ptx::mbar_arrive(bfull);
-                pending = true;
-                pending_phase = (uint32_t)(j & 1);
-                ++j;
             }
             if (*abort_flag && pending) drain_wait(bfull, pending_phase);
         }
@@ -590,7 +624,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
         }
 
         // ---- epilogues of this CTA's segments
-        int i = 0, jb = 0, staged_tb = -1, slotted_tb = -1;
+        int i = 0, jf = 0, staged_tb = -1, slotted_tb = -1;
         bool v_ready = !p.lora;
         for (long long u = u_begin; u < u_end && ok; ++i) {
             const Seg sg = seg_at(u, u_end, KB);
@@ -656,17 +690,19 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
                 if (!(ok = epi_sync())) break;
                 staged_tb = tb;
             }
-            // the LoRA operands of this segment first: the MMA warp adds them to the
-            // accumulator before it signals tfull
-            if (p.lora && !(ok = wait_bounded(bfull, (uint32_t)(jb & 1), abort_flag, p.status, 0x20u))) break;
-            if (p.lora) {
-                const int nsl = s_nslots;
-                if (slotted_tb != tb) {
-                    // per token: its slot (-2: adapter not staged, done on CUDA cores below);
-                    // per slot q: V'_q[t][j] = s_q v[t][j] / sx[t] for its tokens t (zero for the
-                    // other tokens of its 16-aligned column range), K-major bf16. Each thread owns
-                    // at most one token (BN <= 256): it loads that token's v row first, so the
-                    // whole build waits for one round trip to memory, not one per slot
+            // the LoRA operands of this segment, phase by phase: the MMA warp adds each
+            // phase to the accumulator (between its k-blocks) and signals tfull after the last
+            for (int ph = 0; p.lora && ok; ++ph) {
+                if (!(ok = wait_bounded(bfull, (uint32_t)(jf & 1), abort_flag, p.status, 0x20u))) break;
+                ++jf;
+                const int nact = s_nact;
+                const int e0 = ph * p.n_slots, e1 = min(nact, e0 + p.n_slots);
+                if (ph == 0 && slotted_tb != tb) {
+                    // per token: its entry in the block's adapter list (-2: past the list, done on
+                    // CUDA cores below); per entry e: V'_e[t][j] = s_a v[t][j] / sx[t] for its
+                    // tokens t (zero for the other tokens of its 16-aligned column range), K-major
+                    // bf16, for every phase of every segment of this token block. Each token's
+                    // v row is loaded first, so the build waits for one round trip to memory
                     // lane (token pl, copy cp): v_rep consecutive lanes load the copies of one
                     // token's v row and sum them with shuffles (BN * v_rep <= 256)
                     const int pl = etid >> p.lg_rep, cp = etid & (p.v_rep - 1);
@@ -680,7 +716,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
                         const int a = s_a[pl];
                         if (a >= 0) {
                             q_own = -2;
-                            for (int t = 0; t < nsl; ++t)
+                            for (int t = 0; t < nact; ++t)
                                 if (s_slot_adapter[t] == a) { q_own = t; break; }
                         }
                         if (cp == 0) s_q[pl] = q_own;
@@ -692,7 +728,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
                     }
                     // zero every slot's tile and publish its byte offset
                     int off = 0;
-                    for (int q = 0; q < nsl; ++q) {
+                    for (int q = 0; q < nact; ++q) {
                         const int4 lq = s_lq[q];
                         const int w = ((lq.y + 15) & ~15) - (lq.x & ~15);
                         if (etid == 0) s_lq[q].z = off;
@@ -750,40 +786,49 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
                     }
                     slotted_tb = tb;
                 }
-                // B'_q[n][j] = B_q[j][n] / sw[n] in place, K-major: every thread first reads
-                // its (n, slot) columns, then (after a barrier) writes them transposed
-                const float inv_sw2 = (nb * kBlockM + (etid & 127) < p.N) ? 1.f / p.sw[nb * kBlockM + (etid & 127)] : 0.f;
-                for (int q0 = 0; q0 < nsl && ok; q0 += 2) {
-                    const int q = q0 + (etid >> 7), nn = etid & 127;
-                    float col[MAXR];
-                    const bool act = q < nsl;
-                    const int r = act ? s_slot_rank[q] : 0;
-                    const uint16_t* raw = reinterpret_cast<const uint16_t*>(slots + (size_t)(act ? q : 0) * p.r16 * 256) + nn;
+                // B'[n][j] = B_a[j][n] / sw[n] in place, K-major, for the phase's slots: each
+                // thread reads its row n of kSpt slots, then (after a barrier) writes them
+                const int nn = etid & 127, half = etid >> 7;
+                const float inv_sw2 = (nb * kBlockM + nn < p.N) ? 1.f / p.sw[nb * kBlockM + nn] : 0.f;
+                const int nbuf = e1 - e0;
+                constexpr int kSpt = MAXR <= 16 ? 4 : (MAXR <= 32 ? 2 : 1);
+                for (int b0 = 0; b0 < nbuf && ok; b0 += 2 * kSpt) {
+                    uint32_t colw[kSpt][MAXR / 2];
 #pragma unroll
-                    for (int j = 0; j < MAXR; ++j)
-                        col[j] = (j < r) ? __uint_as_float((uint32_t)raw[j * 128] << 16) * inv_sw2 : 0.f;
+                    for (int t = 0; t < kSpt; ++t) {
+                        const int b = b0 + 2 * t + half;
+                        const int r = b < nbuf ? s_slot_rank[e0 + b] : 0;
+                        const uint16_t* raw = reinterpret_cast<const uint16_t*>(slots + (size_t)(b < nbuf ? b : 0) * p.r16 * 256) + nn;
+#pragma unroll
+                        for (int j = 0; j < MAXR; j += 2) {
+                            const float c0 = j < r ? __uint_as_float((uint32_t)raw[j * 128] << 16) * inv_sw2 : 0.f;
+                            const float c1 = j + 1 < r ? __uint_as_float((uint32_t)raw[(j + 1) * 128] << 16) * inv_sw2 : 0.f;
+                            __nv_bfloat162 hv = __floats2bfloat162_rn(c0, c1);
+                            colw[t][j >> 1] = *reinterpret_cast<uint32_t*>(&hv);
+                        }
+                    }
                     if (!(ok = epi_sync())) break;
-                    if (act) {
-                        uint8_t* dst = slots + (size_t)q * p.r16 * 256;
+#pragma unroll
+                    for (int t = 0; t < kSpt; ++t) {
+                        const int b = b0 + 2 * t + half;
+                        if (b >= nbuf) continue;
+                        uint8_t* dst = slots + (size_t)b * p.r16 * 256;
 #pragma unroll
                         for (int kg = 0; kg < MAXR / 8; ++kg) {
                             if (kg >= kgq) break;
-                            uint32_t wv[4];
-#pragma unroll
-                            for (int h = 0; h < 4; ++h) {
-                                __nv_bfloat162 hv = __floats2bfloat162_rn(col[kg * 8 + 2 * h], col[kg * 8 + 2 * h + 1]);
-                                wv[h] = *reinterpret_cast<uint32_t*>(&hv);
-                            }
-                            *reinterpret_cast<uint4*>(dst + kmajor_off(nn, kg, kgq)) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+                            *reinterpret_cast<uint4*>(dst + kmajor_off(nn, kg, kgq)) =
+                                make_uint4(colw[t][4 * kg], colw[t][4 * kg + 1], colw[t][4 * kg + 2], colw[t][4 * kg + 3]);
                         }
                     }
-                    // the next pair reads other slots: no barrier before it
+                    // the next round reads other slots: no barrier before it
                 }
                 if (!ok) break;
                 ptx::fence_proxy_async_smem();  // generic writes, read by the tensor core (async proxy)
                 if (!(ok = epi_sync())) break;
                 if (etid == 0) ptx::mbar_arrive(lready);
+                if (e1 >= nact) break;  // the segment's last phase
             }
+            if (!ok) break;
             if (!(ok = wait_bounded(&tfull[buf], (uint32_t)((i >> 1) & 1), abort_flag, p.status, 0x10u))) break;
             ptx::tc_fence_after();
             // the CTAs after this one that hold later k-blocks of this tile
@@ -918,9 +963,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
             __syncwarp();
             if (lane == 0) {
                 ptx::mbar_arrive(&tempty[buf]);
-                if (p.lora) ptx::mbar_arrive(bempty);
             }
-            ++jb;
         }
     }
 
@@ -1051,35 +1094,61 @@ cudaError_t launch_fp8_gemm(const Fp8GemmArgs& a, cudaStream_t stream)
     const size_t bars = 8 * (2 * kMaxStages + 9);
     // a slot holds one adapter's B[j][128 n] as loaded, then B'[128 n][r16] in place
     const size_t slot_bytes = (size_t)p.r16 * 256;
-    // V' tiles: each staged adapter's 16-aligned token range, r16 bf16 per token
-    auto vq_bytes = [&](int nslots) -> size_t {
-        return a.lora ? align_up(((size_t)p.BN + 32 * (size_t)nslots) * p.r16 * 2, 128) : 0;
+    // V' tiles of va adapters: their token ranges are disjoint and contiguous, so their
+    // 16-aligned windows cover at most BN + 16 (va - 1) token rows of r16 bf16
+    auto vq_bytes = [&](int va) -> size_t {
+        return (a.lora && va > 0) ? align_up(((size_t)p.BN + 16 * (size_t)(va - 1)) * p.r16 * 2, 128) : 0;
     };
-    int want_slots = a.lora ? (a.n_adapters < p.BN ? a.n_adapters : p.BN) : 0;
-    if (want_slots > 256) want_slots = 256;
-    auto fit = [&](int bk, int nslots) -> int {
+    auto fit = [&](int bk, int va, int ns) -> int {
         const size_t stage_bytes = (size_t)kBlockM * bk + (size_t)p.BN * bk;
-        const size_t fixed = 1024 + meta + vq_bytes(nslots) + bars + (size_t)nslots * slot_bytes;
+        const size_t fixed = 1024 + meta + vq_bytes(va) + bars + (size_t)ns * slot_bytes;
         if (fixed >= kSmemMax) return 0;
         const size_t st = (kSmemMax - fixed) / stage_bytes;
         return (int)(st > (size_t)kMaxStages ? kMaxStages : st);
     };
-    // prefer 128-byte k-blocks, then 64-byte ones, with every adapter's B staged
-    // and >= 4 stages; then give up staging slots; then accept 2 stages
-    int BK = 128, slots = want_slots, stages = fit(128, want_slots);
-    if (stages < 4) { BK = 64; stages = fit(64, want_slots); }
-    while (stages < 4 && slots > 0) stages = fit(64, --slots);
-    if (stages < 4) stages = fit(64, 0);
+    // Every adapter of a token block gets a V' tile when they fit (va); their B slices
+    // pass through ns slots, in phases of ns adapters. Preference: 128-byte k-blocks with
+    // >= 4 stages, then with 3 (a tile of 256 tokens), then 64-byte k-blocks; within
+    // each, as many slots as fit; fewer V' tiles only as a last resort.
+    int want_va = a.lora ? (a.n_adapters < p.BN ? a.n_adapters : p.BN) : 0;
+    if (want_va > 256) want_va = 256;
+    int BK = 0, va = 0, ns = 0, stages = 0;
+    if (!a.lora) {
+        BK = 128;
+        stages = fit(128, 0, 0);
+    } else {
+        // a phase costs a few microseconds of latency (load, transform, MMAs): keep at
+        // least 4 slots (or one per adapter) so that a segment needs few phases
+        const int tries[3][2] = {{128, 4}, {128, 3}, {64, 4}};
+        for (int v = want_va; v >= 1 && !BK; v = v > 1 ? (v + 1) / 2 : 0) {
+            for (int t = 0; t < 3 && !BK; ++t) {
+                const int bk = tries[t][0], min_st = tries[t][1];
+                int n = v;
+                while (n >= 1 && fit(bk, v, n) < min_st) --n;
+                if (n >= (v < 4 ? v : 4)) {
+                    BK = bk;
+                    va = v;
+                    ns = n;
+                    stages = fit(bk, v, n);
+                }
+            }
+        }
+        if (!BK) {  // no tensor-core slots at all: every adapter on CUDA cores
+            BK = 64;
+            stages = fit(64, 0, 0);
+        }
+    }
     if (stages < 2) return cudaErrorInvalidConfiguration;
     p.stages = stages;
-    p.n_slots = slots;
+    p.n_slots = ns;
+    p.v_adapters = va;
     p.k_blocks = (a.K + BK - 1) / BK;
     p.units = (long long)p.num_tiles * p.k_blocks;
     const size_t stage_bytes = (size_t)kBlockM * BK + (size_t)p.BN * BK;
     p.ring_off = 0;
     p.slots_off = (uint32_t)align_up((size_t)stages * stage_bytes, 1024);
-    p.v_off = (uint32_t)align_up(p.slots_off + (size_t)slots * slot_bytes, 128);
-    p.meta_off = (uint32_t)(p.v_off + vq_bytes(slots));
+    p.v_off = (uint32_t)align_up(p.slots_off + (size_t)ns * slot_bytes, 128);
+    p.meta_off = (uint32_t)(p.v_off + vq_bytes(va));
     p.bar_off = (uint32_t)align_up(p.meta_off + meta, 8);
     const size_t smem = align_up(p.bar_off + bars, 128) + 1024;  // + alignment slack
 
