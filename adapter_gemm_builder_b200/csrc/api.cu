@@ -89,6 +89,12 @@ int lora_version(void) { return kVersion; }
 
 int lora_tile_tokens(void) { return LORA_TILE_TOKENS; }
 
+int lora_tile_tokens_for(int T, int n_adapters)
+{
+    if (T < 0 || n_adapters < 1) return -1;
+    return tile_tokens_for(T, n_adapters);
+}
+
 int lora_max_tiles(int T, int n_adapters)
 {
     if (T < 0 || n_adapters < 1) return -1;
@@ -108,7 +114,8 @@ int lora_segments_status(const lora_segments_t* seg, lora_stream_t stream, uint3
     if (word) {
         e = cudaMemsetAsync(dev, 0, sizeof(int32_t), (cudaStream_t)stream);
         if (e == cudaSuccess) e = cudaStreamSynchronize((cudaStream_t)stream);
-        return e == cudaSuccess ? LORA_ERR_TIMEOUT : LORA_ERR_CUDA;
+        if (e != cudaSuccess) return LORA_ERR_CUDA;
+        return (word & kSegTooLarge) ? LORA_ERR_INVALID_ARG : LORA_ERR_TIMEOUT;
     }
     return LORA_OK;
 }

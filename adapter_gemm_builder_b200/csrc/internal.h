@@ -65,6 +65,8 @@ int device_sm_count();
 
 // Rows of lora_segments_t.tiles for T tokens over n_adapters.
 int max_tiles_for(int T, int n_adapters);
+// tokens per tile for a batch (LORA_DECODE_TILE_TOKENS for decode-like batches)
+int tile_tokens_for(int T, int n_adapters);
 
 // 2-D tiled tensor map (inner dimension contiguous); false on failure.
 bool encode_tmap_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner,
@@ -78,5 +80,7 @@ bool encode_tmap_3d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, co
 
 // Slot of the device status word in lora_segments_t.counts.
 constexpr int kSegStatusSlot = 4;
+// status bit: a tile held more tokens than the segments' tile size allows
+constexpr int kSegTooLarge = 0x1000;
 
 }  // namespace lora

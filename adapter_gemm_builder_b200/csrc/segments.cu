@@ -24,7 +24,6 @@ namespace lora {
 namespace {
 
 constexpr int kMaxThreads = 1024;
-constexpr int kTile = LORA_TILE_TOKENS;
 
 // Exclusive block-wide scan of one 64-bit value per thread (any blockDim that
 // is a multiple of 32); *total receives the sum. Ends with __syncthreads.
@@ -64,6 +63,7 @@ struct SegOut {
     int32_t* tiles;
     int32_t* tok_adapter;
     int32_t* counts;
+    int tile_t;  // tokens per tile (tile_tokens_for)
 };
 
 // Given per-bin counts hist[0..nb) in shared memory (nb = n_adapters + 1),
@@ -89,7 +89,7 @@ __device__ void finish_tables(const int32_t* hist, int32_t* starts, int n_adapte
     const int ca0 = min(n_adapters, c0), ca1 = min(n_adapters, c1);
     long long pk = 0;
     for (int a = ca0; a < ca1; ++a)
-        if (hist[a] > 0) pk += (1ll << 32) + (hist[a] + kTile - 1) / kTile;
+        if (hist[a] > 0) pk += (1ll << 32) + (hist[a] + o.tile_t - 1) / o.tile_t;
     const long long pbase = block_exclusive_scan(pk, &s_total);
     int pos = (int)(pbase >> 32);
     int tile = (int)(pbase & 0xffffffffll);
@@ -97,9 +97,9 @@ __device__ void finish_tables(const int32_t* hist, int32_t* starts, int n_adapte
         const int c = hist[a];
         if (c > 0) {
             o.active[pos] = a;
-            for (int off = 0; off < c; off += kTile, ++tile)
+            for (int off = 0; off < c; off += o.tile_t, ++tile)
                 reinterpret_cast<int4*>(o.tiles)[tile] =
-                    make_int4(a, starts[a] + off, min(kTile, c - off), pos);
+                    make_int4(a, starts[a] + off, min(o.tile_t, c - off), pos);
             ++pos;
         }
     }
@@ -223,15 +223,22 @@ segments_large_kernel(const int32_t* __restrict__ ids, int T, int n_adapters, in
 
 }  // namespace
 
+int tile_tokens_for(int T, int n_adapters)
+{
+    return (T <= LORA_DECODE_MAX_TOKENS && T <= 2 * n_adapters) ? LORA_DECODE_TILE_TOKENS : LORA_TILE_TOKENS;
+}
+
 int max_tiles_for(int T, int n_adapters)
 {
-    return (n_adapters < T ? n_adapters : T) + (T + kTile - 1) / kTile;
+    const long long t = tile_tokens_for(T, n_adapters);
+    const long long m = n_adapters < T ? n_adapters : T;
+    return (int)(((long long)T + (t - 1) * m) / t);
 }
 
 cudaError_t launch_build_segments(const int32_t* ids, int T, int n_adapters,
                                   const lora_segments_t& seg, cudaStream_t stream)
 {
-    SegOut o{seg.perm, seg.indptr, seg.active, seg.tiles, seg.tok_adapter, seg.counts};
+    SegOut o{seg.perm, seg.indptr, seg.active, seg.tiles, seg.tok_adapter, seg.counts, tile_tokens_for(T, n_adapters)};
     const int nb = n_adapters + 1;
     const int mt = max_tiles_for(T, n_adapters);
     const int threads_small = T <= 64 ? 64 : (T + 31) / 32 * 32;

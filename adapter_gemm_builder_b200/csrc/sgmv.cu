@@ -179,7 +179,10 @@ __device__ bool wait_all(uint64_t* bar, uint32_t parity, volatile int* abort_fla
     return ok;
 }
 
-template <int MODE>
+// kSmallOnly: every tile holds <= kSmallTile tokens (the tiles of a decode-like
+// batch), so the tensor-core path for larger tiles is left out of this variant:
+// a smaller kernel, whose dependent steps wait less on instruction fetch.
+template <int MODE, bool kSmallOnly>
 __global__ void __launch_bounds__(kThreads, 2)
 sgmv_kernel(const __grid_constant__ AMaps am, const SgmvParams p)
 {
@@ -233,7 +236,11 @@ sgmv_kernel(const __grid_constant__ AMaps am, const SgmvParams p)
     r = max(1, min(r, p.r_max));
     const float scale = p.scales ? p.scales[a] : 1.0f;
     const int r8 = round_up(r, 8), r16 = round_up(r, 16);
-    const bool small = nt <= kSmallTile;
+    if (kSmallOnly && nt > kSmallTile) {  // segments not built for this batch size: the
+        if (tid == 0 && rank == 0) atomicOr(status, kSegTooLarge);  // whole cluster leaves
+        return;
+    }
+    const bool small = kSmallOnly || nt <= kSmallTile;
     const int Mt = (nt + 15) >> 4;
     const int Mtr = small ? nt : Mt * 16;  // x / y rows held per stage (tail rows zero)
     if (tid < nt) s_tok[tid] = p.perm[tok0 + tid];
@@ -772,10 +779,10 @@ sgmv_kernel(const __grid_constant__ AMaps am, const SgmvParams p)
 #undef SACC
 #undef ACC
 
-template <int MODE>
+template <int MODE, bool kSmallOnly>
 cudaError_t launch_mode(const AMaps& am, const SgmvParams& p, dim3 grid, int C, size_t smem, cudaStream_t stream)
 {
-    auto kern = sgmv_kernel<MODE>;
+    auto kern = sgmv_kernel<MODE, kSmallOnly>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
@@ -812,7 +819,7 @@ size_t sgmv_smem_per_cta()
     cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev);
     cudaFuncAttributes fa;
     size_t stat = 1024;
-    if (cudaFuncGetAttributes(&fa, sgmv_kernel<SGMV_APPLY>) == cudaSuccess) stat = fa.sharedSizeBytes;
+    if (cudaFuncGetAttributes(&fa, sgmv_kernel<SGMV_APPLY, false>) == cudaSuccess) stat = fa.sharedSizeBytes;
     if (per_sm <= 0) per_sm = 233472;
     const size_t b = (size_t)per_sm / 2 - (size_t)reserved - stat;
     if (dev >= 0 && dev < 64) cached[dev] = b;
@@ -946,10 +953,18 @@ cudaError_t launch_sgmv(int mode, const void* x, int64_t x_slice_stride, const l
     }
 
     const dim3 grid((unsigned)(max_tiles_for(seg.T, pool.n_adapters) * C), (unsigned)pool.n_slices, 1);
+    // segments of a decode-like batch come in tiles of <= kSmallTile tokens
+    if (tile_tokens_for(seg.T, seg.n_adapters) <= kSmallTile) {
+        switch (mode) {
+        case SGMV_SHRINK: return launch_mode<SGMV_SHRINK, true>(am, p, grid, C, smem, stream);
+        case SGMV_EXPAND: return launch_mode<SGMV_EXPAND, true>(am, p, grid, C, smem, stream);
+        default: return launch_mode<SGMV_APPLY, true>(am, p, grid, C, smem, stream);
+        }
+    }
     switch (mode) {
-    case SGMV_SHRINK: return launch_mode<SGMV_SHRINK>(am, p, grid, C, smem, stream);
-    case SGMV_EXPAND: return launch_mode<SGMV_EXPAND>(am, p, grid, C, smem, stream);
-    default: return launch_mode<SGMV_APPLY>(am, p, grid, C, smem, stream);
+    case SGMV_SHRINK: return launch_mode<SGMV_SHRINK, false>(am, p, grid, C, smem, stream);
+    case SGMV_EXPAND: return launch_mode<SGMV_EXPAND, false>(am, p, grid, C, smem, stream);
+    default: return launch_mode<SGMV_APPLY, false>(am, p, grid, C, smem, stream);
     }
 }
 

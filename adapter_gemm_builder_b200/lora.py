@@ -32,7 +32,7 @@ LORA_OP_FP8_GEMM = 3
 EXPORTED = [
     "lora_workspace_size", "lora_workspace_init", "lora_workspace_status", "lora_build_segments",
     "lora_shrink", "lora_expand", "lora_apply", "fp8_quantize_rows", "fp8_gemm_lora_epilogue",
-    "lora_status_string", "lora_version", "lora_tile_tokens", "lora_max_tiles",
+    "lora_status_string", "lora_version", "lora_tile_tokens", "lora_tile_tokens_for", "lora_max_tiles",
     "lora_segments_status", "fp8_gemm_lora_epilogue_noalloc", "lora_noalloc_scratch_bytes",
 ]
 
@@ -90,6 +90,7 @@ def load(path: str = LIB_PATH):
             "lora_status_string": (ctypes.c_char_p, [I]),
             "lora_version": (I, []),
             "lora_tile_tokens": (I, []),
+            "lora_tile_tokens_for": (I, [I, I]),
             "lora_max_tiles": (I, [I, I]),
             "lora_segments_status": (I, [P, P, P]),
             "fp8_gemm_lora_epilogue_noalloc": (I, [P, I, I, I, P, P, P, P, P, P]),
@@ -123,9 +124,14 @@ def tile_tokens() -> int:
     return load().lora_tile_tokens()
 
 
+def tile_tokens_for(T: int, n_adapters: int) -> int:
+    """Tokens per row of Segments.tiles for this batch (lora_tile_tokens_for)."""
+    return load().lora_tile_tokens_for(T, n_adapters)
+
+
 def max_tiles(T: int, n_adapters: int) -> int:
-    """Rows of Segments.tiles (same formula as lora_max_tiles)."""
-    return min(n_adapters, T) + (T + 63) // 64
+    """Rows of Segments.tiles (lora_max_tiles)."""
+    return load().lora_max_tiles(T, n_adapters)
 
 
 class Pool:

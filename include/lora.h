@@ -65,6 +65,8 @@ typedef enum {
 
 /* Implemented limits. */
 #define LORA_TILE_TOKENS 64    /* tokens per work tile of one adapter segment */
+#define LORA_DECODE_TILE_TOKENS 4  /* the same in a decode-like batch (lora_tile_tokens_for) */
+#define LORA_DECODE_MAX_TOKENS 64  /* largest batch that can count as decode-like */
 #define LORA_MAX_RANK 64       /* largest r_max */
 #define LORA_MAX_ADAPTERS 16384
 
@@ -101,7 +103,8 @@ typedef struct {
  *               indptr[n_adapters] = number of tokens with an adapter.
  *   active      int32 [n_adapters]: ids with >= 1 token, ascending; -1 after n_active.
  *   tiles       int32 [lora_max_tiles(T, n_adapters)][4]: every active segment
- *               cut, in order, into runs of at most LORA_TILE_TOKENS tokens:
+ *               cut, in order, into runs of at most
+ *               lora_tile_tokens_for(T, n_adapters) tokens:
  *               {adapter, first position in perm, token count, segment index};
  *               the rows after the last run are {-1, 0, 0, -1}. One row is one
  *               unit of work of the SGMV kernels.
@@ -125,9 +128,11 @@ typedef struct {
 /*
  * Read and clear the status word of a segments object (counts[4]):
  * synchronises `stream`; LORA_OK, or LORA_ERR_TIMEOUT if an SGMV kernel that
- * used these segments gave up on a bounded wait (its output is then
- * undefined). *detail (host, may be NULL) receives the raw word. The word is
- * also cleared by every lora_build_segments on the same object.
+ * used these segments gave up on a bounded wait, or LORA_ERR_INVALID_ARG if a
+ * tile held more tokens than lora_tile_tokens_for(T, n_adapters) allows (the
+ * tiles were not built by lora_build_segments for these sizes); the output is
+ * then undefined. *detail (host, may be NULL) receives the raw word. The word
+ * is also cleared by every lora_build_segments on the same object.
  */
 LORA_API int lora_segments_status(const lora_segments_t* seg, lora_stream_t stream, uint32_t* detail);
 
@@ -268,12 +273,22 @@ LORA_API size_t lora_noalloc_scratch_bytes(void);
 /* Static string for a status code. */
 LORA_API const char* lora_status_string(int status);
 
-/* Library version, and the tile size kernels assume for lora_segments_t.tiles. */
+/* Library version, and the largest tile size (LORA_TILE_TOKENS). */
 LORA_API int lora_version(void);
 LORA_API int lora_tile_tokens(void);
 
+/* Tokens per row of lora_segments_t.tiles for a batch of T tokens over
+ * n_adapters: LORA_DECODE_TILE_TOKENS when the batch is decode-like
+ * (T <= LORA_DECODE_MAX_TOKENS and T <= 2 * n_adapters, so most adapters hold
+ * one or two tokens; the SGMV kernels then run a variant built for tiles that
+ * small), else LORA_TILE_TOKENS. -1 for invalid arguments (T < 0,
+ * n_adapters < 1). */
+LORA_API int lora_tile_tokens_for(int T, int n_adapters);
+
 /* Rows of lora_segments_t.tiles for a batch of T tokens over n_adapters:
- * min(n_adapters, T) + ceil(T / LORA_TILE_TOKENS); -1 for invalid arguments. */
+ * floor((T + (t - 1) * min(n_adapters, T)) / t) with
+ * t = lora_tile_tokens_for(T, n_adapters) (an adapter with c tokens takes
+ * ceil(c / t) <= (c + t - 1) / t rows); -1 for invalid arguments. */
 LORA_API int lora_max_tiles(int T, int n_adapters);
 
 #ifdef __cplusplus

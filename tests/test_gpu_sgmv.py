@@ -16,7 +16,6 @@ from gpu_util import (TOL_BF16, DeviceProblem, assert_close, dev, dev_bf16, f64,
                       oracle_apply, rne_bf16_bits)
 
 pytestmark = pytest.mark.gpu
-TT = 64
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -34,13 +33,18 @@ def _check_segments(ids, n_adapters):
     L.lora_build_segments(dev(ids) if T else torch.empty(0, dtype=torch.int32, device="cuda"),
                           n_adapters, seg)
     torch.cuda.synchronize()
-    want = oracle.build_segments(ids, n_adapters, TT)
+    want = oracle.build_segments(ids, n_adapters, L.tile_tokens_for(T, n_adapters))
     counts = seg.counts.cpu().numpy()
     assert counts[:4].tolist() == want["counts"].tolist()
     assert counts[4:].tolist() == [0, 0, 0, 0]
     assert seg.indptr.cpu().numpy().tolist() == want["indptr"].tolist()
     assert seg.active.cpu().numpy().tolist() == want["active"].tolist()
-    assert seg.tiles.cpu().numpy()[:len(want["tiles"])].tolist() == want["tiles"].tolist()
+    # the tile rows themselves, then padding rows (the two arrays are sized by bounds
+    # of their own)
+    n_tiles = int(want["counts"][3])
+    got_tiles = seg.tiles.cpu().numpy()
+    assert got_tiles[:n_tiles].tolist() == want["tiles"][:n_tiles].tolist()
+    assert all(row == [-1, 0, 0, -1] for row in got_tiles[n_tiles:L.max_tiles(T, n_adapters)].tolist())
     if T:
         assert seg.perm.cpu().numpy()[:T].tolist() == want["perm"].tolist()
         assert seg.tok_adapter.cpu().numpy()[:T].tolist() == want["tok_adapter"].tolist()
@@ -98,6 +102,10 @@ SMALL_CASES = {
                          rank_choices=(16,), kind="uniform"),
     "rank8_pool": dict(seed=18, T=33, n_adapters=4, h_in=256, h_out=136, r_max=8,
                        rank_choices=(3, 8)),
+    # decode-like (T <= 64, T <= 2 n): 4-token tiles on the decode kernel, several tiles
+    # for the adapters with more tokens, mixed ranks and a ragged h_out
+    "decode_zipf": dict(seed=19, T=48, n_adapters=32, kind="zipf", h_in=1024, h_out=520,
+                        r_max=32, rank_choices=(1, 8, 16, 32)),
 }
 
 

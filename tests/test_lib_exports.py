@@ -5,6 +5,8 @@ import ctypes
 import os
 import re
 
+import numpy as np
+
 import pytest
 
 from adapter_gemm_builder_b200 import build as lbuild
@@ -46,8 +48,16 @@ def test_library_is_sm100a_only():
 def test_version_and_constants(lib):
     assert lib.lora_version() >= 1
     assert lib.lora_tile_tokens() == 64
-    assert lib.lora_max_tiles(36, 32) == 32 + 1
-    assert lib.lora_max_tiles(512, 256) == 256 + 8
+    # decode-like batches (T <= 64 and T <= 2 * n_adapters) get 4-token tiles
+    assert lib.lora_tile_tokens_for(36, 32) == 4
+    assert lib.lora_tile_tokens_for(64, 32) == 4
+    assert lib.lora_tile_tokens_for(1, 1) == 4
+    assert lib.lora_tile_tokens_for(64, 4) == 64
+    assert lib.lora_tile_tokens_for(65, 1000) == 64
+    assert lib.lora_tile_tokens_for(-1, 4) == -1 and lib.lora_tile_tokens_for(4, 0) == -1
+    # floor((T + (t - 1) * min(n, T)) / t)
+    assert lib.lora_max_tiles(36, 32) == (36 + 3 * 32) // 4
+    assert lib.lora_max_tiles(512, 256) == (512 + 63 * 256) // 64
     assert lib.lora_max_tiles(-1, 4) == -1
     assert lib.lora_status_string(L.LORA_ERR_TIMEOUT).decode()
 
@@ -156,3 +166,20 @@ def test_binding_fails_loudly_without_library(tmp_path):
             L.load(missing)
     finally:
         L._lib = saved
+
+
+def test_max_tiles_bounds_every_id_mix(lib):
+    """The tile-row bound holds for the worst cases of the tile rule: every adapter
+    one token more than a multiple of the tile size, all tokens on one adapter,
+    and random mixes (tiles counted by the oracle's builder)."""
+    import oracle
+    rng = np.random.default_rng(7)
+    cases = [(36, 32), (64, 32), (48, 24), (5, 2), (64, 4), (300, 7), (1000, 999), (130, 64)]
+    for T, n in cases:
+        t = lib.lora_tile_tokens_for(T, n)
+        bound = lib.lora_max_tiles(T, n)
+        mixes = [rng.integers(0, n, T), np.zeros(T, np.int64), np.arange(T) % n,
+                 np.repeat(np.arange(n), t + 1)[:T]]
+        for ids in mixes:
+            seg = oracle.build_segments(ids.astype(np.int32), n, t)
+            assert seg["counts"][3] <= bound, (T, n, t)
