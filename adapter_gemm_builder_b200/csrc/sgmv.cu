@@ -303,6 +303,15 @@ sgmv_kernel(const __grid_constant__ AMaps am, const SgmvParams p)
         ptx::mbar_arrive_expect_tx(red1, (uint32_t)((one_phase ? C * nt : C * mine) * r8 * 4));
         ptx::mbar_arrive_expect_tx(red2, one_phase ? 0u : (uint32_t)(nt * r8 * 4));
     }
+    // a decode tile's first A block is one contiguous copy that needs nothing but the
+    // geometry: the producer's lane 0 issues it now, ahead of the barrier (its bytes
+    // join stage 0's count; the item-0 pass below leaves it out)
+    const bool a_early = small && !a_tma && nK > 0;
+    if (a_early && warp == kComputeWarps && lane == 0) {
+        const uint32_t bytes = (uint32_t)(min(BK, k_len) * apitch);
+        ptx::mbar_expect_tx(&full[0], bytes);
+        ptx::bulk_g2s(base_u, Ag + (size_t)k_begin * p.r_max, bytes, &full[0]);
+    }
     __syncwarp();
     __syncthreads();
 
@@ -331,8 +340,9 @@ sgmv_kernel(const __grid_constant__ AMaps am, const SgmvParams p)
                 const int kb = min(BK, k_begin + k_len - k0);
                 const int nbox = (kb + 63) >> 6;  // 64-row boxes; rows past h_in read as zero
                 const uint32_t xb = base + (uint32_t)(BK * apitch);
+                const bool a_done = a_early && it == 0;  // issued with the geometry
                 if (lane == 0) {
-                    uint32_t bytes = a_tma ? (uint32_t)(nbox * 64 * apitch) : (uint32_t)(kb * apitch);
+                    uint32_t bytes = a_done ? 0u : (a_tma ? (uint32_t)(nbox * 64 * apitch) : (uint32_t)(kb * apitch));
                     if (small) bytes += (uint32_t)(nt * kb * 2);
                     else if (contig) bytes += (uint32_t)(nbox * Mt * 16 * 128);
                     ptx::mbar_arrive_expect_tx(&full[st], bytes);
@@ -340,7 +350,7 @@ sgmv_kernel(const __grid_constant__ AMaps am, const SgmvParams p)
                 __syncwarp();
                 // one copy instruction per lane (a copy costs ~150 ns of issue to its thread):
                 // lanes 0..nA-1 the A boxes (or the one A bulk copy), then the x boxes or rows
-                const int nA = a_tma ? nbox : 1;
+                const int nA = a_done ? 0 : (a_tma ? nbox : 1);
                 if (lane < nA) {
                     if (a_tma)
                         ptx::tma_load_3d(base + (uint32_t)(lane * 64 * apitch), &am.m[a_map], &full[st], 0,
