@@ -432,8 +432,11 @@ sgmv_kernel(const __grid_constant__ AMaps am, const SgmvParams p)
         const uint32_t vf_u = base_u + p.off_vf, rb_u = base_u + p.off_rb;
         const uint32_t red1_u = ptx::smem_u32(red1), red2_u = ptx::smem_u32(red2);
 
-        // small tiles: thread owns 8 columns (chunk c) of A over rows k = rg, rg + rstride, ...;
-        // chunks per row are padded to a power of two (ncbp) so a warp reduces by shuffles
+        // small tiles, chunks of 8 columns per token padded to a power of two (ncbp).
+        // Decode variant: warp w owns the (token, chunk) pairs w, w + 8, ... and its lanes
+        // stride over the rows (SACC(i, e): column e of its i-th pair), so no reduction
+        // across warps is needed. Otherwise: thread (c_own, rg) owns chunk c_own over rows
+        // rg, rg + rstride, ... for every token (SACC(t, e)), one read of A for all tokens.
         const int ncb = r8 >> 3;
         const int lg = ncb <= 1 ? 0 : (ncb <= 2 ? 1 : (ncb <= 4 ? 2 : 3));
         const int ncbp = 1 << lg;
@@ -443,7 +446,7 @@ sgmv_kernel(const __grid_constant__ AMaps am, const SgmvParams p)
         const int tiles_s = Mt * nNT;
         const int tpw_s = (tiles_s + kComputeWarps - 1) / kComputeWarps;  // <= 4
         // one register file for both paths (a tile takes exactly one of them):
-        // small: R[t*8+e] = token t, column c_own*8+e; large: R[q*4+e] = MMA tile q
+        // small: R[i*8+e] (see above); large: R[q*4+e] = MMA tile q
         float R[kSmallTile * 8];
 #pragma unroll
         for (int i = 0; i < kSmallTile * 8; ++i) R[i] = 0.f;
@@ -473,37 +476,56 @@ sgmv_kernel(const __grid_constant__ AMaps am, const SgmvParams p)
         // ---- partial v of this CTA -> VF, cluster exchange, v in VF (all rows)
         auto reduce_v = [&]() {
             if (small) {
-                // lanes sharing a chunk (lane % ncbp) reduce by shuffles, then warps through VF
-                for (int off = 16; off >= ncbp; off >>= 1)
+                if constexpr (kSmallOnly) {
+                    // each pair of a warp: a shuffle tree over the lanes, then lane 0 writes its 8 sums
 #pragma unroll
-                    for (int t = 0; t < kSmallTile; ++t)
-                        if (t < nt)  // uniform
+                    for (int i = 0; i < kSmallTile * 8 / kComputeWarps; ++i) {
+                        const int q = warp + kComputeWarps * i;
+                        if (q >= nt * ncbp) break;  // uniform per warp
+                        const int t = q >> lg, c = q & (ncbp - 1);
+                        if (c >= ncb) continue;
+                        for (int off = 16; off >= 1; off >>= 1)
 #pragma unroll
-                            for (int e = 0; e < 8; ++e)
-                                SACC(t, e) += __shfl_xor_sync(0xffffffffu, SACC(t, e), off);
-                if (lane < ncbp) {
-#pragma unroll
-                    for (int t = 0; t < kSmallTile; ++t)
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) VF[((warp * ncbp + lane) * kSmallTile + t) * 8 + e] = SACC(t, e);
-                }
-                ptx::named_sync(1, kCompute);
-                // column j = c*8+e of token t: sum the slots of the threads that own chunk c
-                float part[2] = {0.f, 0.f};
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const int idx = tid + h * kCompute;
-                    if (idx < nt * r8) {
-                        const int t = idx / r8, j = idx - t * r8, c = j >> 3, e = j & 7;
-                        for (int w = 0; w < kComputeWarps; ++w)
-                            part[h] += VF[((w * ncbp + c) * kSmallTile + t) * 8 + e];
+                            for (int e = 0; e < 8; ++e) SACC(i, e) += __shfl_xor_sync(0xffffffffu, SACC(i, e), off);
+                        if (lane == 0) {
+                            float4* dst = reinterpret_cast<float4*>(&VF[t * p.rp + c * 8]);
+                            dst[0] = make_float4(SACC(i, 0), SACC(i, 1), SACC(i, 2), SACC(i, 3));
+                            dst[1] = make_float4(SACC(i, 4), SACC(i, 5), SACC(i, 6), SACC(i, 7));
+                        }
                     }
-                }
-                ptx::named_sync(1, kCompute);
+                } else {
+                    // lanes sharing a chunk (lane % ncbp) reduce by shuffles, then warps through VF
+                    for (int off = 16; off >= ncbp; off >>= 1)
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const int idx = tid + h * kCompute;
-                    if (idx < nt * r8) VF[(idx / r8) * p.rp + idx % r8] = part[h];
+                        for (int t = 0; t < kSmallTile; ++t)
+                            if (t < nt)  // uniform
+#pragma unroll
+                                for (int e = 0; e < 8; ++e)
+                                    SACC(t, e) += __shfl_xor_sync(0xffffffffu, SACC(t, e), off);
+                    if (lane < ncbp) {
+#pragma unroll
+                        for (int t = 0; t < kSmallTile; ++t)
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) VF[((warp * ncbp + lane) * kSmallTile + t) * 8 + e] = SACC(t, e);
+                    }
+                    ptx::named_sync(1, kCompute);
+                    // column j = c*8+e of token t: sum the slots of the threads that own chunk c
+                    float part[2] = {0.f, 0.f};
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const int idx = tid + h * kCompute;
+                        if (idx < nt * r8) {
+                            const int t = idx / r8, j = idx - t * r8, c = j >> 3, e = j & 7;
+                            for (int w = 0; w < kComputeWarps; ++w)
+                                part[h] += VF[((w * ncbp + c) * kSmallTile + t) * 8 + e];
+                        }
+                    }
+                    ptx::named_sync(1, kCompute);
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const int idx = tid + h * kCompute;
+                        if (idx < nt * r8) VF[(idx / r8) * p.rp + idx % r8] = part[h];
+                    }
                 }
             } else {
                 const int gq = lane >> 2, tq = lane & 3;
@@ -606,20 +628,43 @@ sgmv_kernel(const __grid_constant__ AMaps am, const SgmvParams p)
             const int kb = min(BK, k_begin + k_len - k0);
             const uint32_t xb = base + (uint32_t)(BK * apitch);
             if (ok && small) {
-                if (c_own < ncb) {
-                    for (int k = rg; k < kb; k += rstride) {
-                        const uint4 av =
-                            *reinterpret_cast<const uint4*>(smem + (base - base_u) + a_chunk(k, c_own, apitch, a_swz));
-                        const float af[8] = {bf16_lo(av.x), bf16_hi(av.x), bf16_lo(av.y), bf16_hi(av.y),
-                                             bf16_lo(av.z), bf16_hi(av.z), bf16_lo(av.w), bf16_hi(av.w)};
+                if constexpr (kSmallOnly) {
+                    // warp w owns the (token, 8-column chunk) pairs w, w + 8, ...: its lanes
+                    // stride over the block's rows, so one shuffle tree finishes each pair
 #pragma unroll
-                        for (int t = 0; t < kSmallTile; ++t) {
-                            if (t < nt) {
-                                const float xv = __uint_as_float(
-                                    (uint32_t)(*reinterpret_cast<const uint16_t*>(smem + (xb - base_u) + t * xp + k * 2))
-                                    << 16);
+                    for (int i = 0; i < kSmallTile * 8 / kComputeWarps; ++i) {
+                        const int q = warp + kComputeWarps * i;
+                        if (q >= nt * ncbp) break;  // uniform per warp
+                        const int t = q >> lg, c = q & (ncbp - 1);
+                        if (c >= ncb) continue;
+                        for (int k = lane; k < kb; k += 32) {
+                            const uint4 av =
+                                *reinterpret_cast<const uint4*>(smem + (base - base_u) + a_chunk(k, c, apitch, a_swz));
+                            const float xv = __uint_as_float(
+                                (uint32_t)(*reinterpret_cast<const uint16_t*>(smem + (xb - base_u) + t * xp + k * 2)) << 16);
+                            const float af[8] = {bf16_lo(av.x), bf16_hi(av.x), bf16_lo(av.y), bf16_hi(av.y),
+                                                 bf16_lo(av.z), bf16_hi(av.z), bf16_lo(av.w), bf16_hi(av.w)};
 #pragma unroll
-                                for (int e = 0; e < 8; ++e) SACC(t, e) = fmaf(xv, af[e], SACC(t, e));
+                            for (int e = 0; e < 8; ++e) SACC(i, e) = fmaf(xv, af[e], SACC(i, e));
+                        }
+                    }
+                } else {
+                    // thread owns 8 columns (chunk c_own) over rows k = rg, rg + rstride, ...
+                    if (c_own < ncb) {
+                        for (int k = rg; k < kb; k += rstride) {
+                            const uint4 av =
+                                *reinterpret_cast<const uint4*>(smem + (base - base_u) + a_chunk(k, c_own, apitch, a_swz));
+                            const float af[8] = {bf16_lo(av.x), bf16_hi(av.x), bf16_lo(av.y), bf16_hi(av.y),
+                                                 bf16_lo(av.z), bf16_hi(av.z), bf16_lo(av.w), bf16_hi(av.w)};
+#pragma unroll
+                            for (int t = 0; t < kSmallTile; ++t) {
+                                if (t < nt) {
+                                    const float xv = __uint_as_float(
+                                        (uint32_t)(*reinterpret_cast<const uint16_t*>(smem + (xb - base_u) + t * xp + k * 2))
+                                        << 16);
+#pragma unroll
+                                    for (int e = 0; e < 8; ++e) SACC(t, e) = fmaf(xv, af[e], SACC(t, e));
+                                }
                             }
                         }
                     }
