@@ -278,6 +278,9 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
         if (lane == 0) {
             ptx::tma_prefetch_desc(&tmW);
             ptx::tma_prefetch_desc(&tmX);
+            // W is read exactly once: first out of L2, which then keeps the reused data
+            // (xq, the stream-K partials, v, the adapters)
+            const uint64_t w_policy = ptx::l2_policy_evict_first();
             int stage = 0;
             uint32_t phase = 0;
             uint32_t issued_phase[kMaxStages];
@@ -309,7 +312,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
                     const uint32_t sW = smem_u + p.ring_off + stage * stage_bytes;
                     const uint32_t sX = sW + kStageW;
                     ptx::mbar_arrive_expect_tx(&full[stage], (uint32_t)stage_bytes);
-                    ptx::tma_load_2d(sW, &tmW, &full[stage], kb * BK, nb * kBlockM);
+                    ptx::tma_load_2d_hint(sW, &tmW, &full[stage], kb * BK, nb * kBlockM, w_policy);
                     if (waited) {
                         ptx::tma_load_2d(sX, &tmX, &full[stage], kb * BK, tb * p.BN);
                     } else {  // first ring pass: stage == n_def
