@@ -1141,6 +1141,10 @@ cudaError_t launch_fp8_gemm(const Fp8GemmArgs& a, cudaStream_t stream)
             stages = fit(64, 0, 0);
         }
     }
+    // At a few tokens the weight stream is HBM-bound with fewer stages in flight as well;
+    // a shallower queue of weight loads shortens the latency of the LoRA term's own loads
+    // (down-projection, v, B): 6 stages rather than 8 measured ~1 us faster at M = 16
+    if (a.lora && p.BN <= 32 && stages > 6) stages = 6;
     if (stages < 2) return cudaErrorInvalidConfiguration;
     p.stages = stages;
     p.n_slots = ns;
