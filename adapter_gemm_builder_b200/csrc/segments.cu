@@ -124,6 +124,126 @@ __device__ __forceinline__ int bin_of(int id, int n_adapters)
     return (id >= 0 && id < n_adapters) ? id : n_adapters;
 }
 
+// Tiny batches (T <= 64, n_adapters <= 64, a decode step): one warp and no block
+// barriers. Lane l holds tokens l and l + 32; match_any groups equal ids, so a
+// token's rank among its id is the number of equal ids before it (the slot-0
+// tokens of its id come first), and a scan over the <= 65 bins (3 per lane)
+// gives starts, indptr, the active list and the tile rows.
+constexpr int kWarpMaxT = 64;
+constexpr int kWarpMaxAdapters = 64;
+
+__device__ __forceinline__ int warp_excl_scan(int v, int* total)
+{
+    const int lane = threadIdx.x & 31;
+    int incl = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int n = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += n;
+    }
+    *total = __shfl_sync(0xffffffffu, incl, 31);
+    return incl - v;
+}
+
+__global__ void __launch_bounds__(32, 1)
+segments_warp_kernel(const int32_t* __restrict__ ids, int T, int n_adapters, int max_tiles, SegOut o)
+{
+    __shared__ int32_t hist[96];    // per bin (n_adapters + 1 <= 65), 3 per lane
+    __shared__ int32_t cnt0[96];    // the same over slot-0 tokens only
+    __shared__ int32_t starts[96];
+    ptx::pdl_wait();
+    ptx::pdl_launch_dependents();
+    const int lane = threadIdx.x;
+    const int nb = n_adapters + 1;
+    for (int b = lane; b < 96; b += 32) hist[b] = 0;
+    __syncwarp();
+
+    int bin[2], rank[2];
+    bool in[2];
+    int nbad = 0;
+#pragma unroll
+    for (int sl = 0; sl < 2; ++sl) {
+        const int t = lane + 32 * sl;
+        in[sl] = t < T;
+        const int id = in[sl] ? ids[t] : -1;
+        bin[sl] = in[sl] ? bin_of(id, n_adapters) : -2 - lane;  // absent tokens match nobody
+        if (in[sl]) {
+            o.tok_adapter[t] = bin[sl] < n_adapters ? id : -1;
+            if (bin[sl] == n_adapters && id != -1) ++nbad;
+        }
+    }
+    nbad = __reduce_add_sync(0xffffffffu, (unsigned)nbad);
+    const unsigned lt = (1u << lane) - 1u;
+    // slot 0: one leader per distinct bin sets its count
+    const unsigned p0 = __match_any_sync(0xffffffffu, bin[0]);
+    rank[0] = __popc(p0 & lt);
+    if (in[0] && lane == __ffs(p0) - 1) hist[bin[0]] = __popc(p0);
+    __syncwarp();
+    for (int b = lane; b < 96; b += 32) cnt0[b] = hist[b];
+    __syncwarp();
+    // slot 1: after every slot-0 token of the same bin
+    const unsigned p1 = __match_any_sync(0xffffffffu, bin[1]);
+    rank[1] = in[1] ? cnt0[bin[1]] + __popc(p1 & lt) : 0;
+    if (in[1] && lane == __ffs(p1) - 1) hist[bin[1]] = cnt0[bin[1]] + __popc(p1);
+    __syncwarp();
+
+    // starts / indptr over bins 3*lane .. 3*lane+2
+    int h[3], sum = 0;
+#pragma unroll
+    for (int i = 0; i < 3; ++i) {
+        const int b = 3 * lane + i;
+        h[i] = b < nb ? hist[b] : 0;
+        sum += h[i];
+    }
+    int n_valid_all;
+    int base = warp_excl_scan(sum, &n_valid_all);
+#pragma unroll
+    for (int i = 0; i < 3; ++i) {
+        const int b = 3 * lane + i;
+        if (b < nb) {
+            starts[b] = base;
+            o.indptr[b] = base;
+        }
+        base += h[i];
+    }
+    // active adapters and their tiles: (#active << 16) | #tiles, scanned over bins
+    int pk = 0;
+#pragma unroll
+    for (int i = 0; i < 3; ++i) {
+        const int b = 3 * lane + i;
+        if (b < n_adapters && h[i] > 0) pk += (1 << 16) + (h[i] + o.tile_t - 1) / o.tile_t;
+    }
+    int pk_total;
+    const int pbase = warp_excl_scan(pk, &pk_total);
+    int pos = pbase >> 16, tile = pbase & 0xffff;
+#pragma unroll
+    for (int i = 0; i < 3; ++i) {
+        const int b = 3 * lane + i;
+        if (b < n_adapters && h[i] > 0) {
+            o.active[pos] = b;
+            for (int off = 0; off < h[i]; off += o.tile_t, ++tile)
+                reinterpret_cast<int4*>(o.tiles)[tile] = make_int4(b, starts[b] + off, min(o.tile_t, h[i] - off), pos);
+            ++pos;
+        }
+    }
+    const int n_active = pk_total >> 16, n_tiles = pk_total & 0xffff;
+    for (int a = n_active + lane; a < n_adapters; a += 32) o.active[a] = -1;
+    for (int g = n_tiles + lane; g < max_tiles; g += 32)
+        reinterpret_cast<int4*>(o.tiles)[g] = make_int4(-1, 0, 0, -1);
+    __syncwarp();  // starts[] complete
+#pragma unroll
+    for (int sl = 0; sl < 2; ++sl)
+        if (in[sl]) o.perm[starts[bin[sl]] + rank[sl]] = lane + 32 * sl;
+    if (lane == 0) {
+        o.counts[0] = starts[n_adapters];
+        o.counts[1] = n_active;
+        o.counts[2] = nbad;
+        o.counts[3] = n_tiles;
+        o.counts[4] = 0;  // device status word
+        o.counts[5] = o.counts[6] = o.counts[7] = 0;
+    }
+}
+
 // Small batches: blockDim >= T, shared memory = (warps + 2) * nb ints.
 __global__ void __launch_bounds__(kMaxThreads, 1)
 segments_small_kernel(const int32_t* __restrict__ ids, int T, int n_adapters, int max_tiles, SegOut o)
@@ -254,6 +374,11 @@ cudaError_t launch_build_segments(const int32_t* ids, int T, int n_adapters,
     cfg.stream = stream;
     cfg.gridDim = dim3(1, 1, 1);
     cudaError_t e;
+    if (T <= kWarpMaxT && n_adapters <= kWarpMaxAdapters) {
+        cfg.blockDim = dim3(32, 1, 1);
+        cfg.dynamicSmemBytes = 0;
+        return cudaLaunchKernelEx(&cfg, segments_warp_kernel, ids, T, n_adapters, mt, o);
+    }
     if (small) {
         cfg.blockDim = dim3(threads_small, 1, 1);
         cfg.dynamicSmemBytes = smem_small;

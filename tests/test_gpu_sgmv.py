@@ -54,6 +54,9 @@ def _check_segments(ids, n_adapters):
     ("distinct", 36, 32), ("identical", 36, 32), ("uniform", 1000, 7), ("zipf", 512, 256),
     ("sorted_zipf", 2300, 8), ("uniform", 5000, 3000), ("zipf", 4097, 1), ("uniform", 1, 5),
     ("zipf", 70000, 16384),
+    # one-warp builder (T <= 64, n <= 64): both tile sizes, a partial second slot of lanes
+    ("zipf", 64, 64), ("uniform", 50, 3), ("zipf", 17, 60), ("sorted_zipf", 40, 8),
+    ("identical", 64, 1), ("uniform", 33, 64), ("distinct", 64, 64),
 ])
 def test_segments_bitexact(kind, T, n):
     rng = np.random.default_rng(T + n)
@@ -68,6 +71,8 @@ def test_segments_edge_cases():
     rng = np.random.default_rng(3)
     bad = rng.integers(-5, 15, size=777).astype(np.int32)    # out-of-range ids
     _check_segments(bad, 10)
+    _check_segments(rng.integers(-5, 15, size=40).astype(np.int32), 10)  # the same, one warp
+    _check_segments(np.full(20, -1, np.int32), 4)            # one warp, nobody has an adapter
 
 
 def test_segments_sync_check_reports_bad_ids():
