@@ -87,6 +87,19 @@ def test_fp8_gemm_lora_full_grid(M, K, N, lora):
     assert_close(f64(y), want, TOL_FP8, f"fp8 M{M} K{K} N{N} lora={lora}")
 
 
+def test_fp8_gemm_adapters_beyond_vq_capacity():
+    """256 tokens over 48 adapters of rank up to 64: the shared-memory plan holds V'
+    tiles for 8 adapters per token block (64-byte k-blocks, 4 slots, two phases), so
+    the others take the CUDA-core path in the epilogue."""
+    M, K, N = 256, 512, 256
+    p, Wq, sw, y = _fp8_case(M, K, N, n_adapters=48, r=64, seed=21, kind="uniform",
+                             rank_choices=(8, 16, 40, 64))
+    rows = np.repeat(np.arange(M), N).astype(np.int32)
+    cols = np.tile(np.arange(N), M).astype(np.int32)
+    want = _oracle_fp8(p, Wq, sw, rows, cols, True).reshape(M, N)
+    assert_close(f64(y), want, TOL_FP8, "adapters beyond V' capacity")
+
+
 def test_fp8_gemm_mixed_ranks_many_adapters():
     p, Wq, sw, y = _fp8_case(96, 512, 256, n_adapters=40, r=64, seed=5, kind="uniform",
                              rank_choices=(8, 16, 64))
