@@ -77,6 +77,7 @@ struct GemmParams {
     float* v;  // fp32 [v_rep][M][r_max], segment (perm) order, zeroed by the quantiser: the
                // down-projection of K chunk q adds into copy q % v_rep (fewer atomics per address)
     int v_rep, lg_rep;  // copies of v (a power of two), log2
+    int lg_lanes;       // log2 of the lanes that sum one token's copies in the V' build
     const uint16_t* B;
     const int32_t* ranks;
     const float* scales;
@@ -706,15 +707,24 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
                     // tokens t (zero for the other tokens of its 16-aligned column range), K-major
                     // bf16, for every phase of every segment of this token block. Each token's
                     // v row is loaded first, so the build waits for one round trip to memory
-                    // lane (token pl, copy cp): v_rep consecutive lanes load the copies of one
-                    // token's v row and sum them with shuffles (BN * v_rep <= 256)
-                    const int pl = etid >> p.lg_rep, cp = etid & (p.v_rep - 1);
+                    // lane (token pl, lane cp of the token's 2^lg_lanes): the lane loads copies
+                    // cp, cp + lanes, ... of the token's v row and adds them, then the token's
+                    // lanes sum by shuffles (BN * lanes <= 256)
+                    const int lanes = 1 << p.lg_lanes, cpl = p.v_rep >> p.lg_lanes;
+                    const int pl = etid >> p.lg_lanes, cp = etid & (lanes - 1);
+                    const size_t cstride = (size_t)lanes * p.M * p.r_max / 4;  // float4s between a lane's copies
                     int q_own = -1;
                     float4 vr[4];  // v[token][0..16) (a larger rank loads the rest later)
 #pragma unroll
                     for (int h = 0; h < 4; ++h) vr[h] = make_float4(0.f, 0.f, 0.f, 0.f);
                     const float4* vg = reinterpret_cast<const float4*>(
                         p.v + ((size_t)cp * p.M + tb * p.BN + min(pl, p.BN - 1)) * p.r_max);
+                    auto add4 = [](float4& a4, const float4 b4) {
+                        a4.x += b4.x;
+                        a4.y += b4.y;
+                        a4.z += b4.z;
+                        a4.w += b4.w;
+                    };
                     if (pl < p.BN) {
                         const int a = s_a[pl];
                         if (a >= 0) {
@@ -724,9 +734,10 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
                         }
                         if (cp == 0) s_q[pl] = q_own;
                         if (q_own >= 0) {
+                            for (int i = 0; i < cpl; ++i)
 #pragma unroll
-                            for (int h = 0; h < 4; ++h)
-                                if (4 * h < p.r_max) vr[h] = __ldcg(vg + h);
+                                for (int h = 0; h < 4; ++h)
+                                    if (4 * h < p.r_max) add4(vr[h], __ldcg(vg + i * cstride + h));
                         }
                     }
                     // zero every slot's tile and publish its byte offset
@@ -741,7 +752,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
                     }
                     if (!(ok = epi_sync())) break;
                     auto sum_copies = [&](float4& f) {
-                        for (int o = 1; o < p.v_rep; o <<= 1) {
+                        for (int o = 1; o < lanes; o <<= 1) {
                             f.x += __shfl_xor_sync(0xffffffffu, f.x, o);
                             f.y += __shfl_xor_sync(0xffffffffu, f.y, o);
                             f.z += __shfl_xor_sync(0xffffffffu, f.z, o);
@@ -765,10 +776,11 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
                                 f0 = vr[2 * kg];
                                 f1 = vr[2 * kg + 1];
                             } else {
-                                if (in_row) {
-                                    f0 = __ldcg(vg + 2 * kg);
-                                    f1 = __ldcg(vg + 2 * kg + 1);
-                                }
+                                if (in_row)
+                                    for (int i = 0; i < cpl; ++i) {
+                                        add4(f0, __ldcg(vg + i * cstride + 2 * kg));
+                                        add4(f1, __ldcg(vg + i * cstride + 2 * kg + 1));
+                                    }
                                 sum_copies(f0);
                                 sum_copies(f1);
                             }
@@ -1037,11 +1049,10 @@ int fp8_gemm_tile_n(int M)
 
 int fp8_gemm_v_copies(int M)
 {
-    // as many copies as the V' build has lanes to spare per token (at most 8)
-    const int bn = fp8_gemm_tile_n(M);
-    int c = 1;
-    while (c < 8 && bn * c * 2 <= kEpiThreads) c *= 2;
-    return c;
+    // 8 copies: the adds of 128 K chunks into one 16-byte piece of v are spread 8 ways;
+    // the V' build sums them (one lane per copy at few tokens, several copies a lane at more)
+    (void)M;
+    return 8;
 }
 
 size_t fp8_gemm_partial_bytes(int M)
@@ -1077,6 +1088,8 @@ cudaError_t launch_fp8_gemm(const Fp8GemmArgs& a, cudaStream_t stream)
     p.v = a.v;
     p.v_rep = fp8_gemm_v_copies(a.M);
     p.lg_rep = __builtin_ctz((unsigned)p.v_rep);
+    p.lg_lanes = p.lg_rep;
+    while ((p.BN << p.lg_lanes) > kEpiThreads) --p.lg_lanes;
     p.B = a.B;
     p.ranks = a.ranks;
     p.scales = a.scales;
