@@ -18,19 +18,25 @@
 //    first thing and raise a flag; the finisher adds them before its epilogue.
 //  * warp roles in each CTA:
 //      warp 0  TMA producer: W and xq k-blocks into a ring of stages
-//              (128- or 64-byte swizzle, matching the MMA descriptors); its
-//              first W loads are issued before the wait on the quantiser;
+//              (128- or 64-byte swizzle, matching the MMA descriptors); W's
+//              tiles carry an L2 evict-first policy (read once); its first W
+//              loads are issued before the wait on the quantiser;
 //      warp 1  TMEM allocator and single-thread tcgen05.mma issuer
 //              (kind::f8f6f4, fp32 accumulators in TMEM, double-buffered so the
-//              epilogue of one segment overlaps the mainloop of the next);
-//      warp 2  B stager: TMA-loads the [r x 128] slices of B_a of every
-//              adapter of the tile's token block into shared memory;
+//              epilogue of one segment overlaps the mainloop of the next); it
+//              also issues the LoRA up-projection (kind::f16) of a segment in
+//              phases between that segment's own k-blocks;
+//      warp 2  B stager: TMA-loads the [r x 128] slices of B_a of the adapters
+//              of the tile's token block into a few shared-memory slots, one
+//              phase of slots at a time (the MMAs of a phase free the slots);
 //      warps 3..10 the down-projection first -- while the first weights
 //              stream, each CTA computes v over its own 64-column slice of K
-//              for every token (bf16 x, fp32 sums, vector atomics into v,
-//              then a completion count) -- and then the epilogue: tcgen05.ld
-//              of the accumulator, per-token and per-channel scales, the LoRA
-//              term on CUDA cores from shared memory, bf16 stores.
+//              for every token (bf16 x, fp32 sums, vector atomics spread over
+//              8 copies of v, then a completion count) -- then, per segment,
+//              the LoRA operands (V' = s_a v / sx per token block, B' = B / sw
+//              per phase) and the epilogue: tcgen05.ld of the accumulator,
+//              stream-K partials, per-token and per-channel scales, bf16 rows
+//              stored 16 bytes at a time.
 //  * tokens are processed in segment order (rows of xq are permuted by the
 //    quantiser, v is kept in that order), so the adapter changes only at
 //    segment boundaries.
