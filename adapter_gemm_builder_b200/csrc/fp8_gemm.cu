@@ -917,7 +917,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
 #pragma unroll
                 for (int e = 0; e < 16; ++e) lo[e] = 0.f;
                 if (p.lora) {
-                    // adapters that found no shared-memory slot: their term on CUDA cores, B
+                    // adapters past the V' capacity of the token block: their term on CUDA cores, B
                     // and v from global memory (the staged ones are in the accumulator)
                     bool far = false;
 #pragma unroll

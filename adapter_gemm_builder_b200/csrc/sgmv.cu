@@ -8,7 +8,11 @@
 //   APPLY   y += s_a * (x.A_a).B_a, with v kept on chip
 //
 // Work. The segment builder cuts every adapter's run of tokens into tiles of
-// at most LORA_TILE_TOKENS tokens (one row of lora_segments_t.tiles each). A
+// at most lora_tile_tokens_for(T, n_adapters) tokens (one row of
+// lora_segments_t.tiles each): 4 for a decode-like batch, which then runs
+// the kernel variant built for such tiles alone (no tensor-core path: a
+// smaller kernel whose short-lived CTAs wait less on instruction fetch), else
+// LORA_TILE_TOKENS. A
 // tile is handled by a thread-block cluster of C CTAs: in the shrink CTA c
 // owns the c-th slice of h_in (split-K) and computes a partial v for the
 // tile's tokens; in the expand it owns the c-th slice of h_out. gridDim.y is
