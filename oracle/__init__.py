@@ -57,7 +57,7 @@ def _load():
             lib.orc_e4m3_encode.restype = ctypes.c_uint8
             lib.orc_e4m3_encode.argtypes = [ctypes.c_float]
             lib.orc_build_segments.restype = None
-            lib.orc_build_segments.argtypes = [P, I, I, I, P, P, P, P, I, P, P]
+            lib.orc_build_segments.argtypes = [P, I, I, P, P, P, P, P]
             lib.orc_lora_shrink.restype = None
             lib.orc_lora_shrink.argtypes = [P, I, I, P, I, I, P, P, P]
             lib.orc_lora_expand.restype = None
@@ -125,26 +125,21 @@ def e4m3_to_f64(a: np.ndarray) -> np.ndarray:
     return _table("orc_e4m3_decode", 256)[np.asarray(a, dtype=np.uint8)]
 
 
-def max_tiles(T: int, n_adapters: int, tile_t: int) -> int:
-    return min(n_adapters, T) + (T + tile_t - 1) // tile_t
-
-
-def build_segments(ids: np.ndarray, n_adapters: int, tile_t: int) -> dict:
+def build_segments(ids: np.ndarray, n_adapters: int) -> dict:
+    """Stable group-by of the tokens by adapter id: perm, indptr, active,
+    tok_adapter and counts = [n_valid, n_active, n_bad]."""
     lib = _load()
     ids = _c(ids, np.int32)
     T = ids.shape[0]
-    mt = max_tiles(T, n_adapters, tile_t)
     out = dict(
         perm=np.zeros(T, np.int32),
         indptr=np.zeros(n_adapters + 1, np.int32),
         active=np.zeros(n_adapters, np.int32),
-        tiles=np.zeros((mt, 4), np.int32),
         tok_adapter=np.zeros(T, np.int32),
-        counts=np.zeros(4, np.int32),
+        counts=np.zeros(3, np.int32),
     )
-    lib.orc_build_segments(_p(ids), T, n_adapters, tile_t, _p(out["perm"]), _p(out["indptr"]),
-                           _p(out["active"]), _p(out["tiles"]), mt, _p(out["tok_adapter"]),
-                           _p(out["counts"]))
+    lib.orc_build_segments(_p(ids), T, n_adapters, _p(out["perm"]), _p(out["indptr"]),
+                           _p(out["active"]), _p(out["tok_adapter"]), _p(out["counts"]))
     return out
 
 

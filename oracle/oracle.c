@@ -110,16 +110,14 @@ uint8_t orc_e4m3_encode(float f)
  *   indptr[n_adapters] = number of valid tokens.
  * active[n_adapters]: ids with at least one token, ascending (first n_active
  *   entries meaningful; the rest are set to -1).
- * tiles[max_tiles][4]: every active segment cut, in order, into chunks of at
- *   most tile_t tokens: {adapter, first position in perm, token count,
- *   segment index}; rows past the last chunk are {-1, 0, 0, -1}.
- *   max_tiles = min(n_adapters, T) + ceil(T / tile_t) bounds the chunk count.
  * tok_adapter[T]: the id each token is served with (-1 for none or bad).
- * counts[4]: n_valid, n_active, n_bad, n_tiles.
+ * counts[3]: n_valid, n_active, n_bad.
+ * This is the grouping the segmented gather needs and nothing more: how a
+ * kernel cuts the segments into units of work is not part of it.
  */
-void orc_build_segments(const int32_t* ids, int T, int n_adapters, int tile_t,
+void orc_build_segments(const int32_t* ids, int T, int n_adapters,
                         int32_t* perm, int32_t* indptr, int32_t* active,
-                        int32_t* tiles, int max_tiles, int32_t* tok_adapter, int32_t* counts)
+                        int32_t* tok_adapter, int32_t* counts)
 {
     int32_t* cnt = (int32_t*)calloc((size_t)n_adapters + 1, sizeof(int32_t));
     int32_t* cursor = (int32_t*)calloc((size_t)n_adapters + 1, sizeof(int32_t));
@@ -148,34 +146,15 @@ void orc_build_segments(const int32_t* ids, int T, int n_adapters, int tile_t,
         int bin = (id >= 0 && id < n_adapters) ? id : n_adapters;
         perm[cursor[bin]++] = t;
     }
-    int n_active = 0, n_tiles = 0;
-    for (int a = 0; a < n_adapters; ++a) {
-        if (cnt[a] > 0) {
-            active[n_active] = a;
-            for (int off = 0; off < cnt[a]; off += tile_t) {
-                int32_t* row = tiles + 4 * (size_t)n_tiles;
-                row[0] = a;
-                row[1] = indptr[a] + off;
-                row[2] = (cnt[a] - off < tile_t) ? cnt[a] - off : tile_t;
-                row[3] = n_active;
-                ++n_tiles;
-            }
-            ++n_active;
-        }
-    }
+    int n_active = 0;
+    for (int a = 0; a < n_adapters; ++a)
+        if (cnt[a] > 0)
+            active[n_active++] = a;
     for (int s = n_active; s < n_adapters; ++s)
         active[s] = -1;
-    for (int g = n_tiles; g < max_tiles; ++g) {
-        int32_t* row = tiles + 4 * (size_t)g;
-        row[0] = -1;
-        row[1] = 0;
-        row[2] = 0;
-        row[3] = -1;
-    }
     counts[0] = indptr[n_adapters];
     counts[1] = n_active;
     counts[2] = n_bad;
-    counts[3] = n_tiles;
     free(cnt);
     free(cursor);
 }

@@ -12,6 +12,7 @@ import torch
 import oracle
 from adapter_gemm_builder_b200 import lora as L
 from adapter_gemm_builder_b200 import workloads as wl
+from tile_rule import expected_tiles, tile_tokens
 from gpu_util import (TOL_BF16, DeviceProblem, assert_close, dev, dev_bf16, f64, host_bf16_bits,
                       oracle_apply, rne_bf16_bits)
 
@@ -28,23 +29,28 @@ def _lib():
 # ------------------------------------------------------------------ segments
 
 def _check_segments(ids, n_adapters):
+    """The grouping (perm, indptr, active, tok_adapter, counts) bit-exact against
+    the oracle; the tile table against the tile rule applied to the oracle's grouping."""
     T = len(ids)
     seg = L.Segments(T, n_adapters)
     L.lora_build_segments(dev(ids) if T else torch.empty(0, dtype=torch.int32, device="cuda"),
                           n_adapters, seg)
     torch.cuda.synchronize()
-    want = oracle.build_segments(ids, n_adapters, L.tile_tokens_for(T, n_adapters))
+    want = oracle.build_segments(ids, n_adapters)
     counts = seg.counts.cpu().numpy()
-    assert counts[:4].tolist() == want["counts"].tolist()
+    t = L.tile_tokens_for(T, n_adapters)
+    assert t == tile_tokens(T, n_adapters)
+    want_tiles = expected_tiles(want["indptr"], want["active"], want["counts"][1], t)
+    assert counts[:3].tolist() == want["counts"].tolist()
+    assert counts[3] == len(want_tiles)
     assert counts[4:].tolist() == [0, 0, 0, 0]
     assert seg.indptr.cpu().numpy().tolist() == want["indptr"].tolist()
     assert seg.active.cpu().numpy().tolist() == want["active"].tolist()
-    # the tile rows themselves, then padding rows (the two arrays are sized by bounds
-    # of their own)
-    n_tiles = int(want["counts"][3])
     got_tiles = seg.tiles.cpu().numpy()
-    assert got_tiles[:n_tiles].tolist() == want["tiles"][:n_tiles].tolist()
-    assert all(row == [-1, 0, 0, -1] for row in got_tiles[n_tiles:L.max_tiles(T, n_adapters)].tolist())
+    n_rows = L.max_tiles(T, n_adapters)
+    assert len(want_tiles) <= n_rows
+    assert got_tiles[:len(want_tiles)].tolist() == want_tiles
+    assert all(row == [-1, 0, 0, -1] for row in got_tiles[len(want_tiles):n_rows].tolist())
     if T:
         assert seg.perm.cpu().numpy()[:T].tolist() == want["perm"].tolist()
         assert seg.tok_adapter.cpu().numpy()[:T].tolist() == want["tok_adapter"].tolist()

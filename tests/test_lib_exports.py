@@ -171,15 +171,18 @@ def test_binding_fails_loudly_without_library(tmp_path):
 def test_max_tiles_bounds_every_id_mix(lib):
     """The tile-row bound holds for the worst cases of the tile rule: every adapter
     one token more than a multiple of the tile size, all tokens on one adapter,
-    and random mixes (tiles counted by the oracle's builder)."""
+    and random mixes (rows counted by the tile rule over the oracle's grouping)."""
     import oracle
+    from tile_rule import expected_tiles, tile_tokens
     rng = np.random.default_rng(7)
     cases = [(36, 32), (64, 32), (48, 24), (5, 2), (64, 4), (300, 7), (1000, 999), (130, 64)]
     for T, n in cases:
         t = lib.lora_tile_tokens_for(T, n)
+        assert t == tile_tokens(T, n), (T, n)
         bound = lib.lora_max_tiles(T, n)
         mixes = [rng.integers(0, n, T), np.zeros(T, np.int64), np.arange(T) % n,
                  np.repeat(np.arange(n), t + 1)[:T]]
         for ids in mixes:
-            seg = oracle.build_segments(ids.astype(np.int32), n, t)
-            assert seg["counts"][3] <= bound, (T, n, t)
+            seg = oracle.build_segments(ids.astype(np.int32), n)
+            rows = expected_tiles(seg["indptr"], seg["active"], seg["counts"][1], t)
+            assert len(rows) <= bound, (T, n, t)

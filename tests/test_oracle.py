@@ -109,19 +109,15 @@ def test_e4m3_encode_ties_to_even_and_saturation():
 
 # ---------------------------------------------------------------- segments
 
-def _segments_by_sort(ids, n_adapters, tile_t):
+def _segments_by_sort(ids, n_adapters):
     T = len(ids)
     key = [(ids[t] if 0 <= ids[t] < n_adapters else n_adapters, t) for t in range(T)]
     order = sorted(range(T), key=lambda t: key[t])  # library sort, stable key
     counts = [sum(1 for t in range(T) if key[t][0] == a) for a in range(n_adapters + 1)]
     indptr = [sum(counts[:a]) for a in range(n_adapters + 1)]
     active = [a for a in range(n_adapters) if counts[a] > 0]
-    tiles = []
-    for s, a in enumerate(active):
-        for off in range(0, counts[a], tile_t):
-            tiles.append([a, indptr[a] + off, min(tile_t, counts[a] - off), s])
     n_bad = sum(1 for i in ids if i != -1 and not (0 <= i < n_adapters))
-    return order, indptr, active, tiles, n_bad
+    return order, indptr, active, n_bad
 
 
 SEG_KINDS = ["distinct", "identical", "uniform", "zipf", "sorted_zipf", "none", "bad", "single"]
@@ -130,7 +126,7 @@ SEG_KINDS = ["distinct", "identical", "uniform", "zipf", "sorted_zipf", "none", 
 @pytest.mark.parametrize("kind", SEG_KINDS)
 def test_segments_match_sorted_order(kind):
     rng = np.random.default_rng(SEG_KINDS.index(kind))
-    n_adapters, tile_t = 12, 4
+    n_adapters = 12
     if kind == "none":
         ids = np.full(17, -1, np.int32)
     elif kind == "bad":
@@ -141,24 +137,23 @@ def test_segments_match_sorted_order(kind):
         ids = wl.make_ids("distinct", rng, 12, n_adapters, none_frac=0.2)
     else:
         ids = wl.make_ids(kind, rng, 50, n_adapters, none_frac=0.1)
-    seg = oracle.build_segments(ids, n_adapters, tile_t)
-    order, indptr, active, tiles, n_bad = _segments_by_sort(list(ids), n_adapters, tile_t)
+    seg = oracle.build_segments(ids, n_adapters)
+    order, indptr, active, n_bad = _segments_by_sort(list(ids), n_adapters)
     assert seg["perm"].tolist() == order
     assert seg["indptr"].tolist() == indptr
     n_active = len(active)
-    assert seg["counts"].tolist() == [indptr[n_adapters], n_active, n_bad, len(tiles)]
+    assert seg["counts"].tolist() == [indptr[n_adapters], n_active, n_bad]
     assert seg["active"][:n_active].tolist() == active
-    assert seg["tiles"][:len(tiles)].tolist() == tiles
-    assert (seg["tiles"][len(tiles):] == [-1, 0, 0, -1]).all()
-    assert len(tiles) <= oracle.max_tiles(len(ids), n_adapters, tile_t)
+    assert (seg["active"][n_active:] == -1).all()
     want_tok = [i if 0 <= i < n_adapters else -1 for i in ids]
     assert seg["tok_adapter"].tolist() == want_tok
 
 
 def test_segments_empty_batch():
-    seg = oracle.build_segments(np.zeros(0, np.int32), 3, 64)
-    assert seg["counts"].tolist() == [0, 0, 0, 0]
+    seg = oracle.build_segments(np.zeros(0, np.int32), 3)
+    assert seg["counts"].tolist() == [0, 0, 0]
     assert seg["indptr"].tolist() == [0, 0, 0, 0]
+    assert seg["active"].tolist() == [-1, -1, -1]
 
 
 # ---------------------------------------------------------------- LoRA algebra
