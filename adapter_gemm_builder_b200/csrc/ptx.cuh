@@ -3,6 +3,7 @@
 // cluster barriers and distributed shared memory, programmatic dependent
 // launch, mbarriers, TMA tensor loads and the tcgen05 (TMEM) tensor-core path.
 #pragma once
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -163,13 +164,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity)
 
 // ------------------------------------------------------------------ TMA
 
-__device__ __forceinline__ void tma_prefetch_desc(const void* tmap)
+// The descriptor arguments are typed: a TMA instruction handed any other
+// address (a local variable, a device pointer) reads garbage as its tensor
+// map, so such a call must not compile.
+
+__device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* tmap)
 {
     asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
 }
 // 2-D tiled tensor load (no multicast) into this CTA's shared memory;
 // completion is signalled as transaction bytes on `bar`.
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, uint64_t* bar, int32_t c0,
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* tmap, uint64_t* bar, int32_t c0,
                                             int32_t c1)
 {
     asm volatile(
@@ -179,7 +184,7 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, uint
         : "memory");
 }
 // The same with an L2 cache policy (from l2_policy_evict_first / _evict_last).
-__device__ __forceinline__ void tma_load_2d_hint(uint32_t dst, const void* tmap, uint64_t* bar, int32_t c0,
+__device__ __forceinline__ void tma_load_2d_hint(uint32_t dst, const CUtensorMap* tmap, uint64_t* bar, int32_t c0,
                                                  int32_t c1, uint64_t policy)
 {
     asm volatile(
@@ -202,7 +207,7 @@ __device__ __forceinline__ uint64_t l2_policy_evict_last()
     return p;
 }
 // 3-D tiled tensor load (no multicast), completion as transaction bytes on `bar`.
-__device__ __forceinline__ void tma_load_3d(uint32_t dst, const void* tmap, uint64_t* bar, int32_t c0,
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* tmap, uint64_t* bar, int32_t c0,
                                             int32_t c1, int32_t c2)
 {
     asm volatile(
