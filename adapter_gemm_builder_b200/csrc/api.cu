@@ -5,6 +5,8 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <atomic>
+
 #include "internal.h"
 #include "lora.h"
 
@@ -67,9 +69,49 @@ size_t fp8_ws_layout(int M, int K, const lora_pool_t* pool, size_t* off_xq, size
     return off;
 }
 
+constexpr unsigned long long kDefaultWaitNs = 2000000000ull;  // 2 s
+std::atomic<unsigned long long> g_wait_limit_ns{kDefaultWaitNs};
+std::atomic<int> g_inject_stall{0};
+
 }  // namespace
 
+namespace lora {
+
+unsigned long long debug_wait_limit_ns() { return g_wait_limit_ns.load(std::memory_order_relaxed); }
+int debug_inject_stall() { return g_inject_stall.load(std::memory_order_relaxed); }
+
+// Checks of fp8_gemm_lora_epilogue's arguments other than the workspace
+// (shared with the entry point that allocates nothing, so both answer alike).
+int fp8_gemm_check_args(const void* x, int M, int K, int N, const uint8_t* Wq, const float* w_scale,
+                        const lora_pool_t* pool, const lora_segments_t* seg, const void* y)
+{
+    if (M < 1 || K < 16 || N < 8 || K % 16 || N % 8) return LORA_ERR_INVALID_ARG;
+    if (!x || !Wq || !w_scale || !y) return LORA_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(Wq) || !aligned16(y)) return LORA_ERR_INVALID_ARG;
+    if (M > (1 << 24)) return LORA_ERR_UNSUPPORTED;
+    if (pool) {
+        int st = check_pool(pool);
+        if (st != LORA_OK) return st;
+        if (pool->n_slices != 1 || pool->h_in != K || pool->h_out != N) return LORA_ERR_INVALID_ARG;
+        if ((st = check_segments(seg, pool->n_adapters)) != LORA_OK) return st;
+        if (seg->T != M) return LORA_ERR_INVALID_ARG;
+    }
+    return LORA_OK;
+}
+
+}  // namespace lora
+
 extern "C" {
+
+int lora_debug_set_wait_limit(uint64_t limit_ns, int inject_stall)
+{
+    if (limit_ns == 0) limit_ns = kDefaultWaitNs;
+    if (limit_ns < 1000 || limit_ns > kDefaultWaitNs) return LORA_ERR_INVALID_ARG;
+    if (inject_stall != 0 && inject_stall != 1) return LORA_ERR_INVALID_ARG;
+    g_wait_limit_ns.store(limit_ns, std::memory_order_relaxed);
+    g_inject_stall.store(inject_stall, std::memory_order_relaxed);
+    return LORA_OK;
+}
 
 const char* lora_status_string(int s)
 {
@@ -251,17 +293,8 @@ int fp8_gemm_lora_epilogue(const void* x, int M, int K, int N, const uint8_t* Wq
                            const lora_segments_t* seg, void* y, void* ws, size_t ws_bytes,
                            lora_stream_t stream)
 {
-    if (M < 1 || K < 16 || N < 8 || K % 16 || N % 8) return LORA_ERR_INVALID_ARG;
-    if (!x || !Wq || !w_scale || !y) return LORA_ERR_INVALID_ARG;
-    if (!aligned16(x) || !aligned16(Wq) || !aligned16(y)) return LORA_ERR_INVALID_ARG;
-    if (M > (1 << 24)) return LORA_ERR_UNSUPPORTED;
-    if (pool) {
-        int st = check_pool(pool);
-        if (st != LORA_OK) return st;
-        if (pool->n_slices != 1 || pool->h_in != K || pool->h_out != N) return LORA_ERR_INVALID_ARG;
-        if ((st = check_segments(seg, pool->n_adapters)) != LORA_OK) return st;
-        if (seg->T != M) return LORA_ERR_INVALID_ARG;
-    }
+    const int st = fp8_gemm_check_args(x, M, K, N, Wq, w_scale, pool, seg, y);
+    if (st != LORA_OK) return st;
     size_t off_xq, off_sx, off_v, off_sync, off_part;
     const size_t need = fp8_ws_layout(M, K, pool, &off_xq, &off_sx, &off_v, &off_sync, &off_part);
     if (!ws || ws_bytes < need || !aligned16(ws)) return LORA_ERR_WORKSPACE;

@@ -58,7 +58,7 @@ constexpr int kEpiThreads = kEpiWarps * 32;
 constexpr int kThreads = (3 + kEpiWarps) * 32;
 constexpr int kMaxStages = 8;
 constexpr int kShrinkCols = 64;  // K columns of the down-projection per work item
-constexpr unsigned long long kTimeoutNs = 2000000000ull;
+constexpr unsigned long long kTimeoutNs = 2000000000ull;  // drains after an abort
 
 struct GemmParams {
     int M, N, K, BN, n_tb, n_nb, num_tiles, k_blocks, stages;
@@ -90,6 +90,8 @@ struct GemmParams {
     int n_adapters, r_max, r8, r16;
     int n_slots;
     uint32_t ring_off, slots_off, v_off, meta_off, bar_off;
+    unsigned long long timeout_ns;  // limit of every bounded wait (2 s unless a test lowers it)
+    int inject_stall;  // test hook: CTA 0's producer first waits on a barrier nothing completes
 };
 
 using ptx::globaltimer;
@@ -116,14 +118,14 @@ __device__ __forceinline__ void transpose8x8(uint32_t (&w)[8], int lane)
 // (another role gave up) or if this wait itself timed out (then it raises the
 // abort flag and records `code` in the status word).
 __device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                             uint32_t* status, uint32_t code)
+                                             uint32_t* status, uint32_t code, unsigned long long limit)
 {
     if (ptx::mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = globaltimer();
     while (true) {
         if (ptx::mbar_try_wait(bar, parity)) return true;
         if (*abort_flag) return false;
-        if (globaltimer() - t0 > kTimeoutNs) {
+        if (globaltimer() - t0 > limit) {
             *abort_flag = 1;
             if (status) atomicOr(status, code);
             return false;
@@ -140,7 +142,7 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity)
 
 // Bounded wait until the global counter reaches `target` (acquire, GPU scope).
 __device__ __forceinline__ bool wait_count(const int* ctr, int target, volatile int* abort_flag,
-                                           uint32_t* status, uint32_t code)
+                                           uint32_t* status, uint32_t code, unsigned long long limit)
 {
     const unsigned long long t0 = globaltimer();
     while (true) {
@@ -148,7 +150,7 @@ __device__ __forceinline__ bool wait_count(const int* ctr, int target, volatile 
         asm volatile("ld.acquire.gpu.global.b32 %0, [%1];\n" : "=r"(v) : "l"(ctr) : "memory");
         if (v >= target) return true;
         if (*abort_flag) return false;
-        if (globaltimer() - t0 > kTimeoutNs) {
+        if (globaltimer() - t0 > limit) {
             *abort_flag = 1;
             if (status) atomicOr(status, code);
             return false;
@@ -243,6 +245,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
     uint64_t* drain = bempty + 1;               // [1]
     uint64_t* epibar = drain + 1;               // [1] epilogue-warps barrier
     uint64_t* lready = epibar + 1;              // [1] LoRA operands of the segment built
+    uint64_t* stall = lready + 1;               // [1] test hook: never completed
     volatile int* abort_flag = &s_abort;
 
     constexpr int kStageW = kBlockM * BK;
@@ -267,6 +270,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
         ptx::mbar_init(drain, 1);
         ptx::mbar_init(epibar, kEpiWarps);
         ptx::mbar_init(lready, 1);
+        ptx::mbar_init(stall, 1);
         ptx::fence_mbar_init();
     }
     if (warp == 1) {
@@ -306,13 +310,17 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
                 }
             };
             bool ok = true;
+            // test hook: before its first load, CTA 0 waits on a barrier that nothing
+            // completes, so the bounded wait runs out and the CTA takes its abort path
+            if (p.inject_stall && cta == 0)
+                ok = wait_bounded(stall, 0, abort_flag, p.status, 0x400u, p.timeout_ns);
             for (long long u = u_begin; u < u_end && ok;) {
                 const Seg sg = seg_at(u, u_end, KB);
                 u += sg.kb1 - sg.kb0;
                 const int nb = sg.tile / p.n_tb, tb = sg.tile - nb * p.n_tb;
                 for (int kb = sg.kb0; kb < sg.kb1; ++kb) {
                     if (!waited && n_def == p.stages) flush_deferred();
-                    if (!wait_bounded(&empty[stage], phase ^ 1, abort_flag, p.status, 0x1u)) {
+                    if (!wait_bounded(&empty[stage], phase ^ 1, abort_flag, p.status, 0x1u, p.timeout_ns)) {
                         ok = false;
                         break;
                     }
@@ -395,7 +403,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
             auto lora_step = [&](bool block) -> bool {
                 if (fq_n == 0 || fq_ph[0] < 0) return true;
                 if (block) {
-                    if (!wait_bounded(lready, (uint32_t)(lj & 1), abort_flag, p.status, 0x200u)) return false;
+                    if (!wait_bounded(lready, (uint32_t)(lj & 1), abort_flag, p.status, 0x200u, p.timeout_ns)) return false;
                 } else if (!ptx::mbar_test_wait(lready, (uint32_t)(lj & 1))) {  // no suspend
                     return true;
                 }
@@ -420,7 +428,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
                     ok = false;
                     break;
                 }
-                if (!wait_bounded(&tempty[buf], bphase ^ 1, abort_flag, p.status, 0x2u)) {
+                if (!wait_bounded(&tempty[buf], bphase ^ 1, abort_flag, p.status, 0x2u, p.timeout_ns)) {
                     ok = false;
                     break;
                 }
@@ -428,7 +436,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
                 const uint32_t d = tmem_base + (uint32_t)(buf * p.BN);
                 for (int kb = sg.kb0; kb < sg.kb1; ++kb) {
                     if (!lora_step(false) ||
-                        !wait_bounded(&full[stage], phase, abort_flag, p.status, 0x4u)) {
+                        !wait_bounded(&full[stage], phase, abort_flag, p.status, 0x4u, p.timeout_ns)) {
                         ok = false;
                         break;
                     }
@@ -489,7 +497,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
                 if (sg.kb0 != 0) continue;  // partial accumulators only: no epilogue here
                 const int nb = sg.tile / p.n_tb, tb = sg.tile - nb * p.n_tb;
                 for (int ph = 0;; ++ph) {
-                    if (!(ok = wait_bounded(bempty, (uint32_t)((j & 1) ^ 1), abort_flag, p.status, 0x8u))) break;
+                    if (!(ok = wait_bounded(bempty, (uint32_t)((j & 1) ^ 1), abort_flag, p.status, 0x8u, p.timeout_ns))) break;
                     if (ph == 0 && tb != slots_tb) {
                         // the adapters of this token block (kept while the block does not change)
                         slots_tb = tb;
@@ -551,7 +559,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
         auto epi_sync = [&]() -> bool {
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(epibar);
-            const bool ok = wait_bounded(epibar, epi_phase, abort_flag, p.status, 0x40u);
+            const bool ok = wait_bounded(epibar, epi_phase, abort_flag, p.status, 0x40u, p.timeout_ns);
             epi_phase ^= 1;
             return ok;
         };
@@ -644,7 +652,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
             const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * p.BN);
             if (sg.kb0 > 0) {
                 // later k-blocks of a tile another CTA finishes: fp32 partials to the workspace
-                if (!wait_bounded(&tfull[buf], (uint32_t)((i >> 1) & 1), abort_flag, p.status, 0x10u)) break;
+                if (!wait_bounded(&tfull[buf], (uint32_t)((i >> 1) & 1), abort_flag, p.status, 0x10u, p.timeout_ns)) break;
                 ptx::tc_fence_after();
                 // per 16-column chunk four planes [128 rows][4 columns]: each store of a
                 // warp covers 512 contiguous bytes
@@ -666,7 +674,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
             }
             if (staged_tb != tb) {
                 if (!v_ready) {  // every CTA's share of the down-projection is in v
-                    if (etid == 0) ok = wait_count(p.v_done, n_chunks, abort_flag, p.status, 0x80u);
+                    if (etid == 0) ok = wait_count(p.v_done, n_chunks, abort_flag, p.status, 0x80u, p.timeout_ns);
                     if (!(ok = epi_sync() && ok)) break;
                     v_ready = true;
                 }
@@ -703,7 +711,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
             // the LoRA operands of this segment, phase by phase: the MMA warp adds each
             // phase to the accumulator (between its k-blocks) and signals tfull after the last
             for (int ph = 0; p.lora && ok; ++ph) {
-                if (!(ok = wait_bounded(bfull, (uint32_t)(jf & 1), abort_flag, p.status, 0x20u))) break;
+                if (!(ok = wait_bounded(bfull, (uint32_t)(jf & 1), abort_flag, p.status, 0x20u, p.timeout_ns))) break;
                 ++jf;
                 const int nact = s_nact;
                 const int e0 = ph * p.n_slots, e1 = min(nact, e0 + p.n_slots);
@@ -850,7 +858,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
                 if (e1 >= nact) break;  // the segment's last phase
             }
             if (!ok) break;
-            if (!(ok = wait_bounded(&tfull[buf], (uint32_t)((i >> 1) & 1), abort_flag, p.status, 0x10u))) break;
+            if (!(ok = wait_bounded(&tfull[buf], (uint32_t)((i >> 1) & 1), abort_flag, p.status, 0x10u, p.timeout_ns))) break;
             ptx::tc_fence_after();
             // the CTAs after this one that hold later k-blocks of this tile
             int c_hi = cta + 1;
@@ -859,7 +867,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
                 while (c_hi < G && unit_begin(p.units, c_hi, G) < tile_end) ++c_hi;
                 if (etid == 0)
                     for (int cc = cta + 1; cc < c_hi && ok; ++cc)
-                        ok = wait_count(p.flags + cc, 1, abort_flag, p.status, 0x100u);
+                        ok = wait_count(p.flags + cc, 1, abort_flag, p.status, 0x100u, p.timeout_ns);
                 if (!(ok = epi_sync() && ok)) break;
             }
 
@@ -1113,7 +1121,7 @@ cudaError_t launch_fp8_gemm(const Fp8GemmArgs& a, cudaStream_t stream)
     if (cudaFuncGetAttributes(&fa, fp8_gemm_kernel<128, 64>) != cudaSuccess) return cudaErrorInvalidValue;
     const size_t kSmemMax = (size_t)(optin > 0 ? optin : 232448) - fa.sharedSizeBytes - 256;
     const size_t meta = align_up((size_t)p.BN * 20, 128);  // token, adapter, rank, slot, sx
-    const size_t bars = 8 * (2 * kMaxStages + 9);
+    const size_t bars = 8 * (2 * kMaxStages + 10);
     // a slot holds one adapter's B[j][128 n] as loaded, then B'[128 n][r16] in place
     const size_t slot_bytes = (size_t)p.r16 * 256;
     // V' tiles of va adapters: their token ranges are disjoint and contiguous, so their
@@ -1193,10 +1201,25 @@ cudaError_t launch_fp8_gemm(const Fp8GemmArgs& a, cudaStream_t stream)
         tmB = tmW;  // unused
     }
 
-    // one persistent CTA per SM (the partial buffers and flags are sized for that)
+    p.timeout_ns = debug_wait_limit_ns();
+    p.inject_stall = debug_inject_stall();
+    // One persistent CTA per SM (the partial buffers and flags are sized for that).
+    // The CTAs wait on one another (the down-projection count, the stream-K flags), so
+    // every CTA of the grid must be resident at once: the grid is at most the SMs times
+    // the CTAs of this kernel that fit on one SM (one, by its shared memory). A context
+    // limited to fewer SMs than the device has (an MPS share, a green context) cannot
+    // hold that grid: its CTAs would wait until the bounded waits give up.
+    const bool small_r = p.r8 <= 16;
+    auto kern = BK == 128 ? (small_r ? fp8_gemm_kernel<128, 16> : fp8_gemm_kernel<128, 64>)
+                          : (small_r ? fp8_gemm_kernel<64, 16> : fp8_gemm_kernel<64, 64>);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, smem);
+    if (e != cudaSuccess) return e;
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
     long long grid = device_sm_count();
     if (grid > p.units) grid = p.units;
-    const bool small_r = p.r8 <= 16;
     if (BK == 128)
         return small_r ? launch_t<128, 16>(p, tmW, tmX, tmB, smem, (int)grid, stream)
                        : launch_t<128, 64>(p, tmW, tmX, tmB, smem, (int)grid, stream);

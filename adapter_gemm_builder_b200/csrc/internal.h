@@ -63,6 +63,12 @@ int fp8_gemm_v_copies(int M);
 
 int device_sm_count();
 
+// Limit of the kernels' bounded waits (2 s unless a test lowered it with
+// lora_debug_set_wait_limit) and the test hook that makes one CTA wait on a
+// barrier that nothing completes.
+unsigned long long debug_wait_limit_ns();
+int debug_inject_stall();
+
 // Rows of lora_segments_t.tiles for T tokens over n_adapters.
 int max_tiles_for(int T, int n_adapters);
 // tokens per tile for a batch (LORA_DECODE_TILE_TOKENS for decode-like batches)
@@ -77,6 +83,10 @@ bool encode_tmap_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, ui
 // out-of-range box elements are filled with zeros. false on failure.
 bool encode_tmap_3d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, const uint64_t dims[3],
                     const uint64_t strides_bytes[2], const uint32_t box[3], CUtensorMapSwizzle swz);
+
+// fp8_gemm_lora_epilogue's argument checks, workspace aside (a lora_status_t).
+int fp8_gemm_check_args(const void* x, int M, int K, int N, const uint8_t* Wq, const float* w_scale,
+                        const lora_pool_t* pool, const lora_segments_t* seg, const void* y);
 
 // Slot of the device status word in lora_segments_t.counts.
 constexpr int kSegStatusSlot = 4;

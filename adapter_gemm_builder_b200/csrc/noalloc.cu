@@ -55,15 +55,26 @@ int fp8_gemm_lora_epilogue_noalloc(const void* x, int M, int K, int N, const uin
                                    const float* w_scale, const lora_pool_t* pool,
                                    const lora_segments_t* seg, void* y, lora_stream_t stream)
 {
+    // the same argument checks, and status codes, as the workspace entry point
+    const int st = lora::fp8_gemm_check_args(x, M, K, N, Wq, w_scale, pool, seg, y);
+    if (st != LORA_OK) return st;
     const size_t need = lora_workspace_size(LORA_OP_FP8_GEMM, M, K, pool);
     if (need == (size_t)-1) return LORA_ERR_INVALID_ARG;
     if (need > kNoAllocScratchBytes) return LORA_ERR_WORKSPACE;  // beyond the built-in scratch
     void* ws = scratch_on_current_device();
     if (!ws) return LORA_ERR_CUDA;
-    // the status word (first 256 bytes) must start at zero; the rest is fully
-    // rewritten by every call before it is read
-    if (cudaMemsetAsync(ws, 0, 256, (cudaStream_t)stream) != cudaSuccess) return LORA_ERR_CUDA;
+    // The status word (the first 256 bytes) starts at zero when the library is loaded
+    // and is cleared only by lora_noalloc_status, so a bounded-wait timeout of any call
+    // stays visible until it is read. Everything else the kernels read is rewritten by
+    // each call before it is read (the quantiser zeroes v and the sync words).
     return fp8_gemm_lora_epilogue(x, M, K, N, Wq, w_scale, pool, seg, y, ws, need, stream);
+}
+
+int lora_noalloc_status(lora_stream_t stream, uint32_t* detail)
+{
+    void* ws = scratch_on_current_device();
+    if (!ws) return LORA_ERR_CUDA;
+    return lora_workspace_status(ws, 256, stream, detail);
 }
 
 }  // extern "C"

@@ -66,7 +66,7 @@ constexpr int kTT = LORA_TILE_TOKENS;    // 64
 constexpr int kMaxCluster = 8;
 constexpr int kOnePhaseBytes = 8192;     // all-to-all exchange of v up to this size per CTA
 constexpr int kSmallTile = 4;            // tiles of <= 4 tokens use CUDA-core FMAs
-constexpr unsigned long long kTimeoutNs = 2000000000ull;
+constexpr unsigned long long kTimeoutNs = 2000000000ull;  // drains after an abort
 
 // Tensor maps of the pools. a[i]: A viewed as {r_max, h_in, n_slices *
 // n_adapters}, box {8 << i, 64, 1} (swizzle = the box row width);
@@ -98,6 +98,8 @@ struct SgmvParams {
     int stage_bytes; // one ring stage
     int xy_maps;     // tensor maps of x and y are valid (consecutive-row tiles use them)
     uint32_t off_rb, off_vf, off_bar;
+    unsigned long long timeout_ns;  // limit of every bounded wait (2 s unless a test lowers it)
+    int inject_stall;  // test hook: one CTA's producer first waits on a barrier nothing completes
 };
 
 __device__ __forceinline__ int round_up(int a, int b) { return (a + b - 1) / b * b; }
@@ -147,9 +149,12 @@ __device__ __forceinline__ void gather_rows(uint32_t dst, const uint16_t* src, s
 
 // Bounded wait by ONE thread; on expiry raises the CTA abort flag and the
 // status word. The clock and the abort flag are read every 256 probes only.
-template <bool kClusterScope>
+// kHonorAbort = false: the wait does not end early when another role of the
+// CTA aborted (used for the v exchange: the peers always send their bytes, and
+// a CTA may not leave while their stores into its shared memory are in flight).
+template <bool kClusterScope, bool kHonorAbort = true>
 __device__ bool wait_one(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int32_t* status,
-                         int code)
+                         int code, unsigned long long limit)
 {
     auto probe = [&]() {
         return kClusterScope ? ptx::mbar_try_wait_cluster(bar, parity) : ptx::mbar_try_wait(bar, parity);
@@ -159,8 +164,8 @@ __device__ bool wait_one(uint64_t* bar, uint32_t parity, volatile int* abort_fla
     for (unsigned n = 1;; ++n) {
         if (probe()) return true;
         if ((n & 255) == 0) {
-            if (*abort_flag) return false;
-            if (ptx::globaltimer() - t0 > kTimeoutNs) {
+            if (kHonorAbort && *abort_flag) return false;
+            if (ptx::globaltimer() - t0 > limit) {
                 *abort_flag = 1;
                 atomicOr(status, code);
                 return false;
@@ -171,12 +176,13 @@ __device__ bool wait_one(uint64_t* bar, uint32_t parity, volatile int* abort_fla
 
 // Bounded wait by a WHOLE warp (all 32 lanes must call it): lane 0 polls,
 // the others then observe the completed phase themselves (acquire).
-template <bool kClusterScope>
+template <bool kClusterScope, bool kHonorAbort = true>
 __device__ bool wait_all(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int32_t* status,
-                         int code)
+                         int code, unsigned long long limit)
 {
     bool ok = true;
-    if ((threadIdx.x & 31) == 0) ok = wait_one<kClusterScope>(bar, parity, abort_flag, status, code);
+    if ((threadIdx.x & 31) == 0)
+        ok = wait_one<kClusterScope, kHonorAbort>(bar, parity, abort_flag, status, code, limit);
     ok = __shfl_sync(0xffffffffu, ok, 0);
     if (ok && (threadIdx.x & 31) != 0)
         kClusterScope ? ptx::mbar_try_wait_cluster(bar, parity) : ptx::mbar_try_wait(bar, parity);
@@ -208,6 +214,7 @@ sgmv_kernel(const __grid_constant__ AMaps am, const SgmvParams p)
     uint64_t* empty = full + kStages;
     uint64_t* red1 = empty + kStages;
     uint64_t* red2 = red1 + 1;
+    uint64_t* stall = red2 + 1;  // test hook: never completed
     volatile int* abort_flag = &s_abort;
     int32_t* status = p.counts + kSegStatusSlot;
 
@@ -219,6 +226,7 @@ sgmv_kernel(const __grid_constant__ AMaps am, const SgmvParams p)
         }
         ptx::mbar_init(red1, 1);
         ptx::mbar_init(red2, 1);
+        ptx::mbar_init(stall, 1);
         ptx::fence_mbar_init();
     }
     __syncwarp();  // __syncthreads is an aligned barrier: warps reach it converged
@@ -332,10 +340,16 @@ sgmv_kernel(const __grid_constant__ AMaps am, const SgmvParams p)
         }
         const int xs = p.x_slice_stride ? slice : 0;
         int issued = 0;
-        for (int it = 0; it < nItems; ++it) {
+        // test hook: the first CTA of the first tile row waits, before its first copy, on
+        // a barrier that nothing completes; the bounded wait runs out and the CTA takes
+        // its abort path (not with an early A copy in flight, which that path cannot drain)
+        bool go = true;
+        if (p.inject_stall && g == 0 && slice == 0 && rank == 0 && !a_early)
+            go = wait_all<false>(stall, 0, abort_flag, status, 0x2000, p.timeout_ns);
+        for (int it = 0; it < nItems && go; ++it) {
             const int st = it % kStages;
             const uint32_t ph = (uint32_t)((it / kStages) & 1);
-            if (!wait_all<false>(&empty[st], ph ^ 1, abort_flag, status, 0x100)) break;
+            if (!wait_all<false>(&empty[st], ph ^ 1, abort_flag, status, 0x100, p.timeout_ns)) break;
             const uint32_t base = base_u + st * SB;
             // lane 0 announces the stage's tensor-map / bulk bytes before any lane issues a
             // copy; then every lane arrives once its own copies have landed (33 arrivals)
@@ -571,7 +585,7 @@ sgmv_kernel(const __grid_constant__ AMaps am, const SgmvParams p)
                 }
             }
             if (one_phase) ptx::cluster_arrive();  // phase 1: this thread's remote stores are issued
-            wait_all<true>(red1, 0, abort_flag, status, 0x200);
+            wait_all<true, false>(red1, 0, abort_flag, status, 0x200, p.timeout_ns);
             ptx::named_sync(1, kCompute);  // every thread of this CTA has sent its share
             if (one_phase) {
                 for (int i = tid; i < nt * q8; i += kCompute) {
@@ -594,7 +608,7 @@ sgmv_kernel(const __grid_constant__ AMaps am, const SgmvParams p)
                         ptx::st_async_f32x4(ptx::mapa(vf_u + off, d), s4, ptx::mapa(red2_u, d));
                 }
                 ptx::cluster_arrive();  // phase 1: this thread's remote stores are issued
-                wait_all<true>(red2, 0, abort_flag, status, 0x400);
+                wait_all<true, false>(red2, 0, abort_flag, status, 0x400, p.timeout_ns);
             }
             ptx::named_sync(1, kCompute);
             if (MODE == SGMV_SHRINK) {
@@ -627,7 +641,7 @@ sgmv_kernel(const __grid_constant__ AMaps am, const SgmvParams p)
             const int st = it % kStages;
             const uint32_t ph = (uint32_t)((it / kStages) & 1);
             const uint32_t base = base_u + st * SB;
-            const bool ok = wait_all<false>(&full[st], ph, abort_flag, status, 0x800) && !*abort_flag;
+            const bool ok = wait_all<false>(&full[st], ph, abort_flag, status, 0x800, p.timeout_ns) && !*abort_flag;
             const int k0 = k_begin + it * BK;
             const int kb = min(BK, k_begin + k_len - k0);
             const uint32_t xb = base + (uint32_t)(BK * apitch);
@@ -738,7 +752,7 @@ sgmv_kernel(const __grid_constant__ AMaps am, const SgmvParams p)
             const int st = it % kStages;
             const uint32_t ph = (uint32_t)((it / kStages) & 1);
             const uint32_t base = base_u + st * SB;
-            const bool ok = wait_all<false>(&full[st], ph, abort_flag, status, 0x800) && !*abort_flag;
+            const bool ok = wait_all<false>(&full[st], ph, abort_flag, status, 0x800, p.timeout_ns) && !*abort_flag;
             const int n0 = n_begin + (it - nK) * BN;
             const int nb = min(BN, n_begin + n_len - n0);
             const uint32_t yb = base + y_off;
@@ -910,6 +924,8 @@ cudaError_t launch_sgmv(int mode, const void* x, int64_t x_slice_stride, const l
     p.h_in = pool.h_in;
     p.h_out = pool.h_out;
     p.r_max = pool.r_max;
+    p.timeout_ns = debug_wait_limit_ns();
+    p.inject_stall = debug_inject_stall();
     // CTAs per tile: up to one per 512 columns of h_in (at most 8). When that would
     // need more than one wave of two CTAs per SM but the tile rows alone fit in one,
     // take as many per tile as keep one wave (no near-empty last wave: prefill gets 5);
@@ -944,7 +960,7 @@ cudaError_t launch_sgmv(int mode, const void* x, int64_t x_slice_stride, const l
     const size_t partials = (size_t)kComputeWarps * 8 * kSmallTile * 8 * 4;  // small-tile warp partials
     if (vf < partials) vf = partials;
     // stages (multiples of 1024 bytes, at most 32 KB) sized so that two CTAs fit on an SM
-    const size_t bars = 8 * (2 * kStages + 2);
+    const size_t bars = 8 * (2 * kStages + 3);
     const size_t fixed = rb + vf + bars + 1024;  // + base alignment slack
     const size_t budget = sgmv_smem_per_cta();
     if (budget <= fixed + (size_t)kStages * 8192) return cudaErrorInvalidConfiguration;

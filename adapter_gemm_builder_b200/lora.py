@@ -34,6 +34,7 @@ EXPORTED = [
     "lora_shrink", "lora_expand", "lora_apply", "fp8_quantize_rows", "fp8_gemm_lora_epilogue",
     "lora_status_string", "lora_version", "lora_tile_tokens", "lora_tile_tokens_for", "lora_max_tiles",
     "lora_segments_status", "fp8_gemm_lora_epilogue_noalloc", "lora_noalloc_scratch_bytes",
+    "lora_noalloc_status", "lora_debug_set_wait_limit",
 ]
 
 
@@ -95,6 +96,8 @@ def load(path: str = LIB_PATH):
             "lora_segments_status": (I, [P, P, P]),
             "fp8_gemm_lora_epilogue_noalloc": (I, [P, I, I, I, P, P, P, P, P, P]),
             "lora_noalloc_scratch_bytes": (Z, []),
+            "lora_noalloc_status": (I, [P, P]),
+            "lora_debug_set_wait_limit": (I, [ctypes.c_uint64, I]),
         }
         for name, (res, args) in sig.items():
             f = getattr(lib, name)
@@ -261,3 +264,16 @@ def fp8_gemm_lora_epilogue_noalloc(x: torch.Tensor, Wq: torch.Tensor, w_scale: t
     _check(load().fp8_gemm_lora_epilogue_noalloc(
         _ptr(x), M, K, N, _ptr(Wq), _ptr(w_scale), ctypes.byref(pool.c) if pool else None,
         ctypes.byref(seg.c) if seg else None, _ptr(y), _stream(stream)))
+
+
+def lora_noalloc_status(stream=None) -> tuple[int, int]:
+    """Read and clear the status word of the no-alloc entry point's scratch array."""
+    detail = ctypes.c_uint32(0)
+    st = load().lora_noalloc_status(_stream(stream), ctypes.byref(detail))
+    return st, detail.value
+
+
+def lora_debug_set_wait_limit(limit_ns: int, inject_stall: bool = False) -> None:
+    """Test hook: limit of the kernels' bounded waits (0 = default 2 s) and the stall
+    that makes one CTA of each later launch run out its wait."""
+    _check(load().lora_debug_set_wait_limit(int(limit_ns), 1 if inject_stall else 0))

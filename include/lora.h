@@ -179,7 +179,8 @@ LORA_API int lora_build_segments(const int32_t* ids, int T, int n_adapters, cons
                         int sync_check, lora_stream_t stream);
 
 /*
- * Shrink (down-projection), for every slice s and token t with adapter a:
+ * Shrink (down-projection; the x_i.A_i half of the added term in the Punica
+ * README, "How?"), for every slice s and token t with adapter a:
  *   v[s][t][j] = sum_k x[s][t][k] * A[s][a][k][j]   for j < r_a  (fp32 accumulate)
  *   v[s][t][j] = 0                                    for r_a <= j < r_max.
  * Rows of tokens without an adapter are not written.
@@ -194,7 +195,9 @@ LORA_API int lora_shrink(const void* x, int64_t x_slice_stride, const lora_pool_
                 lora_stream_t stream);
 
 /*
- * Expand (up-projection), in place on y, for every slice s and token t with adapter a:
+ * Expand (up-projection; the (x_i.A_i).B_i half of the added term in the
+ * Punica README, "How?", added to the base output), in place on y, for every
+ * slice s and token t with adapter a:
  *   y[s][t][n] = bf16( fp32(y[s][t][n]) + s_a * sum_{j < r_a} v[s][t][j] * B[s][a][j][n] )
  * (one rounding, to nearest even); rows of tokens without an adapter are untouched.
  *   v  fp32 [n_slices][T][r_max];  y bf16 [n_slices][T][h_out] (in/out).
@@ -204,7 +207,8 @@ LORA_API int lora_expand(const float* v, const lora_pool_t* pool, const lora_seg
                 void* ws, size_t ws_bytes, lora_stream_t stream);
 
 /*
- * Shrink then expand (y += s_a * (x.A_a).B_a), with v kept on chip in fp32:
+ * Shrink then expand (y += s_a * (x.A_a).B_a; the whole added term of the
+ * Punica README, "How?", for a batch of many adapters), with v kept on chip in fp32:
  * one kernel launch, no workspace. Arguments as lora_shrink / lora_expand.
  */
 LORA_API int lora_apply(const void* x, int64_t x_slice_stride, const lora_pool_t* pool,
@@ -238,6 +242,12 @@ LORA_API int fp8_quantize_rows(const void* x, int M, int K, uint8_t* xq, float* 
  *   seg: required when pool != NULL (built for these M tokens); may be NULL otherwise.
  *   ws: lora_workspace_size(LORA_OP_FP8_GEMM, M, K, pool) bytes.
  * Limits: K % 16 == 0, N % 8 == 0, M >= 1.
+ * The GEMM is a persistent grid of one CTA per SM whose CTAs wait on one
+ * another (the down-projection count, stream-K partials), so all of them must
+ * be resident at once: the context needs every SM of the device. Where fewer
+ * are available (an MPS share, a green context, another kernel holding SMs
+ * for long), the waits give up after 2 s and lora_workspace_status reports
+ * LORA_ERR_TIMEOUT.
  */
 LORA_API int fp8_gemm_lora_epilogue(const void* x, int M, int K, int N, const uint8_t* Wq,
                            const float* w_scale, const lora_pool_t* pool,
@@ -249,26 +259,47 @@ LORA_API int fp8_gemm_lora_epilogue(const void* x, int M, int K, int N, const ui
  * (the pages have no counterpart of this call): for example a plugin inside
  * a serving engine that plans all device memory itself and only hands over
  * inputs and outputs, or a hot path that must not call cudaMalloc, which can
- * synchronise the device. Same arguments and results as
+ * synchronise the device. Same arguments, checks and results as
  * fp8_gemm_lora_epilogue, minus the workspace: the scratch space lives in a
  * fixed array of lora_noalloc_scratch_bytes() (8 MiB) inside the library's
  * own device memory, held by every GPU that loads the library until the
  * process exits. Calls whose workspace would exceed it return
- * LORA_ERR_WORKSPACE. The call allocates nothing (no cudaMalloc or
- * cudaFree); it clears the array's status word with a stream-ordered memset.
+ * LORA_ERR_WORKSPACE (after the other argument checks). The call allocates
+ * nothing (no cudaMalloc or cudaFree).
  * The first call on each device looks up the array's device address (with
  * that device current); make that first call before any stream capture.
  * Every call shares the one array: calls that may overlap on the GPU (other
  * streams, other threads) race on it and must be ordered by the caller.
- * lora_workspace_status() does not apply; a bounded-wait timeout is not
- * reported by this entry point.
+ * The array's status word is zero when the library loads and only
+ * lora_noalloc_status clears it: a bounded-wait timeout of any call since the
+ * last query stays visible until it is read.
  */
 LORA_API int fp8_gemm_lora_epilogue_noalloc(const void* x, int M, int K, int N, const uint8_t* Wq,
                                             const float* w_scale, const lora_pool_t* pool,
                                             const lora_segments_t* seg, void* y, lora_stream_t stream);
 
+/*
+ * Read and clear the status word of the built-in scratch array on the current
+ * device (fp8_gemm_lora_epilogue_noalloc's counterpart of
+ * lora_workspace_status): synchronises `stream`; LORA_OK, or LORA_ERR_TIMEOUT
+ * if a call since the last query gave up on a bounded wait (its output is
+ * then undefined). *detail (host, may be NULL) receives the raw word.
+ */
+LORA_API int lora_noalloc_status(lora_stream_t stream, uint32_t* detail);
+
 /* Bytes of the built-in scratch array used by fp8_gemm_lora_epilogue_noalloc. */
 LORA_API size_t lora_noalloc_scratch_bytes(void);
+
+/*
+ * Test hook for the failure path (not for production use): limit_ns sets the
+ * limit of every bounded device-side wait of later launches (1 us .. 2 s;
+ * 0 restores the default of 2 s); inject_stall = 1 makes one CTA of each
+ * later SGMV (non-decode tiles) and FP8 GEMM launch first wait on a barrier
+ * that nothing completes, so that wait runs out, the kernel takes its abort
+ * path, returns, and the status calls report LORA_ERR_TIMEOUT. Process-wide;
+ * LORA_ERR_INVALID_ARG for values outside those ranges.
+ */
+LORA_API int lora_debug_set_wait_limit(uint64_t limit_ns, int inject_stall);
 
 /* Static string for a status code. */
 LORA_API const char* lora_status_string(int status);

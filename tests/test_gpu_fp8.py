@@ -43,6 +43,9 @@ def test_quantize_rows_bitexact(M, K, std):
     assert np.array_equal(xq.cpu().numpy(), want_q)
 
 
+ORACLE_QUANT_MAX = 1 << 23  # weights up to this many codes are quantised by the oracle
+
+
 def _fp8_case(M, K, N, n_adapters=5, r=16, lora=True, seed=0, kind="zipf", none_frac=0.1,
               rank_choices=None):
     rng = np.random.default_rng(seed + 1000)
@@ -50,7 +53,15 @@ def _fp8_case(M, K, N, n_adapters=5, r=16, lora=True, seed=0, kind="zipf", none_
     p = wl.fp8_problem(M, K=K, N=N, n_adapters=n_adapters, r=r, seed=seed, ids_kind=kind,
                        none_frac=none_frac, W=W, rank_choices=rank_choices)
     x = dev_bf16(p.x)
-    Wq, sw = _quantize_gpu(p.W)
+    if N * K <= ORACLE_QUANT_MAX:
+        # the weight codes and scales come from the oracle (the GPU quantiser has its own
+        # bit-exact test), so nothing the oracle consumes comes from the CUDA path
+        Wq_o, sw_o = oracle.quantize_rows(p.W)
+        Wq, sw = dev(Wq_o), dev(sw_o)
+    else:
+        # the full-size weight (235 M codes) is quantised on the GPU; the tests that use
+        # it check the sampled rows bit-exact against the oracle before using them
+        Wq, sw = _quantize_gpu(p.W)
     y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
     pool = seg = None
     if lora:
@@ -161,3 +172,30 @@ def test_fp8_gemm_rejects_unaligned_y():
     L.fp8_gemm_lora_epilogue(x, Wq, sw, None, None, y_buf[:-1].view(M, N), ws)
     torch.cuda.synchronize()
     assert torch.count_nonzero(y_buf[:-1]).item() == 0  # all-zero x: y = 0
+
+
+@pytest.mark.parametrize("kind", ["all_none", "out_of_range"])
+def test_fp8_gemm_lora_ids_without_adapter(kind):
+    """Every token without an adapter (pure base GEMM through the LoRA path), and ids
+    outside [-1, n_adapters) (served as -1): the oracle leaves those rows base-only."""
+    M, K, N, n_ad = 48, 256, 384, 4
+    rng = np.random.default_rng(77)
+    W = wl.normal_bf16(rng, (N, K), 1.0 / np.sqrt(K))
+    p = wl.fp8_problem(M, K=K, N=N, n_adapters=n_ad, r=16, seed=77, W=W)
+    if kind == "all_none":
+        p.ids[:] = -1
+    else:
+        p.ids[:] = rng.integers(-3, n_ad + 3, size=M).astype(np.int32)
+    Wq_o, sw_o = oracle.quantize_rows(p.W)
+    pool = L.Pool(dev_bf16(p.A), dev_bf16(p.B), dev(p.ranks), dev(p.scales))
+    seg = L.Segments(M, n_ad)
+    L.lora_build_segments(dev(p.ids), n_ad, seg)
+    ws = L.workspace(L.LORA_OP_FP8_GEMM, M, K, pool)
+    y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+    L.fp8_gemm_lora_epilogue(dev_bf16(p.x), dev(Wq_o), dev(sw_o), pool, seg, y, ws)
+    torch.cuda.synchronize()
+    assert L.lora_workspace_status(ws)[0] == L.LORA_OK
+    rows = np.repeat(np.arange(M), N).astype(np.int32)
+    cols = np.tile(np.arange(N), M).astype(np.int32)
+    want = _oracle_fp8(p, Wq_o, sw_o, rows, cols, True).reshape(M, N)
+    assert_close(f64(host_bf16_bits(y)), want, TOL_FP8, f"fp8 ids {kind}")

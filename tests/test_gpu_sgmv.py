@@ -266,3 +266,89 @@ def test_many_tenants_full():
     L.lora_apply(d.x, d.pool, d.seg, y)
     torch.cuda.synchronize()
     assert_close(f64(host_bf16_bits(y)), oracle_apply(p), TOL_BF16, "many_tenants")
+
+
+# ------------------------------------------------------------------ ids without an adapter
+
+@pytest.mark.parametrize("T,n", [(36, 32), (150, 6)])
+def test_apply_all_ids_none_leaves_y_untouched(T, n):
+    """No token has an adapter (decode-like and general batches): y stays bit-exact."""
+    p = _small(51, T=T, n_adapters=n, h_in=512, h_out=264, r_max=16, rank_choices=(16,))
+    p.ids[:] = -1
+    d = DeviceProblem(p)
+    y = d.y_in()
+    L.lora_apply(d.x, d.pool, d.seg, y)
+    torch.cuda.synchronize()
+    assert np.array_equal(host_bf16_bits(y), p.y_in)
+    assert seg_counts(d.seg)[:2] == [0, 0]
+
+
+@pytest.mark.parametrize("T,n", [(40, 24), (300, 7)])
+def test_apply_out_of_range_ids_served_as_none(T, n):
+    """Ids outside [-1, n_adapters) are counted as bad and served as -1."""
+    p = _small(52, T=T, n_adapters=n, h_in=512, h_out=264, r_max=16, rank_choices=(8, 16))
+    rng = np.random.default_rng(52)
+    p.ids[:] = rng.integers(-4, n + 4, size=T).astype(np.int32)
+    d = DeviceProblem(p)
+    y = d.y_in()
+    L.lora_apply(d.x, d.pool, d.seg, y)
+    torch.cuda.synchronize()
+    bad = (p.ids < -1) | (p.ids >= n)
+    assert seg_counts(d.seg)[2] == int(bad.sum())
+    assert_close(f64(host_bf16_bits(y)), oracle_apply(p), TOL_BF16, "out-of-range ids")
+    none = (p.ids < 0) | (p.ids >= n)
+    assert np.array_equal(host_bf16_bits(y)[:, none], p.y_in[:, none])
+
+
+def seg_counts(seg):
+    return seg.counts.cpu().numpy().tolist()
+
+
+# ------------------------------------------------------------------ whole layer
+
+def _whole_layer(p, W, rows):
+    """y = x.W^T (the harness's base GEMM: torch bf16 on the GPU, stored as bf16) plus
+    lora_apply, against the oracle's y_ref = sum_k x.W + s.(x.A).B in fp64, on the
+    given token rows of every slice."""
+    d = DeviceProblem(p)
+    xs = d.x
+    Wd = dev_bf16(W)
+    y = torch.stack([xs[s] @ Wd[s].t() for s in range(p.n_slices)]).contiguous()
+    L.lora_apply(d.x, d.pool, d.seg, y)
+    torch.cuda.synchronize()
+    got = f64(host_bf16_bits(y))[:, rows]
+    zeros = np.zeros((len(rows), p.h_out), np.uint16)
+    cols = np.tile(np.arange(p.h_out), len(rows)).astype(np.int32)
+    rr = np.repeat(np.asarray(rows), p.h_out).astype(np.int32)
+    for s in range(p.n_slices):
+        base = oracle.linear_bf16_sampled(p.x[s], W[s], rr, cols).reshape(len(rows), p.h_out)
+        lora = oracle.lora_apply(p.x[s][rows], p.A[s], p.B[s], p.ranks, p.scales, p.ids[rows], zeros)
+        assert_close(got[s], base + lora, TOL_BF16, f"{p.name} whole layer, slice {s}")
+
+
+def test_whole_layer_sgmv_tiny():
+    p = wl.sgmv_tiny()
+    _whole_layer(p, p.W, np.arange(p.T))
+
+
+def test_whole_layer_bgmv_decode():
+    p = wl.bgmv_decode()
+    W = wl.weight_bf16(p.h_out, p.h_in, seed=101)[None]
+    _whole_layer(p, W, np.arange(p.T))
+
+
+def test_whole_layer_sgmv_prefill_sampled():
+    p = wl.sgmv_prefill()
+    W = wl.weight_bf16(p.h_out, p.h_in, seed=102)[None]
+    starts = np.concatenate([[0], np.cumsum(np.bincount(p.ids))])
+    rng = np.random.default_rng(2)
+    rows = np.unique(np.concatenate([rng.choice(p.T, 12, replace=False), starts[1:-1], starts[1:] - 1]))
+    _whole_layer(p, W, rows)
+
+
+def test_whole_layer_many_tenants_sampled():
+    p = wl.many_tenants()
+    W = np.stack([wl.weight_bf16(p.h_out, p.h_in, seed=103 + s) for s in range(p.n_slices)])
+    rng = np.random.default_rng(4)
+    rows = np.sort(rng.choice(p.T, 24, replace=False))
+    _whole_layer(p, W, rows)

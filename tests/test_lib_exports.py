@@ -186,3 +186,11 @@ def test_max_tiles_bounds_every_id_mix(lib):
             seg = oracle.build_segments(ids.astype(np.int32), n)
             rows = expected_tiles(seg["indptr"], seg["active"], seg["counts"][1], t)
             assert len(rows) <= bound, (T, n, t)
+
+
+def test_debug_wait_limit_validates_and_restores(lib):
+    assert lib.lora_debug_set_wait_limit(999, 0) == L.LORA_ERR_INVALID_ARG       # below 1 us
+    assert lib.lora_debug_set_wait_limit(3_000_000_000, 0) == L.LORA_ERR_INVALID_ARG  # above 2 s
+    assert lib.lora_debug_set_wait_limit(1_000_000, 2) == L.LORA_ERR_INVALID_ARG
+    assert lib.lora_debug_set_wait_limit(1_000_000, 1) == L.LORA_OK
+    assert lib.lora_debug_set_wait_limit(0, 0) == L.LORA_OK                      # default again
