@@ -234,10 +234,15 @@ def lora_expand(v: torch.Tensor, pool: Pool, seg: Segments, y: torch.Tensor, str
 
 
 def lora_apply(x: torch.Tensor, pool: Pool, seg: Segments, y: torch.Tensor, stream=None,
-               x_slice_stride: int | None = None) -> None:
+               x_slice_stride: int | None = None, ws: torch.Tensor | None = None) -> None:
+    """y += s_a (x.A_a).B_a; ws: a workspace of lora_workspace_size(LORA_OP_APPLY, T, 0, pool)
+    bytes (allocated here when None; pass one to keep the call free of allocation)."""
     xs = _slice_stride(x, pool) if x_slice_stride is None else x_slice_stride
-    _check(load().lora_apply(_ptr(x), xs, ctypes.byref(pool.c), ctypes.byref(seg.c), _ptr(y), None,
-                             0, _stream(stream)))
+    if ws is None:
+        n = lora_workspace_size(LORA_OP_APPLY, seg.T, 0, pool)
+        ws = workspace(LORA_OP_APPLY, seg.T, 0, pool, device=y.device, stream=stream) if n else None
+    _check(load().lora_apply(_ptr(x), xs, ctypes.byref(pool.c), ctypes.byref(seg.c), _ptr(y),
+                             _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream)))
 
 
 def fp8_quantize_rows(x: torch.Tensor, xq: torch.Tensor, sx: torch.Tensor, stream=None) -> None:

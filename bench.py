@@ -1,19 +1,24 @@
 #!/usr/bin/env python
 """Benchmark of the multi-tenant LoRA hot path on B200.
 
-Default workload (N=1): the BGMV decode batch -- 36 tokens, 32 of them each
-with its own adapter (32 adapters, rank 16) and 4 with id -1, h_in = h_out =
-4096 (Llama-2-7B q_proj). One step is one pass of the hot path over one batch:
-the segment build (lora_build_segments) and the fused shrink+expand
-(lora_apply). Steps rotate over enough copies of the inputs and adapter pools
-that the working set exceeds the 126 MB L2, and run as CUDA-graph replays.
+Headline workload (N=1): many tenants -- 512 decode tokens over 256 adapters of
+ranks {8, 16, 32, 64} (pool padded to 64), Zipf(1.1) ids with 5% at -1,
+h_in = h_out = 5120 (Llama-2-13B o_proj shape), the q/k/v/o projections applied
+in one call. One step is one pass of the hot path over one batch: the segment
+build (lora_build_segments) and the fused shrink+expand (lora_apply). Steps
+rotate over enough copies of the inputs and adapter pools that the working set
+exceeds the 126 MB L2 (the label says so, or says "L2-resident" when it cannot),
+and run as CUDA-graph replays.
 
 Printed (rank 0): one JSON line with the metric (GB/s of algorithmic bytes),
 the roofline of the dominant kernel against the measured HBM peak, the
 end-to-end number through the public API with host buffers, the fp64 CPU
-oracle timed on the host, SM clocks sampled during the timed region, and the
-fused FP8 GEMM + LoRA epilogue at M = 16/64/256 (K 8192, N 28672): TFLOP/s,
-us per call and the overhead over the same GEMM without LoRA.
+oracle timed on the host (all cores and one core, with the CPU model), SM
+clocks sampled during the timed region, the other workloads of the method
+(BGMV decode, SGMV prefill, SGMV tiny, and Punica's Identical and Uniform
+popularity settings) each with its own roofline, and the fused FP8 GEMM +
+LoRA epilogue at M = 16/64/256 (K 8192, N 28672): TFLOP/s, us per call and the
+overhead over the same GEMM without LoRA.
 
 Multi-GPU: one process per GPU (torchrun); each rank runs an independent
 replica of the workload (no collective on the data path), value = all ranks'
@@ -48,15 +53,15 @@ FALLBACK_BF16 = 1590.0
 def parse_args():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=64000)
-    ap.add_argument("--warmup", type=int, default=320)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="bgmv_decode",
-                    choices=["bgmv_decode", "sgmv_tiny", "sgmv_prefill", "many_tenants"])
+    ap.add_argument("--workload", default="many_tenants", choices=list(WORKLOADS))
+    ap.add_argument("--no-extras", action="store_true", help="skip the other workloads")
     ap.add_argument("--no-fp8", action="store_true", help="skip the FP8 GEMM + LoRA section")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
-    ap.add_argument("--e2e-steps", type=int, default=2000)
+    ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--fp8-only", action="store_true",
                     help="run only the FP8 GEMM + LoRA section and print its JSON")
     ap.add_argument("--fp8-m", type=int, nargs="+", default=[16, 64, 256])
@@ -66,10 +71,25 @@ def parse_args():
 
 # ------------------------------------------------------------------ workloads and byte counts
 
+WORKLOADS = {
+    # name: (generator, keyword arguments)
+    "many_tenants": ("many_tenants", {}),
+    "bgmv_decode": ("bgmv_decode", {}),
+    "sgmv_prefill": ("sgmv_prefill", {}),
+    "sgmv_tiny": ("sgmv_tiny", {}),
+    # Punica's popularity settings on the same shapes: Identical (every token on one
+    # adapter, BGMV decode shapes) and Uniform (ids uniform over the adapters, many-tenant shapes)
+    "identical": ("bgmv_decode", {"ids_kind": "identical"}),
+    "uniform": ("many_tenants", {"ids_kind": "uniform"}),
+}
+
+
 def make_problem(name):
     from adapter_gemm_builder_b200 import workloads as wl
-    return {"bgmv_decode": wl.bgmv_decode, "sgmv_tiny": wl.sgmv_tiny,
-            "sgmv_prefill": wl.sgmv_prefill, "many_tenants": wl.many_tenants}[name]()
+    gen, kw = WORKLOADS[name]
+    p = getattr(wl, gen)(**kw)
+    p.name = name
+    return p
 
 
 def apply_bytes(p, rows=None, col_frac=1.0):
@@ -314,23 +334,30 @@ class _Events:
                                                 ctypes.c_void_p(stream.cuda_stream), 1) == 0
 
 
-def run_ours(args):
+def apply_launches():
+    """Kernels of this library one lora_apply launches (the bench counts them)."""
+    return 1
+
+
+def time_apply(p, dev, steps, warmup, stream, ext, world=1, clocks=None):
+    """Time `steps` steps (segment build + lora_apply) of workload p on device dev.
+    Inputs rotate over R copies whose total exceeds 2.5x the L2 when that takes at
+    most 64 copies (else the label says the working set is L2-resident). Returns
+    a dict with the step time (max over ranks), the apply's own time from events
+    around each launch in the last replay, and the labels."""
     import numpy as np
     import torch
 
     from adapter_gemm_builder_b200 import lora as L
-
-    rank, world, local = dist_setup(args)
-    torch.cuda.set_device(local)
-    L.load()
-    dev = torch.device("cuda", local)
-    hbm_peak, bf16_peak, bf16_sust, peak_src = measured_peaks()
-
-    p = make_problem(args.workload)
-    set_bytes = (p.A.nbytes + p.B.nbytes) // max(1, p.n_adapters) * max(1, len(np.unique(p.ids[p.ids >= 0]))) \
+    act = np.unique(p.ids[p.ids >= 0])
+    set_bytes = (p.A.nbytes + p.B.nbytes) // max(1, p.n_adapters) * max(1, len(act)) \
         + p.x.nbytes + p.y_in.nbytes
-    R = int(min(64, max(1, math.ceil(2.5 * L2_BYTES / max(set_bytes, 1)))))
-    bytes_step = apply_bytes(p)
+    want_r = math.ceil(2.5 * L2_BYTES / max(set_bytes, 1))
+    R = int(min(64, max(1, want_r)))
+    l2_label = (f"rotating {R} input sets ({R * set_bytes / 2**20:.0f} MiB > 2.5 x 126 MB L2)"
+                if R == want_r else
+                f"L2-resident: {R} rotating input sets of {set_bytes / 2**20:.2f} MiB "
+                f"({R * set_bytes / 2**20:.0f} MiB < 126 MB L2)")
 
     def to_dev(a):
         return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
@@ -343,16 +370,14 @@ def run_ours(args):
         d = {key: (v.clone() if k else v) for key, v in base.items()}
         d["pool"] = L.Pool(d["A"], d["B"], d["ranks"], d["scales"])
         d["seg"] = L.Segments(p.T, p.n_adapters, device=dev)
+        d["ws"] = L.workspace(L.LORA_OP_APPLY, p.T, 0, d["pool"], device=dev)
         sets.append(d)
-
-    stream = torch.cuda.Stream(device=dev)
-    ext = _Events()
 
     def step(d):
         L.lora_build_segments(d["ids"], p.n_adapters, d["seg"])
-        L.lora_apply(d["x"], d["pool"], d["seg"], d["y"])
+        L.lora_apply(d["x"], d["pool"], d["seg"], d["y"], ws=d["ws"])
 
-    K, W = args.steps, max(3, args.warmup)
+    K, W = steps, max(3, warmup)
     nfull, rem = divmod(K, R)
     ev_a = [torch.cuda.Event(enable_timing=True) for _ in range(R)]
     ev_b = [torch.cuda.Event(enable_timing=True) for _ in range(R)]
@@ -376,7 +401,7 @@ def run_ours(args):
             for k, d in enumerate(sets):
                 L.lora_build_segments(d["ids"], p.n_adapters, d["seg"])
                 inner_ok &= ext.record_external(ev_a[k], cs)
-                L.lora_apply(d["x"], d["pool"], d["seg"], d["y"])
+                L.lora_apply(d["x"], d["pool"], d["seg"], d["y"], ws=d["ws"])
                 inner_ok &= ext.record_external(ev_b[k], cs)
         g_rem = None
         if rem:
@@ -384,17 +409,13 @@ def run_ours(args):
             with torch.cuda.graph(g_rem, stream=stream):
                 for d in sets[:rem]:
                     step(d)
-        # warm-up (untimed): W steps
-        for _ in range(math.ceil(W / R)):
+        for _ in range(math.ceil(W / R)):  # warm-up (untimed): >= W steps
             g_full.replay()
         g_inst.replay()
         stream.synchronize()
 
-    try:
-        clocks = ClockSampler("GPU-" + str(torch.cuda.get_device_properties(dev).uuid))
-    except Exception:
-        clocks = ClockSampler(str(local))
-    clocks.start()
+    if clocks is not None:
+        clocks.start()
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     dist_barrier(world)
     torch.cuda.synchronize()
@@ -409,12 +430,11 @@ def run_ours(args):
     torch.cuda.synchronize()
     t_host1 = time.time()
     dist_barrier(world)
-    clk = clocks.stop(t_host0, t_host1)
+    clk = clocks.stop(t_host0, t_host1) if clocks is not None else None
     ms = start.elapsed_time(end)
     ms_max = dist_max(ms, world)
+    statuses = [L.lora_segments_status(d["seg"])[0] for d in sets]
 
-    # dominant kernel: lora_apply, events around each launch inside the timed region
-    kernel_ms = None
     timing_src = "events around each lora_apply launch in the last graph replay of the timed region"
     if inner_ok and nfull > 0:
         kernel_ms = statistics.mean(ev_a[k].elapsed_time(ev_b[k]) for k in range(R))
@@ -424,7 +444,7 @@ def run_ours(args):
         with torch.cuda.stream(stream):
             with torch.cuda.graph(g_k, stream=stream):
                 for d in sets:
-                    L.lora_apply(d["x"], d["pool"], d["seg"], d["y"])
+                    L.lora_apply(d["x"], d["pool"], d["seg"], d["y"], ws=d["ws"])
             for _ in range(3):
                 g_k.replay()
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -434,43 +454,129 @@ def run_ours(args):
             b.record(stream)
         torch.cuda.synchronize()
         kernel_ms = a.elapsed_time(b) / (20 * R)
+    return dict(ms_max=ms_max, kernel_ms=kernel_ms, R=R, l2=l2_label, timing=timing_src,
+                clocks=clk, sets=sets, status_ok=all(st == L.LORA_OK for st in statuses),
+                launch=f"CUDA graph of {R} steps")
 
-    value = bytes_step * K * world / (ms_max / 1e3) / 1e9
-    achieved = bytes_step / (kernel_ms / 1e3) / 1e9
-    traffic = profiled_traffic("sgmv.cu", args.workload)
-    roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                "frac": achieved / hbm_peak, "traffic": traffic,
-                "kernel": "sgmv_kernel<APPLY> (lora_apply)", "kernel_us": kernel_ms * 1e3,
-                "algorithmic_bytes_per_launch": bytes_step,
-                "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs, burst copy)",
-                "timing": timing_src}
+
+def roofline_apply(p, t, hbm_peak, peak_src, workload):
+    bytes_step = apply_bytes(p)
+    achieved = bytes_step / (t["kernel_ms"] / 1e3) / 1e9
+    return {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+            "frac": achieved / hbm_peak, "traffic": profiled_traffic("sgmv.cu", workload),
+            "kernel": "lora_apply (sgmv kernels)", "kernel_us": t["kernel_ms"] * 1e3,
+            "algorithmic_bytes_per_launch": bytes_step,
+            "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs, burst copy)",
+            "timing": t["timing"]}
+
+
+def run_ours(args):
+    import torch
+
+    from adapter_gemm_builder_b200 import lora as L
+
+    rank, world, local = dist_setup(args)
+    torch.cuda.set_device(local)
+    L.load()
+    dev = torch.device("cuda", local)
+    hbm_peak, bf16_peak, bf16_sust, peak_src = measured_peaks()
+    stream = torch.cuda.Stream(device=dev)
+    ext = _Events()
+
+    p = make_problem(args.workload)
+    bytes_step = apply_bytes(p)
+    try:
+        clocks = ClockSampler("GPU-" + str(torch.cuda.get_device_properties(dev).uuid))
+    except Exception:
+        clocks = ClockSampler(str(local))
+    t = time_apply(p, dev, args.steps, args.warmup, stream, ext, world, clocks)
+    K, W = args.steps, max(3, args.warmup)
+    value = bytes_step * K * world / (t["ms_max"] / 1e3) / 1e9
+    roofline = roofline_apply(p, t, hbm_peak, peak_src, args.workload)
 
     # end to end through the public API with host buffers
-    e2e = run_e2e(args, p, sets[0], stream, bytes_step)
+    e2e = run_e2e(args, p, t["sets"][0], stream, bytes_step)
+    del t["sets"]
+
+    # the other workloads of the method, each with its own roofline (not the headline)
+    extras = {}
+    if not args.no_extras:
+        for name in WORKLOADS:
+            if name == args.workload:
+                continue
+            q = make_problem(name)
+            tq = time_apply(q, dev, 200, 10, stream, ext, world, None)
+            del tq["sets"]
+            extras[name] = {
+                "config": workload_config(q, name), "l2": tq["l2"],
+                "gb_per_s_step": apply_bytes(q) * 200 / (tq["ms_max"] / 1e3) / 1e9,
+                "us_per_step": tq["ms_max"] * 1e3 / 200,
+                "roofline": roofline_apply(q, tq, hbm_peak, peak_src, name),
+                "status_ok": tq["status_ok"]}
 
     fp8 = None if args.no_fp8 else run_fp8(args, dev, stream, hbm_peak, bf16_peak, bf16_sust, peak_src)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, cores, n = cpu_oracle_throughput(p, args.cpu_seconds)
-        cpu = {"value": v, "unit": "GB/s", "cores": cores, "kind": "oracle",
-               "sample": f"the whole batch ({p.T} tokens, {p.n_slices} slice(s)) x {n} repetitions"}
+        cpu = cpu_baseline(p, args.cpu_seconds)
 
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": K,
-            "warmup": W, "ms_per_step": ms_max / K, "higher_is_better": True, "scaling": "weak",
+            "warmup": W, "ms_per_step": t["ms_max"] / K, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {**workload_config(p, args.workload),
-                       "l2": f"rotating {R} input sets ({R * set_bytes / 2**20:.0f} MiB > 126 MB L2)",
-                       "launch": f"CUDA graph of {R} steps", "parallelism": f"replicas x{world}"},
-            "roofline": roofline, "e2e": e2e, "gpu_launches": 2 * K, "clocks": clk,
-            "cpu_baseline": cpu, "fp8_gemm_lora": fp8,
+            "config": {**workload_config(p, args.workload), "l2": t["l2"], "launch": t["launch"],
+                       "parallelism": f"replicas x{world}"},
+            "roofline": roofline, "e2e": e2e, "gpu_launches": (1 + apply_launches()) * K,
+            "clocks": t["clocks"], "status_ok": t["status_ok"],
+            "cpu_baseline": cpu, "workloads": extras, "fp8_gemm_lora": fp8,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
+
+
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def cpu_baseline(p, seconds):
+    """The fp64 oracle as it stands, on this host: all cores on the whole batch for
+    about `seconds`, and one core on a bounded sample (a few tokens, all slices)."""
+    import numpy as np
+
+    import oracle
+    all_cores = oracle.num_threads()
+    v_all, _, n = cpu_oracle_throughput(p, seconds)
+    oracle.set_num_threads(1)
+    try:
+        rows = np.nonzero(p.ids >= 0)[0][:8]
+        t0 = time.perf_counter()
+        reps = 0
+        while True:
+            for s in range(p.n_slices):
+                oracle.lora_apply(p.x[s][rows], p.A[s], p.B[s], p.ranks, p.scales, p.ids[rows],
+                                  p.y_in[s][rows])
+            reps += 1
+            if time.perf_counter() - t0 >= seconds / 2:
+                break
+        dt = time.perf_counter() - t0
+        v_one = apply_bytes(p, rows=rows) * reps / dt / 1e9
+    finally:
+        oracle.set_num_threads(all_cores)
+    return {"value": v_all, "unit": "GB/s", "cores": all_cores, "kind": "oracle",
+            "sample": f"the whole batch ({p.T} tokens, {p.n_slices} slice(s)) x {n} repetitions",
+            "cpu_model": cpu_model(),
+            "one_core": {"value": v_one, "unit": "GB/s", "cores": 1,
+                         "sample": f"{len(rows)} tokens with an adapter, all slices, x {reps} repetitions"}}
 
 
 def run_e2e(args, p, d, stream, bytes_step):
@@ -519,7 +625,7 @@ def run_e2e(args, p, d, stream, bytes_step):
                 ev_up[k].record(up)
             stream.wait_event(ev_up[k])
             L.lora_build_segments(iv, p.n_adapters, d["seg"])
-            L.lora_apply(xv, d["pool"], d["seg"], yv)
+            L.lora_apply(xv, d["pool"], d["seg"], yv, ws=d["ws"])
             ev_run[k].record(stream)
             with torch.cuda.stream(down):
                 down.wait_event(ev_run[k])
@@ -574,25 +680,39 @@ def run_fp8(args, dev, stream, hbm_peak, bf16_peak, bf16_sust, peak_src):
     for M in args.fp8_m:
         q = wl.fp8_problem(M, K=K, N=N, n_adapters=n_ad, r=r, seed=3, W=np.zeros((1, 1), np.uint16))
         tb = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
-        x = tb(q.x)
-        pool = L.Pool(tb(q.A), tb(q.B), torch.from_numpy(q.ranks).to(dev),
-                      torch.from_numpy(q.scales).to(dev))
-        seg = L.Segments(M, n_ad, device=dev)
-        ids = torch.from_numpy(q.ids).to(dev)
-        L.lora_build_segments(ids, n_ad, seg)
-        y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
-        ws = L.workspace(L.LORA_OP_FP8_GEMM, M, K, pool, device=dev)
-        ws0 = L.workspace(L.LORA_OP_FP8_GEMM, M, K, None, device=dev)
+        act = np.unique(q.ids)
+        lora_bytes = int(len(act)) * r * (K + N) * 2 + M * r * 4
+        # the token activations, the adapters and y rotate over enough copies to pass
+        # the L2 (W, 235 MB, is read once per call anyway)
+        set_bytes = q.x.nbytes + q.A.nbytes + q.B.nbytes + M * N * 2
+        R = int(min(32, max(2, math.ceil(2.5 * L2_BYTES / set_bytes))))
+        base = dict(x=tb(q.x), A=tb(q.A), B=tb(q.B), ids=torch.from_numpy(q.ids).to(dev),
+                    ranks=torch.from_numpy(q.ranks).to(dev), scales=torch.from_numpy(q.scales).to(dev))
+        sets = []
+        for k in range(R):
+            d = {key: (v.clone() if k else v) for key, v in base.items()}
+            d["pool"] = L.Pool(d["A"], d["B"], d["ranks"], d["scales"])
+            d["seg"] = L.Segments(M, n_ad, device=dev)
+            L.lora_build_segments(d["ids"], n_ad, d["seg"])
+            d["y"] = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+            d["ws"] = L.workspace(L.LORA_OP_FP8_GEMM, M, K, d["pool"], device=dev)
+            d["ws0"] = L.workspace(L.LORA_OP_FP8_GEMM, M, K, None, device=dev)
+            sets.append(d)
         res = {}
-        for tag, pl, sg, w in (("lora", pool, seg, ws), ("base", None, None, ws0)):
+        for tag in ("lora", "base"):
+            def call(d):
+                if tag == "lora":
+                    L.fp8_gemm_lora_epilogue(d["x"], Wq, sw, d["pool"], d["seg"], d["y"], d["ws"])
+                else:
+                    L.fp8_gemm_lora_epilogue(d["x"], Wq, sw, None, None, d["y"], d["ws0"])
             with torch.cuda.stream(stream):
-                L.fp8_gemm_lora_epilogue(x, Wq, sw, pl, sg, y, w)
+                for d in sets:
+                    call(d)
                 stream.synchronize()
                 g = torch.cuda.CUDAGraph()
-                reps = 10
                 with torch.cuda.graph(g, stream=stream):
-                    for _ in range(reps):
-                        L.fp8_gemm_lora_epilogue(x, Wq, sw, pl, sg, y, w)
+                    for d in sets:
+                        call(d)
                 for _ in range(min(3, args.fp8_reps)):
                     g.replay()
                 a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -602,11 +722,9 @@ def run_fp8(args, dev, stream, hbm_peak, bf16_peak, bf16_sust, peak_src):
                     g.replay()
                 b.record(stream)
             torch.cuda.synchronize()
-            st, detail = L.lora_workspace_status(w)
-            res[tag] = a.elapsed_time(b) / (n_rep * reps) * 1e3  # us per call
-            res[tag + "_status"] = st
-        act = np.unique(q.ids)
-        lora_bytes = int(len(act)) * r * (K + N) * 2 + M * r * 4
+            res[tag] = a.elapsed_time(b) / (n_rep * R) * 1e3  # us per call
+            res[tag + "_status"] = max(L.lora_workspace_status(d["ws" if tag == "lora" else "ws0"])[0]
+                                       for d in sets)
         bytes_call = N * K + N * 4 + M * K * 2 + M * N * 2 + lora_bytes
         flops = 2.0 * M * N * K
         t = res["lora"] * 1e-6
@@ -616,8 +734,10 @@ def run_fp8(args, dev, stream, hbm_peak, bf16_peak, bf16_sust, peak_src):
             "tflops": flops / t / 1e12, "tensor_frac": flops / t / 1e12 / fp8_peak,
             "hbm_gbs": bytes_call / t / 1e9, "hbm_frac": bytes_call / t / 1e9 / hbm_peak,
             "attainable_frac": (flops / t) / min(fp8_peak * 1e12, flops / bytes_call * hbm_peak * 1e9),
-            "distinct_adapters": int(len(act)), "status_ok": res["lora_status"] == 0,
+            "distinct_adapters": int(len(act)), "status_ok": res["lora_status"] == 0 and res["base_status"] == 0,
+            "l2": f"x, adapters and y rotate over {R} copies ({R * set_bytes / 2**20:.0f} MiB); W read once per call",
         }
+        del sets
     return out
 
 
