@@ -167,8 +167,12 @@ size_t lora_workspace_size(int op, int T, int K, const lora_pool_t* pool)
     if (T < 0) return (size_t)-1;
     switch (op) {
     case LORA_OP_SHRINK:
-    case LORA_OP_EXPAND:
-    case LORA_OP_APPLY: return 0;
+    case LORA_OP_EXPAND: return 0;
+    case LORA_OP_APPLY:
+        // decode-like batches need none; the others, the streaming kernel's counters and v
+        if (!pool || check_pool(pool) != LORA_OK) return (size_t)-1;
+        if (T == 0 || tile_tokens_for(T, pool->n_adapters) <= LORA_DECODE_TILE_TOKENS) return 0;
+        return sgmv_stream_workspace_bytes(T, *pool);
     case LORA_OP_FP8_GEMM: {
         if (K <= 0) return (size_t)-1;
         if (pool && check_pool(pool) != LORA_OK) return (size_t)-1;
@@ -268,16 +272,19 @@ int lora_apply(const void* x, int64_t x_slice_stride, const lora_pool_t* pool,
                const lora_segments_t* seg, void* y, void* ws, size_t ws_bytes,
                lora_stream_t stream)
 {
-    (void)ws;
-    (void)ws_bytes;
     int st = check_pool(pool);
     if (st != LORA_OK) return st;
     if ((st = check_segments(seg, pool->n_adapters)) != LORA_OK) return st;
     if (seg->T == 0) return LORA_OK;
     if ((st = check_x(x, x_slice_stride, pool, seg->T)) != LORA_OK) return st;
     if (!y || !aligned16(y)) return LORA_ERR_INVALID_ARG;
-    return cuda_status(launch_sgmv(SGMV_APPLY, x, x_slice_stride, *pool, *seg, nullptr, y,
-                                   (cudaStream_t)stream, false));
+    if (tile_tokens_for(seg->T, pool->n_adapters) <= LORA_DECODE_TILE_TOKENS)
+        // a decode-like batch: one tile per thread-block cluster, v exchanged on chip
+        return cuda_status(launch_sgmv(SGMV_APPLY, x, x_slice_stride, *pool, *seg, nullptr, y,
+                                       (cudaStream_t)stream, false));
+    const size_t need = sgmv_stream_workspace_bytes(seg->T, *pool);
+    if (!ws || ws_bytes < need || !aligned16(ws)) return LORA_ERR_WORKSPACE;
+    return cuda_status(launch_sgmv_stream(x, x_slice_stride, *pool, *seg, y, ws, (cudaStream_t)stream));
 }
 
 int fp8_quantize_rows(const void* x, int M, int K, uint8_t* xq, float* sx, lora_stream_t stream)

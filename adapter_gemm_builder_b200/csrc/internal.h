@@ -21,6 +21,13 @@ cudaError_t launch_sgmv(int mode, const void* x, int64_t x_slice_stride, const l
                         const lora_segments_t& seg, float* v, void* y, cudaStream_t stream,
                         bool pdl_trigger);
 
+// The fused shrink + expand as a persistent grid streaming work items (batches
+// whose tiles hold up to LORA_TILE_TOKENS tokens); ws holds
+// sgmv_stream_workspace_bytes(T, pool) bytes.
+cudaError_t launch_sgmv_stream(const void* x, int64_t x_slice_stride, const lora_pool_t& pool,
+                               const lora_segments_t& seg, void* y, void* ws, cudaStream_t stream);
+size_t sgmv_stream_workspace_bytes(int T, const lora_pool_t& pool);
+
 // Per-row E4M3 quantisation; row p of the output is row perm[p] of x
 // (perm == NULL: identity). The kernel also zeroes zero_words 32-bit words at
 // `zero` (may be NULL) and lets a programmatic dependent launch start early.

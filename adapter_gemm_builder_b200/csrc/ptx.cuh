@@ -324,6 +324,18 @@ __device__ __forceinline__ void named_sync(int id, int n)
 {
     asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(n) : "memory");
 }
+// Named barrier over `n` threads that also ORs a predicate over them: every
+// participating thread gets the same result.
+__device__ __forceinline__ bool named_sync_or(int id, int n, bool pred)
+{
+    uint32_t r;
+    asm volatile(
+        "{\n.reg .pred p, q;\nsetp.ne.u32 p, %1, 0;\nbar.red.or.pred q, %2, %3, p;\nselp.u32 %0, 1, 0, q;\n}\n"
+        : "=r"(r)
+        : "r"((uint32_t)pred), "r"(id), "r"(n)
+        : "memory");
+    return r != 0;
+}
 __device__ __forceinline__ unsigned long long globaltimer()
 {
     unsigned long long t;

@@ -146,7 +146,8 @@ LORA_API int lora_segments_status(const lora_segments_t* seg, lora_stream_t stre
  * Bytes of workspace an operation needs (0 if it needs none), or (size_t)-1
  * for invalid arguments. For LORA_OP_FP8_GEMM, T is the
  * token count M and `K` the GEMM's reduction size; `pool` may be NULL (no
- * LoRA). The other operations ignore K.
+ * LoRA). LORA_OP_APPLY needs the pool (its counters and v scale with the
+ * slices, the tiles and r_max). The other operations ignore K.
  * A workspace must be zeroed once after allocation (lora_workspace_init);
  * afterwards the library keeps it in a reusable state.
  */
@@ -208,8 +209,14 @@ LORA_API int lora_expand(const float* v, const lora_pool_t* pool, const lora_seg
 
 /*
  * Shrink then expand (y += s_a * (x.A_a).B_a; the whole added term of the
- * Punica README, "How?", for a batch of many adapters), with v kept on chip in fp32:
- * one kernel launch, no workspace. Arguments as lora_shrink / lora_expand.
+ * Punica README, "How?", for a batch of many adapters), v in fp32. Arguments
+ * as lora_shrink / lora_expand, plus a workspace of
+ * lora_workspace_size(LORA_OP_APPLY, T, 0, pool) bytes (none for a
+ * decode-like batch, see lora_tile_tokens_for). A decode-like batch runs one
+ * kernel whose thread-block clusters each take one tile and keep v on chip;
+ * any other batch runs a memset of the workspace's counters and one
+ * persistent kernel that streams shrink and expand parts of every tile,
+ * passing v through the workspace.
  */
 LORA_API int lora_apply(const void* x, int64_t x_slice_stride, const lora_pool_t* pool,
                const lora_segments_t* seg, void* y, void* ws, size_t ws_bytes,
