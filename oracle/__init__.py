@@ -12,6 +12,8 @@ cites the passage of the pages it follows in ``oracle.c``:
   Punica README, section "How?".
 * Per-token adapter ids in one multi-tenant batch, -1 for none:
   EpiLoRA abstract, sentence 1.
+* Token-wise merge of router-selected adapters into the backbone weight:
+  LoRA-Switch abstract (shd-paper.top page).
 * FP8 base GEMM whose epilogue adds each tenant's up-projection:
   EpiLoRA abstract, sentences 2-4 (8-bit format read as E4M3 with per-row
   scales; that reading is stated in ``oracle.c``).
@@ -71,6 +73,8 @@ def _load():
             lib.orc_fp8_gemm_lora_sampled.restype = None
             lib.orc_fp8_gemm_lora_sampled.argtypes = [P, P, P, P, I, P, P, P, I, I, I,
                                                       P, P, P, P, P, I, P]
+            lib.orc_lora_switch_merge.restype = None
+            lib.orc_lora_switch_merge.argtypes = [P, I, I, P, P, I, I, P, P, P, P, I, P]
             lib.orc_num_threads.restype = I
             lib.orc_set_num_threads.argtypes = [I]
             _lib = lib
@@ -223,4 +227,19 @@ def fp8_gemm_lora_sampled(xq, sx, Wq, sw, rows, cols, x=None, A=None, B=None, ra
     lib.orc_fp8_gemm_lora_sampled(_p(xq), _p(sx), _p(Wq), _p(sw), K, _p(x), _p(A), _p(B),
                                   n_adapters, r_max, N, _p(ranks), _p(scales), _p(ids),
                                   _p(rows), _p(cols), rows.shape[0], _p(out))
+    return out
+
+
+def lora_switch_merge(W, A, B, ranks, scales, sel, gates) -> np.ndarray:
+    """W bf16 [N, K]; A bf16 [n_adapters, K, r_max]; B bf16 [n_adapters, r_max, N];
+    sel int32 [n_sel] (-1: none); gates fp32 [n_sel]; returns the merged weight fp64 [N, K]."""
+    lib = _load()
+    W = _c(W, np.uint16); A = _c(A, np.uint16); B = _c(B, np.uint16)
+    ranks = _c(ranks, np.int32); scales = _c(scales, np.float32)
+    sel = _c(sel, np.int32); gates = _c(gates, np.float32)
+    N, K = W.shape
+    n_adapters, _, r_max = A.shape
+    out = np.zeros((N, K), np.float64)
+    lib.orc_lora_switch_merge(_p(W), N, K, _p(A), _p(B), n_adapters, r_max, _p(ranks),
+                              _p(scales), _p(sel), _p(gates), sel.shape[0], _p(out))
     return out

@@ -341,6 +341,45 @@ void orc_fp8_gemm_lora_sampled(const uint8_t* xq, const float* sx,
     }
 }
 
+/*
+ * Token-wise merge of the selected adapters into the backbone (LoRA-Switch
+ * abstract on the shd-paper.top page: for each token a router picks LoRA
+ * adapters, which are merged into the backbone weights before the token is
+ * decoded, all selected adapters in one fused operation). With W stored
+ * [N][K] (y = x.W^T) and the Punica README's identity x.(W + A.B) =
+ * x.W + x.A.B, merging adapter a with router gate g adds g.s_a.(A_a.B_a)^T:
+ *   out[n][k] = W[n][k] + sum_e gates[e] * s_{sel[e]}
+ *                         * sum_{j < r_{sel[e]}} A[sel[e]][k][j] * B[sel[e]][j][n]
+ * over the n_sel selected entries; an entry with sel[e] outside [0, n_adapters)
+ * (-1: no adapter) adds nothing. W, A, B bf16; out fp64 [N][K].
+ */
+void orc_lora_switch_merge(const uint16_t* W, int N, int K, const uint16_t* A,
+                           const uint16_t* B, int n_adapters, int r_max,
+                           const int32_t* ranks, const float* scales,
+                           const int32_t* sel, const float* gates, int n_sel,
+                           double* out)
+{
+#pragma omp parallel for schedule(static)
+    for (int n = 0; n < N; ++n) {
+        for (int k = 0; k < K; ++k) {
+            double w = orc_bf16_decode(W[(size_t)n * K + k]);
+            for (int e = 0; e < n_sel; ++e) {
+                int a = sel[e];
+                if (a < 0 || a >= n_adapters)
+                    continue;
+                int r = rank_of(ranks, a, r_max);
+                double s = scales ? (double)scales[a] : 1.0;
+                double d = 0.0;
+                for (int j = 0; j < r; ++j)
+                    d += orc_bf16_decode(A[((size_t)a * K + k) * r_max + j]) *
+                         orc_bf16_decode(B[((size_t)a * r_max + j) * N + n]);
+                w += (double)gates[e] * s * d;
+            }
+            out[(size_t)n * K + k] = w;
+        }
+    }
+}
+
 /* Threads the OpenMP loops above use. */
 int orc_num_threads(void)
 {

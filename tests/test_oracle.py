@@ -448,3 +448,116 @@ def test_linear_bf16_matches_numpy():
     got = oracle.linear_bf16_sampled(x, W, rows, cols).reshape(5, 7)
     want = oracle.bf16_to_f64(x) @ oracle.bf16_to_f64(W).T
     assert np.allclose(got, want, rtol=1e-13, atol=1e-13)
+
+
+# ---------------------------------------------------------------- token-wise merge (LoRA-Switch)
+
+def _merge_problem(seed, N=6, K=7, n_adapters=4, r_max=3, n_sel=2, ints=False):
+    rng = np.random.default_rng(seed)
+    ranks = rng.integers(1, r_max + 1, size=n_adapters).astype(np.int32)
+    scales = rng.choice(np.array([0.5, 1.0, 2.0, -1.5], np.float32), size=n_adapters)
+
+    def draw(shape, std):
+        if ints:
+            return wl.to_bf16_bits(rng.integers(-2, 3, size=shape).astype(np.float32))
+        return wl.normal_bf16(rng, shape, std)
+    W = draw((N, K), 0.5)
+    A = np.full((n_adapters, K, r_max), wl.BF16_NAN, np.uint16)
+    B = np.full((n_adapters, r_max, N), wl.BF16_NAN, np.uint16)
+    for a in range(n_adapters):
+        A[a, :, :ranks[a]] = draw((K, ranks[a]), 0.4)
+        B[a, :ranks[a], :] = draw((ranks[a], N), 0.6)
+    sel = rng.choice(n_adapters, size=n_sel, replace=False).astype(np.int32)
+    gates = (rng.choice(np.array([0.25, 0.5, 0.75, 1.0], np.float32), size=n_sel) if ints
+             else rng.random(n_sel).astype(np.float32))
+    return W, A, B, ranks, scales, sel, gates
+
+
+def _brute_force_merge(W, A, B, ranks, scales, sel, gates):
+    """Exact rationals: W + sum_e g_e s_a (A_a B_a)^T, elementwise."""
+    N, K = W.shape
+    Wf = _frac_bf16(W)
+    out = [list(row) for row in Wf]
+    for e, a in enumerate(sel):
+        a = int(a)
+        if not 0 <= a < A.shape[0]:
+            continue
+        r = int(ranks[a])
+        Af = _frac_bf16(A[a][:, :r])
+        Bf = _frac_bf16(B[a][:r, :])
+        c = Fraction(float(gates[e])) * Fraction(float(scales[a]))
+        for n in range(N):
+            for k in range(K):
+                out[n][k] += c * sum(Af[k][j] * Bf[j][n] for j in range(r))
+    return out
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_merge_exact_rationals_small_ints(seed):
+    args = _merge_problem(seed, ints=True)
+    got = oracle.lora_switch_merge(*args)
+    assert [[Fraction(float(v)) for v in row] for row in got] == _brute_force_merge(*args)
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_merge_rationals_random_bf16(seed):
+    args = _merge_problem(50 + seed, N=5, K=9, n_sel=3)
+    got = oracle.lora_switch_merge(*args)
+    want = np.array([[float(v) for v in row] for row in _brute_force_merge(*args)])
+    assert np.allclose(got, want, rtol=1e-12, atol=1e-12)
+
+
+def test_merge_zero_gates_and_no_adapter_give_the_backbone():
+    W, A, B, ranks, scales, sel, gates = _merge_problem(9, N=12, K=10)
+    base = oracle.bf16_to_f64(W)
+    assert np.array_equal(oracle.lora_switch_merge(W, A, B, ranks, scales, sel, gates * 0), base)
+    none = np.full_like(sel, -1)
+    assert np.array_equal(oracle.lora_switch_merge(W, A, B, ranks, scales, none, gates), base)
+    bad = np.array([A.shape[0], 99], np.int32)  # ids outside the pool add nothing
+    assert np.array_equal(oracle.lora_switch_merge(W, A, B, ranks, scales, bad, gates), base)
+
+
+def test_merge_is_linear_in_the_gates():
+    W, A, B, ranks, scales, sel, gates = _merge_problem(10, N=16, K=12, n_sel=2)
+    base = oracle.bf16_to_f64(W)
+    both = oracle.lora_switch_merge(W, A, B, ranks, scales, sel, gates) - base
+    one = oracle.lora_switch_merge(W, A, B, ranks, scales, sel[:1], gates[:1]) - base
+    two = oracle.lora_switch_merge(W, A, B, ranks, scales, sel[1:], gates[1:]) - base
+    assert np.allclose(both, one + two, rtol=1e-12, atol=1e-15)
+
+
+def test_merged_weight_reproduces_the_unmerged_layer():
+    """Punica README, "How?": x.(W + A.B) = x.W + x.A.B. A token routed to one adapter
+    with gate 1 gets the same output from the merged backbone as from the base layer
+    plus the separately pinned LoRA apply."""
+    p = _random_problem(11, T=8, n_adapters=4, h_in=24, h_out=20, r_max=8)
+    a = 2
+    merged = oracle.lora_switch_merge(p.W[0], p.A[0], p.B[0], p.ranks, p.scales,
+                                      np.array([a], np.int32), np.array([1.0], np.float32))
+    xf = oracle.bf16_to_f64(p.x[0])
+    y_merged = xf @ merged.T
+    rows = np.repeat(np.arange(p.T), p.h_out).astype(np.int32)
+    cols = np.tile(np.arange(p.h_out), p.T).astype(np.int32)
+    base = oracle.linear_bf16_sampled(p.x[0], p.W[0], rows, cols).reshape(p.T, p.h_out)
+    ids = np.full(p.T, a, np.int32)
+    lora = oracle.lora_apply(p.x[0], p.A[0], p.B[0], p.ranks, p.scales, ids,
+                             np.zeros((p.T, p.h_out), np.uint16))
+    assert np.allclose(y_merged, base + lora, rtol=1e-10, atol=1e-12)
+
+
+def test_merge_rank1_closed_form():
+    """A_a = e_j0 (one nonzero row k0, column 0) and rank 1: the delta is g s B[0][n] at
+    column k0 only."""
+    N, K, r_max = 6, 8, 8
+    W = wl.normal_bf16(np.random.default_rng(3), (N, K), 0.3)
+    A = np.zeros((1, K, r_max), np.uint16)
+    k0 = 5
+    A[0, k0, 0] = wl.to_bf16_bits(np.array([1.0], np.float32))[0]
+    B = np.zeros((1, r_max, N), np.uint16)
+    B[0, 0] = wl.to_bf16_bits(np.linspace(-1, 1, N).astype(np.float32))
+    out = oracle.lora_switch_merge(W, A, B, np.array([1], np.int32), np.array([2.0], np.float32),
+                                   np.array([0], np.int32), np.array([0.5], np.float32))
+    delta = out - oracle.bf16_to_f64(W)
+    want = np.zeros((N, K))
+    want[:, k0] = 0.5 * 2.0 * oracle.bf16_to_f64(B[0, 0])
+    assert np.array_equal(delta, want)
