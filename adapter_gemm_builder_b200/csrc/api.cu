@@ -50,14 +50,14 @@ int check_segments(const lora_segments_t* seg, int n_adapters)
     return LORA_OK;
 }
 
-// FP8 workspace: status | xq | sx | v (with a pool) | sync words | partials.
-// [off_v, off_part) is zeroed by the quantiser on every call.
+// GEMM workspace: status | xq (esz bytes per element) | sx | v (with a pool) |
+// sync words | partials. [off_v, off_part) is zeroed by the quantiser on every call.
 size_t fp8_ws_layout(int M, int K, const lora_pool_t* pool, size_t* off_xq, size_t* off_sx,
-                     size_t* off_v, size_t* off_sync, size_t* off_part)
+                     size_t* off_v, size_t* off_sync, size_t* off_part, int esz = 1)
 {
     size_t off = 256;  // status word block
     *off_xq = off;
-    off += align256((size_t)M * K);
+    off += align256((size_t)M * K * esz);
     *off_sx = off;
     off += align256((size_t)M * 4);
     *off_v = off;
@@ -98,6 +98,67 @@ int fp8_gemm_check_args(const void* x, int M, int K, int N, const uint8_t* Wq, c
     }
     return LORA_OK;
 }
+
+namespace {
+// Both GEMM entry points after their argument checks. esz 1: E4M3 operands
+// (x quantised per token); esz 2: bf16 operands (x copied in segment order).
+int gemm_lora_launch(int esz, const void* x, int M, int K, int N, const uint8_t* Wq, const float* w_scale,
+                     const lora_pool_t* pool, const lora_segments_t* seg, void* y, void* ws,
+                     size_t ws_bytes, lora_stream_t stream)
+{
+    size_t off_xq, off_sx, off_v, off_sync, off_part;
+    const size_t need = fp8_ws_layout(M, K, pool, &off_xq, &off_sx, &off_v, &off_sync, &off_part, esz);
+    if (!ws || ws_bytes < need || !aligned16(ws)) return LORA_ERR_WORKSPACE;
+    uint8_t* w = static_cast<uint8_t*>(ws);
+    uint32_t* status = reinterpret_cast<uint32_t*>(w);
+    uint8_t* xq = w + off_xq;
+    float* sx = reinterpret_cast<float*>(w + off_sx);
+    float* v = pool ? reinterpret_cast<float*>(w + off_v) : nullptr;
+    int* sync = reinterpret_cast<int*>(w + off_sync);
+    cudaStream_t s = (cudaStream_t)stream;
+
+    // 1. activations -> E4M3 (or copied as bf16), rows in segment order when adapters
+    //    are present; the same kernel zeroes v and the GEMM's synchronisation words
+    cudaError_t e = launch_quantize_rows(x, pool ? seg->perm : nullptr, M, K, xq, sx, w + off_v,
+                                         (off_part - off_v) / 4, s, esz == 2);
+    if (e != cudaSuccess) return LORA_ERR_CUDA;
+    // 2. the GEMM, a programmatic dependent of the quantiser: its weights start
+    //    streaming at once, the down-projection runs in its epilogue warps meanwhile
+    //    and the up-projection in its epilogue
+    Fp8GemmArgs a = {};
+    a.M = M;
+    a.N = N;
+    a.K = K;
+    a.esz = esz;
+    a.xq = xq;
+    a.sx = sx;
+    a.Wq = Wq;
+    a.sw = w_scale;
+    a.y = static_cast<uint16_t*>(y);
+    a.status = status;
+    a.partials = reinterpret_cast<float*>(w + off_part);
+    a.v_done = sync;
+    a.flags = sync + 16;
+    a.lora = pool != nullptr;
+    if (pool) {
+        a.perm = seg->perm;
+        a.tok_adapter = seg->tok_adapter;
+        a.indptr = seg->indptr;
+        a.active = seg->active;
+        a.counts = seg->counts;
+        a.v = v;
+        a.x = static_cast<const uint16_t*>(x);
+        a.A = static_cast<const uint16_t*>(pool->A);
+        a.B = static_cast<const uint16_t*>(pool->B);
+        a.ranks = pool->ranks;
+        a.scales = pool->scales;
+        a.n_adapters = pool->n_adapters;
+        a.r_max = pool->r_max;
+    }
+    return cuda_status(launch_fp8_gemm(a, s));
+}
+
+}  // namespace
 
 }  // namespace lora
 
@@ -173,12 +234,13 @@ size_t lora_workspace_size(int op, int T, int K, const lora_pool_t* pool)
         if (!pool || check_pool(pool) != LORA_OK) return (size_t)-1;
         if (T == 0 || tile_tokens_for(T, pool->n_adapters) <= LORA_DECODE_TILE_TOKENS) return 0;
         return sgmv_stream_workspace_bytes(T, *pool);
-    case LORA_OP_FP8_GEMM: {
+    case LORA_OP_FP8_GEMM:
+    case LORA_OP_BF16_GEMM: {
         if (K <= 0) return (size_t)-1;
         if (pool && check_pool(pool) != LORA_OK) return (size_t)-1;
         if (T < 1) return (size_t)-1;
         size_t a, b, c, d, e;
-        return fp8_ws_layout(T, K, pool, &a, &b, &c, &d, &e);
+        return fp8_ws_layout(T, K, pool, &a, &b, &c, &d, &e, op == LORA_OP_BF16_GEMM ? 2 : 1);
     }
     default: return (size_t)-1;
     }
@@ -302,55 +364,42 @@ int fp8_gemm_lora_epilogue(const void* x, int M, int K, int N, const uint8_t* Wq
 {
     const int st = fp8_gemm_check_args(x, M, K, N, Wq, w_scale, pool, seg, y);
     if (st != LORA_OK) return st;
-    size_t off_xq, off_sx, off_v, off_sync, off_part;
-    const size_t need = fp8_ws_layout(M, K, pool, &off_xq, &off_sx, &off_v, &off_sync, &off_part);
-    if (!ws || ws_bytes < need || !aligned16(ws)) return LORA_ERR_WORKSPACE;
-    uint8_t* w = static_cast<uint8_t*>(ws);
-    uint32_t* status = reinterpret_cast<uint32_t*>(w);
-    uint8_t* xq = w + off_xq;
-    float* sx = reinterpret_cast<float*>(w + off_sx);
-    float* v = pool ? reinterpret_cast<float*>(w + off_v) : nullptr;
-    int* sync = reinterpret_cast<int*>(w + off_sync);
-    cudaStream_t s = (cudaStream_t)stream;
+    return gemm_lora_launch(1, x, M, K, N, Wq, w_scale, pool, seg, y, ws, ws_bytes, stream);
+}
 
-    // 1. activations -> E4M3, rows in segment order when adapters are present; the
-    //    same kernel zeroes v and the GEMM's synchronisation words
-    cudaError_t e = launch_quantize_rows(x, pool ? seg->perm : nullptr, M, K, xq, sx, w + off_v,
-                                         (off_part - off_v) / 4, s);
-    if (e != cudaSuccess) return LORA_ERR_CUDA;
-    // 2. the GEMM, a programmatic dependent of the quantiser: its weights start
-    //    streaming at once, the down-projection runs in its epilogue warps meanwhile
-    //    and the up-projection in its epilogue
-    Fp8GemmArgs a = {};
-    a.M = M;
-    a.N = N;
-    a.K = K;
-    a.xq = xq;
-    a.sx = sx;
-    a.Wq = Wq;
-    a.sw = w_scale;
-    a.y = static_cast<uint16_t*>(y);
-    a.status = status;
-    a.partials = reinterpret_cast<float*>(w + off_part);
-    a.v_done = sync;
-    a.flags = sync + 16;
-    a.lora = pool != nullptr;
+int lora_switch_merge(const void* W, int N, int K, const lora_pool_t* pool, const int32_t* sel,
+                      const float* gates, int n_sel, void* W_out, lora_stream_t stream)
+{
+    int st = check_pool(pool);
+    if (st != LORA_OK) return st;
+    if (N < 8 || K < 8 || N % 8 || K % 8 || n_sel < 1) return LORA_ERR_INVALID_ARG;
+    if (pool->n_slices != 1 || pool->h_in != K || pool->h_out != N) return LORA_ERR_INVALID_ARG;
+    if (!W || !W_out || !sel || !gates || !aligned16(W) || !aligned16(W_out)) return LORA_ERR_INVALID_ARG;
+    if (n_sel > LORA_SWITCH_MAX_SELECTED || n_sel * ((pool->r_max + 15) / 16 * 16) > LORA_SWITCH_MAX_RANK_SUM)
+        return LORA_ERR_UNSUPPORTED;
+    // in place or disjoint: a partly overlapping output would be read after it is written
+    const uintptr_t a0 = (uintptr_t)W, b0 = (uintptr_t)W_out, len = (uintptr_t)N * K * 2;
+    if (a0 != b0 && a0 < b0 + len && b0 < a0 + len) return LORA_ERR_INVALID_ARG;
+    return cuda_status(launch_lora_switch_merge(W, N, K, *pool, sel, gates, n_sel, W_out, (cudaStream_t)stream));
+}
+
+int bf16_gemm_lora_epilogue(const void* x, int M, int K, int N, const void* W,
+                            const lora_pool_t* pool, const lora_segments_t* seg, void* y,
+                            void* ws, size_t ws_bytes, lora_stream_t stream)
+{
+    if (M < 1 || K < 8 || N < 8 || K % 8 || N % 8) return LORA_ERR_INVALID_ARG;
+    if (!x || !W || !y) return LORA_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(W) || !aligned16(y)) return LORA_ERR_INVALID_ARG;
+    if (M > (1 << 24)) return LORA_ERR_UNSUPPORTED;
     if (pool) {
-        a.perm = seg->perm;
-        a.tok_adapter = seg->tok_adapter;
-        a.indptr = seg->indptr;
-        a.active = seg->active;
-        a.counts = seg->counts;
-        a.v = v;
-        a.x = static_cast<const uint16_t*>(x);
-        a.A = static_cast<const uint16_t*>(pool->A);
-        a.B = static_cast<const uint16_t*>(pool->B);
-        a.ranks = pool->ranks;
-        a.scales = pool->scales;
-        a.n_adapters = pool->n_adapters;
-        a.r_max = pool->r_max;
+        int st = check_pool(pool);
+        if (st != LORA_OK) return st;
+        if (pool->n_slices != 1 || pool->h_in != K || pool->h_out != N) return LORA_ERR_INVALID_ARG;
+        if ((st = check_segments(seg, pool->n_adapters)) != LORA_OK) return st;
+        if (seg->T != M) return LORA_ERR_INVALID_ARG;
     }
-    return cuda_status(launch_fp8_gemm(a, s));
+    return gemm_lora_launch(2, x, M, K, N, static_cast<const uint8_t*>(W), nullptr, pool, seg, y, ws,
+                            ws_bytes, stream);
 }
 
 }  // extern "C"

@@ -217,7 +217,10 @@ __device__ __forceinline__ Seg seg_at(long long u, long long u_end, int KB)
     return s;
 }
 
-template <int BK, int MAXR>
+// ESZ: bytes per operand element -- 1 for E4M3 (kind::f8f6f4), 2 for bf16
+// (kind::f16). BK is the k-block in bytes either way (128: 128-byte swizzle,
+// 64: 64-byte swizzle), so the shared-memory layouts are the same.
+template <int BK, int MAXR, int ESZ>
 __global__ void __launch_bounds__(kThreads, 1)
 fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                 const __grid_constant__ CUtensorMap tmB, const GemmParams p)
@@ -306,7 +309,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
                 waited = true;
                 for (int d = 0; d < n_def; ++d) {
                     const uint32_t sX = smem_u + p.ring_off + d * stage_bytes + kStageW;
-                    ptx::tma_load_2d(sX, &tmX, &full[d], def_kb[d] * BK, def_tb[d] * p.BN);
+                    ptx::tma_load_2d(sX, &tmX, &full[d], def_kb[d] * (BK / ESZ), def_tb[d] * p.BN);
                 }
             };
             bool ok = true;
@@ -327,9 +330,9 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
                     const uint32_t sW = smem_u + p.ring_off + stage * stage_bytes;
                     const uint32_t sX = sW + kStageW;
                     ptx::mbar_arrive_expect_tx(&full[stage], (uint32_t)stage_bytes);
-                    ptx::tma_load_2d_hint(sW, &tmW, &full[stage], kb * BK, nb * kBlockM, w_policy);
+                    ptx::tma_load_2d_hint(sW, &tmW, &full[stage], kb * (BK / ESZ), nb * kBlockM, w_policy);
                     if (waited) {
-                        ptx::tma_load_2d(sX, &tmX, &full[stage], kb * BK, tb * p.BN);
+                        ptx::tma_load_2d(sX, &tmX, &full[stage], kb * (BK / ESZ), tb * p.BN);
                     } else {  // first ring pass: stage == n_def
                         def_kb[n_def] = kb;
                         def_tb[n_def] = tb;
@@ -353,7 +356,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
         if (lane == 0) {
             int stage = 0;
             uint32_t phase = 0;
-            const uint32_t idesc = make_idesc(p.BN);
+            const uint32_t idesc = ESZ == 1 ? make_idesc(p.BN) : make_idesc_bf16(p.BN);
             bool ok = true, any = false;
             int i = 0, lj = 0;
             const uint32_t slots_u = smem_u + p.slots_off, vq_u = smem_u + p.v_off;
@@ -443,10 +446,16 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
                     ptx::tc_fence_after();
                     const uint32_t sW = smem_u + p.ring_off + stage * stage_bytes;
                     const uint32_t sX = sW + kStageW;
+                    // 32 bytes of K per instruction: 32 E4M3 or 16 bf16 elements
 #pragma unroll
-                    for (int kk = 0; kk < BK / 32; ++kk)
-                        ptx::tc_mma_f8(d, make_desc<BK>(sW + kk * 32), make_desc<BK>(sX + kk * 32), idesc,
-                                       (kb > sg.kb0 || kk != 0) ? 1u : 0u);
+                    for (int kk = 0; kk < BK / 32; ++kk) {
+                        if constexpr (ESZ == 1)
+                            ptx::tc_mma_f8(d, make_desc<BK>(sW + kk * 32), make_desc<BK>(sX + kk * 32), idesc,
+                                           (kb > sg.kb0 || kk != 0) ? 1u : 0u);
+                        else
+                            ptx::tc_mma_f16(d, make_desc<BK>(sW + kk * 32), make_desc<BK>(sX + kk * 32), idesc,
+                                            (kb > sg.kb0 || kk != 0) ? 1u : 0u);
+                    }
                     any = true;
                     ptx::tc_commit(&empty[stage]);
                     if (++stage == p.stages) {
@@ -818,7 +827,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
                 // B'[n][j] = B_a[j][n] / sw[n] in place, K-major, for the phase's slots: each
                 // thread reads its row n of kSpt slots, then (after a barrier) writes them
                 const int nn = etid & 127, half = etid >> 7;
-                const float inv_sw2 = (nb * kBlockM + nn < p.N) ? 1.f / p.sw[nb * kBlockM + nn] : 0.f;
+                const float inv_sw2 = (nb * kBlockM + nn < p.N) ? (p.sw ? 1.f / p.sw[nb * kBlockM + nn] : 1.f) : 0.f;
                 const int nbuf = e1 - e0;
                 constexpr int kSpt = MAXR <= 16 ? 4 : (MAXR <= 32 ? 2 : 1);
                 for (int b0 = 0; b0 < nbuf && ok; b0 += 2 * kSpt) {
@@ -872,7 +881,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
             }
 
             const int n = nb * kBlockM + n_local;
-            const float swn = n < p.N ? p.sw[n] : 0.f;
+            const float swn = n < p.N ? (p.sw ? p.sw[n] : 1.f) : 0.f;
 
             // partial sums of the later k-blocks for 16 columns (zero when nobody else has any);
             // the next chunk's are loaded while this one is processed
@@ -1017,11 +1026,11 @@ bool encode_2d(CUtensorMap* m, CUtensorMapDataType dt, int elem_bytes, const voi
                           box_outer, swz);
 }
 
-template <int BK, int MAXR>
+template <int BK, int MAXR, int ESZ>
 cudaError_t launch_t(const GemmParams& p, const CUtensorMap& tmW, const CUtensorMap& tmX,
                      const CUtensorMap& tmB, size_t smem, int grid, cudaStream_t stream)
 {
-    cudaError_t e = cudaFuncSetAttribute(fp8_gemm_kernel<BK, MAXR>,
+    cudaError_t e = cudaFuncSetAttribute(fp8_gemm_kernel<BK, MAXR, ESZ>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
@@ -1035,7 +1044,7 @@ cudaError_t launch_t(const GemmParams& p, const CUtensorMap& tmW, const CUtensor
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, fp8_gemm_kernel<BK, MAXR>, tmW, tmX, tmB, p);
+    return cudaLaunchKernelEx(&cfg, fp8_gemm_kernel<BK, MAXR, ESZ>, tmW, tmX, tmB, p);
 }
 
 size_t align_up(size_t a, size_t b) { return (a + b - 1) / b * b; }
@@ -1118,7 +1127,7 @@ cudaError_t launch_fp8_gemm(const Fp8GemmArgs& a, cudaStream_t stream)
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
     cudaFuncAttributes fa;
-    if (cudaFuncGetAttributes(&fa, fp8_gemm_kernel<128, 64>) != cudaSuccess) return cudaErrorInvalidValue;
+    if (cudaFuncGetAttributes(&fa, fp8_gemm_kernel<128, 64, 1>) != cudaSuccess) return cudaErrorInvalidValue;
     const size_t kSmemMax = (size_t)(optin > 0 ? optin : 232448) - fa.sharedSizeBytes - 256;
     const size_t meta = align_up((size_t)p.BN * 20, 128);  // token, adapter, rank, slot, sx
     const size_t bars = 8 * (2 * kMaxStages + 10);
@@ -1176,7 +1185,8 @@ cudaError_t launch_fp8_gemm(const Fp8GemmArgs& a, cudaStream_t stream)
     p.stages = stages;
     p.n_slots = ns;
     p.v_adapters = va;
-    p.k_blocks = (a.K + BK - 1) / BK;
+    const int esz = a.esz == 2 ? 2 : 1;
+    p.k_blocks = (a.K * esz + BK - 1) / BK;
     p.units = (long long)p.num_tiles * p.k_blocks;
     const size_t stage_bytes = (size_t)kBlockM * BK + (size_t)p.BN * BK;
     p.ring_off = 0;
@@ -1188,10 +1198,9 @@ cudaError_t launch_fp8_gemm(const Fp8GemmArgs& a, cudaStream_t stream)
 
     CUtensorMap tmW, tmX, tmB;
     const CUtensorMapSwizzle swz = BK == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
-    if (!encode_2d(&tmW, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.Wq, (uint64_t)a.K, (uint64_t)a.N, BK,
-                   kBlockM, swz) ||
-        !encode_2d(&tmX, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.xq, (uint64_t)a.K, (uint64_t)a.M, BK,
-                   (uint32_t)p.BN, swz))
+    const CUtensorMapDataType dt = esz == 2 ? CU_TENSOR_MAP_DATA_TYPE_UINT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+    if (!encode_2d(&tmW, dt, esz, a.Wq, (uint64_t)a.K, (uint64_t)a.N, (uint32_t)(BK / esz), kBlockM, swz) ||
+        !encode_2d(&tmX, dt, esz, a.xq, (uint64_t)a.K, (uint64_t)a.M, (uint32_t)(BK / esz), (uint32_t)p.BN, swz))
         return cudaErrorInvalidValue;
     if (a.lora) {
         if (!encode_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, a.B, (uint64_t)a.N,
@@ -1210,8 +1219,10 @@ cudaError_t launch_fp8_gemm(const Fp8GemmArgs& a, cudaStream_t stream)
     // limited to fewer SMs than the device has (an MPS share, a green context) cannot
     // hold that grid: its CTAs would wait until the bounded waits give up.
     const bool small_r = p.r8 <= 16;
-    auto kern = BK == 128 ? (small_r ? fp8_gemm_kernel<128, 16> : fp8_gemm_kernel<128, 64>)
-                          : (small_r ? fp8_gemm_kernel<64, 16> : fp8_gemm_kernel<64, 64>);
+    auto kern = esz == 1 ? (BK == 128 ? (small_r ? fp8_gemm_kernel<128, 16, 1> : fp8_gemm_kernel<128, 64, 1>)
+                                      : (small_r ? fp8_gemm_kernel<64, 16, 1> : fp8_gemm_kernel<64, 64, 1>))
+                         : (BK == 128 ? (small_r ? fp8_gemm_kernel<128, 16, 2> : fp8_gemm_kernel<128, 64, 2>)
+                                      : (small_r ? fp8_gemm_kernel<64, 16, 2> : fp8_gemm_kernel<64, 64, 2>));
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     int per_sm = 0;
@@ -1220,11 +1231,18 @@ cudaError_t launch_fp8_gemm(const Fp8GemmArgs& a, cudaStream_t stream)
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
     long long grid = device_sm_count();
     if (grid > p.units) grid = p.units;
+    if (esz == 2) {
+        if (BK == 128)
+            return small_r ? launch_t<128, 16, 2>(p, tmW, tmX, tmB, smem, (int)grid, stream)
+                           : launch_t<128, 64, 2>(p, tmW, tmX, tmB, smem, (int)grid, stream);
+        return small_r ? launch_t<64, 16, 2>(p, tmW, tmX, tmB, smem, (int)grid, stream)
+                       : launch_t<64, 64, 2>(p, tmW, tmX, tmB, smem, (int)grid, stream);
+    }
     if (BK == 128)
-        return small_r ? launch_t<128, 16>(p, tmW, tmX, tmB, smem, (int)grid, stream)
-                       : launch_t<128, 64>(p, tmW, tmX, tmB, smem, (int)grid, stream);
-    return small_r ? launch_t<64, 16>(p, tmW, tmX, tmB, smem, (int)grid, stream)
-                   : launch_t<64, 64>(p, tmW, tmX, tmB, smem, (int)grid, stream);
+        return small_r ? launch_t<128, 16, 1>(p, tmW, tmX, tmB, smem, (int)grid, stream)
+                       : launch_t<128, 64, 1>(p, tmW, tmX, tmB, smem, (int)grid, stream);
+    return small_r ? launch_t<64, 16, 1>(p, tmW, tmX, tmB, smem, (int)grid, stream)
+                   : launch_t<64, 64, 1>(p, tmW, tmX, tmB, smem, (int)grid, stream);
 }
 
 }  // namespace lora

@@ -28,18 +28,25 @@ cudaError_t launch_sgmv_stream(const void* x, int64_t x_slice_stride, const lora
                                const lora_segments_t& seg, void* y, void* ws, cudaStream_t stream);
 size_t sgmv_stream_workspace_bytes(int T, const lora_pool_t& pool);
 
+// Token-wise merge of the selected adapters into the backbone (merge.cu).
+cudaError_t launch_lora_switch_merge(const void* W, int N, int K, const lora_pool_t& pool, const int32_t* sel,
+                                     const float* gates, int n_sel, void* W_out, cudaStream_t stream);
+
 // Per-row E4M3 quantisation; row p of the output is row perm[p] of x
 // (perm == NULL: identity). The kernel also zeroes zero_words 32-bit words at
 // `zero` (may be NULL) and lets a programmatic dependent launch start early.
+// copy_bf16: the rows are copied as bf16 instead (xq holds M * K bf16) and sx = 1.
 cudaError_t launch_quantize_rows(const void* x, const int32_t* perm, int M, int K, uint8_t* xq,
-                                 float* sx, void* zero, size_t zero_words, cudaStream_t stream);
+                                 float* sx, void* zero, size_t zero_words, cudaStream_t stream,
+                                 bool copy_bf16 = false);
 
 struct Fp8GemmArgs {
     int M, N, K;
-    const uint8_t* xq;   // e4m3 [M][K], rows in perm order
-    const float* sx;     // [M], perm order
-    const uint8_t* Wq;   // e4m3 [N][K]
-    const float* sw;     // [N]
+    int esz;             // operand element bytes: 1 = E4M3 (kind::f8f6f4), 2 = bf16 (kind::f16)
+    const uint8_t* xq;   // e4m3 (or bf16) [M][K], rows in perm order
+    const float* sx;     // [M], perm order (1 for bf16 operands)
+    const uint8_t* Wq;   // e4m3 (or bf16) [N][K]
+    const float* sw;     // [N]; NULL = 1 (bf16 weights carry no scale)
     uint16_t* y;         // bf16 [M][N]
     uint32_t* status;    // device status word
     float* partials;     // fp32 [SMs][128][fp8_gemm_tile_n(M)] stream-K partials

@@ -17,6 +17,8 @@ namespace {
 
 constexpr int kThreads = 256;
 
+// kCopy: the rows are copied as bf16 (the 16-bit GEMM's operand in segment order), sx = 1.
+template <bool kCopy>
 __global__ void __launch_bounds__(kThreads)
 quantize_rows_kernel(const uint16_t* __restrict__ x, const int32_t* __restrict__ perm, int K,
                      uint8_t* __restrict__ xq, float* __restrict__ sx, uint32_t* __restrict__ zero,
@@ -37,6 +39,12 @@ quantize_rows_kernel(const uint16_t* __restrict__ x, const int32_t* __restrict__
     const int row = perm ? perm[prow] : prow;
     const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)row * K);
     const int n16 = K >> 3;  // 8 bf16 per 16-byte chunk
+    if constexpr (kCopy) {
+        uint4* dst = reinterpret_cast<uint4*>(xq + (size_t)prow * K * 2);
+        for (int i = threadIdx.x; i < n16; i += kThreads) dst[i] = src[i];
+        if (threadIdx.x == 0) sx[prow] = 1.f;
+        return;
+    }
 
     float amax = 0.f;
     for (int i = threadIdx.x; i < n16; i += kThreads) {
@@ -78,7 +86,8 @@ quantize_rows_kernel(const uint16_t* __restrict__ x, const int32_t* __restrict__
 }  // namespace
 
 cudaError_t launch_quantize_rows(const void* x, const int32_t* perm, int M, int K, uint8_t* xq,
-                                 float* sx, void* zero, size_t zero_words, cudaStream_t stream)
+                                 float* sx, void* zero, size_t zero_words, cudaStream_t stream,
+                                 bool copy_bf16)
 {
     if (M == 0) return cudaSuccess;
     cudaLaunchConfig_t cfg = {};
@@ -90,7 +99,10 @@ cudaError_t launch_quantize_rows(const void* x, const int32_t* perm, int M, int 
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, quantize_rows_kernel, static_cast<const uint16_t*>(x), perm, K, xq, sx,
+    if (copy_bf16)
+        return cudaLaunchKernelEx(&cfg, quantize_rows_kernel<true>, static_cast<const uint16_t*>(x), perm, K, xq,
+                                  sx, static_cast<uint32_t*>(zero), zero_words);
+    return cudaLaunchKernelEx(&cfg, quantize_rows_kernel<false>, static_cast<const uint16_t*>(x), perm, K, xq, sx,
                               static_cast<uint32_t*>(zero), zero_words);
 }
 

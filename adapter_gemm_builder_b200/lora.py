@@ -28,13 +28,15 @@ LORA_OP_SHRINK = 0
 LORA_OP_EXPAND = 1
 LORA_OP_APPLY = 2
 LORA_OP_FP8_GEMM = 3
+LORA_OP_BF16_GEMM = 4
 
 EXPORTED = [
     "lora_workspace_size", "lora_workspace_init", "lora_workspace_status", "lora_build_segments",
     "lora_shrink", "lora_expand", "lora_apply", "fp8_quantize_rows", "fp8_gemm_lora_epilogue",
     "lora_status_string", "lora_version", "lora_tile_tokens", "lora_tile_tokens_for", "lora_max_tiles",
     "lora_segments_status", "fp8_gemm_lora_epilogue_noalloc", "lora_noalloc_scratch_bytes",
-    "lora_noalloc_status", "lora_debug_set_wait_limit",
+    "lora_noalloc_status", "lora_debug_set_wait_limit", "bf16_gemm_lora_epilogue",
+    "lora_switch_merge",
 ]
 
 
@@ -98,6 +100,8 @@ def load(path: str = LIB_PATH):
             "lora_noalloc_scratch_bytes": (Z, []),
             "lora_noalloc_status": (I, [P, P]),
             "lora_debug_set_wait_limit": (I, [ctypes.c_uint64, I]),
+            "bf16_gemm_lora_epilogue": (I, [P, I, I, I, P, P, P, P, P, Z, P]),
+            "lora_switch_merge": (I, [P, I, I, P, P, P, I, P, P]),
         }
         for name, (res, args) in sig.items():
             f = getattr(lib, name)
@@ -258,6 +262,25 @@ def fp8_gemm_lora_epilogue(x: torch.Tensor, Wq: torch.Tensor, w_scale: torch.Ten
     _check(load().fp8_gemm_lora_epilogue(
         _ptr(x), M, K, N, _ptr(Wq), _ptr(w_scale), ctypes.byref(pool.c) if pool else None,
         ctypes.byref(seg.c) if seg else None, _ptr(y), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def bf16_gemm_lora_epilogue(x: torch.Tensor, W: torch.Tensor, pool: Pool | None,
+                            seg: Segments | None, y: torch.Tensor, ws: torch.Tensor,
+                            stream=None) -> None:
+    """y = x.W^T + s_a (x.A_a).B_a with bf16 operands (x [M, K], W [N, K])."""
+    M, K = x.shape
+    N = W.shape[0]
+    _check(load().bf16_gemm_lora_epilogue(
+        _ptr(x), M, K, N, _ptr(W), ctypes.byref(pool.c) if pool else None,
+        ctypes.byref(seg.c) if seg else None, _ptr(y), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def lora_switch_merge(W: torch.Tensor, pool: Pool, sel: torch.Tensor, gates: torch.Tensor,
+                      W_out: torch.Tensor, stream=None) -> None:
+    """W_out = W + sum_e gates[e] s_a (A_a B_a)^T over the selected adapters (device sel/gates)."""
+    N, K = W.shape
+    _check(load().lora_switch_merge(_ptr(W), N, K, ctypes.byref(pool.c), _ptr(sel), _ptr(gates),
+                                    sel.numel(), _ptr(W_out), _stream(stream)))
 
 
 def fp8_gemm_lora_epilogue_noalloc(x: torch.Tensor, Wq: torch.Tensor, w_scale: torch.Tensor,

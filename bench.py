@@ -66,6 +66,7 @@ def parse_args():
                     help="run only the FP8 GEMM + LoRA section and print its JSON")
     ap.add_argument("--fp8-m", type=int, nargs="+", default=[16, 64, 256])
     ap.add_argument("--fp8-reps", type=int, default=20, help="graph replays per timing")
+    ap.add_argument("--no-bf16", action="store_true", help="skip the bf16 GEMM + LoRA section")
     return ap.parse_args()
 
 
@@ -515,6 +516,7 @@ def run_ours(args):
                 "status_ok": tq["status_ok"]}
 
     fp8 = None if args.no_fp8 else run_fp8(args, dev, stream, hbm_peak, bf16_peak, bf16_sust, peak_src)
+    bf16 = None if args.no_bf16 else run_bf16(args, dev, stream, hbm_peak, bf16_peak, peak_src)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -529,7 +531,7 @@ def run_ours(args):
                        "parallelism": f"replicas x{world}"},
             "roofline": roofline, "e2e": e2e, "gpu_launches": (1 + apply_launches()) * K,
             "clocks": t["clocks"], "status_ok": t["status_ok"],
-            "cpu_baseline": cpu, "workloads": extras, "fp8_gemm_lora": fp8,
+            "cpu_baseline": cpu, "workloads": extras, "fp8_gemm_lora": fp8, "bf16_gemm_lora": bf16,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -736,6 +738,107 @@ def run_fp8(args, dev, stream, hbm_peak, bf16_peak, bf16_sust, peak_src):
             "attainable_frac": (flops / t) / min(fp8_peak * 1e12, flops / bytes_call * hbm_peak * 1e9),
             "distinct_adapters": int(len(act)), "status_ok": res["lora_status"] == 0 and res["base_status"] == 0,
             "l2": f"x, adapters and y rotate over {R} copies ({R * set_bytes / 2**20:.0f} MiB); W read once per call",
+        }
+        del sets
+    return out
+
+
+BF16_CASES = [
+    # name, M, K, N, adapters, rank choices, r_max, ids kind, fraction of tokens at -1
+    ("llama70b_up_M16", 16, 8192, 28672, 16, (16,), 16, "zipf", 0.0),
+    ("llama70b_up_M64", 64, 8192, 28672, 16, (16,), 16, "zipf", 0.0),
+    ("llama70b_up_M256", 256, 8192, 28672, 16, (16,), 16, "zipf", 0.0),
+    ("bgmv_decode", 36, 4096, 4096, 32, (16,), 16, "distinct36", 0.0),
+    ("many_tenants_one_slice", 512, 5120, 5120, 256, (8, 16, 32, 64), 64, "zipf", 0.05),
+    ("sgmv_prefill", 2704, 4096, 11008, 8, (64,), 64, "prefill", 0.0),
+]
+
+
+def run_bf16(args, dev, stream, hbm_peak, bf16_peak, peak_src):
+    """The 16-bit base GEMM with the fused LoRA term (one call per projection) on the
+    decode shapes of the FP8 section and on the bf16 workloads' shapes, each against the
+    same call without LoRA. Inputs are drawn on the device from a seeded generator with
+    the workloads' distributions; W, x, the adapters and y rotate over enough copies to
+    pass the L2."""
+    import numpy as np
+    import torch
+
+    from adapter_gemm_builder_b200 import lora as L
+    from adapter_gemm_builder_b200 import workloads as wl
+    out = {"peak_tflops_bf16": bf16_peak, "peak_hbm_gbs": hbm_peak,
+           "peak_source": f"{peak_src} (MEASURED_PEAKS.json bf16_tflops, burst cuBLAS)", "cases": {}}
+    gen = torch.Generator(device=dev).manual_seed(11)
+
+    def randn(shape, std):
+        return (torch.randn(shape, generator=gen, device=dev) * std).to(torch.bfloat16)
+
+    for name, M, K, N, n_ad, rchoice, r_max, kind, none_frac in BF16_CASES:
+        rng = np.random.default_rng(M + N)
+        if kind == "distinct36":
+            ids = rng.permutation(np.concatenate([np.arange(32), np.full(4, -1)])).astype(np.int32)
+        elif kind == "prefill":
+            ids = np.repeat(np.arange(8, dtype=np.int32), wl.sgmv_prefill_lengths())
+            M = int(ids.shape[0])
+        else:
+            ids = wl.make_ids(kind, rng, M, n_ad, none_frac)
+        ranks = rng.choice(np.asarray(rchoice, np.int32), size=n_ad).astype(np.int32)
+        act = np.unique(ids[ids >= 0])
+        lora_bytes = int(ranks[act].sum()) * (K + N) * 2 + M * r_max * 4
+        base_bytes = N * K * 2 + M * K * 2 + M * N * 2
+        set_bytes = base_bytes + int(ranks[act].sum()) * (K + N) * 2
+        R = int(min(16, max(1, math.ceil(2.5 * L2_BYTES / set_bytes))))
+        sets = []
+        for k in range(R):
+            d = dict(x=randn((M, K), 1.0), W=randn((N, K), 1.0 / math.sqrt(K)),
+                     A=randn((n_ad, K, r_max), 1.0 / math.sqrt(K)),
+                     B=randn((n_ad, r_max, N), 1.0 / math.sqrt(max(1, r_max))),
+                     y=torch.empty((M, N), dtype=torch.bfloat16, device=dev))
+            d["pool"] = L.Pool(d["A"], d["B"], torch.from_numpy(ranks).to(dev),
+                               torch.full((n_ad,), 2.0, dtype=torch.float32, device=dev))
+            d["seg"] = L.Segments(M, n_ad, device=dev)
+            L.lora_build_segments(torch.from_numpy(ids).to(dev), n_ad, d["seg"])
+            d["ws"] = L.workspace(L.LORA_OP_BF16_GEMM, M, K, d["pool"], device=dev)
+            d["ws0"] = L.workspace(L.LORA_OP_BF16_GEMM, M, K, None, device=dev)
+            sets.append(d)
+        res = {}
+        for tag in ("lora", "base"):
+            def call(d):
+                if tag == "lora":
+                    L.bf16_gemm_lora_epilogue(d["x"], d["W"], d["pool"], d["seg"], d["y"], d["ws"])
+                else:
+                    L.bf16_gemm_lora_epilogue(d["x"], d["W"], None, None, d["y"], d["ws0"])
+            with torch.cuda.stream(stream):
+                for d in sets:
+                    call(d)
+                stream.synchronize()
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=stream):
+                    for d in sets:
+                        call(d)
+                for _ in range(3):
+                    g.replay()
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                reps = max(2, 40 // R)
+                a.record(stream)
+                for _ in range(reps):
+                    g.replay()
+                b.record(stream)
+            torch.cuda.synchronize()
+            res[tag] = a.elapsed_time(b) / (reps * R) * 1e3
+            res[tag + "_status"] = max(L.lora_workspace_status(d["ws" if tag == "lora" else "ws0"])[0]
+                                       for d in sets)
+        t = res["lora"] * 1e-6
+        flops = 2.0 * M * N * K
+        bytes_call = base_bytes + lora_bytes
+        out["cases"][name] = {
+            "M": M, "K": K, "N": N, "adapters": n_ad, "active_adapters": int(len(act)),
+            "us_per_call": res["lora"], "us_per_call_no_lora": res["base"],
+            "overhead_vs_no_lora": res["lora"] / res["base"] - 1.0,
+            "tflops": flops / t / 1e12, "tensor_frac": flops / t / 1e12 / bf16_peak,
+            "hbm_gbs": bytes_call / t / 1e9, "hbm_frac": bytes_call / t / 1e9 / hbm_peak,
+            "attainable_frac": (flops / t) / min(bf16_peak * 1e12, flops / bytes_call * hbm_peak * 1e9),
+            "status_ok": res["lora_status"] == 0 and res["base_status"] == 0,
+            "l2": f"W, x, the adapters and y rotate over {R} copies ({R * set_bytes / 2**20:.0f} MiB)",
         }
         del sets
     return out

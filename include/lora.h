@@ -69,6 +69,8 @@ typedef enum {
 #define LORA_DECODE_MAX_TOKENS 64  /* largest batch that can count as decode-like */
 #define LORA_MAX_RANK 64       /* largest r_max */
 #define LORA_MAX_ADAPTERS 16384
+#define LORA_SWITCH_MAX_SELECTED 8    /* adapters one lora_switch_merge may merge */
+#define LORA_SWITCH_MAX_RANK_SUM 256  /* n_sel * round_up(r_max, 16) */
 
 /*
  * Stacked adapter pool (the pages' per-adapter A_i, B_i, stacked; the
@@ -141,6 +143,7 @@ LORA_API int lora_segments_status(const lora_segments_t* seg, lora_stream_t stre
 #define LORA_OP_EXPAND 1
 #define LORA_OP_APPLY 2
 #define LORA_OP_FP8_GEMM 3
+#define LORA_OP_BF16_GEMM 4
 
 /*
  * Bytes of workspace an operation needs (0 if it needs none), or (size_t)-1
@@ -260,6 +263,50 @@ LORA_API int fp8_gemm_lora_epilogue(const void* x, int M, int K, int N, const ui
                            const float* w_scale, const lora_pool_t* pool,
                            const lora_segments_t* seg, void* y, void* ws, size_t ws_bytes,
                            lora_stream_t stream);
+
+/*
+ * 16-bit base GEMM with the same fused LoRA term (the EpiLoRA abstract,
+ * sentences 3-4, for the engine that keeps activations and weights in 16
+ * bits, sentence 6):
+ *   y[m][n] = bf16( sum_k x[m][k] * W[n][k]
+ *                   + s_a * sum_{j < r_a} v[m][j] * B[0][a][j][n] ),
+ *   v = x.A_a in fp32, a = seg->tok_adapter[m] (no term for -1 or pool == NULL).
+ * The same kernel as fp8_gemm_lora_epilogue with bf16 tensor-core operands
+ * (tcgen05 kind::f16, fp32 accumulation in TMEM) and no scales: a copy kernel
+ * puts x's rows in segment order, then the GEMM runs as its programmatic
+ * dependent with the down-projection on its epilogue warps.
+ *   x bf16 [M][K]; W bf16 [N][K]; y bf16 [M][N] (out).
+ *   pool / seg as for fp8_gemm_lora_epilogue.
+ *   ws: lora_workspace_size(LORA_OP_BF16_GEMM, M, K, pool) bytes.
+ * Limits: K % 8 == 0, N % 8 == 0, M >= 1. The residency note of
+ * fp8_gemm_lora_epilogue applies.
+ */
+LORA_API int bf16_gemm_lora_epilogue(const void* x, int M, int K, int N, const void* W,
+                                     const lora_pool_t* pool, const lora_segments_t* seg, void* y,
+                                     void* ws, size_t ws_bytes, lora_stream_t stream);
+
+/*
+ * Token-wise merge of router-selected adapters into the backbone (LoRA-Switch
+ * abstract, shd-paper.top page: for each token a router switches the LoRA
+ * adapters and their weights and merges them into the backbone, all selected
+ * adapters in one fused kernel):
+ *   W_out[n][k] = bf16( W[n][k] + sum_e gates[e] * s_a
+ *                                * sum_{j < r_a} A[0][a][k][j] * B[0][a][j][n] ),
+ *   a = sel[e]; entries with a outside [0, n_adapters) (-1: none) add nothing.
+ * The gate and scale multiply the fp32 product, so the merged weight is
+ * rounded once, to bf16. The token is then decoded with the merged weight
+ * (e.g. bf16_gemm_lora_epilogue with pool = NULL); W itself stays unchanged
+ * unless W_out == W.
+ *   W bf16 [N][K] (y = x.W^T); W_out bf16 [N][K], W itself or a disjoint buffer.
+ *   pool: n_slices == 1, h_in == K, h_out == N.
+ *   sel int32 [n_sel], gates fp32 [n_sel]: DEVICE arrays (the router's output;
+ *   the kernel waits for the previous kernel in the stream before reading them).
+ * One kernel launch. Limits: N % 8 == 0, K % 8 == 0,
+ * n_sel <= LORA_SWITCH_MAX_SELECTED and n_sel * round_up(r_max, 16) <=
+ * LORA_SWITCH_MAX_RANK_SUM (else LORA_ERR_UNSUPPORTED).
+ */
+LORA_API int lora_switch_merge(const void* W, int N, int K, const lora_pool_t* pool, const int32_t* sel,
+                               const float* gates, int n_sel, void* W_out, lora_stream_t stream);
 
 /*
  * fp8_gemm_lora_epilogue for callers that cannot allocate device memory
