@@ -67,6 +67,7 @@ def parse_args():
     ap.add_argument("--fp8-m", type=int, nargs="+", default=[16, 64, 256])
     ap.add_argument("--fp8-reps", type=int, default=20, help="graph replays per timing")
     ap.add_argument("--no-bf16", action="store_true", help="skip the bf16 GEMM + LoRA section")
+    ap.add_argument("--no-merge", action="store_true", help="skip the adapter-merge section")
     return ap.parse_args()
 
 
@@ -517,6 +518,7 @@ def run_ours(args):
 
     fp8 = None if args.no_fp8 else run_fp8(args, dev, stream, hbm_peak, bf16_peak, bf16_sust, peak_src)
     bf16 = None if args.no_bf16 else run_bf16(args, dev, stream, hbm_peak, bf16_peak, peak_src)
+    merge = None if args.no_merge else run_merge(args, dev, stream, hbm_peak, peak_src)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -532,6 +534,7 @@ def run_ours(args):
             "roofline": roofline, "e2e": e2e, "gpu_launches": (1 + apply_launches()) * K,
             "clocks": t["clocks"], "status_ok": t["status_ok"],
             "cpu_baseline": cpu, "workloads": extras, "fp8_gemm_lora": fp8, "bf16_gemm_lora": bf16,
+            "switch_merge": merge,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -841,6 +844,67 @@ def run_bf16(args, dev, stream, hbm_peak, bf16_peak, peak_src):
             "l2": f"W, x, the adapters and y rotate over {R} copies ({R * set_bytes / 2**20:.0f} MiB)",
         }
         del sets
+    return out
+
+
+MERGE_CASES = [
+    # name, N, K, adapters in the pool, rank, selected (top-k of the router)
+    ("llama7b_q_proj_top2_of_8", 4096, 4096, 8, 16, 2),
+    ("llama70b_up_proj_top2_of_16", 28672, 8192, 16, 16, 2),
+]
+
+
+def run_merge(args, dev, stream, hbm_peak, peak_src):
+    """Token-wise merge of the router-selected adapters into the backbone
+    (lora_switch_merge): GB/s of algorithmic bytes (W read, W_out written, the
+    selected adapters' A and B read) and the fraction of the HBM peak. W and W_out
+    rotate over enough copies to pass the L2."""
+    import numpy as np
+    import torch
+
+    from adapter_gemm_builder_b200 import lora as L
+    gen = torch.Generator(device=dev).manual_seed(13)
+    out = {"peak_hbm_gbs": hbm_peak, "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)",
+           "cases": {}}
+    for name, N, K, n_ad, r, k_sel in MERGE_CASES:
+        A = (torch.randn((n_ad, K, r), generator=gen, device=dev) / math.sqrt(K)).to(torch.bfloat16)
+        B = (torch.randn((n_ad, r, N), generator=gen, device=dev) / math.sqrt(r)).to(torch.bfloat16)
+        pool = L.Pool(A, B, torch.full((n_ad,), r, dtype=torch.int32, device=dev),
+                      torch.full((n_ad,), 2.0, dtype=torch.float32, device=dev))
+        rng = np.random.default_rng(N)
+        sel = torch.from_numpy(rng.choice(n_ad, k_sel, replace=False).astype(np.int32)).to(dev)
+        g = rng.random(k_sel).astype(np.float32)
+        gates = torch.from_numpy(g / g.sum()).to(dev)
+        set_bytes = 2 * N * K * 2
+        R = int(min(16, max(1, math.ceil(2.5 * L2_BYTES / set_bytes))))
+        Ws = [(torch.randn((N, K), generator=gen, device=dev) / math.sqrt(K)).to(torch.bfloat16)
+              for _ in range(R)]
+        Wo = [torch.empty_like(w) for w in Ws]
+        with torch.cuda.stream(stream):
+            for w, o in zip(Ws, Wo):
+                L.lora_switch_merge(w, pool, sel, gates, o)
+            stream.synchronize()
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph, stream=stream):
+                for w, o in zip(Ws, Wo):
+                    L.lora_switch_merge(w, pool, sel, gates, o)
+            for _ in range(3):
+                graph.replay()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            reps = max(3, 60 // R)
+            a.record(stream)
+            for _ in range(reps):
+                graph.replay()
+            b.record(stream)
+        torch.cuda.synchronize()
+        us = a.elapsed_time(b) / (reps * R) * 1e3
+        nbytes = 2 * N * K * 2 + k_sel * r * (K + N) * 2
+        out["cases"][name] = {"N": N, "K": K, "adapters": n_ad, "rank": r, "selected": k_sel,
+                              "us_per_call": us, "algorithmic_bytes": nbytes,
+                              "gbs": nbytes / (us * 1e-6) / 1e9,
+                              "hbm_frac": nbytes / (us * 1e-6) / 1e9 / hbm_peak,
+                              "l2": f"W and W_out rotate over {R} pairs ({R * set_bytes / 2**20:.0f} MiB)"}
+        del Ws, Wo, A, B
     return out
 
 

@@ -14,6 +14,8 @@ cites the passage of the pages it follows in ``oracle.c``:
   EpiLoRA abstract, sentence 1.
 * Token-wise merge of router-selected adapters into the backbone weight:
   LoRA-Switch abstract (shd-paper.top page).
+* Gradients of the layer for training adapters on a frozen FP8 base:
+  EpiLoRA abstract, sentence 6 (with the Punica README's algebra).
 * FP8 base GEMM whose epilogue adds each tenant's up-projection:
   EpiLoRA abstract, sentences 2-4 (8-bit format read as E4M3 with per-row
   scales; that reading is stated in ``oracle.c``).
@@ -75,6 +77,8 @@ def _load():
                                                       P, P, P, P, P, I, P]
             lib.orc_lora_switch_merge.restype = None
             lib.orc_lora_switch_merge.argtypes = [P, I, I, P, P, I, I, P, P, P, P, I, P]
+            lib.orc_lora_backward.restype = None
+            lib.orc_lora_backward.argtypes = [P, P, I, I, I, P, P, P, P, P, P, I, I, P, P, P, P, P, P]
             lib.orc_num_threads.restype = I
             lib.orc_set_num_threads.argtypes = [I]
             _lib = lib
@@ -243,3 +247,23 @@ def lora_switch_merge(W, A, B, ranks, scales, sel, gates) -> np.ndarray:
     lib.orc_lora_switch_merge(_p(W), N, K, _p(A), _p(B), n_adapters, r_max, _p(ranks),
                               _p(scales), _p(sel), _p(gates), sel.shape[0], _p(out))
     return out
+
+
+def lora_backward(x, dY, A, B, ranks, scales, ids, dYq=None, sd=None, WqT=None, swT=None):
+    """x bf16 [M, K]; dY bf16 [M, N]; A bf16 [n_adapters, K, r_max]; B bf16 [n_adapters,
+    r_max, N]; optional base term from dYq/sd (dY quantised per token) and WqT/swT (W^T
+    quantised per input channel). Returns (dX [M, K], dA [n_ad, K, r_max], dB [n_ad, r_max, N])
+    in fp64."""
+    lib = _load()
+    x = _c(x, np.uint16); dY = _c(dY, np.uint16); A = _c(A, np.uint16); B = _c(B, np.uint16)
+    ranks = _c(ranks, np.int32); scales = _c(scales, np.float32); ids = _c(ids, np.int32)
+    dYq = _c(dYq, np.uint8); sd = _c(sd, np.float32); WqT = _c(WqT, np.uint8); swT = _c(swT, np.float32)
+    M, K = x.shape
+    N = dY.shape[1]
+    n_adapters, _, r_max = A.shape
+    dX = np.zeros((M, K), np.float64)
+    dA = np.zeros((n_adapters, K, r_max), np.float64)
+    dB = np.zeros((n_adapters, r_max, N), np.float64)
+    lib.orc_lora_backward(_p(x), _p(dY), M, K, N, _p(dYq), _p(sd), _p(WqT), _p(swT), _p(A), _p(B),
+                          n_adapters, r_max, _p(ranks), _p(scales), _p(ids), _p(dX), _p(dA), _p(dB))
+    return dX, dA, dB

@@ -380,6 +380,97 @@ void orc_lora_switch_merge(const uint16_t* W, int N, int K, const uint16_t* A,
     }
 }
 
+/*
+ * Gradients of the LoRA layer for training adapters on a frozen 8-bit base
+ * (EpiLoRA abstract, sentence 6: a trainer that keeps the base weights in
+ * FP8). The forward is y = x.W^T + s_a.(x.A_a).B_a (the Punica README's
+ * "How?" with a scale); for an upstream gradient dY [M][N] the chain rule
+ * gives, per token m with adapter a (nothing from the adapter term for -1):
+ *   dX[m][k]    = sum_n dY[m][n] W[n][k] + s_a sum_j u[m][j] A_a[k][j],
+ *                 u[m][j] = sum_n dY[m][n] B_a[j][n]            (j < r_a)
+ *   dA_a[k][j]  = s_a sum_{m with adapter a} x[m][k] u[m][j]     (j < r_a)
+ *   dB_a[j][n]  = s_a sum_{m with adapter a} v[m][j] dY[m][n],   v = x.A_a
+ * The base weight's term of dX is the 8-bit GEMM of the backward: W^T
+ * quantised per input channel (WqT [K][N] E4M3 with fp32 scales swT [K], made
+ * once from the frozen W like the forward's Wq) and dY quantised per token
+ * the way the forward quantises x (sd[m] = amax_n |dY[m][n]| / 448, dYq =
+ * E4M3(dY / sd)), both given here:
+ *   base[m][k] = sd[m] swT[k] sum_n E4M3(dYq[m][n]) E4M3(WqT[k][n]).
+ * WqT == NULL leaves the base term out. Entries past each adapter's rank
+ * (padding) are neither read nor written: dA / dB keep zero there, and they
+ * are zero for adapters without tokens. x, dY, A, B bf16; outputs fp64.
+ */
+void orc_lora_backward(const uint16_t* x, const uint16_t* dY, int M, int K, int N,
+                       const uint8_t* dYq, const float* sd, const uint8_t* WqT,
+                       const float* swT, const uint16_t* A, const uint16_t* B,
+                       int n_adapters, int r_max, const int32_t* ranks,
+                       const float* scales, const int32_t* ids, double* dX,
+                       double* dA, double* dB)
+{
+    double* u = (double*)calloc((size_t)M * r_max, sizeof(double));
+    double* v = (double*)calloc((size_t)M * r_max, sizeof(double));
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int m = 0; m < M; ++m) {
+        int a = valid_id(ids, m, n_adapters);
+        if (a < 0)
+            continue;
+        int r = rank_of(ranks, a, r_max);
+        for (int j = 0; j < r; ++j) {
+            double su = 0.0, sv = 0.0;
+            for (int n = 0; n < N; ++n)
+                su += orc_bf16_decode(dY[(size_t)m * N + n]) *
+                      orc_bf16_decode(B[((size_t)a * r_max + j) * N + n]);
+            for (int k = 0; k < K; ++k)
+                sv += orc_bf16_decode(x[(size_t)m * K + k]) *
+                      orc_bf16_decode(A[((size_t)a * K + k) * r_max + j]);
+            u[(size_t)m * r_max + j] = su;
+            v[(size_t)m * r_max + j] = sv;
+        }
+    }
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int m = 0; m < M; ++m) {
+        int a = valid_id(ids, m, n_adapters);
+        int r = a >= 0 ? rank_of(ranks, a, r_max) : 0;
+        double s = (a >= 0 && scales) ? (double)scales[a] : 1.0;
+        for (int k = 0; k < K; ++k) {
+            double g = 0.0;
+            if (WqT != NULL) {
+                double acc = 0.0;
+                for (int n = 0; n < N; ++n)
+                    acc += orc_e4m3_decode(dYq[(size_t)m * N + n]) *
+                           orc_e4m3_decode(WqT[(size_t)k * N + n]);
+                g = (double)sd[m] * (double)swT[k] * acc;
+            }
+            double l = 0.0;
+            for (int j = 0; j < r; ++j)
+                l += u[(size_t)m * r_max + j] * orc_bf16_decode(A[((size_t)a * K + k) * r_max + j]);
+            dX[(size_t)m * K + k] = g + s * l;
+        }
+    }
+    memset(dA, 0, sizeof(double) * (size_t)n_adapters * K * r_max);
+    memset(dB, 0, sizeof(double) * (size_t)n_adapters * r_max * N);
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int a = 0; a < n_adapters; ++a) {
+        int r = rank_of(ranks, a, r_max);
+        double s = scales ? (double)scales[a] : 1.0;
+        for (int m = 0; m < M; ++m) {
+            if (valid_id(ids, m, n_adapters) != a)
+                continue;
+            for (int k = 0; k < K; ++k) {
+                double xv = orc_bf16_decode(x[(size_t)m * K + k]);
+                for (int j = 0; j < r; ++j)
+                    dA[((size_t)a * K + k) * r_max + j] += s * xv * u[(size_t)m * r_max + j];
+            }
+            for (int j = 0; j < r; ++j)
+                for (int n = 0; n < N; ++n)
+                    dB[((size_t)a * r_max + j) * N + n] +=
+                        s * v[(size_t)m * r_max + j] * orc_bf16_decode(dY[(size_t)m * N + n]);
+        }
+    }
+    free(u);
+    free(v);
+}
+
 /* Threads the OpenMP loops above use. */
 int orc_num_threads(void)
 {

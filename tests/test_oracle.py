@@ -561,3 +561,128 @@ def test_merge_rank1_closed_form():
     want = np.zeros((N, K))
     want[:, k0] = 0.5 * 2.0 * oracle.bf16_to_f64(B[0, 0])
     assert np.array_equal(delta, want)
+
+
+# ---------------------------------------------------------------- gradients (adapter training)
+
+def _loss_lora(x, A, B, ranks, scales, ids, dY):
+    """L = sum dY * (s (x A) B) through the separately pinned forward oracle."""
+    y = oracle.lora_apply(x, A, B, ranks, scales, ids, np.zeros(dY.shape, np.uint16))
+    return float(np.sum(oracle.bf16_to_f64(dY) * y))
+
+
+def _int_bits(rng, shape, lo=-2, hi=3):
+    return wl.to_bf16_bits(rng.integers(lo, hi, size=shape).astype(np.float32))
+
+
+def _grad_problem(seed, M=7, K=6, N=5, n_ad=3, r_max=3):
+    rng = np.random.default_rng(seed)
+    x = _int_bits(rng, (M, K))
+    dY = _int_bits(rng, (M, N))
+    ranks = rng.integers(1, r_max + 1, size=n_ad).astype(np.int32)
+    A = np.full((n_ad, K, r_max), wl.BF16_NAN, np.uint16)
+    B = np.full((n_ad, r_max, N), wl.BF16_NAN, np.uint16)
+    for a in range(n_ad):
+        A[a, :, :ranks[a]] = _int_bits(rng, (K, ranks[a]))
+        B[a, :ranks[a], :] = _int_bits(rng, (ranks[a], N))
+    scales = rng.choice(np.array([0.5, 1.0, 2.0, -1.5], np.float32), size=n_ad)
+    ids = rng.integers(-1, n_ad, size=M).astype(np.int32)
+    return rng, x, dY, A, B, ranks, scales, ids
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_backward_adjoint_identities(seed):
+    """The layer is linear in x, in A (B fixed) and in B (A fixed), so for any
+    direction d: L(. + d) - L(.) = <grad, d> exactly (small integers: every value
+    and sum is exact in fp64)."""
+    rng, x, dY, A, B, ranks, scales, ids = _grad_problem(seed)
+    dX, dA, dB = oracle.lora_backward(x, dY, A, B, ranks, scales, ids)
+    L0 = _loss_lora(x, A, B, ranks, scales, ids, dY)
+    d = _int_bits(rng, x.shape, -1, 2)
+    xd = wl.to_bf16_bits((oracle.bf16_to_f64(x) + oracle.bf16_to_f64(d)).astype(np.float32))
+    assert _loss_lora(xd, A, B, ranks, scales, ids, dY) - L0 == float(np.sum(dX * oracle.bf16_to_f64(d)))
+    dAdir = np.zeros(A.shape, np.float64)
+    Ad = A.copy()
+    for a in range(A.shape[0]):
+        r = ranks[a]
+        step = rng.integers(-1, 2, size=(A.shape[1], r)).astype(np.float64)
+        dAdir[a, :, :r] = step
+        Ad[a, :, :r] = wl.to_bf16_bits((oracle.bf16_to_f64(A[a, :, :r]) + step).astype(np.float32))
+    assert _loss_lora(x, Ad, B, ranks, scales, ids, dY) - L0 == float(np.sum(dA * dAdir))
+    dBdir = np.zeros(B.shape, np.float64)
+    Bd = B.copy()
+    for a in range(B.shape[0]):
+        r = ranks[a]
+        step = rng.integers(-1, 2, size=(r, B.shape[2])).astype(np.float64)
+        dBdir[a, :r, :] = step
+        Bd[a, :r, :] = wl.to_bf16_bits((oracle.bf16_to_f64(B[a, :r, :]) + step).astype(np.float32))
+    assert _loss_lora(x, A, Bd, ranks, scales, ids, dY) - L0 == float(np.sum(dB * dBdir))
+
+
+def test_backward_brute_force_rationals():
+    """Every output from its definition in exact rationals (u, v, then the sums)."""
+    rng, x, dY, A, B, ranks, scales, ids = _grad_problem(9, M=5, K=4, N=3)
+    dX, dA, dB = oracle.lora_backward(x, dY, A, B, ranks, scales, ids)
+    X, D = _frac_bf16(x), _frac_bf16(dY)
+    M, K, N = len(X), len(X[0]), len(D[0])
+    n_ad, _, r_max = A.shape
+    wdX = [[Fraction(0)] * K for _ in range(M)]
+    wdA = np.zeros(A.shape, dtype=object); wdA[:] = Fraction(0)
+    wdB = np.zeros(B.shape, dtype=object); wdB[:] = Fraction(0)
+    for m in range(M):
+        a = int(ids[m])
+        if a < 0:
+            continue
+        r = int(ranks[a])
+        Af, Bf = _frac_bf16(A[a][:, :r]), _frac_bf16(B[a][:r, :])
+        s = Fraction(float(scales[a]))
+        u = [sum(D[m][n] * Bf[j][n] for n in range(N)) for j in range(r)]
+        v = [sum(X[m][k] * Af[k][j] for k in range(K)) for j in range(r)]
+        for k in range(K):
+            wdX[m][k] = s * sum(u[j] * Af[k][j] for j in range(r))
+            for j in range(r):
+                wdA[a, k, j] += s * X[m][k] * u[j]
+        for j in range(r):
+            for n in range(N):
+                wdB[a, j, n] += s * v[j] * D[m][n]
+    assert [[Fraction(float(t)) for t in row] for row in dX] == wdX
+    assert all(Fraction(float(g)) == w for g, w in zip(dA.ravel(), wdA.ravel()))
+    assert all(Fraction(float(g)) == w for g, w in zip(dB.ravel(), wdB.ravel()))
+
+
+def test_backward_base_term_is_the_adjoint_of_the_8bit_product():
+    """The base term of dX is the adjoint of y = x . W'^T, W'[n][k] = swT[k] WqT[k][n],
+    under the quantised upstream dY' = sd . dYq: <base, d> = <dY', d . W'^T>."""
+    rng = np.random.default_rng(21)
+    M, K, N = 6, 40, 24
+    x = wl.normal_bf16(rng, (M, K))
+    dY = wl.normal_bf16(rng, (M, N))
+    WT = wl.normal_bf16(rng, (K, N), 0.2)
+    WqT, swT = oracle.quantize_rows(WT)
+    dYq, sd = oracle.quantize_rows(dY)
+    A = np.zeros((1, K, 8), np.uint16)
+    B = np.zeros((1, 8, N), np.uint16)
+    ids = np.full(M, -1, np.int32)
+    dX, dA, dB = oracle.lora_backward(x, dY, A, B, None, None, ids, dYq, sd, WqT, swT)
+    Wp = (swT[:, None].astype(np.float64) * oracle.e4m3_to_f64(WqT)).T   # [N][K]
+    dYp = sd[:, None].astype(np.float64) * oracle.e4m3_to_f64(dYq)       # [M][N]
+    d = rng.standard_normal((M, K))
+    assert np.isclose(np.sum(dX * d), np.sum(dYp * (d @ Wp.T)), rtol=1e-12)
+    assert not dA.any() and not dB.any()   # no token has an adapter
+
+
+def test_backward_invariants():
+    rng, x, dY, A, B, ranks, scales, ids = _grad_problem(12, M=9)
+    dX, dA, dB = oracle.lora_backward(x, dY, A, B, ranks, scales, ids)
+    # tokens without an adapter get no adapter term; permuting tokens permutes dX only
+    assert not dX[ids < 0].any()
+    pi = rng.permutation(len(ids))
+    dX2, dA2, dB2 = oracle.lora_backward(x[pi], dY[pi], A, B, ranks, scales, ids[pi])
+    assert np.array_equal(dX2, dX[pi]) and np.allclose(dA2, dA) and np.allclose(dB2, dB)
+    # B = 0: u = 0, so dX and dA vanish while dB does not
+    B0 = np.where(B == wl.BF16_NAN, B, np.uint16(0))
+    dX0, dA0, dB0 = oracle.lora_backward(x, dY, A, B0, ranks, scales, ids)
+    assert not dX0.any() and not dA0.any() and dB0.any()
+    # the padding past each rank is never written
+    for a in range(A.shape[0]):
+        assert not dA[a, :, ranks[a]:].any() and not dB[a, ranks[a]:, :].any()
