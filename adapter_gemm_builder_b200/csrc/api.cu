@@ -69,6 +69,24 @@ size_t fp8_ws_layout(int M, int K, const lora_pool_t* pool, size_t* off_xq, size
     return off;
 }
 
+// Backward workspace: the forward GEMM's workspace for (M, K' = N, the transposed
+// pool) | A' = B^T [n_adapters][N][r_max] | B' = A^T [n_adapters][r_max][K] | u | v.
+size_t bwd_ws_layout(int M, const lora_pool_t* pool, size_t* off_at, size_t* off_bt, size_t* off_u,
+                     size_t* off_v)
+{
+    size_t a, b, c, d, e;
+    size_t off = align256(fp8_ws_layout(M, pool->h_out, pool, &a, &b, &c, &d, &e));
+    *off_at = off;
+    off += align256((size_t)pool->n_adapters * pool->h_out * pool->r_max * 2);
+    *off_bt = off;
+    off += align256((size_t)pool->n_adapters * pool->r_max * pool->h_in * 2);
+    *off_u = off;
+    off += align256((size_t)M * pool->r_max * 4);
+    *off_v = off;
+    off += align256((size_t)M * pool->r_max * 4);
+    return off;
+}
+
 constexpr unsigned long long kDefaultWaitNs = 2000000000ull;  // 2 s
 std::atomic<unsigned long long> g_wait_limit_ns{kDefaultWaitNs};
 std::atomic<int> g_inject_stall{0};
@@ -234,6 +252,11 @@ size_t lora_workspace_size(int op, int T, int K, const lora_pool_t* pool)
         if (!pool || check_pool(pool) != LORA_OK) return (size_t)-1;
         if (T == 0 || tile_tokens_for(T, pool->n_adapters) <= LORA_DECODE_TILE_TOKENS) return 0;
         return sgmv_stream_workspace_bytes(T, *pool);
+    case LORA_OP_FP8_BACKWARD: {
+        if (!pool || check_pool(pool) != LORA_OK || T < 1) return (size_t)-1;
+        size_t a, b, c, d;
+        return bwd_ws_layout(T, pool, &a, &b, &c, &d);
+    }
     case LORA_OP_FP8_GEMM:
     case LORA_OP_BF16_GEMM: {
         if (K <= 0) return (size_t)-1;
@@ -365,6 +388,54 @@ int fp8_gemm_lora_epilogue(const void* x, int M, int K, int N, const uint8_t* Wq
     const int st = fp8_gemm_check_args(x, M, K, N, Wq, w_scale, pool, seg, y);
     if (st != LORA_OK) return st;
     return gemm_lora_launch(1, x, M, K, N, Wq, w_scale, pool, seg, y, ws, ws_bytes, stream);
+}
+
+int fp8_lora_backward(const void* x, const void* dY, int M, int K, int N, const uint8_t* WqT,
+                      const float* swT, const lora_pool_t* pool, const lora_segments_t* seg, void* dX,
+                      float* dA, float* dB, void* ws, size_t ws_bytes, lora_stream_t stream)
+{
+    int st = check_pool(pool);
+    if (st != LORA_OK) return st;
+    if (pool->n_slices != 1 || pool->h_in != K || pool->h_out != N) return LORA_ERR_INVALID_ARG;
+    if ((st = check_segments(seg, pool->n_adapters)) != LORA_OK) return st;
+    if (M < 1 || seg->T != M || K % 8 || N % 16 || K < 8 || N < 16) return LORA_ERR_INVALID_ARG;
+    if (M > (1 << 24)) return LORA_ERR_UNSUPPORTED;
+    if (!x || !dY || !WqT || !swT || !dX || !dA || !dB) return LORA_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(dY) || !aligned16(WqT) || !aligned16(dX) || !aligned16(dA) ||
+        !aligned16(dB))
+        return LORA_ERR_INVALID_ARG;
+    size_t off_at, off_bt, off_u, off_v;
+    const size_t need = bwd_ws_layout(M, pool, &off_at, &off_bt, &off_u, &off_v);
+    if (!ws || ws_bytes < need || !aligned16(ws)) return LORA_ERR_WORKSPACE;
+    uint8_t* w = static_cast<uint8_t*>(ws);
+    cudaStream_t s = (cudaStream_t)stream;
+    // the transposed pool: A' = B^T (h_in' = N), B' = A^T (h_out' = K)
+    lora_pool_t pt = *pool;
+    pt.A = w + off_at;
+    pt.B = w + off_bt;
+    pt.h_in = N;
+    pt.h_out = K;
+    float* u = reinterpret_cast<float*>(w + off_u);
+    float* v = reinterpret_cast<float*>(w + off_v);
+    const size_t na = (size_t)pool->n_adapters;
+    // 1. the gradients of adapters without tokens are zero
+    if (cudaMemsetAsync(dA, 0, na * K * pool->r_max * 4, s) != cudaSuccess ||
+        cudaMemsetAsync(dB, 0, na * pool->r_max * N * 4, s) != cudaSuccess)
+        return LORA_ERR_CUDA;
+    // 2. A' = B^T and B' = A^T of the active adapters
+    if (launch_transpose_pool(*pool, *seg, const_cast<void*>(pt.A), const_cast<void*>(pt.B), s) != cudaSuccess)
+        return LORA_ERR_CUDA;
+    // 3. dX = dY.W + s (dY.B^T).A^T: the forward's fused 8-bit GEMM of dY with W^T
+    //    (quantised per input channel) and the transposed pool; its workspace leads
+    st = gemm_lora_launch(1, dY, M, N, K, WqT, swT, &pt, seg, dX, w, off_at, stream);
+    if (st != LORA_OK) return st;
+    // 4. u = dY.B^T and v = x.A per token, then dA = s x^T u and dB = s v^T dY per adapter
+    if (launch_sgmv(SGMV_SHRINK, dY, 0, pt, *seg, u, nullptr, s, false) != cudaSuccess ||
+        launch_sgmv(SGMV_SHRINK, x, 0, *pool, *seg, v, nullptr, s, false) != cudaSuccess ||
+        launch_grad_outer(true, x, u, K, *pool, *seg, dA, s) != cudaSuccess ||
+        launch_grad_outer(false, dY, v, N, *pool, *seg, dB, s) != cudaSuccess)
+        return LORA_ERR_CUDA;
+    return LORA_OK;
 }
 
 int lora_switch_merge(const void* W, int N, int K, const lora_pool_t* pool, const int32_t* sel,

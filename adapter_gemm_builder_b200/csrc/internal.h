@@ -32,6 +32,15 @@ size_t sgmv_stream_workspace_bytes(int T, const lora_pool_t& pool);
 cudaError_t launch_lora_switch_merge(const void* W, int N, int K, const lora_pool_t& pool, const int32_t* sel,
                                      const float* gates, int n_sel, void* W_out, cudaStream_t stream);
 
+// Adapter gradients (grad.cu): the transposed pool (A'_a = B_a^T [N][r_max],
+// B'_a = A_a^T [r_max][K]) of the active adapters, and the segmented outer
+// products dA_a = s_a x_a^T u_a ([K][r_max], row_major_long) or
+// dB_a = s_a v_a^T dY_a ([r_max][N]) of the active adapters.
+cudaError_t launch_transpose_pool(const lora_pool_t& pool, const lora_segments_t& seg, void* At, void* Bt,
+                                  cudaStream_t stream);
+cudaError_t launch_grad_outer(bool row_major_long, const void* lng, const float* shrt, int L,
+                              const lora_pool_t& pool, const lora_segments_t& seg, float* out, cudaStream_t stream);
+
 // Per-row E4M3 quantisation; row p of the output is row perm[p] of x
 // (perm == NULL: identity). The kernel also zeroes zero_words 32-bit words at
 // `zero` (may be NULL) and lets a programmatic dependent launch start early.

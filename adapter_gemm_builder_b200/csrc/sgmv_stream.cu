@@ -60,7 +60,6 @@ struct StreamParams {
     int* ctr;     // [0]: next item; [1 + s * n_rows + g]: shrink parts done of tile row g, slice s
     int T, n_adapters, h_in, h_out, r_max, n_slices, n_rows;
     int Pk, Pn, kp, np;  // parts per tile row and their spans (multiples of 64)
-    long long n_shrink, n_items;
     int stage_bytes;
     int xy_maps;
     uint32_t off_vf, off_bar;
@@ -157,15 +156,21 @@ sgmv_stream_kernel(const __grid_constant__ AMaps am, const StreamParams p)
                 if ((8 << i) <= p.r_max) ptx::tma_prefetch_desc(&am.m[i]);
             for (int i = 0; i < 4 && 16 * i < p.r_max; ++i) ptx::tma_prefetch_desc(&am.b[i]);
         }
+        // items are enumerated over the tile rows in use (the segment builder's count);
+        // the next item is claimed while the current one's copies are issued
+        const long long used = p.counts[3];
+        const long long n_shrink = used * p.n_slices * p.Pk;
+        const long long n_items = n_shrink + used * p.n_slices * p.Pn;
+        long long next = 0;
+        if (lane == 0) next = (long long)atomicAdd(p.ctr, 1);
         while (ok) {
-            long long item = 0;
-            if (lane == 0) item = (long long)atomicAdd(p.ctr, 1);
-            item = __shfl_sync(0xffffffffu, item, 0);
-            if (item >= p.n_items) break;
-            const bool shrink = item < p.n_shrink;
-            long long rem = shrink ? item : item - p.n_shrink;
+            const long long item = __shfl_sync(0xffffffffu, next, 0);
+            if (item >= n_items) break;
+            if (lane == 0) next = (long long)atomicAdd(p.ctr, 1);
+            const bool shrink = item < n_shrink;
+            long long rem = shrink ? item : item - n_shrink;
             const int P = shrink ? p.Pk : p.Pn;
-            const long long per_slice = (long long)p.n_rows * P;
+            const long long per_slice = used * P;
             const int slice = (int)(rem / per_slice);
             rem -= (long long)slice * per_slice;
             const int g = (int)(rem / P);
@@ -525,34 +530,51 @@ sgmv_stream_kernel(const __grid_constant__ AMaps am, const StreamParams p)
                 const uint32_t yb = base + (uint32_t)((wb >> 6) * r16 * 128);
                 uint16_t* yg = p.y + (size_t)slice * p.T * p.h_out;
                 if (live && small) {
-                    // one column pair per thread: y[t][n..n+1] += s * sum_j v[t][j] * B[j][n..n+1]
-                    for (int pp = tid; pp < (cw >> 1); pp += kCompute) {
-                        const int n = pp * 2;
+                    // four lanes per column pair, each over every fourth rank index j (its
+                    // loads unrolled by two), then a two-step shuffle sum:
+                    // y[t][n..n+1] += s * sum_j v[t][j] * B[j][n..n+1]
+                    const int jq = tid & 3;
+                    const int npairs = cw >> 1;
+                    for (int pb = 0; pb < npairs; pb += kCompute / 4) {  // uniform trip count
+                        const int pp = pb + (tid >> 2);
+                        const bool on = pp < npairs;
+                        const int n = on ? pp * 2 : 0;
                         float s0[kSmallTile], s1[kSmallTile];
 #pragma unroll
                         for (int t = 0; t < kSmallTile; ++t) s0[t] = s1[t] = 0.f;
-                        const uint32_t bcol = (uint32_t)((n >> 6) * r16 * 128 + (n & 7) * 2);
+                        const uint8_t* bcol = smem + (base - base_u) + (n >> 6) * r16 * 128 + (n & 7) * 2;
                         const int nc = (n >> 3) & 7;
-                        for (int j = 0; j < r; ++j) {
-                            const uint32_t bw = *reinterpret_cast<const uint32_t*>(
-                                smem + (base - base_u) + bcol + j * 128 + ((nc ^ (j & 7)) << 4));
-                            const float b0 = bf16_lo(bw), b1 = bf16_hi(bw);
+                        for (int j = jq; j < r; j += 8) {
+                            const uint32_t bw0 = *reinterpret_cast<const uint32_t*>(bcol + j * 128 + ((nc ^ (j & 7)) << 4));
+                            const int j1 = j + 4;
+                            const uint32_t bw1 = j1 < r ? *reinterpret_cast<const uint32_t*>(
+                                                              bcol + j1 * 128 + ((nc ^ (j1 & 7)) << 4))
+                                                        : 0u;
 #pragma unroll
                             for (int t = 0; t < kSmallTile; ++t)
                                 if (t < nt) {
-                                    const float vv = VF[t * 64 + j];
-                                    s0[t] = fmaf(vv, b0, s0[t]);
-                                    s1[t] = fmaf(vv, b1, s1[t]);
+                                    const float v0 = VF[t * 64 + j], v1 = j1 < r ? VF[t * 64 + j1] : 0.f;
+                                    s0[t] = fmaf(v0, bf16_lo(bw0), fmaf(v1, bf16_lo(bw1), s0[t]));
+                                    s1[t] = fmaf(v0, bf16_hi(bw0), fmaf(v1, bf16_hi(bw1), s1[t]));
                                 }
                         }
 #pragma unroll
-                        for (int t = 0; t < kSmallTile; ++t)
-                            if (t < nt) {
-                                const uint32_t yw = *reinterpret_cast<const uint32_t*>(
-                                    smem + (yb - base_u) + blk_chunk(t, n >> 3, Mtr) + (n & 7) * 2);
-                                *reinterpret_cast<uint32_t*>(yg + (size_t)h.tok[t] * p.h_out + c0 + n) =
-                                    pack_bf16x2(bf16_lo(yw) + scale * s0[t], bf16_hi(yw) + scale * s1[t]);
-                            }
+                        for (int t = 0; t < kSmallTile; ++t) {
+                            s0[t] += __shfl_xor_sync(0xffffffffu, s0[t], 1);
+                            s1[t] += __shfl_xor_sync(0xffffffffu, s1[t], 1);
+                            s0[t] += __shfl_xor_sync(0xffffffffu, s0[t], 2);
+                            s1[t] += __shfl_xor_sync(0xffffffffu, s1[t], 2);
+                        }
+                        if (on && jq < nt) {  // lane jq of the four stores token jq
+#pragma unroll
+                            for (int t = 0; t < kSmallTile; ++t)
+                                if (t == jq) {
+                                    const uint32_t yw = *reinterpret_cast<const uint32_t*>(
+                                        smem + (yb - base_u) + blk_chunk(t, n >> 3, Mtr) + (n & 7) * 2);
+                                    *reinterpret_cast<uint32_t*>(yg + (size_t)h.tok[t] * p.h_out + c0 + n) =
+                                        pack_bf16x2(bf16_lo(yw) + scale * s0[t], bf16_hi(yw) + scale * s1[t]);
+                                }
+                        }
                     }
                 } else if (live) {
                     if (r != r16) {  // B rows r..r16 of every box hold padding or nothing: zero them
@@ -662,19 +684,19 @@ cudaError_t launch_sgmv_stream(const void* x, int64_t x_slice_stride, const lora
     p.inject_stall = debug_inject_stall();
 
     // Parts per tile row: about three shrink and three expand items per CTA of the
-    // grid, counted on the bound of the tile rows (some may be unused).
+    // grid, counted on an estimate of the tile rows in use (at most the bound, and
+    // at most one row per 4 tokens: many adapters hold only a few tokens each).
     const int sms = device_sm_count();
     const long long G = 2LL * sms;
     const long long rows = (long long)p.n_rows * pool.n_slices;
-    long long P = (3 * G + rows - 1) / rows;
+    const long long rows_est = (long long)min(p.n_rows, (seg.T + 3) / 4) * pool.n_slices;
+    long long P = (3 * G + rows_est - 1) / rows_est;
     P = P < 1 ? 1 : (P > 16 ? 16 : P);
     auto span = [&](int h) { return (int)(((h + P - 1) / P + 63) / 64 * 64); };
     p.kp = span(pool.h_in);
     p.np = span(pool.h_out);
     p.Pk = (pool.h_in + p.kp - 1) / p.kp;
     p.Pn = (pool.h_out + p.np - 1) / p.np;
-    p.n_shrink = rows * p.Pk;
-    p.n_items = p.n_shrink + rows * p.Pn;
 
     uint8_t* w = static_cast<uint8_t*>(ws);
     const size_t ctr_bytes = ((1 + (size_t)rows) * 4 + 255) / 256 * 256;
@@ -715,7 +737,7 @@ cudaError_t launch_sgmv_stream(const void* x, int64_t x_slice_stride, const lora
     e = cudaFuncSetAttribute(sgmv_stream_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     long long grid = G;
-    if (grid > p.n_items) grid = p.n_items;
+    if (grid > rows * (p.Pk + p.Pn)) grid = rows * (p.Pk + p.Pn);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid, 1, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);

@@ -29,6 +29,7 @@ LORA_OP_EXPAND = 1
 LORA_OP_APPLY = 2
 LORA_OP_FP8_GEMM = 3
 LORA_OP_BF16_GEMM = 4
+LORA_OP_FP8_BACKWARD = 5
 
 EXPORTED = [
     "lora_workspace_size", "lora_workspace_init", "lora_workspace_status", "lora_build_segments",
@@ -36,7 +37,7 @@ EXPORTED = [
     "lora_status_string", "lora_version", "lora_tile_tokens", "lora_tile_tokens_for", "lora_max_tiles",
     "lora_segments_status", "fp8_gemm_lora_epilogue_noalloc", "lora_noalloc_scratch_bytes",
     "lora_noalloc_status", "lora_debug_set_wait_limit", "bf16_gemm_lora_epilogue",
-    "lora_switch_merge",
+    "lora_switch_merge", "fp8_lora_backward",
 ]
 
 
@@ -102,6 +103,7 @@ def load(path: str = LIB_PATH):
             "lora_debug_set_wait_limit": (I, [ctypes.c_uint64, I]),
             "bf16_gemm_lora_epilogue": (I, [P, I, I, I, P, P, P, P, P, Z, P]),
             "lora_switch_merge": (I, [P, I, I, P, P, P, I, P, P]),
+            "fp8_lora_backward": (I, [P, P, I, I, I, P, P, P, P, P, P, P, P, Z, P]),
         }
         for name, (res, args) in sig.items():
             f = getattr(lib, name)
@@ -273,6 +275,17 @@ def bf16_gemm_lora_epilogue(x: torch.Tensor, W: torch.Tensor, pool: Pool | None,
     _check(load().bf16_gemm_lora_epilogue(
         _ptr(x), M, K, N, _ptr(W), ctypes.byref(pool.c) if pool else None,
         ctypes.byref(seg.c) if seg else None, _ptr(y), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def fp8_lora_backward(x: torch.Tensor, dY: torch.Tensor, WqT: torch.Tensor, swT: torch.Tensor,
+                      pool: Pool, seg: Segments, dX: torch.Tensor, dA: torch.Tensor, dB: torch.Tensor,
+                      ws: torch.Tensor, stream=None) -> None:
+    """Gradients of y = x.W^T + s_a (x.A_a).B_a on a frozen FP8 base (see fp8_lora_backward)."""
+    M, K = x.shape
+    N = dY.shape[1]
+    _check(load().fp8_lora_backward(_ptr(x), _ptr(dY), M, K, N, _ptr(WqT), _ptr(swT),
+                                    ctypes.byref(pool.c), ctypes.byref(seg.c), _ptr(dX), _ptr(dA),
+                                    _ptr(dB), _ptr(ws), ws.numel(), _stream(stream)))
 
 
 def lora_switch_merge(W: torch.Tensor, pool: Pool, sel: torch.Tensor, gates: torch.Tensor,

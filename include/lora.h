@@ -144,6 +144,7 @@ LORA_API int lora_segments_status(const lora_segments_t* seg, lora_stream_t stre
 #define LORA_OP_APPLY 2
 #define LORA_OP_FP8_GEMM 3
 #define LORA_OP_BF16_GEMM 4
+#define LORA_OP_FP8_BACKWARD 5
 
 /*
  * Bytes of workspace an operation needs (0 if it needs none), or (size_t)-1
@@ -284,6 +285,35 @@ LORA_API int fp8_gemm_lora_epilogue(const void* x, int M, int K, int N, const ui
 LORA_API int bf16_gemm_lora_epilogue(const void* x, int M, int K, int N, const void* W,
                                      const lora_pool_t* pool, const lora_segments_t* seg, void* y,
                                      void* ws, size_t ws_bytes, lora_stream_t stream);
+
+/*
+ * Gradients of the LoRA layer for training the adapters on a frozen 8-bit
+ * base (EpiLoRA abstract, sentence 6: a trainer that keeps the base weights
+ * in FP8; the chain rule of y = x.W^T + s_a (x.A_a).B_a of the Punica
+ * README's "How?"). For the upstream gradient dY, per token m with adapter a:
+ *   dX[m][k]   = bf16( sd[m] swT[k] sum_n dYq[m][n] WqT[k][n]
+ *                      + s_a sum_j u[m][j] A_a[k][j] ),  u = dY.B_a^T (fp32)
+ *   dA_a[k][j] = s_a sum_{m with adapter a} x[m][k] u[m][j]    (fp32)
+ *   dB_a[j][n] = s_a sum_{m with adapter a} v[m][j] dY[m][n],  v = x.A_a (fp32)
+ * The base term is the backward's 8-bit GEMM: dY quantised per token as
+ * fp8_quantize_rows does (sd, dYq), and W^T quantised per input channel once
+ * by the caller (WqT = E4M3 [K][N], swT [K], e.g. fp8_quantize_rows of W^T).
+ * Launches: two memsets (dA, dB: adapters without tokens get zero), a
+ * transpose of the active adapters' A and B into the workspace, the fused
+ * GEMM of fp8_gemm_lora_epilogue on (dY, W^T, the transposed pool) for dX,
+ * two shrinks (u, v), and one segmented outer-product kernel each for dA, dB.
+ *   x bf16 [M][K]; dY bf16 [M][N]; dX bf16 [M][K] (out);
+ *   dA fp32 [n_adapters][K][r_max], dB fp32 [n_adapters][r_max][N] (out; the
+ *   padding past each rank is written as zero);
+ *   pool: n_slices == 1, h_in == K, h_out == N; seg built for these M tokens;
+ *   ws: lora_workspace_size(LORA_OP_FP8_BACKWARD, M, K, pool) bytes.
+ * Limits: K % 8 == 0, N % 16 == 0. The residency note of
+ * fp8_gemm_lora_epilogue applies to its GEMM.
+ */
+LORA_API int fp8_lora_backward(const void* x, const void* dY, int M, int K, int N, const uint8_t* WqT,
+                               const float* swT, const lora_pool_t* pool, const lora_segments_t* seg,
+                               void* dX, float* dA, float* dB, void* ws, size_t ws_bytes,
+                               lora_stream_t stream);
 
 /*
  * Token-wise merge of router-selected adapters into the backbone (LoRA-Switch
