@@ -52,8 +52,17 @@ int check_segments(const lora_segments_t* seg, int n_adapters)
 
 // GEMM workspace: status | xq (esz bytes per element) | sx | v (with a pool) |
 // sync words | partials. [off_v, off_part) is zeroed by the quantiser on every call.
+// Batches whose adapters are too many to fold into the GEMM's accumulator (more
+// than kFuseMaxAdapters in the pool and in the batch) run the base GEMM and then
+// the SGMV apply instead (see gemm_lora_launch).
+constexpr int kFuseMaxAdapters = 16;
+bool gemm_split(int M, const lora_pool_t* pool)
+{
+    return pool && pool->n_adapters > kFuseMaxAdapters && M > kFuseMaxAdapters;
+}
+
 size_t fp8_ws_layout(int M, int K, const lora_pool_t* pool, size_t* off_xq, size_t* off_sx,
-                     size_t* off_v, size_t* off_sync, size_t* off_part, int esz = 1)
+                     size_t* off_v, size_t* off_sync, size_t* off_part, int esz = 1, size_t* off_apply = nullptr)
 {
     size_t off = 256;  // status word block
     *off_xq = off;
@@ -66,6 +75,8 @@ size_t fp8_ws_layout(int M, int K, const lora_pool_t* pool, size_t* off_xq, size
     off += align256((size_t)(16 + device_sm_count()) * 4);
     *off_part = off;
     off += align256(fp8_gemm_partial_bytes(M));
+    if (off_apply) *off_apply = off;
+    if (gemm_split(M, pool)) off += align256(sgmv_stream_workspace_bytes(M, *pool));
     return off;
 }
 
@@ -124,9 +135,12 @@ int gemm_lora_launch(int esz, const void* x, int M, int K, int N, const uint8_t*
                      const lora_pool_t* pool, const lora_segments_t* seg, void* y, void* ws,
                      size_t ws_bytes, lora_stream_t stream)
 {
-    size_t off_xq, off_sx, off_v, off_sync, off_part;
-    const size_t need = fp8_ws_layout(M, K, pool, &off_xq, &off_sx, &off_v, &off_sync, &off_part, esz);
+    size_t off_xq, off_sx, off_v, off_sync, off_part, off_apply;
+    const size_t need =
+        fp8_ws_layout(M, K, pool, &off_xq, &off_sx, &off_v, &off_sync, &off_part, esz, &off_apply);
     if (!ws || ws_bytes < need || !aligned16(ws)) return LORA_ERR_WORKSPACE;
+    const bool split = gemm_split(M, pool);
+    const lora_pool_t* fused = split ? nullptr : pool;  // the adapters folded into the GEMM
     uint8_t* w = static_cast<uint8_t*>(ws);
     uint32_t* status = reinterpret_cast<uint32_t*>(w);
     uint8_t* xq = w + off_xq;
@@ -137,7 +151,7 @@ int gemm_lora_launch(int esz, const void* x, int M, int K, int N, const uint8_t*
 
     // 1. activations -> E4M3 (or copied as bf16), rows in segment order when adapters
     //    are present; the same kernel zeroes v and the GEMM's synchronisation words
-    cudaError_t e = launch_quantize_rows(x, pool ? seg->perm : nullptr, M, K, xq, sx, w + off_v,
+    cudaError_t e = launch_quantize_rows(x, fused ? seg->perm : nullptr, M, K, xq, sx, w + off_v,
                                          (off_part - off_v) / 4, s, esz == 2);
     if (e != cudaSuccess) return LORA_ERR_CUDA;
     // 2. the GEMM, a programmatic dependent of the quantiser: its weights start
@@ -157,8 +171,8 @@ int gemm_lora_launch(int esz, const void* x, int M, int K, int N, const uint8_t*
     a.partials = reinterpret_cast<float*>(w + off_part);
     a.v_done = sync;
     a.flags = sync + 16;
-    a.lora = pool != nullptr;
-    if (pool) {
+    a.lora = fused != nullptr;
+    if (fused) {
         a.perm = seg->perm;
         a.tok_adapter = seg->tok_adapter;
         a.indptr = seg->indptr;
@@ -173,7 +187,13 @@ int gemm_lora_launch(int esz, const void* x, int M, int K, int N, const uint8_t*
         a.n_adapters = pool->n_adapters;
         a.r_max = pool->r_max;
     }
-    return cuda_status(launch_fp8_gemm(a, s));
+    e = launch_fp8_gemm(a, s);
+    if (e != cudaSuccess || !split) return cuda_status(e);
+    // 3. many adapters: their term added to the GEMM's bf16 output by the SGMV apply
+    //    (the kernel lora_apply picks for this batch)
+    if (tile_tokens_for(M, pool->n_adapters) <= LORA_DECODE_TILE_TOKENS)
+        return cuda_status(launch_sgmv(SGMV_APPLY, x, 0, *pool, *seg, nullptr, y, s, false));
+    return cuda_status(launch_sgmv_stream(x, 0, *pool, *seg, y, w + off_apply, s));
 }
 
 }  // namespace

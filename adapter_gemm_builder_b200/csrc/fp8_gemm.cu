@@ -58,6 +58,7 @@ constexpr int kEpiThreads = kEpiWarps * 32;
 constexpr int kThreads = (3 + kEpiWarps) * 32;
 constexpr int kMaxStages = 8;
 constexpr int kShrinkCols = 64;  // K columns of the down-projection per work item
+constexpr int kShrinkTok = 64;   // tokens of the down-projection per work item
 constexpr unsigned long long kTimeoutNs = 2000000000ull;  // drains after an abort
 
 struct GemmParams {
@@ -575,24 +576,30 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
         ptx::pdl_wait();  // xq, sx and the zeroed v / flags / count come from the quantiser
         bool ok = true;
 
-        // ---- down-projection: work item q = 64 columns of K for every token
+        // ---- down-projection: work item = 64 columns of K (q) for a block of up to 64
+        // tokens (so that a large M spreads over every CTA)
         const int n_chunks = (p.K + kShrinkCols - 1) / kShrinkCols;
+        const int n_tblk = (p.M + kShrinkTok - 1) / kShrinkTok;
+        const int n_dp = n_chunks * n_tblk;
         if (p.lora) {
             const int ng = p.r_max >> 3;  // groups of 8 rank columns (a power of two)
             const int lg = __ffs(ng) - 1;
-            // with few (token, group) pairs, split the 64 columns over up to 4 threads
-            int ls = 0;
-            while (ls < 2 && (p.M << (lg + ls + 1)) <= kEpiThreads) ++ls;
-            const int kspan = kShrinkCols >> ls;  // 64, 32 or 16 columns per thread
-            const int total = p.M << (lg + ls);
-            for (int q = cta; q < n_chunks && ok; q += G) {
+            for (int it = cta; it < n_dp && ok; it += G) {
+                const int q = it % n_chunks, tblk = it / n_chunks;
+                const int t_base = tblk * kShrinkTok;
+                const int Mtb = min(kShrinkTok, p.M - t_base);
+                // with few (token, group) pairs, split the 64 columns over up to 4 threads
+                int ls = 0;
+                while (ls < 2 && (Mtb << (lg + ls + 1)) <= kEpiThreads) ++ls;
+                const int kspan = kShrinkCols >> ls;  // 64, 32 or 16 columns per thread
+                const int total = Mtb << (lg + ls);
                 float* vcopy = p.v + (size_t)(q & (p.v_rep - 1)) * p.M * p.r_max;
                 // work items w: (token, group of 8 ranks, K sub-range); the 2^ls sub-ranges of
                 // one (token, group) sit in consecutive lanes, the loop is uniform per warp
                 for (int wb = ew * 32; wb < total; wb += kEpiThreads) {
                     const int w = wb + lane;
                     const int pg = w >> ls, sub = w & ((1 << ls) - 1);
-                    const int pp = pg >> lg, g = pg & (ng - 1);
+                    const int pp = t_base + (pg >> lg), g = pg & (ng - 1);
                     const int k0 = q * kShrinkCols + sub * kspan;
                     int kw = min(kspan, p.K - k0);  // a multiple of 16 (or <= 0)
                     int r = 0, m = 0, a = -1;
@@ -683,7 +690,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
             }
             if (staged_tb != tb) {
                 if (!v_ready) {  // every CTA's share of the down-projection is in v
-                    if (etid == 0) ok = wait_count(p.v_done, n_chunks, abort_flag, p.status, 0x80u, p.timeout_ns);
+                    if (etid == 0) ok = wait_count(p.v_done, n_dp, abort_flag, p.status, 0x80u, p.timeout_ns);
                     if (!(ok = epi_sync() && ok)) break;
                     v_ready = true;
                 }

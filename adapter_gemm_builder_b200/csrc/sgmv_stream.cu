@@ -156,34 +156,67 @@ sgmv_stream_kernel(const __grid_constant__ AMaps am, const StreamParams p)
                 if ((8 << i) <= p.r_max) ptx::tma_prefetch_desc(&am.m[i]);
             for (int i = 0; i < 4 && 16 * i < p.r_max; ++i) ptx::tma_prefetch_desc(&am.b[i]);
         }
-        // items are enumerated over the tile rows in use (the segment builder's count);
-        // the next item is claimed while the current one's copies are issued
+        // Items are enumerated over the tile rows in use (the segment builder's count).
+        // The producer's per-item metadata is a chain of dependent loads (claim -> tile
+        // row -> rank, scale, token ids); it is software-pipelined so that each link is
+        // consumed one item after it was issued, while the current item's copies go out:
+        // claims run two items ahead, tile rows one item ahead.
         const long long used = p.counts[3];
         const long long n_shrink = used * p.n_slices * p.Pk;
         const long long n_items = n_shrink + used * p.n_slices * p.Pn;
-        long long next = 0;
-        if (lane == 0) next = (long long)atomicAdd(p.ctr, 1);
-        while (ok) {
-            const long long item = __shfl_sync(0xffffffffu, next, 0);
-            if (item >= n_items) break;
-            if (lane == 0) next = (long long)atomicAdd(p.ctr, 1);
-            const bool shrink = item < n_shrink;
-            long long rem = shrink ? item : item - n_shrink;
-            const int P = shrink ? p.Pk : p.Pn;
+        struct Meta {
+            long long item;
+            int shrink, slice, g, part;
+            int4 tl;
+            int r, t_lo, t_hi;
+            float scale;
+        };
+        auto decode = [&](long long item, Meta& m) {  // issues the tile-row load
+            m.item = item;
+            if (item >= n_items) return;
+            m.shrink = item < n_shrink;
+            long long rem = m.shrink ? item : item - n_shrink;
+            const int P = m.shrink ? p.Pk : p.Pn;
             const long long per_slice = used * P;
-            const int slice = (int)(rem / per_slice);
-            rem -= (long long)slice * per_slice;
-            const int g = (int)(rem / P);
-            const int part = (int)(rem - (long long)g * P);
-            const int4 tl = p.tiles[g];
-            const int nt = tl.z;
-            if (nt <= 0) continue;  // unused tile row
-            const int a = tl.x, tok0 = tl.y;
-            int r = p.ranks ? p.ranks[a] : p.r_max;
-            r = max(1, min(r, p.r_max));
-            const float scale = p.scales ? p.scales[a] : 1.0f;
-            const int t_lo = lane < nt ? p.perm[tok0 + lane] : 0;
-            const int t_hi = lane + 32 < nt ? p.perm[tok0 + lane + 32] : 0;
+            m.slice = (int)(rem / per_slice);
+            rem -= (long long)m.slice * per_slice;
+            m.g = (int)(rem / P);
+            m.part = (int)(rem - (long long)m.g * P);
+            m.tl = p.tiles[m.g];
+        };
+        auto resolve = [&](Meta& m) {  // issues the loads that need the tile row
+            if (m.item >= n_items) return;
+            const int a = m.tl.x, nt = m.tl.z;
+            m.r = p.ranks ? p.ranks[a] : p.r_max;
+            m.scale = p.scales ? p.scales[a] : 1.0f;
+            m.t_lo = lane < nt ? p.perm[m.tl.y + lane] : 0;
+            m.t_hi = lane + 32 < nt ? p.perm[m.tl.y + lane + 32] : 0;
+        };
+        long long claim = 0;
+        Meta m0, m1;
+        if (lane == 0) claim = (long long)atomicAdd(p.ctr, 1);
+        decode(__shfl_sync(0xffffffffu, claim, 0), m0);
+        if (lane == 0) claim = (long long)atomicAdd(p.ctr, 1);
+        decode(__shfl_sync(0xffffffffu, claim, 0), m1);
+        if (lane == 0 && m1.item < n_items) claim = (long long)atomicAdd(p.ctr, 1);
+        resolve(m0);
+        while (ok && m0.item < n_items) {
+            resolve(m1);
+            Meta m2;
+            m2.item = n_items;
+            if (m1.item < n_items) {
+                decode(__shfl_sync(0xffffffffu, claim, 0), m2);
+                if (lane == 0 && m2.item < n_items) claim = (long long)atomicAdd(p.ctr, 1);
+            }
+            const bool shrink = m0.shrink;
+            const int slice = m0.slice, g = m0.g, part = m0.part;
+            const int nt = m0.tl.z;
+            const int a = m0.tl.x;
+            const int r = max(1, min(m0.r, p.r_max));
+            const float scale = m0.scale;
+            const int t_lo = m0.t_lo, t_hi = m0.t_hi;
+            m0 = m1;
+            m1 = m2;
             const bool small = nt <= kSmallTile;
             const int Mt = (nt + 15) >> 4;
             const int Mtr = small ? nt : Mt * 16;
