@@ -14,6 +14,8 @@ cites the passage of the pages it follows in ``oracle.c``:
   EpiLoRA abstract, sentence 1.
 * Token-wise merge of router-selected adapters into the backbone weight:
   LoRA-Switch abstract (shd-paper.top page).
+* 4-bit (OCP MX FP4) weights with the LoRA term, bf16 activations:
+  EpiLoRA abstract, sentences 2 and 6.
 * Gradients of the layer for training adapters on a frozen FP8 base:
   EpiLoRA abstract, sentence 6 (with the Punica README's algebra).
 * FP8 base GEMM whose epilogue adds each tenant's up-projection:
@@ -79,6 +81,16 @@ def _load():
             lib.orc_lora_switch_merge.argtypes = [P, I, I, P, P, I, I, P, P, P, P, I, P]
             lib.orc_lora_backward.restype = None
             lib.orc_lora_backward.argtypes = [P, P, I, I, I, P, P, P, P, P, P, I, I, P, P, P, P, P, P]
+            lib.orc_e2m1_decode.restype = ctypes.c_double
+            lib.orc_e2m1_decode.argtypes = [ctypes.c_uint8]
+            lib.orc_e8m0_decode.restype = ctypes.c_double
+            lib.orc_e8m0_decode.argtypes = [ctypes.c_uint8]
+            lib.orc_e2m1_encode.restype = ctypes.c_uint8
+            lib.orc_e2m1_encode.argtypes = [ctypes.c_double]
+            lib.orc_mxfp4_quantize.restype = None
+            lib.orc_mxfp4_quantize.argtypes = [P, I, I, P, P]
+            lib.orc_mxfp4_gemm_lora_sampled.restype = None
+            lib.orc_mxfp4_gemm_lora_sampled.argtypes = [P, P, P, I, P, P, I, I, I, P, P, P, P, P, I, P]
             lib.orc_num_threads.restype = I
             lib.orc_set_num_threads.argtypes = [I]
             _lib = lib
@@ -267,3 +279,47 @@ def lora_backward(x, dY, A, B, ranks, scales, ids, dYq=None, sd=None, WqT=None, 
     lib.orc_lora_backward(_p(x), _p(dY), M, K, N, _p(dYq), _p(sd), _p(WqT), _p(swT), _p(A), _p(B),
                           n_adapters, r_max, _p(ranks), _p(scales), _p(ids), _p(dX), _p(dA), _p(dB))
     return dX, dA, dB
+
+
+def e2m1_decode(c: int) -> float:
+    return _load().orc_e2m1_decode(int(c))
+
+
+def e8m0_decode(e: int) -> float:
+    return _load().orc_e8m0_decode(int(e))
+
+
+def e2m1_encode(f: float) -> int:
+    return int(_load().orc_e2m1_encode(float(f)))
+
+
+def mxfp4_quantize(W):
+    """W bf16 [N, K] (K % 32 == 0) -> (codes uint8 [N, K], one E2M1 code per byte;
+    scales uint8 [N, K / 32], E8M0)."""
+    lib = _load()
+    W = _c(W, np.uint16)
+    N, K = W.shape
+    codes = np.zeros((N, K), np.uint8)
+    scales = np.zeros((N, K // 32), np.uint8)
+    lib.orc_mxfp4_quantize(_p(W), N, K, _p(codes), _p(scales))
+    return codes, scales
+
+
+def mxfp4_gemm_lora_sampled(x, codes, scales, rows, cols, A=None, B=None, ranks=None,
+                            scales_lora=None, ids=None) -> np.ndarray:
+    lib = _load()
+    x = _c(x, np.uint16); codes = _c(codes, np.uint8); scales = _c(scales, np.uint8)
+    rows = _c(rows, np.int32); cols = _c(cols, np.int32)
+    K = x.shape[1]
+    N = codes.shape[0]
+    if A is not None:
+        A = _c(A, np.uint16); B = _c(B, np.uint16); ranks = _c(ranks, np.int32)
+        scales_lora = _c(scales_lora, np.float32); ids = _c(ids, np.int32)
+        n_adapters, _, r_max = A.shape
+    else:
+        n_adapters, r_max = 0, 0
+    out = np.zeros(rows.shape[0], np.float64)
+    lib.orc_mxfp4_gemm_lora_sampled(_p(x), _p(codes), _p(scales), K, _p(A), _p(B), n_adapters, r_max,
+                                    N, _p(ranks), _p(scales_lora), _p(ids), _p(rows), _p(cols),
+                                    rows.shape[0], _p(out))
+    return out

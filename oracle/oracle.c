@@ -96,6 +96,43 @@ uint8_t orc_e4m3_encode(float f)
     return sign | (uint8_t)best;
 }
 
+/* OCP MX FP4 element (E2M1): 1 sign, 2 exponent bits (bias 1), 1 fraction
+ * bit; no infinities or NaN; magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6. */
+double orc_e2m1_decode(uint8_t c)
+{
+    int s = (c >> 3) & 1;
+    int e = (c >> 1) & 3;
+    int m = c & 1;
+    double v = (e == 0) ? 0.5 * m : ldexp(1.0 + 0.5 * m, e - 1);
+    return s ? -v : v;
+}
+
+/* OCP MX E8M0 block scale: 2^(E - 127); 255 is NaN. */
+double orc_e8m0_decode(uint8_t e)
+{
+    return e == 255 ? NAN : ldexp(1.0, (int)e - 127);
+}
+
+/* Nearest E2M1 code to a (finite) value, ties to the code whose fraction bit
+ * is 0, magnitudes beyond 6 saturated to 6 (brute force over the 8 codes). */
+uint8_t orc_e2m1_encode(double f)
+{
+    uint8_t sign = signbit(f) ? 8 : 0;
+    double a = fabs(f);
+    if (a >= 6.0)
+        return sign | 7;
+    int best = 0;
+    double best_d = a;
+    for (int c = 1; c <= 7; ++c) {
+        double d = fabs(a - orc_e2m1_decode((uint8_t)c));
+        if (d < best_d || (d == best_d && (c & 1) == 0 && (best & 1) == 1)) {
+            best = c;
+            best_d = d;
+        }
+    }
+    return sign | (uint8_t)best;
+}
+
 /* ------------------------------------------------------------------ */
 /* Segments: stable group-by of token indices by adapter id.           */
 /* ------------------------------------------------------------------ */
@@ -469,6 +506,89 @@ void orc_lora_backward(const uint16_t* x, const uint16_t* dY, int M, int K, int 
     }
     free(u);
     free(v);
+}
+
+/*
+ * MXFP4 quantisation of weight rows (the 4-bit base of the EpiLoRA abstract,
+ * sentence 2, read as the OCP MX format): every block of 32 consecutive
+ * values of a row shares one E8M0 scale X = 2^(floor(log2(amax)) - 2) (2 is
+ * the exponent of E2M1's largest value, 6 = 1.5 * 2^2; the E8M0 exponent is
+ * clamped to 0..254, and an all-zero block takes the smallest scale), and
+ * each value is rounded to E2M1 as v / X (nearest, ties to even fraction,
+ * saturating to +-6). W bf16 [N][K], K a multiple of 32; codes [N][K]
+ * (one E2M1 code per byte); scales [N][K / 32] (E8M0 bytes).
+ */
+void orc_mxfp4_quantize(const uint16_t* W, int N, int K, uint8_t* codes, uint8_t* scales)
+{
+#pragma omp parallel for schedule(static)
+    for (int n = 0; n < N; ++n) {
+        for (int b = 0; b < K / 32; ++b) {
+            double amax = 0.0;
+            for (int i = 0; i < 32; ++i) {
+                double a = fabs(orc_bf16_decode(W[(size_t)n * K + b * 32 + i]));
+                if (a > amax)
+                    amax = a;
+            }
+            int e = 0;
+            if (amax > 0.0) {
+                e = (int)floor(log2(amax)) - 2 + 127;
+                if (e < 0)
+                    e = 0;
+                if (e > 254)
+                    e = 254;
+            }
+            scales[(size_t)n * (K / 32) + b] = (uint8_t)e;
+            double x = orc_e8m0_decode((uint8_t)e);
+            for (int i = 0; i < 32; ++i) {
+                double v = orc_bf16_decode(W[(size_t)n * K + b * 32 + i]);
+                codes[(size_t)n * K + b * 32 + i] = orc_e2m1_encode(v / x);
+            }
+        }
+    }
+}
+
+/*
+ * The MXFP4 base GEMM with the LoRA term, at the listed (m, n) samples, with
+ * the activations kept in bf16 (the 16-bit activation engine of the EpiLoRA
+ * abstract, sentence 6):
+ *   y[m][n] = sum_k x[m][k] * E2M1(codes[n][k]) * E8M0(scales[n][k / 32])
+ *           + s_a * sum_{j < r_a} (sum_k x[m][k] A[a][k][j]) * B[a][j][n].
+ * A == NULL: no LoRA term. Layouts as orc_mxfp4_quantize.
+ */
+void orc_mxfp4_gemm_lora_sampled(const uint16_t* x, const uint8_t* codes, const uint8_t* scales,
+                                 int K, const uint16_t* A, const uint16_t* B, int n_adapters,
+                                 int r_max, int h_out, const int32_t* ranks,
+                                 const float* scales_lora, const int32_t* ids,
+                                 const int32_t* rows, const int32_t* cols, int n_samples,
+                                 double* out)
+{
+#pragma omp parallel for schedule(dynamic, 16)
+    for (int i = 0; i < n_samples; ++i) {
+        int m = rows[i], n = cols[i];
+        double acc = 0.0;
+        for (int k = 0; k < K; ++k)
+            acc += orc_bf16_decode(x[(size_t)m * K + k]) *
+                   orc_e2m1_decode(codes[(size_t)n * K + k]) *
+                   orc_e8m0_decode(scales[(size_t)n * (K / 32) + k / 32]);
+        double y = acc;
+        if (A != NULL) {
+            int a = valid_id(ids, m, n_adapters);
+            if (a >= 0) {
+                int r = rank_of(ranks, a, r_max);
+                double s = scales_lora ? (double)scales_lora[a] : 1.0;
+                double l = 0.0;
+                for (int j = 0; j < r; ++j) {
+                    double vj = 0.0;
+                    for (int k = 0; k < K; ++k)
+                        vj += orc_bf16_decode(x[(size_t)m * K + k]) *
+                              orc_bf16_decode(A[((size_t)a * K + k) * r_max + j]);
+                    l += vj * orc_bf16_decode(B[((size_t)a * r_max + j) * h_out + n]);
+                }
+                y += s * l;
+            }
+        }
+        out[i] = y;
+    }
 }
 
 /* Threads the OpenMP loops above use. */

@@ -686,3 +686,109 @@ def test_backward_invariants():
     # the padding past each rank is never written
     for a in range(A.shape[0]):
         assert not dA[a, :, ranks[a]:].any() and not dB[a, ranks[a]:, :].any()
+
+
+# ---------------------------------------------------------------- MX FP4 (4-bit base)
+
+def test_e2m1_decode_golden_values():
+    with open(os.path.join(GOLDEN, "e2m1_values.txt")) as f:
+        rows = [l.split() for l in f if l.strip() and not l.startswith("#")]
+    assert len(rows) == 16
+    for code, val in rows:
+        got = oracle.e2m1_decode(int(code, 16))
+        assert got == float(val) and math.copysign(1, got) == math.copysign(1, float(val)), code
+
+
+def test_e8m0_decode():
+    assert oracle.e8m0_decode(127) == 1.0 and oracle.e8m0_decode(128) == 2.0
+    assert oracle.e8m0_decode(0) == 2.0 ** -127 and oracle.e8m0_decode(254) == 2.0 ** 127
+    assert math.isnan(oracle.e8m0_decode(255))
+
+
+def test_e2m1_encode_round_trip_ties_and_saturation():
+    for c in range(16):
+        assert oracle.e2m1_encode(oracle.e2m1_decode(c)) == (c if c != 8 else 8)
+    # midpoints go to the code with fraction bit 0
+    for mid, want in [(0.25, 0x0), (0.75, 0x2), (1.25, 0x2), (1.75, 0x4), (2.5, 0x4), (3.5, 0x6),
+                      (5.0, 0x6)]:
+        assert oracle.e2m1_encode(mid) == want, mid
+        assert oracle.e2m1_encode(-mid) == want | 8, -mid
+    for big in (6.0, 6.5, 7.9, 100.0):
+        assert oracle.e2m1_encode(big) == 0x7 and oracle.e2m1_encode(-big) == 0xF
+    assert oracle.e2m1_encode(0.26) == 0x1 and oracle.e2m1_encode(0.24) == 0x0
+
+
+def _mx_representable_rows(rng, N, K):
+    """Rows whose every 32-block is E2M1 codes times 2^k with the block's largest
+    magnitude 4 or 6 times 2^k: exactly representable in MXFP4 (and in bf16)."""
+    W = np.zeros((N, K), np.float32)
+    mags = np.array([0, 0.5, 1, 1.5, 2, 3, 4, 6], np.float32)
+    for n in range(N):
+        for b in range(K // 32):
+            k = int(rng.integers(-6, 4))
+            v = rng.choice(mags, 32) * rng.choice([-1.0, 1.0], 32)
+            v[rng.integers(0, 32)] = rng.choice([4.0, 6.0]) * rng.choice([-1.0, 1.0])
+            W[n, b * 32:(b + 1) * 32] = v * 2.0 ** k
+    return wl.to_bf16_bits(W), W
+
+
+def test_mxfp4_quantize_exact_on_representable_blocks():
+    rng = np.random.default_rng(31)
+    Wb, W = _mx_representable_rows(rng, 6, 96)
+    codes, scales = oracle.mxfp4_quantize(Wb)
+    deq = np.vectorize(oracle.e2m1_decode)(codes) * np.repeat(
+        np.vectorize(oracle.e8m0_decode)(scales), 32, axis=1)
+    assert np.array_equal(deq, W.astype(np.float64))
+
+
+def test_mxfp4_quantize_scale_rule_and_zero_block():
+    # amax 1.0 -> X = 2^(0 - 2): 1.0 / 0.25 = 4, code 6
+    W = np.zeros((2, 64), np.float32)
+    W[0, :32] = 1.0
+    W[0, 32:] = np.linspace(-7.9, 7.9, 32)   # amax 7.9: X = 2^(2 - 2) = 1, 7.9 saturates to 6
+    codes, scales = oracle.mxfp4_quantize(wl.to_bf16_bits(W))
+    assert scales[0, 0] == 127 - 2 and (codes[0, :32] == 0x6).all()
+    assert scales[0, 1] == 127 and codes[0, 32] == 0xF and codes[0, 63] == 0x7
+    assert scales[1, 0] == 0 and (codes[1] == 0).all()      # all-zero blocks
+
+
+def test_mxfp4_gemm_equals_bf16_linear_on_representable_weights():
+    """With MXFP4-representable weights the 4-bit GEMM equals the (separately pinned)
+    bf16 linear oracle on the same values."""
+    rng = np.random.default_rng(32)
+    N, K, M = 10, 128, 5
+    Wb, _ = _mx_representable_rows(rng, N, K)
+    x = wl.normal_bf16(rng, (M, K))
+    codes, scales = oracle.mxfp4_quantize(Wb)
+    rows = np.repeat(np.arange(M), N).astype(np.int32)
+    cols = np.tile(np.arange(N), M).astype(np.int32)
+    got = oracle.mxfp4_gemm_lora_sampled(x, codes, scales, rows, cols)
+    want = oracle.linear_bf16_sampled(x, Wb, rows, cols)
+    assert np.allclose(got, want, rtol=1e-13, atol=1e-13)
+
+
+def test_mxfp4_gemm_lora_brute_force_rationals():
+    rng = np.random.default_rng(33)
+    M, K, N, n_ad, r = 3, 64, 4, 2, 2
+    x = wl.to_bf16_bits(rng.integers(-2, 3, (M, K)).astype(np.float32))
+    codes = rng.integers(0, 16, (N, K)).astype(np.uint8)
+    scales = rng.integers(124, 130, (N, K // 32)).astype(np.uint8)
+    A = wl.to_bf16_bits(rng.integers(-2, 3, (n_ad, K, r)).astype(np.float32))
+    B = wl.to_bf16_bits(rng.integers(-2, 3, (n_ad, r, N)).astype(np.float32))
+    ranks = np.array([2, 1], np.int32)
+    sl = np.array([2.0, 0.5], np.float32)
+    ids = np.array([0, -1, 1], np.int32)
+    rows = np.repeat(np.arange(M), N).astype(np.int32)
+    cols = np.tile(np.arange(N), M).astype(np.int32)
+    got = oracle.mxfp4_gemm_lora_sampled(x, codes, scales, rows, cols, A=A, B=B, ranks=ranks,
+                                         scales_lora=sl, ids=ids)
+    X = _frac_bf16(x)
+    E2 = [Fraction(oracle.e2m1_decode(c)) for c in range(16)]
+    for i, (m, n) in enumerate(zip(rows, cols)):
+        y = sum(X[m][k] * E2[codes[n, k]] * Fraction(2) ** (int(scales[n, k // 32]) - 127) for k in range(K))
+        a = int(ids[m])
+        if a >= 0:
+            Af, Bf = _frac_bf16(A[a]), _frac_bf16(B[a])
+            v = [sum(X[m][k] * Af[k][j] for k in range(K)) for j in range(ranks[a])]
+            y += Fraction(float(sl[a])) * sum(v[j] * Bf[j][n] for j in range(ranks[a]))
+        assert Fraction(got[i]) == y
