@@ -4,17 +4,14 @@
 // prefill), as a persistent grid that streams work items.
 //
 // Work items. Every tile row (one run of <= 64 tokens of one adapter, in one
-// slice) is split into Pk shrink parts (a span of h_in) and Pn expand parts (a
-// span of h_out). One global counter hands the items out in a fixed order:
-// every shrink part first, then every expand part. A shrink part computes its
-// span's partial v = x.A_a for the tile's tokens and adds it into a v buffer
-// in the workspace (plain stores when Pk == 1), then counts itself done for
-// its tile. An expand part first waits (bounded) until all Pk shrink parts of
-// its tile are done, then reads v and adds s_a v.B_a to its span of y.
-// A CTA that was handed an expand part has finished every shrink part it was
-// handed, and every shrink part was handed to a running CTA before any expand
-// part was, so the waits cannot form a cycle, whether or not every CTA of the
-// grid is resident.
+// slice) is split into Pk shrink parts (spans of h_in) and Pn expand parts
+// (spans of h_out). The call makes two launches of the kernel, each handing
+// its items out from a global counter: the first runs every shrink part, which
+// computes its span's partial v = x.A_a for the tile's tokens and adds it into
+// a v buffer in the workspace (plain stores when Pk == 1); the second, a
+// programmatic dependent of the first, runs every expand part: its copies of
+// B_a and y start while the first launch finishes, and its compute warps wait
+// for the first launch to complete before they read v.
 //
 // Pipeline. A producer warp claims items, cuts them into chunks of columns
 // sized to one ring stage (wider chunks for small ranks and few tokens) and
@@ -57,7 +54,8 @@ struct StreamParams {
     int32_t* counts;
     uint16_t* y;
     float* vbuf;  // fp32 [n_slices][T][r_max]
-    int* ctr;     // [0]: next item; [1 + s * n_rows + g]: shrink parts done of tile row g, slice s
+    int* ctr;     // [phase]: the next item of this launch
+    int phase;    // 0: the shrink parts; 1: the expand parts (a programmatic dependent of 0)
     int T, n_adapters, h_in, h_out, r_max, n_slices, n_rows;
     int Pk, Pn, kp, np;  // parts per tile row and their spans (multiples of 64)
     int stage_bytes;
@@ -90,32 +88,12 @@ __device__ __forceinline__ int chunk_width(int per_col, int sb)
     return w;
 }
 
-// Bounded wait for a global counter (acquire, GPU scope).
-__device__ bool wait_counter(const int* ctr, int target, volatile int* abort_flag, int32_t* status,
-                             unsigned long long limit)
-{
-    const unsigned long long t0 = ptx::globaltimer();
-    while (true) {
-        int v;
-        asm volatile("ld.acquire.gpu.global.b32 %0, [%1];\n" : "=r"(v) : "l"(ctr) : "memory");
-        if (v >= target) return true;
-        if (*abort_flag) return false;
-        if (ptx::globaltimer() - t0 > limit) {
-            *abort_flag = 1;
-            atomicOr(status, 0x4000);
-            return false;
-        }
-        __nanosleep(100);
-    }
-}
-
 __global__ void __launch_bounds__(kThreads, 2)
 sgmv_stream_kernel(const __grid_constant__ AMaps am, const StreamParams p)
 {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     __shared__ StageHdr s_hdr[kStages];
     __shared__ int s_abort;
-    __shared__ int s_ok;
 
     const uint32_t raw_u = ptx::smem_u32(smem_raw);
     const uint32_t base_u = (raw_u + 1023u) & ~1023u;  // swizzled boxes need 1024-byte alignment
@@ -139,9 +117,13 @@ sgmv_stream_kernel(const __grid_constant__ AMaps am, const StreamParams p)
     }
     __syncwarp();
     __syncthreads();
-    // the segment builder (the previous kernel in the stream) may still run
-    ptx::pdl_wait();
+    // Shrink launch: the segment builder (the previous kernel in the stream) may still
+    // run; the expand launch may start as soon as this one has passed this point. Expand
+    // launch: its copies (B_a and y, which the shrink does not write) start at once; the
+    // compute warps wait for the shrink launch to complete before they read v.
+    if (p.phase == 0) ptx::pdl_wait();
     ptx::pdl_launch_dependents();
+    bool v_ready = p.phase == 0;
 
     if (warp == kComputeWarps) {
         // ================================================================ producer warp
@@ -162,8 +144,8 @@ sgmv_stream_kernel(const __grid_constant__ AMaps am, const StreamParams p)
         // consumed one item after it was issued, while the current item's copies go out:
         // claims run two items ahead, tile rows one item ahead.
         const long long used = p.counts[3];
-        const long long n_shrink = used * p.n_slices * p.Pk;
-        const long long n_items = n_shrink + used * p.n_slices * p.Pn;
+        const long long n_shrink = p.phase == 0 ? used * p.n_slices * p.Pk : 0;
+        const long long n_items = p.phase == 0 ? n_shrink : used * p.n_slices * p.Pn;
         struct Meta {
             long long item;
             int shrink, slice, g, part;
@@ -194,11 +176,11 @@ sgmv_stream_kernel(const __grid_constant__ AMaps am, const StreamParams p)
         };
         long long claim = 0;
         Meta m0, m1;
-        if (lane == 0) claim = (long long)atomicAdd(p.ctr, 1);
+        if (lane == 0) claim = (long long)atomicAdd(p.ctr + p.phase, 1);
         decode(__shfl_sync(0xffffffffu, claim, 0), m0);
-        if (lane == 0) claim = (long long)atomicAdd(p.ctr, 1);
+        if (lane == 0) claim = (long long)atomicAdd(p.ctr + p.phase, 1);
         decode(__shfl_sync(0xffffffffu, claim, 0), m1);
-        if (lane == 0 && m1.item < n_items) claim = (long long)atomicAdd(p.ctr, 1);
+        if (lane == 0 && m1.item < n_items) claim = (long long)atomicAdd(p.ctr + p.phase, 1);
         resolve(m0);
         while (ok && m0.item < n_items) {
             resolve(m1);
@@ -206,7 +188,7 @@ sgmv_stream_kernel(const __grid_constant__ AMaps am, const StreamParams p)
             m2.item = n_items;
             if (m1.item < n_items) {
                 decode(__shfl_sync(0xffffffffu, claim, 0), m2);
-                if (lane == 0 && m2.item < n_items) claim = (long long)atomicAdd(p.ctr, 1);
+                if (lane == 0 && m2.item < n_items) claim = (long long)atomicAdd(p.ctr + p.phase, 1);
             }
             const bool shrink = m0.shrink;
             const int slice = m0.slice, g = m0.g, part = m0.part;
@@ -361,7 +343,7 @@ sgmv_stream_kernel(const __grid_constant__ AMaps am, const StreamParams p)
             const StageHdr& h = s_hdr[st];
             const int kind = h.kind;
             if (kind == kEnd) break;
-            const int slice = h.slice, g = h.g, nt = h.nt, r = h.r, wb = h.wb, c0 = h.c0, cw = h.cw;
+            const int slice = h.slice, nt = h.nt, r = h.r, wb = h.wb, c0 = h.c0, cw = h.cw;
             const bool first = h.first, last = h.last;
             const bool small = nt <= kSmallTile;
             const int Mt = (nt + 15) >> 4;
@@ -504,19 +486,17 @@ sgmv_stream_kernel(const __grid_constant__ AMaps am, const StreamParams p)
                             }
                         }
                     }
-                    __threadfence();
                     ptx::named_sync(1, kCompute);
-                    if (tid == 0) atomicAdd(p.ctr + 1 + slice * p.n_rows + g, 1);
                 }
             } else {
                 // ---------------------------------------------------------- expand chunk
                 const float scale = h.scale;
                 if (first) {
-                    // every shrink part of this tile is done: then v of its tokens
-                    if (tid == 0)
-                        s_ok = wait_counter(p.ctr + 1 + slice * p.n_rows + g, p.Pk, abort_flag, status, p.timeout_ns);
-                    ptx::named_sync(1, kCompute);
-                    live = s_ok;
+                    // the shrink launch has completed: v of every token is in the buffer
+                    if (!v_ready) {
+                        ptx::pdl_wait();
+                        v_ready = true;
+                    }
                     if (live) {
                         if (small) {
                             for (int idx = tid; idx < nt * r16; idx += kCompute) {
@@ -557,8 +537,6 @@ sgmv_stream_kernel(const __grid_constant__ AMaps am, const StreamParams p)
                         }
                     }
                     ptx::named_sync(1, kCompute);
-                } else {
-                    live = s_ok;
                 }
                 const uint32_t yb = base + (uint32_t)((wb >> 6) * r16 * 128);
                 uint16_t* yg = p.y + (size_t)slice * p.T * p.h_out;
@@ -685,10 +663,8 @@ sgmv_stream_kernel(const __grid_constant__ AMaps am, const StreamParams p)
 
 size_t sgmv_stream_workspace_bytes(int T, const lora_pool_t& pool)
 {
-    const size_t n_rows = (size_t)max_tiles_for(T, pool.n_adapters);
-    const size_t ctr = ((1 + (size_t)pool.n_slices * n_rows) * 4 + 255) / 256 * 256;
     const size_t v = (size_t)pool.n_slices * T * pool.r_max * 4;
-    return ctr + (v + 255) / 256 * 256;
+    return 256 + (v + 255) / 256 * 256;  // the two item counters | v
 }
 
 cudaError_t launch_sgmv_stream(const void* x, int64_t x_slice_stride, const lora_pool_t& pool,
@@ -732,11 +708,11 @@ cudaError_t launch_sgmv_stream(const void* x, int64_t x_slice_stride, const lora
     p.Pn = (pool.h_out + p.np - 1) / p.np;
 
     uint8_t* w = static_cast<uint8_t*>(ws);
-    const size_t ctr_bytes = ((1 + (size_t)rows) * 4 + 255) / 256 * 256;
+    const size_t ctr_bytes = 256;
     p.ctr = reinterpret_cast<int*>(w);
     p.vbuf = reinterpret_cast<float*>(w + ctr_bytes);
     const size_t v_bytes = (size_t)pool.n_slices * seg.T * pool.r_max * 4;
-    // the counters start at zero; so does v when several parts add into it
+    // the item counters start at zero; so does v when several parts add into it
     cudaError_t e = cudaMemsetAsync(w, 0, p.Pk > 1 ? ctr_bytes + v_bytes : ctr_bytes, stream);
     if (e != cudaSuccess) return e;
 
@@ -769,19 +745,27 @@ cudaError_t launch_sgmv_stream(const void* x, int64_t x_slice_stride, const lora
 
     e = cudaFuncSetAttribute(sgmv_stream_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    long long grid = G;
-    if (grid > rows * (p.Pk + p.Pn)) grid = rows * (p.Pk + p.Pn);
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)grid, 1, 1);
-    cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, sgmv_stream_kernel, am, p);
+    // two launches of the persistent kernel: the shrink parts, then the expand parts as
+    // its programmatic dependent
+    for (int phase = 0; phase < 2; ++phase) {
+        p.phase = phase;
+        long long grid = G;
+        const long long items = rows * (phase == 0 ? p.Pk : p.Pn);
+        if (grid > items) grid = items;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)grid, 1, 1);
+        cfg.blockDim = dim3(kThreads, 1, 1);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        e = cudaLaunchKernelEx(&cfg, sgmv_stream_kernel, am, p);
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
 }
 
 }  // namespace lora
