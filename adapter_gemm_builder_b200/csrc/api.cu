@@ -76,7 +76,7 @@ size_t fp8_ws_layout(int M, int K, const lora_pool_t* pool, size_t* off_xq, size
     *off_part = off;
     off += align256(fp8_gemm_partial_bytes(M));
     if (off_apply) *off_apply = off;
-    if (gemm_split(M, pool)) off += align256(sgmv_stream_workspace_bytes(M, *pool));
+    if (gemm_split(M, pool)) off += align256(sgmv_warp_workspace_bytes(M, *pool));
     return off;
 }
 
@@ -133,7 +133,7 @@ namespace {
 // (x quantised per token); esz 2: bf16 operands (x copied in segment order).
 int gemm_lora_launch(int esz, const void* x, int M, int K, int N, const uint8_t* Wq, const float* w_scale,
                      const lora_pool_t* pool, const lora_segments_t* seg, void* y, void* ws,
-                     size_t ws_bytes, lora_stream_t stream)
+                     size_t ws_bytes, lora_stream_t stream, const uint8_t* wsc = nullptr, bool w_e4m3 = false)
 {
     size_t off_xq, off_sx, off_v, off_sync, off_part, off_apply;
     const size_t need =
@@ -166,6 +166,8 @@ int gemm_lora_launch(int esz, const void* x, int M, int K, int N, const uint8_t*
     a.sx = sx;
     a.Wq = Wq;
     a.sw = w_scale;
+    a.wsc = wsc;
+    a.w_e4m3 = w_e4m3;
     a.y = static_cast<uint16_t*>(y);
     a.status = status;
     a.partials = reinterpret_cast<float*>(w + off_part);
@@ -193,7 +195,11 @@ int gemm_lora_launch(int esz, const void* x, int M, int K, int N, const uint8_t*
     //    (the kernel lora_apply picks for this batch)
     if (tile_tokens_for(M, pool->n_adapters) <= LORA_DECODE_TILE_TOKENS)
         return cuda_status(launch_sgmv(SGMV_APPLY, x, 0, *pool, *seg, nullptr, y, s, false));
-    return cuda_status(launch_sgmv_stream(x, 0, *pool, *seg, y, w + off_apply, s));
+    void* wa = w + off_apply;
+    if (sgmv_warp_zero(*pool, *seg, wa, s) != cudaSuccess ||
+        launch_sgmv(SGMV_APPLY, x, 0, *pool, *seg, nullptr, y, s, false, kWarpSmallTile) != cudaSuccess)
+        return LORA_ERR_CUDA;
+    return cuda_status(launch_sgmv_warp(x, 0, *pool, *seg, y, wa, s));
 }
 
 }  // namespace
@@ -271,19 +277,21 @@ size_t lora_workspace_size(int op, int T, int K, const lora_pool_t* pool)
         // decode-like batches need none; the others, the streaming kernel's counters and v
         if (!pool || check_pool(pool) != LORA_OK) return (size_t)-1;
         if (T == 0 || tile_tokens_for(T, pool->n_adapters) <= LORA_DECODE_TILE_TOKENS) return 0;
-        return sgmv_stream_workspace_bytes(T, *pool);
+        return sgmv_warp_workspace_bytes(T, *pool);
     case LORA_OP_FP8_BACKWARD: {
         if (!pool || check_pool(pool) != LORA_OK || T < 1) return (size_t)-1;
         size_t a, b, c, d;
         return bwd_ws_layout(T, pool, &a, &b, &c, &d);
     }
     case LORA_OP_FP8_GEMM:
-    case LORA_OP_BF16_GEMM: {
+    case LORA_OP_BF16_GEMM:
+    case LORA_OP_MXFP4_GEMM:
+    case LORA_OP_W8A16_GEMM: {
         if (K <= 0) return (size_t)-1;
         if (pool && check_pool(pool) != LORA_OK) return (size_t)-1;
         if (T < 1) return (size_t)-1;
         size_t a, b, c, d, e;
-        return fp8_ws_layout(T, K, pool, &a, &b, &c, &d, &e, op == LORA_OP_BF16_GEMM ? 2 : 1);
+        return fp8_ws_layout(T, K, pool, &a, &b, &c, &d, &e, op == LORA_OP_FP8_GEMM ? 1 : 2);
     }
     default: return (size_t)-1;
     }
@@ -383,13 +391,19 @@ int lora_apply(const void* x, int64_t x_slice_stride, const lora_pool_t* pool,
     if (seg->T == 0) return LORA_OK;
     if ((st = check_x(x, x_slice_stride, pool, seg->T)) != LORA_OK) return st;
     if (!y || !aligned16(y)) return LORA_ERR_INVALID_ARG;
+    cudaStream_t s = (cudaStream_t)stream;
     if (tile_tokens_for(seg->T, pool->n_adapters) <= LORA_DECODE_TILE_TOKENS)
         // a decode-like batch: one tile per thread-block cluster, v exchanged on chip
-        return cuda_status(launch_sgmv(SGMV_APPLY, x, x_slice_stride, *pool, *seg, nullptr, y,
-                                       (cudaStream_t)stream, false));
-    const size_t need = sgmv_stream_workspace_bytes(seg->T, *pool);
+        return cuda_status(launch_sgmv(SGMV_APPLY, x, x_slice_stride, *pool, *seg, nullptr, y, s, false));
+    const size_t need = sgmv_warp_workspace_bytes(seg->T, *pool);
     if (!ws || ws_bytes < need || !aligned16(ws)) return LORA_ERR_WORKSPACE;
-    return cuda_status(launch_sgmv_stream(x, x_slice_stride, *pool, *seg, y, ws, (cudaStream_t)stream));
+    // the warp kernel's counters are zeroed first; then the tile rows of more than
+    // kWarpSmallTile tokens on the cluster kernel, and alongside it the small ones
+    // on the warp kernel (two launches)
+    if (sgmv_warp_zero(*pool, *seg, ws, s) != cudaSuccess ||
+        launch_sgmv(SGMV_APPLY, x, x_slice_stride, *pool, *seg, nullptr, y, s, false, kWarpSmallTile) != cudaSuccess)
+        return LORA_ERR_CUDA;
+    return cuda_status(launch_sgmv_warp(x, x_slice_stride, *pool, *seg, y, ws, s));
 }
 
 int fp8_quantize_rows(const void* x, int M, int K, uint8_t* xq, float* sx, lora_stream_t stream)
@@ -472,6 +486,49 @@ int lora_switch_merge(const void* W, int N, int K, const lora_pool_t* pool, cons
     const uintptr_t a0 = (uintptr_t)W, b0 = (uintptr_t)W_out, len = (uintptr_t)N * K * 2;
     if (a0 != b0 && a0 < b0 + len && b0 < a0 + len) return LORA_ERR_INVALID_ARG;
     return cuda_status(launch_lora_switch_merge(W, N, K, *pool, sel, gates, n_sel, W_out, (cudaStream_t)stream));
+}
+
+int w8a16_gemm_lora_epilogue(const void* x, int M, int K, int N, const uint8_t* Wq, const float* w_scale,
+                             const lora_pool_t* pool, const lora_segments_t* seg, void* y, void* ws,
+                             size_t ws_bytes, lora_stream_t stream)
+{
+    if (M < 1 || K < 64 || N < 8 || K % 64 || N % 8) return LORA_ERR_INVALID_ARG;
+    if (!x || !Wq || !w_scale || !y) return LORA_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(Wq) || !aligned16(y)) return LORA_ERR_INVALID_ARG;
+    if (M > (1 << 24)) return LORA_ERR_UNSUPPORTED;
+    if (pool) {
+        int st = check_pool(pool);
+        if (st != LORA_OK) return st;
+        if (pool->n_slices != 1 || pool->h_in != K || pool->h_out != N) return LORA_ERR_INVALID_ARG;
+        if ((st = check_segments(seg, pool->n_adapters)) != LORA_OK) return st;
+        if (seg->T != M) return LORA_ERR_INVALID_ARG;
+    }
+    return gemm_lora_launch(2, x, M, K, N, Wq, w_scale, pool, seg, y, ws, ws_bytes, stream, nullptr, true);
+}
+
+int mxfp4_quantize_rows(const void* W, int N, int K, uint8_t* Wp, uint8_t* Wsc, lora_stream_t stream)
+{
+    if (N < 1 || K < 64 || K % 64) return LORA_ERR_INVALID_ARG;
+    if (!W || !Wp || !Wsc || !aligned16(W) || !aligned16(Wp) || !aligned16(Wsc)) return LORA_ERR_INVALID_ARG;
+    return cuda_status(launch_mxfp4_quantize(W, N, K, Wp, Wsc, (cudaStream_t)stream));
+}
+
+int mxfp4_gemm_lora_epilogue(const void* x, int M, int K, int N, const uint8_t* Wp, const uint8_t* Wsc,
+                             const lora_pool_t* pool, const lora_segments_t* seg, void* y, void* ws,
+                             size_t ws_bytes, lora_stream_t stream)
+{
+    if (M < 1 || K < 64 || N < 8 || K % 64 || N % 8) return LORA_ERR_INVALID_ARG;
+    if (!x || !Wp || !Wsc || !y) return LORA_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(Wp) || !aligned16(Wsc) || !aligned16(y)) return LORA_ERR_INVALID_ARG;
+    if (M > (1 << 24)) return LORA_ERR_UNSUPPORTED;
+    if (pool) {
+        int st = check_pool(pool);
+        if (st != LORA_OK) return st;
+        if (pool->n_slices != 1 || pool->h_in != K || pool->h_out != N) return LORA_ERR_INVALID_ARG;
+        if ((st = check_segments(seg, pool->n_adapters)) != LORA_OK) return st;
+        if (seg->T != M) return LORA_ERR_INVALID_ARG;
+    }
+    return gemm_lora_launch(2, x, M, K, N, Wp, nullptr, pool, seg, y, ws, ws_bytes, stream, Wsc);
 }
 
 int bf16_gemm_lora_epilogue(const void* x, int M, int K, int N, const void* W,

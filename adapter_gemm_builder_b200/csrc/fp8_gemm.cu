@@ -56,6 +56,14 @@ constexpr int kBlockM = 128;  // W rows per tile (MMA M)
 constexpr int kEpiWarps = 8;
 constexpr int kEpiThreads = kEpiWarps * 32;
 constexpr int kThreads = (3 + kEpiWarps) * 32;
+constexpr int kCvtWarps = 4;                      // MX FP4 weights: converter warps (one row each lane)
+constexpr int kThreadsW4 = (3 + kEpiWarps + kCvtWarps) * 32;
+constexpr int kPackStage = 5120;                  // packed E2M1 tile (128 x 32 B) + scales (2 x 128 B), 1 KB aligned
+constexpr int kCodeStage = 8192;                  // E4M3 tile of the 8-bit weights under bf16 activations (128 x 64 B)
+// Weight converter modes of the 16-bit MMA path: none (the weights are bf16), MX FP4
+// codes with E8M0 block scales, E4M3 codes with a per-channel scale (W8A16).
+enum { kWcNone = 0, kWcMxfp4 = 1, kWcE4m3 = 2 };
+__host__ __device__ constexpr int wc_stage_bytes(int wc) { return wc == 1 ? kPackStage : (wc == 2 ? kCodeStage : 0); }
 constexpr int kMaxStages = 8;
 constexpr int kShrinkCols = 64;  // K columns of the down-projection per work item
 constexpr int kShrinkTok = 64;   // tokens of the down-projection per work item
@@ -66,6 +74,7 @@ struct GemmParams {
     long long units;  // num_tiles * k_blocks, split evenly over the grid
     const float* sx;
     const float* sw;
+    const uint8_t* wsc;  // MX FP4 block scales (kW4)
     uint16_t* y;
     uint32_t* status;
     float* partials;  // fp32 stream-K partial accumulators, [gridDim.x][BN/16][4][128][4]
@@ -200,6 +209,48 @@ __device__ __forceinline__ uint32_t kmajor_off(int row, int kg, int kg_n)
     return (uint32_t)((((row >> 3) * kg_n + kg) << 7) + ((row & 7) << 4));
 }
 
+// bf16 bit patterns of the 8 E2M1 magnitudes times the block scale 2^(E - 127)
+// (exact: at most two significant bits), split into low and high byte tables
+// of 8 entries for byte permutes.
+__device__ __forceinline__ void e2m1_tables(uint32_t E, uint32_t& lo0, uint32_t& lo1, uint32_t& hi0, uint32_t& hi1)
+{
+    const float S = E == 0 ? __uint_as_float(0x00400000u) : (E == 255 ? __uint_as_float(0x7fc00000u) : __uint_as_float(E << 23));
+    const float mag[8] = {0.f, 0.5f, 1.f, 1.5f, 2.f, 3.f, 4.f, 6.f};
+    uint32_t b[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) b[i] = __float_as_uint(mag[i] * S) >> 16;
+    lo0 = (b[0] & 0xffu) | ((b[1] & 0xffu) << 8) | ((b[2] & 0xffu) << 16) | ((b[3] & 0xffu) << 24);
+    lo1 = (b[4] & 0xffu) | ((b[5] & 0xffu) << 8) | ((b[6] & 0xffu) << 16) | ((b[7] & 0xffu) << 24);
+    hi0 = (b[0] >> 8) | ((b[1] >> 8) << 8) | ((b[2] >> 8) << 16) | ((b[3] >> 8) << 24);
+    hi1 = (b[4] >> 8) | ((b[5] >> 8) << 8) | ((b[6] >> 8) << 16) | ((b[7] >> 8) << 24);
+}
+
+// Eight E2M1 codes (one 32-bit word, element i in nibble i) -> eight bf16 values:
+// byte permutes pick each code's magnitude bytes from the tables, the code's
+// sign bit becomes the bf16 sign, and the low / high bytes are interleaved.
+__device__ __forceinline__ uint4 e2m1x8_to_bf16(uint32_t w, uint32_t lo0, uint32_t lo1, uint32_t hi0, uint32_t hi1)
+{
+    const uint32_t s0 = w & 0x7777u, s1 = (w >> 16) & 0x7777u;
+    const uint32_t w4 = w << 4;
+    const uint32_t L0 = __byte_perm(lo0, lo1, s0), L1 = __byte_perm(lo0, lo1, s1);
+    const uint32_t H0 = __byte_perm(hi0, hi1, s0) | (__byte_perm(w, w4, 0x1504) & 0x80808080u);
+    const uint32_t H1 = __byte_perm(hi0, hi1, s1) | (__byte_perm(w, w4, 0x3726) & 0x80808080u);
+    return make_uint4(__byte_perm(L0, H0, 0x5140), __byte_perm(L0, H0, 0x7362), __byte_perm(L1, H1, 0x5140),
+                      __byte_perm(L1, H1, 0x7362));
+}
+
+// Two E4M3 codes (byte 0 the first) -> two bf16 (the first in the low half):
+// E4M3 -> f16 -> f32 -> bf16, every step exact.
+__device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint16_t c2)
+{
+    uint32_t h2, r;
+    float lo, hi;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(c2));
+    asm("{\n.reg .f16 l, h;\nmov.b32 {l, h}, %2;\ncvt.f32.f16 %0, l;\ncvt.f32.f16 %1, h;\n}" : "=f"(lo), "=f"(hi) : "r"(h2));
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
 // Stream-K schedule: CTA c owns units [c*U/G, (c+1)*U/G) of the (tile,
 // k-block) sequence; a segment is the part of one tile inside that range.
 struct Seg {
@@ -221,8 +272,13 @@ __device__ __forceinline__ Seg seg_at(long long u, long long u_end, int KB)
 // ESZ: bytes per operand element -- 1 for E4M3 (kind::f8f6f4), 2 for bf16
 // (kind::f16). BK is the k-block in bytes either way (128: 128-byte swizzle,
 // 64: 64-byte swizzle), so the shared-memory layouts are the same.
-template <int BK, int MAXR, int ESZ>
-__global__ void __launch_bounds__(kThreads, 1)
+// kW4 (a weight converter mode, with ESZ 2 and BK 128): the weights arrive as
+// codes -- OCP MX FP4 (packed E2M1 codes and E8M0 block scales) or E4M3 (whose
+// per-channel scale the epilogue applies, as on the 8-bit path) -- and four
+// converter warps turn each k-block's codes into the bf16 tile the MMA reads
+// (one row per thread), signalling it on conv[stage].
+template <int BK, int MAXR, int ESZ, int kW4 = kWcNone>
+__global__ void __launch_bounds__(kW4 != kWcNone ? kThreadsW4 : kThreads, 1)
 fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                 const __grid_constant__ CUtensorMap tmB, const GemmParams p)
 {
@@ -250,10 +306,11 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
     uint64_t* epibar = drain + 1;               // [1] epilogue-warps barrier
     uint64_t* lready = epibar + 1;              // [1] LoRA operands of the segment built
     uint64_t* stall = lready + 1;               // [1] test hook: never completed
+    uint64_t* conv = stall + 1;                 // [stages] MX FP4: the k-block's bf16 W tile built
     volatile int* abort_flag = &s_abort;
 
     constexpr int kStageW = kBlockM * BK;
-    const int stage_bytes = kStageW + p.BN * BK;
+    const int stage_bytes = kStageW + p.BN * BK + wc_stage_bytes(kW4);
     const uint32_t ncols = (uint32_t)(2 * p.BN <= 32 ? 32 : (2 * p.BN <= 64 ? 64 : (2 * p.BN <= 128 ? 128 : (2 * p.BN <= 256 ? 256 : 512))));
     const int G = gridDim.x, cta = blockIdx.x, KB = p.k_blocks;
     const long long u_begin = unit_begin(p.units, cta, G), u_end = unit_begin(p.units, cta + 1, G);
@@ -264,6 +321,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
         for (int s = 0; s < p.stages; ++s) {
             ptx::mbar_init(&full[s], 1);
             ptx::mbar_init(&empty[s], 1);
+            if (kW4 != kWcNone) ptx::mbar_init(&conv[s], kCvtWarps);
         }
         for (int b = 0; b < 2; ++b) {
             ptx::mbar_init(&tfull[b], 1);
@@ -330,8 +388,22 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
                     }
                     const uint32_t sW = smem_u + p.ring_off + stage * stage_bytes;
                     const uint32_t sX = sW + kStageW;
-                    ptx::mbar_arrive_expect_tx(&full[stage], (uint32_t)stage_bytes);
-                    ptx::tma_load_2d_hint(sW, &tmW, &full[stage], kb * (BK / ESZ), nb * kBlockM, w_policy);
+                    if constexpr (kW4 == kWcMxfp4) {
+                        // packed codes (128 rows x 32 bytes) and the k-block's two scale blocks
+                        const uint32_t sP = sX + (uint32_t)(p.BN * BK);
+                        ptx::mbar_arrive_expect_tx(&full[stage], (uint32_t)(4096 + 256 + p.BN * BK));
+                        ptx::tma_load_2d_hint(sP, &tmW, &full[stage], kb * 32, nb * kBlockM, w_policy);
+                        ptx::bulk_g2s(sP + 4096, p.wsc + ((size_t)nb * (p.K / 32) + kb * 2) * kBlockM, 256,
+                                      &full[stage]);
+                    } else if constexpr (kW4 == kWcE4m3) {
+                        // E4M3 codes: 128 rows x 64 bytes
+                        const uint32_t sP = sX + (uint32_t)(p.BN * BK);
+                        ptx::mbar_arrive_expect_tx(&full[stage], (uint32_t)(kCodeStage + p.BN * BK));
+                        ptx::tma_load_2d_hint(sP, &tmW, &full[stage], kb * 64, nb * kBlockM, w_policy);
+                    } else {
+                        ptx::mbar_arrive_expect_tx(&full[stage], (uint32_t)stage_bytes);
+                        ptx::tma_load_2d_hint(sW, &tmW, &full[stage], kb * (BK / ESZ), nb * kBlockM, w_policy);
+                    }
                     if (waited) {
                         ptx::tma_load_2d(sX, &tmX, &full[stage], kb * (BK / ESZ), tb * p.BN);
                     } else {  // first ring pass: stage == n_def
@@ -440,7 +512,8 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
                 const uint32_t d = tmem_base + (uint32_t)(buf * p.BN);
                 for (int kb = sg.kb0; kb < sg.kb1; ++kb) {
                     if (!lora_step(false) ||
-                        !wait_bounded(&full[stage], phase, abort_flag, p.status, 0x4u, p.timeout_ns)) {
+                        !wait_bounded(kW4 != kWcNone ? &conv[stage] : &full[stage], phase, abort_flag, p.status, 0x4u,
+                                      p.timeout_ns)) {
                         ok = false;
                         break;
                     }
@@ -549,7 +622,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
             }
             if (*abort_flag && pending) drain_wait(bfull, pending_phase);
         }
-    } else {
+    } else if (kW4 == kWcNone || warp < 3 + kEpiWarps) {
         // ------------------------------------------------------------ epilogue warps
         const int ew = warp - 3;
         const int quarter = warp & 3;         // TMEM lane quarter this warp may access
@@ -1012,6 +1085,74 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
         }
     }
 
+    if constexpr (kW4 != kWcNone) {
+        if (warp >= 3 + kEpiWarps) {
+            // ------------------------------------------------------------ converter warps
+            // thread = one W row of the tile: its 64 codes of the k-block (32 packed bytes)
+            // and its two block scales become 64 bf16 values in the 128-byte swizzled row
+            // the MMA descriptor expects
+            const int row = (warp - 3 - kEpiWarps) * 32 + lane;
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            for (long long u = u_begin; u < u_end && ok;) {
+                const Seg sg = seg_at(u, u_end, KB);
+                u += sg.kb1 - sg.kb0;
+                for (int kb = sg.kb0; kb < sg.kb1; ++kb) {
+                    bool got = true;
+                    if (lane == 0) got = wait_bounded(&full[stage], phase, abort_flag, p.status, 0x800u, p.timeout_ns);
+                    got = __shfl_sync(0xffffffffu, got, 0);
+                    if (!got) {
+                        ok = false;
+                        break;
+                    }
+                    if (lane != 0) drain_wait(&full[stage], phase);  // complete already: acquire
+                    uint8_t* st_base = smem + p.ring_off + (size_t)stage * stage_bytes;
+                    const uint8_t* pk = st_base + kStageW + p.BN * BK;
+                    uint8_t* dst = st_base + row * 128;
+                    const int sw = row & 7;
+                    if constexpr (kW4 == kWcE4m3) {
+                        // 64 E4M3 codes -> bf16 (exact: E4M3 -> f16 -> f32 -> bf16)
+#pragma unroll
+                        for (int h = 0; h < 4; ++h) {
+                            const uint4 q = *reinterpret_cast<const uint4*>(pk + row * 64 + h * 16);
+                            const uint32_t w4[4] = {q.x, q.y, q.z, q.w};
+                            uint32_t o[8];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                o[2 * e] = e4m3x2_to_bf16x2((uint16_t)(w4[e] & 0xffffu));
+                                o[2 * e + 1] = e4m3x2_to_bf16x2((uint16_t)(w4[e] >> 16));
+                            }
+                            *reinterpret_cast<uint4*>(dst + (((2 * h) ^ sw) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+                            *reinterpret_cast<uint4*>(dst + (((2 * h + 1) ^ sw) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
+                        }
+                    } else {
+                    const uint4 q0 = *reinterpret_cast<const uint4*>(pk + row * 32);
+                    const uint4 q1 = *reinterpret_cast<const uint4*>(pk + row * 32 + 16);
+                    uint32_t lo0, lo1, hi0, hi1;
+                    e2m1_tables(pk[4096 + row], lo0, lo1, hi0, hi1);
+                    *reinterpret_cast<uint4*>(dst + ((0 ^ sw) << 4)) = e2m1x8_to_bf16(q0.x, lo0, lo1, hi0, hi1);
+                    *reinterpret_cast<uint4*>(dst + ((1 ^ sw) << 4)) = e2m1x8_to_bf16(q0.y, lo0, lo1, hi0, hi1);
+                    *reinterpret_cast<uint4*>(dst + ((2 ^ sw) << 4)) = e2m1x8_to_bf16(q0.z, lo0, lo1, hi0, hi1);
+                    *reinterpret_cast<uint4*>(dst + ((3 ^ sw) << 4)) = e2m1x8_to_bf16(q0.w, lo0, lo1, hi0, hi1);
+                    e2m1_tables(pk[4096 + 128 + row], lo0, lo1, hi0, hi1);
+                    *reinterpret_cast<uint4*>(dst + ((4 ^ sw) << 4)) = e2m1x8_to_bf16(q1.x, lo0, lo1, hi0, hi1);
+                    *reinterpret_cast<uint4*>(dst + ((5 ^ sw) << 4)) = e2m1x8_to_bf16(q1.y, lo0, lo1, hi0, hi1);
+                    *reinterpret_cast<uint4*>(dst + ((6 ^ sw) << 4)) = e2m1x8_to_bf16(q1.z, lo0, lo1, hi0, hi1);
+                    *reinterpret_cast<uint4*>(dst + ((7 ^ sw) << 4)) = e2m1x8_to_bf16(q1.w, lo0, lo1, hi0, hi1);
+                    }
+                    ptx::fence_proxy_async_smem();  // generic writes, read by the tensor core
+                    __syncwarp();
+                    if (lane == 0) ptx::mbar_arrive(&conv[stage]);
+                    if (++stage == p.stages) {
+                        stage = 0;
+                        phase ^= 1;
+                    }
+                }
+            }
+        }
+    }
+
     // the single-lane roles of warps 0-2 rejoin their warps before the aligned barrier
     // (otherwise a lane arriving late is not held by it)
     __syncwarp();
@@ -1033,16 +1174,16 @@ bool encode_2d(CUtensorMap* m, CUtensorMapDataType dt, int elem_bytes, const voi
                           box_outer, swz);
 }
 
-template <int BK, int MAXR, int ESZ>
+template <int BK, int MAXR, int ESZ, int kW4 = kWcNone>
 cudaError_t launch_t(const GemmParams& p, const CUtensorMap& tmW, const CUtensorMap& tmX,
                      const CUtensorMap& tmB, size_t smem, int grid, cudaStream_t stream)
 {
-    cudaError_t e = cudaFuncSetAttribute(fp8_gemm_kernel<BK, MAXR, ESZ>,
+    cudaError_t e = cudaFuncSetAttribute(fp8_gemm_kernel<BK, MAXR, ESZ, kW4>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid, 1, 1);
-    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.blockDim = dim3(kW4 != kWcNone ? kThreadsW4 : kThreads, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     // a programmatic dependent of the quantiser: the first W loads overlap it
@@ -1051,7 +1192,7 @@ cudaError_t launch_t(const GemmParams& p, const CUtensorMap& tmW, const CUtensor
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, fp8_gemm_kernel<BK, MAXR, ESZ>, tmW, tmX, tmB, p);
+    return cudaLaunchKernelEx(&cfg, fp8_gemm_kernel<BK, MAXR, ESZ, kW4>, tmW, tmX, tmB, p);
 }
 
 size_t align_up(size_t a, size_t b) { return (a + b - 1) / b * b; }
@@ -1102,6 +1243,7 @@ cudaError_t launch_fp8_gemm(const Fp8GemmArgs& a, cudaStream_t stream)
     p.num_tiles = p.n_nb * p.n_tb;
     p.sx = a.sx;
     p.sw = a.sw;
+    p.wsc = a.wsc;
     p.y = a.y;
     p.status = a.status;
     p.partials = a.partials;
@@ -1137,7 +1279,7 @@ cudaError_t launch_fp8_gemm(const Fp8GemmArgs& a, cudaStream_t stream)
     if (cudaFuncGetAttributes(&fa, fp8_gemm_kernel<128, 64, 1>) != cudaSuccess) return cudaErrorInvalidValue;
     const size_t kSmemMax = (size_t)(optin > 0 ? optin : 232448) - fa.sharedSizeBytes - 256;
     const size_t meta = align_up((size_t)p.BN * 20, 128);  // token, adapter, rank, slot, sx
-    const size_t bars = 8 * (2 * kMaxStages + 10);
+    const size_t bars = 8 * (3 * kMaxStages + 10);
     // a slot holds one adapter's B[j][128 n] as loaded, then B'[128 n][r16] in place
     const size_t slot_bytes = (size_t)p.r16 * 256;
     // V' tiles of va adapters: their token ranges are disjoint and contiguous, so their
@@ -1145,8 +1287,11 @@ cudaError_t launch_fp8_gemm(const Fp8GemmArgs& a, cudaStream_t stream)
     auto vq_bytes = [&](int va) -> size_t {
         return (a.lora && va > 0) ? align_up(((size_t)p.BN + 16 * (size_t)(va - 1)) * p.r16 * 2, 128) : 0;
     };
+    const int wc = a.wsc != nullptr ? kWcMxfp4 : (a.esz == 2 && a.w_e4m3 ? kWcE4m3 : kWcNone);
+    const bool w4 = wc != kWcNone;
     auto fit = [&](int bk, int va, int ns) -> int {
-        const size_t stage_bytes = (size_t)kBlockM * bk + (size_t)p.BN * bk;
+        if (w4 && bk != 128) return 0;  // the converter writes 128-byte rows
+        const size_t stage_bytes = (size_t)kBlockM * bk + (size_t)p.BN * bk + wc_stage_bytes(wc);
         const size_t fixed = 1024 + meta + vq_bytes(va) + bars + (size_t)ns * slot_bytes;
         if (fixed >= kSmemMax) return 0;
         const size_t st = (kSmemMax - fixed) / stage_bytes;
@@ -1195,7 +1340,7 @@ cudaError_t launch_fp8_gemm(const Fp8GemmArgs& a, cudaStream_t stream)
     const int esz = a.esz == 2 ? 2 : 1;
     p.k_blocks = (a.K * esz + BK - 1) / BK;
     p.units = (long long)p.num_tiles * p.k_blocks;
-    const size_t stage_bytes = (size_t)kBlockM * BK + (size_t)p.BN * BK;
+    const size_t stage_bytes = (size_t)kBlockM * BK + (size_t)p.BN * BK + wc_stage_bytes(wc);
     p.ring_off = 0;
     p.slots_off = (uint32_t)align_up((size_t)stages * stage_bytes, 1024);
     p.v_off = (uint32_t)align_up(p.slots_off + (size_t)ns * slot_bytes, 128);
@@ -1206,8 +1351,20 @@ cudaError_t launch_fp8_gemm(const Fp8GemmArgs& a, cudaStream_t stream)
     CUtensorMap tmW, tmX, tmB;
     const CUtensorMapSwizzle swz = BK == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
     const CUtensorMapDataType dt = esz == 2 ? CU_TENSOR_MAP_DATA_TYPE_UINT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
-    if (!encode_2d(&tmW, dt, esz, a.Wq, (uint64_t)a.K, (uint64_t)a.N, (uint32_t)(BK / esz), kBlockM, swz) ||
-        !encode_2d(&tmX, dt, esz, a.xq, (uint64_t)a.K, (uint64_t)a.M, (uint32_t)(BK / esz), (uint32_t)p.BN, swz))
+    if (wc == kWcMxfp4) {  // packed codes: [N][K / 2] bytes, boxes of 128 rows x 32 bytes, not swizzled
+        if (esz != 2 || BK != 128 ||
+            !encode_2d(&tmW, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.Wq, (uint64_t)a.K / 2, (uint64_t)a.N, 32, kBlockM,
+                       CU_TENSOR_MAP_SWIZZLE_NONE))
+            return cudaErrorInvalidValue;
+    } else if (wc == kWcE4m3) {  // E4M3 codes: [N][K] bytes, boxes of 128 rows x 64 bytes, not swizzled
+        if (esz != 2 || BK != 128 ||
+            !encode_2d(&tmW, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.Wq, (uint64_t)a.K, (uint64_t)a.N, 64, kBlockM,
+                       CU_TENSOR_MAP_SWIZZLE_NONE))
+            return cudaErrorInvalidValue;
+    } else if (!encode_2d(&tmW, dt, esz, a.Wq, (uint64_t)a.K, (uint64_t)a.N, (uint32_t)(BK / esz), kBlockM, swz)) {
+        return cudaErrorInvalidValue;
+    }
+    if (!encode_2d(&tmX, dt, esz, a.xq, (uint64_t)a.K, (uint64_t)a.M, (uint32_t)(BK / esz), (uint32_t)p.BN, swz))
         return cudaErrorInvalidValue;
     if (a.lora) {
         if (!encode_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, a.B, (uint64_t)a.N,
@@ -1226,18 +1383,26 @@ cudaError_t launch_fp8_gemm(const Fp8GemmArgs& a, cudaStream_t stream)
     // limited to fewer SMs than the device has (an MPS share, a green context) cannot
     // hold that grid: its CTAs would wait until the bounded waits give up.
     const bool small_r = p.r8 <= 16;
-    auto kern = esz == 1 ? (BK == 128 ? (small_r ? fp8_gemm_kernel<128, 16, 1> : fp8_gemm_kernel<128, 64, 1>)
+    auto kern = wc == kWcMxfp4 ? (small_r ? fp8_gemm_kernel<128, 16, 2, kWcMxfp4> : fp8_gemm_kernel<128, 64, 2, kWcMxfp4>)
+              : wc == kWcE4m3 ? (small_r ? fp8_gemm_kernel<128, 16, 2, kWcE4m3> : fp8_gemm_kernel<128, 64, 2, kWcE4m3>)
+              : esz == 1 ? (BK == 128 ? (small_r ? fp8_gemm_kernel<128, 16, 1> : fp8_gemm_kernel<128, 64, 1>)
                                       : (small_r ? fp8_gemm_kernel<64, 16, 1> : fp8_gemm_kernel<64, 64, 1>))
                          : (BK == 128 ? (small_r ? fp8_gemm_kernel<128, 16, 2> : fp8_gemm_kernel<128, 64, 2>)
                                       : (small_r ? fp8_gemm_kernel<64, 16, 2> : fp8_gemm_kernel<64, 64, 2>));
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     int per_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, smem);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, w4 ? kThreadsW4 : kThreads, smem);
     if (e != cudaSuccess) return e;
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
     long long grid = device_sm_count();
     if (grid > p.units) grid = p.units;
+    if (wc == kWcMxfp4)
+        return small_r ? launch_t<128, 16, 2, kWcMxfp4>(p, tmW, tmX, tmB, smem, (int)grid, stream)
+                       : launch_t<128, 64, 2, kWcMxfp4>(p, tmW, tmX, tmB, smem, (int)grid, stream);
+    if (wc == kWcE4m3)
+        return small_r ? launch_t<128, 16, 2, kWcE4m3>(p, tmW, tmX, tmB, smem, (int)grid, stream)
+                       : launch_t<128, 64, 2, kWcE4m3>(p, tmW, tmX, tmB, smem, (int)grid, stream);
     if (esz == 2) {
         if (BK == 128)
             return small_r ? launch_t<128, 16, 2>(p, tmW, tmX, tmB, smem, (int)grid, stream)

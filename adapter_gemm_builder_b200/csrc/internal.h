@@ -16,17 +16,21 @@ cudaError_t launch_build_segments(const int32_t* ids, int T, int n_adapters,
 
 enum SgmvMode { SGMV_SHRINK = 0, SGMV_EXPAND = 1, SGMV_APPLY = 2 };
 
-// x, v, y may be NULL where the mode does not use them.
+// x, v, y may be NULL where the mode does not use them. Tile rows of at most
+// skip_small tokens are left alone (the warp kernel takes them).
 cudaError_t launch_sgmv(int mode, const void* x, int64_t x_slice_stride, const lora_pool_t& pool,
                         const lora_segments_t& seg, float* v, void* y, cudaStream_t stream,
-                        bool pdl_trigger);
+                        bool pdl_trigger, int skip_small = 0);
 
-// The fused shrink + expand as a persistent grid streaming work items (batches
-// whose tiles hold up to LORA_TILE_TOKENS tokens); ws holds
-// sgmv_stream_workspace_bytes(T, pool) bytes.
-cudaError_t launch_sgmv_stream(const void* x, int64_t x_slice_stride, const lora_pool_t& pool,
-                               const lora_segments_t& seg, void* y, void* ws, cudaStream_t stream);
-size_t sgmv_stream_workspace_bytes(int T, const lora_pool_t& pool);
+// The fused shrink + expand of the tile rows of at most kWarpSmallTile tokens
+// (sgmv_warp.cu): one warp per work item, two launches; ws holds
+// sgmv_warp_workspace_bytes(T, pool) bytes, zeroed by sgmv_warp_zero first.
+constexpr int kWarpSmallTile = 8;
+cudaError_t sgmv_warp_zero(const lora_pool_t& pool, const lora_segments_t& seg, void* ws, cudaStream_t stream);
+cudaError_t launch_sgmv_warp(const void* x, int64_t x_slice_stride, const lora_pool_t& pool,
+                             const lora_segments_t& seg, void* y, void* ws, cudaStream_t stream);
+size_t sgmv_warp_workspace_bytes(int T, const lora_pool_t& pool);
+
 
 // Token-wise merge of the selected adapters into the backbone (merge.cu).
 cudaError_t launch_lora_switch_merge(const void* W, int N, int K, const lora_pool_t& pool, const int32_t* sel,
@@ -49,6 +53,10 @@ cudaError_t launch_quantize_rows(const void* x, const int32_t* perm, int M, int 
                                  float* sx, void* zero, size_t zero_words, cudaStream_t stream,
                                  bool copy_bf16 = false);
 
+// OCP MX FP4 quantisation of W bf16 [N][K] (K % 64 == 0): Wp [N][K / 2] packed
+// E2M1 codes (element 2i in the low nibble), Wsc E8M0 [ceil(N / 128)][K / 32][128].
+cudaError_t launch_mxfp4_quantize(const void* W, int N, int K, uint8_t* Wp, uint8_t* Wsc, cudaStream_t stream);
+
 struct Fp8GemmArgs {
     int M, N, K;
     int esz;             // operand element bytes: 1 = E4M3 (kind::f8f6f4), 2 = bf16 (kind::f16)
@@ -56,6 +64,9 @@ struct Fp8GemmArgs {
     const float* sx;     // [M], perm order (1 for bf16 operands)
     const uint8_t* Wq;   // e4m3 (or bf16) [N][K]
     const float* sw;     // [N]; NULL = 1 (bf16 weights carry no scale)
+    const uint8_t* wsc;  // MX FP4 weights (esz 2): Wq holds the packed E2M1 codes
+                         // [N][K / 2] and wsc the E8M0 scales [ceil(N / 128)][K / 32][128]
+    bool w_e4m3;         // esz 2 with E4M3 weight codes (W8A16): converted to bf16 on chip
     uint16_t* y;         // bf16 [M][N]
     uint32_t* status;    // device status word
     float* partials;     // fp32 [SMs][128][fp8_gemm_tile_n(M)] stream-K partials

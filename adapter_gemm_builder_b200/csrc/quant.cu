@@ -83,7 +83,77 @@ quantize_rows_kernel(const uint16_t* __restrict__ x, const int32_t* __restrict__
     }
 }
 
+// OCP MX FP4 quantisation of weight rows: thread = (row n, block b of 32
+// values). X = 2^(floor(log2(amax)) - 2) as an E8M0 exponent clamped to
+// 0..254 (0 for an all-zero block); each value v / X (exact: a power of two)
+// rounded to the nearest E2M1 value, ties to the even fraction bit, magnitudes
+// past 6 saturated. Codes are packed two per byte, element 2i in the low
+// nibble; the scales are stored per group of 128 rows, block-major
+// ([n / 128][b][n % 128]), so one k-block's scales for 128 rows are contiguous.
+__global__ void __launch_bounds__(kThreads)
+mxfp4_quantize_kernel(const uint16_t* __restrict__ W, int N, int K, uint8_t* __restrict__ Wp,
+                      uint8_t* __restrict__ Wsc)
+{
+    const int nb = K / 32;
+    const long long i = (long long)blockIdx.x * kThreads + threadIdx.x;
+    if (i >= (long long)N * nb) return;
+    const int n = (int)(i / nb), b = (int)(i - (long long)n * nb);
+    const uint4* src = reinterpret_cast<const uint4*>(W + (size_t)n * K + b * 32);
+    uint32_t w[16];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const uint4 c = src[q];
+        w[4 * q] = c.x;
+        w[4 * q + 1] = c.y;
+        w[4 * q + 2] = c.z;
+        w[4 * q + 3] = c.w;
+    }
+    float amax = 0.f;
+#pragma unroll
+    for (int q = 0; q < 16; ++q) {
+        amax = fmaxf(amax, fabsf(__uint_as_float(w[q] << 16)));
+        amax = fmaxf(amax, fabsf(__uint_as_float(w[q] & 0xffff0000u)));
+    }
+    int e = 0;
+    if (amax > 0.f) e = min(254, max(0, ilogbf(amax) - 2 + 127));
+    auto code = [&](float v) -> uint32_t {
+        const float a = fabsf(ldexpf(v, 127 - e));
+        uint32_t c;
+        if (a <= 0.25f) c = 0;
+        else if (a < 0.75f) c = 1;
+        else if (a <= 1.25f) c = 2;
+        else if (a < 1.75f) c = 3;
+        else if (a <= 2.5f) c = 4;
+        else if (a < 3.5f) c = 5;
+        else if (a <= 5.0f) c = 6;
+        else c = 7;
+        return c | (signbit(v) ? 8u : 0u);
+    };
+    uint32_t out[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        uint32_t o = 0;
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+            const uint32_t word = w[4 * q + h];
+            o |= code(__uint_as_float(word << 16)) << (8 * h);
+            o |= code(__uint_as_float(word & 0xffff0000u)) << (8 * h + 4);
+        }
+        out[q] = o;
+    }
+    *reinterpret_cast<uint4*>(Wp + (size_t)n * (K / 2) + b * 16) = make_uint4(out[0], out[1], out[2], out[3]);
+    Wsc[((size_t)(n >> 7) * nb + b) * 128 + (n & 127)] = (uint8_t)e;
+}
+
 }  // namespace
+
+cudaError_t launch_mxfp4_quantize(const void* W, int N, int K, uint8_t* Wp, uint8_t* Wsc, cudaStream_t stream)
+{
+    const long long threads = (long long)N * (K / 32);
+    const unsigned blocks = (unsigned)((threads + kThreads - 1) / kThreads);
+    mxfp4_quantize_kernel<<<blocks, kThreads, 0, stream>>>(static_cast<const uint16_t*>(W), N, K, Wp, Wsc);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_quantize_rows(const void* x, const int32_t* perm, int M, int K, uint8_t* xq,
                                  float* sx, void* zero, size_t zero_words, cudaStream_t stream,

@@ -1,7 +1,6 @@
-// sgmv_common.cuh -- pieces shared by the SGMV kernels (sgmv.cu: one tile per
+// sgmv_common.cuh -- pieces of the cluster SGMV kernel (sgmv.cu: one tile per
 // thread-block cluster with the split-K exchange of v in distributed shared
-// memory; sgmv_stream.cu: a persistent grid that streams work items of many
-// tiles): launch constants, the pools' tensor maps, the shared-memory tile
+// memory): launch constants, the pools' tensor maps, the shared-memory tile
 // layouts and the bounded waits.
 #pragma once
 #include <cuda.h>

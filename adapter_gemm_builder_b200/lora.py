@@ -30,6 +30,8 @@ LORA_OP_APPLY = 2
 LORA_OP_FP8_GEMM = 3
 LORA_OP_BF16_GEMM = 4
 LORA_OP_FP8_BACKWARD = 5
+LORA_OP_MXFP4_GEMM = 6
+LORA_OP_W8A16_GEMM = 7
 
 EXPORTED = [
     "lora_workspace_size", "lora_workspace_init", "lora_workspace_status", "lora_build_segments",
@@ -37,7 +39,8 @@ EXPORTED = [
     "lora_status_string", "lora_version", "lora_tile_tokens", "lora_tile_tokens_for", "lora_max_tiles",
     "lora_segments_status", "fp8_gemm_lora_epilogue_noalloc", "lora_noalloc_scratch_bytes",
     "lora_noalloc_status", "lora_debug_set_wait_limit", "bf16_gemm_lora_epilogue",
-    "lora_switch_merge", "fp8_lora_backward",
+    "lora_switch_merge", "fp8_lora_backward", "mxfp4_quantize_rows", "mxfp4_gemm_lora_epilogue",
+    "w8a16_gemm_lora_epilogue",
 ]
 
 
@@ -104,6 +107,9 @@ def load(path: str = LIB_PATH):
             "bf16_gemm_lora_epilogue": (I, [P, I, I, I, P, P, P, P, P, Z, P]),
             "lora_switch_merge": (I, [P, I, I, P, P, P, I, P, P]),
             "fp8_lora_backward": (I, [P, P, I, I, I, P, P, P, P, P, P, P, P, Z, P]),
+            "mxfp4_quantize_rows": (I, [P, I, I, P, P, P]),
+            "mxfp4_gemm_lora_epilogue": (I, [P, I, I, I, P, P, P, P, P, P, Z, P]),
+            "w8a16_gemm_lora_epilogue": (I, [P, I, I, I, P, P, P, P, P, P, Z, P]),
         }
         for name, (res, args) in sig.items():
             f = getattr(lib, name)
@@ -274,6 +280,38 @@ def bf16_gemm_lora_epilogue(x: torch.Tensor, W: torch.Tensor, pool: Pool | None,
     N = W.shape[0]
     _check(load().bf16_gemm_lora_epilogue(
         _ptr(x), M, K, N, _ptr(W), ctypes.byref(pool.c) if pool else None,
+        ctypes.byref(seg.c) if seg else None, _ptr(y), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def w8a16_gemm_lora_epilogue(x: torch.Tensor, Wq: torch.Tensor, w_scale: torch.Tensor,
+                             pool: Pool | None, seg: Segments | None, y: torch.Tensor, ws: torch.Tensor,
+                             stream=None) -> None:
+    """y = w_scale . (x . E4M3(Wq)^T) + s_a (x.A_a).B_a with bf16 x (W8A16)."""
+    M, K = x.shape
+    N = Wq.shape[0]
+    _check(load().w8a16_gemm_lora_epilogue(
+        _ptr(x), M, K, N, _ptr(Wq), _ptr(w_scale), ctypes.byref(pool.c) if pool else None,
+        ctypes.byref(seg.c) if seg else None, _ptr(y), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def mxfp4_scale_bytes(N: int, K: int) -> int:
+    """Bytes of the E8M0 scale array of an [N, K] MX FP4 weight (rows padded to 128)."""
+    return (N + 127) // 128 * 128 * (K // 32)
+
+
+def mxfp4_quantize_rows(W: torch.Tensor, Wp: torch.Tensor, Wsc: torch.Tensor, stream=None) -> None:
+    N, K = W.shape
+    _check(load().mxfp4_quantize_rows(_ptr(W), N, K, _ptr(Wp), _ptr(Wsc), _stream(stream)))
+
+
+def mxfp4_gemm_lora_epilogue(x: torch.Tensor, Wp: torch.Tensor, Wsc: torch.Tensor, pool: Pool | None,
+                             seg: Segments | None, y: torch.Tensor, ws: torch.Tensor,
+                             stream=None) -> None:
+    """y = x.W^T + s_a (x.A_a).B_a with W in MX FP4 (Wp [N, K/2], Wsc) and bf16 x."""
+    M, K = x.shape
+    N = Wp.shape[0]
+    _check(load().mxfp4_gemm_lora_epilogue(
+        _ptr(x), M, K, N, _ptr(Wp), _ptr(Wsc), ctypes.byref(pool.c) if pool else None,
         ctypes.byref(seg.c) if seg else None, _ptr(y), _ptr(ws), ws.numel(), _stream(stream)))
 
 

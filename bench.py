@@ -68,6 +68,7 @@ def parse_args():
     ap.add_argument("--fp8-reps", type=int, default=20, help="graph replays per timing")
     ap.add_argument("--no-bf16", action="store_true", help="skip the bf16 GEMM + LoRA section")
     ap.add_argument("--no-merge", action="store_true", help="skip the adapter-merge section")
+    ap.add_argument("--no-mxfp4", action="store_true", help="skip the MX FP4 GEMM + LoRA section")
     return ap.parse_args()
 
 
@@ -336,9 +337,12 @@ class _Events:
                                                 ctypes.c_void_p(stream.cuda_stream), 1) == 0
 
 
-def apply_launches():
-    """Kernels of this library one lora_apply launches (the bench counts them)."""
-    return 1
+def apply_launches(p):
+    """Kernels of this library one lora_apply launches: one for a decode-like batch
+    (T <= 64 and T <= 2 n_adapters); otherwise the cluster kernel for the larger tiles
+    and the warp kernel's two launches for the small ones (plus a memset of its
+    counters, not counted)."""
+    return 1 if (p.T <= 64 and p.T <= 2 * p.n_adapters) else 3
 
 
 def time_apply(p, dev, steps, warmup, stream, ext, world=1, clocks=None):
@@ -467,6 +471,7 @@ def roofline_apply(p, t, hbm_peak, peak_src, workload):
     return {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
             "frac": achieved / hbm_peak, "traffic": profiled_traffic("sgmv.cu", workload),
             "kernel": "lora_apply (sgmv kernels)", "kernel_us": t["kernel_ms"] * 1e3,
+            "launches_per_call": apply_launches(p),
             "algorithmic_bytes_per_launch": bytes_step,
             "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs, burst copy)",
             "timing": t["timing"]}
@@ -519,6 +524,7 @@ def run_ours(args):
     fp8 = None if args.no_fp8 else run_fp8(args, dev, stream, hbm_peak, bf16_peak, bf16_sust, peak_src)
     bf16 = None if args.no_bf16 else run_bf16(args, dev, stream, hbm_peak, bf16_peak, peak_src)
     merge = None if args.no_merge else run_merge(args, dev, stream, hbm_peak, peak_src)
+    mxfp4 = None if args.no_mxfp4 else run_mxfp4(args, dev, stream, hbm_peak, bf16_peak, peak_src)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -531,10 +537,10 @@ def run_ours(args):
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {**workload_config(p, args.workload), "l2": t["l2"], "launch": t["launch"],
                        "parallelism": f"replicas x{world}"},
-            "roofline": roofline, "e2e": e2e, "gpu_launches": (1 + apply_launches()) * K,
+            "roofline": roofline, "e2e": e2e, "gpu_launches": (1 + apply_launches(p)) * K,
             "clocks": t["clocks"], "status_ok": t["status_ok"],
             "cpu_baseline": cpu, "workloads": extras, "fp8_gemm_lora": fp8, "bf16_gemm_lora": bf16,
-            "switch_merge": merge,
+            "switch_merge": merge, "mxfp4_gemm_lora": mxfp4,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -842,6 +848,87 @@ def run_bf16(args, dev, stream, hbm_peak, bf16_peak, peak_src):
             "attainable_frac": (flops / t) / min(bf16_peak * 1e12, flops / bytes_call * hbm_peak * 1e9),
             "status_ok": res["lora_status"] == 0 and res["base_status"] == 0,
             "l2": f"W, x, the adapters and y rotate over {R} copies ({R * set_bytes / 2**20:.0f} MiB)",
+        }
+        del sets
+    return out
+
+
+def run_mxfp4(args, dev, stream, hbm_peak, bf16_peak, peak_src):
+    """The 4-bit base (OCP MX FP4 weights, bf16 activations) with the fused LoRA term at
+    the FP8 section's decode shapes (K 8192, N 28672, 16 adapters of rank 16, Zipf ids),
+    against the same call without LoRA: us per call, TFLOP/s against the bf16 peak (its
+    MMAs are kind::f16) and the HBM fraction of its algorithmic bytes (packed codes,
+    scales, x, y and the adapters present)."""
+    import numpy as np
+    import torch
+
+    from adapter_gemm_builder_b200 import lora as L
+    from adapter_gemm_builder_b200 import workloads as wl
+    K, N, n_ad, r = 8192, 28672, 16, 16
+    gen = torch.Generator(device=dev).manual_seed(5)
+    W = (torch.randn((N, K), generator=gen, device=dev) * (1.0 / math.sqrt(K))).to(torch.bfloat16)
+    Wp = torch.empty((N, K // 2), dtype=torch.uint8, device=dev)
+    Wsc = torch.zeros(L.mxfp4_scale_bytes(N, K), dtype=torch.uint8, device=dev)
+    L.mxfp4_quantize_rows(W, Wp, Wsc)
+    del W
+    out = {"shape": {"K": K, "N": N, "adapters": n_ad, "r": r, "ids": "zipf(1.1)"},
+           "peak_tflops_bf16": bf16_peak, "peak_hbm_gbs": hbm_peak,
+           "peak_source": f"{peak_src} (MEASURED_PEAKS.json)", "M": {}}
+    for M in args.fp8_m:
+        q = wl.fp8_problem(M, K=K, N=N, n_adapters=n_ad, r=r, seed=3, W=np.zeros((1, 1), np.uint16))
+        tb = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+        act = np.unique(q.ids)
+        set_bytes = q.x.nbytes + q.A.nbytes + q.B.nbytes + M * N * 2
+        R = int(min(32, max(2, math.ceil(2.5 * L2_BYTES / set_bytes))))
+        base = dict(x=tb(q.x), A=tb(q.A), B=tb(q.B), ids=torch.from_numpy(q.ids).to(dev),
+                    ranks=torch.from_numpy(q.ranks).to(dev), scales=torch.from_numpy(q.scales).to(dev))
+        sets = []
+        for k in range(R):
+            d = {key: (v.clone() if k else v) for key, v in base.items()}
+            d["pool"] = L.Pool(d["A"], d["B"], d["ranks"], d["scales"])
+            d["seg"] = L.Segments(M, n_ad, device=dev)
+            L.lora_build_segments(d["ids"], n_ad, d["seg"])
+            d["y"] = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+            d["ws"] = L.workspace(L.LORA_OP_MXFP4_GEMM, M, K, d["pool"], device=dev)
+            d["ws0"] = L.workspace(L.LORA_OP_MXFP4_GEMM, M, K, None, device=dev)
+            sets.append(d)
+        res = {}
+        for tag in ("lora", "base"):
+            def call(d):
+                if tag == "lora":
+                    L.mxfp4_gemm_lora_epilogue(d["x"], Wp, Wsc, d["pool"], d["seg"], d["y"], d["ws"])
+                else:
+                    L.mxfp4_gemm_lora_epilogue(d["x"], Wp, Wsc, None, None, d["y"], d["ws0"])
+            with torch.cuda.stream(stream):
+                for d in sets:
+                    call(d)
+                stream.synchronize()
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=stream):
+                    for d in sets:
+                        call(d)
+                for _ in range(3):
+                    g.replay()
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                for _ in range(args.fp8_reps):
+                    g.replay()
+                b.record(stream)
+            torch.cuda.synchronize()
+            res[tag] = a.elapsed_time(b) / (args.fp8_reps * R) * 1e3
+            res[tag + "_status"] = max(L.lora_workspace_status(d["ws" if tag == "lora" else "ws0"])[0]
+                                       for d in sets)
+        lora_bytes = int(len(act)) * r * (K + N) * 2 + M * r * 4
+        bytes_call = N * K // 2 + L.mxfp4_scale_bytes(N, K) + M * K * 2 + M * N * 2 + lora_bytes
+        flops = 2.0 * M * N * K
+        t = res["lora"] * 1e-6
+        out["M"][str(M)] = {
+            "us_per_call": res["lora"], "us_per_call_no_lora": res["base"],
+            "overhead_vs_no_lora": res["lora"] / res["base"] - 1.0,
+            "tflops": flops / t / 1e12, "tensor_frac": flops / t / 1e12 / bf16_peak,
+            "hbm_gbs": bytes_call / t / 1e9, "hbm_frac": bytes_call / t / 1e9 / hbm_peak,
+            "status_ok": res["lora_status"] == 0 and res["base_status"] == 0,
+            "l2": f"x, adapters and y rotate over {R} copies; the packed weight is read once per call",
         }
         del sets
     return out

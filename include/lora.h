@@ -145,6 +145,8 @@ LORA_API int lora_segments_status(const lora_segments_t* seg, lora_stream_t stre
 #define LORA_OP_FP8_GEMM 3
 #define LORA_OP_BF16_GEMM 4
 #define LORA_OP_FP8_BACKWARD 5
+#define LORA_OP_MXFP4_GEMM 6
+#define LORA_OP_W8A16_GEMM 7
 
 /*
  * Bytes of workspace an operation needs (0 if it needs none), or (size_t)-1
@@ -289,6 +291,59 @@ LORA_API int fp8_gemm_lora_epilogue(const void* x, int M, int K, int N, const ui
 LORA_API int bf16_gemm_lora_epilogue(const void* x, int M, int K, int N, const void* W,
                                      const lora_pool_t* pool, const lora_segments_t* seg, void* y,
                                      void* ws, size_t ws_bytes, lora_stream_t stream);
+
+/*
+ * The 8-bit weights with the activations kept in 16 bits (W8A16: the EpiLoRA
+ * abstract's 8-bit base, sentence 2, under its 16-bit activation engine,
+ * sentence 6) and the fused LoRA term:
+ *   y[m][n] = bf16( w_scale[n] * sum_k x[m][k] * E4M3(Wq[n][k])
+ *                   + s_a * sum_{j < r_a} v[m][j] * B[0][a][j][n] ),  v = x.A_a.
+ * The same weights as fp8_gemm_lora_epilogue (fp8_quantize_rows of W), but x is
+ * not quantised: the kernel of bf16_gemm_lora_epilogue, whose weight tiles
+ * arrive as E4M3 codes and are turned into bf16 on chip (exactly) by four
+ * converter warps before the tcgen05 kind::f16 MMAs; the epilogue applies
+ * w_scale as on the 8-bit path.
+ *   x bf16 [M][K]; Wq e4m3 [N][K]; w_scale fp32 [N]; y bf16 [M][N] (out).
+ *   pool / seg as for fp8_gemm_lora_epilogue (including its many-adapter path).
+ *   ws: lora_workspace_size(LORA_OP_W8A16_GEMM, M, K, pool) bytes.
+ * Limits: K % 64 == 0, N % 8 == 0, M >= 1.
+ */
+LORA_API int w8a16_gemm_lora_epilogue(const void* x, int M, int K, int N, const uint8_t* Wq, const float* w_scale,
+                                      const lora_pool_t* pool, const lora_segments_t* seg, void* y, void* ws,
+                                      size_t ws_bytes, lora_stream_t stream);
+
+/*
+ * OCP MX FP4 quantisation of base weights (the 4-bit base of the EpiLoRA
+ * abstract, sentence 2, read as the MX format): each block of 32 consecutive
+ * values of a row shares the E8M0 scale X = 2^(floor(log2(amax)) - 2)
+ * (exponent clamped to 0..254; 0 for an all-zero block) and each value
+ * becomes the E2M1 code nearest to v / X (ties to the even fraction bit,
+ * saturating at +-6). Finite weights only.
+ *   W bf16 [N][K] (K % 64 == 0);
+ *   Wp uint8 [N][K / 2]: two codes per byte, element 2i in the low nibble;
+ *   Wsc uint8 [ceil(N / 128)][K / 32][128]: the E8M0 scale of block b of row n
+ *   at [n / 128][b][n % 128] (one k-block's scales of 128 rows are contiguous).
+ * One kernel launch.
+ */
+LORA_API int mxfp4_quantize_rows(const void* W, int N, int K, uint8_t* Wp, uint8_t* Wsc, lora_stream_t stream);
+
+/*
+ * 4-bit base GEMM with the fused LoRA term: the weights in OCP MX FP4
+ * (mxfp4_quantize_rows), the activations in bf16 (the EpiLoRA abstract's
+ * 4-bit base, sentence 2, and its 16-bit activation engine, sentence 6):
+ *   y[m][n] = bf16( sum_k x[m][k] * E2M1(Wp[n][k]) * 2^(Wsc[n][k / 32] - 127)
+ *                   + s_a * sum_{j < r_a} v[m][j] * B[0][a][j][n] ),  v = x.A_a.
+ * The kernel of bf16_gemm_lora_epilogue, whose weight tiles arrive as packed
+ * codes and scales (half the bytes of an 8-bit weight) and are turned into
+ * bf16 on chip by four converter warps before the tcgen05 kind::f16 MMAs.
+ *   x bf16 [M][K]; Wp / Wsc as mxfp4_quantize_rows; y bf16 [M][N] (out).
+ *   pool / seg as for fp8_gemm_lora_epilogue (including its many-adapter path).
+ *   ws: lora_workspace_size(LORA_OP_MXFP4_GEMM, M, K, pool) bytes.
+ * Limits: K % 64 == 0, N % 8 == 0, M >= 1.
+ */
+LORA_API int mxfp4_gemm_lora_epilogue(const void* x, int M, int K, int N, const uint8_t* Wp, const uint8_t* Wsc,
+                                      const lora_pool_t* pool, const lora_segments_t* seg, void* y, void* ws,
+                                      size_t ws_bytes, lora_stream_t stream);
 
 /*
  * Gradients of the LoRA layer for training the adapters on a frozen 8-bit

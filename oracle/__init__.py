@@ -91,6 +91,8 @@ def _load():
             lib.orc_mxfp4_quantize.argtypes = [P, I, I, P, P]
             lib.orc_mxfp4_gemm_lora_sampled.restype = None
             lib.orc_mxfp4_gemm_lora_sampled.argtypes = [P, P, P, I, P, P, I, I, I, P, P, P, P, P, I, P]
+            lib.orc_w8a16_gemm_lora_sampled.restype = None
+            lib.orc_w8a16_gemm_lora_sampled.argtypes = [P, P, P, I, P, P, I, I, I, P, P, P, P, P, I, P]
             lib.orc_num_threads.restype = I
             lib.orc_set_num_threads.argtypes = [I]
             _lib = lib
@@ -322,4 +324,25 @@ def mxfp4_gemm_lora_sampled(x, codes, scales, rows, cols, A=None, B=None, ranks=
     lib.orc_mxfp4_gemm_lora_sampled(_p(x), _p(codes), _p(scales), K, _p(A), _p(B), n_adapters, r_max,
                                     N, _p(ranks), _p(scales_lora), _p(ids), _p(rows), _p(cols),
                                     rows.shape[0], _p(out))
+    return out
+
+
+def w8a16_gemm_lora_sampled(x, Wq, sw, rows, cols, A=None, B=None, ranks=None, scales=None,
+                            ids=None) -> np.ndarray:
+    """y = sw . (x . E4M3(Wq)^T) + LoRA with bf16 x (W8A16), at the (rows, cols) samples."""
+    lib = _load()
+    x = _c(x, np.uint16); Wq = _c(Wq, np.uint8); sw = _c(sw, np.float32)
+    rows = _c(rows, np.int32); cols = _c(cols, np.int32)
+    K = x.shape[1]
+    N = Wq.shape[0]
+    if A is not None:
+        A = _c(A, np.uint16); B = _c(B, np.uint16); ranks = _c(ranks, np.int32)
+        scales = _c(scales, np.float32); ids = _c(ids, np.int32)
+        n_adapters, _, r_max = A.shape
+    else:
+        n_adapters, r_max = 0, 0
+    out = np.zeros(rows.shape[0], np.float64)
+    lib.orc_w8a16_gemm_lora_sampled(_p(x), _p(Wq), _p(sw), K, _p(A), _p(B), n_adapters, r_max, N,
+                                    _p(ranks), _p(scales), _p(ids), _p(rows), _p(cols), rows.shape[0],
+                                    _p(out))
     return out

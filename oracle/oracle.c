@@ -591,6 +591,47 @@ void orc_mxfp4_gemm_lora_sampled(const uint16_t* x, const uint8_t* codes, const 
     }
 }
 
+/*
+ * The 8-bit-weight GEMM with the activations kept in bf16 (W8A16: the FP8
+ * weights of the EpiLoRA abstract, sentence 2, under its 16-bit activation
+ * engine, sentence 6) and the LoRA term, at the listed (m, n) samples:
+ *   y[m][n] = sw[n] * sum_k x[m][k] * E4M3(Wq[n][k])
+ *           + s_a * sum_{j < r_a} (sum_k x[m][k] A[a][k][j]) * B[a][j][n].
+ * A == NULL: no LoRA term. Wq / sw as orc_quantize_rows makes them.
+ */
+void orc_w8a16_gemm_lora_sampled(const uint16_t* x, const uint8_t* Wq, const float* sw, int K,
+                                 const uint16_t* A, const uint16_t* B, int n_adapters, int r_max,
+                                 int h_out, const int32_t* ranks, const float* scales,
+                                 const int32_t* ids, const int32_t* rows, const int32_t* cols,
+                                 int n_samples, double* out)
+{
+#pragma omp parallel for schedule(dynamic, 16)
+    for (int i = 0; i < n_samples; ++i) {
+        int m = rows[i], n = cols[i];
+        double acc = 0.0;
+        for (int k = 0; k < K; ++k)
+            acc += orc_bf16_decode(x[(size_t)m * K + k]) * orc_e4m3_decode(Wq[(size_t)n * K + k]);
+        double y = (double)sw[n] * acc;
+        if (A != NULL) {
+            int a = valid_id(ids, m, n_adapters);
+            if (a >= 0) {
+                int r = rank_of(ranks, a, r_max);
+                double s = scales ? (double)scales[a] : 1.0;
+                double l = 0.0;
+                for (int j = 0; j < r; ++j) {
+                    double vj = 0.0;
+                    for (int k = 0; k < K; ++k)
+                        vj += orc_bf16_decode(x[(size_t)m * K + k]) *
+                              orc_bf16_decode(A[((size_t)a * K + k) * r_max + j]);
+                    l += vj * orc_bf16_decode(B[((size_t)a * r_max + j) * h_out + n]);
+                }
+                y += s * l;
+            }
+        }
+        out[i] = y;
+    }
+}
+
 /* Threads the OpenMP loops above use. */
 int orc_num_threads(void)
 {

@@ -792,3 +792,36 @@ def test_mxfp4_gemm_lora_brute_force_rationals():
             v = [sum(X[m][k] * Af[k][j] for k in range(K)) for j in range(ranks[a])]
             y += Fraction(float(sl[a])) * sum(v[j] * Bf[j][n] for j in range(ranks[a]))
         assert Fraction(got[i]) == y
+
+
+# ---------------------------------------------------------------- W8A16 (FP8 weights, bf16 activations)
+
+def test_w8a16_equals_bf16_linear_on_power_of_two_scales():
+    """With power-of-two channel scales every dequantised weight sw * E4M3(code) is a bf16
+    value, and the W8A16 product equals the (separately pinned) bf16 linear oracle."""
+    rng = np.random.default_rng(51)
+    M, K, N = 5, 96, 12
+    x = wl.normal_bf16(rng, (M, K))
+    Wq = rng.integers(0, 256, (N, K)).astype(np.uint8)
+    Wq[(Wq & 0x7F) == 0x7F] = 0x10          # no NaN codes
+    sw = (2.0 ** rng.integers(-8, 3, N)).astype(np.float32)
+    W = wl.to_bf16_bits((oracle.e4m3_to_f64(Wq) * sw[:, None]).astype(np.float32))
+    assert np.array_equal(oracle.bf16_to_f64(W), oracle.e4m3_to_f64(Wq) * sw[:, None])
+    rows = np.repeat(np.arange(M), N).astype(np.int32)
+    cols = np.tile(np.arange(N), M).astype(np.int32)
+    got = oracle.w8a16_gemm_lora_sampled(x, Wq, sw, rows, cols)
+    assert np.allclose(got, oracle.linear_bf16_sampled(x, W, rows, cols), rtol=1e-13, atol=1e-13)
+
+
+def test_w8a16_lora_term_matches_the_apply_oracle():
+    """The LoRA term of W8A16 is the pinned apply oracle's term (zero base weight)."""
+    p = _random_problem(52, T=6, n_adapters=3, h_in=32, h_out=16, r_max=8)
+    Wq = np.zeros((p.h_out, p.h_in), np.uint8)
+    sw = np.ones(p.h_out, np.float32)
+    rows = np.repeat(np.arange(p.T), p.h_out).astype(np.int32)
+    cols = np.tile(np.arange(p.h_out), p.T).astype(np.int32)
+    got = oracle.w8a16_gemm_lora_sampled(p.x[0], Wq, sw, rows, cols, A=p.A[0], B=p.B[0], ranks=p.ranks,
+                                         scales=p.scales, ids=p.ids).reshape(p.T, p.h_out)
+    want = oracle.lora_apply(p.x[0], p.A[0], p.B[0], p.ranks, p.scales, p.ids,
+                             np.zeros((p.T, p.h_out), np.uint16))
+    assert np.allclose(got, want, rtol=1e-12, atol=1e-12)
