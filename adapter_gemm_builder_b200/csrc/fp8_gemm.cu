@@ -75,6 +75,7 @@ struct GemmParams {
     const float* sx;
     const float* sw;
     const uint8_t* wsc;  // MX FP4 block scales (kW4)
+    const uint8_t* Wpk;  // MX FP4 codes in 128 x 64 tiles of 4096 bytes
     uint16_t* y;
     uint32_t* status;
     float* partials;  // fp32 stream-K partial accumulators, [gridDim.x][BN/16][4][128][4]
@@ -392,7 +393,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
                         // packed codes (128 rows x 32 bytes) and the k-block's two scale blocks
                         const uint32_t sP = sX + (uint32_t)(p.BN * BK);
                         ptx::mbar_arrive_expect_tx(&full[stage], (uint32_t)(4096 + 256 + p.BN * BK));
-                        ptx::tma_load_2d_hint(sP, &tmW, &full[stage], kb * 32, nb * kBlockM, w_policy);
+                        ptx::bulk_g2s(sP, p.Wpk + ((size_t)nb * (p.K / 64) + kb) * 4096, 4096, &full[stage]);
                         ptx::bulk_g2s(sP + 4096, p.wsc + ((size_t)nb * (p.K / 32) + kb * 2) * kBlockM, 256,
                                       &full[stage]);
                     } else if constexpr (kW4 == kWcE4m3) {
@@ -1244,6 +1245,7 @@ cudaError_t launch_fp8_gemm(const Fp8GemmArgs& a, cudaStream_t stream)
     p.sx = a.sx;
     p.sw = a.sw;
     p.wsc = a.wsc;
+    p.Wpk = a.Wq;
     p.y = a.y;
     p.status = a.status;
     p.partials = a.partials;
@@ -1351,11 +1353,11 @@ cudaError_t launch_fp8_gemm(const Fp8GemmArgs& a, cudaStream_t stream)
     CUtensorMap tmW, tmX, tmB;
     const CUtensorMapSwizzle swz = BK == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
     const CUtensorMapDataType dt = esz == 2 ? CU_TENSOR_MAP_DATA_TYPE_UINT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
-    if (wc == kWcMxfp4) {  // packed codes: [N][K / 2] bytes, boxes of 128 rows x 32 bytes, not swizzled
-        if (esz != 2 || BK != 128 ||
-            !encode_2d(&tmW, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.Wq, (uint64_t)a.K / 2, (uint64_t)a.N, 32, kBlockM,
-                       CU_TENSOR_MAP_SWIZZLE_NONE))
-            return cudaErrorInvalidValue;
+    if (!encode_2d(&tmX, dt, esz, a.xq, (uint64_t)a.K, (uint64_t)a.M, (uint32_t)(BK / esz), (uint32_t)p.BN, swz))
+        return cudaErrorInvalidValue;
+    if (wc == kWcMxfp4) {  // packed codes in 4096-byte tiles: 1-D bulk copies, no tensor map
+        if (esz != 2 || BK != 128) return cudaErrorInvalidValue;
+        tmW = tmX;  // a valid map the kernel never loads through
     } else if (wc == kWcE4m3) {  // E4M3 codes: [N][K] bytes, boxes of 128 rows x 64 bytes, not swizzled
         if (esz != 2 || BK != 128 ||
             !encode_2d(&tmW, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.Wq, (uint64_t)a.K, (uint64_t)a.N, 64, kBlockM,
@@ -1364,8 +1366,6 @@ cudaError_t launch_fp8_gemm(const Fp8GemmArgs& a, cudaStream_t stream)
     } else if (!encode_2d(&tmW, dt, esz, a.Wq, (uint64_t)a.K, (uint64_t)a.N, (uint32_t)(BK / esz), kBlockM, swz)) {
         return cudaErrorInvalidValue;
     }
-    if (!encode_2d(&tmX, dt, esz, a.xq, (uint64_t)a.K, (uint64_t)a.M, (uint32_t)(BK / esz), (uint32_t)p.BN, swz))
-        return cudaErrorInvalidValue;
     if (a.lora) {
         if (!encode_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, a.B, (uint64_t)a.N,
                        (uint64_t)a.n_adapters * a.r_max, 128, 8, CU_TENSOR_MAP_SWIZZLE_NONE))

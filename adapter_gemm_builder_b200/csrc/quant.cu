@@ -88,8 +88,11 @@ quantize_rows_kernel(const uint16_t* __restrict__ x, const int32_t* __restrict__
 // 0..254 (0 for an all-zero block); each value v / X (exact: a power of two)
 // rounded to the nearest E2M1 value, ties to the even fraction bit, magnitudes
 // past 6 saturated. Codes are packed two per byte, element 2i in the low
-// nibble; the scales are stored per group of 128 rows, block-major
-// ([n / 128][b][n % 128]), so one k-block's scales for 128 rows are contiguous.
+// nibble, in tiles of 128 rows x 64 values (the GEMM's k-block): tile (n / 128,
+// k / 64) is 4096 contiguous bytes, row n % 128 at 32-byte pitch, so one
+// k-block's weights arrive as one contiguous copy. The scales are stored per
+// group of 128 rows, block-major ([n / 128][b][n % 128]), so one k-block's
+// scales for 128 rows are contiguous too.
 __global__ void __launch_bounds__(kThreads)
 mxfp4_quantize_kernel(const uint16_t* __restrict__ W, int N, int K, uint8_t* __restrict__ Wp,
                       uint8_t* __restrict__ Wsc)
@@ -141,7 +144,8 @@ mxfp4_quantize_kernel(const uint16_t* __restrict__ W, int N, int K, uint8_t* __r
         }
         out[q] = o;
     }
-    *reinterpret_cast<uint4*>(Wp + (size_t)n * (K / 2) + b * 16) = make_uint4(out[0], out[1], out[2], out[3]);
+    *reinterpret_cast<uint4*>(Wp + ((size_t)(n >> 7) * (K / 64) + (b >> 1)) * 4096 + (n & 127) * 32 + (b & 1) * 16) =
+        make_uint4(out[0], out[1], out[2], out[3]);
     Wsc[((size_t)(n >> 7) * nb + b) * 128 + (n & 127)] = (uint8_t)e;
 }
 

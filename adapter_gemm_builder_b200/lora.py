@@ -294,6 +294,11 @@ def w8a16_gemm_lora_epilogue(x: torch.Tensor, Wq: torch.Tensor, w_scale: torch.T
         ctypes.byref(seg.c) if seg else None, _ptr(y), _ptr(ws), ws.numel(), _stream(stream)))
 
 
+def mxfp4_code_bytes(N: int, K: int) -> int:
+    """Bytes of the packed E2M1 codes of an [N, K] MX FP4 weight (128 x 64 tiles)."""
+    return (N + 127) // 128 * 128 * (K // 2)
+
+
 def mxfp4_scale_bytes(N: int, K: int) -> int:
     """Bytes of the E8M0 scale array of an [N, K] MX FP4 weight (rows padded to 128)."""
     return (N + 127) // 128 * 128 * (K // 32)
@@ -307,9 +312,10 @@ def mxfp4_quantize_rows(W: torch.Tensor, Wp: torch.Tensor, Wsc: torch.Tensor, st
 def mxfp4_gemm_lora_epilogue(x: torch.Tensor, Wp: torch.Tensor, Wsc: torch.Tensor, pool: Pool | None,
                              seg: Segments | None, y: torch.Tensor, ws: torch.Tensor,
                              stream=None) -> None:
-    """y = x.W^T + s_a (x.A_a).B_a with W in MX FP4 (Wp [N, K/2], Wsc) and bf16 x."""
+    """y = x.W^T + s_a (x.A_a).B_a with W in MX FP4 (Wp, Wsc as mxfp4_quantize_rows makes
+    them; N = the weight's rows, read from y) and bf16 x."""
     M, K = x.shape
-    N = Wp.shape[0]
+    N = y.shape[1]
     _check(load().mxfp4_gemm_lora_epilogue(
         _ptr(x), M, K, N, _ptr(Wp), _ptr(Wsc), ctypes.byref(pool.c) if pool else None,
         ctypes.byref(seg.c) if seg else None, _ptr(y), _ptr(ws), ws.numel(), _stream(stream)))

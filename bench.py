@@ -867,7 +867,7 @@ def run_mxfp4(args, dev, stream, hbm_peak, bf16_peak, peak_src):
     K, N, n_ad, r = 8192, 28672, 16, 16
     gen = torch.Generator(device=dev).manual_seed(5)
     W = (torch.randn((N, K), generator=gen, device=dev) * (1.0 / math.sqrt(K))).to(torch.bfloat16)
-    Wp = torch.empty((N, K // 2), dtype=torch.uint8, device=dev)
+    Wp = torch.zeros(L.mxfp4_code_bytes(N, K), dtype=torch.uint8, device=dev)
     Wsc = torch.zeros(L.mxfp4_scale_bytes(N, K), dtype=torch.uint8, device=dev)
     L.mxfp4_quantize_rows(W, Wp, Wsc)
     del W

@@ -320,9 +320,13 @@ LORA_API int w8a16_gemm_lora_epilogue(const void* x, int M, int K, int N, const 
  * becomes the E2M1 code nearest to v / X (ties to the even fraction bit,
  * saturating at +-6). Finite weights only.
  *   W bf16 [N][K] (K % 64 == 0);
- *   Wp uint8 [N][K / 2]: two codes per byte, element 2i in the low nibble;
+ *   Wp uint8, ceil(N / 128) * 128 * K / 2 bytes: two codes per byte (element 2i
+ *   in the low nibble) in tiles of 128 rows x 64 values, tile (n / 128, k / 64)
+ *   at byte ((n / 128) * (K / 64) + k / 64) * 4096, row n % 128 at 32-byte
+ *   pitch (one k-block of 128 rows is one contiguous 4 KB copy for the GEMM);
  *   Wsc uint8 [ceil(N / 128)][K / 32][128]: the E8M0 scale of block b of row n
  *   at [n / 128][b][n % 128] (one k-block's scales of 128 rows are contiguous).
+ *   The padding rows of the last 128-row group are not written.
  * One kernel launch.
  */
 LORA_API int mxfp4_quantize_rows(const void* W, int N, int K, uint8_t* Wp, uint8_t* Wsc, lora_stream_t stream);
