@@ -62,7 +62,7 @@ bool gemm_split(int M, const lora_pool_t* pool)
 }
 
 size_t fp8_ws_layout(int M, int K, const lora_pool_t* pool, size_t* off_xq, size_t* off_sx,
-                     size_t* off_v, size_t* off_sync, size_t* off_part, int esz = 1, size_t* off_apply = nullptr)
+                     size_t* off_v, size_t* off_sync, size_t* off_part, int esz = 1)
 {
     size_t off = 256;  // status word block
     *off_xq = off;
@@ -75,8 +75,6 @@ size_t fp8_ws_layout(int M, int K, const lora_pool_t* pool, size_t* off_xq, size
     off += align256((size_t)(16 + device_sm_count()) * 4);
     *off_part = off;
     off += align256(fp8_gemm_partial_bytes(M));
-    if (off_apply) *off_apply = off;
-    if (gemm_split(M, pool)) off += align256(sgmv_warp_workspace_bytes(M, *pool));
     return off;
 }
 
@@ -135,9 +133,9 @@ int gemm_lora_launch(int esz, const void* x, int M, int K, int N, const uint8_t*
                      const lora_pool_t* pool, const lora_segments_t* seg, void* y, void* ws,
                      size_t ws_bytes, lora_stream_t stream, const uint8_t* wsc = nullptr, bool w_e4m3 = false)
 {
-    size_t off_xq, off_sx, off_v, off_sync, off_part, off_apply;
+    size_t off_xq, off_sx, off_v, off_sync, off_part;
     const size_t need =
-        fp8_ws_layout(M, K, pool, &off_xq, &off_sx, &off_v, &off_sync, &off_part, esz, &off_apply);
+        fp8_ws_layout(M, K, pool, &off_xq, &off_sx, &off_v, &off_sync, &off_part, esz);
     if (!ws || ws_bytes < need || !aligned16(ws)) return LORA_ERR_WORKSPACE;
     const bool split = gemm_split(M, pool);
     const lora_pool_t* fused = split ? nullptr : pool;  // the adapters folded into the GEMM
@@ -192,14 +190,7 @@ int gemm_lora_launch(int esz, const void* x, int M, int K, int N, const uint8_t*
     e = launch_fp8_gemm(a, s);
     if (e != cudaSuccess || !split) return cuda_status(e);
     // 3. many adapters: their term added to the GEMM's bf16 output by the SGMV apply
-    //    (the kernel lora_apply picks for this batch)
-    if (tile_tokens_for(M, pool->n_adapters) <= LORA_DECODE_TILE_TOKENS)
-        return cuda_status(launch_sgmv(SGMV_APPLY, x, 0, *pool, *seg, nullptr, y, s, false));
-    void* wa = w + off_apply;
-    if (sgmv_warp_zero(*pool, *seg, wa, s) != cudaSuccess ||
-        launch_sgmv(SGMV_APPLY, x, 0, *pool, *seg, nullptr, y, s, false, kWarpSmallTile) != cudaSuccess)
-        return LORA_ERR_CUDA;
-    return cuda_status(launch_sgmv_warp(x, 0, *pool, *seg, y, wa, s));
+    return cuda_status(launch_sgmv(SGMV_APPLY, x, 0, *pool, *seg, nullptr, y, s, false));
 }
 
 }  // namespace
@@ -274,10 +265,9 @@ size_t lora_workspace_size(int op, int T, int K, const lora_pool_t* pool)
     case LORA_OP_SHRINK:
     case LORA_OP_EXPAND: return 0;
     case LORA_OP_APPLY:
-        // decode-like batches need none; the others, the streaming kernel's counters and v
+        // v stays on chip (exchanged inside each thread-block cluster): no workspace
         if (!pool || check_pool(pool) != LORA_OK) return (size_t)-1;
-        if (T == 0 || tile_tokens_for(T, pool->n_adapters) <= LORA_DECODE_TILE_TOKENS) return 0;
-        return sgmv_warp_workspace_bytes(T, *pool);
+        return 0;
     case LORA_OP_FP8_BACKWARD: {
         if (!pool || check_pool(pool) != LORA_OK || T < 1) return (size_t)-1;
         size_t a, b, c, d;
@@ -392,18 +382,10 @@ int lora_apply(const void* x, int64_t x_slice_stride, const lora_pool_t* pool,
     if ((st = check_x(x, x_slice_stride, pool, seg->T)) != LORA_OK) return st;
     if (!y || !aligned16(y)) return LORA_ERR_INVALID_ARG;
     cudaStream_t s = (cudaStream_t)stream;
-    if (tile_tokens_for(seg->T, pool->n_adapters) <= LORA_DECODE_TILE_TOKENS)
-        // a decode-like batch: one tile per thread-block cluster, v exchanged on chip
-        return cuda_status(launch_sgmv(SGMV_APPLY, x, x_slice_stride, *pool, *seg, nullptr, y, s, false));
-    const size_t need = sgmv_warp_workspace_bytes(seg->T, *pool);
-    if (!ws || ws_bytes < need || !aligned16(ws)) return LORA_ERR_WORKSPACE;
-    // the warp kernel's counters are zeroed first; then the tile rows of more than
-    // kWarpSmallTile tokens on the cluster kernel, and alongside it the small ones
-    // on the warp kernel (two launches)
-    if (sgmv_warp_zero(*pool, *seg, ws, s) != cudaSuccess ||
-        launch_sgmv(SGMV_APPLY, x, x_slice_stride, *pool, *seg, nullptr, y, s, false, kWarpSmallTile) != cudaSuccess)
-        return LORA_ERR_CUDA;
-    return cuda_status(launch_sgmv_warp(x, x_slice_stride, *pool, *seg, y, ws, s));
+    // one tile row per thread-block cluster, v exchanged on chip (ws is not used)
+    (void)ws;
+    (void)ws_bytes;
+    return cuda_status(launch_sgmv(SGMV_APPLY, x, x_slice_stride, *pool, *seg, nullptr, y, s, false));
 }
 
 int fp8_quantize_rows(const void* x, int M, int K, uint8_t* xq, float* sx, lora_stream_t stream)

@@ -56,7 +56,7 @@ constexpr int kBlockM = 128;  // W rows per tile (MMA M)
 constexpr int kEpiWarps = 8;
 constexpr int kEpiThreads = kEpiWarps * 32;
 constexpr int kThreads = (3 + kEpiWarps) * 32;
-constexpr int kCvtWarps = 4;                      // MX FP4 weights: converter warps (one row each lane)
+constexpr int kCvtWarps = 8;                      // weight converter warps: half a W row per lane
 constexpr int kThreadsW4 = (3 + kEpiWarps + kCvtWarps) * 32;
 constexpr int kPackStage = 5120;                  // packed E2M1 tile (128 x 32 B) + scales (2 x 128 B), 1 KB aligned
 constexpr int kCodeStage = 8192;                  // E4M3 tile of the 8-bit weights under bf16 activations (128 x 64 B)
@@ -64,6 +64,11 @@ constexpr int kCodeStage = 8192;                  // E4M3 tile of the 8-bit weig
 // codes with E8M0 block scales, E4M3 codes with a per-channel scale (W8A16).
 enum { kWcNone = 0, kWcMxfp4 = 1, kWcE4m3 = 2 };
 __host__ __device__ constexpr int wc_stage_bytes(int wc) { return wc == 1 ? kPackStage : (wc == 2 ? kCodeStage : 0); }
+// MX FP4: the byte-permute tables of all 256 block scales (uint4 each), built once per CTA
+constexpr int kE2m1TabBytes = 256 * 16;
+// W8A16: the converter writes each E4M3 weight as bf16 times 2^-112 (the exponent of its
+// exact f16 form read as a bf16 exponent), and the per-channel scale carries the 2^112
+__host__ __device__ constexpr float e4m3_bf16_shift() { return 5.192296858534828e33f; }  // 2^112
 constexpr int kMaxStages = 8;
 constexpr int kShrinkCols = 64;  // K columns of the down-projection per work item
 constexpr int kShrinkTok = 64;   // tokens of the down-projection per work item
@@ -100,7 +105,7 @@ struct GemmParams {
     const float* scales;
     int n_adapters, r_max, r8, r16;
     int n_slots;
-    uint32_t ring_off, slots_off, v_off, meta_off, bar_off;
+    uint32_t ring_off, slots_off, v_off, meta_off, bar_off, tab_off;
     unsigned long long timeout_ns;  // limit of every bounded wait (2 s unless a test lowers it)
     int inject_stall;  // test hook: CTA 0's producer first waits on a barrier nothing completes
 };
@@ -252,6 +257,18 @@ __device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint16_t c2)
     return r;
 }
 
+// Four E4M3 codes (byte i the i-th) -> four bf16 equal to the codes' values times
+// 2^-112: each pair goes to f16 (exact; every E4M3 value, subnormals included, is a
+// normal f16 or zero), whose exponent and top mantissa bits, shifted into bf16
+// position, read as value * 2^(15 - 127) (E4M3 has 3 mantissa bits, so none is lost).
+__device__ __forceinline__ uint2 e4m3x4_to_bf16_shifted(uint32_t w)
+{
+    uint32_t h0, h1;
+    asm("{\n.reg .b16 lo, hi;\nmov.b32 {lo, hi}, %2;\ncvt.rn.f16x2.e4m3x2 %0, lo;\ncvt.rn.f16x2.e4m3x2 %1, hi;\n}"
+        : "=r"(h0), "=r"(h1) : "r"(w));
+    return make_uint2(((h0 >> 3) & 0x0fff0fffu) | (h0 & 0x80008000u), ((h1 >> 3) & 0x0fff0fffu) | (h1 & 0x80008000u));
+}
+
 // Stream-K schedule: CTA c owns units [c*U/G, (c+1)*U/G) of the (tile,
 // k-block) sequence; a segment is the part of one tile inside that range.
 struct Seg {
@@ -312,6 +329,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
 
     constexpr int kStageW = kBlockM * BK;
     const int stage_bytes = kStageW + p.BN * BK + wc_stage_bytes(kW4);
+    constexpr float kWShift = kW4 == kWcE4m3 ? e4m3_bf16_shift() : 1.f;  // see e4m3x4_to_bf16_shifted
     const uint32_t ncols = (uint32_t)(2 * p.BN <= 32 ? 32 : (2 * p.BN <= 64 ? 64 : (2 * p.BN <= 128 ? 128 : (2 * p.BN <= 256 ? 256 : 512))));
     const int G = gridDim.x, cta = blockIdx.x, KB = p.k_blocks;
     const long long u_begin = unit_begin(p.units, cta, G), u_end = unit_begin(p.units, cta + 1, G);
@@ -908,7 +926,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
                 // B'[n][j] = B_a[j][n] / sw[n] in place, K-major, for the phase's slots: each
                 // thread reads its row n of kSpt slots, then (after a barrier) writes them
                 const int nn = etid & 127, half = etid >> 7;
-                const float inv_sw2 = (nb * kBlockM + nn < p.N) ? (p.sw ? 1.f / p.sw[nb * kBlockM + nn] : 1.f) : 0.f;
+                const float inv_sw2 = (nb * kBlockM + nn < p.N) ? 1.f / ((p.sw ? p.sw[nb * kBlockM + nn] : 1.f) * kWShift) : 0.f;
                 const int nbuf = e1 - e0;
                 constexpr int kSpt = MAXR <= 16 ? 4 : (MAXR <= 32 ? 2 : 1);
                 for (int b0 = 0; b0 < nbuf && ok; b0 += 2 * kSpt) {
@@ -962,7 +980,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
             }
 
             const int n = nb * kBlockM + n_local;
-            const float swn = n < p.N ? (p.sw ? p.sw[n] : 1.f) : 0.f;
+            const float swn = n < p.N ? (p.sw ? p.sw[n] : 1.f) * kWShift : 0.f;
 
             // partial sums of the later k-blocks for 16 columns (zero when nobody else has any);
             // the next chunk's are loaded while this one is processed
@@ -1089,10 +1107,22 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
     if constexpr (kW4 != kWcNone) {
         if (warp >= 3 + kEpiWarps) {
             // ------------------------------------------------------------ converter warps
-            // thread = one W row of the tile: its 64 codes of the k-block (32 packed bytes)
-            // and its two block scales become 64 bf16 values in the 128-byte swizzled row
-            // the MMA descriptor expects
-            const int row = (warp - 3 - kEpiWarps) * 32 + lane;
+            // thread = half of one W row of the tile: its 32 codes of the k-block (and, for
+            // MX FP4, their block scale) become 32 bf16 values, four 16-byte chunks of the
+            // 128-byte swizzled row the MMA descriptor expects
+            constexpr int kCvtThreads = kCvtWarps * 32;
+            static_assert(kCvtThreads == 128 || kCvtThreads == 256, "a thread converts one or two half rows");
+            const int ct = (warp - 3 - kEpiWarps) * 32 + lane;
+            const int row = ct & 127;
+            const uint4* tab = reinterpret_cast<const uint4*>(smem + p.tab_off);
+            if constexpr (kW4 == kWcMxfp4) {
+                for (int e = ct; e < 256; e += kCvtThreads) {
+                    uint32_t lo0, lo1, hi0, hi1;
+                    e2m1_tables((uint32_t)e, lo0, lo1, hi0, hi1);
+                    *reinterpret_cast<uint4*>(smem + p.tab_off + e * 16) = make_uint4(lo0, lo1, hi0, hi1);
+                }
+                ptx::named_sync(1, kCvtThreads);  // the table is complete
+            }
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
@@ -1112,35 +1142,27 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
                     const uint8_t* pk = st_base + kStageW + p.BN * BK;
                     uint8_t* dst = st_base + row * 128;
                     const int sw = row & 7;
-                    if constexpr (kW4 == kWcE4m3) {
-                        // 64 E4M3 codes -> bf16 (exact: E4M3 -> f16 -> f32 -> bf16)
 #pragma unroll
-                        for (int h = 0; h < 4; ++h) {
-                            const uint4 q = *reinterpret_cast<const uint4*>(pk + row * 64 + h * 16);
-                            const uint32_t w4[4] = {q.x, q.y, q.z, q.w};
-                            uint32_t o[8];
+                    for (int half = ct >> 7; half < 2; half += kCvtThreads / 128) {
+                        const int c0 = 4 * half;
+                        if constexpr (kW4 == kWcE4m3) {
+                            // 32 E4M3 codes -> bf16 times 2^-112 (exact)
 #pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                o[2 * e] = e4m3x2_to_bf16x2((uint16_t)(w4[e] & 0xffffu));
-                                o[2 * e + 1] = e4m3x2_to_bf16x2((uint16_t)(w4[e] >> 16));
+                            for (int h = 0; h < 2; ++h) {
+                                const uint4 q = *reinterpret_cast<const uint4*>(pk + row * 64 + half * 32 + h * 16);
+                                const uint2 a = e4m3x4_to_bf16_shifted(q.x), b = e4m3x4_to_bf16_shifted(q.y);
+                                const uint2 c = e4m3x4_to_bf16_shifted(q.z), d = e4m3x4_to_bf16_shifted(q.w);
+                                *reinterpret_cast<uint4*>(dst + (((c0 + 2 * h) ^ sw) << 4)) = make_uint4(a.x, a.y, b.x, b.y);
+                                *reinterpret_cast<uint4*>(dst + (((c0 + 2 * h + 1) ^ sw) << 4)) = make_uint4(c.x, c.y, d.x, d.y);
                             }
-                            *reinterpret_cast<uint4*>(dst + (((2 * h) ^ sw) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
-                            *reinterpret_cast<uint4*>(dst + (((2 * h + 1) ^ sw) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
+                        } else {
+                            const uint4 q = *reinterpret_cast<const uint4*>(pk + row * 32 + half * 16);
+                            const uint4 t = tab[pk[4096 + half * 128 + row]];
+                            *reinterpret_cast<uint4*>(dst + (((c0 + 0) ^ sw) << 4)) = e2m1x8_to_bf16(q.x, t.x, t.y, t.z, t.w);
+                            *reinterpret_cast<uint4*>(dst + (((c0 + 1) ^ sw) << 4)) = e2m1x8_to_bf16(q.y, t.x, t.y, t.z, t.w);
+                            *reinterpret_cast<uint4*>(dst + (((c0 + 2) ^ sw) << 4)) = e2m1x8_to_bf16(q.z, t.x, t.y, t.z, t.w);
+                            *reinterpret_cast<uint4*>(dst + (((c0 + 3) ^ sw) << 4)) = e2m1x8_to_bf16(q.w, t.x, t.y, t.z, t.w);
                         }
-                    } else {
-                    const uint4 q0 = *reinterpret_cast<const uint4*>(pk + row * 32);
-                    const uint4 q1 = *reinterpret_cast<const uint4*>(pk + row * 32 + 16);
-                    uint32_t lo0, lo1, hi0, hi1;
-                    e2m1_tables(pk[4096 + row], lo0, lo1, hi0, hi1);
-                    *reinterpret_cast<uint4*>(dst + ((0 ^ sw) << 4)) = e2m1x8_to_bf16(q0.x, lo0, lo1, hi0, hi1);
-                    *reinterpret_cast<uint4*>(dst + ((1 ^ sw) << 4)) = e2m1x8_to_bf16(q0.y, lo0, lo1, hi0, hi1);
-                    *reinterpret_cast<uint4*>(dst + ((2 ^ sw) << 4)) = e2m1x8_to_bf16(q0.z, lo0, lo1, hi0, hi1);
-                    *reinterpret_cast<uint4*>(dst + ((3 ^ sw) << 4)) = e2m1x8_to_bf16(q0.w, lo0, lo1, hi0, hi1);
-                    e2m1_tables(pk[4096 + 128 + row], lo0, lo1, hi0, hi1);
-                    *reinterpret_cast<uint4*>(dst + ((4 ^ sw) << 4)) = e2m1x8_to_bf16(q1.x, lo0, lo1, hi0, hi1);
-                    *reinterpret_cast<uint4*>(dst + ((5 ^ sw) << 4)) = e2m1x8_to_bf16(q1.y, lo0, lo1, hi0, hi1);
-                    *reinterpret_cast<uint4*>(dst + ((6 ^ sw) << 4)) = e2m1x8_to_bf16(q1.z, lo0, lo1, hi0, hi1);
-                    *reinterpret_cast<uint4*>(dst + ((7 ^ sw) << 4)) = e2m1x8_to_bf16(q1.w, lo0, lo1, hi0, hi1);
                     }
                     ptx::fence_proxy_async_smem();  // generic writes, read by the tensor core
                     __syncwarp();
@@ -1294,7 +1316,8 @@ cudaError_t launch_fp8_gemm(const Fp8GemmArgs& a, cudaStream_t stream)
     auto fit = [&](int bk, int va, int ns) -> int {
         if (w4 && bk != 128) return 0;  // the converter writes 128-byte rows
         const size_t stage_bytes = (size_t)kBlockM * bk + (size_t)p.BN * bk + wc_stage_bytes(wc);
-        const size_t fixed = 1024 + meta + vq_bytes(va) + bars + (size_t)ns * slot_bytes;
+        const size_t fixed = 1024 + meta + vq_bytes(va) + bars + (size_t)ns * slot_bytes +
+                             (wc == kWcMxfp4 ? (size_t)kE2m1TabBytes + 16 : 0);
         if (fixed >= kSmemMax) return 0;
         const size_t st = (kSmemMax - fixed) / stage_bytes;
         return (int)(st > (size_t)kMaxStages ? kMaxStages : st);
@@ -1348,7 +1371,8 @@ cudaError_t launch_fp8_gemm(const Fp8GemmArgs& a, cudaStream_t stream)
     p.v_off = (uint32_t)align_up(p.slots_off + (size_t)ns * slot_bytes, 128);
     p.meta_off = (uint32_t)(p.v_off + vq_bytes(va));
     p.bar_off = (uint32_t)align_up(p.meta_off + meta, 8);
-    const size_t smem = align_up(p.bar_off + bars, 128) + 1024;  // + alignment slack
+    p.tab_off = (uint32_t)align_up(p.bar_off + bars, 16);
+    const size_t smem = align_up(p.tab_off + (wc == kWcMxfp4 ? (size_t)kE2m1TabBytes : 0), 128) + 1024;  // + alignment slack
 
     CUtensorMap tmW, tmX, tmB;
     const CUtensorMapSwizzle swz = BK == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;

@@ -16,21 +16,10 @@ cudaError_t launch_build_segments(const int32_t* ids, int T, int n_adapters,
 
 enum SgmvMode { SGMV_SHRINK = 0, SGMV_EXPAND = 1, SGMV_APPLY = 2 };
 
-// x, v, y may be NULL where the mode does not use them. Tile rows of at most
-// skip_small tokens are left alone (the warp kernel takes them).
+// x, v, y may be NULL where the mode does not use them.
 cudaError_t launch_sgmv(int mode, const void* x, int64_t x_slice_stride, const lora_pool_t& pool,
                         const lora_segments_t& seg, float* v, void* y, cudaStream_t stream,
-                        bool pdl_trigger, int skip_small = 0);
-
-// The fused shrink + expand of the tile rows of at most kWarpSmallTile tokens
-// (sgmv_warp.cu): one warp per work item, two launches; ws holds
-// sgmv_warp_workspace_bytes(T, pool) bytes, zeroed by sgmv_warp_zero first.
-constexpr int kWarpSmallTile = 8;
-cudaError_t sgmv_warp_zero(const lora_pool_t& pool, const lora_segments_t& seg, void* ws, cudaStream_t stream);
-cudaError_t launch_sgmv_warp(const void* x, int64_t x_slice_stride, const lora_pool_t& pool,
-                             const lora_segments_t& seg, void* y, void* ws, cudaStream_t stream);
-size_t sgmv_warp_workspace_bytes(int T, const lora_pool_t& pool);
-
+                        bool pdl_trigger);
 
 // Token-wise merge of the selected adapters into the backbone (merge.cu).
 cudaError_t launch_lora_switch_merge(const void* W, int N, int K, const lora_pool_t& pool, const int32_t* sel,

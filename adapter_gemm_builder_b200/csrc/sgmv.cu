@@ -80,7 +80,6 @@ struct SgmvParams {
     int rp;          // round_up(r_max, 16): row pitch (floats) of the v buffers
     int stage_bytes; // one ring stage
     int xy_maps;     // tensor maps of x and y are valid (consecutive-row tiles use them)
-    int skip_small;  // tile rows of at most this many tokens belong to the warp kernel
     uint32_t off_rb, off_vf, off_bar;
     unsigned long long timeout_ns;  // limit of every bounded wait (2 s unless a test lowers it)
     int inject_stall;  // test hook: one CTA's producer first waits on a barrier nothing completes
@@ -139,7 +138,7 @@ sgmv_kernel(const __grid_constant__ AMaps am, const SgmvParams p)
 
     const int4 tl = p.tiles[g];
     const int nt = tl.z;
-    if (nt <= 0 || nt <= p.skip_small) return;  // unused row, or the warp kernel's: the cluster leaves together
+    if (nt <= 0) return;  // unused row: the cluster leaves together
     const int a = tl.x, tok0 = tl.y;
     int r = p.ranks ? p.ranks[a] : p.r_max;
     r = max(1, min(r, p.r_max));
@@ -796,7 +795,7 @@ size_t sgmv_smem_per_cta()
 
 cudaError_t launch_sgmv(int mode, const void* x, int64_t x_slice_stride, const lora_pool_t& pool,
                         const lora_segments_t& seg, float* v, void* y, cudaStream_t stream,
-                        bool pdl_trigger, int skip_small)
+                        bool pdl_trigger)
 {
     (void)pdl_trigger;
     if (seg.T == 0) return cudaSuccess;
@@ -819,7 +818,6 @@ cudaError_t launch_sgmv(int mode, const void* x, int64_t x_slice_stride, const l
     p.r_max = pool.r_max;
     p.timeout_ns = debug_wait_limit_ns();
     p.inject_stall = debug_inject_stall();
-    p.skip_small = skip_small;
     // CTAs per tile: up to one per 512 columns of h_in (at most 8). When that would
     // need more than one wave of two CTAs per SM but the tile rows alone fit in one,
     // take as many per tile as keep one wave (no near-empty last wave: prefill gets 5);

@@ -248,7 +248,7 @@ def lora_expand(v: torch.Tensor, pool: Pool, seg: Segments, y: torch.Tensor, str
 def lora_apply(x: torch.Tensor, pool: Pool, seg: Segments, y: torch.Tensor, stream=None,
                x_slice_stride: int | None = None, ws: torch.Tensor | None = None) -> None:
     """y += s_a (x.A_a).B_a; ws: a workspace of lora_workspace_size(LORA_OP_APPLY, T, 0, pool)
-    bytes (allocated here when None; pass one to keep the call free of allocation)."""
+    bytes (none today: v stays on chip; allocated here when None and the size is not 0)."""
     xs = _slice_stride(x, pool) if x_slice_stride is None else x_slice_stride
     if ws is None:
         n = lora_workspace_size(LORA_OP_APPLY, seg.T, 0, pool)

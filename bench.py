@@ -68,7 +68,7 @@ def parse_args():
     ap.add_argument("--fp8-reps", type=int, default=20, help="graph replays per timing")
     ap.add_argument("--no-bf16", action="store_true", help="skip the bf16 GEMM + LoRA section")
     ap.add_argument("--no-merge", action="store_true", help="skip the adapter-merge section")
-    ap.add_argument("--no-mxfp4", action="store_true", help="skip the MX FP4 GEMM + LoRA section")
+    ap.add_argument("--no-mxfp4", action="store_true", help="skip the MX FP4 and W8A16 GEMM + LoRA sections")
     return ap.parse_args()
 
 
@@ -338,11 +338,8 @@ class _Events:
 
 
 def apply_launches(p):
-    """Kernels of this library one lora_apply launches: one for a decode-like batch
-    (T <= 64 and T <= 2 n_adapters); otherwise the cluster kernel for the larger tiles
-    and the warp kernel's two launches for the small ones (plus a memset of its
-    counters, not counted)."""
-    return 1 if (p.T <= 64 and p.T <= 2 * p.n_adapters) else 3
+    """Kernels of this library one lora_apply launches: one (the cluster kernel)."""
+    return 1
 
 
 def time_apply(p, dev, steps, warmup, stream, ext, world=1, clocks=None):
@@ -525,6 +522,7 @@ def run_ours(args):
     bf16 = None if args.no_bf16 else run_bf16(args, dev, stream, hbm_peak, bf16_peak, peak_src)
     merge = None if args.no_merge else run_merge(args, dev, stream, hbm_peak, peak_src)
     mxfp4 = None if args.no_mxfp4 else run_mxfp4(args, dev, stream, hbm_peak, bf16_peak, peak_src)
+    w8a16 = None if args.no_mxfp4 else run_mxfp4(args, dev, stream, hbm_peak, bf16_peak, peak_src, "w8a16")
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -540,7 +538,7 @@ def run_ours(args):
             "roofline": roofline, "e2e": e2e, "gpu_launches": (1 + apply_launches(p)) * K,
             "clocks": t["clocks"], "status_ok": t["status_ok"],
             "cpu_baseline": cpu, "workloads": extras, "fp8_gemm_lora": fp8, "bf16_gemm_lora": bf16,
-            "switch_merge": merge, "mxfp4_gemm_lora": mxfp4,
+            "switch_merge": merge, "mxfp4_gemm_lora": mxfp4, "w8a16_gemm_lora": w8a16,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -853,12 +851,13 @@ def run_bf16(args, dev, stream, hbm_peak, bf16_peak, peak_src):
     return out
 
 
-def run_mxfp4(args, dev, stream, hbm_peak, bf16_peak, peak_src):
-    """The 4-bit base (OCP MX FP4 weights, bf16 activations) with the fused LoRA term at
-    the FP8 section's decode shapes (K 8192, N 28672, 16 adapters of rank 16, Zipf ids),
-    against the same call without LoRA: us per call, TFLOP/s against the bf16 peak (its
-    MMAs are kind::f16) and the HBM fraction of its algorithmic bytes (packed codes,
-    scales, x, y and the adapters present)."""
+def run_mxfp4(args, dev, stream, hbm_peak, bf16_peak, peak_src, fmt="mxfp4"):
+    """A low-bit weight base with bf16 activations and the fused LoRA term at the FP8
+    section's decode shapes (K 8192, N 28672, 16 adapters of rank 16, Zipf ids), against
+    the same call without LoRA: us per call, TFLOP/s against the bf16 peak (its MMAs are
+    kind::f16) and the HBM fraction of its algorithmic bytes (weight codes and scales, x,
+    y and the adapters present). fmt "mxfp4": OCP MX FP4 weights; "w8a16": E4M3 weights
+    with one fp32 scale per output channel."""
     import numpy as np
     import torch
 
@@ -867,9 +866,18 @@ def run_mxfp4(args, dev, stream, hbm_peak, bf16_peak, peak_src):
     K, N, n_ad, r = 8192, 28672, 16, 16
     gen = torch.Generator(device=dev).manual_seed(5)
     W = (torch.randn((N, K), generator=gen, device=dev) * (1.0 / math.sqrt(K))).to(torch.bfloat16)
-    Wp = torch.zeros(L.mxfp4_code_bytes(N, K), dtype=torch.uint8, device=dev)
-    Wsc = torch.zeros(L.mxfp4_scale_bytes(N, K), dtype=torch.uint8, device=dev)
-    L.mxfp4_quantize_rows(W, Wp, Wsc)
+    if fmt == "mxfp4":
+        Wp = torch.zeros(L.mxfp4_code_bytes(N, K), dtype=torch.uint8, device=dev)
+        Wsc = torch.zeros(L.mxfp4_scale_bytes(N, K), dtype=torch.uint8, device=dev)
+        L.mxfp4_quantize_rows(W, Wp, Wsc)
+        w_bytes = N * K // 2 + L.mxfp4_scale_bytes(N, K)
+        op = L.LORA_OP_MXFP4_GEMM
+    else:
+        Wp = torch.empty((N, K), dtype=torch.uint8, device=dev)
+        Wsc = torch.empty((N,), dtype=torch.float32, device=dev)
+        L.fp8_quantize_rows(W, Wp, Wsc)
+        w_bytes = N * K + N * 4
+        op = L.LORA_OP_W8A16_GEMM
     del W
     out = {"shape": {"K": K, "N": N, "adapters": n_ad, "r": r, "ids": "zipf(1.1)"},
            "peak_tflops_bf16": bf16_peak, "peak_hbm_gbs": hbm_peak,
@@ -889,16 +897,18 @@ def run_mxfp4(args, dev, stream, hbm_peak, bf16_peak, peak_src):
             d["seg"] = L.Segments(M, n_ad, device=dev)
             L.lora_build_segments(d["ids"], n_ad, d["seg"])
             d["y"] = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
-            d["ws"] = L.workspace(L.LORA_OP_MXFP4_GEMM, M, K, d["pool"], device=dev)
-            d["ws0"] = L.workspace(L.LORA_OP_MXFP4_GEMM, M, K, None, device=dev)
+            d["ws"] = L.workspace(op, M, K, d["pool"], device=dev)
+            d["ws0"] = L.workspace(op, M, K, None, device=dev)
             sets.append(d)
         res = {}
         for tag in ("lora", "base"):
+            fn = L.mxfp4_gemm_lora_epilogue if fmt == "mxfp4" else L.w8a16_gemm_lora_epilogue
+
             def call(d):
                 if tag == "lora":
-                    L.mxfp4_gemm_lora_epilogue(d["x"], Wp, Wsc, d["pool"], d["seg"], d["y"], d["ws"])
+                    fn(d["x"], Wp, Wsc, d["pool"], d["seg"], d["y"], d["ws"])
                 else:
-                    L.mxfp4_gemm_lora_epilogue(d["x"], Wp, Wsc, None, None, d["y"], d["ws0"])
+                    fn(d["x"], Wp, Wsc, None, None, d["y"], d["ws0"])
             with torch.cuda.stream(stream):
                 for d in sets:
                     call(d)
@@ -919,7 +929,7 @@ def run_mxfp4(args, dev, stream, hbm_peak, bf16_peak, peak_src):
             res[tag + "_status"] = max(L.lora_workspace_status(d["ws" if tag == "lora" else "ws0"])[0]
                                        for d in sets)
         lora_bytes = int(len(act)) * r * (K + N) * 2 + M * r * 4
-        bytes_call = N * K // 2 + L.mxfp4_scale_bytes(N, K) + M * K * 2 + M * N * 2 + lora_bytes
+        bytes_call = w_bytes + M * K * 2 + M * N * 2 + lora_bytes
         flops = 2.0 * M * N * K
         t = res["lora"] * 1e-6
         out["M"][str(M)] = {
@@ -928,7 +938,7 @@ def run_mxfp4(args, dev, stream, hbm_peak, bf16_peak, peak_src):
             "tflops": flops / t / 1e12, "tensor_frac": flops / t / 1e12 / bf16_peak,
             "hbm_gbs": bytes_call / t / 1e9, "hbm_frac": bytes_call / t / 1e9 / hbm_peak,
             "status_ok": res["lora_status"] == 0 and res["base_status"] == 0,
-            "l2": f"x, adapters and y rotate over {R} copies; the packed weight is read once per call",
+            "l2": f"x, adapters and y rotate over {R} copies; the weight codes are read once per call",
         }
         del sets
     return out

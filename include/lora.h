@@ -152,8 +152,8 @@ LORA_API int lora_segments_status(const lora_segments_t* seg, lora_stream_t stre
  * Bytes of workspace an operation needs (0 if it needs none), or (size_t)-1
  * for invalid arguments. For LORA_OP_FP8_GEMM, T is the
  * token count M and `K` the GEMM's reduction size; `pool` may be NULL (no
- * LoRA). LORA_OP_APPLY needs the pool (its counters and v scale with the
- * slices, the tiles and r_max). The other operations ignore K.
+ * LoRA). LORA_OP_APPLY needs a valid pool and returns 0 (v stays on chip).
+ * The other operations ignore K.
  * A workspace must be zeroed once after allocation (lora_workspace_init);
  * afterwards the library keeps it in a reusable state.
  */
@@ -217,12 +217,10 @@ LORA_API int lora_expand(const float* v, const lora_pool_t* pool, const lora_seg
  * Shrink then expand (y += s_a * (x.A_a).B_a; the whole added term of the
  * Punica README, "How?", for a batch of many adapters), v in fp32. Arguments
  * as lora_shrink / lora_expand, plus a workspace of
- * lora_workspace_size(LORA_OP_APPLY, T, 0, pool) bytes (none for a
- * decode-like batch, see lora_tile_tokens_for). A decode-like batch runs one
- * kernel whose thread-block clusters each take one tile and keep v on chip;
- * any other batch runs a memset of the workspace's counters and one
- * persistent kernel that streams shrink and expand parts of every tile,
- * passing v through the workspace.
+ * lora_workspace_size(LORA_OP_APPLY, T, 0, pool) bytes (0 today; ws may be
+ * NULL). One kernel launch: each thread-block cluster takes one tile row
+ * (lora_tile_tokens_for) and keeps its v on chip, the partial v of its CTAs
+ * exchanged through distributed shared memory.
  */
 LORA_API int lora_apply(const void* x, int64_t x_slice_stride, const lora_pool_t* pool,
                const lora_segments_t* seg, void* y, void* ws, size_t ws_bytes,
@@ -257,8 +255,8 @@ LORA_API int fp8_quantize_rows(const void* x, int M, int K, uint8_t* xq, float* 
  * Limits: K % 16 == 0, N % 8 == 0, M >= 1.
  * Many adapters: when the pool holds more than 16 adapters and M > 16, the
  * adapters' term is not folded into the GEMM's accumulator; the call runs the
- * base GEMM and then the SGMV apply of lora_apply on its output (three or four
- * launches, the workspace covering both), so y = bf16(bf16(base) + term).
+ * base GEMM and then the SGMV apply of lora_apply on its output (three
+ * launches), so y = bf16(bf16(base) + term).
  * The GEMM is a persistent grid of one CTA per SM whose CTAs wait on one
  * another (the down-projection count, stream-K partials), so all of them must
  * be resident at once: the context needs every SM of the device. Where fewer

@@ -188,3 +188,58 @@ def test_w8a16_gemm_lora_full_grid(M, K, N, n_ad, lora):
     ka = dict(A=p.A, B=p.B, ranks=p.ranks, scales=p.scales, ids=p.ids) if lora else {}
     want = oracle.w8a16_gemm_lora_sampled(p.x, Wq, sw, rows, cols, **ka).reshape(M, N)
     assert_close(f64(host_bf16_bits(y)), want, TOL_FP8, f"w8a16 M{M} K{K} N{N} lora={lora}")
+
+
+def test_w8a16_gemm_small_integers_exact():
+    """Integer weights that E4M3 holds exactly, power-of-two channel scales and activations
+    in -2..2: every product and partial sum is exact in fp32, so y must equal the oracle
+    rounded once to bf16."""
+    rng = np.random.default_rng(43)
+    M, K, N = 24, 192, 136
+    x = wl.to_bf16_bits(rng.integers(-2, 3, (M, K)).astype(np.float32))
+    ints = rng.integers(-4, 5, (N, K))
+    Wq = np.vectorize(oracle.e4m3_encode)(ints.astype(np.float64)).astype(np.uint8)
+    sw = np.float32(2.0) ** rng.integers(-2, 3, N).astype(np.float32)
+    ws = L.workspace(L.LORA_OP_W8A16_GEMM, M, K, None)
+    y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+    L.w8a16_gemm_lora_epilogue(dev_bf16(x), dev(Wq), dev(sw), None, None, y, ws)
+    torch.cuda.synchronize()
+    assert L.lora_workspace_status(ws)[0] == L.LORA_OK
+    rows = np.repeat(np.arange(M), N).astype(np.int32)
+    cols = np.tile(np.arange(N), M).astype(np.int32)
+    want = oracle.w8a16_gemm_lora_sampled(x, Wq, sw, rows, cols).reshape(M, N)
+    assert np.array_equal(host_bf16_bits(y), rne_bf16_bits(want))
+
+
+def test_w8a16_gemm_lora_decode_shape_sampled():
+    """K 8192, N 28672, M 16, 16 adapters of rank 16, Zipf ids; the weight quantised by
+    the library (its sampled rows checked bit-exact against the oracle's quantiser)."""
+    M, K, N = 16, 8192, 28672
+    W = wl.weight_bf16(N, K, seed=3 + 7000)
+    Wq = torch.empty((N, K), dtype=torch.uint8, device="cuda")
+    sw = torch.empty((N,), dtype=torch.float32, device="cuda")
+    L.fp8_quantize_rows(dev_bf16(W), Wq, sw)
+    p = wl.fp8_problem(M, K=K, N=N, n_adapters=16, r=16, seed=3, none_frac=0.0, W=np.zeros((1, 1), np.uint16))
+    rng = np.random.default_rng(77)
+    rows = rng.integers(0, M, 1200).astype(np.int32)
+    cols = rng.integers(0, N, 1200).astype(np.int32)
+    cols[:8] = np.arange(N - 8, N)
+    need = np.unique(cols)
+    q_need, s_need = oracle.quantize_rows(W[need])
+    assert np.array_equal(Wq[torch.from_numpy(need).cuda()].cpu().numpy(), q_need)
+    assert np.array_equal(sw[torch.from_numpy(need).cuda()].cpu().numpy(), s_need)
+    pool = L.Pool(dev_bf16(p.A), dev_bf16(p.B), dev(p.ranks), dev(p.scales))
+    seg = L.Segments(M, 16)
+    L.lora_build_segments(dev(p.ids), 16, seg)
+    ws = L.workspace(L.LORA_OP_W8A16_GEMM, M, K, pool)
+    y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+    L.w8a16_gemm_lora_epilogue(dev_bf16(p.x), Wq, sw, pool, seg, y, ws)
+    torch.cuda.synchronize()
+    assert L.lora_workspace_status(ws)[0] == L.LORA_OK
+    full_q = np.zeros((N, K), np.uint8)
+    full_q[need] = q_need
+    full_s = np.ones(N, np.float32)
+    full_s[need] = s_need
+    want = oracle.w8a16_gemm_lora_sampled(p.x, full_q, full_s, rows, cols, A=p.A, B=p.B, ranks=p.ranks,
+                                          scales=p.scales, ids=p.ids)
+    assert_close(f64(host_bf16_bits(y)[rows, cols]), want, TOL_FP8, "w8a16 decode shape")
