@@ -226,7 +226,7 @@ sgmv_kernel(const __grid_constant__ AMaps am, const SgmvParams p)
     if (warp == kComputeWarps) {
         // ================================================================ producer warp
         if (lane == 0 && a_tma && nK > 0) ptx::tma_prefetch_desc(&am.m[a_map]);
-        if (lane == 0 && !small && nN > 0) ptx::tma_prefetch_desc(&am.b[b_map]);
+        if (lane == 0 && nN > 0) ptx::tma_prefetch_desc(&am.b[b_map]);
         // consecutive token rows (a pre-sorted batch): x and y rows come as tensor-map boxes
         bool contig = false;
         if (!small && p.xy_maps) {
@@ -292,15 +292,18 @@ sgmv_kernel(const __grid_constant__ AMaps am, const SgmvParams p)
                 const int nb = min(BN, n_begin + n_len - n0);
                 const uint32_t yb = base + y_off;
                 if (small) {
-                    if (lane == 0) ptx::mbar_arrive_expect_tx(&full[st], (uint32_t)((r + nt) * nb * 2));
+                    // B as tensor-map boxes of 64 columns x rB rows (one request per box, not
+                    // one per rank row), the tile's y rows as 1-D copies
+                    const int nbox = (nb + 63) >> 6;
+                    if (lane == 0)
+                        ptx::mbar_arrive_expect_tx(&full[st], (uint32_t)(nbox * 64 * rB * 2 + nt * nb * 2));
                     __syncwarp();
-                    for (int i = lane; i < r + nt; i += 32) {
-                        if (i < r)
-                            ptx::bulk_g2s(base + i * bp, Bg + (size_t)i * p.h_out + n0, (uint32_t)(nb * 2), &full[st]);
-                        else
-                            ptx::bulk_g2s(yb + (i - r) * bp, yg + (size_t)s_tok[i - r] * p.h_out + n0,
-                                          (uint32_t)(nb * 2), &full[st]);
-                    }
+                    if (lane < nbox)
+                        ptx::tma_load_3d(base + (uint32_t)(lane * r16 * 128), &am.b[b_map], &full[st], n0 + lane * 64,
+                                         0, (int)sa);
+                    for (int i = lane; i < nt; i += 32)
+                        ptx::bulk_g2s(yb + i * bp, yg + (size_t)s_tok[i] * p.h_out + n0, (uint32_t)(nb * 2),
+                                      &full[st]);
                     ptx::mbar_arrive(&full[st]);
                 } else {
                     const int nbox = (nb + 63) >> 6;
@@ -659,9 +662,12 @@ sgmv_kernel(const __grid_constant__ AMaps am, const SgmvParams p)
                     float s0[kSmallTile], s1[kSmallTile];
 #pragma unroll
                     for (int t = 0; t < kSmallTile; ++t) s0[t] = s1[t] = 0.f;
-                    const uint8_t* bcol = smem + (base - base_u) + n * 2;
+                    // B(j, n..n+1) in its 64-column box: row j of 128 bytes, 16-byte chunk
+                    // (n / 8) % 8 XOR (j % 8) (the box's 128-byte swizzle)
+                    const uint8_t* bbox = smem + (base - base_u) + (n >> 6) * r16 * 128 + ((n & 7) << 1);
+                    const int bchunk = (n >> 3) & 7;
                     for (int j = 0; j < r; ++j) {
-                        const uint32_t bw = *reinterpret_cast<const uint32_t*>(bcol + j * bp);
+                        const uint32_t bw = *reinterpret_cast<const uint32_t*>(bbox + j * 128 + ((bchunk ^ (j & 7)) << 4));
                         const float b0 = bf16_lo(bw), b1 = bf16_hi(bw);
 #pragma unroll
                         for (int t = 0; t < kSmallTile; ++t)
