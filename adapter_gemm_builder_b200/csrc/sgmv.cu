@@ -181,16 +181,18 @@ sgmv_kernel(const __grid_constant__ AMaps am, const SgmvParams p)
     const int xp = BK * 2 + 16;  // x row pitch of decode tiles (bytes)
     const int n_begin = min(p.h_out, rank * p.nc);
     const int n_len = min(p.h_out, n_begin + p.nc) - n_begin;
-    // expand blocks: decode tiles keep B rows j < r and y rows at the padded pitch bp;
+    // expand blocks: small tiles keep B in unswizzled boxes of kSmallBoxCols columns (r16
+    // rows each) and their y rows at the padded pitch bp;
     // tensor-core tiles keep B (r16 rows) and y (Mtr rows) in swizzled 64-column blocks
     int BN;
     if (small) {
-        BN = ((SB / (r16 + Mtr) - 16) / 2) / 64 * 64;
+        // whole boxes of kSmallBoxCols columns (B arrives in such boxes)
+        BN = ((SB / (r16 + Mtr) - 16) / 2) / kSmallBoxCols * kSmallBoxCols;
     } else {
         BN = 64;  // a power of two, so the gathers need no division
         while (BN < 256 && 2 * BN * (2 * r16 + 2 * Mtr) <= SB) BN *= 2;
     }
-    BN = min(BN, round_up(max(n_len, 1), 64));
+    BN = min(BN, round_up(max(n_len, 1), small ? kSmallBoxCols : 64));
     const int nN = (MODE == SGMV_SHRINK) ? 0 : (n_len + BN - 1) / BN;
     const int bp = BN * 2 + 16;  // y row pitch (and B row pitch of decode tiles), bytes
     const int b_map = (r16 >> 4) - 1;
@@ -226,7 +228,7 @@ sgmv_kernel(const __grid_constant__ AMaps am, const SgmvParams p)
     if (warp == kComputeWarps) {
         // ================================================================ producer warp
         if (lane == 0 && a_tma && nK > 0) ptx::tma_prefetch_desc(&am.m[a_map]);
-        if (lane == 0 && nN > 0) ptx::tma_prefetch_desc(&am.b[b_map]);
+        if (lane == 0 && nN > 0) ptx::tma_prefetch_desc(small ? &am.bs[b_map] : &am.b[b_map]);
         // consecutive token rows (a pre-sorted batch): x and y rows come as tensor-map boxes
         bool contig = false;
         if (!small && p.xy_maps) {
@@ -292,15 +294,15 @@ sgmv_kernel(const __grid_constant__ AMaps am, const SgmvParams p)
                 const int nb = min(BN, n_begin + n_len - n0);
                 const uint32_t yb = base + y_off;
                 if (small) {
-                    // B as tensor-map boxes of 64 columns x rB rows (one request per box, not
-                    // one per rank row), the tile's y rows as 1-D copies
-                    const int nbox = (nb + 63) >> 6;
+                    // B as tensor-map boxes of kSmallBoxCols columns x rB rows (one request per
+                    // box, 256 contiguous bytes of each rank row), the tile's y rows as 1-D copies
+                    const int nbox = (nb + kSmallBoxCols - 1) / kSmallBoxCols;
                     if (lane == 0)
-                        ptx::mbar_arrive_expect_tx(&full[st], (uint32_t)(nbox * 64 * rB * 2 + nt * nb * 2));
+                        ptx::mbar_arrive_expect_tx(&full[st], (uint32_t)(nbox * kSmallBoxCols * rB * 2 + nt * nb * 2));
                     __syncwarp();
                     if (lane < nbox)
-                        ptx::tma_load_3d(base + (uint32_t)(lane * r16 * 128), &am.b[b_map], &full[st], n0 + lane * 64,
-                                         0, (int)sa);
+                        ptx::tma_load_3d(base + (uint32_t)(lane * r16 * kSmallBoxCols * 2), &am.bs[b_map], &full[st],
+                                         n0 + lane * kSmallBoxCols, 0, (int)sa);
                     for (int i = lane; i < nt; i += 32)
                         ptx::bulk_g2s(yb + i * bp, yg + (size_t)s_tok[i] * p.h_out + n0, (uint32_t)(nb * 2),
                                       &full[st]);
@@ -662,12 +664,11 @@ sgmv_kernel(const __grid_constant__ AMaps am, const SgmvParams p)
                     float s0[kSmallTile], s1[kSmallTile];
 #pragma unroll
                     for (int t = 0; t < kSmallTile; ++t) s0[t] = s1[t] = 0.f;
-                    // B(j, n..n+1) in its 64-column box: row j of 128 bytes, 16-byte chunk
-                    // (n / 8) % 8 XOR (j % 8) (the box's 128-byte swizzle)
-                    const uint8_t* bbox = smem + (base - base_u) + (n >> 6) * r16 * 128 + ((n & 7) << 1);
-                    const int bchunk = (n >> 3) & 7;
+                    // B(j, n..n+1) in its box of kSmallBoxCols columns: rows of 2 kSmallBoxCols bytes
+                    const uint8_t* bbox = smem + (base - base_u) + (n / kSmallBoxCols) * r16 * kSmallBoxCols * 2 +
+                                          (n % kSmallBoxCols) * 2;
                     for (int j = 0; j < r; ++j) {
-                        const uint32_t bw = *reinterpret_cast<const uint32_t*>(bbox + j * 128 + ((bchunk ^ (j & 7)) << 4));
+                        const uint32_t bw = *reinterpret_cast<const uint32_t*>(bbox + j * kSmallBoxCols * 2);
                         const float b0 = bf16_lo(bw), b1 = bf16_hi(bw);
 #pragma unroll
                         for (int t = 0; t < kSmallTile; ++t)

@@ -26,10 +26,14 @@ constexpr unsigned long long kTimeoutNs = 2000000000ull;  // drains after an abo
 // n_adapters}, box {8 << i, 64, 1} (swizzle = the box row width);
 // b[i]: B viewed as {h_out, r_max, n_slices * n_adapters}, box
 // {64, min(16 (i + 1), r_max), 1}, 128-byte swizzle.
+// bs[i]: B as b[i], box {128, min(16 (i + 1), r_max), 1}, not swizzled (small tiles:
+// 256 contiguous bytes of each rank row per request).
 // x: {h_in, T, slices of x}, y: {h_out, T, n_slices}, box {64, 16, 1}, 128-byte swizzle.
+constexpr int kSmallBoxCols = 128;
 struct AMaps {
     CUtensorMap m[4];
     CUtensorMap b[4];
+    CUtensorMap bs[4];
     CUtensorMap x, y;
 };
 
@@ -150,6 +154,10 @@ inline bool build_pool_maps(AMaps& am, const lora_pool_t& pool, bool shrink, boo
             const uint32_t box[3] = {64, (uint32_t)rows, 1};
             if (!encode_tmap_3d(&am.b[i], CU_TENSOR_MAP_DATA_TYPE_UINT16, pool.B, dims, strides, box,
                                 CU_TENSOR_MAP_SWIZZLE_128B))
+                return false;
+            const uint32_t box_s[3] = {(uint32_t)kSmallBoxCols, (uint32_t)rows, 1};
+            if (!encode_tmap_3d(&am.bs[i], CU_TENSOR_MAP_DATA_TYPE_UINT16, pool.B, dims, strides, box_s,
+                                CU_TENSOR_MAP_SWIZZLE_NONE))
                 return false;
         }
     }
