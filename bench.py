@@ -64,6 +64,8 @@ def parse_args():
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--fp8-only", action="store_true",
                     help="run only the FP8 GEMM + LoRA section and print its JSON")
+    ap.add_argument("--section", choices=["fp8", "bf16", "w8a16", "mxfp4", "merge"],
+                    help="run only this GEMM / merge section and print its JSON (profiling aid)")
     ap.add_argument("--fp8-m", type=int, nargs="+", default=[16, 64, 256])
     ap.add_argument("--fp8-reps", type=int, default=20, help="graph replays per timing")
     ap.add_argument("--no-bf16", action="store_true", help="skip the bf16 GEMM + LoRA section")
@@ -1007,6 +1009,20 @@ def run_merge(args, dev, stream, hbm_peak, peak_src):
 
 def main():
     args = parse_args()
+    if args.section:
+        import torch
+        from adapter_gemm_builder_b200 import lora as L
+        L.load()
+        dev = torch.device("cuda", 0)
+        hbm, bf16, sust, src = measured_peaks()
+        st = torch.cuda.Stream(device=dev)
+        run = {"fp8": lambda: run_fp8(args, dev, st, hbm, bf16, sust, src),
+               "bf16": lambda: run_bf16(args, dev, st, hbm, bf16, src),
+               "mxfp4": lambda: run_mxfp4(args, dev, st, hbm, bf16, src),
+               "w8a16": lambda: run_mxfp4(args, dev, st, hbm, bf16, src, "w8a16"),
+               "merge": lambda: run_merge(args, dev, st, hbm, src)}[args.section]
+        print(json.dumps(run()))
+        return
     if args.fp8_only:
         import torch
         from adapter_gemm_builder_b200 import lora as L
