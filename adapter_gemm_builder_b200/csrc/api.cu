@@ -265,9 +265,10 @@ size_t lora_workspace_size(int op, int T, int K, const lora_pool_t* pool)
     case LORA_OP_SHRINK:
     case LORA_OP_EXPAND: return 0;
     case LORA_OP_APPLY:
-        // v stays on chip (exchanged inside each thread-block cluster): no workspace
+        // v stays on chip; a general batch's tile rows in cost order (optional workspace)
         if (!pool || check_pool(pool) != LORA_OK) return (size_t)-1;
-        return 0;
+        if (T == 0 || tile_tokens_for(T, pool->n_adapters) <= LORA_DECODE_TILE_TOKENS) return 0;
+        return align256(sgmv_order_bytes(T, pool->n_adapters));
     case LORA_OP_FP8_BACKWARD: {
         if (!pool || check_pool(pool) != LORA_OK || T < 1) return (size_t)-1;
         size_t a, b, c, d;
@@ -382,10 +383,14 @@ int lora_apply(const void* x, int64_t x_slice_stride, const lora_pool_t* pool,
     if ((st = check_x(x, x_slice_stride, pool, seg->T)) != LORA_OK) return st;
     if (!y || !aligned16(y)) return LORA_ERR_INVALID_ARG;
     cudaStream_t s = (cudaStream_t)stream;
-    // one tile row per thread-block cluster, v exchanged on chip (ws is not used)
-    (void)ws;
-    (void)ws_bytes;
-    return cuda_status(launch_sgmv(SGMV_APPLY, x, x_slice_stride, *pool, *seg, nullptr, y, s, false));
+    // one tile row per thread-block cluster, v exchanged on chip; with a workspace, a
+    // general batch's tile rows run in descending cost (a small ordering kernel first)
+    void* order = nullptr;
+    if (ws && tile_tokens_for(seg->T, pool->n_adapters) > LORA_DECODE_TILE_TOKENS) {
+        if (ws_bytes < sgmv_order_bytes(seg->T, pool->n_adapters) || !aligned16(ws)) return LORA_ERR_WORKSPACE;
+        order = ws;
+    }
+    return cuda_status(launch_sgmv(SGMV_APPLY, x, x_slice_stride, *pool, *seg, nullptr, y, s, false, order));
 }
 
 int fp8_quantize_rows(const void* x, int M, int K, uint8_t* xq, float* sx, lora_stream_t stream)

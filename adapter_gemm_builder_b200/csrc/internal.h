@@ -16,10 +16,14 @@ cudaError_t launch_build_segments(const int32_t* ids, int T, int n_adapters,
 
 enum SgmvMode { SGMV_SHRINK = 0, SGMV_EXPAND = 1, SGMV_APPLY = 2 };
 
-// x, v, y may be NULL where the mode does not use them.
+// x, v, y may be NULL where the mode does not use them. order: NULL, or
+// sgmv_order_bytes(T, n_adapters) bytes of device memory (16-byte aligned) into which
+// a small kernel first writes the tile rows in descending cost, which the SGMV
+// kernel then walks (long rows first, no tail of a few long CTAs).
 cudaError_t launch_sgmv(int mode, const void* x, int64_t x_slice_stride, const lora_pool_t& pool,
                         const lora_segments_t& seg, float* v, void* y, cudaStream_t stream,
-                        bool pdl_trigger);
+                        bool pdl_trigger, void* order = nullptr);
+size_t sgmv_order_bytes(int T, int n_adapters);
 
 // Token-wise merge of the selected adapters into the backbone (merge.cu).
 cudaError_t launch_lora_switch_merge(const void* W, int N, int K, const lora_pool_t& pool, const int32_t* sel,

@@ -11,10 +11,11 @@
 //      for the tile's columns and of their B columns for the tile's rows into
 //      padded shared-memory tiles (no bank conflicts for ldmatrix);
 //   2. per selected adapter, bf16 mma.sync (m16n8k16, fp32 accumulate) of
-//      D^T[k][n] = sum_j A[k][j] B[j][n] over its rank, then D += g s D_e in
+//      D[n][k] = sum_j B[j][n] A[k][j] over its rank, then D += g s D_e in
 //      fp32 (the gate and scale are applied to the fp32 product, so the only
 //      rounding of the merged weight is the final one to bf16);
-//   3. the tile updated in shared memory and stored with 16-byte stores.
+//   3. the tile updated in shared memory, a pair of consecutive k per access,
+//      and stored with 16-byte stores.
 // W_out may be W itself (each CTA reads its whole tile before writing it).
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -51,7 +52,7 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi)
     return *reinterpret_cast<uint32_t*>(&h);
 }
 
-__global__ void __launch_bounds__(kThreadsM)
+__global__ void __launch_bounds__(kThreadsM, 4)
 merge_kernel(const MergeParams p)
 {
     extern __shared__ __align__(16) uint8_t smem[];
@@ -135,51 +136,64 @@ merge_kernel(const MergeParams p)
     }
     __syncthreads();
 
-    // ---- 2. warp w: D^T rows k = 16 w .. 16 w + 15, all 64 columns n (8 MMA tiles of 8)
-    float acc[8][4], part[8][4];
+    // ---- 2. warp w: D rows n = 16 (w % 4) .. + 15, columns k = 64 (w / 4) .. + 63, in two
+    // passes of 32 columns (4 MMA tiles of 8; fewer live accumulators): D[n][k] =
+    // sum_j B[j][n] A[k][j], so a thread's accumulator pairs are pairs of consecutive k,
+    // contiguous in W's row n
+    const int mt = warp & 3, kh = warp >> 2;
+    const int gq = lane >> 2, tq = lane & 3;
+    // A operand (n x j, from B stored [j][n]): transposed 8x8 loads, lane -> row j, n block
+    const uint32_t a_row = ptx::smem_u32(Bs + ((lane & 7) + ((lane >> 4) << 3)) * kBPitch +
+                                         (mt * 16 + ((lane >> 3) & 1) * 8) * 2);
+    for (int pass = 0; pass < 2; ++pass) {
+        const int kq = kh * 64 + pass * 32;  // first column of this pass
+        // B operand (j x k, from A stored [k][j]): two k tiles per 4-matrix load
+        const uint32_t b_row = ptx::smem_u32(As + (kq + ((lane >> 4) << 3) + (lane & 7)) * p.a_pitch +
+                                             ((lane >> 3) & 1) * 16);
+        float acc[4][4], part[4][4];
 #pragma unroll
-    for (int t = 0; t < 8; ++t)
+        for (int t = 0; t < 4; ++t)
 #pragma unroll
-        for (int i = 0; i < 4; ++i) acc[t][i] = 0.f;
-    const uint32_t a_row = ptx::smem_u32(As + (warp * 16 + (lane & 15)) * p.a_pitch + (lane >> 4) * 16);
-    const uint32_t b_row = ptx::smem_u32(Bs + (lane & 15) * kBPitch);
-    for (int e = 0; e < ne; ++e) {
-        const int r16 = (s_r[e] + 15) & ~15, j0 = s_j0[e];
+            for (int i = 0; i < 4; ++i) acc[t][i] = 0.f;
+        for (int e = 0; e < ne; ++e) {
+            const int r16 = (s_r[e] + 15) & ~15, j0 = s_j0[e];
 #pragma unroll
-        for (int t = 0; t < 8; ++t)
+            for (int t = 0; t < 4; ++t)
 #pragma unroll
-            for (int i = 0; i < 4; ++i) part[t][i] = 0.f;
-        for (int ks = 0; ks < r16 / 16; ++ks) {
-            const int j = j0 + ks * 16;
-            uint32_t af[4];
-            ptx::ldsm_x4(a_row + j * 2, af[0], af[1], af[2], af[3]);
+                for (int i = 0; i < 4; ++i) part[t][i] = 0.f;
+            for (int ks = 0; ks < r16 / 16; ++ks) {
+                const int j = j0 + ks * 16;
+                uint32_t af[4];
+                ptx::ldsm_x4_t(a_row + j * kBPitch, af[0], af[1], af[2], af[3]);
 #pragma unroll
-            for (int t = 0; t < 8; ++t) {
-                uint32_t b0, b1;
-                ptx::ldsm_x2_t(b_row + j * kBPitch + t * 16, b0, b1);
-                ptx::mma_bf16_16816(part[t], af, b0, b1);
+                for (int t = 0; t < 4; t += 2) {
+                    uint32_t b[4];
+                    ptx::ldsm_x4(b_row + t * 8 * p.a_pitch + j * 2, b[0], b[1], b[2], b[3]);
+                    ptx::mma_bf16_16816(part[t], af, b[0], b[1]);
+                    ptx::mma_bf16_16816(part[t + 1], af, b[2], b[3]);
+                }
             }
+            const float c = s_c[e];
+#pragma unroll
+            for (int t = 0; t < 4; ++t)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) acc[t][i] = fmaf(c, part[t][i], acc[t][i]);
         }
-        const float c = s_c[e];
+        // ---- 3. W tile += D: the fragment's pairs (n = gq or gq + 8, k = 2 tq, 2 tq + 1)
+        if (ne > 0) {
 #pragma unroll
-        for (int t = 0; t < 8; ++t)
+            for (int t = 0; t < 4; ++t)
 #pragma unroll
-            for (int i = 0; i < 4; ++i) acc[t][i] = fmaf(c, part[t][i], acc[t][i]);
-    }
-    // ---- 3. W tile += D (D^T fragment: rows k = gq, gq + 8; columns n = 2 tq, 2 tq + 1)
-    if (ne > 0) {
-        const int gq = lane >> 2, tq = lane & 3;
-#pragma unroll
-        for (int t = 0; t < 8; ++t)
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int k = warp * 16 + gq + (i >> 1) * 8;
-                const int n = t * 8 + tq * 2 + (i & 1);
-                uint16_t* w = reinterpret_cast<uint16_t*>(Ws + n * kWPitch + k * 2);
-                const float f = __uint_as_float((uint32_t)*w << 16) + acc[t][i];
-                __nv_bfloat16 h = __float2bfloat16_rn(f);
-                *w = *reinterpret_cast<uint16_t*>(&h);
-            }
+                for (int h = 0; h < 2; ++h) {
+                    const int n = mt * 16 + gq + h * 8;
+                    const int k = kq + t * 8 + tq * 2;
+                    uint32_t* w = reinterpret_cast<uint32_t*>(Ws + n * kWPitch + k * 2);
+                    const uint32_t wv = *w;
+                    const float f0 = __uint_as_float(wv << 16) + acc[t][2 * h];
+                    const float f1 = __uint_as_float(wv & 0xffff0000u) + acc[t][2 * h + 1];
+                    *w = pack2(f0, f1);
+                }
+        }
     }
     __syncthreads();
     for (int i = tid; i < kTN * wchunks; i += kThreadsM) {

@@ -15,8 +15,9 @@
 // LORA_TILE_TOKENS. A
 // tile is handled by a thread-block cluster of C CTAs: in the shrink CTA c
 // owns the c-th slice of h_in (split-K) and computes a partial v for the
-// tile's tokens; in the expand it owns the c-th slice of h_out. gridDim.y is
-// the slice (projection) index, so q/k/v/o run in one launch.
+// tile's tokens; in the expand it owns the c-th slice of h_out. The grid covers
+// every (tile row, slice) pair, the slices of a row adjacent, so q/k/v/o run in
+// one launch.
 //
 // Memory path (the kernel is bound by HBM bytes and by latency). A producer
 // warp fills a ring of 3 stages whose copies all complete on the stage's
@@ -70,11 +71,12 @@ struct SgmvParams {
     const int32_t* ranks;
     const float* scales;
     const int32_t* perm;
-    const int4* tiles;
+    const int4* tiles;  // the segments' tile rows, or the same rows in cost order (tile_order_kernel)
     int32_t* counts;
     float* v;
     uint16_t* y;
     int T, n_adapters, h_in, h_out, r_max;
+    int n_slices;
     int csize;       // CTAs per tile
     int kc, nc;      // h_in / h_out slice per CTA (kc a multiple of 128, nc of 64)
     int rp;          // round_up(r_max, 16): row pitch (floats) of the v buffers
@@ -103,8 +105,10 @@ sgmv_kernel(const __grid_constant__ AMaps am, const SgmvParams p)
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int C = p.csize;
     const int rank = kClustered ? (int)ptx::cluster_ctarank() : (int)(blockIdx.x % C);
-    const int g = blockIdx.x / C;
-    const int slice = blockIdx.y;
+    // blockIdx.x = ((tile row * n_slices) + slice) * C + rank: the slices of a tile row
+    // launch together (with the rows in cost order, every slice's long rows start first)
+    const int g = (blockIdx.x / C) / p.n_slices;
+    const int slice = (blockIdx.x / C) - g * p.n_slices;
     const int SB = p.stage_bytes;
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + p.off_bar);
     uint64_t* empty = full + kStages;
@@ -755,6 +759,58 @@ sgmv_kernel(const __grid_constant__ AMaps am, const SgmvParams p)
 #undef SACC
 #undef ACC
 
+// The tile rows of a general batch in descending cost, so that the long rows start
+// first and the grid has no tail of a few long CTAs: the tensor-core rows (more than
+// kSmallTile tokens), then the small rows by descending rank (round_up(r, 8)), each
+// class in table order (a stable counting sort, one CTA). Results do not depend on
+// the order: every row writes only its own tokens' outputs. The unused rows keep
+// their places after the last used one; above kOrderMax used rows the table is copied
+// as it is.
+constexpr int kOrderThreads = 1024;
+constexpr int kOrderMax = kOrderThreads;
+constexpr int kOrderClasses = 9;
+__global__ void __launch_bounds__(kOrderThreads)
+tile_order_kernel(const int4* tiles, const int32_t* counts, const int32_t* ranks, int r_max, int max_tiles, int4* out)
+{
+    __shared__ int s_cnt[kOrderClasses][kOrderThreads / 32];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    ptx::pdl_wait();  // the segment builder wrote the tile rows
+    const int n = min(max(counts[3], 0), max_tiles);
+    if (n > kOrderMax) {
+        for (int i = tid; i < max_tiles; i += kOrderThreads) out[i] = tiles[i];
+        ptx::pdl_launch_dependents();
+        return;
+    }
+    const bool valid = tid < n;
+    const int4 tl = valid ? tiles[tid] : make_int4(-1, 0, 0, -1);
+    int key = kOrderClasses;  // none
+    if (valid) {
+        int r = ranks ? ranks[tl.x] : r_max;
+        r = max(1, min(r, r_max));
+        key = tl.z > kSmallTile ? 0 : 1 + (64 - ((r + 7) & ~7)) / 8;  // 0 .. 8
+    }
+    unsigned mine = 0;
+    for (int c = 0; c < kOrderClasses; ++c) {
+        const unsigned b = __ballot_sync(0xffffffffu, key == c);
+        if (key == c) mine = b;
+        if (lane == 0) s_cnt[c][warp] = __popc(b);
+    }
+    __syncthreads();
+    if (tid == 0) {  // exclusive prefix in (class, warp) order
+        int run = 0;
+        for (int c = 0; c < kOrderClasses; ++c)
+            for (int w = 0; w < kOrderThreads / 32; ++w) {
+                const int v = s_cnt[c][w];
+                s_cnt[c][w] = run;
+                run += v;
+            }
+    }
+    __syncthreads();
+    if (valid) out[s_cnt[key][warp] + __popc(mine & ((1u << lane) - 1u))] = tl;
+    for (int i = n + tid; i < max_tiles; i += kOrderThreads) out[i] = tiles[i];
+    ptx::pdl_launch_dependents();
+}
+
 template <int MODE, bool kSmallOnly>
 cudaError_t launch_mode(const AMaps& am, const SgmvParams& p, dim3 grid, int C, size_t smem, cudaStream_t stream)
 {
@@ -800,9 +856,14 @@ size_t sgmv_smem_per_cta()
 
 }  // namespace
 
+size_t sgmv_order_bytes(int T, int n_adapters)
+{
+    return (size_t)max_tiles_for(T, n_adapters) * sizeof(int4);
+}
+
 cudaError_t launch_sgmv(int mode, const void* x, int64_t x_slice_stride, const lora_pool_t& pool,
                         const lora_segments_t& seg, float* v, void* y, cudaStream_t stream,
-                        bool pdl_trigger)
+                        bool pdl_trigger, void* order)
 {
     (void)pdl_trigger;
     if (seg.T == 0) return cudaSuccess;
@@ -815,6 +876,26 @@ cudaError_t launch_sgmv(int mode, const void* x, int64_t x_slice_stride, const l
     p.scales = pool.scales;
     p.perm = seg.perm;
     p.tiles = reinterpret_cast<const int4*>(seg.tiles);
+    // the tile rows in cost order first (one small CTA, a programmatic dependent), when
+    // there are more rows than one wave of two CTAs per SM holds (else order cannot help)
+    if (order && (long long)max_tiles_for(seg.T, pool.n_adapters) * pool.n_slices <= 2LL * device_sm_count())
+        order = nullptr;
+    if (order) {
+        const int mt = max_tiles_for(seg.T, pool.n_adapters);
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(1, 1, 1);
+        cfg.blockDim = dim3(kOrderThreads, 1, 1);
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        const cudaError_t e = cudaLaunchKernelEx(&cfg, tile_order_kernel, p.tiles, (const int32_t*)seg.counts,
+                                                 pool.ranks, pool.r_max, mt, static_cast<int4*>(order));
+        if (e != cudaSuccess) return e;
+        p.tiles = static_cast<const int4*>(order);
+    }
     p.counts = seg.counts;
     p.v = v;
     p.y = static_cast<uint16_t*>(y);
@@ -877,7 +958,8 @@ cudaError_t launch_sgmv(int mode, const void* x, int64_t x_slice_stride, const l
     if (!build_pool_maps(am, pool, mode != SGMV_EXPAND, mode != SGMV_SHRINK)) return cudaErrorInvalidValue;
     p.xy_maps = build_xy_maps(am, pool, seg.T, x, x_slice_stride, y, mode != SGMV_EXPAND, mode != SGMV_SHRINK) ? 1 : 0;
 
-    const dim3 grid((unsigned)(max_tiles_for(seg.T, pool.n_adapters) * C), (unsigned)pool.n_slices, 1);
+    p.n_slices = pool.n_slices;
+    const dim3 grid((unsigned)((long long)max_tiles_for(seg.T, pool.n_adapters) * pool.n_slices * C), 1, 1);
     // segments of a decode-like batch come in tiles of <= kSmallTile tokens
     if (tile_tokens_for(seg.T, seg.n_adapters) <= kSmallTile) {
         switch (mode) {

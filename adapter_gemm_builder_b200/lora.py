@@ -246,11 +246,14 @@ def lora_expand(v: torch.Tensor, pool: Pool, seg: Segments, y: torch.Tensor, str
 
 
 def lora_apply(x: torch.Tensor, pool: Pool, seg: Segments, y: torch.Tensor, stream=None,
-               x_slice_stride: int | None = None, ws: torch.Tensor | None = None) -> None:
+               x_slice_stride: int | None = None, ws: torch.Tensor | None | bool = None) -> None:
     """y += s_a (x.A_a).B_a; ws: a workspace of lora_workspace_size(LORA_OP_APPLY, T, 0, pool)
-    bytes (none today: v stays on chip; allocated here when None and the size is not 0)."""
+    bytes, in which a general batch's tile rows are put in cost order (allocated here when
+    None and the size is not 0; False: none, the rows run in table order)."""
     xs = _slice_stride(x, pool) if x_slice_stride is None else x_slice_stride
-    if ws is None:
+    if ws is False:  # explicitly none: the tile rows run in table order
+        ws = None
+    elif ws is None:
         n = lora_workspace_size(LORA_OP_APPLY, seg.T, 0, pool)
         ws = workspace(LORA_OP_APPLY, seg.T, 0, pool, device=y.device, stream=stream) if n else None
     _check(load().lora_apply(_ptr(x), xs, ctypes.byref(pool.c), ctypes.byref(seg.c), _ptr(y),

@@ -152,8 +152,9 @@ LORA_API int lora_segments_status(const lora_segments_t* seg, lora_stream_t stre
  * Bytes of workspace an operation needs (0 if it needs none), or (size_t)-1
  * for invalid arguments. For LORA_OP_FP8_GEMM, T is the
  * token count M and `K` the GEMM's reduction size; `pool` may be NULL (no
- * LoRA). LORA_OP_APPLY needs a valid pool and returns 0 (v stays on chip).
- * The other operations ignore K.
+ * LoRA). LORA_OP_APPLY needs a valid pool; it returns 0 for a decode-like
+ * batch (lora_tile_tokens_for) and otherwise the bytes of the tile rows in cost
+ * order (16 per row of lora_max_tiles). The other operations ignore K.
  * A workspace must be zeroed once after allocation (lora_workspace_init);
  * afterwards the library keeps it in a reusable state.
  */
@@ -216,11 +217,16 @@ LORA_API int lora_expand(const float* v, const lora_pool_t* pool, const lora_seg
 /*
  * Shrink then expand (y += s_a * (x.A_a).B_a; the whole added term of the
  * Punica README, "How?", for a batch of many adapters), v in fp32. Arguments
- * as lora_shrink / lora_expand, plus a workspace of
- * lora_workspace_size(LORA_OP_APPLY, T, 0, pool) bytes (0 today; ws may be
- * NULL). One kernel launch: each thread-block cluster takes one tile row
- * (lora_tile_tokens_for) and keeps its v on chip, the partial v of its CTAs
- * exchanged through distributed shared memory.
+ * as lora_shrink / lora_expand, plus an optional workspace of
+ * lora_workspace_size(LORA_OP_APPLY, T, 0, pool) bytes. The SGMV kernel: each
+ * thread-block cluster takes one tile row (lora_tile_tokens_for) and keeps its
+ * v on chip, the partial v of its CTAs exchanged through distributed shared
+ * memory. With a workspace (ws != NULL, ws_bytes at least that size, 16-byte
+ * aligned, else LORA_ERR_WORKSPACE), a batch that is not decode-like and whose
+ * tile rows times slices exceed two per SM first runs a one-CTA kernel that writes
+ * its tile rows into ws in descending cost (rows of more than four tokens, then
+ * by descending rank), so that the long rows start first; the results are the
+ * same either way. ws NULL: one launch, table order.
  */
 LORA_API int lora_apply(const void* x, int64_t x_slice_stride, const lora_pool_t* pool,
                const lora_segments_t* seg, void* y, void* ws, size_t ws_bytes,

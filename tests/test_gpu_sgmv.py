@@ -352,3 +352,40 @@ def test_whole_layer_many_tenants_sampled():
     rng = np.random.default_rng(4)
     rows = np.sort(rng.choice(p.T, 24, replace=False))
     _whole_layer(p, W, rows)
+
+
+# ------------------------------------------------------------------ tile rows in cost order
+
+def _expected_order(tiles, n_used, ranks, r_max):
+    """The order lora_apply's workspace holds: the used tile rows stably sorted by class
+    (rows of more than four tokens first, then small rows by descending round_up(r, 8)),
+    then the unused rows in place."""
+    def key(row):
+        if row[2] > 4:
+            return 0
+        r = max(1, min(int(ranks[row[0]]), r_max))
+        return 1 + (64 - ((r + 7) & ~7)) // 8
+    used = sorted(range(n_used), key=lambda i: key(tiles[i]))  # Python's sort is stable
+    return np.concatenate([tiles[used], tiles[n_used:]]) if n_used < len(tiles) else tiles[used]
+
+
+@pytest.mark.parametrize("ids_kind", ["zipf", "uniform"])
+def test_apply_tile_order_same_results_and_cost_order(ids_kind):
+    """With a workspace, a general batch's tile rows run in cost order: the output is
+    bit-identical to the table-order launch (no workspace), and the workspace holds the
+    rows in the stated order."""
+    p = wl.many_tenants(seed=11, T=300, n_adapters=96, h=1024, ids_kind=ids_kind)
+    d = DeviceProblem(p)
+    y0 = d.y_in()
+    L.lora_apply(d.x, d.pool, d.seg, y0, ws=False)
+    ws = L.workspace(L.LORA_OP_APPLY, p.T, 0, d.pool)
+    y1 = d.y_in()
+    L.lora_apply(d.x, d.pool, d.seg, y1, ws=ws)
+    torch.cuda.synchronize()
+    assert L.lora_segments_status(d.seg)[0] == L.LORA_OK
+    assert np.array_equal(host_bf16_bits(y0), host_bf16_bits(y1))
+    tiles = d.seg.tiles.cpu().numpy()
+    n_used = int(d.seg.counts[3].item())
+    got = ws[: tiles.size * 4].view(torch.int32).cpu().numpy().reshape(-1, 4)
+    assert np.array_equal(got, _expected_order(tiles, n_used, p.ranks, p.r_max))
+    assert_close(f64(host_bf16_bits(y1)), oracle_apply(p), TOL_BF16, f"ordered apply {ids_kind}")

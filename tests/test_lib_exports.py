@@ -75,7 +75,9 @@ def test_workspace_sizes(lib):
     assert lib.lora_workspace_size(L.LORA_OP_APPLY, 10, 0, None) == ctypes.c_size_t(-1).value
     pa = _pool(n_slices=4, n_adapters=256, h_in=5120, h_out=5120, r_max=64)
     assert lib.lora_workspace_size(L.LORA_OP_APPLY, 36, 0, ctypes.byref(_pool(n_adapters=32))) == 0
-    assert lib.lora_workspace_size(L.LORA_OP_APPLY, 512, 0, ctypes.byref(pa)) == 0  # v stays on chip
+    # a general batch: the tile rows in cost order, 16 bytes per row of lora_max_tiles
+    n = lib.lora_workspace_size(L.LORA_OP_APPLY, 512, 0, ctypes.byref(pa))
+    assert n >= 16 * lib.lora_max_tiles(512, 256) and n % 256 == 0
     p = _pool(h_in=8192, h_out=28672)
     n = lib.lora_workspace_size(L.LORA_OP_FP8_GEMM, 256, 8192, ctypes.byref(p))
     assert n >= 256 + 256 * 8192 + 256 * 4 + 256 * 16 * 4
