@@ -592,15 +592,17 @@ sgmv_kernel(const __grid_constant__ AMaps am, const SgmvParams p)
                         }
                     }
                 }
-            } else if (ok) {
+            } else if (!small && (kb & 15)) {
+                // last block of h_in: x columns kb..kb+8 may hold stale bytes; zero them (the
+                // barrier does not depend on ok, so every compute thread meets it)
+                if (ok && tid < nt)
+                    *reinterpret_cast<uint4*>(smem + (xb - base_u) + blk_chunk(tid, kb >> 3, Mtr)) =
+                        make_uint4(0, 0, 0, 0);
+                ptx::fence_proxy_async_smem();  // generic writes to a stage that bulk copies refill
+                ptx::named_sync(1, kCompute);
+            }
+            if (ok && !small) {
                 const int ksteps = (kb + 15) >> 4;
-                if (kb & 15) {  // last block of h_in: x columns kb..kb+8 may hold stale bytes; zero them
-                    if (tid < nt)
-                        *reinterpret_cast<uint4*>(smem + (xb - base_u) + blk_chunk(tid, kb >> 3, Mtr)) =
-                            make_uint4(0, 0, 0, 0);
-                    ptx::fence_proxy_async_smem();  // generic writes to a stage that bulk copies refill
-                    ptx::named_sync(1, kCompute);
-                }
                 // x rows in swizzled 64-column blocks: row (l_mt*16 + lane%16), k chunk 2*ks + lane/16
                 uint32_t xrow[4], aaddr[4];
 #pragma unroll
@@ -690,18 +692,18 @@ sgmv_kernel(const __grid_constant__ AMaps am, const SgmvParams p)
                                 pack_bf16x2(bf16_lo(yw) + scale * s0[t], bf16_hi(yw) + scale * s1[t]);
                         }
                 }
-            } else if (ok) {
+            } else if (!small) {
                 if (r != r16) {  // B rows r..r16 of every box hold padding or nothing: zero them
                     const int zr = r16 - r, nbx = (nb + 63) >> 6;
-                    for (int i = tid; i < nbx * zr * 8; i += kCompute) {
+                    for (int i = tid; ok && i < nbx * zr * 8; i += kCompute) {
                         const int bx = i / (zr * 8), rem = i - bx * zr * 8;
                         *reinterpret_cast<uint4*>(smem + (base - base_u) + bx * r16 * 128 + (r + (rem >> 3)) * 128 +
                                                   (rem & 7) * 16) = make_uint4(0, 0, 0, 0);
                     }
                     ptx::fence_proxy_async_smem();  // generic writes to a stage that bulk copies refill
-                    ptx::named_sync(1, kCompute);
+                    ptx::named_sync(1, kCompute);    // met by every compute thread, whatever ok
                 }
-                const int nNTe = (nb + 7) >> 3;
+                const int nNTe = ok ? (nb + 7) >> 3 : 0;
                 const int gq = lane >> 2, tq = lane & 3;
                 for (int ntl = ntl0; ntl < nNTe; ntl += nw_mt) {
                     // row j = ks*16 + (lane & 15) of box ntl/8, 16-byte chunk ntl%8 XOR (j & 7)
