@@ -53,16 +53,19 @@ int check_segments(const lora_segments_t* seg, int n_adapters)
 // GEMM workspace: status | xq (esz bytes per element) | sx | v (with a pool) |
 // sync words | partials. [off_v, off_part) is zeroed by the quantiser on every call.
 // Batches whose adapters are too many to fold into the GEMM's accumulator (more
-// than kFuseMaxAdapters in the pool and in the batch) run the base GEMM and then
-// the SGMV apply instead (see gemm_lora_launch).
+// than kFuseMaxAdapters in the pool and in the batch), and batches of more than
+// kFuseMaxTokens tokens (prefill: the down-projection of that many tokens on the
+// epilogue warps costs more than the SGMV apply), run the base GEMM and then the SGMV
+// apply instead (see gemm_lora_launch).
 constexpr int kFuseMaxAdapters = 16;
+constexpr int kFuseMaxTokens = 1024;
 bool gemm_split(int M, const lora_pool_t* pool)
 {
-    return pool && pool->n_adapters > kFuseMaxAdapters && M > kFuseMaxAdapters;
+    return pool && ((pool->n_adapters > kFuseMaxAdapters && M > kFuseMaxAdapters) || M > kFuseMaxTokens);
 }
 
 size_t fp8_ws_layout(int M, int K, const lora_pool_t* pool, size_t* off_xq, size_t* off_sx,
-                     size_t* off_v, size_t* off_sync, size_t* off_part, int esz = 1)
+                     size_t* off_v, size_t* off_sync, size_t* off_part, int esz = 1, size_t* off_order = nullptr)
 {
     size_t off = 256;  // status word block
     *off_xq = off;
@@ -75,6 +78,8 @@ size_t fp8_ws_layout(int M, int K, const lora_pool_t* pool, size_t* off_xq, size
     off += align256((size_t)(16 + device_sm_count()) * 4);
     *off_part = off;
     off += align256(fp8_gemm_partial_bytes(M));
+    if (off_order) *off_order = off;  // the split path's apply: tile rows in cost order
+    if (gemm_split(M, pool)) off += align256(sgmv_order_bytes(M, pool->n_adapters));
     return off;
 }
 
@@ -133,9 +138,9 @@ int gemm_lora_launch(int esz, const void* x, int M, int K, int N, const uint8_t*
                      const lora_pool_t* pool, const lora_segments_t* seg, void* y, void* ws,
                      size_t ws_bytes, lora_stream_t stream, const uint8_t* wsc = nullptr, bool w_e4m3 = false)
 {
-    size_t off_xq, off_sx, off_v, off_sync, off_part;
+    size_t off_xq, off_sx, off_v, off_sync, off_part, off_order;
     const size_t need =
-        fp8_ws_layout(M, K, pool, &off_xq, &off_sx, &off_v, &off_sync, &off_part, esz);
+        fp8_ws_layout(M, K, pool, &off_xq, &off_sx, &off_v, &off_sync, &off_part, esz, &off_order);
     if (!ws || ws_bytes < need || !aligned16(ws)) return LORA_ERR_WORKSPACE;
     const bool split = gemm_split(M, pool);
     const lora_pool_t* fused = split ? nullptr : pool;  // the adapters folded into the GEMM
@@ -189,8 +194,10 @@ int gemm_lora_launch(int esz, const void* x, int M, int K, int N, const uint8_t*
     }
     e = launch_fp8_gemm(a, s);
     if (e != cudaSuccess || !split) return cuda_status(e);
-    // 3. many adapters: their term added to the GEMM's bf16 output by the SGMV apply
-    return cuda_status(launch_sgmv(SGMV_APPLY, x, 0, *pool, *seg, nullptr, y, s, false));
+    // 3. many adapters or tokens: their term added to the GEMM's bf16 output by the SGMV
+    //    apply (a general batch's tile rows in cost order, in the workspace)
+    void* order = tile_tokens_for(M, pool->n_adapters) > LORA_DECODE_TILE_TOKENS ? w + off_order : nullptr;
+    return cuda_status(launch_sgmv(SGMV_APPLY, x, 0, *pool, *seg, nullptr, y, s, false, order));
 }
 
 }  // namespace

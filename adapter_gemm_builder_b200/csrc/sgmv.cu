@@ -878,10 +878,37 @@ cudaError_t launch_sgmv(int mode, const void* x, int64_t x_slice_stride, const l
     p.scales = pool.scales;
     p.perm = seg.perm;
     p.tiles = reinterpret_cast<const int4*>(seg.tiles);
+    p.counts = seg.counts;
+    p.v = v;
+    p.y = static_cast<uint16_t*>(y);
+    p.T = seg.T;
+    p.n_adapters = pool.n_adapters;
+    p.h_in = pool.h_in;
+    p.h_out = pool.h_out;
+    p.r_max = pool.r_max;
+    p.timeout_ns = debug_wait_limit_ns();
+    p.inject_stall = debug_inject_stall();
+    // CTAs per tile: up to one per 512 columns of h_in (at most 8). When that would
+    // need more than one wave of two CTAs per SM but the tile rows alone fit in one,
+    // take as many per tile as keep one wave (no near-empty last wave: prefill gets 5),
+    // but not fewer than 2 (one CTA per row makes long chains); with more tile rows than
+    // that (many tenants), 2 per tile, then 1 beyond eight waves
+    int C = (pool.h_in + 511) / 512;
+    C = C < 1 ? 1 : (C > kMaxCluster ? kMaxCluster : C);
+    const long long rows = (long long)max_tiles_for(seg.T, pool.n_adapters) * pool.n_slices;
+    const long long slots = 2LL * device_sm_count();
+    if (rows * C > slots) {
+        if (rows <= slots) {
+            const int c1 = (int)(slots / rows), c2 = C < 2 ? C : 2;
+            C = c1 > c2 ? c1 : c2;
+        } else {
+            C = C < 2 ? C : 2;
+            if (rows * C > 8 * slots) C = 1;
+        }
+    }
     // the tile rows in cost order first (one small CTA, a programmatic dependent), when
-    // there are more rows than one wave of two CTAs per SM holds (else order cannot help)
-    if (order && (long long)max_tiles_for(seg.T, pool.n_adapters) * pool.n_slices <= 2LL * device_sm_count())
-        order = nullptr;
+    // their CTAs need more than one wave of two per SM (else the order cannot help)
+    if (order && rows * C <= slots) order = nullptr;
     if (order) {
         const int mt = max_tiles_for(seg.T, pool.n_adapters);
         cudaLaunchConfig_t cfg = {};
@@ -897,34 +924,6 @@ cudaError_t launch_sgmv(int mode, const void* x, int64_t x_slice_stride, const l
                                                  pool.ranks, pool.r_max, mt, static_cast<int4*>(order));
         if (e != cudaSuccess) return e;
         p.tiles = static_cast<const int4*>(order);
-    }
-    p.counts = seg.counts;
-    p.v = v;
-    p.y = static_cast<uint16_t*>(y);
-    p.T = seg.T;
-    p.n_adapters = pool.n_adapters;
-    p.h_in = pool.h_in;
-    p.h_out = pool.h_out;
-    p.r_max = pool.r_max;
-    p.timeout_ns = debug_wait_limit_ns();
-    p.inject_stall = debug_inject_stall();
-    // CTAs per tile: up to one per 512 columns of h_in (at most 8). When that would
-    // need more than one wave of two CTAs per SM but the tile rows alone fit in one,
-    // take as many per tile as keep one wave (no near-empty last wave: prefill gets 5);
-    // with more tile rows than that (many tenants), 2 per tile, then 1
-    int C = (pool.h_in + 511) / 512;
-    C = C < 1 ? 1 : (C > kMaxCluster ? kMaxCluster : C);
-    {
-        const long long rows = (long long)max_tiles_for(seg.T, pool.n_adapters) * pool.n_slices;
-        const long long slots = 2LL * device_sm_count();
-        if (rows * C > slots) {
-            if (rows <= slots) {
-                C = (int)(slots / rows);
-            } else {
-                C = C < 2 ? C : 2;
-                if (rows * C > 8 * slots) C = 1;
-            }
-        }
     }
     p.csize = C;
     p.kc = ((pool.h_in + C - 1) / C + 127) / 128 * 128;

@@ -739,6 +739,7 @@ def run_fp8(args, dev, stream, hbm_peak, bf16_peak, bf16_sust, peak_src):
         bytes_call = N * K + N * 4 + M * K * 2 + M * N * 2 + lora_bytes
         flops = 2.0 * M * N * K
         t = res["lora"] * 1e-6
+        lib_ref = library_fp8_gemm(dev, stream, sets[0]["x"], Wq, sw, args.fp8_reps)
         out["M"][str(M)] = {
             "us_per_call": res["lora"], "us_per_call_no_lora": res["base"],
             "overhead_vs_no_lora": res["lora"] / res["base"] - 1.0,
@@ -747,9 +748,46 @@ def run_fp8(args, dev, stream, hbm_peak, bf16_peak, bf16_sust, peak_src):
             "attainable_frac": (flops / t) / min(fp8_peak * 1e12, flops / bytes_call * hbm_peak * 1e9),
             "distinct_adapters": int(len(act)), "status_ok": res["lora_status"] == 0 and res["base_status"] == 0,
             "l2": f"x, adapters and y rotate over {R} copies ({R * set_bytes / 2**20:.0f} MiB); W read once per call",
+            "library_base": lib_ref,
         }
         del sets
     return out
+
+
+def library_fp8_gemm(dev, stream, x, Wq, sw, reps):
+    """The base GEMM alone through a library kernel on the same box, as a side
+    comparison for the call without LoRA: torch._scaled_mm on the same E4M3 operands
+    (x quantised per token by this library's quantiser) with per-row and per-channel
+    scales, bf16 out. A library GEMM; nothing of it is on this library's path."""
+    import torch
+
+    from adapter_gemm_builder_b200 import lora as L
+    M, K = x.shape
+    N = Wq.shape[0]
+    xq = torch.empty((M, K), dtype=torch.uint8, device=dev)
+    sx = torch.empty(M, dtype=torch.float32, device=dev)
+    L.fp8_quantize_rows(x, xq, sx)
+    a = xq.view(torch.float8_e4m3fn)
+    b = Wq.view(torch.float8_e4m3fn).t()
+    try:
+        def f():
+            return torch._scaled_mm(a, b, scale_a=sx.view(M, 1), scale_b=sw.view(1, N), out_dtype=torch.bfloat16)
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                f()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            n = max(5, reps)
+            e0.record(stream)
+            for _ in range(n):
+                f()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        us = e0.elapsed_time(e1) / n * 1e3
+        return {"kernel": "torch._scaled_mm, row-wise scales (library GEMM)", "us_per_call": us,
+                "tflops": 2.0 * M * N * K / (us * 1e-6) / 1e12,
+                "note": "same weights back to back: W (235 MB) exceeds L2, x and y stay L2-warm"}
+    except Exception as exc:  # a library without this path on this box: say so
+        return {"kernel": "torch._scaled_mm", "unavailable": str(exc).splitlines()[0][:200]}
 
 
 BF16_CASES = [

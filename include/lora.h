@@ -259,10 +259,11 @@ LORA_API int fp8_quantize_rows(const void* x, int M, int K, uint8_t* xq, float* 
  *   seg: required when pool != NULL (built for these M tokens); may be NULL otherwise.
  *   ws: lora_workspace_size(LORA_OP_FP8_GEMM, M, K, pool) bytes.
  * Limits: K % 16 == 0, N % 8 == 0, M >= 1.
- * Many adapters: when the pool holds more than 16 adapters and M > 16, the
- * adapters' term is not folded into the GEMM's accumulator; the call runs the
- * base GEMM and then the SGMV apply of lora_apply on its output (three
- * launches), so y = bf16(bf16(base) + term).
+ * Many adapters or tokens: when the pool holds more than 16 adapters and
+ * M > 16, or M > 1024, the adapters' term is not folded into the GEMM's
+ * accumulator; the call runs the base GEMM and then the SGMV apply of
+ * lora_apply on its output (three or four launches, the workspace holding the
+ * apply's tile order), so y = bf16(bf16(base) + term).
  * The GEMM is a persistent grid of one CTA per SM whose CTAs wait on one
  * another (the down-projection count, stream-K partials), so all of them must
  * be resident at once: the context needs every SM of the device. Where fewer
