@@ -339,9 +339,22 @@ class _Events:
                                                 ctypes.c_void_p(stream.cuda_stream), 1) == 0
 
 
-def apply_launches(p):
-    """Kernels of this library one lora_apply launches: one (the cluster kernel)."""
-    return 1
+def apply_launches(p, sm_count=None):
+    """Kernels of this library one lora_apply (with its workspace) launches: the cluster
+    kernel, preceded by the tile-ordering kernel when the batch is not decode-like and
+    its clusters need more than one wave of two CTAs per SM (the library's rule)."""
+    from adapter_gemm_builder_b200 import lora as L
+    if p.T <= 64 and p.T <= 2 * p.n_adapters:
+        return 1
+    if sm_count is None:
+        import torch
+        sm_count = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    rows = L.max_tiles(p.T, p.n_adapters) * p.n_slices
+    slots = 2 * sm_count
+    c = min(8, max(1, (p.h_in + 511) // 512))
+    if rows * c > slots:
+        c = max(slots // rows, min(c, 2)) if rows <= slots else (1 if rows * min(c, 2) > 8 * slots else min(c, 2))
+    return 2 if rows * c > slots else 1
 
 
 def time_apply(p, dev, steps, warmup, stream, ext, world=1, clocks=None):
