@@ -292,9 +292,9 @@ __device__ __forceinline__ Seg seg_at(long long u, long long u_end, int KB)
 // 64: 64-byte swizzle), so the shared-memory layouts are the same.
 // kW4 (a weight converter mode, with ESZ 2 and BK 128): the weights arrive as
 // codes -- OCP MX FP4 (packed E2M1 codes and E8M0 block scales) or E4M3 (whose
-// per-channel scale the epilogue applies, as on the 8-bit path) -- and four
+// per-channel scale the epilogue applies, as on the 8-bit path) -- and eight
 // converter warps turn each k-block's codes into the bf16 tile the MMA reads
-// (one row per thread), signalling it on conv[stage].
+// (half a row per thread), signalling it on conv[stage].
 template <int BK, int MAXR, int ESZ, int kW4 = kWcNone>
 __global__ void __launch_bounds__(kW4 != kWcNone ? kThreadsW4 : kThreads, 1)
 fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
@@ -324,7 +324,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
     uint64_t* epibar = drain + 1;               // [1] epilogue-warps barrier
     uint64_t* lready = epibar + 1;              // [1] LoRA operands of the segment built
     uint64_t* stall = lready + 1;               // [1] test hook: never completed
-    uint64_t* conv = stall + 1;                 // [stages] MX FP4: the k-block's bf16 W tile built
+    uint64_t* conv = stall + 1;                 // [stages] converter paths: the k-block's bf16 W tile built
     volatile int* abort_flag = &s_abort;
 
     constexpr int kStageW = kBlockM * BK;

@@ -305,9 +305,10 @@ LORA_API int bf16_gemm_lora_epilogue(const void* x, int M, int K, int N, const v
  *                   + s_a * sum_{j < r_a} v[m][j] * B[0][a][j][n] ),  v = x.A_a.
  * The same weights as fp8_gemm_lora_epilogue (fp8_quantize_rows of W), but x is
  * not quantised: the kernel of bf16_gemm_lora_epilogue, whose weight tiles
- * arrive as E4M3 codes and are turned into bf16 on chip (exactly) by four
- * converter warps before the tcgen05 kind::f16 MMAs; the epilogue applies
- * w_scale as on the 8-bit path.
+ * arrive as E4M3 codes and are turned on chip by eight converter warps into
+ * bf16 tiles holding the codes' values times 2^-112 (exact: each pair goes
+ * through f16) before the tcgen05 kind::f16 MMAs; the epilogue applies
+ * w_scale * 2^112 (in fp32), as the 8-bit path applies w_scale.
  *   x bf16 [M][K]; Wq e4m3 [N][K]; w_scale fp32 [N]; y bf16 [M][N] (out).
  *   pool / seg as for fp8_gemm_lora_epilogue (including its many-adapter path).
  *   ws: lora_workspace_size(LORA_OP_W8A16_GEMM, M, K, pool) bytes.
@@ -344,7 +345,7 @@ LORA_API int mxfp4_quantize_rows(const void* W, int N, int K, uint8_t* Wp, uint8
  *                   + s_a * sum_{j < r_a} v[m][j] * B[0][a][j][n] ),  v = x.A_a.
  * The kernel of bf16_gemm_lora_epilogue, whose weight tiles arrive as packed
  * codes and scales (half the bytes of an 8-bit weight) and are turned into
- * bf16 on chip by four converter warps before the tcgen05 kind::f16 MMAs.
+ * bf16 on chip by eight converter warps before the tcgen05 kind::f16 MMAs.
  *   x bf16 [M][K]; Wp / Wsc as mxfp4_quantize_rows; y bf16 [M][N] (out).
  *   pool / seg as for fp8_gemm_lora_epilogue (including its many-adapter path).
  *   ws: lora_workspace_size(LORA_OP_MXFP4_GEMM, M, K, pool) bytes.
