@@ -64,7 +64,8 @@ def parse_args():
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--fp8-only", action="store_true",
                     help="run only the FP8 GEMM + LoRA section and print its JSON")
-    ap.add_argument("--section", choices=["fp8", "bf16", "w8a16", "mxfp4", "merge"],
+    ap.add_argument("--no-backward", action="store_true", help="skip the FP8 backward section")
+    ap.add_argument("--section", choices=["fp8", "bf16", "w8a16", "mxfp4", "merge", "backward"],
                     help="run only this GEMM / merge section and print its JSON (profiling aid)")
     ap.add_argument("--fp8-m", type=int, nargs="+", default=[16, 64, 256])
     ap.add_argument("--fp8-reps", type=int, default=20, help="graph replays per timing")
@@ -538,6 +539,7 @@ def run_ours(args):
     merge = None if args.no_merge else run_merge(args, dev, stream, hbm_peak, peak_src)
     mxfp4 = None if args.no_mxfp4 else run_mxfp4(args, dev, stream, hbm_peak, bf16_peak, peak_src)
     w8a16 = None if args.no_mxfp4 else run_mxfp4(args, dev, stream, hbm_peak, bf16_peak, peak_src, "w8a16")
+    backward = None if args.no_backward else run_backward(args, dev, stream, hbm_peak, bf16_peak, peak_src)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -554,6 +556,7 @@ def run_ours(args):
             "clocks": t["clocks"], "status_ok": t["status_ok"],
             "cpu_baseline": cpu, "workloads": extras, "fp8_gemm_lora": fp8, "bf16_gemm_lora": bf16,
             "switch_merge": merge, "mxfp4_gemm_lora": mxfp4, "w8a16_gemm_lora": w8a16,
+            "fp8_lora_backward": backward,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -1004,6 +1007,77 @@ MERGE_CASES = [
 ]
 
 
+def run_backward(args, dev, stream, hbm_peak, bf16_peak, peak_src):
+    """The adapters' backward on the frozen 8-bit base (fp8_lora_backward: dX, dA, dB) at
+    the FP8 section's shapes (K 8192, N 28672, 16 adapters of rank 16, Zipf ids): us per
+    call, TFLOP/s of dX's 8-bit GEMM against the FP8 peak, and the HBM fraction of its
+    algorithmic bytes (WqT and swT, x, dY and dX, the adapters read and transposed, dA
+    and dB written in full)."""
+    import numpy as np
+    import torch
+
+    from adapter_gemm_builder_b200 import lora as L
+    from adapter_gemm_builder_b200 import workloads as wl
+    K, N, n_ad, r = 8192, 28672, 16, 16
+    gen = torch.Generator(device=dev).manual_seed(9)
+    Wt = (torch.randn((K, N), generator=gen, device=dev) * (1.0 / math.sqrt(K))).to(torch.bfloat16)
+    WqT = torch.empty((K, N), dtype=torch.uint8, device=dev)
+    swT = torch.empty(K, dtype=torch.float32, device=dev)
+    L.fp8_quantize_rows(Wt, WqT, swT)  # W^T quantised per input channel, once
+    del Wt
+    fp8_peak = 2.0 * bf16_peak
+    out = {"shape": {"K": K, "N": N, "adapters": n_ad, "r": r, "ids": "zipf(1.1)"},
+           "peak_tflops_fp8": fp8_peak, "peak_hbm_gbs": hbm_peak,
+           "peak_source": f"{peak_src}: FP8 = 2 x bf16_tflops (nominal dense ratio)", "M": {}}
+    for M in args.fp8_m:
+        q = wl.fp8_problem(M, K=K, N=N, n_adapters=n_ad, r=r, seed=4, W=np.zeros((1, 1), np.uint16))
+        tb = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+        pool = L.Pool(tb(q.A), tb(q.B), torch.from_numpy(q.ranks).to(dev), torch.from_numpy(q.scales).to(dev))
+        seg = L.Segments(M, n_ad, device=dev)
+        L.lora_build_segments(torch.from_numpy(q.ids).to(dev), n_ad, seg)
+        sets = []
+        for k in range(2):
+            g = torch.Generator(device=dev).manual_seed(100 + k)
+            sets.append(dict(
+                x=tb(q.x), dY=torch.randn((M, N), generator=g, device=dev).to(torch.bfloat16),
+                dX=torch.empty((M, K), dtype=torch.bfloat16, device=dev),
+                dA=torch.empty((n_ad, K, r), device=dev), dB=torch.empty((n_ad, r, N), device=dev),
+                ws=L.workspace(L.LORA_OP_FP8_BACKWARD, M, K, pool, device=dev)))
+
+        def call(d):
+            L.fp8_lora_backward(d["x"], d["dY"], WqT, swT, pool, seg, d["dX"], d["dA"], d["dB"], d["ws"])
+        with torch.cuda.stream(stream):
+            for d in sets:
+                call(d)
+            stream.synchronize()
+            gr = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gr, stream=stream):
+                for d in sets:
+                    call(d)
+            for _ in range(3):
+                gr.replay()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for _ in range(args.fp8_reps):
+                gr.replay()
+            b.record(stream)
+        torch.cuda.synchronize()
+        us = a.elapsed_time(b) / (args.fp8_reps * len(sets)) * 1e3
+        status = max(L.lora_workspace_status(d["ws"])[0] for d in sets)
+        act = int(len(np.unique(q.ids)))
+        bytes_call = (K * N + K * 4 + M * N * 2 + M * K * 2 * 2 + act * r * (K + N) * 2 * 3
+                      + n_ad * r * (K + N) * 4)
+        flops = 2.0 * M * N * K
+        t = us * 1e-6
+        out["M"][str(M)] = {"us_per_call": us, "tflops": flops / t / 1e12,
+                            "tensor_frac": flops / t / 1e12 / fp8_peak,
+                            "hbm_gbs": bytes_call / t / 1e9, "hbm_frac": bytes_call / t / 1e9 / hbm_peak,
+                            "status_ok": status == 0,
+                            "l2": "two input sets; WqT (235 MB) read once per call"}
+        del sets
+    return out
+
+
 def run_merge(args, dev, stream, hbm_peak, peak_src):
     """Token-wise merge of the router-selected adapters into the backbone
     (lora_switch_merge): GB/s of algorithmic bytes (W read, W_out written, the
@@ -1071,7 +1145,8 @@ def main():
                "bf16": lambda: run_bf16(args, dev, st, hbm, bf16, src),
                "mxfp4": lambda: run_mxfp4(args, dev, st, hbm, bf16, src),
                "w8a16": lambda: run_mxfp4(args, dev, st, hbm, bf16, src, "w8a16"),
-               "merge": lambda: run_merge(args, dev, st, hbm, src)}[args.section]
+               "merge": lambda: run_merge(args, dev, st, hbm, src),
+               "backward": lambda: run_backward(args, dev, st, hbm, bf16, src)}[args.section]
         print(json.dumps(run()))
         return
     if args.fp8_only:

@@ -199,3 +199,15 @@ def test_fp8_gemm_lora_ids_without_adapter(kind):
     cols = np.tile(np.arange(N), M).astype(np.int32)
     want = _oracle_fp8(p, Wq_o, sw_o, rows, cols, True).reshape(M, N)
     assert_close(f64(host_bf16_bits(y)), want, TOL_FP8, f"fp8 ids {kind}")
+
+
+def test_fp8_gemm_lora_many_tokens_split_path():
+    """More than 1024 tokens: the call runs the base GEMM, then the SGMV apply on its
+    output with the tile rows in cost order from the GEMM workspace; y = bf16(bf16(base)
+    + term), within the FP8 bar on every element."""
+    M, K, N = 1100, 256, 264
+    p, Wq, sw, y = _fp8_case(M, K, N, n_adapters=6, r=16, seed=17, none_frac=0.1)
+    rows = np.repeat(np.arange(M), N).astype(np.int32)
+    cols = np.tile(np.arange(N), M).astype(np.int32)
+    want = _oracle_fp8(p, Wq, sw, rows, cols, True).reshape(M, N)
+    assert_close(f64(y), want, TOL_FP8, "fp8 split path, 1100 tokens")
