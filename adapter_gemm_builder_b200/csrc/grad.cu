@@ -11,7 +11,8 @@
 // thread l keeps the r_a sums of one row of the output and walks the adapter's
 // tokens, 32 at a time: the tokens' short vectors (u or v, fp32) are staged in
 // shared memory and each thread reads its token rows' bf16 element of x or dY
-// (coalesced across the block). Bound by HBM: x or dY rows of the adapter's
+// (coalesced across the block; eight tokens' loads are issued before their
+// FMAs, so their latencies overlap). Bound by HBM: x or dY rows of the adapter's
 // tokens in, the gradient rows out.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -38,12 +39,13 @@ struct GradParams {
     int L, r_max, n_adapters;
 };
 
-// kRowMajorLong: the output is [L][r_max] (dA); else [r_max][L] (dB).
-template <bool kRowMajorLong>
+// kRowMajorLong: the output is [L][r_max] (dA); else [r_max][L] (dB). MAXR: the
+// pool's r_max rounded up to 16 or 64 (the sums a thread keeps).
+template <bool kRowMajorLong, int MAXR>
 __global__ void __launch_bounds__(kGThreads)
 grad_outer_kernel(const GradParams p)
 {
-    __shared__ float s_short[kTokChunk][64];
+    __shared__ float s_short[kTokChunk][MAXR];
     __shared__ int s_tok[kTokChunk];
     ptx::pdl_wait();  // the shrinks that produced u / v come first in the stream
     const int slot = blockIdx.y;
@@ -54,25 +56,33 @@ grad_outer_kernel(const GradParams p)
     const float s = p.scales ? p.scales[a] : 1.f;
     const int l = blockIdx.x * kGThreads + threadIdx.x;
     const int t0 = p.indptr[a], t1 = p.indptr[a + 1];
-    float acc[64];
+    float acc[MAXR];
 #pragma unroll
-    for (int j = 0; j < 64; ++j) acc[j] = 0.f;
+    for (int j = 0; j < MAXR; ++j) acc[j] = 0.f;
     for (int c0 = t0; c0 < t1; c0 += kTokChunk) {
         const int nc = min(kTokChunk, t1 - c0);
         __syncthreads();  // the previous chunk's short vectors are consumed
         if (threadIdx.x < nc) s_tok[threadIdx.x] = p.perm[c0 + threadIdx.x];
         __syncthreads();
-        for (int i = threadIdx.x; i < nc * 64; i += kGThreads) {
-            const int t = i >> 6, j = i & 63;
+        for (int i = threadIdx.x; i < nc * MAXR; i += kGThreads) {
+            const int t = i / MAXR, j = i % MAXR;
             s_short[t][j] = j < r ? p.shrt[(size_t)s_tok[t] * p.r_max + j] : 0.f;
         }
         __syncthreads();
         if (l < p.L) {
-            for (int t = 0; t < nc; ++t) {
-                const float lv = __uint_as_float((uint32_t)p.lng[(size_t)s_tok[t] * p.L + l] << 16);
+            // eight tokens at a time: their long elements first (independent loads, in
+            // flight together), then the FMAs (columns past the rank hold zeros)
+            for (int t0 = 0; t0 < nc; t0 += 8) {
+                float lv[8];
 #pragma unroll
-                for (int j = 0; j < 64; ++j)
-                    if (j < p.r_max) acc[j] = fmaf(lv, s_short[t][j], acc[j]);
+                for (int u = 0; u < 8; ++u)
+                    lv[u] = t0 + u < nc ? __uint_as_float((uint32_t)p.lng[(size_t)s_tok[t0 + u] * p.L + l] << 16)
+                                        : 0.f;
+#pragma unroll
+                for (int u = 0; u < 8; ++u)
+                    if (t0 + u < nc)
+#pragma unroll
+                        for (int j = 0; j < MAXR; ++j) acc[j] = fmaf(lv[u], s_short[t0 + u][j], acc[j]);
             }
         }
     }
@@ -81,13 +91,13 @@ grad_outer_kernel(const GradParams p)
     if (kRowMajorLong) {
         float4* o = reinterpret_cast<float4*>(p.out + ((size_t)a * p.L + l) * p.r_max);
 #pragma unroll
-        for (int j = 0; j < 64; j += 4)
+        for (int j = 0; j < MAXR; j += 4)
             if (j < p.r_max)
                 o[j >> 2] = make_float4(j < r ? s * acc[j] : 0.f, j + 1 < r ? s * acc[j + 1] : 0.f,
                                         j + 2 < r ? s * acc[j + 2] : 0.f, j + 3 < r ? s * acc[j + 3] : 0.f);
     } else {
 #pragma unroll
-        for (int j = 0; j < 64; ++j)
+        for (int j = 0; j < MAXR; ++j)
             if (j < p.r_max) p.out[((size_t)a * p.r_max + j) * p.L + l] = j < r ? s * acc[j] : 0.f;
     }
 }
@@ -169,8 +179,10 @@ cudaError_t launch_grad_outer(bool row_major_long, const void* lng, const float*
     p.n_adapters = pool.n_adapters;
     const dim3 grid((unsigned)((L + kGThreads - 1) / kGThreads), (unsigned)pool.n_adapters, 1);
     void* args[] = {&p};
-    return launch_pdl(row_major_long ? (const void*)grad_outer_kernel<true> : (const void*)grad_outer_kernel<false>,
-                      grid, args, stream);
+    const bool r16 = pool.r_max <= 16;
+    const void* kern = row_major_long ? (r16 ? (const void*)grad_outer_kernel<true, 16> : (const void*)grad_outer_kernel<true, 64>)
+                                      : (r16 ? (const void*)grad_outer_kernel<false, 16> : (const void*)grad_outer_kernel<false, 64>);
+    return launch_pdl(kern, grid, args, stream);
 }
 
 }  // namespace lora
