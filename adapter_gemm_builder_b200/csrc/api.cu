@@ -457,9 +457,19 @@ int fp8_lora_backward(const void* x, const void* dY, int M, int K, int N, const 
     //    (quantised per input channel) and the transposed pool; its workspace leads
     st = gemm_lora_launch(1, dY, M, N, K, WqT, swT, &pt, seg, dX, w, off_at, stream);
     if (st != LORA_OK) return st;
-    // 4. u = dY.B^T and v = x.A per token, then dA = s x^T u and dB = s v^T dY per adapter
-    if (launch_sgmv(SGMV_SHRINK, dY, 0, pt, *seg, u, nullptr, s, false) != cudaSuccess ||
-        launch_sgmv(SGMV_SHRINK, x, 0, *pool, *seg, v, nullptr, s, false) != cudaSuccess ||
+    // 4. u = dY.B^T per token: the GEMM's own down-projection when it folded the adapters
+    //    into its accumulator (summed from its workspace copies), else a shrink of dY
+    cudaError_t eu;
+    if (!gemm_split(M, &pt)) {
+        size_t g_xq, g_sx, g_v, g_sync, g_part;
+        fp8_ws_layout(M, N, &pt, &g_xq, &g_sx, &g_v, &g_sync, &g_part, 1);
+        eu = launch_gather_u(reinterpret_cast<const float*>(w + g_v), fp8_gemm_v_copies(M), *seg, M, pool->r_max, u, s);
+    } else {
+        eu = launch_sgmv(SGMV_SHRINK, dY, 0, pt, *seg, u, nullptr, s, false);
+    }
+    if (eu != cudaSuccess) return LORA_ERR_CUDA;
+    // 5. v = x.A per token, then dA = s x^T u and dB = s v^T dY per adapter
+    if (launch_sgmv(SGMV_SHRINK, x, 0, *pool, *seg, v, nullptr, s, false) != cudaSuccess ||
         launch_grad_outer(true, x, u, K, *pool, *seg, dA, s) != cudaSuccess ||
         launch_grad_outer(false, dY, v, N, *pool, *seg, dB, s) != cudaSuccess)
         return LORA_ERR_CUDA;

@@ -129,6 +129,25 @@ transpose_pool_kernel(const uint16_t* A, const uint16_t* B, uint16_t* At, uint16
     ptx::pdl_launch_dependents();
 }
 
+// u[t][j] = sum_c vg[c][pos][j] for the token t = perm[pos] of every position with an
+// adapter: the down-projection the backward's fused GEMM already computed (dY.B^T
+// with the transposed pool, in its workspace as v_rep partial copies in segment
+// order), so no second shrink of dY is needed.
+__global__ void __launch_bounds__(kGThreads)
+gather_u_kernel(const float* vg, int v_rep, const int32_t* perm, const int32_t* counts, int M, int r_max, float* u)
+{
+    ptx::pdl_wait();  // the GEMM wrote vg
+    const int n_valid = counts[0];
+    const int i = blockIdx.x * kGThreads + threadIdx.x;
+    const int pos = i / r_max, j = i - pos * r_max;
+    if (pos < n_valid && pos < M) {
+        float acc = 0.f;
+        for (int c = 0; c < v_rep; ++c) acc += vg[((size_t)c * M + pos) * r_max + j];
+        u[(size_t)perm[pos] * r_max + j] = acc;
+    }
+    ptx::pdl_launch_dependents();
+}
+
 cudaError_t launch_pdl(const void* kern, dim3 grid, void** args, cudaStream_t stream)
 {
     cudaLaunchConfig_t cfg = {};
@@ -159,6 +178,17 @@ cudaError_t launch_transpose_pool(const lora_pool_t& pool, const lora_segments_t
     int k = K, n = N, r = pool.r_max;
     void* args[] = {&A, &B, &at, &bt, &active, &counts, &k, &n, &r};
     return launch_pdl((const void*)transpose_pool_kernel, grid, args, stream);
+}
+
+cudaError_t launch_gather_u(const float* vg, int v_rep, const lora_segments_t& seg, int M, int r_max, float* u,
+                            cudaStream_t stream)
+{
+    const dim3 grid((unsigned)(((long long)M * r_max + kGThreads - 1) / kGThreads), 1, 1);
+    const int32_t* perm = seg.perm;
+    const int32_t* counts = seg.counts;
+    int m = M, r = r_max;
+    void* args[] = {&vg, &v_rep, &perm, &counts, &m, &r, &u};
+    return launch_pdl((const void*)gather_u_kernel, grid, args, stream);
 }
 
 cudaError_t launch_grad_outer(bool row_major_long, const void* lng, const float* shrt, int L,

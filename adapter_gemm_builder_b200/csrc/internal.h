@@ -35,6 +35,10 @@ cudaError_t launch_lora_switch_merge(const void* W, int N, int K, const lora_poo
 // dB_a = s_a v_a^T dY_a ([r_max][N]) of the active adapters.
 cudaError_t launch_transpose_pool(const lora_pool_t& pool, const lora_segments_t& seg, void* At, void* Bt,
                                   cudaStream_t stream);
+// u[perm[pos]][j] = sum over the v_rep copies of vg[c][pos][j] (the fused GEMM's
+// down-projection, segment order) for every position with an adapter (grad.cu).
+cudaError_t launch_gather_u(const float* vg, int v_rep, const lora_segments_t& seg, int M, int r_max, float* u,
+                            cudaStream_t stream);
 cudaError_t launch_grad_outer(bool row_major_long, const void* lng, const float* shrt, int L,
                               const lora_pool_t& pool, const lora_segments_t& seg, float* out, cudaStream_t stream);
 
