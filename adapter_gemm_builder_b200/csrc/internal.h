@@ -24,6 +24,11 @@ cudaError_t launch_sgmv(int mode, const void* x, int64_t x_slice_stride, const l
                         const lora_segments_t& seg, float* v, void* y, cudaStream_t stream,
                         bool pdl_trigger, void* order = nullptr);
 size_t sgmv_order_bytes(int T, int n_adapters);
+// The expand on the tcgen05 tensor cores (sgmv_tc.cu) for batches of long segments:
+// whether a batch qualifies, and the launch (v fp32 [n_slices][T][r_max], y in place).
+bool sgmv_expand_tc_eligible(int T, const lora_pool_t& pool);
+cudaError_t launch_sgmv_expand_tc(const float* v, const lora_pool_t& pool, const lora_segments_t& seg, void* y,
+                                  cudaStream_t stream);
 
 // Token-wise merge of the selected adapters into the backbone (merge.cu).
 cudaError_t launch_lora_switch_merge(const void* W, int N, int K, const lora_pool_t& pool, const int32_t* sel,

@@ -341,12 +341,15 @@ class _Events:
 
 
 def apply_launches(p, sm_count=None):
-    """Kernels of this library one lora_apply (with its workspace) launches: the cluster
+    """Kernels of this library one lora_apply (with its workspace) launches: for a batch
+    of long segments the shrink and the tensor-core expand; otherwise the cluster
     kernel, preceded by the tile-ordering kernel when the batch is not decode-like and
-    its clusters need more than one wave of two CTAs per SM (the library's rule)."""
+    its clusters need more than one wave of two CTAs per SM (the library's rules)."""
     from adapter_gemm_builder_b200 import lora as L
     if p.T <= 64 and p.T <= 2 * p.n_adapters:
         return 1
+    if p.T >= 32 * p.n_adapters and p.h_out >= 128:
+        return 2
     if sm_count is None:
         import torch
         sm_count = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count

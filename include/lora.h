@@ -153,8 +153,10 @@ LORA_API int lora_segments_status(const lora_segments_t* seg, lora_stream_t stre
  * for invalid arguments. For LORA_OP_FP8_GEMM, T is the
  * token count M and `K` the GEMM's reduction size; `pool` may be NULL (no
  * LoRA). LORA_OP_APPLY needs a valid pool; it returns 0 for a decode-like
- * batch (lora_tile_tokens_for) and otherwise the bytes of the tile rows in cost
- * order (16 per row of lora_max_tiles). The other operations ignore K.
+ * batch (lora_tile_tokens_for), for a batch of long segments (T >= 32 *
+ * n_adapters, h_out >= 128) the bytes of v in fp32 (n_slices * T * r_max * 4,
+ * rounded up to 256; see lora_apply), and otherwise the bytes of the tile rows
+ * in cost order (16 per row of lora_max_tiles). The other operations ignore K.
  * A workspace must be zeroed once after allocation (lora_workspace_init);
  * afterwards the library keeps it in a reusable state.
  */
@@ -209,7 +211,11 @@ LORA_API int lora_shrink(const void* x, int64_t x_slice_stride, const lora_pool_
  *   y[s][t][n] = bf16( fp32(y[s][t][n]) + s_a * sum_{j < r_a} v[s][t][j] * B[s][a][j][n] )
  * (one rounding, to nearest even); rows of tokens without an adapter are untouched.
  *   v  fp32 [n_slices][T][r_max];  y bf16 [n_slices][T][h_out] (in/out).
- * Needs no workspace. One kernel launch.
+ * Needs no workspace. One kernel launch: for a batch of long segments (not
+ * decode-like, T >= 32 * n_adapters, h_out >= 128) the tcgen05 expand (the
+ * 128-column blocks of every tile row as MMAs with B_a read in place by TMA
+ * and v split into bf16 halves hi + lo, so ~16 bits of v; the grid's CTAs
+ * take equal runs of (tile row, slice, block)), else the cluster SGMV kernel.
  */
 LORA_API int lora_expand(const float* v, const lora_pool_t* pool, const lora_segments_t* seg, void* y,
                 void* ws, size_t ws_bytes, lora_stream_t stream);
@@ -227,6 +233,12 @@ LORA_API int lora_expand(const float* v, const lora_pool_t* pool, const lora_seg
  * its tile rows into ws in descending cost (rows of more than four tokens, then
  * by descending rank), so that the long rows start first; the results are the
  * same either way. ws NULL: one launch, table order.
+ * A batch of long segments (as for lora_expand's tensor-core path) with a
+ * workspace of lora_workspace_size(LORA_OP_APPLY, ...) bytes instead runs the
+ * shrink into the workspace (v fp32 [n_slices][T][r_max]) and then the
+ * tcgen05 expand as its programmatic dependent: two launches, the same
+ * results up to fp32 rounding order. With a smaller workspace (at least the
+ * tile-order bytes) such a batch takes the cluster kernel.
  */
 LORA_API int lora_apply(const void* x, int64_t x_slice_stride, const lora_pool_t* pool,
                const lora_segments_t* seg, void* y, void* ws, size_t ws_bytes,

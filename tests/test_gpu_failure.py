@@ -78,6 +78,26 @@ def test_sgmv_shrink_wait_runs_out_then_next_call_is_correct():
     assert_close(v.cpu().numpy()[0][has].astype(np.float64), want[has], TOL_BF16, "shrink")
 
 
+def test_sgmv_tc_expand_wait_runs_out_then_next_call_is_correct():
+    # 300 tokens on 3 adapters: long segments, so lora_expand runs the tensor-core expand
+    # (its stalled CTA drains its copies and MMAs and releases TMEM before it leaves)
+    p = wl.make_lora_problem("t", 13, T=300, n_adapters=3, h_in=256, h_out=392, r_max=32,
+                             ids_kind="zipf", none_frac=0.1, rank_choices=(5, 32))
+    d = DeviceProblem(p)
+    rng = np.random.default_rng(13)
+    v = rng.standard_normal((1, p.T, p.r_max)).astype(np.float32)
+    y = d.y_in()
+    _stalled(lambda: L.lora_expand(dev(v), d.pool, d.seg, y))
+    st, detail = L.lora_segments_status(d.seg)
+    assert st == L.LORA_ERR_TIMEOUT and detail & SGMV_WAIT_BITS, hex(detail)
+    y = d.y_in()
+    L.lora_expand(dev(v), d.pool, d.seg, y)
+    torch.cuda.synchronize()
+    assert L.lora_segments_status(d.seg)[0] == L.LORA_OK
+    want = oracle.lora_expand(v[0], p.B[0], p.ranks, p.scales, p.ids, p.y_in[0])
+    assert_close(f64(host_bf16_bits(y))[0], want, TOL_BF16, "tc expand after a timeout")
+
+
 def test_fp8_gemm_wait_runs_out_then_next_call_is_correct():
     M, K, N = 64, 512, 640
     rng = np.random.default_rng(5)

@@ -389,3 +389,101 @@ def test_apply_tile_order_same_results_and_cost_order(ids_kind):
     got = ws[: tiles.size * 4].view(torch.int32).cpu().numpy().reshape(-1, 4)
     assert np.array_equal(got, _expected_order(tiles, n_used, p.ranks, p.r_max))
     assert_close(f64(host_bf16_bits(y1)), oracle_apply(p), TOL_BF16, f"ordered apply {ids_kind}")
+
+
+# ------------------------------------------------------------------ tensor-core expand (long segments)
+
+# Batches of long segments (on average half a tile or more per adapter, h_out >= 128):
+# lora_expand runs the tcgen05 expand, and lora_apply with its workspace runs the shrink
+# into the workspace and then that expand. Ragged column blocks, ranks that are not
+# multiples of 16, a pool padded to 8 (rank rows past the box), several slices, gathered
+# and pre-sorted tokens, tiles whose token count is not a multiple of 16.
+TC_CASES = {
+    "tc_ragged_mixed": dict(seed=61, T=400, n_adapters=6, h_in=264, h_out=392, r_max=32),
+    "tc_rank64_slices": dict(seed=62, T=600, n_adapters=9, h_in=320, h_out=520, r_max=64,
+                             rank_choices=(8, 16, 40, 48, 64), n_slices=3),
+    "tc_rank8_pool": dict(seed=63, T=200, n_adapters=4, h_in=256, h_out=136, r_max=8,
+                          rank_choices=(3, 8)),
+    "tc_sorted_long": dict(seed=64, T=700, n_adapters=2, h_in=512, h_out=1024, r_max=16,
+                           rank_choices=(16,), kind="sorted_zipf", none_frac=0.0),
+    "tc_uniform_partial": dict(seed=65, T=130, n_adapters=4, h_in=128, h_out=264, r_max=16,
+                               rank_choices=(1, 16), kind="uniform"),
+}
+
+
+def test_tc_cases_take_the_tensor_core_path():
+    """The workspace of lora_apply on these batches holds v (fp32, every slice)."""
+    for case, kw in TC_CASES.items():
+        p = _small(**kw)
+        d = DeviceProblem(p, build=False)
+        n = L.lora_workspace_size(L.LORA_OP_APPLY, p.T, 0, d.pool)
+        assert n == -(-p.n_slices * p.T * p.r_max * 4 // 256) * 256, case
+
+
+@pytest.mark.parametrize("case", list(TC_CASES))
+def test_expand_tc_parity(case):
+    p = _small(**TC_CASES[case])
+    d = DeviceProblem(p)
+    rng = np.random.default_rng(7)
+    v = rng.standard_normal((p.n_slices, p.T, p.r_max)).astype(np.float32)
+    y = d.y_in()
+    L.lora_expand(dev(v), d.pool, d.seg, y)
+    torch.cuda.synchronize()
+    assert L.lora_segments_status(d.seg)[0] == L.LORA_OK
+    got = f64(host_bf16_bits(y))
+    for s in range(p.n_slices):
+        want = oracle.lora_expand(v[s], p.B[s], p.ranks, p.scales, p.ids, p.y_in[s])
+        assert_close(got[s], want, TOL_BF16, f"{case} slice {s}")
+    none = p.ids == -1
+    assert np.array_equal(host_bf16_bits(y)[:, none], p.y_in[:, none])
+
+
+@pytest.mark.parametrize("case", list(TC_CASES))
+@pytest.mark.parametrize("ws", [None, False], ids=["shrink+tc_expand", "cluster"])
+def test_apply_tc_parity(case, ws):
+    p = _small(**TC_CASES[case])
+    d = DeviceProblem(p)
+    y = d.y_in()
+    L.lora_apply(d.x, d.pool, d.seg, y, ws=ws)
+    torch.cuda.synchronize()
+    assert L.lora_segments_status(d.seg)[0] == L.LORA_OK
+    assert_close(f64(host_bf16_bits(y)), oracle_apply(p), TOL_BF16, case)
+    none = p.ids == -1
+    assert np.array_equal(host_bf16_bits(y)[:, none], p.y_in[:, none])
+
+
+def test_apply_tc_exact_small_integers():
+    """Small integers through the shrink and the tensor-core expand: v is an integer
+    below 2^16, which its two bf16 halves hold exactly, every product and sum is exact
+    in fp32, so y must be the exact value rounded once to bf16."""
+    rng = np.random.default_rng(66)
+    T, n_adapters, h_in, h_out, r_max = 300, 3, 1024, 392, 16
+    p = _small(66, T=T, n_adapters=n_adapters, h_in=h_in, h_out=h_out, r_max=r_max,
+               rank_choices=(5, 16))
+    p.x[:] = wl.to_bf16_bits(rng.integers(-2, 3, size=p.x.shape).astype(np.float32))
+    for a in range(n_adapters):
+        r = p.ranks[a]
+        p.A[:, a, :, :r] = wl.to_bf16_bits(rng.integers(-2, 3, size=(1, h_in, r)).astype(np.float32))
+        p.B[:, a, :r, :] = wl.to_bf16_bits(rng.integers(-2, 3, size=(1, r, h_out)).astype(np.float32))
+    p.y_in[:] = wl.to_bf16_bits(rng.integers(-8, 9, size=p.y_in.shape).astype(np.float32))
+    p.scales[:] = 0.5
+    d = DeviceProblem(p)
+    y = d.y_in()
+    L.lora_apply(d.x, d.pool, d.seg, y)
+    torch.cuda.synchronize()
+    assert np.array_equal(host_bf16_bits(y), rne_bf16_bits(oracle_apply(p)))
+
+
+@pytest.mark.parametrize("ws", [None, False], ids=["shrink+tc_expand", "cluster"])
+def test_sgmv_prefill_both_paths_sampled_tokens(ws):
+    p = wl.sgmv_prefill()
+    d = DeviceProblem(p)
+    y = d.y_in()
+    L.lora_apply(d.x, d.pool, d.seg, y, ws=ws)
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(1)
+    rows = np.sort(rng.choice(p.T, size=160, replace=False))
+    starts = np.concatenate([[0], np.cumsum(np.bincount(p.ids))])
+    rows = np.unique(np.concatenate([rows, starts[:-1], starts[1:] - 1]))
+    got = f64(host_bf16_bits(y))[:, rows]
+    assert_close(got, oracle_apply(p, rows=rows), TOL_BF16, "sgmv_prefill")

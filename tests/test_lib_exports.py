@@ -78,6 +78,15 @@ def test_workspace_sizes(lib):
     # a general batch: the tile rows in cost order, 16 bytes per row of lora_max_tiles
     n = lib.lora_workspace_size(L.LORA_OP_APPLY, 512, 0, ctypes.byref(pa))
     assert n >= 16 * lib.lora_max_tiles(512, 256) and n % 256 == 0
+    # long segments (T >= 32 n_adapters, h_out >= 128): v in fp32 for the shrink and the
+    # tensor-core expand, n_slices x T x r_max x 4 bytes rounded up to 256
+    pl = _pool(n_slices=2, n_adapters=8, h_in=4096, h_out=11008, r_max=64)
+    assert lib.lora_workspace_size(L.LORA_OP_APPLY, 2704, 0, ctypes.byref(pl)) == -(-2 * 2704 * 64 * 4 // 256) * 256
+    # ... but not with a narrow y (h_out < 128) or fewer tokens per adapter
+    assert lib.lora_workspace_size(L.LORA_OP_APPLY, 2704, 0, ctypes.byref(_pool(n_adapters=8, h_out=120))) \
+        == -(-16 * lib.lora_max_tiles(2704, 8) // 256) * 256
+    assert lib.lora_workspace_size(L.LORA_OP_APPLY, 255, 0, ctypes.byref(_pool(n_adapters=8, h_out=256))) \
+        == -(-16 * lib.lora_max_tiles(255, 8) // 256) * 256
     p = _pool(h_in=8192, h_out=28672)
     n = lib.lora_workspace_size(L.LORA_OP_FP8_GEMM, 256, 8192, ctypes.byref(p))
     assert n >= 256 + 256 * 8192 + 256 * 4 + 256 * 16 * 4
