@@ -22,12 +22,10 @@ int cuda_status(cudaError_t e) { return e == cudaSuccess ? LORA_OK : LORA_ERR_CU
 
 size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
-// fp32 v [n_slices][T][r_max] of lora_apply's two-launch path (at least the tile-order bytes)
-size_t apply_v_bytes(int T, const lora_pool_t& pool)
+// `parts` planes of fp32 v [n_slices][T][r_max] for lora_apply's two-launch path
+size_t apply_v_bytes(int T, const lora_pool_t& pool, int parts)
 {
-    const size_t v = (size_t)pool.n_slices * T * pool.r_max * 4;
-    const size_t o = sgmv_order_bytes(T, pool.n_adapters);
-    return v > o ? v : o;
+    return (size_t)parts * pool.n_slices * T * pool.r_max * 4;
 }
 
 // Checks shared by every call that reads the pool.
@@ -284,7 +282,11 @@ size_t lora_workspace_size(int op, int T, int K, const lora_pool_t* pool)
         if (!pool || check_pool(pool) != LORA_OK) return (size_t)-1;
         if (T == 0 || tile_tokens_for(T, pool->n_adapters) <= LORA_DECODE_TILE_TOKENS) return 0;
         // long segments: v through the workspace (shrink, then the tensor-core expand)
-        if (sgmv_expand_tc_eligible(T, *pool)) return align256(apply_v_bytes(T, *pool));
+        if (sgmv_expand_tc_eligible(T, *pool)) {
+            const size_t v = apply_v_bytes(T, *pool, sgmv_shrink_tc_parts(*pool));
+            const size_t o = sgmv_order_bytes(T, pool->n_adapters);
+            return align256(v > o ? v : o);
+        }
         return align256(sgmv_order_bytes(T, pool->n_adapters));
     case LORA_OP_FP8_BACKWARD: {
         if (!pool || check_pool(pool) != LORA_OK || T < 1) return (size_t)-1;
@@ -386,7 +388,7 @@ int lora_expand(const float* v, const lora_pool_t* pool, const lora_segments_t* 
     if (seg->T == 0) return LORA_OK;
     if (!v || !aligned16(v) || !y || !aligned16(y)) return LORA_ERR_INVALID_ARG;
     if (sgmv_expand_tc_eligible(seg->T, *pool))  // long segments: the tensor-core expand
-        return cuda_status(launch_sgmv_expand_tc(v, *pool, *seg, y, (cudaStream_t)stream));
+        return cuda_status(launch_sgmv_expand_tc(v, 1, *pool, *seg, y, (cudaStream_t)stream));
     return cuda_status(launch_sgmv(SGMV_EXPAND, nullptr, 0, *pool, *seg, const_cast<float*>(v), y,
                                    (cudaStream_t)stream, false));
 }
@@ -404,14 +406,25 @@ int lora_apply(const void* x, int64_t x_slice_stride, const lora_pool_t* pool,
     cudaStream_t s = (cudaStream_t)stream;
     // one tile row per thread-block cluster, v exchanged on chip; with a workspace, a
     // general batch's tile rows run in descending cost (a small ordering kernel first)
-    // long segments with room for v in the workspace: the shrink, then the tensor-core
-    // expand as its programmatic dependent
-    if (ws && sgmv_expand_tc_eligible(seg->T, *pool) && ws_bytes >= apply_v_bytes(seg->T, *pool) &&
+    // long segments with room for v in the workspace: the shrink into planes of v (on the
+    // tensor cores; with room for one plane only, or if the pool's tensor map is refused,
+    // the cluster shrink), then the tensor-core expand as its programmatic dependent
+    if (ws && sgmv_expand_tc_eligible(seg->T, *pool) && ws_bytes >= apply_v_bytes(seg->T, *pool, 1) &&
         aligned16(ws)) {
         float* v = static_cast<float*>(ws);
-        const cudaError_t e = launch_sgmv(SGMV_SHRINK, x, x_slice_stride, *pool, *seg, v, nullptr, s, false);
-        if (e != cudaSuccess) return cuda_status(e);
-        return cuda_status(launch_sgmv_expand_tc(v, *pool, *seg, y, s));
+        const int parts = sgmv_shrink_tc_parts(*pool);
+        int planes = 0;
+        if (ws_bytes >= apply_v_bytes(seg->T, *pool, parts)) {
+            const cudaError_t e = launch_sgmv_shrink_tc(x, x_slice_stride, *pool, *seg, v, parts, s);
+            if (e == cudaSuccess) planes = parts;
+            else if (e != cudaErrorInvalidValue) return cuda_status(e);
+        }
+        if (planes == 0) {
+            const cudaError_t e = launch_sgmv(SGMV_SHRINK, x, x_slice_stride, *pool, *seg, v, nullptr, s, false);
+            if (e != cudaSuccess) return cuda_status(e);
+            planes = 1;
+        }
+        return cuda_status(launch_sgmv_expand_tc(v, planes, *pool, *seg, y, s));
     }
     void* order = nullptr;
     if (ws && tile_tokens_for(seg->T, pool->n_adapters) > LORA_DECODE_TILE_TOKENS) {

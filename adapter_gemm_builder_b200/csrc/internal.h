@@ -26,9 +26,16 @@ cudaError_t launch_sgmv(int mode, const void* x, int64_t x_slice_stride, const l
 size_t sgmv_order_bytes(int T, int n_adapters);
 // The expand on the tcgen05 tensor cores (sgmv_tc.cu) for batches of long segments:
 // whether a batch qualifies, and the launch (v fp32 [n_slices][T][r_max], y in place).
+// v may come as v_parts planes of [n_slices][T][r_max] (the shrink below) that the
+// expand sums in plane order.
 bool sgmv_expand_tc_eligible(int T, const lora_pool_t& pool);
-cudaError_t launch_sgmv_expand_tc(const float* v, const lora_pool_t& pool, const lora_segments_t& seg, void* y,
-                                  cudaStream_t stream);
+cudaError_t launch_sgmv_expand_tc(const float* v, int v_parts, const lora_pool_t& pool, const lora_segments_t& seg,
+                                  void* y, cudaStream_t stream);
+// The shrink on the tensor cores for the same batches, into `parts` planes of v (at most
+// sgmv_shrink_tc_parts(pool)); cudaErrorInvalidValue if the pool's tensor map is refused.
+int sgmv_shrink_tc_parts(const lora_pool_t& pool);
+cudaError_t launch_sgmv_shrink_tc(const void* x, int64_t x_slice_stride, const lora_pool_t& pool,
+                                  const lora_segments_t& seg, float* v, int parts, cudaStream_t stream);
 
 // Token-wise merge of the selected adapters into the backbone (merge.cu).
 cudaError_t launch_lora_switch_merge(const void* W, int N, int K, const lora_pool_t& pool, const int32_t* sel,

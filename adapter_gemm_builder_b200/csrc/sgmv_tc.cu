@@ -54,9 +54,12 @@ constexpr int kTcBBytes = (kTcBlockN / 64) * 64 * 128;  // 64-column boxes of up
 constexpr int kTcYBytes = kTT * kTcBlockN * 2;          // the tile's y rows of one block
 constexpr int kTcStageBytes = kTcBBytes + kTcYBytes;
 constexpr int kTcTmemCols = 2 * kTcBlockN;              // two accumulators
+constexpr int kTcMaxPlanes = 8;                         // planes of v the expand sums
 
 struct TcExpandParams {
-    const float* v;
+    const float* v;        // v_parts planes of v, v_part_stride floats apart; v is their sum
+    long long v_part_stride;
+    int v_parts;
     uint16_t* y;
     const int32_t* ranks;
     const float* scales;
@@ -337,30 +340,33 @@ sgmv_expand_tc_kernel(const __grid_constant__ AMaps am, const TcExpandParams p)
                 // Every MMA of the previous row is complete (its last block was drained).
                 const int cpr = w.r16 >> 3;
                 const int n_items = w.nt16 * cpr;
-                float4 f[4][2];
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const int idx = et + 128 * k;
-                    const int tv = idx / cpr, c = idx - tv * cpr;
-                    f[k][0] = make_float4(0.f, 0.f, 0.f, 0.f);
-                    f[k][1] = f[k][0];
-                    if (idx < n_items && tv < w.nt && 8 * c < w.r) {
-                        const float4* src = reinterpret_cast<const float4*>(
-                            p.v + ((size_t)slice * p.T + p.perm[w.tok0 + tv]) * p.r_max + 8 * c);
-                        f[k][0] = src[0];
-                        f[k][1] = src[1];
-                    }
-                }
-#pragma unroll
                 for (int k = 0; k < 4; ++k) {
                     const int idx = et + 128 * k;
                     if (idx >= n_items) break;
                     const int tv = idx / cpr, c = idx - tv * cpr;
-                    float fv[8] = {f[k][0].x, f[k][0].y, f[k][0].z, f[k][0].w,
-                                   f[k][1].x, f[k][1].y, f[k][1].z, f[k][1].w};
+                    float fv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                    if (tv < w.nt && 8 * c < w.r) {
+                        // the planes' loads first, then their sum in plane order
+                        const float4* src = reinterpret_cast<const float4*>(
+                            p.v + ((size_t)slice * p.T + p.perm[w.tok0 + tv]) * p.r_max + 8 * c);
+                        float4 g[kTcMaxPlanes][2];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e)
-                        if (8 * c + e >= w.r) fv[e] = 0.f;
+                        for (int pl = 0; pl < kTcMaxPlanes; ++pl)
+                            if (pl < p.v_parts) {
+                                const float4* sp = src + (size_t)pl * (p.v_part_stride >> 2);
+                                g[pl][0] = sp[0];
+                                g[pl][1] = sp[1];
+                            }
+#pragma unroll
+                        for (int pl = 0; pl < kTcMaxPlanes; ++pl)
+                            if (pl < p.v_parts) {
+                                fv[0] += g[pl][0].x; fv[1] += g[pl][0].y; fv[2] += g[pl][0].z; fv[3] += g[pl][0].w;
+                                fv[4] += g[pl][1].x; fv[5] += g[pl][1].y; fv[6] += g[pl][1].z; fv[7] += g[pl][1].w;
+                            }
+#pragma unroll
+                        for (int e = 0; e < 8; ++e)
+                            if (8 * c + e >= w.r) fv[e] = 0.f;
+                    }
                     uint32_t hi[4], lo[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
@@ -445,6 +451,186 @@ sgmv_expand_tc_kernel(const __grid_constant__ AMaps am, const TcExpandParams p)
     }
 }
 
+// ---------------------------------------------------------------------------- shrink
+// Planes of v = x.A_a for the same batches: CTA (tile row, slice, part) sums the
+// k-blocks [part nkb / P, (part + 1) nkb / P) of 64 h_in columns into plane `part`
+// (P <= 8 planes; the expand adds them in plane order, so the result does not depend
+// on timing). D[t][j] = sum_k x[t][k] A_a[k][j] with M = 128, N = 64, K = 16 per MMA:
+// the tile's tokens are rows 64..127 of the x operand, whose descriptor starts 8 KB
+// before the x tile (rows 0..63 read the stage's A box as filler and their results
+// are dropped), so drain warps 2 and 3 read valid TMEM lanes. A_a's k rows arrive by
+// TMA as one 64-column box with the 128-byte swizzle (the MN-major operand; columns
+// past the rank, pool padding or past r_max, are dropped from the result); the
+// tile's x rows by cp.async into the K-major 128-byte-swizzled layout.
+constexpr int kShThreads = 128;
+constexpr int kShStages = 4;
+constexpr int kShBox = 64 * 64 * 2;           // 64 k rows x 64 columns of A_a, or 64 tokens x 64 k of x
+constexpr int kShStageBytes = 2 * kShBox;     // A box, then the x tile
+constexpr int kShTmemCols = 64;
+
+struct TcShrinkParams {
+    const uint16_t* x;
+    long long x_slice_stride;
+    const int32_t* ranks;
+    const int32_t* perm;
+    const int4* tiles;
+    int32_t* counts;
+    float* v;  // parts planes of [n_slices][T][r_max]
+    long long v_part_stride;
+    int T, n_adapters, h_in, r_max, n_slices;
+    int parts, nkb;  // planes; 64-column k-blocks of h_in
+    unsigned long long timeout_ns;
+    int inject_stall;
+};
+
+__global__ void __launch_bounds__(kShThreads, 3)
+sgmv_shrink_tc_kernel(const __grid_constant__ CUtensorMap a_map, const TcShrinkParams p)
+{
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    __shared__ int s_tok[kTT];
+    __shared__ int s_abort;
+    __shared__ uint32_t s_tmem;
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int per_row = p.n_slices * p.parts;
+    const int g = blockIdx.x / per_row;
+    const int slice = (blockIdx.x - g * per_row) / p.parts;
+    const int part = blockIdx.x - g * per_row - slice * p.parts;
+
+    // the previous kernel in the stream (the segment builder, the producer of x) may still run
+    ptx::pdl_wait();
+    ptx::pdl_launch_dependents();
+    const int4 tl = p.tiles[g];
+    const int nt = tl.z;
+    if (nt <= 0) return;  // unused tile row
+    int32_t* status = p.counts + kSegStatusSlot;
+    if (nt > kTT || tl.x < 0 || tl.x >= p.n_adapters) {  // segments not built for this batch size
+        if (tid == 0 && part == 0 && slice == 0) atomicOr(status, kSegTooLarge);
+        return;
+    }
+    const int kb0 = (int)((long long)part * p.nkb / p.parts);
+    const int nkb = (int)((long long)(part + 1) * p.nkb / p.parts) - kb0;  // >= 1 (parts <= nkb)
+    const int a = tl.x, tok0 = tl.y;
+    int r = p.ranks ? p.ranks[a] : p.r_max;
+    r = max(1, min(r, p.r_max));
+    const int sa = slice * p.n_adapters + a;
+
+    const uint32_t raw_u = ptx::smem_u32(smem_raw);
+    const uint32_t base_u = (raw_u + 1023u) & ~1023u;
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem_raw + (base_u - raw_u) + kShStages * kShStageBytes);
+    uint64_t* empty = full + kShStages;
+    uint64_t* dfull = empty + kShStages;
+    uint64_t* stall = dfull + 1;  // test hook: never completed
+    volatile int* abort_flag = &s_abort;
+
+    if (tid == 0) {
+        s_abort = 0;
+        for (int s = 0; s < kShStages; ++s) {
+            ptx::mbar_init(&full[s], 1 + 32);  // lane 0's expect_tx + every producer lane's copies
+            ptx::mbar_init(&empty[s], 1);      // the MMAs' commit
+        }
+        ptx::mbar_init(dfull, 1);
+        ptx::mbar_init(stall, 1);
+        ptx::fence_mbar_init();
+    }
+    if (tid < nt) s_tok[tid] = p.perm[tok0 + tid];
+    if (warp == 1) {
+        ptx::tmem_alloc(&s_tmem, kShTmemCols);
+        ptx::tmem_relinquish();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = s_tmem;
+
+    if (warp == 0) {
+        // ================================================================ producer
+        if (lane == 0) ptx::tma_prefetch_desc(&a_map);
+        const uint16_t* xs = p.x + (size_t)(p.x_slice_stride ? slice : 0) * p.x_slice_stride;
+        int issued[kShStages] = {};
+        bool go = true;
+        if (p.inject_stall && blockIdx.x == 0)  // test hook: a wait that runs out
+            go = wait_all<false>(stall, 0, abort_flag, status, 0x2000, p.timeout_ns);
+        for (int i = 0; i < nkb && go; ++i) {
+            const int st = i % kShStages;
+            if (i >= kShStages &&
+                !wait_all<false>(&empty[st], (uint32_t)(((i / kShStages) - 1) & 1), abort_flag, status, 0x100,
+                                 p.timeout_ns))
+                break;
+            const int k0 = (kb0 + i) * 64;
+            const uint32_t sA = base_u + (uint32_t)(st * kShStageBytes), sx = sA + kShBox;
+            if (lane == 0) ptx::mbar_arrive_expect_tx(&full[st], (uint32_t)kShBox);
+            __syncwarp();
+            // k rows past h_in and columns past r_max read as zero
+            if (lane == 0) ptx::tma_load_3d(sA, &a_map, &full[st], 0, k0, sa);
+            // x rows: 8 chunks of 16 bytes each, chunk index XOR row (the 128-byte swizzle);
+            // chunks past h_in are zero-filled
+            for (int idx = lane; idx < nt * 8; idx += 32) {
+                const int t = idx >> 3, c = idx & 7, col = k0 + 8 * c;
+                const uint16_t* src = xs + (size_t)s_tok[t] * p.h_in + (col < p.h_in ? col : 0);
+                ptx::cp_async16(sx + (uint32_t)(t * 128 + ((c ^ (t & 7)) << 4)), src, col < p.h_in ? 16u : 0u);
+            }
+            ptx::cp_async_arrive_noinc(&full[st]);
+            ++issued[st];
+        }
+        // let every copy this CTA issued land before it leaves
+        for (int st = 0; st < kShStages; ++st)
+            if (issued[st]) wait_all<false, false>(&full[st], (uint32_t)((issued[st] - 1) & 1), abort_flag, status,
+                                                   0x800, p.timeout_ns);
+    } else if (warp == 1) {
+        // ================================================================ MMA issuer
+        const uint32_t idesc = idesc_mn_b(64);
+        for (int i = 0; i < nkb; ++i) {
+            const int st = i % kShStages;
+            if (!wait_all<false>(&full[st], (uint32_t)((i / kShStages) & 1), abort_flag, status, 0x800,
+                                 p.timeout_ns))
+                break;
+            if (lane == 0) {
+                ptx::tc_fence_after();
+                const uint32_t sA = base_u + (uint32_t)(st * kShStageBytes);
+                for (int ks = 0; ks < 4; ++ks)
+                    ptx::tc_mma_f16(tmem, desc_k_sw128(sA + (uint32_t)(ks * 32)),
+                                    desc_mn_sw128(sA + (uint32_t)(ks * 2048), (uint32_t)kShBox), idesc,
+                                    (i | ks) ? 1u : 0u);
+                ptx::tc_commit(&empty[st]);
+            }
+            __syncwarp();
+        }
+        // the accumulator is complete (or, after an abort, every issued MMA is)
+        if (lane == 0) ptx::tc_commit(dfull);
+        __syncwarp();
+    } else {
+        // ================================================================ drain: plane rows
+        const int q = warp & 3;  // 2 or 3: TMEM lanes 64..127, the tile's tokens
+        const int t = (q - 2) * 32 + lane;
+        const bool ok = wait_all<false, false>(dfull, 0, abort_flag, status, 0x200, p.timeout_ns);
+        ptx::tc_fence_after();
+        float d[64];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) ptx::tmem_ld16(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(c * 16), d + c * 16);
+        if (ok && !*abort_flag && t < nt) {
+            float* dst = p.v + (size_t)part * p.v_part_stride + ((size_t)slice * p.T + s_tok[t]) * p.r_max;
+#pragma unroll
+            for (int j = 0; j < 64; j += 4) {
+                if (j >= p.r_max) break;
+                float4 o;
+                o.x = j < r ? d[j] : 0.f;
+                o.y = j + 1 < r ? d[j + 1] : 0.f;
+                o.z = j + 2 < r ? d[j + 2] : 0.f;
+                o.w = j + 3 < r ? d[j + 3] : 0.f;
+                *reinterpret_cast<float4*>(dst + j) = o;
+            }
+        }
+    }
+
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem, kShTmemCols);
+    }
+}
+
 }  // namespace
 
 bool sgmv_expand_tc_eligible(int T, const lora_pool_t& pool)
@@ -455,12 +641,14 @@ bool sgmv_expand_tc_eligible(int T, const lora_pool_t& pool)
            pool.h_out >= kTcBlockN;
 }
 
-cudaError_t launch_sgmv_expand_tc(const float* v, const lora_pool_t& pool, const lora_segments_t& seg, void* y,
-                                  cudaStream_t stream)
+cudaError_t launch_sgmv_expand_tc(const float* v, int v_parts, const lora_pool_t& pool, const lora_segments_t& seg,
+                                  void* y, cudaStream_t stream)
 {
     if (seg.T == 0) return cudaSuccess;
     TcExpandParams p = {};
     p.v = v;
+    p.v_parts = v_parts;
+    p.v_part_stride = (long long)pool.n_slices * seg.T * pool.r_max;
     p.y = static_cast<uint16_t*>(y);
     p.ranks = pool.ranks;
     p.scales = pool.scales;
@@ -498,6 +686,60 @@ cudaError_t launch_sgmv_expand_tc(const float* v, const lora_pool_t& pool, const
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, kern, am, p);
+}
+
+int sgmv_shrink_tc_parts(const lora_pool_t& pool)
+{
+    const int nkb = (pool.h_in + 63) / 64;
+    return nkb < kTcMaxPlanes ? nkb : kTcMaxPlanes;
+}
+
+cudaError_t launch_sgmv_shrink_tc(const void* x, int64_t x_slice_stride, const lora_pool_t& pool,
+                                  const lora_segments_t& seg, float* v, int parts, cudaStream_t stream)
+{
+    if (seg.T == 0) return cudaSuccess;
+    TcShrinkParams p = {};
+    p.x = static_cast<const uint16_t*>(x);
+    p.x_slice_stride = x_slice_stride;
+    p.ranks = pool.ranks;
+    p.perm = seg.perm;
+    p.tiles = reinterpret_cast<const int4*>(seg.tiles);
+    p.counts = seg.counts;
+    p.v = v;
+    p.v_part_stride = (long long)pool.n_slices * seg.T * pool.r_max;
+    p.T = seg.T;
+    p.n_adapters = pool.n_adapters;
+    p.h_in = pool.h_in;
+    p.r_max = pool.r_max;
+    p.n_slices = pool.n_slices;
+    p.nkb = (pool.h_in + 63) / 64;
+    p.parts = parts < 1 ? 1 : (parts > p.nkb ? p.nkb : parts);
+    p.timeout_ns = debug_wait_limit_ns();
+    p.inject_stall = debug_inject_stall();
+    // A as {r_max, h_in, slices x adapters}, box {64, 64, 1}, 128-byte swizzle (columns past
+    // r_max and rows past h_in read as zero)
+    CUtensorMap a_map;
+    const uint64_t dims[3] = {(uint64_t)pool.r_max, (uint64_t)pool.h_in,
+                              (uint64_t)pool.n_slices * (uint64_t)pool.n_adapters};
+    const uint64_t strides[2] = {(uint64_t)pool.r_max * 2, (uint64_t)pool.h_in * pool.r_max * 2};
+    const uint32_t box[3] = {64, 64, 1};
+    if (!encode_tmap_3d(&a_map, CU_TENSOR_MAP_DATA_TYPE_UINT16, pool.A, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    const size_t smem = (size_t)kShStages * kShStageBytes + 8 * (2 * kShStages + 2) + 1024;
+    auto kern = sgmv_shrink_tc_kernel;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)((long long)max_tiles_for(seg.T, pool.n_adapters) * pool.n_slices * p.parts), 1, 1);
+    cfg.blockDim = dim3(kShThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, a_map, p);
 }
 
 }  // namespace lora

@@ -348,7 +348,7 @@ def apply_launches(p, sm_count=None):
     from adapter_gemm_builder_b200 import lora as L
     if p.T <= 64 and p.T <= 2 * p.n_adapters:
         return 1
-    if p.T >= 32 * p.n_adapters and p.h_out >= 128:
+    if tc_path(p):
         return 2
     if sm_count is None:
         import torch
@@ -481,12 +481,21 @@ def time_apply(p, dev, steps, warmup, stream, ext, world=1, clocks=None):
                 launch=f"CUDA graph of {R} steps")
 
 
+def tc_path(p):
+    """lora_apply (with its workspace) takes the tensor-core shrink and expand: a batch of
+    long segments (not decode-like, T >= 32 n_adapters, h_out >= 128; the library's rule)."""
+    return not (p.T <= 64 and p.T <= 2 * p.n_adapters) and p.T >= 32 * p.n_adapters and p.h_out >= 128
+
+
 def roofline_apply(p, t, hbm_peak, peak_src, workload):
     bytes_step = apply_bytes(p)
     achieved = bytes_step / (t["kernel_ms"] / 1e3) / 1e9
+    tc = tc_path(p)
     return {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-            "frac": achieved / hbm_peak, "traffic": profiled_traffic("sgmv.cu", workload),
-            "kernel": "lora_apply (sgmv kernels)", "kernel_us": t["kernel_ms"] * 1e3,
+            "frac": achieved / hbm_peak,
+            "traffic": profiled_traffic("sgmv_tc.cu" if tc else "sgmv.cu", workload),
+            "kernel": "lora_apply (tensor-core shrink + expand)" if tc else "lora_apply (sgmv kernels)",
+            "kernel_us": t["kernel_ms"] * 1e3,
             "launches_per_call": apply_launches(p),
             "algorithmic_bytes_per_launch": bytes_step,
             "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs, burst copy)",

@@ -98,6 +98,23 @@ def test_sgmv_tc_expand_wait_runs_out_then_next_call_is_correct():
     assert_close(f64(host_bf16_bits(y))[0], want, TOL_BF16, "tc expand after a timeout")
 
 
+def test_sgmv_tc_apply_wait_runs_out_then_next_call_is_correct():
+    # long segments with a workspace: the tensor-core shrink into planes of v, then the
+    # tensor-core expand; one CTA of each launch stalls
+    p = wl.make_lora_problem("t", 14, T=300, n_adapters=3, h_in=640, h_out=392, r_max=64,
+                             ids_kind="zipf", none_frac=0.1, rank_choices=(8, 40, 64))
+    d = DeviceProblem(p)
+    y = d.y_in()
+    _stalled(lambda: L.lora_apply(d.x, d.pool, d.seg, y))
+    st, detail = L.lora_segments_status(d.seg)
+    assert st == L.LORA_ERR_TIMEOUT and detail & SGMV_WAIT_BITS, hex(detail)
+    y = d.y_in()
+    L.lora_apply(d.x, d.pool, d.seg, y)
+    torch.cuda.synchronize()
+    assert L.lora_segments_status(d.seg)[0] == L.LORA_OK
+    assert_close(f64(host_bf16_bits(y)), oracle_apply(p), TOL_BF16, "tc apply after a timeout")
+
+
 def test_fp8_gemm_wait_runs_out_then_next_call_is_correct():
     M, K, N = 64, 512, 640
     rng = np.random.default_rng(5)

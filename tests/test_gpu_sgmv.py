@@ -411,13 +411,33 @@ TC_CASES = {
 }
 
 
+def _tc_planes(h_in):
+    return min(8, -(-h_in // 64))
+
+
 def test_tc_cases_take_the_tensor_core_path():
-    """The workspace of lora_apply on these batches holds v (fp32, every slice)."""
+    """The workspace of lora_apply on these batches holds the shrink's planes of v (fp32,
+    every slice; one plane per part of h_in, at most 8)."""
     for case, kw in TC_CASES.items():
         p = _small(**kw)
         d = DeviceProblem(p, build=False)
         n = L.lora_workspace_size(L.LORA_OP_APPLY, p.T, 0, d.pool)
-        assert n == -(-p.n_slices * p.T * p.r_max * 4 // 256) * 256, case
+        v = _tc_planes(p.h_in) * p.n_slices * p.T * p.r_max * 4
+        assert n == -(-max(v, 16 * L.max_tiles(p.T, p.n_adapters)) // 256) * 256, case
+
+
+@pytest.mark.parametrize("case", ["tc_ragged_mixed", "tc_rank64_slices"])
+def test_apply_tc_one_plane_workspace(case):
+    """A workspace with room for one plane of v only: the cluster shrink, then the
+    tensor-core expand."""
+    p = _small(**TC_CASES[case])
+    d = DeviceProblem(p)
+    ws = torch.zeros(p.n_slices * p.T * p.r_max * 4, dtype=torch.uint8, device="cuda")
+    y = d.y_in()
+    L.lora_apply(d.x, d.pool, d.seg, y, ws=ws)
+    torch.cuda.synchronize()
+    assert L.lora_segments_status(d.seg)[0] == L.LORA_OK
+    assert_close(f64(host_bf16_bits(y)), oracle_apply(p), TOL_BF16, case)
 
 
 @pytest.mark.parametrize("case", list(TC_CASES))

@@ -78,10 +78,13 @@ def test_workspace_sizes(lib):
     # a general batch: the tile rows in cost order, 16 bytes per row of lora_max_tiles
     n = lib.lora_workspace_size(L.LORA_OP_APPLY, 512, 0, ctypes.byref(pa))
     assert n >= 16 * lib.lora_max_tiles(512, 256) and n % 256 == 0
-    # long segments (T >= 32 n_adapters, h_out >= 128): v in fp32 for the shrink and the
-    # tensor-core expand, n_slices x T x r_max x 4 bytes rounded up to 256
+    # long segments (T >= 32 n_adapters, h_out >= 128): the shrink's planes of v in fp32
+    # (one per part of h_in, at most 8), n_slices x T x r_max x 4 bytes each, rounded up to 256
     pl = _pool(n_slices=2, n_adapters=8, h_in=4096, h_out=11008, r_max=64)
-    assert lib.lora_workspace_size(L.LORA_OP_APPLY, 2704, 0, ctypes.byref(pl)) == -(-2 * 2704 * 64 * 4 // 256) * 256
+    assert lib.lora_workspace_size(L.LORA_OP_APPLY, 2704, 0, ctypes.byref(pl)) == \
+        -(-8 * 2 * 2704 * 64 * 4 // 256) * 256
+    pl = _pool(n_slices=1, n_adapters=2, h_in=192, h_out=128, r_max=16)
+    assert lib.lora_workspace_size(L.LORA_OP_APPLY, 64, 0, ctypes.byref(pl)) == -(-3 * 64 * 16 * 4 // 256) * 256
     # ... but not with a narrow y (h_out < 128) or fewer tokens per adapter
     assert lib.lora_workspace_size(L.LORA_OP_APPLY, 2704, 0, ctypes.byref(_pool(n_adapters=8, h_out=120))) \
         == -(-16 * lib.lora_max_tiles(2704, 8) // 256) * 256
