@@ -152,11 +152,13 @@ LORA_API int lora_segments_status(const lora_segments_t* seg, lora_stream_t stre
  * Bytes of workspace an operation needs (0 if it needs none), or (size_t)-1
  * for invalid arguments. For LORA_OP_FP8_GEMM, T is the
  * token count M and `K` the GEMM's reduction size; `pool` may be NULL (no
- * LoRA). LORA_OP_APPLY needs a valid pool; it returns 0 for a decode-like
- * batch (lora_tile_tokens_for), for a batch of long segments (T >= 32 *
- * n_adapters, h_out >= 128) the bytes of v in fp32 (n_slices * T * r_max * 4,
- * rounded up to 256; see lora_apply), and otherwise the bytes of the tile rows
- * in cost order (16 per row of lora_max_tiles). The other operations ignore K.
+ * LoRA). LORA_OP_APPLY needs a valid pool. It returns:
+ *   0 for a decode-like batch (lora_tile_tokens_for);
+ *   for a batch of long segments (T >= 32 * n_adapters, h_out >= 128), the bytes of
+ *   P = min(8, ceil(h_in / 64)) planes of fp32 v (P * n_slices * T * r_max * 4,
+ *   at least the tile-order bytes, rounded up to 256; see lora_apply);
+ *   otherwise the bytes of the tile rows in cost order (16 per row of
+ *   lora_max_tiles). The other operations ignore K.
  * A workspace must be zeroed once after allocation (lora_workspace_init);
  * afterwards the library keeps it in a reusable state.
  */
@@ -234,11 +236,15 @@ LORA_API int lora_expand(const float* v, const lora_pool_t* pool, const lora_seg
  * by descending rank), so that the long rows start first; the results are the
  * same either way. ws NULL: one launch, table order.
  * A batch of long segments (as for lora_expand's tensor-core path) with a
- * workspace of lora_workspace_size(LORA_OP_APPLY, ...) bytes instead runs the
- * shrink into the workspace (v fp32 [n_slices][T][r_max]) and then the
- * tcgen05 expand as its programmatic dependent: two launches, the same
- * results up to fp32 rounding order. With a smaller workspace (at least the
- * tile-order bytes) such a batch takes the cluster kernel.
+ * workspace of lora_workspace_size(LORA_OP_APPLY, ...) bytes instead runs two
+ * launches. First the tcgen05 shrink writes P = min(8, ceil(h_in / 64)) planes
+ * of fp32 v [n_slices][T][r_max] into the workspace, each the sum over one
+ * part of h_in. Then the tcgen05 expand, as its programmatic dependent, adds
+ * the planes in plane order (deterministic) and applies the term. The results
+ * equal the one-launch path's up to fp32 rounding order.
+ * With a workspace of one plane (n_slices * T * r_max * 4 bytes), the cluster
+ * shrink writes v and the tensor-core expand follows. With a smaller workspace
+ * (at least the tile-order bytes), such a batch takes the cluster kernel.
  */
 LORA_API int lora_apply(const void* x, int64_t x_slice_stride, const lora_pool_t* pool,
                const lora_segments_t* seg, void* y, void* ws, size_t ws_bytes,
