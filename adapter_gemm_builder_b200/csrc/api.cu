@@ -84,8 +84,15 @@ size_t fp8_ws_layout(int M, int K, const lora_pool_t* pool, size_t* off_xq, size
     off += align256((size_t)(16 + device_sm_count()) * 4);
     *off_part = off;
     off += align256(fp8_gemm_partial_bytes(M));
-    if (off_order) *off_order = off;  // the split path's apply: tile rows in cost order
-    if (gemm_split(M, pool)) off += align256(sgmv_order_bytes(M, pool->n_adapters));
+    if (off_order) *off_order = off;  // the split path's apply: tile rows in cost order, or
+    if (gemm_split(M, pool)) {        // for long segments the tensor-core shrink's planes of v
+        size_t o = sgmv_order_bytes(M, pool->n_adapters);
+        if (sgmv_expand_tc_eligible(M, *pool)) {
+            const size_t v = apply_v_bytes(M, *pool, sgmv_shrink_tc_parts(*pool));
+            if (v > o) o = v;
+        }
+        off += align256(o);
+    }
     return off;
 }
 
@@ -201,7 +208,20 @@ int gemm_lora_launch(int esz, const void* x, int M, int K, int N, const uint8_t*
     e = launch_fp8_gemm(a, s);
     if (e != cudaSuccess || !split) return cuda_status(e);
     // 3. many adapters or tokens: their term added to the GEMM's bf16 output by the SGMV
-    //    apply (a general batch's tile rows in cost order, in the workspace)
+    //    apply: for long segments the tensor-core shrink into planes of v (in the
+    //    workspace) and the tensor-core expand, else the cluster kernel (a general batch's
+    //    tile rows in cost order, in the workspace)
+    if (sgmv_expand_tc_eligible(M, *pool)) {
+        float* vp = reinterpret_cast<float*>(w + off_order);
+        int planes = sgmv_shrink_tc_parts(*pool);
+        e = launch_sgmv_shrink_tc(x, 0, *pool, *seg, vp, planes, s);
+        if (e == cudaErrorInvalidValue) {  // the pool's tensor map was refused: the cluster shrink
+            e = launch_sgmv(SGMV_SHRINK, x, 0, *pool, *seg, vp, nullptr, s, false);
+            planes = 1;
+        }
+        if (e != cudaSuccess) return LORA_ERR_CUDA;
+        return cuda_status(launch_sgmv_expand_tc(vp, planes, *pool, *seg, y, s));
+    }
     void* order = tile_tokens_for(M, pool->n_adapters) > LORA_DECODE_TILE_TOKENS ? w + off_order : nullptr;
     return cuda_status(launch_sgmv(SGMV_APPLY, x, 0, *pool, *seg, nullptr, y, s, false, order));
 }

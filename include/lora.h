@@ -280,8 +280,10 @@ LORA_API int fp8_quantize_rows(const void* x, int M, int K, uint8_t* xq, float* 
  * Many adapters or tokens: when the pool holds more than 16 adapters and
  * M > 16, or M > 1024, the adapters' term is not folded into the GEMM's
  * accumulator; the call runs the base GEMM and then the SGMV apply of
- * lora_apply on its output (three or four launches, the workspace holding the
- * apply's tile order), so y = bf16(bf16(base) + term).
+ * lora_apply on its output, so y = bf16(bf16(base) + term). That is three or
+ * four launches: the workspace holds the apply's tile order, or, for a batch
+ * of long segments (M >= 32 * n_adapters), the tensor-core shrink's planes of
+ * v, followed by the tensor-core expand.
  * The GEMM is a persistent grid of one CTA per SM whose CTAs wait on one
  * another (the down-projection count, stream-K partials), so all of them must
  * be resident at once: the context needs every SM of the device. Where fewer
