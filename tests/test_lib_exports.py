@@ -211,3 +211,23 @@ def test_debug_wait_limit_validates_and_restores(lib):
     assert lib.lora_debug_set_wait_limit(1_000_000, 2) == L.LORA_ERR_INVALID_ARG
     assert lib.lora_debug_set_wait_limit(1_000_000, 1) == L.LORA_OK
     assert lib.lora_debug_set_wait_limit(0, 0) == L.LORA_OK                      # default again
+
+
+def test_bench_launch_rule_matches_the_library(lib):
+    """bench.py counts this library's launches per apply (gpu_launches) with its own copy
+    of the rule that sends a batch to the tensor-core shrink and expand; the library's
+    rule shows in the APPLY workspace size (planes of v instead of the tile order)."""
+    import sys
+    from types import SimpleNamespace
+    sys.path.insert(0, ROOT)
+    import bench
+    for T, n, h_in, h_out in [(2704, 8, 4096, 11008), (512, 256, 5120, 5120), (36, 32, 4096, 4096),
+                              (64, 2, 4096, 4096), (63, 2, 4096, 4096), (256, 8, 512, 128),
+                              (256, 8, 512, 120), (255, 8, 512, 128), (1100, 16, 8192, 28672),
+                              (64, 64, 1024, 1024), (4096, 1, 64, 200)]:
+        pool = _pool(n_adapters=n, h_in=h_in, h_out=h_out, r_max=64)
+        got = lib.lora_workspace_size(L.LORA_OP_APPLY, T, 0, ctypes.byref(pool))
+        planes = min(8, -(-h_in // 64))
+        tc_size = -(-max(planes * T * 64 * 4, 16 * lib.lora_max_tiles(T, n)) // 256) * 256
+        p = SimpleNamespace(T=T, n_adapters=n, h_in=h_in, h_out=h_out)
+        assert bench.tc_path(p) == (got == tc_size and got != 0), (T, n, h_in, h_out, got)
