@@ -340,6 +340,14 @@ sgmv_expand_tc_kernel(const __grid_constant__ AMaps am, const TcExpandParams p)
                 // Every MMA of the previous row is complete (its last block was drained).
                 const int cpr = w.r16 >> 3;
                 const int n_items = w.nt16 * cpr;
+                // the items' token indices first (independent loads), then each item's planes
+                int tokv[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const int idx = et + 128 * k, tv = idx / cpr;
+                    tokv[k] = idx < n_items && tv < w.nt ? p.perm[w.tok0 + tv] : 0;
+                }
+#pragma unroll
                 for (int k = 0; k < 4; ++k) {
                     const int idx = et + 128 * k;
                     if (idx >= n_items) break;
@@ -348,7 +356,7 @@ sgmv_expand_tc_kernel(const __grid_constant__ AMaps am, const TcExpandParams p)
                     if (tv < w.nt && 8 * c < w.r) {
                         // the planes' loads first, then their sum in plane order
                         const float4* src = reinterpret_cast<const float4*>(
-                            p.v + ((size_t)slice * p.T + p.perm[w.tok0 + tv]) * p.r_max + 8 * c);
+                            p.v + ((size_t)slice * p.T + tokv[k]) * p.r_max + 8 * c);
                         float4 g[kTcMaxPlanes][2];
 #pragma unroll
                         for (int pl = 0; pl < kTcMaxPlanes; ++pl)
