@@ -95,6 +95,13 @@ def test_workspace_sizes(lib):
     assert n >= 256 + 256 * 8192 + 256 * 4 + 256 * 16 * 4
     n0 = lib.lora_workspace_size(L.LORA_OP_FP8_GEMM, 256, 8192, None)
     assert n0 < n
+    # a prefill through a GEMM call (M > 1024, long segments): the split path's apply
+    # holds the tensor-core shrink's eight planes of v in the same workspace
+    pp = _pool(n_adapters=8, h_in=4096, h_out=11008, r_max=64)
+    for op in (L.LORA_OP_FP8_GEMM, L.LORA_OP_BF16_GEMM):
+        big = lib.lora_workspace_size(op, 2704, 4096, ctypes.byref(pp))
+        base = lib.lora_workspace_size(op, 2704, 4096, None)
+        assert big - base >= 8 * 2704 * 64 * 4
     assert lib.lora_workspace_size(99, 1, 1, None) == ctypes.c_size_t(-1).value
     assert lib.lora_workspace_size(L.LORA_OP_FP8_GEMM, 4, 0, None) == ctypes.c_size_t(-1).value
 
