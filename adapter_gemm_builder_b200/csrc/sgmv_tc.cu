@@ -1,19 +1,19 @@
-// sgmv_tc.cu -- the expand half of SGMV (Punica README, "How?": the added term
-// x_i.A_i.B_i of every adapter's segment, here its up-projection
-// y += s_a * v.B_a with v = x.A_a given) on the tcgen05 tensor cores, for
-// batches whose segments are long (prefill-like: the 64-token tiles of
-// lora_segments_t fill the MMAs).
+// sgmv_tc.cu -- SGMV (Punica README, "How?": the added term x_i.A_i.B_i of
+// every adapter's segment) on the tcgen05 tensor cores, for batches whose
+// segments are long (prefill-like: the 64-token tiles of lora_segments_t fill
+// the MMAs): the expand y += s_a * v.B_a, and (at the end of the file) the
+// shrink v = x.A_a into planes of v that the expand sums.
 //
-// One MMA per block of 128 output columns: D[t][n] = sum_j v[t][j] * B_a[j][n]
+// Expand. One MMA per block of 128 output columns: D[t][n] = sum_j v[t][j] * B_a[j][n]
 // (M = 128 rows, N = 128 columns, K = the adapter's rank rounded up to 16),
 // accumulated in TMEM. A tile has at most 64 tokens, so v's rows fill M twice
 // (rows 64..127 repeat rows 0..63): each of the four drain warps then reads
 // valid TMEM lanes, two warps per half of the columns. B_a's rows (rank index
 // j, columns contiguous) arrive by TMA as two 64-column boxes with the
 // 128-byte swizzle, which is the MN-major operand layout as it stands, so
-// B_a is read straight from the pool. v (fp32) is split once per CTA into
-// bf16 halves v = hi + lo (~16 bits of v), kept as K-major 128-byte-swizzled
-// operands; both halves go into the same accumulator.
+// B_a is read straight from the pool. v (fp32) is split, once per tile row a
+// CTA works on, into bf16 halves v = hi + lo (~16 bits of v), kept as K-major
+// 128-byte-swizzled operands; both halves go into the same accumulator.
 //
 // y rows of a block come into shared memory as 16-byte cp.async copies from
 // all lanes of the producer (two 256-byte rows per instruction; a 1-D bulk
@@ -28,8 +28,9 @@
 // rows by cp.async) on mbarriers; warp 1 owns TMEM (two accumulators of 128
 // columns) and its lane 0 issues the MMAs; warps 2..5 build v's operands,
 // then drain each accumulator into y (warp w reads TMEM lanes 32 (w % 4) ..
-// + 31). A CTA takes one tile row of one slice and a contiguous run of column
-// blocks. Every wait is bounded; on expiry the CTA records a status word in
+// + 31). The persistent grid (two CTAs per SM) splits the sequence of (tile
+// row, slice, column block) units evenly, a CTA's run crossing rows where it
+// must. Every wait is bounded; on expiry the CTA records a status word in
 // lora_segments_t.counts, drains what it issued and leaves.
 #include <cuda.h>
 #include <cuda_bf16.h>
