@@ -195,8 +195,9 @@ def source_hash(*names):
 
 
 def profiled_traffic(kernel_file, workload):
-    """DRAM bytes per launch from the committed ncu summary of this kernel and
-    workload, if the kernel source has not changed since (else None)."""
+    """DRAM bytes per lora_apply call (its one launch, or both launches of the
+    tensor-core pair) from the committed ncu summary of this kernel source and
+    workload, if the source has not changed since (else None)."""
     path = os.path.join(ROOT, "profiles", f"{os.path.splitext(kernel_file)[0]}_{workload}.md")
     if not os.path.exists(path):
         return None
@@ -497,7 +498,7 @@ def roofline_apply(p, t, hbm_peak, peak_src, workload):
             "kernel": "lora_apply (tensor-core shrink + expand)" if tc else "lora_apply (sgmv kernels)",
             "kernel_us": t["kernel_ms"] * 1e3,
             "launches_per_call": apply_launches(p),
-            "algorithmic_bytes_per_launch": bytes_step,
+            "algorithmic_bytes_per_call": bytes_step,  # every launch of one lora_apply together
             "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs, burst copy)",
             "timing": t["timing"]}
 
