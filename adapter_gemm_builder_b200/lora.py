@@ -248,8 +248,10 @@ def lora_expand(v: torch.Tensor, pool: Pool, seg: Segments, y: torch.Tensor, str
 def lora_apply(x: torch.Tensor, pool: Pool, seg: Segments, y: torch.Tensor, stream=None,
                x_slice_stride: int | None = None, ws: torch.Tensor | None | bool = None) -> None:
     """y += s_a (x.A_a).B_a; ws: a workspace of lora_workspace_size(LORA_OP_APPLY, T, 0, pool)
-    bytes, in which a general batch's tile rows are put in cost order (allocated here when
-    None and the size is not 0; False: none, the rows run in table order)."""
+    bytes (allocated here when None and the size is not 0; False: none). A batch of long
+    segments uses it for the tensor-core shrink's planes of v, then the tensor-core expand;
+    another general batch, for its tile rows in cost order. Without one, one launch of the
+    cluster kernel, rows in table order."""
     xs = _slice_stride(x, pool) if x_slice_stride is None else x_slice_stride
     if ws is False:  # explicitly none: the tile rows run in table order
         ws = None
