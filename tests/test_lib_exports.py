@@ -238,3 +238,23 @@ def test_bench_launch_rule_matches_the_library(lib):
         tc_size = -(-max(planes * T * 64 * 4, 16 * lib.lora_max_tiles(T, n)) // 256) * 256
         p = SimpleNamespace(T=T, n_adapters=n, h_in=h_in, h_out=h_out)
         assert bench.tc_path(p) == (got == tc_size and got != 0), (T, n, h_in, h_out, got)
+
+
+def test_bench_launches_per_apply(lib):
+    """The launches per lora_apply that bench.py multiplies into gpu_launches, on the
+    bench workloads' shapes (148 SMs): the decode kernel alone; the tile-ordering kernel
+    and the cluster kernel when the clusters need more than one wave; the tensor-core
+    shrink and expand for long segments; the cluster kernel alone otherwise."""
+    import sys
+    from types import SimpleNamespace as NS
+    sys.path.insert(0, ROOT)
+    import bench
+    cases = {
+        "bgmv_decode": (NS(T=36, n_adapters=32, n_slices=1, h_in=4096, h_out=4096), 1),
+        "identical": (NS(T=36, n_adapters=32, n_slices=1, h_in=4096, h_out=4096), 1),
+        "sgmv_tiny": (NS(T=64, n_adapters=4, n_slices=1, h_in=1024, h_out=1024), 1),
+        "sgmv_prefill": (NS(T=2704, n_adapters=8, n_slices=1, h_in=4096, h_out=11008), 2),
+        "many_tenants": (NS(T=512, n_adapters=256, n_slices=4, h_in=5120, h_out=5120), 2),
+    }
+    for name, (p, want) in cases.items():
+        assert bench.apply_launches(p, sm_count=148) == want, name
